@@ -1,0 +1,368 @@
+#!/usr/bin/env python
+"""Benchmark: one GLM-5.2-shape quantised MoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one forward of the whole layer (Q8_0 of x, router, bucketing, expert
+gate/up + SiLU + Q8_0 of h, expert down, combine) over one batch of the
+workload's tokens, with all weights resident in HBM.  L2 is flushed (a write of
+twice its size) before every timed step, so the selected experts' weights come
+from HBM as in a real decode.  Each step is timed on the device with CUDA
+events recorded by the library at its phase boundaries; the phase events also
+give the live duration of the dominant kernel for the roofline.
+
+N > 1: one process per GPU (torchrun); each rank runs an independent replica of
+the layer on its own tokens (the layer forward has no exchange step), the
+ranks' times are max-reduced and value = tokens of all ranks / that time.
+
+--impl reference times the CPU oracle (plain C, fp64) on the host cores on a
+bounded sample of the same workload; on N > 1 only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "GLM-5.2-shape MoE layer tokens/s; expert-weight HBM GB/s vs B200 peak"
+DEFAULT_WORKLOAD = "glm52_decode_int4_t1"
+SPEC_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ----------------------------------------------------------------------------
+# helpers (host-side logic, covered by CPU tests)
+# ----------------------------------------------------------------------------
+def measured_peak_hbm() -> tuple[float, str]:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def dist_env() -> tuple[int, int, int]:
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(tokens_per_rank: int, steps: int, world: int, max_total_ms: float) -> float:
+    """Whole-job tokens/s: every rank ran `steps` steps of `tokens_per_rank`."""
+    return world * tokens_per_rank * steps / (max_total_ms / 1e3)
+
+
+def expert_bytes(shape) -> int:
+    return shape.expert_bytes
+
+
+def gateup_bytes(shape) -> int:
+    """Algorithmic bytes of one expert's gate+up matrices and their row scales."""
+    return 2 * shape.matrix_bytes(shape.inter, shape.hidden) + 2 * 4 * shape.inter
+
+
+def kernel_sources_sha() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "quantized_routed_expert_group_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str) -> float | None:
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it
+    was taken on the current kernel sources; otherwise None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(p) as f:
+            doc = json.load(f)
+    except Exception:
+        return None
+    for row in doc.get("kernels", []):
+        if row.get("kernel") == kernel and row.get("workload") == workload and \
+                row.get("sources_sha") == kernel_sources_sha():
+            return float(row["dram_bytes_per_launch"])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_id: str | None, period_ms: int = 50):
+        self.proc = None
+        if gpu_id is None:
+            return
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gpu_id, f"--query-gpu={','.join(self.FIELDS)}",
+                 "--format=csv,noheader,nounits", "-lms", str(period_ms)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        return parse_clock_samples(out)
+
+
+def parse_clock_samples(text: str) -> dict | None:
+    rows = [r.split(",") for r in text.strip().splitlines() if r.count(",") >= 8]
+    if not rows:
+        return None
+    sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+    mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if "Active" in v and "Not" not in v})
+    return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+            "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------
+# our implementation
+# ----------------------------------------------------------------------------
+def run_ours(args) -> dict | None:
+    import torch
+    import torch.distributed as dist
+
+    from quantized_routed_expert_group_b200 import moe, synth
+
+    rank, world, local = dist_env()
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = synth.WORKLOADS[args.workload]
+    s = wl.shape
+    # replicas: same weights, each rank its own tokens
+    wl_x = synth.Workload(wl.name, s, wl.T, wl.seed + 7919 * rank, wl.x_kind, wl.bias_kind)
+    layer = moe.synth_layer(wl, dev)
+    x = torch.from_numpy(synth.make_x(wl_x)).to(dev)
+    out = torch.empty_like(x)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+
+    # warm-up
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        layer.forward(x, out)
+    torch.cuda.synchronize()
+    assert layer.device_error() == 0
+    n_active = int((layer.view(wl.T)["counts"] > 0).sum().item())
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.PROFILE_PHASES + 1)] for _ in range(K)]
+    for row in evs:  # torch creates the CUDA event on first record
+        for ev in row:
+            ev.record()
+    gpu_uuid = None
+    try:
+        gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        if not gpu_uuid.startswith("GPU-"):
+            gpu_uuid = "GPU-" + gpu_uuid
+    except Exception:
+        pass
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(gpu_uuid)
+    time.sleep(0.15)
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        moe.profile_events(evs[i])
+        layer.forward(x, out)
+    moe.profile_events(None)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    step_ms = [evs[i][0].elapsed_time(evs[i][-1]) for i in range(K)]
+    phase_ms = [[evs[i][p].elapsed_time(evs[i][p + 1]) for i in range(K)] for p in range(moe.PROFILE_PHASES)]
+    total_ms = sum(step_ms)
+    max_total = reduce_max(total_ms, dev)
+    value = throughput(wl.T, K, world, max_total)
+
+    # end to end through the host-buffer entry point (pinned host x / out)
+    K_e2e = max(1, min(K, 200))
+    xh = x.cpu().pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    e2e_s = 0.0
+    for i in range(K_e2e):
+        flush.fill_(i & 0xFF)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        layer.forward_host(xh, oh)
+        e2e_s += time.perf_counter() - t0
+    e2e_max = reduce_max(e2e_s * 1e3, dev)
+    e2e_value = throughput(wl.T, K_e2e, world, e2e_max)
+
+    # roofline of the dominant kernel (expert gate/up: 2/3 of the expert bytes)
+    peak, peak_kind = measured_peak_hbm()
+    gu_ms = statistics.mean(phase_ms[2])
+    gu_bytes = (n_active + s.n_shared) * gateup_bytes(s)
+    achieved = gu_bytes / (gu_ms * 1e-3) / 1e9
+    layer_bytes = (n_active + s.n_shared) * expert_bytes(s)
+    ms_step = statistics.mean(step_ms)
+    layer_gbs = layer_bytes / (ms_step * 1e-3) / 1e9
+    if rank != 0:
+        return None
+    res = {
+        "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded; random-init weights of the layer's shape)",
+        "config": {"workload": wl.name, "tokens": wl.T, "hidden": s.hidden, "inter": s.inter,
+                   "experts": s.n_experts, "top_k": s.top_k, "shared": s.n_shared, "weights": f"int{s.wbits}",
+                   "activations": "Q8_0 int8", "unique_experts_per_step": n_active,
+                   "l2": "flushed before every step (write of 2x L2)", "parallelism": f"replicas x{world}"},
+        "layer_hbm": {"algorithmic_bytes": layer_bytes, "gbs": round(layer_gbs, 1),
+                      "frac_measured": round(layer_gbs / peak, 4), "frac_spec_8tbs": round(layer_gbs / SPEC_HBM_GBS, 4)},
+        "phases_ms": {n: round(statistics.mean(v), 5) for n, v in zip(moe.PHASE_NAMES, phase_ms)},
+        "roofline": {"kernel": "k_gateup", "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "algorithmic_bytes_per_launch": gu_bytes,
+                     "traffic": ncu_traffic("k_gateup", wl.name)},
+        "e2e": {"value": round(e2e_value, 3), "unit": "tokens/s", "h2d_bytes_per_step": x.numel() * 4,
+                "d2h_bytes_per_step": out.numel() * 4, "steps": K_e2e},
+        "gpu_launches": K * moe.forward_launches(layer.cfg, wl.T),
+        "clocks": clocks,
+    }
+    return res
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle (reference arm and cpu_baseline leg)
+# ----------------------------------------------------------------------------
+def oracle_sample(wl, n_tokens: int):
+    """Host inputs for the oracle on the first n_tokens of the workload: router
+    weights, and the routed experts those tokens select plus the shared one,
+    packed by the oracle's own quantiser (untimed set-up)."""
+    from oracle import oracle as orc
+    from quantized_routed_expert_group_b200 import synth
+    s = wl.shape
+    x = synth.make_x(wl)[:n_tokens]
+    Wr, bias = synth.make_router_w(wl), synth.make_bias(wl)
+    idx, _ = orc.router(x, Wr, bias, s.n_groups, s.topk_groups, s.top_k, s.rsf)
+    routed = {}
+    for e in sorted(set(idx.reshape(-1).tolist())):
+        routed[e] = orc.pack_expert(*(synth.make_expert_matrix(wl, e, m) for m in range(3)), s.wbits)
+    shared = orc.pack_expert(*(synth.make_expert_matrix(wl, 0, m, True) for m in range(3)), s.wbits) \
+        if s.n_shared else None
+    return x, Wr, bias, routed, shared
+
+
+def time_oracle(wl, n_tokens: int, budget_s: float, max_steps: int | None = None, warmup: int = 0):
+    from oracle import oracle as orc
+    x, Wr, bias, routed, shared = oracle_sample(wl, n_tokens)
+    for _ in range(warmup):
+        orc.layer_forward(wl.shape, x, Wr, bias, routed, shared)
+    times = []
+    t_start = time.perf_counter()
+    while True:
+        t0 = time.perf_counter()
+        orc.layer_forward(wl.shape, x, Wr, bias, routed, shared)
+        times.append(time.perf_counter() - t0)
+        if max_steps is not None and len(times) >= max_steps:
+            break
+        if time.perf_counter() - t_start >= budget_s:
+            break
+    return times, orc.num_threads()
+
+
+def cpu_baseline(wl, budget_s: float = 12.0) -> dict:
+    n_tok = 1
+    times, cores = time_oracle(wl, n_tok, budget_s)
+    tps = n_tok * len(times) / sum(times)
+    return {"value": round(tps, 4), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {n_tok} token(s) of {wl.name}, {len(times)} forward(s) of the C oracle "
+                      f"(plain C, fp64 sums, OpenMP over output rows), {sum(times):.1f} s"}
+
+
+def run_reference(args) -> dict | None:
+    from quantized_routed_expert_group_b200 import synth
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    wl = synth.WORKLOADS[args.workload]
+    # each step is the oracle's forward of one token of the workload; the run
+    # stops after the requested steps or ~3 minutes, whichever comes first
+    times, cores = time_oracle(wl, 1, budget_s=180.0, max_steps=args.steps, warmup=min(args.warmup, 1))
+    K = len(times)
+    total = sum(times)
+    value = K / total
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "steps_requested": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total / K * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": wl.name, "tokens": wl.T, "hidden": wl.shape.hidden, "inter": wl.shape.inter,
+                   "experts": wl.shape.n_experts, "weights": f"int{wl.shape.wbits}",
+                   "parallelism": "host cores (OpenMP)"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"one token of {wl.name} per step, {K} steps"},
+        "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        res = run_reference(args)
+    else:
+        res = run_ours(args)
+        if res is not None and res["n_gpus"] == 1 and not args.no_cpu_baseline:
+            from quantized_routed_expert_group_b200 import synth
+            res["cpu_baseline"] = cpu_baseline(synth.WORKLOADS[args.workload])
+    if res is not None:
+        print(json.dumps(res), flush=True)
+    try:
+        import torch.distributed as dist
+        if dist.is_available() and dist.is_initialized():
+            dist.destroy_process_group()
+    except Exception:
+        pass
+
+
+if __name__ == "__main__":
+    main()

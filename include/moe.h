@@ -1,0 +1,233 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) quantised mixture-of-experts layer.
+ *
+ * One MoE layer forward of the GLM-5.2 744B model as run by the colibri
+ * engine: DeepSeek-V3-style sigmoid router (noaux_tc grouped top-k with a
+ * correction bias, routed_scaling_factor, one shared expert) -> batch-union
+ * bucketing of tokens by expert -> SwiGLU experts whose int8 / packed int4
+ * weights carry per-row fp32 scales and are dequantised on use, fed by Q8_0
+ * int8 activations through integer dot products -> weighted combine.
+ *
+ * Sources, by page title and section:
+ *  [GN] GeekNews "Show HN: 느린 컴퓨터에서 GLM 5.2 실행하기" -- §구현된 주요 기능
+ *       (router, shared expert, quantisation kernels, integer-dot kernel with
+ *       Q8_0-style int8 activations, batch-union MoE), §디스크 스트리밍 기반 MoE
+ *       실행 방식 (~19 MB per int4 expert).
+ *  [WP] wpnews.pro "Colibri — รัน GLM-5.2 (744B MoE) บนเครื่อง 25GB RAM ด้วย
+ *       Pure C ไฟล์เดียว" -- spec table (256 experts, 8 active + 1 shared,
+ *       Router: DeepSeek-V3-style sigmoid (noaux_tc)), kernel table (int8
+ *       Q8_0-style; int4 packed, dequant-on-use; routing matmul in f32),
+ *       "Batch-Union MoE".
+ *
+ * Conventions for every entry point:
+ *  - Pointers are DEVICE pointers unless the name says host; the caller owns
+ *    all memory.  Arrays are dense, row-major.  Calls are asynchronous on
+ *    `stream` (a cudaStream_t passed as void*; NULL = legacy default stream)
+ *    unless stated otherwise.
+ *  - Arguments are validated on the host before anything is launched; a bad
+ *    argument returns MOE_EINVAL / MOE_EUNSUPPORTED and launches nothing.  A
+ *    failed launch returns MOE_ECUDA.  No call allocates device memory on the
+ *    forward path, and no call throws.
+ *  - Floating point: fp32 inputs and outputs; no fast-math anywhere.
+ *  - Non-finite activations or weights give undefined (but memory-safe)
+ *    results; the CPU test oracle rejects them.
+ *  - Concurrent calls are safe as long as each has its own workspace.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_EINVAL = -1,       /* null / misaligned pointer, negative or inconsistent size */
+    MOE_EUNSUPPORTED = -2, /* well-formed but outside what the kernels support */
+    MOE_EWORKSPACE = -3,   /* workspace smaller than moe_workspace_bytes() */
+    MOE_ECUDA = -4,        /* a CUDA runtime call or kernel launch failed */
+    MOE_EDEVICE = -5       /* a kernel recorded a fault (see moe_get_device_error) */
+} moe_status;
+
+/* Layer hyper-parameters.  The GLM-5.2 layer is hidden 6144, inter 2048,
+ * 256 experts in 8 groups, top-4 groups, top-8, 1 shared, rsf 2.5.
+ * Supported: hidden and inter multiples of 32 (up to 16384); n_experts <= 1024
+ * and a multiple of n_groups; 2 <= n_experts/n_groups; 1 <= topk_groups <=
+ * n_groups <= 32; 1 <= top_k <= min(32, topk_groups * n_experts / n_groups);
+ * n_shared 0 or 1; wbits 8 or 4. */
+typedef struct {
+    int hidden;
+    int inter;
+    int n_experts;
+    int n_groups;
+    int topk_groups;
+    int top_k;
+    int n_shared;
+    float routed_scaling_factor;
+    int wbits;
+} moe_config;
+
+/* Packed expert weights for n experts, laid out expert-major:
+ *   w_gate, w_up : [n][inter][hidden * wbits / 8] bytes
+ *   w_down       : [n][hidden][inter * wbits / 8] bytes
+ *   s_gate, s_up : [n][inter] fp32 row scales;  s_down : [n][hidden]
+ * Codes are two's complement; int4 packs element 2j in the low nibble and
+ * 2j+1 in the high nibble of byte j ([GN] quantisation-kernel bullet: int8 /
+ * packed int4 / packed int2 with per-row scales; the bit layout is this
+ * library's).  Weight pointers must be 16-byte aligned, scale pointers
+ * 4-byte aligned. */
+typedef struct {
+    const uint8_t *w_gate;
+    const uint8_t *w_up;
+    const uint8_t *w_down;
+    const float *s_gate;
+    const float *s_up;
+    const float *s_down;
+} moe_experts;
+
+/* Q8_0 activation quantiser ([GN] integer-dot kernel bullet; [WP] kernel table
+ * "int8 (Q8_0-style)").  For each block of 32 consecutive values of each of the
+ * n_rows rows of x [n_rows][cols]: d = amax/127 (fp32 IEEE divide), q =
+ * round-half-away-from-zero(x * (1/d)) in [-127, 127]; a block with amax below
+ * FLT_MIN stores d = 0, q = 0.  Outputs q [n_rows][cols] int8 and d
+ * [n_rows][cols/32] fp32.  cols must be a multiple of 32; x 16-byte aligned. */
+int moe_quantize_act_q8_0(const float *x, int64_t n_rows, int cols, int8_t *q, float *d, void *stream);
+
+/* Per-row symmetric weight quantiser and packer (the converter's requantise
+ * step; [GN] §구현된 주요 기능, offline converter bullet).  For each row of
+ * w [rows][cols] fp32: s = amax / qmax (qmax 127 for int8, 7 for int4, 1 for
+ * int2), code = round-half-away(w * (1/s)) clamped to [-2^(wbits-1), qmax],
+ * s = 0 and codes 0 when amax < FLT_MIN.  Outputs packed
+ * [rows][cols * wbits / 8] and scales [rows].  wbits is 8, 4 or 2; cols a
+ * multiple of 32. */
+int moe_pack_weights(const float *w, int64_t rows, int cols, int wbits, uint8_t *packed, float *scales,
+                     void *stream);
+
+/* Bytes of device workspace that moe_router_select needs for T tokens. */
+size_t moe_router_workspace_bytes(const moe_config *cfg, int T);
+
+/* Router: DeepSeek-V3-style sigmoid with noaux_tc grouped top-k ([GN]
+ * §구현된 주요 기능; [WP] spec table, Router row).  For each token t of
+ * x [T][hidden]:
+ *   logit[e] = sum_j x[t,j] * router_w[e,j]   (fp32 inputs, fp64 sum)
+ *   s[e] = sigmoid(logit[e]), c[e] = s[e] + router_bias[e]      (fp64)
+ *   group score = sum of the two largest c in the group; keep the topk_groups
+ *   best groups; pick the top_k largest c among their experts (ties: lower
+ *   index first).  idx[t][j] (int32) lists them in descending c order and
+ *   w[t][j] = s / sum(s) * routed_scaling_factor (fp32, unbiased s).
+ * router_w [n_experts][hidden] fp32, router_bias [n_experts] fp32.
+ * workspace: >= moe_router_workspace_bytes(cfg, T) bytes, 256-byte aligned. */
+int moe_router_select(const moe_config *cfg, const float *x, int T, const float *router_w,
+                      const float *router_bias, int32_t *idx, float *w, void *workspace, size_t ws_bytes,
+                      void *stream);
+
+/* Batch-union bucketing ([GN] "Batch-union MoE"; [WP] "Batch-Union MoE"):
+ * a stable counting sort of the T*top_k (token, slot) pairs of idx [T][top_k]
+ * by expert.  counts [n_experts], offsets [n_experts+1] (exclusive prefix
+ * sums, offsets[n_experts] = T*top_k) and perm [T*top_k], where perm lists
+ * t*top_k + j for expert 0's pairs in increasing t, then expert 1's, etc.
+ * Supports n_experts * ceil(T/32) <= 24576 (T <= 3072 at 256 experts). */
+int moe_bucket_tokens(const moe_config *cfg, const int32_t *idx, int T, int32_t *counts, int32_t *offsets,
+                      int32_t *perm, void *stream);
+
+/* Bytes of device workspace that moe_layer_forward needs for up to T_max
+ * tokens (0 on an invalid config). */
+size_t moe_workspace_bytes(const moe_config *cfg, int T_max);
+
+/* One MoE layer forward ([GN] §구현된 주요 기능; [WP] spec table, kernel table,
+ * "Batch-Union MoE"):
+ *   route (as moe_router_select), bucket (as moe_bucket_tokens), then for every
+ *   selected expert e and token t routed to it, and for the shared expert on
+ *   every token:
+ *     g = Wg.x, u = Wu.x   with x as Q8_0 (per-block int32 dots, then
+ *                          s_row * sum_b d_b * isum_b)
+ *     h = silu(g) * u, quantised to Q8_0, y = Wd.h  (same integer-dot form)
+ *   out[t] = sum_j w[t,j] * y_{idx[t,j]}(t) + y_shared(t)   (no residual).
+ * x [T][hidden] fp32 (16-byte aligned), out [T][hidden] fp32.  routed holds
+ * n_experts experts, shared n_shared (ignored when n_shared == 0).
+ * workspace: >= moe_workspace_bytes(cfg, T) bytes, 256-byte aligned; it holds
+ * every intermediate of the call (see moe_workspace_view) and its error word.
+ * 0 <= T; T = 0 returns MOE_OK without launching. */
+int moe_layer_forward(const moe_config *cfg, const float *x, int T, const float *router_w,
+                      const float *router_bias, const moe_experts *routed, const moe_experts *shared,
+                      float *out, void *workspace, size_t ws_bytes, void *stream);
+
+/* moe_layer_forward with HOST activations: copies x_host [T][hidden] to the
+ * workspace, runs the forward, copies the result to out_host [T][hidden] and
+ * synchronises `stream`.  Host buffers should be pinned (cudaHostAlloc) for
+ * asynchronous copies; pageable memory works but is slower.  Weights and the
+ * workspace are device memory as for moe_layer_forward. */
+int moe_layer_forward_host(const moe_config *cfg, const float *x_host, int T, const float *router_w,
+                           const float *router_bias, const moe_experts *routed, const moe_experts *shared,
+                           float *out_host, void *workspace, size_t ws_bytes, void *stream);
+
+/* Device pointers to the intermediates a moe_layer_forward call leaves in its
+ * workspace (valid after the call completes, until the next call on the same
+ * workspace).  Slots: routed (token, slot) pairs occupy bucket positions
+ * 0 .. T*top_k-1 (the order of perm); the shared expert of token t is slot
+ * T*top_k + t. */
+typedef struct {
+    int8_t *xq;        /* [T][hidden]   Q8_0 codes of x */
+    float *xd;         /* [T][hidden/32] Q8_0 scales of x */
+    int32_t *idx;      /* [T][top_k]    selected experts */
+    float *w;          /* [T][top_k]    combine weights */
+    int32_t *counts;   /* [n_experts] */
+    int32_t *offsets;  /* [n_experts+1] */
+    int32_t *perm;     /* [T*top_k] */
+    int8_t *hq;        /* [slots][inter]    Q8_0 codes of h per slot */
+    float *hd;         /* [slots][inter/32] Q8_0 scales of h per slot */
+    float *y;          /* [slots][hidden]   expert outputs per slot (unweighted) */
+    int32_t *error;    /* device error word (0 = none) */
+} moe_workspace_layout;
+
+int moe_workspace_view(const moe_config *cfg, int T, void *workspace, size_t ws_bytes,
+                       moe_workspace_layout *view);
+
+/* Per-block int32 dot products of one packed matrix with Q8_0 codes, computed
+ * by the same device routine as the expert kernels ([GN] integer-dot kernel):
+ * out[t][r][b] = sum_{i<32} code(W[r, 32b+i]) * q[t, 32b+i] for W packed
+ * [rows][cols * wbits / 8] (wbits 8 or 4) and q [n][cols] int8. */
+int moe_block_dots(const uint8_t *packed, int64_t rows, int cols, int wbits, const int8_t *q, int n,
+                   int32_t *out, void *stream);
+
+/* Synchronises `stream` and reads the workspace's device error word into
+ * *code (0 = none).  Returns MOE_OK when it is 0, MOE_EDEVICE otherwise.
+ * Codes: 1 = an index out of range reached a kernel, 2 = a device-side wait
+ * ran out of iterations. */
+int moe_get_device_error(void *workspace, void *stream, int32_t *code);
+
+/* Device copy of the seeded input generator (SplitMix64, counter-based; see
+ * the package's synth module): out[i] = sigma * z(seed, tid, offset + i) with z
+ * the centred Irwin-Hall sum of twelve 16-bit uniforms.  Used to draw
+ * multi-GB synthetic expert weights directly in HBM; bit-identical to the
+ * host generator. */
+int moe_synth_normal(uint64_t seed, uint64_t tid, int64_t offset, int64_t n, float sigma, float *out,
+                     void *stream);
+
+/* Tracing hook: CUDA events at the phase boundaries of moe_layer_forward.
+ * events points to MOE_PROFILE_PHASES + 1 cudaEvent_t handles (passed as
+ * void*), or is NULL to switch tracing off; the setting belongs to the calling
+ * host thread.  While it is set, every forward issued from that thread records
+ * events[0] on its stream before its first launch and events[i] after phase i:
+ *   1 Q8_0 of x + router, 2 bucketing, 3 expert gate/up (+ SiLU, Q8_0 of h),
+ *   4 expert down, 5 combine.
+ * The caller keeps the events alive until they have completed.  n_events must
+ * be MOE_PROFILE_PHASES + 1 (or 0 with events NULL). */
+#define MOE_PROFILE_PHASES 5
+int moe_profile_events(void *const *events, int n_events);
+
+/* Number of kernel launches one moe_layer_forward with T tokens issues
+ * (0 for T = 0; negative status on an invalid config). */
+int moe_forward_launches(const moe_config *cfg, int T);
+
+/* Human-readable name of a status code. */
+const char *moe_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,346 @@
+// moe_api.cu -- the library's C ABI (include/moe.h): argument validation,
+// workspace layout and the launch sequence of one MoE layer forward.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "moe_internal.h"
+
+#define MOE_API extern "C" __attribute__((visibility("default")))
+
+namespace moe {
+
+static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+Layout make_layout(const moe_config& c, int T) {
+    Layout L;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align256(off + bytes);
+        return o;
+    };
+    const size_t t = (size_t)T, H = (size_t)c.hidden, I = (size_t)c.inter, E = (size_t)c.n_experts,
+                 k = (size_t)c.top_k;
+    const size_t slots = t * k + t * (size_t)c.n_shared;
+    L.err = take(64);
+    L.xin = take(t * H * 4);
+    L.outbuf = take(t * H * 4);
+    L.xq = take(t * H);
+    L.xd = take(t * (H / 32) * 4);
+    L.logits = take(t * E * 8);
+    L.idx = take(t * k * 4);
+    L.w = take(t * k * 4);
+    L.counts = take(E * 4);
+    L.offsets = take((E + 1) * 4);
+    L.perm = take(t * k * 4);
+    L.inv_perm = take(t * k * 4);
+    L.active = take((E + 2) * 4);
+    L.hq = take(slots * I);
+    L.hd = take(slots * (I / 32) * 4);
+    L.y = take(slots * H * 4);
+    L.total = off;
+    return L;
+}
+
+const DeviceInfo& device_info() {
+    static DeviceInfo infos[64];
+    static bool done[64];
+    static std::mutex mu;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!done[dev]) {
+        DeviceInfo d{148, 227 * 1024};
+        cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
+        cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        infos[dev] = d;
+        done[dev] = true;
+    }
+    return infos[dev];
+}
+
+static bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+static int check_config(const moe_config* c) {
+    if (!c) return MOE_EINVAL;
+    if (c->hidden <= 0 || c->inter <= 0 || c->n_experts <= 0 || c->n_groups <= 0 || c->topk_groups <= 0 ||
+        c->top_k <= 0 || c->n_shared < 0)
+        return MOE_EINVAL;
+    if (c->n_experts % c->n_groups != 0 || c->topk_groups > c->n_groups) return MOE_EINVAL;
+    if (c->top_k > c->topk_groups * (c->n_experts / c->n_groups)) return MOE_EINVAL;
+    if (!std::isfinite(c->routed_scaling_factor)) return MOE_EINVAL;
+    if (c->hidden % 32 || c->inter % 32 || c->hidden > 16384 || c->inter > 16384) return MOE_EUNSUPPORTED;
+    if (c->n_experts > 1024 || c->n_groups > 32 || c->n_experts / c->n_groups < 2 || c->top_k > 32 ||
+        c->n_shared > 1)
+        return MOE_EUNSUPPORTED;
+    if (c->wbits != 4 && c->wbits != 8) return MOE_EUNSUPPORTED;
+    return MOE_OK;
+}
+
+static int check_experts(const moe_experts* ex) {
+    if (!ex) return MOE_EINVAL;
+    if (!ex->w_gate || !ex->w_up || !ex->w_down || !ex->s_gate || !ex->s_up || !ex->s_down) return MOE_EINVAL;
+    if (!aligned(ex->w_gate, 16) || !aligned(ex->w_up, 16) || !aligned(ex->w_down, 16)) return MOE_EINVAL;
+    if (!aligned(ex->s_gate, 4) || !aligned(ex->s_up, 4) || !aligned(ex->s_down, 4)) return MOE_EINVAL;
+    return MOE_OK;
+}
+
+static int status_of(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ECUDA; }
+
+// Per-thread tracing events (see moe_profile_events).
+static thread_local cudaEvent_t g_trace[MOE_PROFILE_PHASES + 1];
+static thread_local bool g_trace_on = false;
+
+static cudaError_t trace(int i, cudaStream_t s) {
+    return g_trace_on ? cudaEventRecord(g_trace[i], s) : cudaSuccess;
+}
+
+static int check_bucket_fits(const moe_config& c, int T) {
+    if (T > (1 << 20)) return MOE_EUNSUPPORTED;
+    const size_t words = (size_t)c.n_experts * (size_t)((T + 31) / 32);
+    if (words > 24576) return MOE_EUNSUPPORTED;
+    if (bucket_smem_bytes(c, T) > (size_t)device_info().max_smem_optin) return MOE_EUNSUPPORTED;
+    return MOE_OK;
+}
+
+// The forward on a device-resident x; used by both public forwards.
+static int forward_device(const moe_config& c, const float* x, int T, const float* router_w,
+                          const float* router_bias, const moe_experts& routed, const moe_experts* shared,
+                          float* out, char* ws, const Layout& L, cudaStream_t s) {
+    int32_t* err = reinterpret_cast<int32_t*>(ws + L.err);
+    if (trace(0, s) != cudaSuccess) return MOE_ECUDA;
+    if (cudaMemsetAsync(err, 0, 64, s) != cudaSuccess) return MOE_ECUDA;
+    int8_t* xq = reinterpret_cast<int8_t*>(ws + L.xq);
+    float* xd = reinterpret_cast<float*>(ws + L.xd);
+    int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
+    float* w = reinterpret_cast<float*>(ws + L.w);
+    int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
+    int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+    int32_t* perm = reinterpret_cast<int32_t*>(ws + L.perm);
+    int32_t* inv_perm = reinterpret_cast<int32_t*>(ws + L.inv_perm);
+    int32_t* active = reinterpret_cast<int32_t*>(ws + L.active);
+    int st = status_of(launch_quantize_q8_0(x, T, c.hidden, xq, xd, s));
+    if (st) return st;
+    st = status_of(launch_router(c, x, T, router_w, router_bias, reinterpret_cast<double*>(ws + L.logits), idx, w, s));
+    if (!st) st = status_of(trace(1, s));
+    if (st) return st;
+    st = status_of(launch_bucket(c, idx, T, counts, offsets, perm, inv_perm, active, err, s));
+    if (!st) st = status_of(trace(2, s));
+    if (st) return st;
+    ExpertArgs a;
+    a.cfg = &c;
+    a.T = T;
+    a.xq = xq;
+    a.xd = xd;
+    a.w = w;
+    a.offsets = offsets;
+    a.perm = perm;
+    a.inv_perm = inv_perm;
+    a.active = active;
+    a.routed = routed;
+    a.shared = shared ? *shared : routed;
+    a.hq = reinterpret_cast<int8_t*>(ws + L.hq);
+    a.hd = reinterpret_cast<float*>(ws + L.hd);
+    a.y = reinterpret_cast<float*>(ws + L.y);
+    a.out = out;
+    a.err = err;
+    return status_of(launch_experts(a, s, g_trace_on ? &g_trace[3] : nullptr));
+}
+
+static int check_forward_args(const moe_config* cfg, const void* x, int T, const float* router_w,
+                              const float* router_bias, const moe_experts* routed, const moe_experts* shared,
+                              const void* out, const void* workspace, size_t ws_bytes, Layout* L) {
+    int st = check_config(cfg);
+    if (st) return st;
+    if (T < 0) return MOE_EINVAL;
+    if (T > 0 && (!x || !out)) return MOE_EINVAL;  // empty batches may pass null activations
+    if (!router_w || !router_bias || !workspace) return MOE_EINVAL;
+    if (!aligned(router_w, 16) || !aligned(router_bias, 4) || !aligned(workspace, 256)) return MOE_EINVAL;
+    st = check_experts(routed);
+    if (st) return st;
+    if (cfg->n_shared) {
+        st = check_experts(shared);
+        if (st) return st;
+    }
+    st = check_bucket_fits(*cfg, T);
+    if (st) return st;
+    *L = make_layout(*cfg, T);
+    if (ws_bytes < L->total) return MOE_EWORKSPACE;
+    return MOE_OK;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+MOE_API int moe_quantize_act_q8_0(const float* x, int64_t n_rows, int cols, int8_t* q, float* d, void* stream) {
+    if (n_rows < 0 || cols <= 0 || cols % 32) return MOE_EINVAL;
+    if (n_rows == 0) return MOE_OK;
+    if (!x || !q || !d || !aligned(x, 4) || !aligned(d, 4)) return MOE_EINVAL;
+    return status_of(launch_quantize_q8_0(x, n_rows, cols, q, d, (cudaStream_t)stream));
+}
+
+MOE_API int moe_pack_weights(const float* w, int64_t rows, int cols, int wbits, uint8_t* packed, float* scales,
+                             void* stream) {
+    if (rows < 0 || cols <= 0 || cols % 32) return MOE_EINVAL;
+    if (wbits != 8 && wbits != 4 && wbits != 2) return MOE_EUNSUPPORTED;
+    if (rows == 0) return MOE_OK;
+    if (!w || !packed || !scales || !aligned(w, 16) || !aligned(packed, 16) || !aligned(scales, 4))
+        return MOE_EINVAL;
+    return status_of(launch_pack_weights(w, rows, cols, wbits, packed, scales, (cudaStream_t)stream));
+}
+
+MOE_API size_t moe_router_workspace_bytes(const moe_config* cfg, int T) {
+    if (check_config(cfg) != MOE_OK || T < 0) return 0;
+    return align256((size_t)T * (size_t)cfg->n_experts * sizeof(double));
+}
+
+MOE_API int moe_router_select(const moe_config* cfg, const float* x, int T, const float* router_w,
+                              const float* router_bias, int32_t* idx, float* w, void* workspace, size_t ws_bytes,
+                              void* stream) {
+    int st = check_config(cfg);
+    if (st) return st;
+    if (T < 0) return MOE_EINVAL;
+    if (T == 0) return MOE_OK;
+    if (!x || !router_w || !router_bias || !idx || !w || !workspace) return MOE_EINVAL;
+    if (!aligned(x, 16) || !aligned(router_w, 16) || !aligned(workspace, 256)) return MOE_EINVAL;
+    if (ws_bytes < moe_router_workspace_bytes(cfg, T)) return MOE_EWORKSPACE;
+    return status_of(launch_router(*cfg, x, T, router_w, router_bias, reinterpret_cast<double*>(workspace), idx,
+                                   w, (cudaStream_t)stream));
+}
+
+MOE_API int moe_bucket_tokens(const moe_config* cfg, const int32_t* idx, int T, int32_t* counts, int32_t* offsets,
+                              int32_t* perm, void* stream) {
+    int st = check_config(cfg);
+    if (st) return st;
+    if (T < 0) return MOE_EINVAL;
+    if (!counts || !offsets || (T > 0 && (!idx || !perm))) return MOE_EINVAL;
+    st = check_bucket_fits(*cfg, T);
+    if (st) return st;
+    // inv_perm and the active-expert list are internal to the forward: not written here.
+    return status_of(launch_bucket(*cfg, idx, T, counts, offsets, perm, nullptr, nullptr, nullptr,
+                                   (cudaStream_t)stream));
+}
+
+MOE_API size_t moe_workspace_bytes(const moe_config* cfg, int T_max) {
+    if (check_config(cfg) != MOE_OK || T_max < 0) return 0;
+    return make_layout(*cfg, T_max).total;
+}
+
+MOE_API int moe_layer_forward(const moe_config* cfg, const float* x, int T, const float* router_w,
+                              const float* router_bias, const moe_experts* routed, const moe_experts* shared,
+                              float* out, void* workspace, size_t ws_bytes, void* stream) {
+    Layout L;
+    int st = check_forward_args(cfg, x, T, router_w, router_bias, routed, shared, out, workspace, ws_bytes, &L);
+    if (st) return st;
+    if (T == 0) return MOE_OK;
+    if (!aligned(x, 16) || !aligned(out, 4)) return MOE_EINVAL;
+    return forward_device(*cfg, x, T, router_w, router_bias, *routed, cfg->n_shared ? shared : nullptr, out,
+                          static_cast<char*>(workspace), L, (cudaStream_t)stream);
+}
+
+MOE_API int moe_layer_forward_host(const moe_config* cfg, const float* x_host, int T, const float* router_w,
+                                   const float* router_bias, const moe_experts* routed, const moe_experts* shared,
+                                   float* out_host, void* workspace, size_t ws_bytes, void* stream) {
+    Layout L;
+    int st = check_forward_args(cfg, x_host, T, router_w, router_bias, routed, shared, out_host, workspace,
+                                ws_bytes, &L);
+    if (st) return st;
+    if (T == 0) return MOE_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    char* ws = static_cast<char*>(workspace);
+    const size_t bytes = (size_t)T * cfg->hidden * sizeof(float);
+    float* xdev = reinterpret_cast<float*>(ws + L.xin);
+    float* odev = reinterpret_cast<float*>(ws + L.outbuf);
+    if (cudaMemcpyAsync(xdev, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return MOE_ECUDA;
+    st = forward_device(*cfg, xdev, T, router_w, router_bias, *routed, cfg->n_shared ? shared : nullptr, odev, ws, L,
+                        s);
+    if (st) return st;
+    if (cudaMemcpyAsync(out_host, odev, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ECUDA;
+    return status_of(cudaStreamSynchronize(s));
+}
+
+MOE_API int moe_workspace_view(const moe_config* cfg, int T, void* workspace, size_t ws_bytes,
+                               moe_workspace_layout* view) {
+    int st = check_config(cfg);
+    if (st) return st;
+    if (T < 0 || !workspace || !view) return MOE_EINVAL;
+    const Layout L = make_layout(*cfg, T);
+    if (ws_bytes < L.total) return MOE_EWORKSPACE;
+    char* ws = static_cast<char*>(workspace);
+    view->xq = reinterpret_cast<int8_t*>(ws + L.xq);
+    view->xd = reinterpret_cast<float*>(ws + L.xd);
+    view->idx = reinterpret_cast<int32_t*>(ws + L.idx);
+    view->w = reinterpret_cast<float*>(ws + L.w);
+    view->counts = reinterpret_cast<int32_t*>(ws + L.counts);
+    view->offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+    view->perm = reinterpret_cast<int32_t*>(ws + L.perm);
+    view->hq = reinterpret_cast<int8_t*>(ws + L.hq);
+    view->hd = reinterpret_cast<float*>(ws + L.hd);
+    view->y = reinterpret_cast<float*>(ws + L.y);
+    view->error = reinterpret_cast<int32_t*>(ws + L.err);
+    return MOE_OK;
+}
+
+MOE_API int moe_block_dots(const uint8_t* packed, int64_t rows, int cols, int wbits, const int8_t* q, int n,
+                           int32_t* out, void* stream) {
+    if (rows < 0 || n < 0 || cols <= 0 || cols % 32) return MOE_EINVAL;
+    if (wbits != 4 && wbits != 8) return MOE_EUNSUPPORTED;
+    if (rows == 0 || n == 0) return MOE_OK;
+    if (!packed || !q || !out || !aligned(packed, 16) || !aligned(q, 16) || !aligned(out, 4)) return MOE_EINVAL;
+    return status_of(launch_block_dots(packed, rows, cols, wbits, q, n, out, (cudaStream_t)stream));
+}
+
+MOE_API int moe_get_device_error(void* workspace, void* stream, int32_t* code) {
+    if (!workspace || !code) return MOE_EINVAL;
+    cudaStream_t s = (cudaStream_t)stream;
+    int32_t v = 0;
+    if (cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ECUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ECUDA;
+    *code = v;
+    return v == 0 ? MOE_OK : MOE_EDEVICE;
+}
+
+MOE_API int moe_synth_normal(uint64_t seed, uint64_t tid, int64_t offset, int64_t n, float sigma, float* out,
+                             void* stream) {
+    if (n < 0 || offset < 0) return MOE_EINVAL;
+    if (n == 0) return MOE_OK;
+    if (!out || !aligned(out, 4)) return MOE_EINVAL;
+    return status_of(launch_synth_normal(seed, tid, offset, n, sigma, out, (cudaStream_t)stream));
+}
+
+MOE_API int moe_profile_events(void* const* events, int n_events) {
+    if (!events) {
+        if (n_events != 0) return MOE_EINVAL;
+        g_trace_on = false;
+        return MOE_OK;
+    }
+    if (n_events != MOE_PROFILE_PHASES + 1) return MOE_EINVAL;
+    for (int i = 0; i <= MOE_PROFILE_PHASES; ++i) {
+        if (!events[i]) return MOE_EINVAL;
+        g_trace[i] = static_cast<cudaEvent_t>(events[i]);
+    }
+    g_trace_on = true;
+    return MOE_OK;
+}
+
+MOE_API int moe_forward_launches(const moe_config* cfg, int T) {
+    const int st = check_config(cfg);
+    if (st) return st;
+    if (T < 0) return MOE_EINVAL;
+    return T == 0 ? 0 : kForwardLaunches;
+}
+
+MOE_API const char* moe_status_string(int status) {
+    switch (status) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_EINVAL: return "MOE_EINVAL: invalid argument";
+        case MOE_EUNSUPPORTED: return "MOE_EUNSUPPORTED: unsupported shape or bit width";
+        case MOE_EWORKSPACE: return "MOE_EWORKSPACE: workspace too small";
+        case MOE_ECUDA: return "MOE_ECUDA: CUDA call failed";
+        case MOE_EDEVICE: return "MOE_EDEVICE: a kernel recorded a fault";
+        default: return "unknown moe status";
+    }
+}

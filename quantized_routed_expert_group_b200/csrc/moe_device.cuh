@@ -1,0 +1,199 @@
+// moe_device.cuh -- device helpers shared by the MoE layer kernels (sm_100a).
+//
+// The arithmetic here is the integer-dot form of the colibri engine's expert
+// matmuls (GeekNews "Show HN: 느린 컴퓨터에서 GLM 5.2 실행하기", §구현된 주요 기능:
+// Q8_0-style int8 activations times int8 / packed int4 weights with per-row
+// scales, dequantised on use), restated for CUDA cores: __dp4a on four int8
+// lanes instead of AVX2 maddubs.
+#pragma once
+
+#include <cfloat>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace moe {
+
+constexpr int kQBlock = 32;           // Q8_0 block length
+constexpr unsigned kFull = 0xffffffffu;
+
+// Error codes written to the workspace error word.
+constexpr int kErrIndex = 1;
+constexpr int kErrTimeout = 2;
+
+__device__ __forceinline__ void set_error(int32_t* err, int code) {
+    if (err) atomicCAS(reinterpret_cast<int*>(err), 0, code);
+}
+
+// 128-bit read-only streaming load: weights are read once per call, so they
+// bypass L1 and ask L2 for 256-byte sector prefetch.
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+    uint4 r;
+    asm("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p));
+    return r;
+}
+
+// 128-bit read-only load that may stay in L1 (activations, reused across rows).
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+    return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+// Activation block of 32 int8 codes, kept in the order the weight format wants:
+// for int8 weights the natural order (8 words of 4 codes), for int4 weights the
+// even and odd elements of each group of 8 split apart, matching the low and
+// high nibbles of one packed 32-bit weight word.
+struct ActBlock {
+    uint32_t v[8];
+};
+
+__device__ __forceinline__ ActBlock act_natural(uint4 lo, uint4 hi) {
+    ActBlock a;
+    a.v[0] = lo.x; a.v[1] = lo.y; a.v[2] = lo.z; a.v[3] = lo.w;
+    a.v[4] = hi.x; a.v[5] = hi.y; a.v[6] = hi.z; a.v[7] = hi.w;
+    return a;
+}
+
+// Natural -> nibble order: word pair (x[8k..8k+3], x[8k+4..8k+7]) becomes
+// (x[8k], x[8k+2], x[8k+4], x[8k+6]) and (x[8k+1], x[8k+3], x[8k+5], x[8k+7]).
+__device__ __forceinline__ ActBlock act_nibble_order(uint4 lo, uint4 hi) {
+    const uint32_t n[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+    ActBlock a;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        a.v[2 * k] = __byte_perm(n[2 * k], n[2 * k + 1], 0x6420);
+        a.v[2 * k + 1] = __byte_perm(n[2 * k], n[2 * k + 1], 0x7531);
+    }
+    return a;
+}
+
+// Exact int32 dot of one packed-int4 block (16 bytes = 32 codes, element 2j in
+// the low nibble of byte j) with a nibble-ordered activation block.  Each
+// nibble is moved to the top of its byte, which makes the byte 16 * code as a
+// signed int8; the sum is therefore 16 * dot and the final shift is exact.
+__device__ __forceinline__ int dot_block_i4(uint4 w, const ActBlock& a) {
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    int acc = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int lo16 = static_cast<int>((ww[k] << 4) & 0xF0F0F0F0u);
+        const int hi16 = static_cast<int>(ww[k] & 0xF0F0F0F0u);
+        acc = __dp4a(lo16, static_cast<int>(a.v[2 * k]), acc);
+        acc = __dp4a(hi16, static_cast<int>(a.v[2 * k + 1]), acc);
+    }
+    return acc >> 4;
+}
+
+// Exact int32 dot of one int8 block (32 bytes) with a natural-order block.
+__device__ __forceinline__ int dot_block_i8(uint4 w0, uint4 w1, const ActBlock& a) {
+    int acc = 0;
+    acc = __dp4a(static_cast<int>(w0.x), static_cast<int>(a.v[0]), acc);
+    acc = __dp4a(static_cast<int>(w0.y), static_cast<int>(a.v[1]), acc);
+    acc = __dp4a(static_cast<int>(w0.z), static_cast<int>(a.v[2]), acc);
+    acc = __dp4a(static_cast<int>(w0.w), static_cast<int>(a.v[3]), acc);
+    acc = __dp4a(static_cast<int>(w1.x), static_cast<int>(a.v[4]), acc);
+    acc = __dp4a(static_cast<int>(w1.y), static_cast<int>(a.v[5]), acc);
+    acc = __dp4a(static_cast<int>(w1.z), static_cast<int>(a.v[6]), acc);
+    acc = __dp4a(static_cast<int>(w1.w), static_cast<int>(a.v[7]), acc);
+    return acc;
+}
+
+template <int WBITS>
+__device__ __forceinline__ ActBlock load_act_block(const int8_t* q) {
+    const uint4 lo = ld_nc_v4(q);
+    const uint4 hi = ld_nc_v4(q + 16);
+    if constexpr (WBITS == 4) return act_nibble_order(lo, hi);
+    else return act_natural(lo, hi);
+}
+
+// One weight block of a row: 32 codes = 16 bytes (int4) or 32 bytes (int8).
+template <int WBITS>
+struct WBlock {
+    uint4 a, b;
+};
+
+template <int WBITS>
+__device__ __forceinline__ WBlock<WBITS> load_w_block(const uint8_t* row, int blk) {
+    WBlock<WBITS> w;
+    if constexpr (WBITS == 4) {
+        w.a = ld_stream_v4(row + 16 * blk);
+        w.b = make_uint4(0, 0, 0, 0);
+    } else {
+        w.a = ld_stream_v4(row + 32 * blk);
+        w.b = ld_stream_v4(row + 32 * blk + 16);
+    }
+    return w;
+}
+
+template <int WBITS>
+__device__ __forceinline__ int dot_block(const WBlock<WBITS>& w, const ActBlock& a) {
+    if constexpr (WBITS == 4) return dot_block_i4(w.a, a);
+    else return dot_block_i8(w.a, w.b, a);
+}
+
+// Q8_0 of one block held one value per lane: d = amax/127 (IEEE divide),
+// q = round-half-away(v * (1/d)) clamped to [-127, 127]; amax < FLT_MIN
+// gives d = 0, q = 0.  Every lane of the warp must call it.
+__device__ __forceinline__ void q8_0_warp(float v, int8_t& q, float& d) {
+    float a = fabsf(v);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, o));
+    if (!(a >= FLT_MIN)) {
+        d = 0.0f;
+        q = 0;
+        return;
+    }
+    d = __fdiv_rn(a, 127.0f);
+    const float id = __fdiv_rn(1.0f, d);
+    float r = roundf(__fmul_rn(v, id));
+    r = fminf(fmaxf(r, -127.0f), 127.0f);
+    q = static_cast<int8_t>(static_cast<int>(r));
+}
+
+// Butterfly reduction of V per-lane values across the warp (V a power of two,
+// 1 <= V <= 32): afterwards every lane holds the full sum of value index
+// (lane >> (5 - log2 V)).  Costs V - 1 + (5 - log2 V) shuffles instead of
+// 5 V for V independent reductions.
+template <int V>
+__device__ __forceinline__ float warp_reduce_many(float (&v)[V], int lane) {
+    int n = V;
+    int off = 16;
+#pragma unroll
+    for (; n > 1; n >>= 1, off >>= 1) {
+        const bool upper = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < n / 2; ++i) {
+            const float send = upper ? v[i] : v[i + n / 2];
+            const float keep = upper ? v[i + n / 2] : v[i];
+            v[i] = keep + __shfl_xor_sync(kFull, send, off);
+        }
+    }
+    float r = v[0];
+#pragma unroll
+    for (; off > 0; off >>= 1) r += __shfl_xor_sync(kFull, r, off);
+    return r;
+}
+
+template <int V>
+struct Log2 {
+    static constexpr int value = V <= 1 ? 0 : 1 + Log2<V / 2>::value;
+};
+template <>
+struct Log2<1> {
+    static constexpr int value = 0;
+};
+
+// Arg-max over the warp with ties to the lower index.
+__device__ __forceinline__ void warp_argmax(double& v, int& i) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const double ov = __shfl_xor_sync(kFull, v, o);
+        const int oi = __shfl_xor_sync(kFull, i, o);
+        if (ov > v || (ov == v && oi < i)) {
+            v = ov;
+            i = oi;
+        }
+    }
+}
+
+}  // namespace moe

@@ -1,0 +1,81 @@
+// moe_internal.h -- launchers and workspace layout shared by the library's
+// translation units (not part of the public ABI).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// Workspace regions for a call with T tokens.  Every region starts on a
+// 256-byte boundary.  "slots" = T*top_k routed pairs + T*n_shared shared.
+struct Layout {
+    size_t err;        // int32[16]: [0] error word, [1..] counters
+    size_t xin;        // fp32 [T][H]  host-copied activations (forward_host)
+    size_t outbuf;     // fp32 [T][H]  result staged for the host copy
+    size_t xq;         // int8 [T][H]
+    size_t xd;         // fp32 [T][H/32]
+    size_t logits;     // fp64 [T][E]
+    size_t idx;        // int32 [T][k]
+    size_t w;          // fp32 [T][k]
+    size_t counts;     // int32 [E]
+    size_t offsets;    // int32 [E+1]
+    size_t perm;       // int32 [T*k]
+    size_t inv_perm;   // int32 [T*k]
+    size_t active;     // int32 [1 + E + 1]: count, then expert ids (shared = -1 last)
+    size_t hq;         // int8 [slots][I]
+    size_t hd;         // fp32 [slots][I/32]
+    size_t y;          // fp32 [slots][H]
+    size_t total;
+};
+
+Layout make_layout(const moe_config& c, int T);
+
+struct DeviceInfo {
+    int sm_count;
+    int max_smem_optin;
+};
+const DeviceInfo& device_info();
+
+// ---- launchers (return cudaError_t of the launch) ----
+cudaError_t launch_quantize_q8_0(const float* x, int64_t n_rows, int cols, int8_t* q, float* d,
+                                 cudaStream_t s);
+cudaError_t launch_pack_weights(const float* w, int64_t rows, int cols, int wbits, uint8_t* packed,
+                                float* scales, cudaStream_t s);
+cudaError_t launch_router(const moe_config& c, const float* x, int T, const float* router_w,
+                          const float* bias, double* logits, int32_t* idx, float* w, cudaStream_t s);
+cudaError_t launch_bucket(const moe_config& c, const int32_t* idx, int T, int32_t* counts,
+                          int32_t* offsets, int32_t* perm, int32_t* inv_perm, int32_t* active,
+                          int32_t* err, cudaStream_t s);
+size_t bucket_smem_bytes(const moe_config& c, int T);
+
+struct ExpertArgs {
+    const moe_config* cfg;
+    int T;
+    const int8_t* xq;
+    const float* xd;
+    const float* w;
+    const int32_t* offsets;
+    const int32_t* perm;
+    const int32_t* inv_perm;
+    const int32_t* active;
+    moe_experts routed;
+    moe_experts shared;
+    int8_t* hq;
+    float* hd;
+    float* y;
+    float* out;
+    int32_t* err;
+};
+// ev (optional, 3 events): recorded after gate/up, down and combine.
+cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t s, cudaEvent_t const* ev);
+constexpr int kForwardLaunches = 7;  // quantise, logits, select, bucket, gate/up, down, combine
+cudaError_t launch_block_dots(const uint8_t* packed, int64_t rows, int cols, int wbits, const int8_t* q,
+                              int n, int32_t* out, cudaStream_t s);
+cudaError_t launch_synth_normal(uint64_t seed, uint64_t tid, int64_t offset, int64_t n, float sigma,
+                                float* out, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,133 @@
+// moe_quant.cu -- Q8_0 activation quantiser and per-row weight quantiser.
+//
+// Q8_0: GeekNews "Show HN: 느린 컴퓨터에서 GLM 5.2 실행하기", §구현된 주요 기능
+// (integer-dot kernel with Q8_0-style int8 activations); wpnews.pro "Colibri —
+// รัน GLM-5.2 ...", kernel table.  Weight quantiser: same page, quantisation
+// kernel bullet (int8 / packed int4 / packed int2, per-row scales) and the
+// offline converter that requantises the FP8 checkpoint.
+#include "moe_device.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+// One warp per Q8_0 block of 32 values; 8 blocks per CTA, grid-stride.
+__global__ void __launch_bounds__(256) k_quantize_q8_0(const float* __restrict__ x, int64_t nblk,
+                                                       int8_t* __restrict__ q, float* __restrict__ d) {
+    const int lane = threadIdx.x & 31;
+    for (int64_t b = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); b < nblk; b += (int64_t)gridDim.x * 8) {
+        const float v = x[b * kQBlock + lane];
+        int8_t qq;
+        float dd;
+        q8_0_warp(v, qq, dd);
+        q[b * kQBlock + lane] = qq;
+        if (lane == 0) d[b] = dd;
+    }
+}
+
+cudaError_t launch_quantize_q8_0(const float* x, int64_t n_rows, int cols, int8_t* q, float* d,
+                                 cudaStream_t s) {
+    const int64_t nblk = n_rows * (cols / kQBlock);
+    if (nblk == 0) return cudaSuccess;
+    const int64_t want = (nblk + 7) / 8;
+    const int grid = (int)(want < 65535 * 8 ? want : 65535 * 8);
+    k_quantize_q8_0<<<grid, 256, 0, s>>>(x, nblk, q, d);
+    return cudaGetLastError();
+}
+
+// Per-row quantiser: one CTA per row.  s = amax / qmax, code =
+// round-half-away(w * (1/s)) clamped to [-2^(b-1), qmax], packed two's
+// complement with the lowest element in the lowest bits.
+template <int WBITS>
+__global__ void __launch_bounds__(256) k_pack_rows(const float* __restrict__ w, int64_t rows, int cols,
+                                                   uint8_t* __restrict__ packed, float* __restrict__ scales) {
+    constexpr int qmax = WBITS == 8 ? 127 : WBITS == 4 ? 7 : 1;
+    constexpr float qminf = -(float)(1 << (WBITS - 1));
+    __shared__ float red[8];
+    __shared__ float s_is[2];
+    const int64_t row_bytes = (int64_t)cols * WBITS / 8;
+    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+        const float* wr = w + r * cols;
+        float a = 0.0f;
+        for (int i = threadIdx.x * 4; i < cols; i += blockDim.x * 4) {
+            const float4 v = *reinterpret_cast<const float4*>(wr + i);
+            a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, o));
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float m = red[0];
+            for (int i = 1; i < (int)(blockDim.x >> 5); ++i) m = fmaxf(m, red[i]);
+            float sc = 0.0f, is = 0.0f;
+            if (m >= FLT_MIN) {
+                sc = __fdiv_rn(m, (float)qmax);
+                is = __fdiv_rn(1.0f, sc);
+            }
+            scales[r] = sc;
+            s_is[0] = is;
+            s_is[1] = sc;
+        }
+        __syncthreads();
+        const float is = s_is[0];
+        const bool zero = !(s_is[1] > 0.0f);
+        // each thread packs groups of 32 codes
+        for (int g = threadIdx.x; g < cols / 32; g += blockDim.x) {
+            int codes[32];
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+                const float4 v = *reinterpret_cast<const float4*>(wr + 32 * g + i);
+                const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float c = roundf(__fmul_rn(vv[j], is));
+                    c = fminf(fmaxf(c, qminf), (float)qmax);
+                    codes[i + j] = zero ? 0 : (int)c;
+                }
+            }
+            uint8_t* dst = packed + r * row_bytes + (int64_t)g * 32 * WBITS / 8;
+            if constexpr (WBITS == 8) {
+                uint32_t out[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    out[k] = (uint32_t)(codes[4 * k] & 0xFF) | ((uint32_t)(codes[4 * k + 1] & 0xFF) << 8) |
+                             ((uint32_t)(codes[4 * k + 2] & 0xFF) << 16) | ((uint32_t)(codes[4 * k + 3] & 0xFF) << 24);
+                reinterpret_cast<uint4*>(dst)[0] = make_uint4(out[0], out[1], out[2], out[3]);
+                reinterpret_cast<uint4*>(dst)[1] = make_uint4(out[4], out[5], out[6], out[7]);
+            } else if constexpr (WBITS == 4) {
+                uint32_t out[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    uint32_t word = 0;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) word |= (uint32_t)(codes[8 * k + j] & 0xF) << (4 * j);
+                    out[k] = word;
+                }
+                reinterpret_cast<uint4*>(dst)[0] = make_uint4(out[0], out[1], out[2], out[3]);
+            } else {
+                uint32_t out[2];
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    uint32_t word = 0;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) word |= (uint32_t)(codes[16 * k + j] & 0x3) << (2 * j);
+                    out[k] = word;
+                }
+                reinterpret_cast<uint2*>(dst)[0] = make_uint2(out[0], out[1]);
+            }
+        }
+        __syncthreads();
+    }
+}
+
+cudaError_t launch_pack_weights(const float* w, int64_t rows, int cols, int wbits, uint8_t* packed,
+                                float* scales, cudaStream_t s) {
+    if (rows == 0) return cudaSuccess;
+    const int grid = (int)(rows < 1048576 ? rows : 1048576);
+    if (wbits == 8) k_pack_rows<8><<<grid, 256, 0, s>>>(w, rows, cols, packed, scales);
+    else if (wbits == 4) k_pack_rows<4><<<grid, 256, 0, s>>>(w, rows, cols, packed, scales);
+    else k_pack_rows<2><<<grid, 256, 0, s>>>(w, rows, cols, packed, scales);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,83 @@
+"""GPU vs oracle at the GLM-5.2 layer's full sizes (hidden 6144, intermediate
+2048, 256 experts resident in HBM), in the launch configuration bench.py times.
+
+All 256 experts are drawn and packed on the GPU; the oracle regenerates on the
+host only the experts the sampled tokens need and packs them itself.  Checked:
+packed bytes of those experts (bit-exact), expert indices and bucketing for
+every token (bit-exact), per-block int32 dots of gate/up and down rows
+(bit-exact), and the sampled tokens' fp32 outputs (1e-3 of their RMS)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as orc
+from parity_helpers import OUT_TOL, host_expert_mats, rel_rms_err
+from quantized_routed_expert_group_b200 import moe, synth
+
+pytestmark = pytest.mark.gpu
+
+FULL = ["glm52_decode_int4_t1", "glm52_verify_int4_t4", "glm52_int8_t16_outliers", "glm52_prefill_int4_t512_zipf"]
+
+
+@pytest.fixture(scope="module", params=FULL)
+def full(request):
+    wl = synth.WORKLOADS[request.param]
+    layer = moe.synth_layer(wl)
+    x = synth.make_x(wl)
+    out = layer.forward(torch.from_numpy(x).cuda())
+    torch.cuda.synchronize()
+    assert layer.device_error() == 0
+    view = {k: v.cpu().numpy() for k, v in layer.view(wl.T).items()}
+    yield wl, layer, x, out.cpu().numpy(), view
+    del layer, out
+    torch.cuda.empty_cache()
+
+
+def _sample_tokens(T):
+    return sorted(set([0, T - 1, T // 2]))[: 3 if T > 64 else 2]
+
+
+def test_full_router_and_bucket(full):
+    wl, layer, x, out, v = full
+    s = wl.shape
+    io, wo, c, gs = orc.router(x, synth.make_router_w(wl), synth.make_bias(wl), s.n_groups, s.topk_groups,
+                               s.top_k, s.rsf, want_scores=True)
+    np.testing.assert_array_equal(v["idx"], io)
+    np.testing.assert_allclose(v["w"], wo, rtol=1e-6)
+    counts, offsets, perm = orc.bucket(io, s.n_experts)
+    np.testing.assert_array_equal(v["counts"], counts)
+    np.testing.assert_array_equal(v["offsets"], offsets)
+    np.testing.assert_array_equal(v["perm"], perm)
+    print(wl.name, "unique experts:", int((counts > 0).sum()), "max tokens/expert:", int(counts.max()))
+
+
+def test_full_sampled_outputs(full):
+    wl, layer, x, out, v = full
+    s = wl.shape
+    toks = _sample_tokens(wl.T)
+    need = sorted(set(v["idx"][toks].reshape(-1).tolist()))
+    routed = {}
+    for e in need:
+        ex = orc.pack_expert(*host_expert_mats(wl, e), s.wbits)
+        routed[e] = ex
+        # the GPU packed the device-generated weights to the same bytes
+        np.testing.assert_array_equal(layer.routed.w_gate[e].cpu().numpy(), ex.wg)
+        np.testing.assert_array_equal(layer.routed.w_up[e].cpu().numpy(), ex.wu)
+        np.testing.assert_array_equal(layer.routed.w_down[e].cpu().numpy(), ex.wd)
+        np.testing.assert_array_equal(layer.routed.s_down[e].cpu().numpy().view(np.uint32), ex.sd.view(np.uint32))
+    shared = orc.pack_expert(*host_expert_mats(wl, 0, shared=True), s.wbits)
+    np.testing.assert_array_equal(layer.shared.w_gate[0].cpu().numpy(), shared.wg)
+    tr = orc.layer_forward(s, x[toks], synth.make_router_w(wl), synth.make_bias(wl), routed, shared)
+    err = rel_rms_err(out[toks], tr.out)
+    print(wl.name, "tokens", toks, "max err / rms =", err)
+    assert err <= OUT_TOL
+    # per-block int32 dots, bit-exact: gate rows on x's codes, down rows on the
+    # oracle's own h codes (h itself may round differently by a few ulp)
+    t0, e0 = toks[0], int(v["idx"][toks[0], 0])
+    ex = routed[e0]
+    xq = torch.from_numpy(tr.xq[0:1]).cuda()
+    got = moe.block_dots(layer.routed.w_gate[e0], s.hidden, s.wbits, xq).cpu().numpy()
+    np.testing.assert_array_equal(got, orc.block_dots(ex.wg, s.hidden, s.wbits, tr.xq[0:1]))
+    hq = np.ascontiguousarray(tr.hq[0, 0:1])
+    got = moe.block_dots(layer.routed.w_down[e0], s.inter, s.wbits, torch.from_numpy(hq).cuda()).cpu().numpy()
+    np.testing.assert_array_equal(got, orc.block_dots(ex.wd, s.inter, s.wbits, hq))
