@@ -164,6 +164,34 @@ int moe_layer_forward_host(const moe_config *cfg, const float *x_host, int T, co
                            const float *router_bias, const moe_experts *routed, const moe_experts *shared,
                            float *out_host, void *workspace, size_t ws_bytes, void *stream);
 
+/* moe_layer_forward without a caller-provided workspace.  (The pages have no
+ * counterpart: this exists for callers of this library.)
+ *
+ * Some callers cannot allocate device memory when they want to run the layer:
+ * a host framework whose allocator has already reserved the device and owns
+ * every buffer, a plugin that is handed only input and output buffers, or a
+ * latency-critical loop where cudaMalloc (which can synchronise the device)
+ * is not allowed.  This variant allocates nothing: its scratch is a fixed
+ * 8 MiB array in the library's device memory (a file-scope __device__ array),
+ * which every GPU that loads the library holds until the process exits.  The
+ * caller still passes x, out and the weights as for moe_layer_forward.
+ *
+ * Limit: the layer's workspace for T tokens must fit in 8 MiB
+ * (moe_workspace_bytes(cfg, T) <= 8388608); larger T returns MOE_EWORKSPACE
+ * and launches nothing.  For the GLM-5.2 layer (hidden 6144, 256 experts,
+ * top-8 + 1 shared) that allows T <= 27.
+ *
+ * The first call on each device looks up the array's device address with that
+ * device current (once per device); make that first call before any stream
+ * capture.  Every call shares the one array and it keeps the last call's
+ * contents; each call clears what must start at zero.  Calls whose executions
+ * overlap on the GPU (different streams, or different host threads) race on
+ * the array and give wrong results: serialise them.  The intermediates are not
+ * reachable through moe_workspace_view or moe_get_device_error. */
+int moe_layer_forward_noalloc(const moe_config *cfg, const float *x, int T, const float *router_w,
+                              const float *router_bias, const moe_experts *routed, const moe_experts *shared,
+                              float *out, void *stream);
+
 /* Device pointers to the intermediates a moe_layer_forward call leaves in its
  * workspace (valid after the call completes, until the next call on the same
  * workspace).  Slots: routed (token, slot) pairs occupy bucket positions

@@ -262,6 +262,57 @@ MOE_API int moe_layer_forward_host(const moe_config* cfg, const float* x_host, i
     return status_of(cudaStreamSynchronize(s));
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free forward: the scratch is a fixed file-scope device array.
+// In host code g_noalloc_scratch names a host-side stand-in, not the device
+// array, so its device address is looked up with cudaGetSymbolAddress, once
+// per device, with that device current, and passed to the kernels.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoallocScratchBytes = (size_t)8 << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+static void* noalloc_scratch_address(int* status) {
+    static void* addr[64];
+    static bool ready[64];
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        *status = MOE_ECUDA;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ready[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+            *status = MOE_ECUDA;
+            return nullptr;
+        }
+        addr[dev] = p;
+        ready[dev] = true;
+    }
+    *status = MOE_OK;
+    return addr[dev];
+}
+
+MOE_API int moe_layer_forward_noalloc(const moe_config* cfg, const float* x, int T, const float* router_w,
+                                      const float* router_bias, const moe_experts* routed,
+                                      const moe_experts* shared, float* out, void* stream) {
+    int st = check_config(cfg);
+    if (st) return st;
+    if (T < 0) return MOE_EINVAL;
+    if (make_layout(*cfg, T).total > kNoallocScratchBytes) return MOE_EWORKSPACE;
+    void* scratch = noalloc_scratch_address(&st);
+    if (st) return st;
+    Layout L;
+    st = check_forward_args(cfg, x, T, router_w, router_bias, routed, shared, out, scratch, kNoallocScratchBytes,
+                            &L);
+    if (st) return st;
+    if (T == 0) return MOE_OK;
+    if (!aligned(x, 16) || !aligned(out, 4)) return MOE_EINVAL;
+    return forward_device(*cfg, x, T, router_w, router_bias, *routed, cfg->n_shared ? shared : nullptr, out,
+                          static_cast<char*>(scratch), L, (cudaStream_t)stream);
+}
+
 MOE_API int moe_workspace_view(const moe_config* cfg, int T, void* workspace, size_t ws_bytes,
                                moe_workspace_layout* view) {
     int st = check_config(cfg);

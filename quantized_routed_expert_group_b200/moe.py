@@ -54,6 +54,8 @@ _SIGS = {
                            ctypes.POINTER(MoeExperts), _vp, _vp, _sz, _vp], _int),
     "moe_layer_forward_host": ([ctypes.POINTER(MoeConfig), _vp, _int, _vp, _vp, ctypes.POINTER(MoeExperts),
                                 ctypes.POINTER(MoeExperts), _vp, _vp, _sz, _vp], _int),
+    "moe_layer_forward_noalloc": ([ctypes.POINTER(MoeConfig), _vp, _int, _vp, _vp, ctypes.POINTER(MoeExperts),
+                                   ctypes.POINTER(MoeExperts), _vp, _vp], _int),
     "moe_workspace_view": ([ctypes.POINTER(MoeConfig), _int, _vp, _sz, ctypes.POINTER(MoeWorkspaceLayout)], _int),
     "moe_block_dots": ([_vp, _i64, _int, _int, _vp, _int, _vp, _vp], _int),
     "moe_get_device_error": ([_vp, _vp, ctypes.POINTER(ctypes.c_int32)], _int),
@@ -311,6 +313,16 @@ class MoeLayer:
                                        ctypes.byref(self._routed_s), ctypes.byref(self._shared_s), _ptr(out),
                                        _ptr(self.workspace), self.workspace.numel(), _stream(stream)),
                "layer_forward")
+        return out
+
+    def forward_noalloc(self, x: torch.Tensor, out: torch.Tensor, stream=None) -> torch.Tensor:
+        """The layer through the allocation-free entry point (library-owned
+        fixed scratch instead of this object's workspace)."""
+        _cuda(x, torch.float32, "x")
+        _check(lib().moe_layer_forward_noalloc(ctypes.byref(self.cfg), _ptr(x), x.shape[0], _ptr(self.router_w),
+                                               _ptr(self.bias), ctypes.byref(self._routed_s),
+                                               ctypes.byref(self._shared_s), _ptr(out), _stream(stream)),
+               "layer_forward_noalloc")
         return out
 
     def forward_host(self, x_host: torch.Tensor, out_host: torch.Tensor, stream=None) -> torch.Tensor:
