@@ -184,7 +184,9 @@ def run_ours(args) -> dict | None:
     n_active = int((layer.view(wl.T)["counts"] > 0).sum().item())
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.PROFILE_PHASES + 1)] for _ in range(K)]
+    phases = moe.forward_phases(layer.cfg, wl.T)
+    P = len(phases)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.PROFILE_MAX_EVENTS)] for _ in range(K)]
     for row in evs:  # torch creates the CUDA event on first record
         for ev in row:
             ev.record()
@@ -209,8 +211,8 @@ def run_ours(args) -> dict | None:
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
-    step_ms = [evs[i][0].elapsed_time(evs[i][-1]) for i in range(K)]
-    phase_ms = [[evs[i][p].elapsed_time(evs[i][p + 1]) for i in range(K)] for p in range(moe.PROFILE_PHASES)]
+    step_ms = [evs[i][0].elapsed_time(evs[i][P]) for i in range(K)]
+    phase_ms = [[evs[i][p].elapsed_time(evs[i][p + 1]) for i in range(K)] for p in range(P)]
     total_ms = sum(step_ms)
     max_total = reduce_max(total_ms, dev)
     value = throughput(wl.T, K, world, max_total)
@@ -229,12 +231,18 @@ def run_ours(args) -> dict | None:
     e2e_max = reduce_max(e2e_s * 1e3, dev)
     e2e_value = throughput(wl.T, K_e2e, world, e2e_max)
 
-    # roofline of the dominant kernel (expert gate/up: 2/3 of the expert bytes)
+    # roofline of the dominant phase's kernel: the fused kernel (whole layer)
+    # on the small-batch path, the gate/up GEMV on the multi-kernel path
     peak, peak_kind = measured_peak_hbm()
-    gu_ms = statistics.mean(phase_ms[2])
-    gu_bytes = (n_active + s.n_shared) * gateup_bytes(s)
-    achieved = gu_bytes / (gu_ms * 1e-3) / 1e9
+    router_bytes = s.n_experts * s.hidden * 4
     layer_bytes = (n_active + s.n_shared) * expert_bytes(s)
+    if phases == ["fused"]:
+        dom_kernel, dom_ms = "k_moe_small", statistics.mean(phase_ms[0])
+        dom_bytes = layer_bytes + router_bytes
+    else:
+        dom_kernel, dom_ms = "k_gateup", statistics.mean(phase_ms[phases.index("gate_up")])
+        dom_bytes = (n_active + s.n_shared) * gateup_bytes(s)
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     ms_step = statistics.mean(step_ms)
     layer_gbs = layer_bytes / (ms_step * 1e-3) / 1e9
     if rank != 0:
@@ -249,11 +257,11 @@ def run_ours(args) -> dict | None:
                    "l2": "flushed before every step (write of 2x L2)", "parallelism": f"replicas x{world}"},
         "layer_hbm": {"algorithmic_bytes": layer_bytes, "gbs": round(layer_gbs, 1),
                       "frac_measured": round(layer_gbs / peak, 4), "frac_spec_8tbs": round(layer_gbs / SPEC_HBM_GBS, 4)},
-        "phases_ms": {n: round(statistics.mean(v), 5) for n, v in zip(moe.PHASE_NAMES, phase_ms)},
-        "roofline": {"kernel": "k_gateup", "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+        "phases_ms": {n: round(statistics.mean(v), 5) for n, v in zip(phases, phase_ms)},
+        "roofline": {"kernel": dom_kernel, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "algorithmic_bytes_per_launch": gu_bytes,
-                     "traffic": ncu_traffic("k_gateup", wl.name)},
+                     "algorithmic_bytes_per_launch": dom_bytes,
+                     "traffic": ncu_traffic(dom_kernel, wl.name)},
         "e2e": {"value": round(e2e_value, 3), "unit": "tokens/s", "h2d_bytes_per_step": x.numel() * 4,
                 "d2h_bytes_per_step": out.numel() * 4, "steps": K_e2e},
         "gpu_launches": K * moe.forward_launches(layer.cfg, wl.T),

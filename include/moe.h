@@ -236,16 +236,23 @@ int moe_synth_normal(uint64_t seed, uint64_t tid, int64_t offset, int64_t n, flo
                      void *stream);
 
 /* Tracing hook: CUDA events at the phase boundaries of moe_layer_forward.
- * events points to MOE_PROFILE_PHASES + 1 cudaEvent_t handles (passed as
- * void*), or is NULL to switch tracing off; the setting belongs to the calling
- * host thread.  While it is set, every forward issued from that thread records
- * events[0] on its stream before its first launch and events[i] after phase i:
- *   1 Q8_0 of x + router, 2 bucketing, 3 expert gate/up (+ SiLU, Q8_0 of h),
- *   4 expert down, 5 combine.
- * The caller keeps the events alive until they have completed.  n_events must
- * be MOE_PROFILE_PHASES + 1 (or 0 with events NULL). */
-#define MOE_PROFILE_PHASES 5
+ * events points to MOE_PROFILE_MAX_EVENTS cudaEvent_t handles (passed as
+ * void*), or is NULL (with n_events 0) to switch tracing off; the setting
+ * belongs to the calling host thread.  While it is set, every forward issued
+ * from that thread records events[0] on its stream before its first launch
+ * and events[i] after phase i, for i = 1 .. moe_forward_phases(cfg, T).  The
+ * phases depend on the path the forward takes: the fused small-batch path
+ * (T <= 4) has one phase, "fused" (both of its kernels); the multi-kernel path
+ * has five: "route" (Q8_0 of x, logits, selection), "bucket", "gate_up",
+ * "down", "combine".  The caller keeps the events alive until they have
+ * completed. */
+#define MOE_PROFILE_MAX_EVENTS 8
 int moe_profile_events(void *const *events, int n_events);
+
+/* Number of traced phases of a forward with T tokens, and the name of phase
+ * i (0-based; "" when out of range).  Negative status on an invalid config. */
+int moe_forward_phases(const moe_config *cfg, int T);
+const char *moe_forward_phase_name(const moe_config *cfg, int T, int i);
 
 /* Number of kernel launches one moe_layer_forward with T tokens issues
  * (0 for T = 0; negative status on an invalid config). */

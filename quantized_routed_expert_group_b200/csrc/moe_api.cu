@@ -36,6 +36,8 @@ Layout make_layout(const moe_config& c, int T) {
     L.perm = take(t * k * 4);
     L.inv_perm = take(t * k * 4);
     L.active = take((E + 2) * 4);
+    L.ctrl = take(small_ctrl_bytes(c, T));
+    L.hbuf = take(slots * I * 4);
     L.hq = take(slots * I);
     L.hd = take(slots * (I / 32) * 4);
     L.y = take(slots * H * 4);
@@ -53,8 +55,10 @@ const DeviceInfo& device_info() {
     std::lock_guard<std::mutex> lock(mu);
     if (!done[dev]) {
         DeviceInfo d{148, 227 * 1024};
-        cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
-        cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) d.sm_count = v;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess && v > 0)
+            d.max_smem_optin = v;
         infos[dev] = d;
         done[dev] = true;
     }
@@ -90,7 +94,7 @@ static int check_experts(const moe_experts* ex) {
 static int status_of(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ECUDA; }
 
 // Per-thread tracing events (see moe_profile_events).
-static thread_local cudaEvent_t g_trace[MOE_PROFILE_PHASES + 1];
+static thread_local cudaEvent_t g_trace[MOE_PROFILE_MAX_EVENTS];
 static thread_local bool g_trace_on = false;
 
 static cudaError_t trace(int i, cudaStream_t s) {
@@ -110,8 +114,6 @@ static int forward_device(const moe_config& c, const float* x, int T, const floa
                           const float* router_bias, const moe_experts& routed, const moe_experts* shared,
                           float* out, char* ws, const Layout& L, cudaStream_t s) {
     int32_t* err = reinterpret_cast<int32_t*>(ws + L.err);
-    if (trace(0, s) != cudaSuccess) return MOE_ECUDA;
-    if (cudaMemsetAsync(err, 0, 64, s) != cudaSuccess) return MOE_ECUDA;
     int8_t* xq = reinterpret_cast<int8_t*>(ws + L.xq);
     float* xd = reinterpret_cast<float*>(ws + L.xd);
     int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
@@ -121,6 +123,39 @@ static int forward_device(const moe_config& c, const float* x, int T, const floa
     int32_t* perm = reinterpret_cast<int32_t*>(ws + L.perm);
     int32_t* inv_perm = reinterpret_cast<int32_t*>(ws + L.inv_perm);
     int32_t* active = reinterpret_cast<int32_t*>(ws + L.active);
+    if (small_path_supported(c, T)) {
+        SmallArgs a;
+        a.cfg = &c;
+        a.T = T;
+        a.x = x;
+        a.router_w = router_w;
+        a.bias = router_bias;
+        a.routed = routed;
+        a.shared = shared ? *shared : routed;
+        a.xq = xq;
+        a.xd = xd;
+        a.logits = reinterpret_cast<double*>(ws + L.logits);
+        a.idx = idx;
+        a.w = w;
+        a.counts = counts;
+        a.offsets = offsets;
+        a.perm = perm;
+        a.inv_perm = inv_perm;
+        a.active = active;
+        a.hbuf = reinterpret_cast<float*>(ws + L.hbuf);
+        a.hq = reinterpret_cast<int8_t*>(ws + L.hq);
+        a.hd = reinterpret_cast<float*>(ws + L.hd);
+        a.y = reinterpret_cast<float*>(ws + L.y);
+        a.out = out;
+        a.ctrl = reinterpret_cast<int*>(ws + L.ctrl);
+        a.err = err;
+        int st2 = status_of(trace(0, s));
+        if (!st2) st2 = status_of(launch_small(a, s));
+        if (!st2) st2 = status_of(trace(1, s));
+        return st2;
+    }
+    if (trace(0, s) != cudaSuccess) return MOE_ECUDA;
+    if (cudaMemsetAsync(err, 0, 64, s) != cudaSuccess) return MOE_ECUDA;
     int st = status_of(launch_quantize_q8_0(x, T, c.hidden, xq, xd, s));
     if (st) return st;
     st = status_of(launch_router(c, x, T, router_w, router_bias, reinterpret_cast<double*>(ws + L.logits), idx, w, s));
@@ -368,8 +403,8 @@ MOE_API int moe_profile_events(void* const* events, int n_events) {
         g_trace_on = false;
         return MOE_OK;
     }
-    if (n_events != MOE_PROFILE_PHASES + 1) return MOE_EINVAL;
-    for (int i = 0; i <= MOE_PROFILE_PHASES; ++i) {
+    if (n_events != MOE_PROFILE_MAX_EVENTS) return MOE_EINVAL;
+    for (int i = 0; i < MOE_PROFILE_MAX_EVENTS; ++i) {
         if (!events[i]) return MOE_EINVAL;
         g_trace[i] = static_cast<cudaEvent_t>(events[i]);
     }
@@ -381,7 +416,23 @@ MOE_API int moe_forward_launches(const moe_config* cfg, int T) {
     const int st = check_config(cfg);
     if (st) return st;
     if (T < 0) return MOE_EINVAL;
-    return T == 0 ? 0 : kForwardLaunches;
+    if (T == 0) return 0;
+    return small_path_supported(*cfg, T) ? kSmallLaunches : kForwardLaunches;
+}
+
+MOE_API int moe_forward_phases(const moe_config* cfg, int T) {
+    const int st = check_config(cfg);
+    if (st) return st;
+    if (T < 0) return MOE_EINVAL;
+    if (T == 0) return 0;
+    return small_path_supported(*cfg, T) ? 1 : 5;
+}
+
+MOE_API const char* moe_forward_phase_name(const moe_config* cfg, int T, int i) {
+    static const char* multi[5] = {"route", "bucket", "gate_up", "down", "combine"};
+    const int n = moe_forward_phases(cfg, T);
+    if (i < 0 || i >= n) return "";
+    return n == 1 ? "fused" : multi[i];
 }
 
 MOE_API const char* moe_status_string(int status) {

@@ -183,6 +183,53 @@ struct Log2<1> {
     static constexpr int value = 0;
 };
 
+// SwiGLU activation of one row: silu(g) * u = g / (1 + e^-g) * u, in fp32
+// (accurate expf and IEEE division; no fast-math).
+__device__ __forceinline__ float silu_mul(float g, float u) {
+    return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+}
+
+// Compensated ("double-float") dot-product accumulation in fp32.  The
+// product of two fp32 values is split exactly into hi + lo with one fma
+// (TwoProduct) and added into a running (sum, err) pair with TwoSum (Knuth),
+// so the pair carries the running sum to about 2^-48 relative instead of
+// fp32's 2^-24, using only fp32 instructions (fp64 arithmetic on CUDA cores is
+// a narrow pipe on B200).  The pair is folded into fp64 at the end.
+struct DFAcc {
+    float hi = 0.0f, lo = 0.0f;
+    __device__ __forceinline__ void add_prod(float a, float b) {
+        const float p = __fmul_rn(a, b);
+        const float pe = __fmaf_rn(a, b, -p);  // exact product error
+        const float t = __fadd_rn(hi, p);
+        const float bp = __fsub_rn(t, hi);
+        const float e = __fadd_rn(__fsub_rn(hi, __fsub_rn(t, bp)), __fsub_rn(p, bp));  // exact sum error
+        hi = t;
+        lo = __fadd_rn(lo, __fadd_rn(e, pe));
+    }
+    __device__ __forceinline__ double value() const { return (double)hi + (double)lo; }
+};
+
+// Order-preserving unsigned key of a double (larger value -> larger key;
+// -0.0 is folded into +0.0 so that equal values give equal keys).
+__device__ __forceinline__ unsigned long long order_key(double v) {
+    v = v + 0.0;
+    const long long b = __double_as_longlong(v);
+    return b >= 0 ? (unsigned long long)b ^ 0x8000000000000000ull : ~(unsigned long long)b;
+}
+
+// Arg-max of (key, index) over the warp: larger key wins, ties to the lower index.
+__device__ __forceinline__ void warp_argmax_key(unsigned long long& k, int& i) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long ok = __shfl_xor_sync(kFull, k, o);
+        const int oi = __shfl_xor_sync(kFull, i, o);
+        if (ok > k || (ok == k && oi < i)) {
+            k = ok;
+            i = oi;
+        }
+    }
+}
+
 // Arg-max over the warp with ties to the lower index.
 __device__ __forceinline__ void warp_argmax(double& v, int& i) {
 #pragma unroll

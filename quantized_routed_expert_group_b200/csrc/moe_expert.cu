@@ -119,10 +119,7 @@ __global__ void __launch_bounds__(256) k_gateup(ExpertParams p) {
                 const int rd = vi / TCH, i = vi % TCH;
                 const int row = row0 + rd;
                 const int64_t so = (int64_t)eo * p.I + row;
-                const float g = ex.s_gate[so] * v;
-                const float u = ex.s_up[so] * vu;
-                const double gd = (double)g;
-                hs[i][warp * 4 + rd] = (float)(gd / (1.0 + exp(-gd)) * (double)u);
+                hs[i][warp * 4 + rd] = silu_mul(ex.s_gate[so] * v, ex.s_up[so] * vu);
             }
             __syncthreads();
             if (warp < nv) {
@@ -198,19 +195,19 @@ __global__ void __launch_bounds__(256) k_down(ExpertParams p) {
     }
 }
 
-// out[t][c] = sum_j w[t][j] * y[slot(t,j)][c] + y[T*k + t][c]  (fp64 sum in
-// slot order, then the shared expert; rounded once to fp32).
+// out[t][c] = sum_j w[t][j] * y[slot(t,j)][c] + y[T*k + t][c]  (fp32, in
+// slot order, then the shared expert).
 __global__ void k_combine(ExpertParams p) {
     const int64_t n = (int64_t)p.T * p.H;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
         const int t = (int)(i / p.H), c = (int)(i % p.H);
-        double acc = 0.0;
+        float acc = 0.0f;
         for (int j = 0; j < p.k; ++j) {
             const int slot = p.inv_perm[t * p.k + j];
-            acc += (double)p.w[t * p.k + j] * (double)p.y[(int64_t)slot * p.H + c];
+            acc = fmaf(p.w[t * p.k + j], p.y[(int64_t)slot * p.H + c], acc);
         }
-        if (p.ns) acc += (double)p.y[((int64_t)p.T * p.k + t) * p.H + c];
-        p.out[i] = (float)acc;
+        if (p.ns) acc += p.y[((int64_t)p.T * p.k + t) * p.H + c];
+        p.out[i] = acc;
     }
 }
 

@@ -25,7 +25,9 @@ struct Layout {
     size_t offsets;    // int32 [E+1]
     size_t perm;       // int32 [T*k]
     size_t inv_perm;   // int32 [T*k]
-    size_t active;     // int32 [1 + E + 1]: count, then expert ids (shared = -1 last)
+    size_t active;     // int32 [1 + E + 1]: count, then expert ids
+    size_t ctrl;       // int32 control words of the fused small-batch kernel
+    size_t hbuf;       // fp32 [slots][I]  h before quantisation (fused kernel)
     size_t hq;         // int8 [slots][I]
     size_t hd;         // fp32 [slots][I/32]
     size_t y;          // fp32 [slots][H]
@@ -73,6 +75,38 @@ struct ExpertArgs {
 // ev (optional, 3 events): recorded after gate/up, down and combine.
 cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t s, cudaEvent_t const* ev);
 constexpr int kForwardLaunches = 7;  // quantise, logits, select, bucket, gate/up, down, combine
+// Fused small-batch forward (T <= 4), moe_small.cu.
+struct SmallArgs {
+    const moe_config* cfg;
+    int T;
+    const float* x;
+    const float* router_w;
+    const float* bias;
+    moe_experts routed;
+    moe_experts shared;
+    int8_t* xq;
+    float* xd;
+    double* logits;
+    int32_t* idx;
+    float* w;
+    int32_t* counts;
+    int32_t* offsets;
+    int32_t* perm;
+    int32_t* inv_perm;
+    int32_t* active;
+    float* hbuf;
+    int8_t* hq;
+    float* hd;
+    float* y;
+    float* out;
+    int* ctrl;
+    int32_t* err;
+};
+bool small_path_supported(const moe_config& c, int T);
+size_t small_ctrl_bytes(const moe_config& c, int T);
+cudaError_t launch_small(const SmallArgs& a, cudaStream_t s);
+constexpr int kSmallLaunches = 2;  // prologue + persistent kernel
+
 cudaError_t launch_block_dots(const uint8_t* packed, int64_t rows, int cols, int wbits, const int8_t* q,
                               int n, int32_t* out, cudaStream_t s);
 cudaError_t launch_synth_normal(uint64_t seed, uint64_t tid, int64_t offset, int64_t n, float sigma,

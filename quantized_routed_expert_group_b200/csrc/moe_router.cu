@@ -4,8 +4,9 @@
 // router, noaux_tc, routed_scaling_factor, shared expert); wpnews.pro "Colibri
 // — รัน GLM-5.2 ...", spec table (Router: DeepSeek-V3-style sigmoid (noaux_tc);
 // 256 experts, 8 active + 1 shared) and kernel table (the routing matmul stays
-// in f32).  The logits keep fp32 inputs and sum in fp64 so that the expert
-// choice does not depend on the summation order.
+// in f32).  The logits keep fp32 inputs and are summed to about 2^-48
+// relative (compensated fp32, then fp64) so that the expert choice does not
+// depend on the summation order.
 #include <cmath>
 
 #include "moe_device.cuh"
@@ -17,9 +18,10 @@ constexpr int kRouterExpertsPerCta = 2;
 constexpr int kRouterKSplit = 4;
 constexpr int kRouterTokens = 8;
 
-// logits[t][e] = sum_j x[t][j] * Wr[e][j] (fp64).  CTA = 2 experts x 4 K-splits
-// (one warp each) x up to 8 tokens; the K-split partials are added in a fixed
-// order so the result is deterministic.
+// logits[t][e] = sum_j x[t][j] * Wr[e][j], accumulated per lane with the
+// compensated fp32 pair (about 2^-48 relative) and combined in fp64.  CTA = 2
+// experts x 4 K-splits (one warp each) x up to 8 tokens; the K-split partials
+// are added in a fixed order so the result is deterministic.
 __global__ void __launch_bounds__(256) k_router_logits(const float* __restrict__ x, int T, int H,
                                                        const float* __restrict__ Wr, int E,
                                                        double* __restrict__ logits) {
@@ -32,9 +34,7 @@ __global__ void __launch_bounds__(256) k_router_logits(const float* __restrict__
     const int n4 = H / 4;
     const int per = (n4 + kRouterKSplit - 1) / kRouterKSplit;
     const int j0 = ks * per, j1 = min(n4, j0 + per);
-    double acc[kRouterTokens];
-#pragma unroll
-    for (int t = 0; t < kRouterTokens; ++t) acc[t] = 0.0;
+    DFAcc acc[kRouterTokens];
     if (e < E) {
         const float4* wr = reinterpret_cast<const float4*>(Wr + (int64_t)e * H);
         for (int j = j0 + lane; j < j1; j += 32) {
@@ -43,19 +43,17 @@ __global__ void __launch_bounds__(256) k_router_logits(const float* __restrict__
             for (int t = 0; t < kRouterTokens; ++t) {
                 if (t < nt) {
                     const float4 xv = __ldg(reinterpret_cast<const float4*>(x + (int64_t)(t0 + t) * H) + j);
-                    double a = acc[t];
-                    a = fma((double)xv.x, (double)wv.x, a);
-                    a = fma((double)xv.y, (double)wv.y, a);
-                    a = fma((double)xv.z, (double)wv.z, a);
-                    a = fma((double)xv.w, (double)wv.w, a);
-                    acc[t] = a;
+                    acc[t].add_prod(xv.x, wv.x);
+                    acc[t].add_prod(xv.y, wv.y);
+                    acc[t].add_prod(xv.z, wv.z);
+                    acc[t].add_prod(xv.w, wv.w);
                 }
             }
         }
     }
 #pragma unroll
     for (int t = 0; t < kRouterTokens; ++t) {
-        double v = acc[t];
+        double v = acc[t].value();
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
         if (lane == 0) part[ks][el][t] = v;

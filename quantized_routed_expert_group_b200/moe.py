@@ -62,11 +62,12 @@ _SIGS = {
     "moe_synth_normal": ([_u64, _u64, _i64, _i64, _flt, _vp, _vp], _int),
     "moe_profile_events": ([ctypes.POINTER(_vp), _int], _int),
     "moe_forward_launches": ([ctypes.POINTER(MoeConfig), _int], _int),
+    "moe_forward_phases": ([ctypes.POINTER(MoeConfig), _int], _int),
+    "moe_forward_phase_name": ([ctypes.POINTER(MoeConfig), _int, _int], ctypes.c_char_p),
     "moe_status_string": ([_int], ctypes.c_char_p),
 }
 
-PROFILE_PHASES = 5
-PHASE_NAMES = ["route", "bucket", "gate_up", "down", "combine"]
+PROFILE_MAX_EVENTS = 8
 
 _LIB = None
 
@@ -182,7 +183,7 @@ def synth_normal(seed: int, tid: int, n: int, sigma: float, offset: int = 0, out
 
 def profile_events(events) -> None:
     """Record torch.cuda.Event objects at the forward's phase boundaries
-    (PROFILE_PHASES + 1 events, created with enable_timing=True), or stop
+    (PROFILE_MAX_EVENTS events, created with enable_timing=True), or stop
     when events is None."""
     if events is None:
         _check(lib().moe_profile_events(None, 0), "profile_events")
@@ -192,6 +193,13 @@ def profile_events(events) -> None:
             ev.record()
     arr = (_vp * len(events))(*[ev.cuda_event for ev in events])
     _check(lib().moe_profile_events(arr, len(events)), "profile_events")
+
+
+def forward_phases(cfg: MoeConfig, T: int) -> list[str]:
+    n = lib().moe_forward_phases(ctypes.byref(cfg), T)
+    if n < 0:
+        _check(n, "forward_phases")
+    return [lib().moe_forward_phase_name(ctypes.byref(cfg), T, i).decode() for i in range(n)]
 
 
 def forward_launches(cfg: MoeConfig, T: int) -> int:

@@ -127,3 +127,16 @@ def test_other_entry_point_errors(L):
     assert lib.moe_synth_normal(1, 2, -1, 4, 1.0, 0x1000, None) == -1
     code = ctypes.c_int32(0)
     assert lib.moe_get_device_error(None, None, ctypes.byref(code)) == -1
+
+
+def test_forward_paths_and_phases(L):
+    """T <= 4 takes the fused small-batch path (2 launches, one traced phase);
+    larger batches the multi-kernel path (7 launches, five phases)."""
+    c = _cfg(L)
+    assert L.forward_phases(c, 1) == ["fused"] and L.forward_launches(c, 1) == 2
+    assert L.forward_phases(c, 4) == ["fused"]
+    assert L.forward_phases(c, 5) == ["route", "bucket", "gate_up", "down", "combine"]
+    assert L.forward_launches(c, 16) == 7 and L.forward_launches(c, 0) == 0
+    big = _cfg(L, n_experts=512, n_groups=16)   # beyond the fused path's 256 experts
+    assert L.forward_phases(big, 1) == ["route", "bucket", "gate_up", "down", "combine"]
+    assert L.lib().moe_profile_events(None, 3) == -1

@@ -49,8 +49,9 @@ def test_tiny_zero_tokens(tiny):
     assert out.shape == (0, 256)
 
 
-def test_tiny_deterministic(tiny):
-    x = torch.from_numpy(tiny.x).cuda()
+@pytest.mark.parametrize("T", [1, 4, 9])
+def test_tiny_deterministic(tiny, T):
+    x = torch.from_numpy(synth.make_x(tiny.wl.with_tokens(T))).cuda()
     a = tiny.layer.forward(x).clone()
     b = tiny.layer.forward(x).clone()
     torch.cuda.synchronize()
@@ -66,8 +67,13 @@ def test_tiny_host_entry_point(tiny):
 
 
 @pytest.mark.parametrize("shape,T,seed,x_kind", [
-    (MID4, 37, 11, "normal"), (MID8, 19, 12, "normal"), (MID4, 4, 13, "correlated"),
-    (MID4_NOSHARED, 5, 14, "normal"), (FULLGROUPS, 9, 15, "normal"), (MID8, 1, 16, "normal"),
+    # multi-kernel path (T > 4)
+    (MID4, 37, 11, "normal"), (MID8, 19, 12, "normal"), (MID4_NOSHARED, 5, 14, "normal"),
+    (FULLGROUPS, 9, 15, "normal"),
+    # fused small-batch path (T <= 4)
+    (MID4, 4, 13, "correlated"), (MID8, 1, 16, "normal"), (MID4, 1, 17, "normal"), (MID4, 2, 18, "normal"),
+    (MID4, 3, 19, "normal"), (MID8, 2, 20, "normal"), (MID8, 4, 21, "correlated"),
+    (MID4_NOSHARED, 3, 22, "normal"), (FULLGROUPS, 2, 23, "normal"),
 ])
 def test_mid_layers(shape, T, seed, x_kind):
     wl = make_workload(f"mid_{shape.wbits}_{T}", shape, T, seed, x_kind=x_kind)
