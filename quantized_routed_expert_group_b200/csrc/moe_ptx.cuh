@@ -74,6 +74,12 @@ __device__ __forceinline__ void bulk_g2s_nohint(void* dst, const void* src, uint
                  : "memory");
 }
 
+// Ask L2 to fetch a range ahead of its use (no destination, no completion
+// signal).  src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Order this thread's earlier generic-proxy view of global memory (e.g. an
 // acquire of data written by other CTAs) before later bulk-copy reads.
 __device__ __forceinline__ void fence_proxy_async_global() {

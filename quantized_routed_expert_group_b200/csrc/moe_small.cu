@@ -1,34 +1,39 @@
 // moe_small.cu -- the whole MoE layer forward for small batches (T <= 4:
-// decode and speculative verify) as one persistent kernel.
+// decode and speculative verify) as one persistent kernel with a static
+// schedule.
 //
 // What it computes is the layer of moe_api.cu (router, batch-union bucketing,
 // SwiGLU experts on Q8_0 activations, combine; GeekNews "Show HN: 느린 컴퓨터에서
 // GLM 5.2 실행하기", §구현된 주요 기능; wpnews.pro "Colibri — รัน GLM-5.2 ...",
 // spec and kernel tables, "Batch-Union MoE").  How it is scheduled is B200's:
 //
-// * At one to four tokens the layer is a stream of ~170-360 MB of expert
+// * At one to four tokens the layer is a stream of ~170-400 MB of expert
 //   weights, so the goal is to keep HBM busy from the first cycle to the
-//   last.  Each CTA (one per SM) has a producer warp that streams work items
-//   with bulk asynchronous copies (cp.async.bulk, the 1-D TMA form) into a
-//   ring of 48 KB shared-memory slots, and eight consumer warps doing the
-//   integer dots on __dp4a.
-// * Items come from one global queue in dependency order: router rows,
-//   SELECT, shared-expert gate/up rows, QUANTISE(shared), routed gate/up rows,
-//   QUANTISE(routed), shared down rows, routed down rows, COMBINE.  An item
-//   only waits on items with smaller queue indices, which running CTAs have
-//   already taken, so no wait can deadlock; every wait is bounded and records
-//   an error code when it runs out.
-// * Nothing on the consumers' path waits for a global round trip: they signal
-//   completion with fire-and-forget release reductions; the waiting is done by
-//   the producer of the item that depends on them (it polls, then copies the
-//   inputs the item needs - h rows, h codes, partial outputs - into its slot).
-// * The producer prefetches its next queue index one item ahead and keeps the
-//   routing schedule in shared memory, so issuing an item costs no round trip.
-// * COMBINE sums the per-expert outputs of a tile of rows in a fixed order in
-//   fp64: no float atomics, results are bit-reproducible.
+//   last.  Each CTA (one per SM) has a producer warp that streams the CTA's
+//   share of the weights with bulk asynchronous copies (cp.async.bulk, the
+//   1-D TMA form) into a ring of 48 KB shared-memory slots, and eight
+//   consumer warps that do the integer dots on __dp4a.
+// * The schedule is static; no CTA takes work from a queue:
+//   - router: CTA c computes the logits of experts 2c and 2c+1;
+//   - selection: every CTA routes all tokens itself from the published
+//     logits (identical decisions everywhere), so the routing costs one
+//     grid-wide wait and no broadcast;
+//   - gate/up: cut into units of 32 rows of one expert (one Q8_0 block of h);
+//     unit u belongs to CTA u mod grid, which finishes it: SwiGLU, Q8_0 of
+//     the 32 h values, published with one release counter per expert;
+//   - down + combine: CTA c owns output rows [H c / grid, H (c+1) / grid) of
+//     every expert and combines them itself at the end, so no partial output
+//     crosses CTAs: no float atomics, bit-reproducible results.
+// * The only waits: the selection waits for every router item, and each
+//   down chunk waits for its expert's h (the producer polls, then copies the
+//   h codes into the slot with the weights).  Every wait is bounded and
+//   records a timeout in the error word.
+// * Weights known before the routing (the shared expert's) are issued first,
+//   and the CTA's shared-expert down rows are prefetched into L2 while the
+//   routing is computed.
 // * A tiny prologue kernel (Q8_0 of x, control-block reset) runs first; the
-//   main kernel is launched as its programmatic dependent and prefetches its
-//   first, routing-independent item before waiting for it.
+//   main kernel is its programmatic dependent and issues its router rows
+//   before waiting for it.
 #include <cmath>
 
 #include "moe_device.cuh"
@@ -42,51 +47,65 @@ constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kSmallThreads = kConsumers + 32;
 constexpr int kSlotWeightBytes = 48 * 1024;
 constexpr int kMaxSlots = 4;
+constexpr int kUnit = 32;          // gate/up rows per unit: one Q8_0 block of h
+constexpr int kMaxOwnedRows = 64;  // output rows one CTA owns
+constexpr int kScaleWin = 160;     // 16-byte aligned window over <= 32 fp32 scales
+constexpr int kMaxEntryWords = 5;  // ready bitmask words (entries <= 160)
 // Bounds of every wait (legitimate waits last microseconds): mbarrier
 // try_wait iterations, and polls of a global word with a short sleep each.
 constexpr uint32_t kWaitLimit = 1u << 20;
 constexpr uint32_t kSpinLimit = 1u << 21;
 // Consumers only ever wait for their producer, whose own waits are bounded
 // and end in a DONE marker, so their bound is far larger and never reached
-// unless the device misbehaves.
+// unless the device misbehaves; the producer's wait for the consumers'
+// routing uses the same bound.
 constexpr uint32_t kConsumerWaitLimit = 1u << 24;
-// Per-item completion signals: every consumer warp of an item adds one.
-constexpr int kWarpSignals = kConsumerWarps;
 
 enum ItemKind : int {
     kItemRouter = 1,
     kItemSelect = 2,
     kItemGateUp = 3,
-    kItemQuant = 4,
-    kItemDown = 5,
-    kItemCombine = 6,
-    kItemDone = 7
+    kItemDown = 4,
+    kItemCombine = 5,
+    kItemDone = 6
 };
 
 // Control block (int32 words, zeroed by the prologue on every call):
-// [queue, router_done, routing, -, gu_done[nent], hq_ready[nent], tile_done[n_dn]]
-enum : int { kCQueue = 0, kCRouterDone = 1, kCRouting = 2, kCHeader = 4 };
+// [router_done, -, -, -, gu_done[nent]]; gu_done[e] counts (unit, token)
+// pairs of entry e whose h codes are published.
+enum : int { kCRouterDone = 0, kCHeader = 4 };
+
+// One expert of the batch union: entry 0 is the shared expert, entry 1 + a
+// the a-th routed expert in ascending id order.
+struct EntryInfo {
+    int expert;  // routed expert id, -1 for the shared expert
+    int slot0;   // first h / y slot (bucketed position)
+    int n;       // tokens
+    int tok[4];
+    int pad;
+};
 
 struct SmallGeom {
-    int nent;       // 1 + max routed entries (entry 0 = shared expert)
-    int n_router;   // router items (2 experts each)
-    int rg;         // gate/up rows per item (per matrix)
-    int ks;         // K-splits per gate/up row (warps per row)
-    int n_gu;       // gate/up items per expert
-    int rd;         // down rows per item (= combine tile)
-    int n_dn;       // down items per expert (= output tiles)
-    int n_static;   // items per CTA taken before the queue (0 or 1)
-    int pos_sel;    // queue index of SELECT
-    int n_fixed;    // items before the routing-dependent part
-    int nslot;      // ring slots
-    int act_bytes;  // per-slot activation area (down items)
+    int grid;
+    int tmax;
+    int nent;      // 1 + max routed entries
+    int n_router;  // router items (2 experts each)
+    int rg;        // gate/up row pairs per chunk
+    int ks;        // warps per pair (K split)
+    int ppw;       // pairs per warp
+    int cpu;       // chunks per unit
+    int nu;        // units per expert
+    int rpc;       // max output rows a CTA owns
+    int rd;        // down rows per chunk
+    int nys;       // output slots (T*k routed + T shared)
+    int nslot;
+    int a_hd;  // act-area offset of the h-scale window (down chunks)
+    int a_sd;  // act-area offset of the row-scale window (down chunks)
+    int act_bytes;
     int slot_bytes;
     int ctrl_words;
-    int sched_words;  // routing schedule record (after the control words)
-    int sched_w_off;  // word offset of the padded weights inside the record
-    int tk_pad;       // T*k rounded up to 4
+    int o_xq, o_xd, o_bar, o_meta, o_rpart, o_gpart, o_usc, o_ent, o_selw, o_inv, o_ys, o_misc;
     int smem_bytes;
-    int tmax;
 };
 
 struct SmallParams {
@@ -107,13 +126,11 @@ struct SmallParams {
     int32_t* perm;
     int32_t* inv_perm;
     int32_t* active;
-    float* hbuf;
     int8_t* hq;
     float* hd;
     float* y;
     float* out;
     int* ctrl;
-    int* sched;
     int32_t* err;
     SmallGeom g;
 };
@@ -122,11 +139,14 @@ struct SlotMeta {
     int kind;
     int entry;   // 0 shared, 1 + a routed
     int expert;  // routed expert id; -1 shared; first expert for router items
-    int row0;
+    int row0;    // first weight row of the chunk (combine: first output row)
     int nrows;
-    int n;       // tokens
-    int slot0;   // first h / y slot
-    int aux;     // down: byte offset of the h scales in the activation area
+    int n;       // tokens of the entry
+    int slot0;   // first h / y slot of the entry
+    int blk;     // gate/up: unit block (h block index); down: row offset inside the CTA's rows
+    int last;    // gate/up: last chunk of its unit
+    int off_a;   // byte offset in the slot: gate scales / h scales
+    int off_b;   // byte offset in the slot: up scales / down row scales
     int tok[4];
 };
 
@@ -134,60 +154,94 @@ struct SlotMeta {
 // Geometry
 // ---------------------------------------------------------------------------
 static int round_up(int v, int a) { return (v + a - 1) / a * a; }
-__host__ __device__ __forceinline__ int round_up_dev(int v, int a) { return (v + a - 1) / a * a; }
 
-SmallGeom small_geometry(const moe_config& c, int T, int sm_count) {
+SmallGeom small_geometry(const moe_config& c, int T, int grid) {
     SmallGeom g{};
     const int H = c.hidden, I = c.inter, E = c.n_experts;
-    const int rbI = I * c.wbits / 8;
+    const int rowH = H * c.wbits / 8, rowI = I * c.wbits / 8;
+    g.grid = grid;
     g.tmax = T <= 1 ? 1 : T <= 2 ? 2 : 4;
     g.nent = 1 + (E < T * c.top_k ? E : T * c.top_k);
     g.n_router = (E + 1) / 2;
-    g.ks = c.wbits == 8 ? 2 : 1;
-    g.rg = kConsumerWarps / g.ks;
-    g.n_gu = I / g.rg;
-    int rd = kSlotWeightBytes / rbI;
-    rd = rd > 64 ? 64 : rd;
-    g.rd = rd / 8 * 8;
-    g.n_dn = (H + g.rd - 1) / g.rd;
-    const int n_sgu = c.n_shared ? g.n_gu : 0;
-    g.n_static = (g.n_router + n_sgu) >= sm_count ? 1 : 0;
-    const int S = g.n_static * sm_count;
-    g.pos_sel = S > g.n_router ? S : g.n_router;
-    g.n_fixed = g.n_router + 1 + (c.n_shared ? n_sgu + 1 : 0);
-    g.nslot = g.tmax == 1 ? 4 : 3;
-    g.act_bytes = round_up(g.tmax * I + g.tmax * (I / 32) * 4 + 32 + 64 * 4, 128);
+    int rg = kSlotWeightBytes / (2 * rowH);
+    rg = rg > kUnit ? kUnit : rg;
+    int p2 = 1;
+    while (p2 * 2 <= rg) p2 *= 2;
+    g.rg = rg >= 1 ? p2 : 0;
+    g.ks = g.rg >= 8 ? 1 : (g.rg > 0 ? 8 / g.rg : 0);
+    g.ppw = g.rg >= 8 ? g.rg / 8 : 1;
+    g.cpu = g.rg > 0 ? kUnit / g.rg : 0;
+    g.nu = I / kUnit;
+    g.rpc = (H + grid - 1) / grid;
+    const int rd = kSlotWeightBytes / rowI;
+    g.rd = rd > kMaxOwnedRows ? kMaxOwnedRows : rd;
+    g.nys = T * c.top_k + T * c.n_shared;
+    g.nslot = kMaxSlots;
+    const int nbI = I / 32;
+    g.a_hd = round_up(g.tmax * I, 16);
+    g.a_sd = g.a_hd + round_up(g.tmax * nbI * 4 + 32, 16);
+    g.act_bytes = round_up(g.a_sd + kMaxOwnedRows * 4 + 32, 128);
+    if (g.act_bytes < 2 * kScaleWin) g.act_bytes = round_up(2 * kScaleWin, 128);
     g.slot_bytes = kSlotWeightBytes + g.act_bytes;
-    g.ctrl_words = round_up(kCHeader + 2 * g.nent + g.n_dn, 4);
-    g.tk_pad = round_up(T * c.top_k, 4);
-    g.sched_w_off = round_up(1 + 8 * (g.nent - 1), 4);
-    g.sched_words = g.sched_w_off + 2 * g.tk_pad;
-    const int nb = H / 32;
-    const int xq_bytes = round_up(g.tmax * H, 128);
-    const int xd_bytes = round_up(g.tmax * nb * 4, 128);
-    const int scratch = 8192;
-    g.smem_bytes = g.nslot * g.slot_bytes + xq_bytes + xd_bytes + scratch;
+    g.ctrl_words = round_up(kCHeader + g.nent, 4);
+    int o = 0;
+    g.o_xq = o;
+    o += round_up(g.tmax * H, 128);
+    g.o_xd = o;
+    o += round_up(g.tmax * (H / 32) * 4, 128);
+    g.o_bar = o;
+    o += 128;  // full[4], empty[4], routing
+    g.o_meta = o;
+    o += round_up((int)sizeof(SlotMeta) * kMaxSlots, 128);
+    g.o_rpart = o;
+    o += 32 * 8;
+    g.o_gpart = o;
+    o += 2 * kUnit * 2 * 8 * 4;  // [buffer][pair][half][gate/up][token]
+    g.o_usc = o;
+    o += 2 * kUnit * 2 * 4;  // [buffer][pair][gate/up] row scales
+    g.o_ent = o;
+    o += round_up(g.nent * (int)sizeof(EntryInfo), 128);
+    g.o_selw = o;
+    o += round_up(T * c.top_k * 4, 128);
+    g.o_inv = o;
+    o += round_up(T * c.top_k * 4, 128);
+    g.o_ys = o;
+    o += round_up(g.nys * g.rpc * 4, 128);
+    g.o_misc = o;
+    o += 128;
+    // as many ring slots (up to four) as the shared memory holds
+    const int smem_max = device_info().max_smem_optin;
+    while (g.nslot > 2 && o + g.nslot * g.slot_bytes > smem_max) --g.nslot;
+    const int ring = g.nslot * g.slot_bytes;
+    g.o_xq += ring; g.o_xd += ring; g.o_bar += ring; g.o_meta += ring; g.o_rpart += ring; g.o_gpart += ring;
+    g.o_usc += ring; g.o_ent += ring; g.o_selw += ring; g.o_inv += ring; g.o_ys += ring; g.o_misc += ring;
+    g.smem_bytes = o + ring;
     return g;
 }
+
+// Scratch the selection needs inside its ring slot (T*E doubles x 3 + tables).
+static int select_scratch_bytes(int T, int E) { return 3 * T * E * 8 + 4 * 32 * 8 + 4 * 128 * 4 + 3 * 256 * 4 + 64; }
 
 bool small_path_supported(const moe_config& c, int T) {
     if (T < 1 || T > 4) return false;
     if (c.hidden > 6144 || c.n_experts > 256 || c.n_groups > 32 || c.top_k > 32) return false;
-    const int rbI = c.inter * c.wbits / 8;
-    if (8 * rbI > kSlotWeightBytes) return false;
-    const int tmax = T <= 1 ? 1 : T <= 2 ? 2 : 4;
-    if (tmax * c.inter * 4 > kSlotWeightBytes) return false;  // h rows of a QUANTISE item
-    return small_geometry(c, T, 148).smem_bytes <= device_info().max_smem_optin;
+    if (2 * c.hidden * 4 > kSlotWeightBytes) return false;  // a router item is two fp32 rows
+    const SmallGeom g = small_geometry(c, T, device_info().sm_count);
+    if (g.rg < 4) return false;  // a gate/up pair is split over at most two warps
+    if (g.rd < 1 || g.rpc > kMaxOwnedRows) return false;
+    if (g.nent > 32 * kMaxEntryWords) return false;
+    if (select_scratch_bytes(T, c.n_experts) > g.slot_bytes) return false;
+    return g.smem_bytes <= device_info().max_smem_optin;
 }
 
 size_t small_ctrl_bytes(const moe_config& c, int T) {
-    const SmallGeom g = small_geometry(c, T > 0 ? T : 1, 148);
-    return (size_t)(g.ctrl_words + g.sched_words) * 4;
+    const SmallGeom g = small_geometry(c, T > 0 ? T : 1, device_info().sm_count);
+    return (size_t)g.ctrl_words * 4;
 }
 
 // ---------------------------------------------------------------------------
 // Prologue: reset the control block and quantise x (launches its dependent
-// right away so the main kernel can start prefetching).
+// right away so the main kernel can start streaming).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_small_prologue(const float* __restrict__ x, int64_t nblk,
                                                         int8_t* __restrict__ xq, float* __restrict__ xd, int* ctrl,
@@ -211,83 +265,81 @@ __global__ void __launch_bounds__(256) k_small_prologue(const float* __restrict_
 // ---------------------------------------------------------------------------
 struct SmemPtrs {
     uint8_t* slots;
-    uint8_t* xq;   // [tmax][2][nb][16]: each 32-code block split in halves
-    float* xd;     // [tmax][nb]
+    uint8_t* xq;  // [tmax][2][nb][16]: each 32-code block split in halves
+    float* xd;    // [tmax][nb]
     uint64_t* full;
     uint64_t* empty;
+    uint64_t* routing;  // consumers -> producer: the routing tables are ready
     SlotMeta* meta;
-    double* rpart;  // [2][4][4]
-    float* gpart;   // [4][2][8]
-    int* sel_idx;   // [4][32]
-    int* cnt;       // [256]
-    int* off;       // [260]
-    int* flags;     // [16] broadcast words
-    int* sched;     // producer's copy of the routing schedule record [1 + 8*128]
+    double* rpart;   // [2][4][4] router partials
+    float* gpart;    // [2][32][2][2][4] gate/up partial dots of a unit
+    float* usc;      // [2][32][2] gate/up row scales of a unit
+    EntryInfo* ent;  // [nent]
+    float* selw;     // [T*k] routing weights
+    int* inv;        // [T*k] slot of pair (t, j)
+    float* ys;       // [nys][rpc] down outputs of the CTA's rows
+    int* misc;       // [0] = routed entries U
 };
 
-__device__ __forceinline__ SmemPtrs carve(uint8_t* base, const SmallGeom& g, int H) {
+__device__ __forceinline__ SmemPtrs carve(uint8_t* base, const SmallGeom& g) {
     SmemPtrs s;
-    uint8_t* p = base;
-    s.slots = p;
-    p += g.nslot * g.slot_bytes;
-    s.xq = p;
-    p += round_up_dev(g.tmax * H, 128);
-    s.xd = reinterpret_cast<float*>(p);
-    p += round_up_dev(g.tmax * (H / 32) * 4, 128);
-    s.full = reinterpret_cast<uint64_t*>(p);
-    p += 8 * kMaxSlots;
-    s.empty = reinterpret_cast<uint64_t*>(p);
-    p += 8 * kMaxSlots;
-    s.rpart = reinterpret_cast<double*>(p);
-    p += sizeof(double) * 32;
-    s.meta = reinterpret_cast<SlotMeta*>(p);
-    p += sizeof(SlotMeta) * kMaxSlots;
-    s.gpart = reinterpret_cast<float*>(p);
-    p += sizeof(float) * 64;
-    s.sel_idx = reinterpret_cast<int*>(p);
-    p += sizeof(int) * 128;
-    s.cnt = reinterpret_cast<int*>(p);
-    p += sizeof(int) * 256;
-    s.off = reinterpret_cast<int*>(p);
-    p += sizeof(int) * 260;
-    s.flags = reinterpret_cast<int*>(p);
-    p += sizeof(int) * 16;
-    s.sched = reinterpret_cast<int*>(p);
+    s.slots = base;
+    s.xq = base + g.o_xq;
+    s.xd = reinterpret_cast<float*>(base + g.o_xd);
+    s.full = reinterpret_cast<uint64_t*>(base + g.o_bar);
+    s.empty = s.full + kMaxSlots;
+    s.routing = s.empty + kMaxSlots;
+    s.meta = reinterpret_cast<SlotMeta*>(base + g.o_meta);
+    s.rpart = reinterpret_cast<double*>(base + g.o_rpart);
+    s.gpart = reinterpret_cast<float*>(base + g.o_gpart);
+    s.usc = reinterpret_cast<float*>(base + g.o_usc);
+    s.ent = reinterpret_cast<EntryInfo*>(base + g.o_ent);
+    s.selw = reinterpret_cast<float*>(base + g.o_selw);
+    s.inv = reinterpret_cast<int*>(base + g.o_inv);
+    s.ys = reinterpret_cast<float*>(base + g.o_ys);
+    s.misc = reinterpret_cast<int*>(base + g.o_misc);
     return s;
 }
 
 // ---------------------------------------------------------------------------
-// Producer: the whole warp runs the loop in lockstep; lane 0 alone touches the
-// queue, the barriers and the copy engine, the other lanes help with polls of
-// many words and with loading the routing schedule.
+// Producer: the whole warp runs the schedule in lockstep; lane 0 owns the
+// barriers, lanes 0..3 issue one copy each, all lanes help poll.
 // ---------------------------------------------------------------------------
+struct Copy {
+    const void* src;
+    uint32_t bytes;
+    uint32_t dst;  // byte offset in the slot
+    bool stream;   // read-once weights: L2 evict-first
+    int first;     // windows: slot offset of the first requested value
+};
+
+__device__ __forceinline__ Copy no_copy() { return Copy{nullptr, 0u, 0u, false, 0}; }
+
+// A 16-byte aligned window over `count` fp32 values at src, placed at slot
+// offset dst.
+__device__ __forceinline__ Copy window(const float* src, int count, uint32_t dst) {
+    const uintptr_t lo = reinterpret_cast<uintptr_t>(src);
+    const uintptr_t hi = lo + (uintptr_t)count * 4u;
+    const uintptr_t alo = lo & ~uintptr_t(15), ahi = (hi + 15) & ~uintptr_t(15);
+    return Copy{reinterpret_cast<const void*>(alo), count > 0 ? (uint32_t)(ahi - alo) : 0u, dst, false,
+                (int)dst + (int)(lo - alo)};
+}
+
 struct Producer {
     const SmallParams& p;
-    SmemPtrs& s;
+    const SmemPtrs& s;
     const int lane;
     uint64_t pol;
     int slot = 0;
     uint32_t pe = 1;  // parity to wait on the empty barriers (fresh ring: all empty)
-    bool routed_known = false;
-    bool aborted = false;  // a wait ran out: stop issuing, drain and exit
-    int U = 0;
-    uint64_t hq_ready_lo = 0, hq_ready_hi = 0, hq_ready_top = 0;  // entries 0..63, 64..127, 128
-    uint32_t issued_mask = 0, issued_par = 0;  // per slot: a copy was issued / its phase parity
+    bool aborted = false;
+    bool need_proxy_fence = false;  // set after acquiring data that later copies read
+    uint32_t issued_mask = 0, issued_par = 0;
+    uint32_t rdy0 = 0, rdy1 = 0, rdy2 = 0, rdy3 = 0, rdy4 = 0;  // entries whose h codes are all published
 
-    __forceinline__ __device__ Producer(const SmallParams& p_, SmemPtrs& s_, int lane_) : p(p_), s(s_), lane(lane_) {
+    __forceinline__ __device__ Producer(const SmallParams& p_, const SmemPtrs& s_, int lane_)
+        : p(p_), s(s_), lane(lane_) {
         pol = l2_evict_first_policy();
-    }
-
-    __forceinline__ __device__ void mark_issued() {
-        issued_mask |= 1u << slot;
-        issued_par = (issued_par & ~(1u << slot)) | ((pe ^ 1u) << slot);
-    }
-
-    __forceinline__ __device__ void advance() {
-        if (++slot == p.g.nslot) {
-            slot = 0;
-            pe ^= 1u;
-        }
     }
 
     __forceinline__ __device__ void fail() {
@@ -295,290 +347,169 @@ struct Producer {
         aborted = true;
     }
 
-    bool need_proxy_fence = false;  // set after acquiring data that the next copies read
-
-    // Poll until *f >= target (lane 0 polls; the result is broadcast).
-    __forceinline__ __device__ bool wait_geq(const int* f, int target) {
-        int ok = 0;
-        need_proxy_fence = true;
-        if (lane == 0) {
-            for (uint32_t i = 0; i < kSpinLimit; ++i) {
-                if (ld_acquire_gpu(f) >= target) {
-                    ok = 1;
-                    break;
-                }
-                __nanosleep(64);
-            }
-        }
-        ok = __shfl_sync(kFull, ok, 0);
-        __syncwarp();
-        if (!ok) fail();
-        return ok != 0;
-    }
-
-    __forceinline__ __device__ bool entry_ready(int e) const {
-        if (e < 64) return (hq_ready_lo >> e) & 1ull;
-        if (e < 128) return (hq_ready_hi >> (e - 64)) & 1ull;
-        return hq_ready_top != 0;
-    }
-
-    // Wait until entry e's h codes are published; every poll reads all
-    // entries' flags at once (one round trip for the whole warp).
-    __forceinline__ __device__ bool wait_hq(int e) {
-        const int* flags = p.ctrl + kCHeader + p.g.nent;
-        if (!entry_ready(e)) need_proxy_fence = true;
-        for (uint32_t it = 0; it < kSpinLimit && !entry_ready(e); ++it) {
-            const bool f0 = lane < p.g.nent && ld_acquire_gpu(flags + lane) >= kWarpSignals;
-            const bool f1 = lane + 32 < p.g.nent && ld_acquire_gpu(flags + lane + 32) >= kWarpSignals;
-            const bool f2 = lane + 64 < p.g.nent && ld_acquire_gpu(flags + lane + 64) >= kWarpSignals;
-            const bool f3 = lane + 96 < p.g.nent && ld_acquire_gpu(flags + lane + 96) >= kWarpSignals;
-            const bool f4 = lane == 0 && 128 < p.g.nent && ld_acquire_gpu(flags + 128) >= kWarpSignals;
-            hq_ready_lo = (uint64_t)__ballot_sync(kFull, f0) | ((uint64_t)__ballot_sync(kFull, f1) << 32);
-            hq_ready_hi = (uint64_t)__ballot_sync(kFull, f2) | ((uint64_t)__ballot_sync(kFull, f3) << 32);
-            hq_ready_top = __ballot_sync(kFull, f4);
-            if (!entry_ready(e)) __nanosleep(128);
-        }
-        __syncwarp();
-        if (!entry_ready(e)) {
-            fail();
-            return false;
-        }
-        return true;
-    }
-
-    __forceinline__ __device__ bool know_routing() {
-        if (routed_known) return true;
-        if (!wait_geq(p.ctrl + kCRouting, 1)) return false;
-        const int words = 1 + 8 * (p.g.nent - 1);
-        for (int i = lane; i < words; i += 32) s.sched[i] = __ldcg(p.sched + i);
-        __syncwarp();
-        const int umax = p.g.nent - 1;
-        const int u = s.sched[0];
-        U = u < 0 ? 0 : (u > umax ? umax : u);
-        routed_known = true;
-        return true;
-    }
-
-    // Tokens of an entry: 0 = shared (every token), 1 + a = routed expert a.
-    __forceinline__ __device__ void entry_tokens(SlotMeta& m, int entry) {
-        if (entry == 0) {
-            m.expert = -1;
-            m.slot0 = p.T * p.k;
-            m.n = p.T;
-            for (int i = 0; i < 4; ++i) m.tok[i] = i < p.T ? i : 0;
-            return;
-        }
-        const int* r = s.sched + 1 + 8 * (entry - 1);
-        int e = r[0], n = r[2];
-        m.expert = (e < 0 || e >= p.E) ? 0 : e;
-        m.slot0 = r[1] < 0 ? 0 : r[1];
-        m.n = n < 0 ? 0 : (n > p.g.tmax ? p.g.tmax : n);
-        for (int i = 0; i < 4; ++i) {
-            const int t = r[3 + i];
-            m.tok[i] = (t < 0 || t >= p.T) ? 0 : t;
-        }
-    }
-
-    // Issue item q (called by the whole warp); returns false once it has
-    // issued the DONE marker or aborted.
-    __forceinline__ __device__ bool issue(int q) {
-        if (aborted) return false;
-        const SmallGeom& g = p.g;
+    __forceinline__ __device__ SlotMeta blank(int kind) const {
         SlotMeta m;
-        m.kind = kItemDone;
+        m.kind = kind;
         m.entry = 0;
         m.expert = -1;
         m.row0 = 0;
         m.nrows = 0;
         m.n = 0;
         m.slot0 = 0;
-        m.aux = 0;
+        m.blk = 0;
+        m.last = 0;
+        m.off_a = 0;
+        m.off_b = 0;
         for (int i = 0; i < 4; ++i) m.tok[i] = 0;
-        const int64_t rowH = (int64_t)p.H * p.wbits / 8, rowI = (int64_t)p.I * p.wbits / 8;
-        const int n_sgu = p.ns ? g.n_gu : 0;
-        // at most 3 fixed copies, plus one per output slot for COMBINE
-        const void *src0 = nullptr, *src1 = nullptr, *src2 = nullptr, *src3 = nullptr;
-        uint32_t by0 = 0, by1 = 0, by2 = 0, by3 = 0;
-        uint32_t dof0 = 0, dof1 = 0, dof2 = 0, dof3 = 0;
-        int ncopy = 0;
-        bool combine_copies = false;
-        if (q < g.n_router) {
-            m.kind = kItemRouter;
-            m.expert = 2 * q;
-            m.nrows = (p.E - 2 * q) < 2 ? (p.E - 2 * q) : 2;
-            src0 = p.router_w + (int64_t)m.expert * p.H;
-            by0 = (uint32_t)(m.nrows * p.H * 4);
-            ncopy = 1;
-        } else if (q == g.pos_sel) {
-            m.kind = kItemSelect;
-        } else if (q < g.n_router + n_sgu + 1) {
-            const int i = q < g.pos_sel ? q - g.n_router : q - g.n_router - 1;
-            m.kind = kItemGateUp;
-            m.entry = 0;
-            m.row0 = i * g.rg;
-            m.nrows = g.rg;
-            entry_tokens(m, 0);
-            src0 = p.shared.w_gate + (int64_t)m.row0 * rowH;
-            src1 = p.shared.w_up + (int64_t)m.row0 * rowH;
-            by0 = by1 = (uint32_t)(g.rg * rowH);
-            dof1 = by0;
-            src2 = p.shared.s_gate + m.row0;
-            src3 = p.shared.s_up + m.row0;
-            by2 = by3 = (uint32_t)(g.rg * 4);
-            dof2 = kSlotWeightBytes;
-            dof3 = kSlotWeightBytes + 64;
-            ncopy = 4;
-        } else {
-            int entry = -1;  // QUANTISE entry
-            if (p.ns && q == g.n_router + n_sgu + 1) {
-                entry = 0;
-            } else {
-                if (!know_routing()) return finish();
-                int r = q - g.n_fixed;
-                // gate/up items of entry b, each followed by the QUANTISE of
-                // entry b-1 (one entry of lag, so that its inputs are done):
-                // G(0) | G(1) Q(0) | G(2) Q(1) | ... | G(U-1) Q(U-2) | Q(U-1)
-                int gu_entry = -1, gu_tile = 0;
-                if (r < g.n_gu) {
-                    gu_entry = 0;
-                    gu_tile = r;
-                } else if (r < U * g.n_gu + U) {
-                    const int r2 = r - g.n_gu, b = 1 + r2 / (g.n_gu + 1), pos = r2 % (g.n_gu + 1);
-                    if (b < U && pos < g.n_gu) {
-                        gu_entry = b;
-                        gu_tile = pos;
-                    } else {
-                        entry = 1 + (b - 1);  // QUANTISE of routed entry b-1
-                    }
-                }
-                if (gu_entry >= 0) {
-                    m.kind = kItemGateUp;
-                    m.entry = 1 + gu_entry;
-                    entry_tokens(m, m.entry);
-                    m.row0 = gu_tile * g.rg;
-                    m.nrows = g.rg;
-                    src0 = p.routed.w_gate + ((int64_t)m.expert * p.I + m.row0) * rowH;
-                    src1 = p.routed.w_up + ((int64_t)m.expert * p.I + m.row0) * rowH;
-                    by0 = by1 = (uint32_t)(g.rg * rowH);
-                    dof1 = by0;
-                    src2 = p.routed.s_gate + (int64_t)m.expert * p.I + m.row0;
-                    src3 = p.routed.s_up + (int64_t)m.expert * p.I + m.row0;
-                    by2 = by3 = (uint32_t)(g.rg * 4);
-                    dof2 = kSlotWeightBytes;
-                    dof3 = kSlotWeightBytes + 64;
-                    ncopy = 4;
-                } else if (entry >= 1) {
-                    // handled below (QUANTISE)
-                } else {
-                    r -= U * g.n_gu + U;  // past the gate/up + QUANTISE region
-                    int down_entry = -1, tile = -1;
-                    if (p.ns && r < g.n_dn) {
-                        down_entry = 0;
-                        tile = r;
-                    } else {
-                        if (p.ns) r -= g.n_dn;
-                        if (r < U * g.n_dn) {
-                            down_entry = 1 + r / g.n_dn;
-                            tile = r % g.n_dn;
-                        } else if ((r -= U * g.n_dn) < g.n_dn) {
-                            // COMBINE of tile r
-                            if (!wait_geq(p.ctrl + kCHeader + 2 * g.nent + r, (U + p.ns) * kWarpSignals))
-                                return finish();
-                            m.kind = kItemCombine;
-                            m.row0 = r * g.rd;
-                            m.nrows = (p.H - m.row0) < g.rd ? (p.H - m.row0) : g.rd;
-                            combine_copies = true;
-                        }
-                    }
-                    if (tile >= 0) {
-                        if (!wait_hq(down_entry)) return finish();
-                        m.kind = kItemDown;
-                        m.entry = down_entry;
-                        entry_tokens(m, down_entry);
-                        m.row0 = tile * g.rd;
-                        m.nrows = (p.H - m.row0) < g.rd ? (p.H - m.row0) : g.rd;
-                        const moe_experts& ex = down_entry ? p.routed : p.shared;
-                        const int eo = down_entry ? m.expert : 0;
-                        src0 = ex.w_down + ((int64_t)eo * p.H + m.row0) * rowI;
-                        by0 = (uint32_t)(m.nrows * rowI);
-                        src1 = p.hq + (int64_t)m.slot0 * p.I;  // h codes (contiguous slots)
-                        by1 = (uint32_t)(m.n * p.I);
-                        dof1 = kSlotWeightBytes;
-                        // h scales: a 16-byte aligned window covering the rows
-                        const int nbI = p.I / 32;
-                        const uintptr_t lo = reinterpret_cast<uintptr_t>(p.hd + (int64_t)m.slot0 * nbI);
-                        const uintptr_t hi = reinterpret_cast<uintptr_t>(p.hd + (int64_t)(m.slot0 + m.n) * nbI);
-                        const uintptr_t alo = lo & ~uintptr_t(15), ahi = (hi + 15) & ~uintptr_t(15);
-                        src2 = reinterpret_cast<const void*>(alo);
-                        by2 = (uint32_t)(ahi - alo);
-                        dof2 = kSlotWeightBytes + round_up_dev(g.tmax * p.I, 16);
-                        m.aux = (int)(dof2 - kSlotWeightBytes) + (int)(lo - alo);
-                        // row scales of the down rows, after the h scales
-                        src3 = ex.s_down + (int64_t)eo * p.H + m.row0;
-                        by3 = (uint32_t)(m.nrows * 4);
-                        dof3 = (uint32_t)(g.act_bytes - 64 * 4) + kSlotWeightBytes;
-                        ncopy = 4;
-                        if (m.n == 0) by1 = by2 = 0;
-                    }
-                }
-            }
-            if (entry >= 0) {
-                // QUANTISE: wait for every gate/up item of the entry, then
-                // bring its h rows (fp32) into the slot
-                if (!wait_geq(p.ctrl + kCHeader + entry, g.n_gu * kWarpSignals)) return finish();
-                if (entry > 0 && !know_routing()) return finish();
-                m.kind = kItemQuant;
-                m.entry = entry;
-                entry_tokens(m, entry);
-                src0 = p.hbuf + (int64_t)m.slot0 * p.I;
-                by0 = (uint32_t)(m.n * p.I * 4);
-                ncopy = 1;
-            }
-        }
-        // ------------------------- hand the item over -------------------------
-        bool ok = true;
-        if (lane == 0) ok = mbar_wait(&s.empty[slot], pe, kWaitLimit);
-        ok = __shfl_sync(kFull, (int)ok, 0) != 0;
+        return m;
+    }
+
+    __forceinline__ __device__ void set_entry(SlotMeta& m, int entry, const EntryInfo& ei) const {
+        m.entry = entry;
+        m.expert = ei.expert;
+        m.n = ei.n;
+        m.slot0 = ei.slot0;
+        for (int i = 0; i < 4; ++i) m.tok[i] = ei.tok[i];
+    }
+
+    // Hand one item over: wait for its slot, publish the meta, arm the full
+    // barrier with the byte count and start the copies (lane i issues copy i).
+    __forceinline__ __device__ bool push(const SlotMeta& m, const Copy& c0, const Copy& c1, const Copy& c2,
+                                         const Copy& c3) {
+        if (aborted) return false;
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait(&s.empty[slot], pe, kWaitLimit) ? 1 : 0;
+        ok = __shfl_sync(kFull, ok, 0);
+        __syncwarp();
         if (!ok) {
             fail();
             return false;
         }
-        uint8_t* dst = s.slots + (size_t)slot * g.slot_bytes;
-        const int ns_slots = p.T * p.k + p.T * p.ns;
-        const uint32_t rb = (uint32_t)m.nrows * 4;
+        uint8_t* dst = s.slots + (size_t)slot * p.g.slot_bytes;
         if (lane == 0) {
             s.meta[slot] = m;
-            uint32_t total = (ncopy > 0 ? by0 : 0u) + (ncopy > 1 ? by1 : 0u) + (ncopy > 2 ? by2 : 0u) +
-                             (ncopy > 3 ? by3 : 0u);
-            if (combine_copies) total = (uint32_t)ns_slots * rb + 2u * (uint32_t)g.tk_pad * 4u;
+            const uint32_t total = c0.bytes + c1.bytes + c2.bytes + c3.bytes;
             if (total == 0) mbar_arrive(&s.full[slot]);
             else mbar_arrive_expect_tx(&s.full[slot], total);
         }
         __syncwarp();
-        // the copies go out from several lanes at once
-        if (need_proxy_fence && lane < 32) fence_proxy_async_global();
-        if (combine_copies) {
-            for (int sl = lane; sl < ns_slots; sl += 32)
-                bulk_g2s_nohint(dst + (size_t)sl * rb, p.y + (int64_t)sl * p.H + m.row0, rb, &s.full[slot]);
-            if (lane == 31)
-                bulk_g2s_nohint(dst + (size_t)ns_slots * rb, p.sched + g.sched_w_off, (uint32_t)g.tk_pad * 8u,
-                                &s.full[slot]);
-        } else if (lane < ncopy) {
-            const void* sp = lane == 0 ? src0 : lane == 1 ? src1 : lane == 2 ? src2 : src3;
-            const uint32_t bb = lane == 0 ? by0 : lane == 1 ? by1 : lane == 2 ? by2 : by3;
-            const uint32_t dd = lane == 0 ? dof0 : lane == 1 ? dof1 : lane == 2 ? dof2 : dof3;
-            if (bb) bulk_g2s(dst + dd, sp, bb, &s.full[slot], pol);
+        if (lane < 4) {
+            const void* src = lane == 0 ? c0.src : lane == 1 ? c1.src : lane == 2 ? c2.src : c3.src;
+            const uint32_t bytes = lane == 0 ? c0.bytes : lane == 1 ? c1.bytes : lane == 2 ? c2.bytes : c3.bytes;
+            const uint32_t off = lane == 0 ? c0.dst : lane == 1 ? c1.dst : lane == 2 ? c2.dst : c3.dst;
+            const bool stream = lane == 0 ? c0.stream : lane == 1 ? c1.stream : lane == 2 ? c2.stream : c3.stream;
+            if (bytes) {
+                if (need_proxy_fence) fence_proxy_async_global();
+                if (stream) bulk_g2s(dst + off, src, bytes, &s.full[slot], pol);
+                else bulk_g2s_nohint(dst + off, src, bytes, &s.full[slot]);
+            }
         }
         __syncwarp();
         need_proxy_fence = false;
-        mark_issued();
-        advance();
-        return m.kind != kItemDone;
+        issued_mask |= 1u << slot;
+        issued_par = (issued_par & ~(1u << slot)) | ((pe ^ 1u) << slot);
+        if (++slot == p.g.nslot) {
+            slot = 0;
+            pe ^= 1u;
+        }
+        return true;
+    }
+
+    __forceinline__ __device__ bool marker(int kind) {
+        return push(blank(kind), no_copy(), no_copy(), no_copy(), no_copy());
+    }
+
+    __forceinline__ __device__ bool router(int q) {
+        SlotMeta m = blank(kItemRouter);
+        m.expert = 2 * q;
+        m.nrows = (p.E - 2 * q) < 2 ? (p.E - 2 * q) : 2;
+        const Copy c0{p.router_w + (int64_t)m.expert * p.H, (uint32_t)(m.nrows * p.H * 4), 0u, true, 0};
+        return push(m, c0, no_copy(), no_copy(), no_copy());
+    }
+
+    // Chunk ch of gate/up unit blk of an entry: rg rows of Wg and of Wu and
+    // their row scales.
+    __forceinline__ __device__ bool gateup(int entry, const EntryInfo& ei, int blk, int ch) {
+        const SmallGeom& g = p.g;
+        SlotMeta m = blank(kItemGateUp);
+        set_entry(m, entry, ei);
+        m.blk = blk;
+        m.last = ch == g.cpu - 1;
+        m.row0 = blk * kUnit + ch * g.rg;
+        m.nrows = g.rg;
+        const moe_experts& ex = entry ? p.routed : p.shared;
+        const int64_t r = (int64_t)(entry ? ei.expert : 0) * p.I + m.row0;
+        const int64_t rowH = (int64_t)p.H * p.wbits / 8;
+        const uint32_t wb = (uint32_t)(g.rg * rowH);
+        const Copy c0{ex.w_gate + r * rowH, wb, 0u, true, 0};
+        const Copy c1{ex.w_up + r * rowH, wb, wb, true, 0};
+        const Copy c2 = window(ex.s_gate + r, g.rg, kSlotWeightBytes);
+        const Copy c3 = window(ex.s_up + r, g.rg, kSlotWeightBytes + kScaleWin);
+        m.off_a = c2.first;
+        m.off_b = c3.first;
+        return push(m, c0, c1, c2, c3);
+    }
+
+    // nrows down rows of an entry starting at row0, with the entry's h codes
+    // and scales and the rows' scales.  lrow = row0 - first owned row.
+    __forceinline__ __device__ bool down(int entry, const EntryInfo& ei, int row0, int nrows, int lrow) {
+        const SmallGeom& g = p.g;
+        SlotMeta m = blank(kItemDown);
+        set_entry(m, entry, ei);
+        m.row0 = row0;
+        m.nrows = nrows;
+        m.blk = lrow;
+        const moe_experts& ex = entry ? p.routed : p.shared;
+        const int64_t eo = entry ? ei.expert : 0;
+        const int64_t rowI = (int64_t)p.I * p.wbits / 8;
+        const int nbI = p.I / 32;
+        const Copy c0{ex.w_down + (eo * p.H + row0) * rowI, (uint32_t)(nrows * rowI), 0u, true, 0};
+        const Copy c1{p.hq + (int64_t)ei.slot0 * p.I, (uint32_t)(ei.n * p.I), (uint32_t)kSlotWeightBytes, false, 0};
+        const Copy c2 = window(p.hd + (int64_t)ei.slot0 * nbI, ei.n * nbI, kSlotWeightBytes + g.a_hd);
+        const Copy c3 = window(ex.s_down + eo * p.H + row0, nrows, kSlotWeightBytes + g.a_sd);
+        m.off_a = c2.first;
+        m.off_b = c3.first;
+        return push(m, c0, c1, c2, c3);
+    }
+
+    // Wait until every unit of entry e has published its h codes.  Each poll
+    // reads all entries' counters at once (one round trip for the warp).
+    __forceinline__ __device__ bool is_ready(int e) const {
+        const int wi = e >> 5;
+        const uint32_t w = wi == 0 ? rdy0 : wi == 1 ? rdy1 : wi == 2 ? rdy2 : wi == 3 ? rdy3 : rdy4;
+        return (w >> (e & 31)) & 1u;
+    }
+
+    __forceinline__ __device__ bool entry_done(int i, int U) const {
+        return i <= U && ld_acquire_gpu(p.ctrl + kCHeader + i) >= p.g.nu * s.ent[i].n;
+    }
+
+    // Wait until every unit of entry e has published its h codes.  Each poll
+    // reads all entries' counters at once (one round trip for the warp).
+    __forceinline__ __device__ bool wait_entry(int e, int U) {
+        if (is_ready(e)) return true;
+        need_proxy_fence = true;
+        for (uint32_t it = 0; it < kSpinLimit; ++it) {
+            const bool f0 = entry_done(lane, U), f1 = entry_done(lane + 32, U), f2 = entry_done(lane + 64, U);
+            const bool f3 = entry_done(lane + 96, U), f4 = entry_done(lane + 128, U);
+            rdy0 = __ballot_sync(kFull, f0);
+            rdy1 = __ballot_sync(kFull, f1);
+            rdy2 = __ballot_sync(kFull, f2);
+            rdy3 = __ballot_sync(kFull, f3);
+            rdy4 = __ballot_sync(kFull, f4);
+            if (is_ready(e)) {
+                __syncwarp();  // the polling lanes' acquires order the copying lanes' reads
+                return true;
+            }
+            __nanosleep(128);
+        }
+        fail();
+        return false;
     }
 
     // After a timeout: hand the consumers a DONE marker if a slot frees up in
-    // time (otherwise they time out on their own), and stop issuing.
-    __forceinline__ __device__ bool finish() {
+    // time (otherwise they time out on their own).
+    __forceinline__ __device__ void finish() {
         int ok = 0;
         if (lane == 0 && mbar_wait(&s.empty[slot], pe, kWaitLimit)) {
             s.meta[slot].kind = kItemDone;
@@ -587,11 +518,9 @@ struct Producer {
         }
         ok = __shfl_sync(kFull, ok, 0);
         if (ok) {
-            mark_issued();
-            advance();
+            issued_mask |= 1u << slot;
+            issued_par = (issued_par & ~(1u << slot)) | ((pe ^ 1u) << slot);
         }
-        aborted = true;
-        return false;
     }
 
     // Before the CTA exits: wait (bounded) for every copy it issued.
@@ -603,24 +532,26 @@ struct Producer {
 };
 
 // ---------------------------------------------------------------------------
-// Consumer helpers
+// Consumer items
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void consumers_sync() { named_barrier(1, kConsumers); }
 
-// SELECT: wait for every router item, then route all tokens and bucket them;
-// publish the schedule record and raise the routing flag.  Same decisions as
-// the multi-kernel router and the reference (group score = two largest c,
-// keep topk_groups groups, then top_k experts in descending c, ties to the
-// lower index, w = s / sum(s) * rsf).  Every decision is a rank: each thread
-// owns one (token, expert) and counts the candidates that beat it, so there
-// are no serial argmax rounds; the item's own ring slot is the scratch.
 __device__ __forceinline__ bool beats(unsigned long long ka, int ia, unsigned long long kb, int ib) {
     return ka > kb || (ka == kb && ia < ib);
 }
 
-__device__ __forceinline__ void do_select(const SmallParams& p, SmemPtrs& s, uint8_t* scratch, int tid) {
+// SELECT: wait for every router item, then route all tokens and bucket them
+// into this CTA's tables (the same in every CTA; CTA 0 also publishes them to
+// the workspace).  Same decisions as the multi-kernel router and the
+// reference: group score = sum of the two largest c = s + bias, keep
+// topk_groups groups, then top_k experts in descending c, ties to the lower
+// index, w = s / sum(s) * rsf with the unbiased s.  Every decision is a rank:
+// each thread owns one (token, expert) and counts the candidates that beat
+// it.  The item's ring slot is the scratch.
+__device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& s, uint8_t* scratch, int tid) {
     const int E = p.E, T = p.T, k = p.k, G = p.G, per = E / G;
     const int TE = T * E;
+    const bool publish = blockIdx.x == 0;
     double* sc = reinterpret_cast<double*>(scratch);                         // [T][E] c = s + bias
     double* ss = sc + TE;                                                     // [T][E] s
     unsigned long long* key = reinterpret_cast<unsigned long long*>(ss + TE);  // [T][E] order key of c
@@ -649,7 +580,7 @@ __device__ __forceinline__ void do_select(const SmallParams& p, SmemPtrs& s, uin
     for (int i = tid; i < TE; i += kConsumers) {
         const double l = __ldcg(p.logits + i);
         const double sv = 1.0 / (1.0 + exp(-l));
-        const double cv = sv + (double)p.bias[i % E];
+        const double cv = sv + (double)__ldg(p.bias + i % E);
         ss[i] = sv;
         sc[i] = cv;
         key[i] = order_key(cv);
@@ -669,7 +600,9 @@ __device__ __forceinline__ void do_select(const SmallParams& p, SmemPtrs& s, uin
     consumers_sync();
     if (tid < T * 32) {
         const int t = tid >> 5, g = tid & 31;
-        if (g < G) gkey[t * 32 + g] = order_key(sc[(size_t)t * E + top1[t * 32 + g]] + sc[(size_t)t * E + top2[t * 32 + g]]);
+        if (g < G)
+            gkey[t * 32 + g] =
+                order_key(sc[(size_t)t * E + top1[t * 32 + g]] + sc[(size_t)t * E + top2[t * 32 + g]]);
     }
     consumers_sync();
     if (tid < T * 32) {
@@ -703,11 +636,12 @@ __device__ __forceinline__ void do_select(const SmallParams& p, SmemPtrs& s, uin
         for (int j = 0; j < k; ++j) ssum += ss[(size_t)t * E + sel[t * 32 + j]];
         const int e = sel[t * 32 + lane];
         const float wv = (float)(ss[(size_t)t * E + e] / ssum * (double)p.rsf);
-        p.idx[(int64_t)t * k + lane] = e;
-        p.w[(int64_t)t * k + lane] = wv;
-        reinterpret_cast<float*>(p.sched + p.g.sched_w_off)[t * k + lane] = wv;
+        s.selw[t * k + lane] = wv;
+        if (publish) {
+            p.idx[(int64_t)t * k + lane] = e;
+            p.w[(int64_t)t * k + lane] = wv;
+        }
     }
-    consumers_sync();
     const int n = T * k;
     if (tid < n) atomicAdd(&cnt[sel[(tid / k) * 32 + tid % k]], 1);
     consumers_sync();
@@ -737,20 +671,29 @@ __device__ __forceinline__ void do_select(const SmallParams& p, SmemPtrs& s, uin
             const int o = b1 + a1 - cv, ai = b2 + a2 - nz;
             off[tid] = o;
             ent[tid] = ai;
-            p.offsets[tid] = o;
-            p.counts[tid] = cv;
             if (cv > 0) {
-                int* r = p.sched + 1 + 8 * ai;  // schedule record of routed entry ai
-                r[0] = tid;
-                r[1] = o;
-                r[2] = cv;
-                p.active[1 + ai] = tid;
+                EntryInfo& ei = s.ent[1 + ai];
+                ei.expert = tid;
+                ei.slot0 = o;
+                ei.n = cv;
             }
-            if (tid == E - 1) {
-                p.offsets[E] = o + cv;
-                p.active[0] = ai + nz;
-                p.sched[0] = ai + nz;
+            if (tid == E - 1) s.misc[0] = ai + nz;
+            if (publish) {
+                p.offsets[tid] = o;
+                p.counts[tid] = cv;
+                if (cv > 0) p.active[1 + ai] = tid;
+                if (tid == E - 1) {
+                    p.offsets[E] = o + cv;
+                    p.active[0] = ai + nz;
+                }
             }
+        }
+        if (tid == 0) {
+            EntryInfo& e0 = s.ent[0];
+            e0.expert = -1;
+            e0.slot0 = n;
+            e0.n = T;
+            for (int i = 0; i < 4; ++i) e0.tok[i] = i < T ? i : 0;
         }
     }
     consumers_sync();
@@ -761,22 +704,23 @@ __device__ __forceinline__ void do_select(const SmallParams& p, SmemPtrs& s, uin
         for (int t2 = 0; t2 < t; ++t2)
             for (int j2 = 0; j2 < k; ++j2) rank += sel[t2 * 32 + j2] == e ? 1 : 0;
         const int pos = off[e] + rank;
-        p.perm[pos] = tid;
-        p.inv_perm[tid] = pos;
-        (p.sched + p.g.sched_w_off + p.g.tk_pad)[tid] = pos;
-        if (rank < 4) p.sched[1 + 8 * ent[e] + 3 + rank] = t;
+        s.inv[tid] = pos;
+        if (rank < 4) s.ent[1 + ent[e]].tok[rank] = t;
+        if (publish) {
+            p.perm[pos] = tid;
+            p.inv_perm[tid] = pos;
+        }
     }
-    consumers_sync();  // every schedule write is done
-    if (tid == 0) st_release_gpu(p.ctrl + kCRouting, 1);
+    consumers_sync();  // every table is written
+    if (tid == 0) mbar_arrive(s.routing);
 }
 
 // ---- router item: logits of two experts for all tokens ----
 // Each lane accumulates its products with the compensated fp32 pair (about
-// 2^-48 relative), the warps' partials are combined in fp64 in a fixed order.
-// Uses shared scratch across warps, so it synchronises the consumer warps.
+// 2^-48 relative); the warps' partials are combined in fp64 in a fixed order.
 template <int TM>
-__device__ __forceinline__ void do_router(const SmallParams& p, SmemPtrs& s, const SlotMeta& m, const uint8_t* slot, int tid,
-                          uint64_t* empty) {
+__device__ __forceinline__ void do_router(const SmallParams& p, const SmemPtrs& s, const SlotMeta& m,
+                                          const uint8_t* slot, int tid, uint64_t* empty) {
     const int warp = tid >> 5, lane = tid & 31;
     const int el = warp >> 2, qq = warp & 3;
     DFAcc acc[TM];
@@ -829,165 +773,111 @@ __device__ __forceinline__ void do_router(const SmallParams& p, SmemPtrs& s, con
     if (tid == 0) red_add_release_gpu(p.ctrl + kCRouterDone, 1);
 }
 
-// Completion signals of one consumer warp, published in batches: the warp's
-// global writes are ordered before one fence, then every pending counter gets
-// a relaxed add (a release pattern).  The batch is flushed every few items and
-// always before the warp could block, so no other item ever waits on a
-// signal that is still held back.
-struct Signals {
-    int* p0 = nullptr;
-    int* p1 = nullptr;
-    int c0 = 0, c1 = 0;
-    int age = 0;
-    __device__ __forceinline__ void flush(int lane) {
-        if (!p0) return;
-        __syncwarp();
-        if (lane == 0) {
-            fence_acq_rel_gpu();
-            red_add_relaxed_gpu(p0, c0);
-            if (p1) red_add_relaxed_gpu(p1, c1);
-        }
-        __syncwarp();
-        p0 = p1 = nullptr;
-        c0 = c1 = 0;
-        age = 0;
-    }
-    __device__ __forceinline__ void add(int* c, int lane) {
-        if (p1 == c) {
-            ++c1;
-        } else if (!p1 && p0 == c) {
-            ++c0;
-        } else if (!p0) {
-            p0 = c;
-            c0 = 1;
-        } else if (!p1) {
-            p1 = c;
-            c1 = 1;
-        } else {
-            flush(lane);
-            p0 = c;
-            c0 = 1;
-        }
-        if (++age >= 4) flush(lane);
-    }
-};
-
-// ---- gate/up item: rg rows of Wg and Wu for the entry's tokens -> h ----
+// ---- gate/up chunk: rg row pairs of one unit -> partial dots; the unit's
+// last chunk turns the 32 rows into h = silu(g) * u, quantises the block and
+// publishes it ----
 template <int WBITS, int TM>
-__device__ __forceinline__ void do_gateup(const SmallParams& p, SmemPtrs& s, const SlotMeta& m, const uint8_t* slot, int tid,
-                          uint64_t* empty, Signals& sig) {
+__device__ __forceinline__ void do_gateup(const SmallParams& p, const SmemPtrs& s, const SlotMeta& m,
+                                          const uint8_t* slot, int tid, uint64_t* empty, int buf) {
     constexpr int V = 2 * TM;
     constexpr int SHIFT = 5 - Log2<V>::value;
     const int warp = tid >> 5, lane = tid & 31;
     const SmallGeom& g = p.g;
-    const int pair = warp % g.rg, half = warp / g.rg;
     const int nb = p.H / 32;
+    const int half = g.ks == 1 ? 0 : warp / g.rg;
     const int per_half = (nb + g.ks - 1) / g.ks;
     const int b_lo = half * per_half, b_hi = min(nb, b_lo + per_half);
     const int64_t rbH = (int64_t)p.H * WBITS / 8;
-    const uint8_t* wg = slot + (size_t)pair * rbH;
-    const uint8_t* wu = slot + (size_t)(g.rg + pair) * rbH;
-    const float* sg = reinterpret_cast<const float*>(slot + kSlotWeightBytes);
-    const float* su = reinterpret_cast<const float*>(slot + kSlotWeightBytes + 64);
-    float acc[V];
+    const float* sg = reinterpret_cast<const float*>(slot + m.off_a);
+    const float* su = reinterpret_cast<const float*>(slot + m.off_b);
+    const int first = m.row0 - m.blk * kUnit;  // first pair of the chunk inside its unit
+    for (int pp = 0; pp < g.ppw; ++pp) {
+        const int pair = g.ks == 1 ? warp + 8 * pp : warp % g.rg;
+        const uint8_t* wg = slot + (size_t)pair * rbH;
+        const uint8_t* wu = slot + (size_t)(g.rg + pair) * rbH;
+        float acc[V];
 #pragma unroll
-    for (int i = 0; i < V; ++i) acc[i] = 0.0f;
-    for (int b = b_lo + lane; b < b_hi; b += 32) {
-        WBlock<WBITS> bg, bu;
-        if constexpr (WBITS == 4) {
-            bg.a = *reinterpret_cast<const uint4*>(wg + 16 * b);
-            bu.a = *reinterpret_cast<const uint4*>(wu + 16 * b);
-        } else {
-            bg.a = *reinterpret_cast<const uint4*>(wg + 32 * b);
-            bg.b = *reinterpret_cast<const uint4*>(wg + 32 * b + 16);
-            bu.a = *reinterpret_cast<const uint4*>(wu + 32 * b);
-            bu.b = *reinterpret_cast<const uint4*>(wu + 32 * b + 16);
-        }
+        for (int i = 0; i < V; ++i) acc[i] = 0.0f;
+        for (int b = b_lo + lane; b < b_hi; b += 32) {
+            WBlock<WBITS> bg, bu;
+            if constexpr (WBITS == 4) {
+                bg.a = *reinterpret_cast<const uint4*>(wg + 16 * b);
+                bu.a = *reinterpret_cast<const uint4*>(wu + 16 * b);
+            } else {
+                bg.a = *reinterpret_cast<const uint4*>(wg + 32 * b);
+                bg.b = *reinterpret_cast<const uint4*>(wg + 32 * b + 16);
+                bu.a = *reinterpret_cast<const uint4*>(wu + 32 * b);
+                bu.b = *reinterpret_cast<const uint4*>(wu + 32 * b + 16);
+            }
 #pragma unroll
-        for (int i = 0; i < TM; ++i) {
-            if (i < m.n) {
-                const int t = m.tok[i];
-                const uint4 lo = *reinterpret_cast<const uint4*>(s.xq + ((size_t)(t * 2 + 0) * nb + b) * 16);
-                const uint4 hi = *reinterpret_cast<const uint4*>(s.xq + ((size_t)(t * 2 + 1) * nb + b) * 16);
-                ActBlock a;
-                if constexpr (WBITS == 4) a = act_nibble_order(lo, hi);
-                else a = act_natural(lo, hi);
-                const float dx = s.xd[t * nb + b];
-                acc[i] = fmaf(dx, (float)dot_block<WBITS>(bg, a), acc[i]);
-                acc[TM + i] = fmaf(dx, (float)dot_block<WBITS>(bu, a), acc[TM + i]);
+            for (int i = 0; i < TM; ++i) {
+                if (i < m.n) {
+                    const int t = m.tok[i];
+                    const uint4 lo = *reinterpret_cast<const uint4*>(s.xq + ((size_t)(t * 2 + 0) * nb + b) * 16);
+                    const uint4 hi = *reinterpret_cast<const uint4*>(s.xq + ((size_t)(t * 2 + 1) * nb + b) * 16);
+                    ActBlock a;
+                    if constexpr (WBITS == 4) a = act_nibble_order(lo, hi);
+                    else a = act_natural(lo, hi);
+                    const float dx = s.xd[t * nb + b];
+                    acc[i] = fmaf(dx, (float)dot_block<WBITS>(bg, a), acc[i]);
+                    acc[TM + i] = fmaf(dx, (float)dot_block<WBITS>(bu, a), acc[TM + i]);
+                }
             }
         }
-    }
-    const float v = warp_reduce_many<V>(acc, lane);
-    const float vu = __shfl_down_sync(kFull, v, 16);
-    const int vi = lane >> SHIFT;
-    const bool rep = lane < 16 && (lane & ((1 << SHIFT) - 1)) == 0;  // one lane per (g, token)
-    int* counter = p.ctrl + kCHeader + m.entry;
-    if (g.ks == 1) {
-        const float sgv = sg[pair], suv = su[pair];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty);
+        const float v = warp_reduce_many<V>(acc, lane);
+        const float vu = __shfl_down_sync(kFull, v, 16);
+        const int vi = lane >> SHIFT;
+        const bool rep = lane < 16 && (lane & ((1 << SHIFT) - 1)) == 0;  // one lane per token
+        const int up = first + pair;
         if (rep && vi < m.n) {
-            const float gv = sgv * v, uv = suv * vu;
-            p.hbuf[(int64_t)(m.slot0 + vi) * p.I + m.row0 + pair] = silu_mul(gv, uv);
+            float* gp = s.gpart + ((buf * kUnit + up) * 2 + half) * 8;
+            gp[vi] = v;
+            gp[4 + vi] = vu;
         }
-        sig.add(counter, lane);
-    } else {
-        if (rep) {
-            s.gpart[(pair * 2 + half) * 8 + vi] = v;
-            s.gpart[(pair * 2 + half) * 8 + 4 + vi] = vu;
+        if (half == 0 && lane == 0) {
+            s.usc[(buf * kUnit + up) * 2] = sg[pair];
+            s.usc[(buf * kUnit + up) * 2 + 1] = su[pair];
         }
-        consumers_sync();
-        if (tid < g.rg * TM) {
-            const int pr = tid / TM, i = tid % TM;
-            if (i < m.n) {
-                const float gsum = s.gpart[(pr * 2) * 8 + i] + s.gpart[(pr * 2 + 1) * 8 + i];
-                const float usum = s.gpart[(pr * 2) * 8 + 4 + i] + s.gpart[(pr * 2 + 1) * 8 + 4 + i];
-                p.hbuf[(int64_t)(m.slot0 + i) * p.I + m.row0 + pr] = silu_mul(sg[pr] * gsum, su[pr] * usum);
-            }
-        }
-        consumers_sync();  // h written by the first warp; gpart free for the next item
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty);
-        sig.add(counter, lane);
-    }
-}
-
-// ---- QUANTISE: Q8_0 of an entry's h rows (in the slot), published ----
-__device__ __forceinline__ void do_quant(const SmallParams& p, const SlotMeta& m, const uint8_t* slot, int tid, uint64_t* empty,
-                         Signals& sig) {
-    const int warp = tid >> 5, lane = tid & 31;
-    const int nbI = p.I / 32;
-    const float* h = reinterpret_cast<const float*>(slot);
-    for (int job = warp; job < m.n * nbI; job += kConsumerWarps) {
-        const int i = job / nbI, bb = job % nbI;
-        int8_t q;
-        float d;
-        q8_0_warp(h[(size_t)i * p.I + bb * 32 + lane], q, d);
-        const int64_t sl = m.slot0 + i;
-        p.hq[sl * p.I + bb * 32 + lane] = q;
-        if (lane == 0) p.hd[sl * nbI + bb] = d;
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty);
-    sig.add(p.ctrl + kCHeader + p.g.nent + m.entry, lane);
-    sig.flush(lane);  // a whole expert's down items wait for this one
+    if (!m.last) return;
+    consumers_sync();  // every pair of the unit is in gpart
+    if (warp < m.n) {
+        const int i = warp;
+        const float* gp = s.gpart + ((buf * kUnit + lane) * 2) * 8;
+        float gs = gp[i], us = gp[4 + i];
+        if (g.ks == 2) {
+            gs = gs + gp[8 + i];
+            us = us + gp[12 + i];
+        }
+        const float h = silu_mul(s.usc[(buf * kUnit + lane) * 2] * gs, s.usc[(buf * kUnit + lane) * 2 + 1] * us);
+        int8_t q;
+        float d;
+        q8_0_warp(h, q, d);
+        const int64_t sl = m.slot0 + i;
+        p.hq[sl * p.I + m.blk * kUnit + lane] = q;
+        if (lane == 0) p.hd[sl * (p.I / 32) + m.blk] = d;
+        __syncwarp();
+        if (lane == 0) {
+            fence_acq_rel_gpu();  // the warp's h codes before the count (release pattern)
+            red_add_relaxed_gpu(p.ctrl + kCHeader + m.entry, 1);
+        }
+    }
 }
 
-// ---- down item: rd rows of Wd for the entry's tokens -> y ----
+// ---- down chunk: nrows rows of Wd for the entry's tokens -> y ----
 template <int WBITS, int TM>
-__device__ __forceinline__ void do_down(const SmallParams& p, const SlotMeta& m, const uint8_t* slot, int tid, uint64_t* empty,
-                        Signals& sig) {
+__device__ __forceinline__ void do_down(const SmallParams& p, const SmemPtrs& s, const SlotMeta& m,
+                                        const uint8_t* slot, int tid, uint64_t* empty) {
     constexpr int V = 8 * TM;
     constexpr int SHIFT = 5 - Log2<V>::value;
     const int warp = tid >> 5, lane = tid & 31;
-    const SmallGeom& g = p.g;
     const int nbI = p.I / 32;
     const int64_t rbI = (int64_t)p.I * WBITS / 8;
     const uint8_t* act = slot + kSlotWeightBytes;
-    const float* hdv = reinterpret_cast<const float*>(act + m.aux);
-    const float* sdv = reinterpret_cast<const float*>(act + g.act_bytes - 64 * 4);
-    const int rpw = g.rd / 8;
+    const float* hdv = reinterpret_cast<const float*>(slot + m.off_a);
+    const float* sdv = reinterpret_cast<const float*>(slot + m.off_b);
     float acc[V];
 #pragma unroll
     for (int i = 0; i < V; ++i) acc[i] = 0.0f;
@@ -1007,7 +897,7 @@ __device__ __forceinline__ void do_down(const SmallParams& p, const SlotMeta& m,
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int r = warp + 8 * j;
-            if (j < rpw && r < m.nrows) {
+            if (r < m.nrows) {
                 const uint8_t* row = slot + (size_t)r * rbI;
                 WBlock<WBITS> wb;
                 if constexpr (WBITS == 4) {
@@ -1026,30 +916,31 @@ __device__ __forceinline__ void do_down(const SmallParams& p, const SlotMeta& m,
     const int vi = lane >> SHIFT;
     const int j = vi / TM, i = vi % TM;
     const int r = warp + 8 * j;
-    const bool mine = (lane & ((1 << SHIFT) - 1)) == 0 && j < rpw && r < m.nrows && i < m.n;
+    const bool mine = (lane & ((1 << SHIFT) - 1)) == 0 && r < m.nrows && i < m.n;
     const float sd = mine ? sdv[r] : 0.0f;
     __syncwarp();
     if (lane == 0) mbar_arrive(empty);
-    if (mine) p.y[(int64_t)(m.slot0 + i) * p.H + m.row0 + r] = sd * v;
-    sig.add(p.ctrl + kCHeader + 2 * g.nent + m.row0 / g.rd, lane);
+    if (mine) {
+        const float yv = sd * v;
+        s.ys[(m.slot0 + i) * p.g.rpc + m.blk + r] = yv;
+        p.y[(int64_t)(m.slot0 + i) * p.H + m.row0 + r] = yv;
+    }
 }
 
-// ---- COMBINE: out rows of one tile from every slot's y (in the slot) ----
-__device__ __forceinline__ void do_combine(const SmallParams& p, const SlotMeta& m, const uint8_t* slot, int tid, uint64_t* empty) {
-    const int rows = m.nrows;
-    const int ns_slots = p.T * p.k + p.T * p.ns;
-    const float* ys = reinterpret_cast<const float*>(slot);
-    const float* wv = ys + (size_t)ns_slots * rows;
-    const int* inv = reinterpret_cast<const int*>(wv + p.g.tk_pad);
-    for (int idx = tid; idx < p.T * rows; idx += kConsumers) {
-        const int t = idx / rows, r = idx % rows;
+// ---- COMBINE: the CTA's output rows from its per-slot down outputs ----
+__device__ __forceinline__ void do_combine(const SmallParams& p, const SmemPtrs& s, const SlotMeta& m, int tid,
+                                           uint64_t* empty) {
+    consumers_sync();  // every warp's down outputs are in ys
+    const int rows = m.nrows, T = p.T, k = p.k, rpc = p.g.rpc;
+    for (int idx = tid; idx < T * rows; idx += kConsumers) {
+        const int t = idx / rows, r = idx - t * rows;
         float acc = 0.0f;  // fixed order: slots 0..k-1, then the shared expert
-        for (int j = 0; j < p.k; ++j) {
-            int sl = inv[t * p.k + j];
-            sl = (sl < 0 || sl >= p.T * p.k) ? 0 : sl;
-            acc = fmaf(wv[t * p.k + j], ys[(size_t)sl * rows + r], acc);
+        for (int j = 0; j < k; ++j) {
+            int sl = s.inv[t * k + j];
+            sl = (sl < 0 || sl >= T * k) ? 0 : sl;
+            acc = fmaf(s.selw[t * k + j], s.ys[sl * rpc + r], acc);
         }
-        if (p.ns) acc += ys[(size_t)(p.T * p.k + t) * rows + r];
+        if (p.ns) acc += s.ys[(T * k + t) * rpc + r];
         p.out[(int64_t)t * p.H + m.row0 + r] = acc;
     }
     __syncwarp();
@@ -1062,14 +953,18 @@ __device__ __forceinline__ void do_combine(const SmallParams& p, const SlotMeta&
 template <int WBITS, int TM>
 __global__ void __launch_bounds__(kSmallThreads, 1) k_moe_small(const __grid_constant__ SmallParams p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    SmemPtrs s = carve(smem_raw, p.g, p.H);
+    const SmemPtrs s = carve(smem_raw, p.g);
+    const SmallGeom& g = p.g;
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x, grid = gridDim.x;
+    const int r0 = (int)((int64_t)p.H * c / grid), r1 = (int)((int64_t)p.H * (c + 1) / grid);
     if (tid == 0) {
-        for (int i = 0; i < p.g.nslot; ++i) {
+        for (int i = 0; i < g.nslot; ++i) {
             mbar_init(&s.full[i], 1);
             mbar_init(&s.empty[i], kConsumerWarps);
         }
+        mbar_init(s.routing, 1);
         fence_barrier_init();
     }
     __syncthreads();
@@ -1077,20 +972,54 @@ __global__ void __launch_bounds__(kSmallThreads, 1) k_moe_small(const __grid_con
     if (warp == kConsumerWarps) {
         // ------------------------- producer -------------------------
         Producer pr(p, s, lane);
-        // the first item depends on nothing from the prologue
-        if (p.g.n_static) pr.issue(blockIdx.x);
+        // router rows depend on nothing from the prologue
+        for (int q = c; q < g.n_router; q += grid) pr.router(q);
+        const int64_t rowI = (int64_t)p.I * p.wbits / 8;
+        if (p.ns && lane == 0 && r1 > r0)
+            bulk_prefetch_l2(p.shared.w_down + (int64_t)r0 * rowI, (uint32_t)((r1 - r0) * rowI));
         pdl_wait();
-        const int base = p.g.n_static * gridDim.x;
-        // two consecutive items per queue atomic; the next batch index is
-        // requested one batch ahead so its round trip overlaps the issue
-        int pending = 0;
-        if (lane == 0) pending = atom_add_relaxed_gpu(p.ctrl + kCQueue, 1);
-        while (true) {
-            const int q = base + 2 * __shfl_sync(kFull, pending, 0);
-            if (lane == 0) pending = atom_add_relaxed_gpu(p.ctrl + kCQueue, 1);
-            if (!pr.issue(q)) break;
-            if (!pr.issue(q + 1)) break;
+        pr.marker(kItemSelect);
+        // the shared expert's gate/up units need no routing
+        EntryInfo e0;
+        e0.expert = -1;
+        e0.slot0 = p.T * p.k;
+        e0.n = p.T;
+        for (int i = 0; i < 4; ++i) e0.tok[i] = i < p.T ? i : 0;
+        const int n_pre = p.ns ? g.nu : 0;
+        for (int u = c; u < n_pre; u += grid)
+            for (int ch = 0; ch < g.cpu; ++ch) pr.gateup(0, e0, u, ch);
+        // the routed part of the schedule needs this CTA's routing tables
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait(s.routing, 0, kConsumerWaitLimit) ? 1 : 0;
+        ok = __shfl_sync(kFull, ok, 0);
+        __syncwarp();  // lane 0's acquire of the tables orders the other lanes' reads
+        if (!ok) pr.fail();
+        const int umax = g.nent - 1;
+        int U = s.misc[0];
+        U = U < 0 ? 0 : (U > umax ? umax : U);
+        const int first = p.ns ? 0 : 1;
+        const int n_units = (p.ns + U) * g.nu;
+        for (int u = c; u < n_units && !pr.aborted; u += grid) {
+            if (u < n_pre) continue;
+            const int entry = first + u / g.nu, blk = u % g.nu;
+            const EntryInfo ei = s.ent[entry];
+            for (int ch = 0; ch < g.cpu; ++ch) pr.gateup(entry, ei, blk, ch);
         }
+        for (int entry = first; entry <= U && !pr.aborted; ++entry) {
+            const EntryInfo ei = s.ent[entry];
+            for (int rr = r0; rr < r1; rr += g.rd) {
+                if (!pr.wait_entry(entry, U)) break;
+                pr.down(entry, ei, rr, (r1 - rr) < g.rd ? (r1 - rr) : g.rd, rr - r0);
+            }
+        }
+        if (!pr.aborted) {
+            SlotMeta m = pr.blank(kItemCombine);
+            m.row0 = r0;
+            m.nrows = r1 - r0;
+            pr.push(m, no_copy(), no_copy(), no_copy(), no_copy());
+        }
+        if (!pr.aborted) pr.marker(kItemDone);
+        if (pr.aborted) pr.finish();
         pr.drain();
         return;
     }
@@ -1109,48 +1038,38 @@ __global__ void __launch_bounds__(kSmallThreads, 1) k_moe_small(const __grid_con
         for (int job = tid; job < p.T * nb; job += kConsumers) s.xd[job] = __ldcg(p.xd + job);
     }
     consumers_sync();
-    // Every consumer warp walks the ring on its own; only items that combine
-    // partial results across warps (router, select, int8 gate/up) synchronise.
     int slot = 0;
     uint32_t pf = 0;
-    Signals sig;
+    int buf = 0;  // gate/up partials double buffer, flipped after each unit
     while (true) {
-        if (!mbar_try_wait(&s.full[slot], pf)) {
-            sig.flush(lane);  // about to block: publish what this warp has done
-            if (!mbar_wait(&s.full[slot], pf, kConsumerWaitLimit)) {
-                set_error(p.err, kErrTimeout);
-                break;
-            }
+        if (!mbar_wait(&s.full[slot], pf, kConsumerWaitLimit)) {
+            set_error(p.err, kErrTimeout);
+            break;
         }
         const SlotMeta m = s.meta[slot];
-        const uint8_t* data = s.slots + (size_t)slot * p.g.slot_bytes;
+        uint8_t* data = s.slots + (size_t)slot * g.slot_bytes;
         uint64_t* empty = &s.empty[slot];
         if (m.kind == kItemGateUp) {
-            if (p.g.ks != 1) sig.flush(lane);  // this item synchronises the warps
-            do_gateup<WBITS, TM>(p, s, m, data, tid, empty, sig);
+            do_gateup<WBITS, TM>(p, s, m, data, tid, empty, buf);
+            if (m.last) buf ^= 1;
         } else if (m.kind == kItemDown) {
-            do_down<WBITS, TM>(p, m, data, tid, empty, sig);
+            do_down<WBITS, TM>(p, s, m, data, tid, empty);
         } else if (m.kind == kItemRouter) {
-            sig.flush(lane);
             do_router<TM>(p, s, m, data, tid, empty);
-        } else if (m.kind == kItemQuant) {
-            do_quant(p, m, data, tid, empty, sig);
-        } else if (m.kind == kItemCombine) {
-            do_combine(p, m, data, tid, empty);
         } else if (m.kind == kItemSelect) {
-            sig.flush(lane);
-            do_select(p, s, const_cast<uint8_t*>(data), tid);
+            do_select(p, s, data, tid);
             __syncwarp();
             if (lane == 0) mbar_arrive(empty);  // the slot was the scratch
+        } else if (m.kind == kItemCombine) {
+            do_combine(p, s, m, tid, empty);
         } else {
             break;  // DONE (or an unknown marker)
         }
-        if (++slot == p.g.nslot) {
+        if (++slot == g.nslot) {
             slot = 0;
             pf ^= 1u;
         }
     }
-    sig.flush(lane);
 }
 
 // ---------------------------------------------------------------------------
@@ -1169,7 +1088,7 @@ static cudaError_t launch_small_t(const SmallParams& prm, cudaStream_t st) {
         attr_done[dev] = true;
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(device_info().sm_count);
+    cfg.gridDim = dim3(prm.g.grid);
     cfg.blockDim = dim3(kSmallThreads);
     cfg.dynamicSmemBytes = prm.g.smem_bytes;
     cfg.stream = st;
@@ -1189,9 +1108,8 @@ cudaError_t launch_small(const SmallArgs& a, cudaStream_t st) {
     p.x = a.x; p.router_w = a.router_w; p.bias = a.bias; p.routed = a.routed; p.shared = a.shared;
     p.xq = a.xq; p.xd = a.xd; p.logits = a.logits; p.idx = a.idx; p.w = a.w; p.counts = a.counts;
     p.offsets = a.offsets; p.perm = a.perm; p.inv_perm = a.inv_perm; p.active = a.active;
-    p.hbuf = a.hbuf; p.hq = a.hq; p.hd = a.hd; p.y = a.y; p.out = a.out; p.ctrl = a.ctrl; p.err = a.err;
+    p.hq = a.hq; p.hd = a.hd; p.y = a.y; p.out = a.out; p.ctrl = a.ctrl; p.err = a.err;
     p.g = small_geometry(c, a.T, device_info().sm_count);
-    p.sched = a.ctrl + p.g.ctrl_words;
     if (p.g.smem_bytes > device_info().max_smem_optin) return cudaErrorInvalidConfiguration;
     const int64_t nblk = (int64_t)a.T * (c.hidden / 32);
     const int grid = (int)((nblk + 7) / 8) > 1 ? (int)((nblk + 7) / 8) : 1;
