@@ -51,6 +51,17 @@ constexpr int kUnit = 32;          // gate/up rows per unit: one Q8_0 block of h
 constexpr int kMaxOwnedRows = 64;  // output rows one CTA owns
 constexpr int kScaleWin = 160;     // 16-byte aligned window over <= 32 fp32 scales
 constexpr int kMaxEntryWords = 5;  // ready bitmask words (entries <= 160)
+// Thread layout of the gate/up and down chunks: the 64 threads of a warp
+// pair (w, w+1) split the columns (K blocks c, c + 64, ...), the 4 warp pairs
+// split the rows.  Each thread loads its activation blocks once per chunk and
+// reuses them for all its rows; its dots are independent chains.  A row's
+// sum is the two warps' butterfly sums, added half 0 + half 1.
+constexpr int kColThreads = 64;
+constexpr int kRowGroups = 4;  // = consumer warps / 2
+constexpr int kRowBatch = 4;       // rows reduced together
+constexpr int kMaxGuBlocks = 3;    // hidden / 32 <= 192 blocks over 64 column threads
+constexpr int kMaxDownBlocks = 8;  // inter / 32 <= 512
+
 // Bounds of every wait (legitimate waits last microseconds): mbarrier
 // try_wait iterations, and polls of a global word with a short sleep each.
 constexpr uint32_t kWaitLimit = 1u << 20;
@@ -91,8 +102,6 @@ struct SmallGeom {
     int nent;      // 1 + max routed entries
     int n_router;  // router items (2 experts each)
     int rg;        // gate/up row pairs per chunk
-    int ks;        // warps per pair (K split)
-    int ppw;       // pairs per warp
     int cpu;       // chunks per unit
     int nu;        // units per expert
     int rpc;       // max output rows a CTA owns
@@ -168,8 +177,6 @@ SmallGeom small_geometry(const moe_config& c, int T, int grid) {
     int p2 = 1;
     while (p2 * 2 <= rg) p2 *= 2;
     g.rg = rg >= 1 ? p2 : 0;
-    g.ks = g.rg >= 8 ? 1 : (g.rg > 0 ? 8 / g.rg : 0);
-    g.ppw = g.rg >= 8 ? g.rg / 8 : 1;
     g.cpu = g.rg > 0 ? kUnit / g.rg : 0;
     g.nu = I / kUnit;
     g.rpc = (H + grid - 1) / grid;
@@ -206,7 +213,7 @@ SmallGeom small_geometry(const moe_config& c, int T, int grid) {
     g.o_inv = o;
     o += round_up(T * c.top_k * 4, 128);
     g.o_ys = o;
-    o += round_up(g.nys * g.rpc * 4, 128);
+    o += round_up(g.nys * g.rpc * 8, 128);
     g.o_misc = o;
     o += 128;
     // as many ring slots (up to four) as the shared memory holds
@@ -227,7 +234,8 @@ bool small_path_supported(const moe_config& c, int T) {
     if (c.hidden > 6144 || c.n_experts > 256 || c.n_groups > 32 || c.top_k > 32) return false;
     if (2 * c.hidden * 4 > kSlotWeightBytes) return false;  // a router item is two fp32 rows
     const SmallGeom g = small_geometry(c, T, device_info().sm_count);
-    if (g.rg < 4) return false;  // a gate/up pair is split over at most two warps
+    if (g.rg < 4) return false;  // at least one gate/up row per row group
+    if (c.hidden / 32 > kColThreads * kMaxGuBlocks || c.inter / 32 > kColThreads * kMaxDownBlocks) return false;
     if (g.rd < 1 || g.rpc > kMaxOwnedRows) return false;
     if (g.nent > 32 * kMaxEntryWords) return false;
     if (select_scratch_bytes(T, c.n_experts) > g.slot_bytes) return false;
@@ -265,19 +273,19 @@ __global__ void __launch_bounds__(256) k_small_prologue(const float* __restrict_
 // ---------------------------------------------------------------------------
 struct SmemPtrs {
     uint8_t* slots;
-    uint8_t* xq;  // [tmax][2][nb][16]: each 32-code block split in halves
+    uint8_t* xq;  // [tmax][2][nb][16]: each 32-code block in the weights' order, split in halves
     float* xd;    // [tmax][nb]
     uint64_t* full;
     uint64_t* empty;
     uint64_t* routing;  // consumers -> producer: the routing tables are ready
     SlotMeta* meta;
     double* rpart;   // [2][4][4] router partials
-    float* gpart;    // [2][32][2][2][4] gate/up partial dots of a unit
+    float* gpart;    // [2][32][2][2][4] gate/up partial dots of a unit: [buffer][pair][gate/up][half][token]
     float* usc;      // [2][32][2] gate/up row scales of a unit
     EntryInfo* ent;  // [nent]
     float* selw;     // [T*k] routing weights
     int* inv;        // [T*k] slot of pair (t, j)
-    float* ys;       // [nys][rpc] down outputs of the CTA's rows
+    float* ys;       // [nys][rpc][2] down outputs of the CTA's rows, per column half
     int* misc;       // [0] = routed entries U
 };
 
@@ -773,70 +781,94 @@ __device__ __forceinline__ void do_router(const SmallParams& p, const SmemPtrs& 
     if (tid == 0) red_add_release_gpu(p.ctrl + kCRouterDone, 1);
 }
 
+// m.tok[i] with a run-time i, without indexing a local array.
+__device__ __forceinline__ int tok_at(const SlotMeta& m, int i) {
+    return i == 0 ? m.tok[0] : i == 1 ? m.tok[1] : i == 2 ? m.tok[2] : m.tok[3];
+}
+
+template <int WBITS>
+__device__ __forceinline__ WBlock<WBITS> load_block_smem(const uint8_t* row, int b) {
+    WBlock<WBITS> w;
+    if constexpr (WBITS == 4) {
+        w.a = *reinterpret_cast<const uint4*>(row + 16 * b);
+        w.b = make_uint4(0, 0, 0, 0);
+    } else {
+        w.a = *reinterpret_cast<const uint4*>(row + 32 * b);
+        w.b = *reinterpret_cast<const uint4*>(row + 32 * b + 16);
+    }
+    return w;
+}
+
 // ---- gate/up chunk: rg row pairs of one unit -> partial dots; the unit's
 // last chunk turns the 32 rows into h = silu(g) * u, quantises the block and
 // publishes it ----
 template <int WBITS, int TM>
 __device__ __forceinline__ void do_gateup(const SmallParams& p, const SmemPtrs& s, const SlotMeta& m,
                                           const uint8_t* slot, int tid, uint64_t* empty, int buf) {
-    constexpr int V = 2 * TM;
+    constexpr int V = kRowBatch * TM;
     constexpr int SHIFT = 5 - Log2<V>::value;
     const int warp = tid >> 5, lane = tid & 31;
     const SmallGeom& g = p.g;
     const int nb = p.H / 32;
-    const int half = g.ks == 1 ? 0 : warp / g.rg;
-    const int per_half = (nb + g.ks - 1) / g.ks;
-    const int b_lo = half * per_half, b_hi = min(nb, b_lo + per_half);
+    const int half = warp & 1, q = warp >> 1;
+    const int c = half * 32 + lane;
     const int64_t rbH = (int64_t)p.H * WBITS / 8;
+    const int rpg = 2 * g.rg / kRowGroups;  // rows per group: gate rows 0..rg-1, then up rows
+    const int first = m.row0 - m.blk * kUnit;  // first pair of the chunk inside its unit
     const float* sg = reinterpret_cast<const float*>(slot + m.off_a);
     const float* su = reinterpret_cast<const float*>(slot + m.off_b);
-    const int first = m.row0 - m.blk * kUnit;  // first pair of the chunk inside its unit
-    for (int pp = 0; pp < g.ppw; ++pp) {
-        const int pair = g.ks == 1 ? warp + 8 * pp : warp % g.rg;
-        const uint8_t* wg = slot + (size_t)pair * rbH;
-        const uint8_t* wu = slot + (size_t)(g.rg + pair) * rbH;
+    // Branch-free inner loops (so that the independent dots interleave):
+    // out-of-range blocks are clamped and get a zero scale, out-of-range rows
+    // and tokens are clamped and their sums are never stored.
+    const int nlast = m.n > 0 ? m.n - 1 : 0;
+    for (int rb = 0; rb < rpg; rb += kRowBatch) {
         float acc[V];
 #pragma unroll
-        for (int i = 0; i < V; ++i) acc[i] = 0.0f;
-        for (int b = b_lo + lane; b < b_hi; b += 32) {
-            WBlock<WBITS> bg, bu;
-            if constexpr (WBITS == 4) {
-                bg.a = *reinterpret_cast<const uint4*>(wg + 16 * b);
-                bu.a = *reinterpret_cast<const uint4*>(wu + 16 * b);
-            } else {
-                bg.a = *reinterpret_cast<const uint4*>(wg + 32 * b);
-                bg.b = *reinterpret_cast<const uint4*>(wg + 32 * b + 16);
-                bu.a = *reinterpret_cast<const uint4*>(wu + 32 * b);
-                bu.b = *reinterpret_cast<const uint4*>(wu + 32 * b + 16);
-            }
+        for (int v = 0; v < V; ++v) acc[v] = 0.0f;
+        const uint8_t* rowp[kRowBatch];
+#pragma unroll
+        for (int rr = 0; rr < kRowBatch; ++rr) {
+            const int r = min(q * rpg + rb + rr, q * rpg + rpg - 1);
+            rowp[rr] = slot + (size_t)r * rbH;
+        }
+#pragma unroll
+        for (int j = 0; j < kMaxGuBlocks; ++j) {
+            const int bj = c + kColThreads * j;
+            const bool okb = bj < nb;
+            const int b = okb ? bj : 0;
+            ActBlock a[TM];
+            float dx[TM];
+            int cr[TM];
 #pragma unroll
             for (int i = 0; i < TM; ++i) {
-                if (i < m.n) {
-                    const int t = m.tok[i];
-                    const uint4 lo = *reinterpret_cast<const uint4*>(s.xq + ((size_t)(t * 2 + 0) * nb + b) * 16);
-                    const uint4 hi = *reinterpret_cast<const uint4*>(s.xq + ((size_t)(t * 2 + 1) * nb + b) * 16);
-                    ActBlock a;
-                    if constexpr (WBITS == 4) a = act_nibble_order(lo, hi);
-                    else a = act_natural(lo, hi);
-                    const float dx = s.xd[t * nb + b];
-                    acc[i] = fmaf(dx, (float)dot_block<WBITS>(bg, a), acc[i]);
-                    acc[TM + i] = fmaf(dx, (float)dot_block<WBITS>(bu, a), acc[TM + i]);
-                }
+                const int t = tok_at(m, i < nlast ? i : nlast);
+                a[i] = act_natural(*reinterpret_cast<const uint4*>(s.xq + ((size_t)(t * 2 + 0) * nb + b) * 16),
+                                   *reinterpret_cast<const uint4*>(s.xq + ((size_t)(t * 2 + 1) * nb + b) * 16));
+                dx[i] = okb ? s.xd[t * nb + b] * dot_unscale<WBITS>() : 0.0f;
+                cr[i] = act_corr<WBITS>(a[i]);
+            }
+#pragma unroll
+            for (int rr = 0; rr < kRowBatch; ++rr) {
+                const WBlock<WBITS> w = load_block_smem<WBITS>(rowp[rr], b);
+#pragma unroll
+                for (int i = 0; i < TM; ++i)
+                    acc[rr * TM + i] = fmaf(dx[i], (float)dot_block_scaled<WBITS>(w, a[i], cr[i]), acc[rr * TM + i]);
             }
         }
         const float v = warp_reduce_many<V>(acc, lane);
-        const float vu = __shfl_down_sync(kFull, v, 16);
         const int vi = lane >> SHIFT;
-        const bool rep = lane < 16 && (lane & ((1 << SHIFT) - 1)) == 0;  // one lane per token
-        const int up = first + pair;
-        if (rep && vi < m.n) {
-            float* gp = s.gpart + ((buf * kUnit + up) * 2 + half) * 8;
-            gp[vi] = v;
-            gp[4 + vi] = vu;
+        const int rr = vi / TM, i = vi % TM;
+        if ((lane & ((1 << SHIFT) - 1)) == 0 && rb + rr < rpg && i < m.n) {
+            const int r = q * rpg + rb + rr;
+            const int gu = r < g.rg ? 0 : 1;
+            const int up = first + (gu ? r - g.rg : r);
+            s.gpart[(((buf * kUnit + up) * 2 + gu) * 2 + half) * 4 + i] = v;
         }
-        if (half == 0 && lane == 0) {
-            s.usc[(buf * kUnit + up) * 2] = sg[pair];
-            s.usc[(buf * kUnit + up) * 2 + 1] = su[pair];
+        if (half == 0 && lane < kRowBatch && rb + lane < rpg) {
+            const int r = q * rpg + rb + lane;
+            const int gu = r < g.rg ? 0 : 1;
+            const int up = first + (gu ? r - g.rg : r);
+            s.usc[(buf * kUnit + up) * 2 + gu] = gu ? su[r - g.rg] : sg[r];
         }
     }
     __syncwarp();
@@ -845,18 +877,15 @@ __device__ __forceinline__ void do_gateup(const SmallParams& p, const SmemPtrs& 
     consumers_sync();  // every pair of the unit is in gpart
     if (warp < m.n) {
         const int i = warp;
-        const float* gp = s.gpart + ((buf * kUnit + lane) * 2) * 8;
-        float gs = gp[i], us = gp[4 + i];
-        if (g.ks == 2) {
-            gs = gs + gp[8 + i];
-            us = us + gp[12 + i];
-        }
+        const float* gp = s.gpart + (buf * kUnit + lane) * 16;  // [gate/up][half][token]
+        const float gs = gp[i] + gp[4 + i];
+        const float us = gp[8 + i] + gp[12 + i];
         const float h = silu_mul(s.usc[(buf * kUnit + lane) * 2] * gs, s.usc[(buf * kUnit + lane) * 2 + 1] * us);
-        int8_t q;
+        int8_t qv;
         float d;
-        q8_0_warp(h, q, d);
+        q8_0_warp(h, qv, d);
         const int64_t sl = m.slot0 + i;
-        p.hq[sl * p.I + m.blk * kUnit + lane] = q;
+        p.hq[sl * p.I + m.blk * kUnit + lane] = qv;
         if (lane == 0) p.hd[sl * (p.I / 32) + m.blk] = d;
         __syncwarp();
         if (lane == 0) {
@@ -866,82 +895,121 @@ __device__ __forceinline__ void do_gateup(const SmallParams& p, const SmemPtrs& 
     }
 }
 
+// Activation block b of the down chunk's h codes (natural order in the slot)
+// for every token, in the weights' order; blocks past the end get zero scale.
+template <int WBITS, int TM>
+__device__ __forceinline__ void down_act(const uint8_t* act, const float* hdv, int I, int nbI, int n, int bj,
+                                         ActBlock (&a)[TM], float (&dh)[TM], int (&cr)[TM]) {
+    const bool okb = bj < nbI;
+    const int b = okb ? bj : 0;
+#pragma unroll
+    for (int i = 0; i < TM; ++i) {
+        const int ii = i < n ? i : 0;
+        const uint4 lo = *reinterpret_cast<const uint4*>(act + (size_t)ii * I + 32 * b);
+        const uint4 hi = *reinterpret_cast<const uint4*>(act + (size_t)ii * I + 32 * b + 16);
+        if constexpr (WBITS == 4) a[i] = act_nibble_order(lo, hi);
+        else a[i] = act_natural(lo, hi);
+        dh[i] = okb ? hdv[ii * nbI + b] * dot_unscale<WBITS>() : 0.0f;
+        cr[i] = act_corr<WBITS>(a[i]);
+    }
+}
+
+// acc[rr][i] += dh[i] * dot(row rr, block b; token i) for a batch of rows.
+template <int WBITS, int TM>
+__device__ __forceinline__ void rows_dot(const uint8_t* const (&rowp)[kRowBatch], int b, const ActBlock (&a)[TM],
+                                         const float (&dh)[TM], const int (&cr)[TM], float (&acc)[kRowBatch * TM]) {
+#pragma unroll
+    for (int rr = 0; rr < kRowBatch; ++rr) {
+        const WBlock<WBITS> w = load_block_smem<WBITS>(rowp[rr], b);
+#pragma unroll
+        for (int i = 0; i < TM; ++i)
+            acc[rr * TM + i] = fmaf(dh[i], (float)dot_block_scaled<WBITS>(w, a[i], cr[i]), acc[rr * TM + i]);
+    }
+}
+
 // ---- down chunk: nrows rows of Wd for the entry's tokens -> y ----
+// Rows are dealt to the row groups round-robin (r = q + 4 k); the half-1
+// warp of a pair hands its sums to the half-0 warp through shared memory.
 template <int WBITS, int TM>
 __device__ __forceinline__ void do_down(const SmallParams& p, const SmemPtrs& s, const SlotMeta& m,
                                         const uint8_t* slot, int tid, uint64_t* empty) {
-    constexpr int V = 8 * TM;
+    constexpr int V = kRowBatch * TM;
     constexpr int SHIFT = 5 - Log2<V>::value;
     const int warp = tid >> 5, lane = tid & 31;
     const int nbI = p.I / 32;
+    const int half = warp & 1, q = warp >> 1;
+    const int c = half * 32 + lane;
     const int64_t rbI = (int64_t)p.I * WBITS / 8;
     const uint8_t* act = slot + kSlotWeightBytes;
     const float* hdv = reinterpret_cast<const float*>(slot + m.off_a);
     const float* sdv = reinterpret_cast<const float*>(slot + m.off_b);
-    float acc[V];
+    // branch-free inner loops, as in the gate/up chunk; column block 0 of
+    // the thread is loaded once, further ones (inter > 2048) per row batch
+    const int nbj = (nbI + kColThreads - 1) / kColThreads;
+    ActBlock a0[TM];
+    float dh0[TM];
+    int cr0[TM];
+    const int b0 = c < nbI ? c : 0;
+    down_act<WBITS, TM>(act, hdv, p.I, nbI, m.n, c, a0, dh0, cr0);
+    const int nk = (m.nrows - q + kRowGroups - 1) / kRowGroups;  // rows of this group
+    const int klast = nk > 0 ? nk - 1 : 0;
+    for (int kb = 0; kb < nk; kb += kRowBatch) {
+        float acc[V];
 #pragma unroll
-    for (int i = 0; i < V; ++i) acc[i] = 0.0f;
-    for (int b = lane; b < nbI; b += 32) {
-        ActBlock a[TM];
-        float dh[TM];
+        for (int v = 0; v < V; ++v) acc[v] = 0.0f;
+        const uint8_t* rowp[kRowBatch];
 #pragma unroll
-        for (int i = 0; i < TM; ++i) {
-            if (i < m.n) {
-                const uint4 lo = *reinterpret_cast<const uint4*>(act + (size_t)i * p.I + 32 * b);
-                const uint4 hi = *reinterpret_cast<const uint4*>(act + (size_t)i * p.I + 32 * b + 16);
-                if constexpr (WBITS == 4) a[i] = act_nibble_order(lo, hi);
-                else a[i] = act_natural(lo, hi);
-                dh[i] = hdv[i * nbI + b];
-            }
+        for (int rr = 0; rr < kRowBatch; ++rr) {
+            const int k = kb + rr < klast ? kb + rr : klast;
+            rowp[rr] = slot + (size_t)(q + kRowGroups * k) * rbI;
         }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int r = warp + 8 * j;
-            if (r < m.nrows) {
-                const uint8_t* row = slot + (size_t)r * rbI;
-                WBlock<WBITS> wb;
-                if constexpr (WBITS == 4) {
-                    wb.a = *reinterpret_cast<const uint4*>(row + 16 * b);
-                } else {
-                    wb.a = *reinterpret_cast<const uint4*>(row + 32 * b);
-                    wb.b = *reinterpret_cast<const uint4*>(row + 32 * b + 16);
-                }
-#pragma unroll
-                for (int i = 0; i < TM; ++i)
-                    if (i < m.n) acc[j * TM + i] = fmaf(dh[i], (float)dot_block<WBITS>(wb, a[i]), acc[j * TM + i]);
-            }
+        rows_dot<WBITS, TM>(rowp, b0, a0, dh0, cr0, acc);
+        for (int j = 1; j < nbj; ++j) {
+            ActBlock aj[TM];
+            float dhj[TM];
+            int crj[TM];
+            const int bj = c + kColThreads * j;
+            down_act<WBITS, TM>(act, hdv, p.I, nbI, m.n, bj, aj, dhj, crj);
+            rows_dot<WBITS, TM>(rowp, bj < nbI ? bj : 0, aj, dhj, crj, acc);
         }
+        const float v = warp_reduce_many<V>(acc, lane);
+        const int vi = lane >> SHIFT;
+        const int rr = vi / TM, i = vi % TM;
+        const int r = q + kRowGroups * (kb + rr);
+        if ((lane & ((1 << SHIFT) - 1)) == 0 && kb + rr < nk && i < m.n)
+            s.ys[((m.slot0 + i) * p.g.rpc + m.blk + r) * 2 + half] = sdv[r] * v;
     }
-    const float v = warp_reduce_many<V>(acc, lane);
-    const int vi = lane >> SHIFT;
-    const int j = vi / TM, i = vi % TM;
-    const int r = warp + 8 * j;
-    const bool mine = (lane & ((1 << SHIFT) - 1)) == 0 && r < m.nrows && i < m.n;
-    const float sd = mine ? sdv[r] : 0.0f;
     __syncwarp();
     if (lane == 0) mbar_arrive(empty);
-    if (mine) {
-        const float yv = sd * v;
-        s.ys[(m.slot0 + i) * p.g.rpc + m.blk + r] = yv;
-        p.y[(int64_t)(m.slot0 + i) * p.H + m.row0 + r] = yv;
-    }
 }
 
-// ---- COMBINE: the CTA's output rows from its per-slot down outputs ----
+// ---- COMBINE: the CTA's output rows from its per-slot down outputs (the
+// two column halves of each row are added here, half 0 + half 1) ----
 __device__ __forceinline__ void do_combine(const SmallParams& p, const SmemPtrs& s, const SlotMeta& m, int tid,
                                            uint64_t* empty) {
     consumers_sync();  // every warp's down outputs are in ys
     const int rows = m.nrows, T = p.T, k = p.k, rpc = p.g.rpc;
+    const float2* ys = reinterpret_cast<const float2*>(s.ys);
     for (int idx = tid; idx < T * rows; idx += kConsumers) {
         const int t = idx / rows, r = idx - t * rows;
         float acc = 0.0f;  // fixed order: slots 0..k-1, then the shared expert
         for (int j = 0; j < k; ++j) {
             int sl = s.inv[t * k + j];
             sl = (sl < 0 || sl >= T * k) ? 0 : sl;
-            acc = fmaf(s.selw[t * k + j], s.ys[sl * rpc + r], acc);
+            const float2 h = ys[sl * rpc + r];
+            acc = fmaf(s.selw[t * k + j], h.x + h.y, acc);
         }
-        if (p.ns) acc += s.ys[(T * k + t) * rpc + r];
+        if (p.ns) {
+            const float2 h = ys[(T * k + t) * rpc + r];
+            acc += h.x + h.y;
+        }
         p.out[(int64_t)t * p.H + m.row0 + r] = acc;
+    }
+    // the per-slot outputs of these rows, for inspection
+    for (int idx = tid; idx < p.g.nys * rows; idx += kConsumers) {
+        const int sl = idx / rows, r = idx - sl * rows;
+        const float2 h = ys[sl * rpc + r];
+        p.y[(int64_t)sl * p.H + m.row0 + r] = h.x + h.y;
     }
     __syncwarp();
     if ((tid & 31) == 0) mbar_arrive(empty);
@@ -1030,10 +1098,13 @@ __global__ void __launch_bounds__(kSmallThreads, 1) k_moe_small(const __grid_con
         // Q8_0 activations of all tokens into shared memory, each 32-code
         // block split in 16-byte halves so that lanes read consecutive words
         const int nb = p.H / 32;
-        for (int job = tid; job < p.T * nb * 2; job += kConsumers) {
-            const int t = job / (2 * nb), rem = job % (2 * nb), half = rem / nb, b = rem % nb;
-            const uint4 v = __ldcg(reinterpret_cast<const uint4*>(p.xq + (int64_t)t * p.H + b * 32 + half * 16));
-            *reinterpret_cast<uint4*>(s.xq + ((size_t)(t * 2 + half) * nb + b) * 16) = v;
+        for (int job = tid; job < p.T * nb; job += kConsumers) {
+            const int t = job / nb, b = job % nb;
+            const uint4 lo = __ldcg(reinterpret_cast<const uint4*>(p.xq + (int64_t)t * p.H + b * 32));
+            const uint4 hi = __ldcg(reinterpret_cast<const uint4*>(p.xq + (int64_t)t * p.H + b * 32 + 16));
+            const ActBlock a = WBITS == 4 ? act_nibble_order(lo, hi) : act_natural(lo, hi);
+            *reinterpret_cast<uint4*>(s.xq + ((size_t)(t * 2 + 0) * nb + b) * 16) = make_uint4(a.v[0], a.v[1], a.v[2], a.v[3]);
+            *reinterpret_cast<uint4*>(s.xq + ((size_t)(t * 2 + 1) * nb + b) * 16) = make_uint4(a.v[4], a.v[5], a.v[6], a.v[7]);
         }
         for (int job = tid; job < p.T * nb; job += kConsumers) s.xd[job] = __ldcg(p.xd + job);
     }
