@@ -197,7 +197,7 @@ SmallGeom small_geometry(const moe_config& c, int T, int grid) {
     g.o_xd = o;
     o += round_up(g.tmax * (H / 32) * 4, 128);
     g.o_bar = o;
-    o += 128;  // full[4], empty[4], routing
+    o += 128;  // full[4], empty[4], routing, ufull[2], ufree[2]
     g.o_meta = o;
     o += round_up((int)sizeof(SlotMeta) * kMaxSlots, 128);
     g.o_rpart = o;
@@ -227,7 +227,7 @@ SmallGeom small_geometry(const moe_config& c, int T, int grid) {
 }
 
 // Scratch the selection needs inside its ring slot (T*E doubles x 3 + tables).
-static int select_scratch_bytes(int T, int E) { return 3 * T * E * 8 + 4 * 32 * 8 + 4 * 128 * 4 + 3 * 256 * 4 + 64; }
+static int select_scratch_bytes(int T, int E) { return 3 * T * E * 8 + 4 * 32 * 8 + T * E * 4 + 2 * 128 * 4 + 3 * 256 * 4 + 64 + T * E * 12; }
 
 bool small_path_supported(const moe_config& c, int T) {
     if (T < 1 || T > 4) return false;
@@ -278,6 +278,8 @@ struct SmemPtrs {
     uint64_t* full;
     uint64_t* empty;
     uint64_t* routing;  // consumers -> producer: the routing tables are ready
+    uint64_t* ufull;    // [2] every consumer warp has written its partials of a unit
+    uint64_t* ufree;    // [2] the unit's finisher has read them
     SlotMeta* meta;
     double* rpart;   // [2][4][4] router partials
     float* gpart;    // [2][32][2][2][4] gate/up partial dots of a unit: [buffer][pair][gate/up][half][token]
@@ -297,6 +299,8 @@ __device__ __forceinline__ SmemPtrs carve(uint8_t* base, const SmallGeom& g) {
     s.full = reinterpret_cast<uint64_t*>(base + g.o_bar);
     s.empty = s.full + kMaxSlots;
     s.routing = s.empty + kMaxSlots;
+    s.ufull = s.routing + 1;
+    s.ufree = s.ufull + 2;
     s.meta = reinterpret_cast<SlotMeta*>(base + g.o_meta);
     s.rpart = reinterpret_cast<double*>(base + g.o_rpart);
     s.gpart = reinterpret_cast<float*>(base + g.o_gpart);
@@ -544,8 +548,20 @@ struct Producer {
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void consumers_sync() { named_barrier(1, kConsumers); }
 
+// (ka, ia) ranks before (kb, ib): larger key, ties to the lower index.
+// Branch-free, so that unrolled compare loops pipeline their loads.
 __device__ __forceinline__ bool beats(unsigned long long ka, int ia, unsigned long long kb, int ib) {
-    return ka > kb || (ka == kb && ia < ib);
+    return (ka > kb) | ((ka == kb) & (ia < ib));
+}
+
+// Arg-max of 64-bit keys over the warp, ties to the lower index: the key's
+// halves go through the warp max-reduction one after the other, the index
+// through a min-reduction over the lanes that hold the maximum.
+__device__ __forceinline__ int warp_argmax_u64(unsigned long long key, int idx) {
+    const uint32_t hi = (uint32_t)(key >> 32), lo = (uint32_t)key;
+    const uint32_t mh = __reduce_max_sync(kFull, hi);
+    const uint32_t ml = __reduce_max_sync(kFull, hi == mh ? lo : 0u);
+    return (int)__reduce_min_sync(kFull, (hi == mh && lo == ml) ? (uint32_t)idx : 0x7FFFFFFFu);
 }
 
 // SELECT: wait for every router item, then route all tokens and bucket them
@@ -553,38 +569,56 @@ __device__ __forceinline__ bool beats(unsigned long long ka, int ia, unsigned lo
 // the workspace).  Same decisions as the multi-kernel router and the
 // reference: group score = sum of the two largest c = s + bias, keep
 // topk_groups groups, then top_k experts in descending c, ties to the lower
-// index, w = s / sum(s) * rsf with the unbiased s.  Every decision is a rank:
-// each thread owns one (token, expert) and counts the candidates that beat
-// it.  The item's ring slot is the scratch.
+// index, w = s / sum(s) * rsf with the unbiased s.  Keys are order-preserving
+// 64-bit images of c.  Every decision is a rank computed by one thread with
+// independent compares, in short phases that keep all warps busy:
+//   1. s, c, keys;  2. each expert's rank inside its group (the best
+//   kc = min(max(top_k, 2), group size) of each group are listed in order);
+//   3. group keys, then each group's rank (kept = rank < topk_groups);
+//   4. each listed expert of a kept group: its rank among the listed experts
+//   of the kept groups (only those can reach the top_k);  5. bucketing.
+// With groups of 32 experts (one warp each) phases 2-4 use warp arg-max
+// rounds instead: k rounds list each group's best k in order, and one warp
+// per token ranks the kept groups' lists with shuffles.
+// The producer is released as soon as the tables it needs are written; the
+// routing weights, needed only by the combine, come last.  The item's ring
+// slot is the scratch.
 __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& s, uint8_t* scratch, int tid) {
-    const int E = p.E, T = p.T, k = p.k, G = p.G, per = E / G;
+    const int E = p.E, T = p.T, k = p.k, G = p.G, per = E / G, tg = p.tg;
     const int TE = T * E;
+    const int kc = min(max(k, 2), per);  // listed experts per group
+    const int kk = min(k, per);          // of which can reach the top_k
     const bool publish = blockIdx.x == 0;
+    const bool fast = per == 32 && G <= kConsumerWarps && tg * kk <= 32;
     double* sc = reinterpret_cast<double*>(scratch);                         // [T][E] c = s + bias
     double* ss = sc + TE;                                                     // [T][E] s
     unsigned long long* key = reinterpret_cast<unsigned long long*>(ss + TE);  // [T][E] order key of c
     unsigned long long* gkey = key + TE;                                      // [T][32] group-score keys
-    int* top1 = reinterpret_cast<int*>(gkey + 4 * 32);                        // [T][32]
-    int* top2 = top1 + 4 * 32;                                                // [T][32]
-    int* kept = top2 + 4 * 32;                                                // [T][32]
-    int* sel = kept + 4 * 32;                                                 // [T][32] picks, by rank
+    int* cand = reinterpret_cast<int*>(gkey + 4 * 32);                        // [T][G][kc] listed experts
+    int* kg = cand + TE;                                                      // [T][32] kept groups
+    int* sel = kg + 4 * 32;                                                   // [T][32] picks, by rank
     int* cnt = sel + 4 * 32;                                                  // [E]
     int* off = cnt + 256;                                                     // [E] exclusive scan of counts
     int* ent = off + 256;                                                     // [E] entry index
     int* wsum = ent + 256;                                                    // [8][2] warp totals
+    unsigned long long* lkey = reinterpret_cast<unsigned long long*>(wsum + 16);  // [T][tg*kk] listed keys
+    int* lid = reinterpret_cast<int*>(lkey + T * p.tg * min(k, per));            // [T][tg*kk] listed ids
     const int warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         int ok = 0;
+#pragma unroll 1
         for (uint32_t i = 0; i < kSpinLimit; ++i) {
             if (ld_acquire_gpu(p.ctrl + kCRouterDone) >= p.g.n_router) {
                 ok = 1;
                 break;
             }
-            __nanosleep(64);
+            __nanosleep(32);
         }
         if (!ok) set_error(p.err, kErrTimeout);  // route on whatever is there; never hang
     }
     consumers_sync();
+    // 1. s, c and keys
+#pragma unroll 1
     for (int i = tid; i < TE; i += kConsumers) {
         const double l = __ldcg(p.logits + i);
         const double sv = 1.0 / (1.0 + exp(-l));
@@ -593,54 +627,257 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
         sc[i] = cv;
         key[i] = order_key(cv);
     }
+#pragma unroll 1
     for (int e = tid; e < E; e += kConsumers) cnt[e] = 0;
     consumers_sync();
-    // group top-2: rank of each expert inside its group
-    for (int i = tid; i < TE; i += kConsumers) {
-        const int t = i / E, e = i - t * E, g = e / per;
-        const unsigned long long* kt = key + (size_t)t * E;
-        const unsigned long long ke = kt[e];
-        int rank = 0;
-        for (int e2 = g * per; e2 < (g + 1) * per; ++e2) rank += beats(kt[e2], e2, ke, e) ? 1 : 0;
-        if (rank == 0) top1[t * 32 + g] = e;
-        if (rank == 1) top2[t * 32 + g] = e;
-    }
-    consumers_sync();
-    if (tid < T * 32) {
-        const int t = tid >> 5, g = tid & 31;
-        if (g < G)
-            gkey[t * 32 + g] =
-                order_key(sc[(size_t)t * E + top1[t * 32 + g]] + sc[(size_t)t * E + top2[t * 32 + g]]);
-    }
-    consumers_sync();
-    if (tid < T * 32) {
-        const int t = tid >> 5, g = tid & 31;
-        if (g < G) {
-            const unsigned long long kg = gkey[t * 32 + g];
+    if (fast) {
+        // GLM-like shape: warp g owns group g (32 experts, one per lane).
+        // 2. each (token, group): its best kc experts in order by k arg-max
+        // rounds (the first two give the group score)
+        if (warp < G) {
+            const int g = warp, e = g * 32 + lane;
+#pragma unroll 1
+            for (int t = 0; t < T; ++t) {
+                unsigned long long kk2 = key[(size_t)t * E + e];
+                const double cme = sc[(size_t)t * E + e];
+                double c12 = 0.0;
+#pragma unroll 1
+                for (int r = 0; r < kc; ++r) {
+                    const int ew = warp_argmax_u64(kk2, e);
+                    if (lane == 0) cand[(t * G + g) * kc + r] = ew;
+                    if (r < 2) c12 += __shfl_sync(kFull, cme, ew & 31);
+                    if (e == ew) kk2 = 0ull;
+                }
+                if (lane == 0) gkey[t * 32 + g] = order_key(c12);
+            }
+        }
+        consumers_sync();
+        // 3. kept groups: each group's rank among the groups of its token
+        if (warp < G && lane < T) {
+            const int g = warp, t = lane;
+            const unsigned long long kgk = gkey[t * 32 + g];
             int rank = 0;
-            for (int g2 = 0; g2 < G; ++g2) rank += beats(gkey[t * 32 + g2], g2, kg, g) ? 1 : 0;
-            kept[t * 32 + g] = rank < p.tg ? 1 : 0;
+#pragma unroll 1
+            for (int g2 = 0; g2 < G; ++g2) rank += beats(gkey[t * 32 + g2], g2, kgk, g) ? 1 : 0;
+            if (rank < tg) kg[t * 32 + rank] = g;
         }
-    }
-    consumers_sync();
-    // top_k experts of the kept groups: rank among the kept experts
-    for (int i = tid; i < TE; i += kConsumers) {
-        const int t = i / E, e = i - t * E;
-        if (!kept[t * 32 + e / per]) continue;
-        const unsigned long long* kt = key + (size_t)t * E;
-        const unsigned long long ke = kt[e];
-        int rank = 0;
-        for (int g2 = 0; g2 < G; ++g2) {
-            if (!kept[t * 32 + g2]) continue;
-            for (int e2 = g2 * per; e2 < (g2 + 1) * per; ++e2) rank += beats(kt[e2], e2, ke, e) ? 1 : 0;
+        consumers_sync();
+        // 4. one warp per token ranks the listed experts of its kept groups
+        if (warp < T) {
+            const int t = warp, nl = tg * kk;
+            const bool act = lane < nl;
+            const int q = act ? lane / kk : 0, r = act ? lane - q * kk : 0;
+            const int e = act ? cand[(t * G + kg[t * 32 + q]) * kc + r] : 0x7FFFFFFF;
+            const unsigned long long ke = act ? key[(size_t)t * E + e] : 0ull;
+            int rank = 0;
+#pragma unroll 1
+            for (int j = 0; j < 32; ++j) {
+                const unsigned long long kj = __shfl_sync(kFull, ke, j);
+                const int ej = __shfl_sync(kFull, e, j);
+                rank += beats(kj, ej, ke, e) ? 1 : 0;
+            }
+            if (act && rank < k) sel[t * 32 + rank] = e;
         }
-        if (rank < k) sel[t * 32 + rank] = e;
+        consumers_sync();
+    } else {
+        // 2. rank inside the group
+    #pragma unroll 1
+        for (int i = tid; i < TE; i += kConsumers) {
+            const int t = i / E, e = i - t * E, g = e / per;
+            const unsigned long long* kt = key + (size_t)t * E + g * per;
+            const unsigned long long ke = kt[e - g * per];
+            int rank = 0;
+    #pragma unroll 1
+            for (int r2 = 0; r2 < per; ++r2) rank += beats(kt[r2], g * per + r2, ke, e) ? 1 : 0;
+            if (rank < kc) cand[(t * G + g) * kc + rank] = e;
+        }
+        consumers_sync();
+        // 3. group keys, then group ranks
+        if (tid < T * G) {
+            const int t = tid / G, g = tid - t * G;
+            const int* cg = cand + (t * G + g) * kc;
+            gkey[t * 32 + g] = order_key(sc[(size_t)t * E + cg[0]] + sc[(size_t)t * E + cg[1]]);
+        }
+        consumers_sync();
+        if (tid < T * G) {
+            const int t = tid / G, g = tid - t * G;
+            const unsigned long long kgk = gkey[t * 32 + g];
+            int rank = 0;
+    #pragma unroll 1
+            for (int g2 = 0; g2 < G; ++g2) rank += beats(gkey[t * 32 + g2], g2, kgk, g) ? 1 : 0;
+            if (rank < tg) kg[t * 32 + rank] = g;
+        }
+        consumers_sync();
+        // 4. final ranks among the listed experts of the kept groups (their keys
+        // and ids gathered first into one contiguous list per token)
+        const int nl = tg * kk;
+    #pragma unroll 1
+        for (int i = tid; i < T * nl; i += kConsumers) {
+            const int t = i / nl, rem = i - t * nl, q = rem / kk, r = rem - q * kk;
+            const int e = cand[(t * G + kg[t * 32 + q]) * kc + r];
+            lkey[i] = key[(size_t)t * E + e];
+            lid[i] = e;
+        }
+        consumers_sync();
+    #pragma unroll 1
+        for (int i = tid; i < T * nl; i += kConsumers) {
+            const int t = i / nl;
+            const unsigned long long* lk = lkey + t * nl;
+            const int* li = lid + t * nl;
+            const unsigned long long ke = lkey[i];
+            const int e = lid[i];
+            int rank = 0;
+    #pragma unroll 1
+            for (int j = 0; j < nl; ++j) rank += beats(lk[j], li[j], ke, e) ? 1 : 0;
+            if (rank < k) sel[t * 32 + rank] = e;
+        }
+        consumers_sync();
     }
-    consumers_sync();
-    // weights from the unbiased sigmoid, summed in pick order
+    // 5. bucketing
+    const int n = T * k;
+    if (n <= 32) {
+        // one warp, lane = pick t * k + j: same-expert lanes found with a
+        // match, positions from counts over the other lanes
+        if (warp == 0) {
+            const bool act = lane < n;
+            const int e = act ? sel[(lane / k) * 32 + lane % k] : 0x7FFFFFFF;
+            const uint32_t same = __match_any_sync(kFull, e);
+            const int lead = __ffs(same) - 1;
+            const int rank = __popc(same & ((1u << lane) - 1u));  // earlier picks (tokens) of this expert
+            int less = 0, dless = 0;  // picks / distinct experts below e
+#pragma unroll 1
+            for (int l2 = 0; l2 < 32; ++l2) {
+                const int e2 = __shfl_sync(kFull, e, l2);
+                const int lead2 = __shfl_sync(kFull, lead, l2);
+                less += e2 < e ? 1 : 0;
+                dless += (e2 < e && lead2 == l2) ? 1 : 0;
+            }
+            if (act) {
+                const int pos = less + rank;
+                s.inv[lane] = pos;
+                if (lane == lead) {
+                    EntryInfo& ei = s.ent[1 + dless];
+                    ei.expert = e;
+                    ei.slot0 = less;
+                    ei.n = __popc(same);
+                }
+                if (publish) {
+                    p.perm[pos] = lane;
+                    p.inv_perm[lane] = pos;
+                    if (lane == lead) p.active[1 + dless] = e;
+                }
+            }
+            __syncwarp();
+            if (act && rank < 4) s.ent[1 + dless].tok[rank] = lane / k;
+            const int U = __popc(__ballot_sync(kFull, act && lane == lead));
+            if (lane == 0) {
+                s.misc[0] = U;
+                if (publish) p.active[0] = U;
+                EntryInfo& e0 = s.ent[0];
+                e0.expert = -1;
+                e0.slot0 = n;
+                e0.n = T;
+#pragma unroll 1
+                for (int i = 0; i < 4; ++i) e0.tok[i] = i < T ? i : 0;
+            }
+        }
+        consumers_sync();  // every table the producer reads is written
+        if (tid == 0) mbar_arrive(s.routing);
+        if (publish) {
+#pragma unroll 1
+            for (int e = tid; e <= E; e += kConsumers) {
+                int o = 0, cv = 0;
+#pragma unroll 1
+                for (int j = 0; j < n; ++j) {
+                    const int ej = sel[(j / k) * 32 + j % k];
+                    o += ej < e ? 1 : 0;
+                    cv += ej == e ? 1 : 0;
+                }
+                p.offsets[e] = o;
+                if (e < E) p.counts[e] = cv;
+            }
+        }
+    } else {
+        if (tid < n) atomicAdd(&cnt[sel[(tid / k) * 32 + tid % k]], 1);
+        consumers_sync();
+        // block-wide exclusive scans over experts (one thread per expert, E <= 256)
+        {
+            const int cv = tid < E ? cnt[tid] : 0, nz = cv > 0 ? 1 : 0;
+            int a1 = cv, a2 = nz;
+    #pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u1 = __shfl_up_sync(kFull, a1, o), u2 = __shfl_up_sync(kFull, a2, o);
+                if (lane >= o) {
+                    a1 += u1;
+                    a2 += u2;
+                }
+            }
+            if (lane == 31) {
+                wsum[warp * 2] = a1;
+                wsum[warp * 2 + 1] = a2;
+            }
+            consumers_sync();
+            int b1 = 0, b2 = 0;
+#pragma unroll 1
+            for (int w = 0; w < warp; ++w) {
+                b1 += wsum[w * 2];
+                b2 += wsum[w * 2 + 1];
+            }
+            if (tid < E) {
+                const int o = b1 + a1 - cv, ai = b2 + a2 - nz;
+                off[tid] = o;
+                ent[tid] = ai;
+                if (cv > 0) {
+                    EntryInfo& ei = s.ent[1 + ai];
+                    ei.expert = tid;
+                    ei.slot0 = o;
+                    ei.n = cv;
+                }
+                if (tid == E - 1) s.misc[0] = ai + nz;
+                if (publish) {
+                    p.offsets[tid] = o;
+                    p.counts[tid] = cv;
+                    if (cv > 0) p.active[1 + ai] = tid;
+                    if (tid == E - 1) {
+                        p.offsets[E] = o + cv;
+                        p.active[0] = ai + nz;
+                    }
+                }
+            }
+            if (tid == 0) {
+                EntryInfo& e0 = s.ent[0];
+                e0.expert = -1;
+                e0.slot0 = n;
+                e0.n = T;
+#pragma unroll 1
+                for (int i = 0; i < 4; ++i) e0.tok[i] = i < T ? i : 0;
+            }
+        }
+        consumers_sync();
+        if (tid < n) {
+            const int t = tid / k;
+            const int e = sel[t * 32 + tid % k];
+            int rank = 0;
+#pragma unroll 1
+            for (int t2 = 0; t2 < t; ++t2)
+#pragma unroll 1
+                for (int j2 = 0; j2 < k; ++j2) rank += sel[t2 * 32 + j2] == e ? 1 : 0;
+            const int pos = off[e] + rank;
+            s.inv[tid] = pos;
+            if (rank < 4) s.ent[1 + ent[e]].tok[rank] = t;
+            if (publish) {
+                p.perm[pos] = tid;
+                p.inv_perm[tid] = pos;
+            }
+        }
+        consumers_sync();  // every table the producer reads is written
+        if (tid == 0) mbar_arrive(s.routing);
+    }
+    // routing weights from the unbiased sigmoid, summed in pick order
     if (warp < T && lane < k) {
         const int t = warp;
         double ssum = 0.0;
+#pragma unroll 1
         for (int j = 0; j < k; ++j) ssum += ss[(size_t)t * E + sel[t * 32 + j]];
         const int e = sel[t * 32 + lane];
         const float wv = (float)(ss[(size_t)t * E + e] / ssum * (double)p.rsf);
@@ -650,125 +887,78 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
             p.w[(int64_t)t * k + lane] = wv;
         }
     }
-    const int n = T * k;
-    if (tid < n) atomicAdd(&cnt[sel[(tid / k) * 32 + tid % k]], 1);
-    consumers_sync();
-    // block-wide exclusive scans over experts (one thread per expert, E <= 256)
-    {
-        const int cv = tid < E ? cnt[tid] : 0, nz = cv > 0 ? 1 : 0;
-        int a1 = cv, a2 = nz;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int u1 = __shfl_up_sync(kFull, a1, o), u2 = __shfl_up_sync(kFull, a2, o);
-            if (lane >= o) {
-                a1 += u1;
-                a2 += u2;
-            }
-        }
-        if (lane == 31) {
-            wsum[warp * 2] = a1;
-            wsum[warp * 2 + 1] = a2;
-        }
-        consumers_sync();
-        int b1 = 0, b2 = 0;
-        for (int w = 0; w < warp; ++w) {
-            b1 += wsum[w * 2];
-            b2 += wsum[w * 2 + 1];
-        }
-        if (tid < E) {
-            const int o = b1 + a1 - cv, ai = b2 + a2 - nz;
-            off[tid] = o;
-            ent[tid] = ai;
-            if (cv > 0) {
-                EntryInfo& ei = s.ent[1 + ai];
-                ei.expert = tid;
-                ei.slot0 = o;
-                ei.n = cv;
-            }
-            if (tid == E - 1) s.misc[0] = ai + nz;
-            if (publish) {
-                p.offsets[tid] = o;
-                p.counts[tid] = cv;
-                if (cv > 0) p.active[1 + ai] = tid;
-                if (tid == E - 1) {
-                    p.offsets[E] = o + cv;
-                    p.active[0] = ai + nz;
-                }
-            }
-        }
-        if (tid == 0) {
-            EntryInfo& e0 = s.ent[0];
-            e0.expert = -1;
-            e0.slot0 = n;
-            e0.n = T;
-            for (int i = 0; i < 4; ++i) e0.tok[i] = i < T ? i : 0;
-        }
-    }
-    consumers_sync();
-    if (tid < n) {
-        const int t = tid / k;
-        const int e = sel[t * 32 + tid % k];
-        int rank = 0;
-        for (int t2 = 0; t2 < t; ++t2)
-            for (int j2 = 0; j2 < k; ++j2) rank += sel[t2 * 32 + j2] == e ? 1 : 0;
-        const int pos = off[e] + rank;
-        s.inv[tid] = pos;
-        if (rank < 4) s.ent[1 + ent[e]].tok[rank] = t;
-        if (publish) {
-            p.perm[pos] = tid;
-            p.inv_perm[tid] = pos;
-        }
-    }
-    consumers_sync();  // every table is written
-    if (tid == 0) mbar_arrive(s.routing);
 }
 
 // ---- router item: logits of two experts for all tokens ----
-// Each lane accumulates its products with the compensated fp32 pair (about
-// 2^-48 relative); the warps' partials are combined in fp64 in a fixed order.
-template <int TM>
+// Warp w takes expert w / 4 of the item and quarter w % 4 of the hidden
+// dimension; each lane keeps four compensated fp32 sums per token (one per
+// float4 component, about 2^-48 relative each), folded into fp64 in a fixed
+// order, and the warps' partials are combined in fp64 in a fixed order.
+// x comes from shared memory (xs, two tokens at a time) when the caller has
+// staged it, else straight from global memory.  The loops stay rolled (this
+// code runs once per call).
+__device__ __forceinline__ void stage_x(const SmallParams& p, float* xs, int t0, int tid) {
+    const int nt = p.T - t0 < 2 ? p.T - t0 : 2;
+    const int n4 = nt * p.H / 4;
+    const float4* src = reinterpret_cast<const float4*>(p.x + (int64_t)t0 * p.H);
+#pragma unroll 4
+    for (int i = tid; i < n4; i += kConsumers) reinterpret_cast<float4*>(xs)[i] = __ldg(src + i);
+}
+
+__device__ __forceinline__ void dfacc4_add(DFAcc (&acc)[4], float4 x, float4 w) {
+    acc[0].add_prod(x.x, w.x);
+    acc[1].add_prod(x.y, w.y);
+    acc[2].add_prod(x.z, w.z);
+    acc[3].add_prod(x.w, w.w);
+}
+
+__device__ __forceinline__ double dfacc4_value(const DFAcc (&acc)[4]) {
+    return (acc[0].value() + acc[1].value()) + (acc[2].value() + acc[3].value());
+}
+
 __device__ __forceinline__ void do_router(const SmallParams& p, const SmemPtrs& s, const SlotMeta& m,
-                                          const uint8_t* slot, int tid, uint64_t* empty) {
+                                          const uint8_t* slot, int tid, uint64_t* empty, float* xs, bool staged) {
     const int warp = tid >> 5, lane = tid & 31;
     const int el = warp >> 2, qq = warp & 3;
-    DFAcc acc[TM];
-    if (el < m.nrows) {
-        const float4* wr = reinterpret_cast<const float4*>(slot) + (size_t)el * (p.H / 4);
-        const int nq = p.H / 16;
-        // 4 float4 per lane per step, all loads issued before the arithmetic
-        for (int j0 = qq * nq + lane; j0 < (qq + 1) * nq; j0 += 4 * 32) {
-#pragma unroll
-            for (int t = 0; t < TM; ++t) {
-                if (t < p.T) {
-                    const float4* xr = reinterpret_cast<const float4*>(p.x + (int64_t)t * p.H);
-                    float4 xv[4], wv[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int j = j0 + 32 * u;
-                        const bool ok = j < (qq + 1) * nq;
-                        xv[u] = ok ? __ldg(xr + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-                        wv[u] = ok ? wr[j] : make_float4(0.f, 0.f, 0.f, 0.f);
-                    }
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        acc[t].add_prod(xv[u].x, wv[u].x);
-                        acc[t].add_prod(xv[u].y, wv[u].y);
-                        acc[t].add_prod(xv[u].z, wv[u].z);
-                        acc[t].add_prod(xv[u].w, wv[u].w);
-                    }
-                }
+    const int nq = p.H / 16;  // float4 per quarter
+    const float4* wr = reinterpret_cast<const float4*>(slot) + (size_t)(el < m.nrows ? el : 0) * (p.H / 4) + qq * nq;
+#pragma unroll 1
+    for (int t0 = 0; t0 < p.T; t0 += 2) {
+        const bool two = t0 + 1 < p.T;
+        const float4* x0;
+        const float4* x1;
+        if (xs) {
+            if (!(staged && t0 == 0)) {
+                consumers_sync();  // the previous pair is no longer read
+                stage_x(p, xs, t0, tid);
+                consumers_sync();
             }
+            x0 = reinterpret_cast<const float4*>(xs) + qq * nq;
+            x1 = x0 + (two ? p.H / 4 : 0);
+        } else {
+            x0 = reinterpret_cast<const float4*>(p.x + (int64_t)t0 * p.H) + qq * nq;
+            x1 = reinterpret_cast<const float4*>(p.x + (int64_t)(two ? t0 + 1 : t0) * p.H) + qq * nq;
+        }
+        DFAcc a0[4], a1[4];
+#pragma unroll 1
+        for (int j = lane; j < nq; j += 32) {
+            const float4 w = wr[j];
+            dfacc4_add(a0, x0[j], w);
+            dfacc4_add(a1, x1[j], w);
+        }
+        double v0 = dfacc4_value(a0), v1 = dfacc4_value(a1);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            v0 += __shfl_xor_sync(kFull, v0, o);
+            v1 += __shfl_xor_sync(kFull, v1, o);
+        }
+        if (lane == 0) {
+            s.rpart[(el * 4 + qq) * 4 + t0] = v0;
+            if (two) s.rpart[(el * 4 + qq) * 4 + t0 + 1] = v1;
         }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty);
-#pragma unroll
-    for (int t = 0; t < TM; ++t) {
-        double v = acc[t].value();
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
-        if (lane == 0) s.rpart[(el * 4 + qq) * 4 + t] = v;
-    }
     consumers_sync();
     if (tid < m.nrows * p.T) {
         const int e2 = tid / p.T, t = tid % p.T;
@@ -804,8 +994,9 @@ __device__ __forceinline__ WBlock<WBITS> load_block_smem(const uint8_t* row, int
 // publishes it ----
 template <int WBITS, int TM>
 __device__ __forceinline__ void do_gateup(const SmallParams& p, const SmemPtrs& s, const SlotMeta& m,
-                                          const uint8_t* slot, int tid, uint64_t* empty, int buf) {
+                                          const uint8_t* slot, int tid, uint64_t* empty, int uc) {
     constexpr int V = kRowBatch * TM;
+    const int buf = uc & 1;
     constexpr int SHIFT = 5 - Log2<V>::value;
     const int warp = tid >> 5, lane = tid & 31;
     const SmallGeom& g = p.g;
@@ -817,6 +1008,9 @@ __device__ __forceinline__ void do_gateup(const SmallParams& p, const SmemPtrs& 
     const int first = m.row0 - m.blk * kUnit;  // first pair of the chunk inside its unit
     const float* sg = reinterpret_cast<const float*>(slot + m.off_a);
     const float* su = reinterpret_cast<const float*>(slot + m.off_b);
+    // the partials buffer of this unit was last read by the finisher of unit uc - 2
+    if (first == 0 && uc >= 2 && !mbar_wait(&s.ufree[buf], ((uc >> 1) - 1) & 1, kConsumerWaitLimit))
+        set_error(p.err, kErrTimeout);
     // Branch-free inner loops (so that the independent dots interleave):
     // out-of-range blocks are clamped and get a zero scale, out-of-range rows
     // and tokens are clamped and their sums are never stored.
@@ -874,24 +1068,30 @@ __device__ __forceinline__ void do_gateup(const SmallParams& p, const SmemPtrs& 
     __syncwarp();
     if (lane == 0) mbar_arrive(empty);
     if (!m.last) return;
-    consumers_sync();  // every pair of the unit is in gpart
-    if (warp < m.n) {
-        const int i = warp;
-        const float* gp = s.gpart + (buf * kUnit + lane) * 16;  // [gate/up][half][token]
+    // Unit end: every warp reports its partials; one warp (rotating, so that
+    // the wait for the slowest warp and the release fence fall on each warp in
+    // turn) finishes the unit while the others go on with the next chunks.
+    if (lane == 0) mbar_arrive(&s.ufull[buf]);
+    if (warp != (uc & (kConsumerWarps - 1))) return;
+    if (!mbar_wait(&s.ufull[buf], (uc >> 1) & 1, kConsumerWaitLimit)) set_error(p.err, kErrTimeout);
+    const float* gp = s.gpart + (buf * kUnit + lane) * 16;  // [gate/up][half][token]
+    const float sgl = s.usc[(buf * kUnit + lane) * 2], sul = s.usc[(buf * kUnit + lane) * 2 + 1];
+    for (int i = 0; i < m.n; ++i) {
         const float gs = gp[i] + gp[4 + i];
         const float us = gp[8 + i] + gp[12 + i];
-        const float h = silu_mul(s.usc[(buf * kUnit + lane) * 2] * gs, s.usc[(buf * kUnit + lane) * 2 + 1] * us);
+        const float h = silu_mul(sgl * gs, sul * us);
         int8_t qv;
         float d;
         q8_0_warp(h, qv, d);
         const int64_t sl = m.slot0 + i;
         p.hq[sl * p.I + m.blk * kUnit + lane] = qv;
         if (lane == 0) p.hd[sl * (p.I / 32) + m.blk] = d;
-        __syncwarp();
-        if (lane == 0) {
-            fence_acq_rel_gpu();  // the warp's h codes before the count (release pattern)
-            red_add_relaxed_gpu(p.ctrl + kCHeader + m.entry, 1);
-        }
+    }
+    __syncwarp();
+    if (lane == 0) {
+        mbar_arrive(&s.ufree[buf]);
+        fence_acq_rel_gpu();  // the warp's h codes before the count (release pattern)
+        red_add_relaxed_gpu(p.ctrl + kCHeader + m.entry, m.n);
     }
 }
 
@@ -915,11 +1115,11 @@ __device__ __forceinline__ void down_act(const uint8_t* act, const float* hdv, i
 }
 
 // acc[rr][i] += dh[i] * dot(row rr, block b; token i) for a batch of rows.
-template <int WBITS, int TM>
-__device__ __forceinline__ void rows_dot(const uint8_t* const (&rowp)[kRowBatch], int b, const ActBlock (&a)[TM],
-                                         const float (&dh)[TM], const int (&cr)[TM], float (&acc)[kRowBatch * TM]) {
+template <int WBITS, int TM, int RB>
+__device__ __forceinline__ void rows_dot(const uint8_t* const (&rowp)[RB], int b, const ActBlock (&a)[TM],
+                                         const float (&dh)[TM], const int (&cr)[TM], float (&acc)[RB * TM]) {
 #pragma unroll
-    for (int rr = 0; rr < kRowBatch; ++rr) {
+    for (int rr = 0; rr < RB; ++rr) {
         const WBlock<WBITS> w = load_block_smem<WBITS>(rowp[rr], b);
 #pragma unroll
         for (int i = 0; i < TM; ++i)
@@ -933,7 +1133,8 @@ __device__ __forceinline__ void rows_dot(const uint8_t* const (&rowp)[kRowBatch]
 template <int WBITS, int TM>
 __device__ __forceinline__ void do_down(const SmallParams& p, const SmemPtrs& s, const SlotMeta& m,
                                         const uint8_t* slot, int tid, uint64_t* empty) {
-    constexpr int V = kRowBatch * TM;
+    constexpr int RB = TM == 1 ? 16 : TM == 2 ? 8 : 4;  // rows of a group reduced together (all at decode)
+    constexpr int V = RB * TM;
     constexpr int SHIFT = 5 - Log2<V>::value;
     const int warp = tid >> 5, lane = tid & 31;
     const int nbI = p.I / 32;
@@ -953,24 +1154,24 @@ __device__ __forceinline__ void do_down(const SmallParams& p, const SmemPtrs& s,
     down_act<WBITS, TM>(act, hdv, p.I, nbI, m.n, c, a0, dh0, cr0);
     const int nk = (m.nrows - q + kRowGroups - 1) / kRowGroups;  // rows of this group
     const int klast = nk > 0 ? nk - 1 : 0;
-    for (int kb = 0; kb < nk; kb += kRowBatch) {
+    for (int kb = 0; kb < nk; kb += RB) {
         float acc[V];
 #pragma unroll
         for (int v = 0; v < V; ++v) acc[v] = 0.0f;
-        const uint8_t* rowp[kRowBatch];
+        const uint8_t* rowp[RB];
 #pragma unroll
-        for (int rr = 0; rr < kRowBatch; ++rr) {
+        for (int rr = 0; rr < RB; ++rr) {
             const int k = kb + rr < klast ? kb + rr : klast;
             rowp[rr] = slot + (size_t)(q + kRowGroups * k) * rbI;
         }
-        rows_dot<WBITS, TM>(rowp, b0, a0, dh0, cr0, acc);
+        rows_dot<WBITS, TM, RB>(rowp, b0, a0, dh0, cr0, acc);
         for (int j = 1; j < nbj; ++j) {
             ActBlock aj[TM];
             float dhj[TM];
             int crj[TM];
             const int bj = c + kColThreads * j;
             down_act<WBITS, TM>(act, hdv, p.I, nbI, m.n, bj, aj, dhj, crj);
-            rows_dot<WBITS, TM>(rowp, bj < nbI ? bj : 0, aj, dhj, crj, acc);
+            rows_dot<WBITS, TM, RB>(rowp, bj < nbI ? bj : 0, aj, dhj, crj, acc);
         }
         const float v = warp_reduce_many<V>(acc, lane);
         const int vi = lane >> SHIFT;
@@ -1033,6 +1234,10 @@ __global__ void __launch_bounds__(kSmallThreads, 1) k_moe_small(const __grid_con
             mbar_init(&s.empty[i], kConsumerWarps);
         }
         mbar_init(s.routing, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s.ufull[i], kConsumerWarps);
+            mbar_init(&s.ufree[i], 1);
+        }
         fence_barrier_init();
     }
     __syncthreads();
@@ -1046,7 +1251,14 @@ __global__ void __launch_bounds__(kSmallThreads, 1) k_moe_small(const __grid_con
         if (p.ns && lane == 0 && r1 > r0)
             bulk_prefetch_l2(p.shared.w_down + (int64_t)r0 * rowI, (uint32_t)((r1 - r0) * rowI));
         pdl_wait();
-        pr.marker(kItemSelect);
+        if (c < g.n_router) {
+            // the SELECT slot also brings x (up to two tokens) for the router item
+            const int nt = p.T < 2 ? p.T : 2;
+            const Copy cx{p.x, (uint32_t)(nt * p.H * 4), 0u, false, 0};
+            pr.push(pr.blank(kItemSelect), cx, no_copy(), no_copy(), no_copy());
+        } else {
+            pr.marker(kItemSelect);
+        }
         // the shared expert's gate/up units need no routing
         EntryInfo e0;
         e0.expert = -1;
@@ -1111,7 +1323,24 @@ __global__ void __launch_bounds__(kSmallThreads, 1) k_moe_small(const __grid_con
     consumers_sync();
     int slot = 0;
     uint32_t pf = 0;
-    int buf = 0;  // gate/up partials double buffer, flipped after each unit
+    int uc = 0;  // gate/up units started by this CTA
+    if (blockIdx.x < g.n_router) {
+        // the first item of a CTA with router work is its router item, the
+        // second its SELECT, whose copy brings x (the first two tokens)
+        float* xs = reinterpret_cast<float*>(s.slots + g.slot_bytes);
+        if (!mbar_wait(&s.full[0], 0, kConsumerWaitLimit)) {
+            set_error(p.err, kErrTimeout);
+            return;
+        }
+        const SlotMeta m = s.meta[0];
+        if (m.kind != kItemRouter) return;  // the producer gave up before its first item
+        if (!mbar_wait(&s.full[1], 0, kConsumerWaitLimit)) {
+            set_error(p.err, kErrTimeout);
+            return;
+        }
+        do_router(p, s, m, s.slots, tid, &s.empty[0], xs, true);
+        slot = 1;
+    }
     while (true) {
         if (!mbar_wait(&s.full[slot], pf, kConsumerWaitLimit)) {
             set_error(p.err, kErrTimeout);
@@ -1121,12 +1350,12 @@ __global__ void __launch_bounds__(kSmallThreads, 1) k_moe_small(const __grid_con
         uint8_t* data = s.slots + (size_t)slot * g.slot_bytes;
         uint64_t* empty = &s.empty[slot];
         if (m.kind == kItemGateUp) {
-            do_gateup<WBITS, TM>(p, s, m, data, tid, empty, buf);
-            if (m.last) buf ^= 1;
+            do_gateup<WBITS, TM>(p, s, m, data, tid, empty, uc);
+            if (m.last) ++uc;
         } else if (m.kind == kItemDown) {
             do_down<WBITS, TM>(p, s, m, data, tid, empty);
         } else if (m.kind == kItemRouter) {
-            do_router<TM>(p, s, m, data, tid, empty);
+            do_router(p, s, m, data, tid, empty, nullptr, false);
         } else if (m.kind == kItemSelect) {
             do_select(p, s, data, tid);
             __syncwarp();

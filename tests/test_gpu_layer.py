@@ -18,6 +18,9 @@ MID4 = synth.LayerShape(1056, 160, 32, 4, 2, 4, 1, 2.5, 4)
 MID8 = synth.LayerShape(1056, 160, 32, 4, 2, 4, 1, 1.0, 8)
 MID4_NOSHARED = synth.LayerShape(512, 96, 24, 3, 2, 3, 0, 1.5, 4)
 FULLGROUPS = synth.LayerShape(256, 64, 16, 4, 2, 8, 1, 2.5, 4)   # top_k = every expert of the kept groups
+# groups of 32 experts (one warp per group in the fused selection), as in the GLM-5.2 shape
+GROUP32 = synth.LayerShape(512, 96, 128, 4, 2, 8, 1, 2.5, 4)
+GROUP32_K16 = synth.LayerShape(256, 64, 64, 2, 1, 16, 1, 1.0, 8)   # one kept group, top_k 16 of its 32
 
 
 @pytest.fixture(scope="module")
@@ -74,6 +77,9 @@ def test_tiny_host_entry_point(tiny):
     (MID4, 4, 13, "correlated"), (MID8, 1, 16, "normal"), (MID4, 1, 17, "normal"), (MID4, 2, 18, "normal"),
     (MID4, 3, 19, "normal"), (MID8, 2, 20, "normal"), (MID8, 4, 21, "correlated"),
     (MID4_NOSHARED, 3, 22, "normal"), (FULLGROUPS, 2, 23, "normal"),
+    (GROUP32, 1, 24, "normal"), (GROUP32, 2, 25, "normal"), (GROUP32, 3, 26, "normal"),
+    (GROUP32, 4, 27, "correlated"), (GROUP32_K16, 1, 28, "normal"), (GROUP32_K16, 4, 29, "normal"),
+    (GROUP32, 6, 30, "normal"),
 ])
 def test_mid_layers(shape, T, seed, x_kind):
     wl = make_workload(f"mid_{shape.wbits}_{T}", shape, T, seed, x_kind=x_kind)
