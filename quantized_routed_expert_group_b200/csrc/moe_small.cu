@@ -657,7 +657,7 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
             const int g = warp, t = lane;
             const unsigned long long kgk = gkey[t * 32 + g];
             int rank = 0;
-#pragma unroll 1
+#pragma unroll 8
             for (int g2 = 0; g2 < G; ++g2) rank += beats(gkey[t * 32 + g2], g2, kgk, g) ? 1 : 0;
             if (rank < tg) kg[t * 32 + rank] = g;
         }
@@ -670,8 +670,8 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
             const int e = act ? cand[(t * G + kg[t * 32 + q]) * kc + r] : 0x7FFFFFFF;
             const unsigned long long ke = act ? key[(size_t)t * E + e] : 0ull;
             int rank = 0;
-#pragma unroll 1
-            for (int j = 0; j < 32; ++j) {
+#pragma unroll 8
+            for (int j = 0; j < 32; ++j) {  // partly unrolled: the shuffles pipeline
                 const unsigned long long kj = __shfl_sync(kFull, ke, j);
                 const int ej = __shfl_sync(kFull, e, j);
                 rank += beats(kj, ej, ke, e) ? 1 : 0;
@@ -745,8 +745,8 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
             const int lead = __ffs(same) - 1;
             const int rank = __popc(same & ((1u << lane) - 1u));  // earlier picks (tokens) of this expert
             int less = 0, dless = 0;  // picks / distinct experts below e
-#pragma unroll 1
-            for (int l2 = 0; l2 < 32; ++l2) {
+#pragma unroll 8
+            for (int l2 = 0; l2 < 32; ++l2) {  // partly unrolled: the shuffles pipeline
                 const int e2 = __shfl_sync(kFull, e, l2);
                 const int lead2 = __shfl_sync(kFull, lead, l2);
                 less += e2 < e ? 1 : 0;
@@ -877,7 +877,7 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
     if (warp < T && lane < k) {
         const int t = warp;
         double ssum = 0.0;
-#pragma unroll 1
+#pragma unroll 8
         for (int j = 0; j < k; ++j) ssum += ss[(size_t)t * E + sel[t * 32 + j]];
         const int e = sel[t * 32 + lane];
         const float wv = (float)(ss[(size_t)t * E + e] / ssum * (double)p.rsf);
