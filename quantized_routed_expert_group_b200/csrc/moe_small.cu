@@ -564,6 +564,25 @@ __device__ __forceinline__ int warp_argmax_u64(unsigned long long key, int idx) 
     return (int)__reduce_min_sync(kFull, (hi == mh && lo == ml) ? (uint32_t)idx : 0x7FFFFFFFu);
 }
 
+// Bitonic sort of the warp's 32 (key, index) pairs, best first (larger key,
+// ties to the lower index): lane r ends with the r-th best.
+__device__ __forceinline__ void warp_sort_desc(unsigned long long& k, int& i, int lane) {
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+        for (int st = size >> 1; st > 0; st >>= 1) {
+            const unsigned long long ok = __shfl_xor_sync(kFull, k, st);
+            const int oi = __shfl_xor_sync(kFull, i, st);
+            const bool keep_best = ((lane & st) == 0) == ((lane & size) == 0);
+            const bool other_better = beats(ok, oi, k, i);
+            if (keep_best == other_better) {
+                k = ok;
+                i = oi;
+            }
+        }
+    }
+}
+
 // SELECT: wait for every router item, then route all tokens and bucket them
 // into this CTA's tables (the same in every CTA; CTA 0 also publishes them to
 // the workspace).  Same decisions as the multi-kernel router and the
@@ -632,23 +651,18 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
     consumers_sync();
     if (fast) {
         // GLM-like shape: warp g owns group g (32 experts, one per lane).
-        // 2. each (token, group): its best kc experts in order by k arg-max
-        // rounds (the first two give the group score)
+        // 2. each (token, group): its experts sorted best first; the best kc
+        // are listed, the best two give the group score
         if (warp < G) {
             const int g = warp, e = g * 32 + lane;
 #pragma unroll 1
             for (int t = 0; t < T; ++t) {
-                unsigned long long kk2 = key[(size_t)t * E + e];
-                const double cme = sc[(size_t)t * E + e];
-                double c12 = 0.0;
-#pragma unroll 1
-                for (int r = 0; r < kc; ++r) {
-                    const int ew = warp_argmax_u64(kk2, e);
-                    if (lane == 0) cand[(t * G + g) * kc + r] = ew;
-                    if (r < 2) c12 += __shfl_sync(kFull, cme, ew & 31);
-                    if (e == ew) kk2 = 0ull;
-                }
-                if (lane == 0) gkey[t * 32 + g] = order_key(c12);
+                unsigned long long kv = key[(size_t)t * E + e];
+                int iv = e;
+                warp_sort_desc(kv, iv, lane);
+                if (lane < kc) cand[(t * G + g) * kc + lane] = iv;
+                const int b1 = __shfl_sync(kFull, iv, 0), b2 = __shfl_sync(kFull, iv, 1);
+                if (lane == 0) gkey[t * 32 + g] = order_key(sc[(size_t)t * E + b1] + sc[(size_t)t * E + b2]);
             }
         }
         consumers_sync();
@@ -784,17 +798,21 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
         consumers_sync();  // every table the producer reads is written
         if (tid == 0) mbar_arrive(s.routing);
         if (publish) {
+            // counts and offsets of every expert: the first entry (entries are
+            // in ascending expert order) whose expert is not below e
+            const int U = s.misc[0];
 #pragma unroll 1
             for (int e = tid; e <= E; e += kConsumers) {
-                int o = 0, cv = 0;
+                int lo = 1, hi = U + 1;
 #pragma unroll 1
-                for (int j = 0; j < n; ++j) {
-                    const int ej = sel[(j / k) * 32 + j % k];
-                    o += ej < e ? 1 : 0;
-                    cv += ej == e ? 1 : 0;
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (s.ent[mid].expert < e) lo = mid + 1;
+                    else hi = mid;
                 }
-                p.offsets[e] = o;
-                if (e < E) p.counts[e] = cv;
+                const bool in = lo <= U;
+                p.offsets[e] = in ? s.ent[lo].slot0 : n;
+                if (e < E) p.counts[e] = (in && s.ent[lo].expert == e) ? s.ent[lo].n : 0;
             }
         }
     } else {
@@ -940,11 +958,16 @@ __device__ __forceinline__ void do_router(const SmallParams& p, const SmemPtrs& 
             x1 = reinterpret_cast<const float4*>(p.x + (int64_t)(two ? t0 + 1 : t0) * p.H) + qq * nq;
         }
         DFAcc a0[4], a1[4];
-#pragma unroll 1
-        for (int j = lane; j < nq; j += 32) {
-            const float4 w = wr[j];
-            dfacc4_add(a0, x0[j], w);
-            dfacc4_add(a1, x1[j], w);
+        if (two) {
+#pragma unroll 2
+            for (int j = lane; j < nq; j += 32) {
+                const float4 w = wr[j];
+                dfacc4_add(a0, x0[j], w);
+                dfacc4_add(a1, x1[j], w);
+            }
+        } else {
+#pragma unroll 4
+            for (int j = lane; j < nq; j += 32) dfacc4_add(a0, x0[j], wr[j]);
         }
         double v0 = dfacc4_value(a0), v1 = dfacc4_value(a1);
 #pragma unroll
