@@ -34,6 +34,14 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
     return r;
 }
 
+__device__ __forceinline__ float4 ld_stream_f4(const float4* p) {
+    float4 r;
+    asm("ld.global.nc.L1::no_allocate.L2::256B.v4.f32 {%0, %1, %2, %3}, [%4];"
+        : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+        : "l"(p));
+    return r;
+}
+
 // 128-bit read-only load that may stay in L1 (activations, reused across rows).
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
     return __ldg(reinterpret_cast<const uint4*>(p));

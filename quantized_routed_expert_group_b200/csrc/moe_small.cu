@@ -73,7 +73,6 @@ constexpr uint32_t kSpinLimit = 1u << 21;
 constexpr uint32_t kConsumerWaitLimit = 1u << 24;
 
 enum ItemKind : int {
-    kItemRouter = 1,
     kItemSelect = 2,
     kItemGateUp = 3,
     kItemDown = 4,
@@ -82,9 +81,9 @@ enum ItemKind : int {
 };
 
 // Control block (int32 words, zeroed by the prologue on every call):
-// [router_done, -, -, -, gu_done[nent]]; gu_done[e] counts (unit, token)
-// pairs of entry e whose h codes are published.
-enum : int { kCRouterDone = 0, kCHeader = 4 };
+// [-, -, -, -, gu_done[nent]]; gu_done[e] counts (unit, token) pairs of
+// entry e whose h codes are published.
+enum : int { kCHeader = 4 };
 
 // One expert of the batch union: entry 0 is the shared expert, entry 1 + a
 // the a-th routed expert in ascending id order.
@@ -100,7 +99,6 @@ struct SmallGeom {
     int grid;
     int tmax;
     int nent;      // 1 + max routed entries
-    int n_router;  // router items (2 experts each)
     int rg;        // gate/up row pairs per chunk
     int cpu;       // chunks per unit
     int nu;        // units per expert
@@ -113,7 +111,7 @@ struct SmallGeom {
     int act_bytes;
     int slot_bytes;
     int ctrl_words;
-    int o_xq, o_xd, o_bar, o_meta, o_rpart, o_gpart, o_usc, o_ent, o_selw, o_inv, o_ys, o_misc;
+    int o_xq, o_xd, o_bar, o_meta, o_gpart, o_usc, o_ent, o_selw, o_inv, o_ys, o_misc;
     int smem_bytes;
 };
 
@@ -171,7 +169,6 @@ SmallGeom small_geometry(const moe_config& c, int T, int grid) {
     g.grid = grid;
     g.tmax = T <= 1 ? 1 : T <= 2 ? 2 : 4;
     g.nent = 1 + (E < T * c.top_k ? E : T * c.top_k);
-    g.n_router = (E + 1) / 2;
     int rg = kSlotWeightBytes / (2 * rowH);
     rg = rg > kUnit ? kUnit : rg;
     int p2 = 1;
@@ -200,8 +197,6 @@ SmallGeom small_geometry(const moe_config& c, int T, int grid) {
     o += 128;  // full[4], empty[4], routing, ufull[2], ufree[2]
     g.o_meta = o;
     o += round_up((int)sizeof(SlotMeta) * kMaxSlots, 128);
-    g.o_rpart = o;
-    o += 32 * 8;
     g.o_gpart = o;
     o += 2 * kUnit * 2 * 8 * 4;  // [buffer][pair][half][gate/up][token]
     g.o_usc = o;
@@ -220,7 +215,7 @@ SmallGeom small_geometry(const moe_config& c, int T, int grid) {
     const int smem_max = device_info().max_smem_optin;
     while (g.nslot > 2 && o + g.nslot * g.slot_bytes > smem_max) --g.nslot;
     const int ring = g.nslot * g.slot_bytes;
-    g.o_xq += ring; g.o_xd += ring; g.o_bar += ring; g.o_meta += ring; g.o_rpart += ring; g.o_gpart += ring;
+    g.o_xq += ring; g.o_xd += ring; g.o_bar += ring; g.o_meta += ring; g.o_gpart += ring;
     g.o_usc += ring; g.o_ent += ring; g.o_selw += ring; g.o_inv += ring; g.o_ys += ring; g.o_misc += ring;
     g.smem_bytes = o + ring;
     return g;
@@ -232,7 +227,6 @@ static int select_scratch_bytes(int T, int E) { return 3 * T * E * 8 + 4 * 32 * 
 bool small_path_supported(const moe_config& c, int T) {
     if (T < 1 || T > 4) return false;
     if (c.hidden > 6144 || c.n_experts > 256 || c.n_groups > 32 || c.top_k > 32) return false;
-    if (2 * c.hidden * 4 > kSlotWeightBytes) return false;  // a router item is two fp32 rows
     const SmallGeom g = small_geometry(c, T, device_info().sm_count);
     if (g.rg < 4) return false;  // at least one gate/up row per row group
     if (c.hidden / 32 > kColThreads * kMaxGuBlocks || c.inter / 32 > kColThreads * kMaxDownBlocks) return false;
@@ -248,23 +242,82 @@ size_t small_ctrl_bytes(const moe_config& c, int T) {
 }
 
 // ---------------------------------------------------------------------------
-// Prologue: reset the control block and quantise x (launches its dependent
-// right away so the main kernel can start streaming).
+// Prologue: reset the control block, quantise x and compute the router
+// logits.  It launches its dependent (the main kernel) right away; its blocks
+// need no shared memory and few registers, so they run beside the main
+// kernel's persistent CTAs, which meanwhile stream the shared expert.  The
+// main kernel reads the logits after waiting for this grid.
+//
+// Router logits (the router row of expert e dotted with x, per token): block
+// b takes experts b, b + grid, ...; warp w takes eighth w of the hidden
+// dimension, each lane holds its weights (float4) in registers and keeps four
+// compensated fp32 sums per token (one per float4 component, about 2^-48
+// relative each), folded into fp64; the eighths are added in fp64 in a fixed
+// order.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k_small_prologue(const float* __restrict__ x, int64_t nblk,
-                                                        int8_t* __restrict__ xq, float* __restrict__ xd, int* ctrl,
-                                                        int ctrl_words, int32_t* err) {
+constexpr int kPrologueThreads = 256;
+constexpr int kRouterVec = 6;  // float4 of one router row per lane: hidden / 8 / 4 / 32 <= 6
+
+__device__ __forceinline__ void dfacc4_add(DFAcc (&acc)[4], float4 x, float4 w) {
+    acc[0].add_prod(x.x, w.x);
+    acc[1].add_prod(x.y, w.y);
+    acc[2].add_prod(x.z, w.z);
+    acc[3].add_prod(x.w, w.w);
+}
+
+__global__ void __launch_bounds__(kPrologueThreads) k_small_prologue(const float* __restrict__ x, int T, int H, int E,
+                                                                     const float* __restrict__ router_w,
+                                                                     double* __restrict__ logits,
+                                                                     int8_t* __restrict__ xq, float* __restrict__ xd,
+                                                                     int* ctrl, int ctrl_words, int32_t* err) {
     pdl_launch_dependents();
+    __shared__ double part[8][4];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gtid = blockIdx.x * blockDim.x + threadIdx.x;
     for (int i = gtid; i < ctrl_words; i += gridDim.x * blockDim.x) ctrl[i] = 0;
     if (gtid == 0) *err = 0;
-    const int lane = threadIdx.x & 31;
-    for (int64_t b = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); b < nblk; b += (int64_t)gridDim.x * 8) {
+    // Q8_0 of x, one block of 32 per warp
+    const int64_t nblk = (int64_t)T * (H / 32);
+    for (int64_t b = (int64_t)blockIdx.x * 8 + warp; b < nblk; b += (int64_t)gridDim.x * 8) {
         int8_t q;
         float d;
         q8_0_warp(x[b * kQBlock + lane], q, d);
         xq[b * kQBlock + lane] = q;
         if (lane == 0) xd[b] = d;
+    }
+    // router logits
+    const int n8 = H / 32;  // float4 per eighth
+#pragma unroll 1
+    for (int e = blockIdx.x; e < E; e += gridDim.x) {
+        const float4* wr = reinterpret_cast<const float4*>(router_w + (int64_t)e * H) + warp * n8;
+        float4 w[kRouterVec];
+#pragma unroll
+        for (int u = 0; u < kRouterVec; ++u) {
+            const int j = lane + 32 * u;
+            w[u] = j < n8 ? ld_stream_f4(wr + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll 1
+        for (int t = 0; t < T; ++t) {
+            const float4* xr = reinterpret_cast<const float4*>(x + (int64_t)t * H) + warp * n8;
+            DFAcc acc[4];
+#pragma unroll
+            for (int u = 0; u < kRouterVec; ++u) {
+                const int j = lane + 32 * u;
+                dfacc4_add(acc, j < n8 ? __ldg(xr + j) : make_float4(0.f, 0.f, 0.f, 0.f), w[u]);
+            }
+            double v = (acc[0].value() + acc[1].value()) + (acc[2].value() + acc[3].value());
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+            if (lane == 0) part[warp][t] = v;
+        }
+        __syncthreads();
+        if ((int)threadIdx.x < T) {
+            double v = 0.0;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v += part[k][threadIdx.x];
+            logits[(int64_t)threadIdx.x * E + e] = v;
+        }
+        __syncthreads();
     }
 }
 
@@ -281,7 +334,6 @@ struct SmemPtrs {
     uint64_t* ufull;    // [2] every consumer warp has written its partials of a unit
     uint64_t* ufree;    // [2] the unit's finisher has read them
     SlotMeta* meta;
-    double* rpart;   // [2][4][4] router partials
     float* gpart;    // [2][32][2][2][4] gate/up partial dots of a unit: [buffer][pair][gate/up][half][token]
     float* usc;      // [2][32][2] gate/up row scales of a unit
     EntryInfo* ent;  // [nent]
@@ -302,7 +354,6 @@ __device__ __forceinline__ SmemPtrs carve(uint8_t* base, const SmallGeom& g) {
     s.ufull = s.routing + 1;
     s.ufree = s.ufull + 2;
     s.meta = reinterpret_cast<SlotMeta*>(base + g.o_meta);
-    s.rpart = reinterpret_cast<double*>(base + g.o_rpart);
     s.gpart = reinterpret_cast<float*>(base + g.o_gpart);
     s.usc = reinterpret_cast<float*>(base + g.o_usc);
     s.ent = reinterpret_cast<EntryInfo*>(base + g.o_ent);
@@ -429,14 +480,6 @@ struct Producer {
 
     __forceinline__ __device__ bool marker(int kind) {
         return push(blank(kind), no_copy(), no_copy(), no_copy(), no_copy());
-    }
-
-    __forceinline__ __device__ bool router(int q) {
-        SlotMeta m = blank(kItemRouter);
-        m.expert = 2 * q;
-        m.nrows = (p.E - 2 * q) < 2 ? (p.E - 2 * q) : 2;
-        const Copy c0{p.router_w + (int64_t)m.expert * p.H, (uint32_t)(m.nrows * p.H * 4), 0u, true, 0};
-        return push(m, c0, no_copy(), no_copy(), no_copy());
     }
 
     // Chunk ch of gate/up unit blk of an entry: rg rows of Wg and of Wu and
@@ -623,19 +666,7 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
     unsigned long long* lkey = reinterpret_cast<unsigned long long*>(wsum + 16);  // [T][tg*kk] listed keys
     int* lid = reinterpret_cast<int*>(lkey + T * p.tg * min(k, per));            // [T][tg*kk] listed ids
     const int warp = tid >> 5, lane = tid & 31;
-    if (tid == 0) {
-        int ok = 0;
-#pragma unroll 1
-        for (uint32_t i = 0; i < kSpinLimit; ++i) {
-            if (ld_acquire_gpu(p.ctrl + kCRouterDone) >= p.g.n_router) {
-                ok = 1;
-                break;
-            }
-            __nanosleep(32);
-        }
-        if (!ok) set_error(p.err, kErrTimeout);  // route on whatever is there; never hang
-    }
-    consumers_sync();
+    // the logits are the prologue's: the consumers waited for its grid
     // 1. s, c and keys
 #pragma unroll 1
     for (int i = tid; i < TE; i += kConsumers) {
@@ -905,93 +936,6 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
             p.w[(int64_t)t * k + lane] = wv;
         }
     }
-}
-
-// ---- router item: logits of two experts for all tokens ----
-// Warp w takes expert w / 4 of the item and quarter w % 4 of the hidden
-// dimension; each lane keeps four compensated fp32 sums per token (one per
-// float4 component, about 2^-48 relative each), folded into fp64 in a fixed
-// order, and the warps' partials are combined in fp64 in a fixed order.
-// x comes from shared memory (xs, two tokens at a time) when the caller has
-// staged it, else straight from global memory.  The loops stay rolled (this
-// code runs once per call).
-__device__ __forceinline__ void stage_x(const SmallParams& p, float* xs, int t0, int tid) {
-    const int nt = p.T - t0 < 2 ? p.T - t0 : 2;
-    const int n4 = nt * p.H / 4;
-    const float4* src = reinterpret_cast<const float4*>(p.x + (int64_t)t0 * p.H);
-#pragma unroll 4
-    for (int i = tid; i < n4; i += kConsumers) reinterpret_cast<float4*>(xs)[i] = __ldg(src + i);
-}
-
-__device__ __forceinline__ void dfacc4_add(DFAcc (&acc)[4], float4 x, float4 w) {
-    acc[0].add_prod(x.x, w.x);
-    acc[1].add_prod(x.y, w.y);
-    acc[2].add_prod(x.z, w.z);
-    acc[3].add_prod(x.w, w.w);
-}
-
-__device__ __forceinline__ double dfacc4_value(const DFAcc (&acc)[4]) {
-    return (acc[0].value() + acc[1].value()) + (acc[2].value() + acc[3].value());
-}
-
-__device__ __forceinline__ void do_router(const SmallParams& p, const SmemPtrs& s, const SlotMeta& m,
-                                          const uint8_t* slot, int tid, uint64_t* empty, float* xs, bool staged) {
-    const int warp = tid >> 5, lane = tid & 31;
-    const int el = warp >> 2, qq = warp & 3;
-    const int nq = p.H / 16;  // float4 per quarter
-    const float4* wr = reinterpret_cast<const float4*>(slot) + (size_t)(el < m.nrows ? el : 0) * (p.H / 4) + qq * nq;
-#pragma unroll 1
-    for (int t0 = 0; t0 < p.T; t0 += 2) {
-        const bool two = t0 + 1 < p.T;
-        const float4* x0;
-        const float4* x1;
-        if (xs) {
-            if (!(staged && t0 == 0)) {
-                consumers_sync();  // the previous pair is no longer read
-                stage_x(p, xs, t0, tid);
-                consumers_sync();
-            }
-            x0 = reinterpret_cast<const float4*>(xs) + qq * nq;
-            x1 = x0 + (two ? p.H / 4 : 0);
-        } else {
-            x0 = reinterpret_cast<const float4*>(p.x + (int64_t)t0 * p.H) + qq * nq;
-            x1 = reinterpret_cast<const float4*>(p.x + (int64_t)(two ? t0 + 1 : t0) * p.H) + qq * nq;
-        }
-        DFAcc a0[4], a1[4];
-        if (two) {
-#pragma unroll 2
-            for (int j = lane; j < nq; j += 32) {
-                const float4 w = wr[j];
-                dfacc4_add(a0, x0[j], w);
-                dfacc4_add(a1, x1[j], w);
-            }
-        } else {
-#pragma unroll 4
-            for (int j = lane; j < nq; j += 32) dfacc4_add(a0, x0[j], wr[j]);
-        }
-        double v0 = dfacc4_value(a0), v1 = dfacc4_value(a1);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            v0 += __shfl_xor_sync(kFull, v0, o);
-            v1 += __shfl_xor_sync(kFull, v1, o);
-        }
-        if (lane == 0) {
-            s.rpart[(el * 4 + qq) * 4 + t0] = v0;
-            if (two) s.rpart[(el * 4 + qq) * 4 + t0 + 1] = v1;
-        }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(empty);
-    consumers_sync();
-    if (tid < m.nrows * p.T) {
-        const int e2 = tid / p.T, t = tid % p.T;
-        double v = 0.0;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) v += s.rpart[(e2 * 4 + k) * 4 + t];
-        p.logits[(int64_t)t * p.E + m.expert + e2] = v;
-    }
-    consumers_sync();  // logits written; rpart free for the next item
-    if (tid == 0) red_add_release_gpu(p.ctrl + kCRouterDone, 1);
 }
 
 // m.tok[i] with a run-time i, without indexing a local array.
@@ -1268,20 +1212,10 @@ __global__ void __launch_bounds__(kSmallThreads, 1) k_moe_small(const __grid_con
     if (warp == kConsumerWarps) {
         // ------------------------- producer -------------------------
         Producer pr(p, s, lane);
-        // router rows depend on nothing from the prologue
-        for (int q = c; q < g.n_router; q += grid) pr.router(q);
         const int64_t rowI = (int64_t)p.I * p.wbits / 8;
         if (p.ns && lane == 0 && r1 > r0)
             bulk_prefetch_l2(p.shared.w_down + (int64_t)r0 * rowI, (uint32_t)((r1 - r0) * rowI));
-        pdl_wait();
-        if (c < g.n_router) {
-            // the SELECT slot also brings x (up to two tokens) for the router item
-            const int nt = p.T < 2 ? p.T : 2;
-            const Copy cx{p.x, (uint32_t)(nt * p.H * 4), 0u, false, 0};
-            pr.push(pr.blank(kItemSelect), cx, no_copy(), no_copy(), no_copy());
-        } else {
-            pr.marker(kItemSelect);
-        }
+        pr.marker(kItemSelect);
         // the shared expert's gate/up units need no routing
         EntryInfo e0;
         e0.expert = -1;
@@ -1292,6 +1226,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1) k_moe_small(const __grid_con
         for (int u = c; u < n_pre; u += grid)
             for (int ch = 0; ch < g.cpu; ++ch) pr.gateup(0, e0, u, ch);
         // the routed part of the schedule needs this CTA's routing tables
+        // (and the control block the prologue reset)
+        pdl_wait();
         int ok = 1;
         if (lane == 0) ok = mbar_wait(s.routing, 0, kConsumerWaitLimit) ? 1 : 0;
         ok = __shfl_sync(kFull, ok, 0);
@@ -1347,23 +1283,6 @@ __global__ void __launch_bounds__(kSmallThreads, 1) k_moe_small(const __grid_con
     int slot = 0;
     uint32_t pf = 0;
     int uc = 0;  // gate/up units started by this CTA
-    if (blockIdx.x < g.n_router) {
-        // the first item of a CTA with router work is its router item, the
-        // second its SELECT, whose copy brings x (the first two tokens)
-        float* xs = reinterpret_cast<float*>(s.slots + g.slot_bytes);
-        if (!mbar_wait(&s.full[0], 0, kConsumerWaitLimit)) {
-            set_error(p.err, kErrTimeout);
-            return;
-        }
-        const SlotMeta m = s.meta[0];
-        if (m.kind != kItemRouter) return;  // the producer gave up before its first item
-        if (!mbar_wait(&s.full[1], 0, kConsumerWaitLimit)) {
-            set_error(p.err, kErrTimeout);
-            return;
-        }
-        do_router(p, s, m, s.slots, tid, &s.empty[0], xs, true);
-        slot = 1;
-    }
     while (true) {
         if (!mbar_wait(&s.full[slot], pf, kConsumerWaitLimit)) {
             set_error(p.err, kErrTimeout);
@@ -1377,8 +1296,6 @@ __global__ void __launch_bounds__(kSmallThreads, 1) k_moe_small(const __grid_con
             if (m.last) ++uc;
         } else if (m.kind == kItemDown) {
             do_down<WBITS, TM>(p, s, m, data, tid, empty);
-        } else if (m.kind == kItemRouter) {
-            do_router(p, s, m, data, tid, empty, nullptr, false);
         } else if (m.kind == kItemSelect) {
             do_select(p, s, data, tid);
             __syncwarp();
@@ -1434,9 +1351,8 @@ cudaError_t launch_small(const SmallArgs& a, cudaStream_t st) {
     p.hq = a.hq; p.hd = a.hd; p.y = a.y; p.out = a.out; p.ctrl = a.ctrl; p.err = a.err;
     p.g = small_geometry(c, a.T, device_info().sm_count);
     if (p.g.smem_bytes > device_info().max_smem_optin) return cudaErrorInvalidConfiguration;
-    const int64_t nblk = (int64_t)a.T * (c.hidden / 32);
-    const int grid = (int)((nblk + 7) / 8) > 1 ? (int)((nblk + 7) / 8) : 1;
-    k_small_prologue<<<grid, 256, 0, st>>>(a.x, nblk, a.xq, a.xd, a.ctrl, p.g.ctrl_words, a.err);
+    k_small_prologue<<<p.g.grid, kPrologueThreads, 0, st>>>(a.x, a.T, c.hidden, c.n_experts, a.router_w, a.logits,
+                                                            a.xq, a.xd, a.ctrl, p.g.ctrl_words, a.err);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int tm = p.g.tmax;
