@@ -44,7 +44,9 @@ namespace moe {
 
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kSmallThreads = kConsumers + 32;
+constexpr int kProducerWarp = kConsumerWarps;      // streams the items
+constexpr int kFinisherWarp = kConsumerWarps + 1;  // finishes gate/up units
+constexpr int kSmallThreads = kConsumers + 64;
 constexpr int kSlotWeightBytes = 48 * 1024;
 constexpr int kMaxSlots = 4;
 constexpr int kUnit = 32;          // gate/up rows per unit: one Q8_0 block of h
@@ -95,6 +97,14 @@ struct EntryInfo {
     int pad;
 };
 
+// A gate/up unit handed from the consumer warps to the finisher warp.
+struct UnitRec {
+    int entry;  // < 0: no more units
+    int blk;
+    int slot0;
+    int n;
+};
+
 struct SmallGeom {
     int grid;
     int tmax;
@@ -111,7 +121,7 @@ struct SmallGeom {
     int act_bytes;
     int slot_bytes;
     int ctrl_words;
-    int o_xq, o_xd, o_bar, o_meta, o_gpart, o_usc, o_ent, o_selw, o_inv, o_ys, o_misc;
+    int o_xq, o_xd, o_bar, o_meta, o_urec, o_gpart, o_usc, o_ent, o_selw, o_inv, o_ys, o_misc;
     int smem_bytes;
 };
 
@@ -197,6 +207,8 @@ SmallGeom small_geometry(const moe_config& c, int T, int grid) {
     o += 128;  // full[4], empty[4], routing, ufull[2], ufree[2]
     g.o_meta = o;
     o += round_up((int)sizeof(SlotMeta) * kMaxSlots, 128);
+    g.o_urec = o;
+    o += 128;  // UnitRec[2]
     g.o_gpart = o;
     o += 2 * kUnit * 2 * 8 * 4;  // [buffer][pair][half][gate/up][token]
     g.o_usc = o;
@@ -215,7 +227,7 @@ SmallGeom small_geometry(const moe_config& c, int T, int grid) {
     const int smem_max = device_info().max_smem_optin;
     while (g.nslot > 2 && o + g.nslot * g.slot_bytes > smem_max) --g.nslot;
     const int ring = g.nslot * g.slot_bytes;
-    g.o_xq += ring; g.o_xd += ring; g.o_bar += ring; g.o_meta += ring; g.o_gpart += ring;
+    g.o_xq += ring; g.o_xd += ring; g.o_bar += ring; g.o_meta += ring; g.o_urec += ring; g.o_gpart += ring;
     g.o_usc += ring; g.o_ent += ring; g.o_selw += ring; g.o_inv += ring; g.o_ys += ring; g.o_misc += ring;
     g.smem_bytes = o + ring;
     return g;
@@ -332,7 +344,8 @@ struct SmemPtrs {
     uint64_t* empty;
     uint64_t* routing;  // consumers -> producer: the routing tables are ready
     uint64_t* ufull;    // [2] every consumer warp has written its partials of a unit
-    uint64_t* ufree;    // [2] the unit's finisher has read them
+    uint64_t* ufree;    // [2] the finisher warp has read them
+    UnitRec* urec;      // [2] the unit to finish
     SlotMeta* meta;
     float* gpart;    // [2][32][2][2][4] gate/up partial dots of a unit: [buffer][pair][gate/up][half][token]
     float* usc;      // [2][32][2] gate/up row scales of a unit
@@ -354,6 +367,7 @@ __device__ __forceinline__ SmemPtrs carve(uint8_t* base, const SmallGeom& g) {
     s.ufull = s.routing + 1;
     s.ufree = s.ufull + 2;
     s.meta = reinterpret_cast<SlotMeta*>(base + g.o_meta);
+    s.urec = reinterpret_cast<UnitRec*>(base + g.o_urec);
     s.gpart = reinterpret_cast<float*>(base + g.o_gpart);
     s.usc = reinterpret_cast<float*>(base + g.o_usc);
     s.ent = reinterpret_cast<EntryInfo*>(base + g.o_ent);
@@ -1035,30 +1049,51 @@ __device__ __forceinline__ void do_gateup(const SmallParams& p, const SmemPtrs& 
     __syncwarp();
     if (lane == 0) mbar_arrive(empty);
     if (!m.last) return;
-    // Unit end: every warp reports its partials; one warp (rotating, so that
-    // the wait for the slowest warp and the release fence fall on each warp in
-    // turn) finishes the unit while the others go on with the next chunks.
-    if (lane == 0) mbar_arrive(&s.ufull[buf]);
-    if (warp != (uc & (kConsumerWarps - 1))) return;
-    if (!mbar_wait(&s.ufull[buf], (uc >> 1) & 1, kConsumerWaitLimit)) set_error(p.err, kErrTimeout);
-    const float* gp = s.gpart + (buf * kUnit + lane) * 16;  // [gate/up][half][token]
-    const float sgl = s.usc[(buf * kUnit + lane) * 2], sul = s.usc[(buf * kUnit + lane) * 2 + 1];
-    for (int i = 0; i < m.n; ++i) {
-        const float gs = gp[i] + gp[4 + i];
-        const float us = gp[8 + i] + gp[12 + i];
-        const float h = silu_mul(sgl * gs, sul * us);
-        int8_t qv;
-        float d;
-        q8_0_warp(h, qv, d);
-        const int64_t sl = m.slot0 + i;
-        p.hq[sl * p.I + m.blk * kUnit + lane] = qv;
-        if (lane == 0) p.hd[sl * (p.I / 32) + m.blk] = d;
-    }
+    // Unit end: every warp reports its partials and goes on; the finisher
+    // warp turns them into h codes and publishes them
+    if (warp == 0 && lane == 0) s.urec[buf] = UnitRec{m.entry, m.blk, m.slot0, m.n};
     __syncwarp();
-    if (lane == 0) {
-        mbar_arrive(&s.ufree[buf]);
-        fence_acq_rel_gpu();  // the warp's h codes before the count (release pattern)
-        red_add_relaxed_gpu(p.ctrl + kCHeader + m.entry, m.n);
+    if (lane == 0) mbar_arrive(&s.ufull[buf]);
+}
+
+// ---- the finisher warp: for each gate/up unit of the CTA (in order), wait
+// until every consumer warp has reported its partials, then h = silu(g) * u
+// for the 32 rows (lane = row) of each token, Q8_0 of the block, and the
+// release of the codes to the other CTAs; the consumer warps never wait for
+// this (nor for the release fence) ----
+__device__ __forceinline__ void finisher(const SmallParams& p, const SmemPtrs& s, int lane) {
+    pdl_wait();  // the control block was reset by the prologue
+#pragma unroll 1
+    for (int k = 0;; ++k) {
+        const int buf = k & 1;
+        if (!mbar_wait(&s.ufull[buf], (k >> 1) & 1, kConsumerWaitLimit)) {
+            if (lane == 0) set_error(p.err, kErrTimeout);
+            return;
+        }
+        const UnitRec r = s.urec[buf];
+        if (r.entry < 0) return;
+        const float* gp = s.gpart + (buf * kUnit + lane) * 16;  // [gate/up][half][token]
+        const float sgl = s.usc[(buf * kUnit + lane) * 2], sul = s.usc[(buf * kUnit + lane) * 2 + 1];
+        const int n = r.n < 4 ? r.n : 4;
+#pragma unroll 1
+        for (int i = 0; i < n; ++i) {
+            const float gs = gp[i] + gp[4 + i];
+            const float us = gp[8 + i] + gp[12 + i];
+            const float h = silu_mul(sgl * gs, sul * us);
+            int8_t qv;
+            float d;
+            q8_0_warp(h, qv, d);
+            const int64_t sl = r.slot0 + i;
+            p.hq[sl * p.I + r.blk * kUnit + lane] = qv;
+            if (lane == 0) p.hd[sl * (p.I / 32) + r.blk] = d;
+        }
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&s.ufree[buf]);
+            fence_acq_rel_gpu();  // the warp's h codes before the count (release pattern)
+            red_add_relaxed_gpu(p.ctrl + kCHeader + r.entry, n);
+        }
+        __syncwarp();
     }
 }
 
@@ -1209,7 +1244,11 @@ __global__ void __launch_bounds__(kSmallThreads, 1) k_moe_small(const __grid_con
     }
     __syncthreads();
 
-    if (warp == kConsumerWarps) {
+    if (warp == kFinisherWarp) {
+        finisher(p, s, lane);
+        return;
+    }
+    if (warp == kProducerWarp) {
         // ------------------------- producer -------------------------
         Producer pr(p, s, lane);
         const int64_t rowI = (int64_t)p.I * p.wbits / 8;
@@ -1310,6 +1349,13 @@ __global__ void __launch_bounds__(kSmallThreads, 1) k_moe_small(const __grid_con
             pf ^= 1u;
         }
     }
+    // no more units: hand the finisher a terminal record (its buffer was last
+    // used by unit uc - 2, which the finisher must have read first)
+    const int buf = uc & 1;
+    if (uc >= 2 && !mbar_wait(&s.ufree[buf], ((uc >> 1) - 1) & 1, kConsumerWaitLimit)) set_error(p.err, kErrTimeout);
+    if (warp == 0 && lane == 0) s.urec[buf] = UnitRec{-1, 0, 0, 0};
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.ufull[buf]);
 }
 
 // ---------------------------------------------------------------------------
