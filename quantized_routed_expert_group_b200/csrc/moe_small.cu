@@ -1116,19 +1116,6 @@ __device__ __forceinline__ void down_act(const uint8_t* act, const float* hdv, i
     }
 }
 
-// acc[rr][i] += dh[i] * dot(row rr, block b; token i) for a batch of rows.
-template <int WBITS, int TM, int RB>
-__device__ __forceinline__ void rows_dot(const uint8_t* const (&rowp)[RB], int b, const ActBlock (&a)[TM],
-                                         const float (&dh)[TM], const int (&cr)[TM], float (&acc)[RB * TM]) {
-#pragma unroll
-    for (int rr = 0; rr < RB; ++rr) {
-        const WBlock<WBITS> w = load_block_smem<WBITS>(rowp[rr], b);
-#pragma unroll
-        for (int i = 0; i < TM; ++i)
-            acc[rr * TM + i] = fmaf(dh[i], (float)dot_block_scaled<WBITS>(w, a[i], cr[i]), acc[rr * TM + i]);
-    }
-}
-
 // ---- down chunk: nrows rows of Wd for the entry's tokens -> y ----
 // Rows are dealt to the row groups round-robin (r = q + 4 k); the half-1
 // warp of a pair hands its sums to the half-0 warp through shared memory.
@@ -1160,20 +1147,42 @@ __device__ __forceinline__ void do_down(const SmallParams& p, const SmemPtrs& s,
         float acc[V];
 #pragma unroll
         for (int v = 0; v < V; ++v) acc[v] = 0.0f;
-        const uint8_t* rowp[RB];
+        // sub-batches of 4 rows; one wholly past the group's rows is skipped
+        // (a uniform branch), so a group of 10-11 rows computes 12
 #pragma unroll
-        for (int rr = 0; rr < RB; ++rr) {
-            const int k = kb + rr < klast ? kb + rr : klast;
-            rowp[rr] = slot + (size_t)(q + kRowGroups * k) * rbI;
-        }
-        rows_dot<WBITS, TM, RB>(rowp, b0, a0, dh0, cr0, acc);
-        for (int j = 1; j < nbj; ++j) {
-            ActBlock aj[TM];
-            float dhj[TM];
-            int crj[TM];
-            const int bj = c + kColThreads * j;
-            down_act<WBITS, TM>(act, hdv, p.I, nbI, m.n, bj, aj, dhj, crj);
-            rows_dot<WBITS, TM, RB>(rowp, bj < nbI ? bj : 0, aj, dhj, crj, acc);
+        for (int sb = 0; sb < RB / 4; ++sb) {
+            if (kb + 4 * sb < nk) {
+                const uint8_t* rowp[4];
+#pragma unroll
+                for (int rr = 0; rr < 4; ++rr) {
+                    const int k = kb + 4 * sb + rr < klast ? kb + 4 * sb + rr : klast;
+                    rowp[rr] = slot + (size_t)(q + kRowGroups * k) * rbI;
+                }
+#pragma unroll
+                for (int rr = 0; rr < 4; ++rr) {
+                    const WBlock<WBITS> w = load_block_smem<WBITS>(rowp[rr], b0);
+#pragma unroll
+                    for (int i = 0; i < TM; ++i)
+                        acc[(4 * sb + rr) * TM + i] =
+                            fmaf(dh0[i], (float)dot_block_scaled<WBITS>(w, a0[i], cr0[i]), acc[(4 * sb + rr) * TM + i]);
+                }
+                for (int j = 1; j < nbj; ++j) {
+                    ActBlock aj[TM];
+                    float dhj[TM];
+                    int crj[TM];
+                    const int bj = c + kColThreads * j;
+                    down_act<WBITS, TM>(act, hdv, p.I, nbI, m.n, bj, aj, dhj, crj);
+                    const int bc = bj < nbI ? bj : 0;
+#pragma unroll
+                    for (int rr = 0; rr < 4; ++rr) {
+                        const WBlock<WBITS> w = load_block_smem<WBITS>(rowp[rr], bc);
+#pragma unroll
+                        for (int i = 0; i < TM; ++i)
+                            acc[(4 * sb + rr) * TM + i] =
+                                fmaf(dhj[i], (float)dot_block_scaled<WBITS>(w, aj[i], crj[i]), acc[(4 * sb + rr) * TM + i]);
+                    }
+                }
+            }
         }
         const float v = warp_reduce_many<V>(acc, lane);
         const int vi = lane >> SHIFT;
