@@ -258,6 +258,9 @@ def run_ours(args) -> dict | None:
     router_bytes = s.n_experts * s.hidden * 4
     layer_bytes = (n_active + s.n_shared) * expert_bytes(s)
     if phases == ["fused"]:
+        # the fused phase: the prologue (Q8_0 of x, router logits over the
+        # router weights) and the persistent kernel (the experts), which run
+        # overlapped; bytes and ncu traffic cover both
         dom_kernel, dom_ms = "k_moe_small", statistics.mean(phase_ms[0])
         dom_bytes = layer_bytes + router_bytes
     else:

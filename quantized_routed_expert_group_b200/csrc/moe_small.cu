@@ -13,14 +13,18 @@
 //   share of the weights with bulk asynchronous copies (cp.async.bulk, the
 //   1-D TMA form) into a ring of 48 KB shared-memory slots, and eight
 //   consumer warps that do the integer dots on __dp4a.
-// * The schedule is static; no CTA takes work from a queue:
+// * The schedule is static except for the routed gate/up units at T > 1:
 //   - router: CTA c computes the logits of experts 2c and 2c+1;
 //   - selection: every CTA routes all tokens itself from the published
 //     logits (identical decisions everywhere), so the routing costs one
 //     grid-wide wait and no broadcast;
 //   - gate/up: cut into units of 32 rows of one expert (one Q8_0 block of h);
-//     unit u belongs to CTA u mod grid, which finishes it: SwiGLU, Q8_0 of
-//     the 32 h values, published with one release counter per expert;
+//     the shared expert's unit c belongs to CTA c (it needs no routing); at
+//     one token the routed experts' units continue the round robin (unit u
+//     to CTA u mod grid), at more tokens they are taken from a global counter
+//     (one atomic per unit), so that SMs with more bandwidth take more; the CTA
+//     finishes its units: SwiGLU, Q8_0 of the 32 h values, published with
+//     one release counter per expert;
 //   - down + combine: CTA c owns output rows [H c / grid, H (c+1) / grid) of
 //     every expert and combines them itself at the end, so no partial output
 //     crosses CTAs: no float atomics, bit-reproducible results.
@@ -83,9 +87,10 @@ enum ItemKind : int {
 };
 
 // Control block (int32 words, zeroed by the prologue on every call):
-// [-, -, -, -, gu_done[nent]]; gu_done[e] counts (unit, token) pairs of
-// entry e whose h codes are published.
-enum : int { kCHeader = 4 };
+// [units, -, -, -, gu_done[nent]]; units counts the routed gate/up units
+// taken; gu_done[e] counts (unit, token) pairs of entry e whose h codes are
+// published.
+enum : int { kCUnits = 0, kCHeader = 4 };
 
 // One expert of the batch union: entry 0 is the shared expert, entry 1 + a
 // the a-th routed expert in ascending id order.
@@ -277,6 +282,17 @@ __device__ __forceinline__ void dfacc4_add(DFAcc (&acc)[4], float4 x, float4 w) 
     acc[3].add_prod(x.w, w.w);
 }
 
+__device__ __forceinline__ void load_router_row(const float* router_w, int e, int E, int H, int warp, int lane,
+                                                float4 (&w)[kRouterVec]) {
+    const int n8 = H / 32;  // float4 per eighth
+    const float4* wr = reinterpret_cast<const float4*>(router_w + (int64_t)(e < E ? e : 0) * H) + warp * n8;
+#pragma unroll
+    for (int u = 0; u < kRouterVec; ++u) {
+        const int j = lane + 32 * u;
+        w[u] = (e < E && j < n8) ? ld_stream_f4(wr + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
 __global__ void __launch_bounds__(kPrologueThreads) k_small_prologue(const float* __restrict__ x, int T, int H, int E,
                                                                      const float* __restrict__ router_w,
                                                                      double* __restrict__ logits,
@@ -285,6 +301,13 @@ __global__ void __launch_bounds__(kPrologueThreads) k_small_prologue(const float
     pdl_launch_dependents();
     __shared__ double part[8][4];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // the block's first router row is requested first (its latency covers
+    // the rest of the setup), its later rows go to L2 meanwhile
+    float4 w[kRouterVec];
+    load_router_row(router_w, blockIdx.x, E, H, warp, lane, w);
+    if (threadIdx.x == 0)
+        for (int e = blockIdx.x + gridDim.x; e < E; e += gridDim.x)
+            bulk_prefetch_l2(router_w + (int64_t)e * H, (uint32_t)(H * 4));
     const int gtid = blockIdx.x * blockDim.x + threadIdx.x;
     for (int i = gtid; i < ctrl_words; i += gridDim.x * blockDim.x) ctrl[i] = 0;
     if (gtid == 0) *err = 0;
@@ -301,13 +324,7 @@ __global__ void __launch_bounds__(kPrologueThreads) k_small_prologue(const float
     const int n8 = H / 32;  // float4 per eighth
 #pragma unroll 1
     for (int e = blockIdx.x; e < E; e += gridDim.x) {
-        const float4* wr = reinterpret_cast<const float4*>(router_w + (int64_t)e * H) + warp * n8;
-        float4 w[kRouterVec];
-#pragma unroll
-        for (int u = 0; u < kRouterVec; ++u) {
-            const int j = lane + 32 * u;
-            w[u] = j < n8 ? ld_stream_f4(wr + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
+        if (e != (int)blockIdx.x) load_router_row(router_w, e, E, H, warp, lane, w);
 #pragma unroll 1
         for (int t = 0; t < T; ++t) {
             const float4* xr = reinterpret_cast<const float4*>(x + (int64_t)t * H) + warp * n8;
@@ -1285,12 +1302,33 @@ __global__ void __launch_bounds__(kSmallThreads, 1) k_moe_small(const __grid_con
         int U = s.misc[0];
         U = U < 0 ? 0 : (U > umax ? umax : U);
         const int first = p.ns ? 0 : 1;
-        const int n_units = (p.ns + U) * g.nu;
-        for (int u = c; u < n_units && !pr.aborted; u += grid) {
-            if (u < n_pre) continue;
-            const int entry = first + u / g.nu, blk = u % g.nu;
-            const EntryInfo ei = s.ent[entry];
-            for (int ch = 0; ch < g.cpu; ++ch) pr.gateup(entry, ei, blk, ch);
+        const int n_routed = U * g.nu;
+        if (p.T > 1) {
+            // the routed experts' units are taken from a global counter, one
+            // at a time (requested one unit ahead): SMs that stream faster
+            // take more, so every CTA reaches its down chunks at about the
+            // same time
+            int next = 0;
+            if (lane == 0) next = atom_add_relaxed_gpu(p.ctrl + kCUnits, 1);
+            next = __shfl_sync(kFull, next, 0);
+            while (next < n_routed && !pr.aborted) {
+                const int r = next;
+                if (lane == 0) next = atom_add_relaxed_gpu(p.ctrl + kCUnits, 1);
+                const int entry = 1 + r / g.nu, blk = r % g.nu;
+                const EntryInfo ei = s.ent[entry];
+                for (int ch = 0; ch < g.cpu; ++ch) pr.gateup(entry, ei, blk, ch);
+                next = __shfl_sync(kFull, next, 0);
+            }
+        } else {
+            // one token: a static round robin over the units of all experts
+            // (the shared expert's first, issued above) measured as fast
+            const int n_pre_all = p.ns ? g.nu : 0;
+            for (int u = c; u < n_pre_all + n_routed && !pr.aborted; u += grid) {
+                if (u < n_pre_all) continue;
+                const int entry = 1 + (u - n_pre_all) / g.nu, blk = (u - n_pre_all) % g.nu;
+                const EntryInfo ei = s.ent[entry];
+                for (int ch = 0; ch < g.cpu; ++ch) pr.gateup(entry, ei, blk, ch);
+            }
         }
         for (int entry = first; entry <= U && !pr.aborted; ++entry) {
             const EntryInfo ei = s.ent[entry];
