@@ -58,11 +58,16 @@ def lib():
             "orc_block_dots": [_vp, _i64, _i64, _int, _vp, _i64, _vp],
             "orc_qmatvec": [_vp, _vp, _i64, _i64, _int, _vp, _vp, _vp],
             "orc_router": [_vp, _int, _int, _vp, _vp, _int, _int, _int, _int, _flt, _vp, _vp, _vp, _vp],
+            "orc_router_topp": [_vp, _int, _int, _vp, _vp, _int, _int, _int, _int, _flt, _flt,
+                                _vp, _vp, _vp, _vp],
             "orc_bucket": [_vp, _int, _int, _int, _vp, _vp, _vp],
             "orc_expert_ffn": [ctypes.POINTER(_OrcExpert), _int, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp],
             "orc_layer_forward": [_int, _int, _int, _int, _int, _int, _int, _flt, _int,
                                   _vp, _int, _vp, _vp, ctypes.POINTER(_OrcExpert), ctypes.POINTER(_OrcExpert),
                                   _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
+            "orc_layer_forward_topp": [_int, _int, _int, _int, _int, _int, _int, _flt, _int, _flt,
+                                       _vp, _int, _vp, _vp, ctypes.POINTER(_OrcExpert),
+                                       ctypes.POINTER(_OrcExpert), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
             "orc_num_threads": [],
             "orc_set_num_threads": [_int],
         }
@@ -148,7 +153,10 @@ def qmatvec(packed, scales, cols: int, wbits: int, q, d):
     return y
 
 
-def router(x, Wr, bias, n_groups: int, topk_groups: int, top_k: int, rsf: float, want_scores: bool = False):
+def router(x, Wr, bias, n_groups: int, topk_groups: int, top_k: int, rsf: float, want_scores: bool = False,
+           topp: float = 0.0):
+    """Routing of every token: idx, w [T][top_k] (with topp in (0, 1), dropped
+    picks have idx -1 and w 0)."""
     x = _c(x, np.float32)
     Wr = _c(Wr, np.float32)
     bias = _c(bias, np.float32)
@@ -158,8 +166,8 @@ def router(x, Wr, bias, n_groups: int, topk_groups: int, top_k: int, rsf: float,
     w = np.empty((T, top_k), np.float32)
     c = np.empty((T, E), np.float64) if want_scores else None
     gs = np.empty((T, n_groups), np.float64) if want_scores else None
-    _check(lib().orc_router(_p(x), T, H, _p(Wr), _p(bias), E, n_groups, topk_groups, top_k, rsf,
-                            _p(idx), _p(w), _p(c), _p(gs)), "router")
+    _check(lib().orc_router_topp(_p(x), T, H, _p(Wr), _p(bias), E, n_groups, topk_groups, top_k, rsf, topp,
+                                 _p(idx), _p(w), _p(c), _p(gs)), "router")
     if want_scores:
         return idx, w, c, gs
     return idx, w
@@ -243,8 +251,9 @@ def layer_forward(shape, x, Wr, bias, routed: dict, shared: PackedExpert | None)
     ys = np.empty((T, S, H), np.float32)
     hq = np.empty((T, S, I), np.int8)
     hd = np.empty((T, S, I // 32), np.float32)
-    rc = lib().orc_layer_forward(H, I, E, shape.n_groups, shape.topk_groups, k, ns, shape.rsf, shape.wbits,
-                                 _p(x), T, _p(Wr), _p(bias), arr, ctypes.byref(sh), _p(out),
-                                 _p(idx), _p(w), _p(xq), _p(xd), _p(ys), _p(hq), _p(hd))
+    topp = float(getattr(shape, "topp", 0.0))
+    rc = lib().orc_layer_forward_topp(H, I, E, shape.n_groups, shape.topk_groups, k, ns, shape.rsf, shape.wbits,
+                                      topp, _p(x), T, _p(Wr), _p(bias), arr, ctypes.byref(sh), _p(out),
+                                      _p(idx), _p(w), _p(xq), _p(xd), _p(ys), _p(hq), _p(hd))
     _check(rc, "layer_forward")
     return LayerTrace(out, idx, w, xq, xd, ys, hq, hd)

@@ -132,6 +132,7 @@ class LayerShape:
     n_shared: int
     rsf: float
     wbits: int
+    topp: float = 0.0  # adaptive expert top-p in (0, 1); 0 keeps all top_k picks
 
     def matrix_bytes(self, rows: int, cols: int) -> int:
         return rows * cols * self.wbits // 8
@@ -168,6 +169,9 @@ WORKLOADS = {
     "glm52_decode_int4_t1": Workload(
         "glm52_decode_int4_t1", GLM_INT4, 1, 1,
         description="GLM-5.2 shape (6144/2048, 256 experts, 8 groups, top-4 groups, top-8 + 1 shared), int4, 1 token"),
+    "glm52_decode_int4_t1_topp07": Workload(
+        "glm52_decode_int4_t1_topp07", replace(GLM_INT4, topp=0.7), 1, 1,
+        description="glm52_decode_int4_t1 with the adaptive expert top-p at 0.7 (the kept picks' shares reach 0.7)"),
     "glm52_verify_int4_t4": Workload(
         "glm52_verify_int4_t4", GLM_INT4, 4, 2, x_kind="correlated",
         description="GLM-5.2 shape, int4, 4 tokens (1 + 3 drafts) with 0.8-correlated activations"),
