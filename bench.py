@@ -310,9 +310,9 @@ def oracle_sample(wl, n_tokens: int):
     s = wl.shape
     x = synth.make_x(wl)[:n_tokens]
     Wr, bias = synth.make_router_w(wl), synth.make_bias(wl)
-    idx, _ = orc.router(x, Wr, bias, s.n_groups, s.topk_groups, s.top_k, s.rsf)
+    idx, _ = orc.router(x, Wr, bias, s.n_groups, s.topk_groups, s.top_k, s.rsf, topp=s.topp)
     routed = {}
-    for e in sorted(set(idx.reshape(-1).tolist())):
+    for e in sorted(set(idx.reshape(-1).tolist()) - {-1}):  # -1: dropped by the top-p
         routed[e] = orc.pack_expert(*(synth.make_expert_matrix(wl, e, m) for m in range(3)), s.wbits)
     shared = orc.pack_expert(*(synth.make_expert_matrix(wl, 0, m, True) for m in range(3)), s.wbits) \
         if s.n_shared else None

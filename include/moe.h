@@ -57,7 +57,13 @@ typedef enum {
  * Supported: hidden and inter multiples of 32 (up to 16384); n_experts <= 1024
  * and a multiple of n_groups; 2 <= n_experts/n_groups; 1 <= topk_groups <=
  * n_groups <= 32; 1 <= top_k <= min(32, topk_groups * n_experts / n_groups);
- * n_shared 0 or 1; wbits 8 or 4. */
+ * n_shared 0 or 1; wbits 8 or 4.
+ * expert_topp: the adaptive expert top-p ([GN] §모델 다운로드와 실행, option
+ * list: "--topp", an adaptive expert top-p that reads 30-40% fewer experts;
+ * the pages give no rule, this library reads it as nucleus selection over the
+ * top_k picks, see moe_router_select).  0, or any value >= 1, keeps every
+ * pick; it must be finite and >= 0.  The field was added last so that the
+ * members before it keep their offsets. */
 typedef struct {
     int hidden;
     int inter;
@@ -68,6 +74,7 @@ typedef struct {
     int n_shared;
     float routed_scaling_factor;
     int wbits;
+    float expert_topp;
 } moe_config;
 
 /* Packed expert weights for n experts, laid out expert-major:
@@ -118,6 +125,12 @@ size_t moe_router_workspace_bytes(const moe_config *cfg, int T);
  *   best groups; pick the top_k largest c among their experts (ties: lower
  *   index first).  idx[t][j] (int32) lists them in descending c order and
  *   w[t][j] = s / sum(s) * routed_scaling_factor (fp32, unbiased s).
+ * With 0 < expert_topp < 1 each token's picks are then ordered by their share
+ *   q = s / sum(s) (fp64; larger first, ties: the earlier pick), the shortest
+ *   prefix whose running sum of q (fp64, in that order) reaches expert_topp is
+ *   kept (at least one pick), and the kept weights are renormalised:
+ *   w[t][j] = s / sum_kept(s) * routed_scaling_factor (kept s summed in pick
+ *   order).  A dropped pick keeps its position j with idx = -1 and w = 0.
  * router_w [n_experts][hidden] fp32, router_bias [n_experts] fp32.
  * workspace: >= moe_router_workspace_bytes(cfg, T) bytes, 256-byte aligned. */
 int moe_router_select(const moe_config *cfg, const float *x, int T, const float *router_w,
@@ -127,8 +140,11 @@ int moe_router_select(const moe_config *cfg, const float *x, int T, const float 
 /* Batch-union bucketing ([GN] "Batch-union MoE"; [WP] "Batch-Union MoE"):
  * a stable counting sort of the T*top_k (token, slot) pairs of idx [T][top_k]
  * by expert.  counts [n_experts], offsets [n_experts+1] (exclusive prefix
- * sums, offsets[n_experts] = T*top_k) and perm [T*top_k], where perm lists
- * t*top_k + j for expert 0's pairs in increasing t, then expert 1's, etc.
+ * sums, offsets[n_experts] = the number n of routed pairs, T*top_k unless
+ * the top-p dropped some) and perm [T*top_k], where perm lists t*top_k + j
+ * for expert 0's pairs in increasing t, then expert 1's, etc., and ends with
+ * -1 for each dropped pair.  idx = -1 marks a dropped pair; any other value
+ * outside [0, n_experts) records MOE_EDEVICE's index fault.
  * Supports n_experts * ceil(T/32) <= 24576 (T <= 3072 at 256 experts). */
 int moe_bucket_tokens(const moe_config *cfg, const int32_t *idx, int T, int32_t *counts, int32_t *offsets,
                       int32_t *perm, void *stream);
@@ -145,7 +161,8 @@ size_t moe_workspace_bytes(const moe_config *cfg, int T_max);
  *     g = Wg.x, u = Wu.x   with x as Q8_0 (per-block int32 dots, then
  *                          s_row * sum_b d_b * isum_b)
  *     h = silu(g) * u, quantised to Q8_0, y = Wd.h  (same integer-dot form)
- *   out[t] = sum_j w[t,j] * y_{idx[t,j]}(t) + y_shared(t)   (no residual).
+ *   out[t] = sum_j w[t,j] * y_{idx[t,j]}(t) + y_shared(t)   (no residual;
+ *   the sum skips the pairs the top-p dropped, whose experts are not read).
  * x [T][hidden] fp32 (16-byte aligned), out [T][hidden] fp32.  routed holds
  * n_experts experts, shared n_shared (ignored when n_shared == 0).
  * workspace: >= moe_workspace_bytes(cfg, T) bytes, 256-byte aligned; it holds
@@ -195,8 +212,9 @@ int moe_layer_forward_noalloc(const moe_config *cfg, const float *x, int T, cons
 /* Device pointers to the intermediates a moe_layer_forward call leaves in its
  * workspace (valid after the call completes, until the next call on the same
  * workspace).  Slots: routed (token, slot) pairs occupy bucket positions
- * 0 .. T*top_k-1 (the order of perm); the shared expert of token t is slot
- * T*top_k + t. */
+ * 0 .. n-1 (the order of perm, n = offsets[n_experts]; positions n ..
+ * T*top_k-1 are unused when the top-p dropped pairs); the shared expert of
+ * token t is slot T*top_k + t. */
 typedef struct {
     int8_t *xq;        /* [T][hidden]   Q8_0 codes of x */
     float *xd;         /* [T][hidden/32] Q8_0 scales of x */

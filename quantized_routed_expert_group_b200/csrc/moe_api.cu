@@ -75,6 +75,7 @@ static int check_config(const moe_config* c) {
     if (c->n_experts % c->n_groups != 0 || c->topk_groups > c->n_groups) return MOE_EINVAL;
     if (c->top_k > c->topk_groups * (c->n_experts / c->n_groups)) return MOE_EINVAL;
     if (!std::isfinite(c->routed_scaling_factor)) return MOE_EINVAL;
+    if (!std::isfinite(c->expert_topp) || c->expert_topp < 0.f) return MOE_EINVAL;
     if (c->hidden % 32 || c->inter % 32 || c->hidden > 16384 || c->inter > 16384) return MOE_EUNSUPPORTED;
     if (c->n_experts > 1024 || c->n_groups > 32 || c->n_experts / c->n_groups < 2 || c->top_k > 32 ||
         c->n_shared > 1)

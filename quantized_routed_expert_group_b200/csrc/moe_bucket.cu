@@ -7,7 +7,8 @@
 // an expert, pairs keep increasing token order.  A token never picks the same
 // expert twice, so the rank of (t, j) inside bucket e is the number of earlier
 // tokens that picked e: one bit per (expert, token) and a popcount give it
-// without atomics on the order.
+// without atomics on the order.  A pair the adaptive top-p dropped (idx -1)
+// is in no bucket: it gets inv_perm -1, and perm ends with -1 for each.
 #include "moe_device.cuh"
 #include "moe_internal.h"
 
@@ -70,7 +71,7 @@ __global__ void __launch_bounds__(kBucketThreads) k_bucket(const int32_t* __rest
     for (int i = tid; i < n; i += kBucketThreads) {
         const int e = idx[i];
         if (e < 0 || e >= E) {
-            set_error(err, kErrIndex);
+            if (e != -1) set_error(err, kErrIndex);
             continue;
         }
         const int t = i / k;
@@ -92,7 +93,10 @@ __global__ void __launch_bounds__(kBucketThreads) k_bucket(const int32_t* __rest
     }
     for (int i = tid; i < n; i += kBucketThreads) {
         const int e = idx[i];
-        if (e < 0 || e >= E) continue;
+        if (e < 0 || e >= E) {
+            if (inv_perm) inv_perm[i] = -1;
+            continue;
+        }
         const int t = i / k;
         const uint32_t* m = mask + (size_t)e * W;
         int r = __popc(m[t >> 5] & ((1u << (t & 31)) - 1u));
@@ -101,6 +105,7 @@ __global__ void __launch_bounds__(kBucketThreads) k_bucket(const int32_t* __rest
         perm[p] = i;
         if (inv_perm) inv_perm[i] = p;
     }
+    for (int i = total + tid; i < n; i += kBucketThreads) perm[i] = -1;  // dropped pairs
     // active experts (count > 0) in increasing id order
     if (!active) return;  // uniform across the CTA
     __syncthreads();

@@ -286,6 +286,42 @@ __device__ __forceinline__ unsigned long long order_key(double v) {
     return b >= 0 ? (unsigned long long)b ^ 0x8000000000000000ull : ~(unsigned long long)b;
 }
 
+// Adaptive expert top-p of one token's k <= 32 picks, by the token's warp
+// (GeekNews "Show HN: 느린 컴퓨터에서 GLM 5.2 실행하기", §모델 다운로드와 실행,
+// option list: an adaptive expert top-p; the rule is this library's nucleus
+// reading).  Lane j < k holds pick j's unbiased s (sj); ssum is the sum of all
+// k picks' s in pick order.  The picks are ranked by s (larger first, ties to
+// the earlier pick); the first m in rank order are kept, m the smallest count
+// whose running sum of s / ssum (fp64, in rank order) reaches topp, or k.
+// Returns whether lane j's pick is kept and sets *skept to the kept picks' s
+// summed in pick order.  Lanes >= k get false.
+__device__ __forceinline__ bool topp_keep(double sj, double ssum, int k, float topp, int lane, double* skept) {
+    int rank = 0;
+    for (int i = 0; i < k; ++i) {
+        const double si = __shfl_sync(kFull, sj, i);
+        rank += (si > sj || (si == sj && i < lane)) ? 1 : 0;
+    }
+    if (lane >= k) rank = 32;
+    double cum = 0.0;
+    int m = k;
+    for (int r = 0; r < k; ++r) {  // the same values in every lane: a uniform exit
+        const int who = __ffs(__ballot_sync(kFull, rank == r)) - 1;
+        cum += __shfl_sync(kFull, sj, who < 0 ? 0 : who) / ssum;
+        if (cum >= (double)topp) {
+            m = r + 1;
+            break;
+        }
+    }
+    const bool keep = rank < m;
+    double sk = 0.0;
+    for (int i = 0; i < k; ++i) {
+        const double si = __shfl_sync(kFull, sj, i);
+        if (__shfl_sync(kFull, keep ? 1 : 0, i)) sk += si;
+    }
+    *skept = sk;
+    return keep;
+}
+
 // Arg-max of (key, index) over the warp: larger key wins, ties to the lower index.
 __device__ __forceinline__ void warp_argmax_key(unsigned long long& k, int& i) {
 #pragma unroll

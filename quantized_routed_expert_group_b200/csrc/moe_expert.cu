@@ -204,6 +204,7 @@ __global__ void k_combine(ExpertParams p) {
         float acc = 0.0f;
         for (int j = 0; j < p.k; ++j) {
             const int slot = p.inv_perm[t * p.k + j];
+            if (slot < 0) continue;  // dropped by the adaptive top-p
             acc = fmaf(p.w[t * p.k + j], p.y[(int64_t)slot * p.H + c], acc);
         }
         if (p.ns) acc += p.y[((int64_t)p.T * p.k + t) * p.H + c];

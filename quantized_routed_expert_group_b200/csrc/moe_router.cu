@@ -74,11 +74,13 @@ __global__ void __launch_bounds__(256) k_router_logits(const float* __restrict__
 // Selection: one warp per token.  s = sigmoid(logit), c = s + bias; group
 // score = sum of the two largest c (first the maximum, then the largest of the
 // rest, ties to the lower index); keep the topk_groups best groups; take the
-// top_k largest c in them, best first; w = s / sum(s) * rsf.
+// top_k largest c in them, best first; w = s / sum(s) * rsf.  With topp in
+// (0, 1) the adaptive expert top-p then drops the picks past the share
+// prefix that reaches topp (idx -1, w 0) and renormalises the rest.
 __global__ void __launch_bounds__(128) k_router_select(const double* __restrict__ logits,
                                                        const float* __restrict__ bias, int T, int E, int G,
-                                                       int tg, int k, float rsf, int32_t* __restrict__ idx,
-                                                       float* __restrict__ wout) {
+                                                       int tg, int k, float rsf, float topp,
+                                                       int32_t* __restrict__ idx, float* __restrict__ wout) {
     extern __shared__ double sm[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = blockIdx.x * 4 + warp;
@@ -133,6 +135,16 @@ __global__ void __launch_bounds__(128) k_router_select(const double* __restrict_
         if (lane == n) sel_mine = i;
         ssum += ss[i];  // same order as the picks: s_0 + s_1 + ...
     }
+    if (topp > 0.f && topp < 1.f) {
+        const double sj = lane < k ? ss[sel_mine] : 0.0;
+        double skept;
+        const bool keep = topp_keep(sj, ssum, k, topp, lane, &skept);
+        if (lane < k) {
+            idx[(int64_t)t * k + lane] = keep ? sel_mine : -1;
+            wout[(int64_t)t * k + lane] = keep ? (float)(sj / skept * (double)rsf) : 0.f;
+        }
+        return;
+    }
     if (lane < k) {
         idx[(int64_t)t * k + lane] = sel_mine;
         wout[(int64_t)t * k + lane] = (float)(ss[sel_mine] / ssum * (double)rsf);
@@ -153,7 +165,7 @@ cudaError_t launch_router(const moe_config& c, const float* x, int T, const floa
         if (e != cudaSuccess) return e;
     }
     k_router_select<<<(T + 3) / 4, 128, smem, s>>>(logits, bias, T, c.n_experts, c.n_groups, c.topk_groups,
-                                                   c.top_k, c.routed_scaling_factor, idx, w);
+                                                   c.top_k, c.routed_scaling_factor, c.expert_topp, idx, w);
     return cudaGetLastError();
 }
 

@@ -133,6 +133,7 @@ struct SmallGeom {
 struct SmallParams {
     int T, H, I, E, G, tg, k, ns, wbits;
     float rsf;
+    float topp;  // adaptive expert top-p; outside (0, 1): keep every pick
     const float* x;
     const float* router_w;
     const float* bias;
@@ -809,14 +810,39 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
         }
         consumers_sync();
     }
-    // 5. bucketing
+    // 4b. adaptive expert top-p (one warp per token): the dropped picks leave
+    // sel as -1 before the bucketing, and the weights are final here
+    const bool topp_on = p.topp > 0.f && p.topp < 1.f;
+    if (topp_on) {
+        if (warp < T) {
+            const int t = warp;
+            const int e = lane < k ? sel[t * 32 + lane] : 0;
+            const double sj = lane < k ? ss[(size_t)t * E + e] : 0.0;
+            double ssum = 0.0;
+            for (int j = 0; j < k; ++j) ssum += __shfl_sync(kFull, sj, j);  // pick order
+            double skept;
+            const bool keep = topp_keep(sj, ssum, k, p.topp, lane, &skept);
+            if (lane < k) {
+                const float wv = keep ? (float)(sj / skept * (double)p.rsf) : 0.f;
+                s.selw[t * k + lane] = wv;
+                if (!keep) sel[t * 32 + lane] = -1;
+                if (publish) {
+                    p.idx[(int64_t)t * k + lane] = keep ? e : -1;
+                    p.w[(int64_t)t * k + lane] = wv;
+                }
+            }
+        }
+        consumers_sync();
+    }
+    // 5. bucketing (a dropped pick, sel -1, is in no bucket: inv -1)
     const int n = T * k;
     if (n <= 32) {
         // one warp, lane = pick t * k + j: same-expert lanes found with a
         // match, positions from counts over the other lanes
         if (warp == 0) {
-            const bool act = lane < n;
-            const int e = act ? sel[(lane / k) * 32 + lane % k] : 0x7FFFFFFF;
+            const int e_in = lane < n ? sel[(lane / k) * 32 + lane % k] : -1;
+            const bool act = e_in >= 0;
+            const int e = act ? e_in : 0x7FFFFFFF;
             const uint32_t same = __match_any_sync(kFull, e);
             const int lead = __ffs(same) - 1;
             const int rank = __popc(same & ((1u << lane) - 1u));  // earlier picks (tokens) of this expert
@@ -842,7 +868,13 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
                     p.inv_perm[lane] = pos;
                     if (lane == lead) p.active[1 + dless] = e;
                 }
+            } else if (lane < n) {  // dropped by the top-p
+                s.inv[lane] = -1;
+                if (publish) p.inv_perm[lane] = -1;
             }
+            const int n_act = __popc(__ballot_sync(kFull, act));  // routed pairs
+            if (publish && lane >= n_act && lane < n) p.perm[lane] = -1;
+            if (lane == 0) s.misc[1] = n_act;
             __syncwarp();
             if (act && rank < 4) s.ent[1 + dless].tok[rank] = lane / k;
             const int U = __popc(__ballot_sync(kFull, act && lane == lead));
@@ -862,7 +894,7 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
         if (publish) {
             // counts and offsets of every expert: the first entry (entries are
             // in ascending expert order) whose expert is not below e
-            const int U = s.misc[0];
+            const int U = s.misc[0], n_act = s.misc[1];
 #pragma unroll 1
             for (int e = tid; e <= E; e += kConsumers) {
                 int lo = 1, hi = U + 1;
@@ -873,12 +905,12 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
                     else hi = mid;
                 }
                 const bool in = lo <= U;
-                p.offsets[e] = in ? s.ent[lo].slot0 : n;
+                p.offsets[e] = in ? s.ent[lo].slot0 : n_act;
                 if (e < E) p.counts[e] = (in && s.ent[lo].expert == e) ? s.ent[lo].n : 0;
             }
         }
     } else {
-        if (tid < n) atomicAdd(&cnt[sel[(tid / k) * 32 + tid % k]], 1);
+        if (tid < n && sel[(tid / k) * 32 + tid % k] >= 0) atomicAdd(&cnt[sel[(tid / k) * 32 + tid % k]], 1);
         consumers_sync();
         // block-wide exclusive scans over experts (one thread per expert, E <= 256)
         {
@@ -913,7 +945,10 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
                     ei.slot0 = o;
                     ei.n = cv;
                 }
-                if (tid == E - 1) s.misc[0] = ai + nz;
+                if (tid == E - 1) {
+                    s.misc[0] = ai + nz;
+                    s.misc[1] = o + cv;  // routed pairs
+                }
                 if (publish) {
                     p.offsets[tid] = o;
                     p.counts[tid] = cv;
@@ -934,7 +969,11 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
             }
         }
         consumers_sync();
-        if (tid < n) {
+        if (publish && tid < n && tid >= s.misc[1]) p.perm[tid] = -1;  // the dropped pairs' tail
+        if (tid < n && sel[(tid / k) * 32 + tid % k] < 0) {  // dropped by the top-p
+            s.inv[tid] = -1;
+            if (publish) p.inv_perm[tid] = -1;
+        } else if (tid < n) {
             const int t = tid / k;
             const int e = sel[t * 32 + tid % k];
             int rank = 0;
@@ -953,8 +992,9 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
         consumers_sync();  // every table the producer reads is written
         if (tid == 0) mbar_arrive(s.routing);
     }
-    // routing weights from the unbiased sigmoid, summed in pick order
-    if (warp < T && lane < k) {
+    // routing weights from the unbiased sigmoid, summed in pick order (with the
+    // top-p they were written before the bucketing)
+    if (!topp_on && warp < T && lane < k) {
         const int t = warp;
         double ssum = 0.0;
 #pragma unroll 8
@@ -1223,8 +1263,8 @@ __device__ __forceinline__ void do_combine(const SmallParams& p, const SmemPtrs&
         const int t = idx / rows, r = idx - t * rows;
         float acc = 0.0f;  // fixed order: slots 0..k-1, then the shared expert
         for (int j = 0; j < k; ++j) {
-            int sl = s.inv[t * k + j];
-            sl = (sl < 0 || sl >= T * k) ? 0 : sl;
+            const int sl = s.inv[t * k + j];
+            if (sl < 0 || sl >= T * k) continue;  // dropped by the adaptive top-p
             const float2 h = ys[sl * rpc + r];
             acc = fmaf(s.selw[t * k + j], h.x + h.y, acc);
         }
@@ -1437,7 +1477,7 @@ cudaError_t launch_small(const SmallArgs& a, cudaStream_t st) {
     const moe_config& c = *a.cfg;
     SmallParams p;
     p.T = a.T; p.H = c.hidden; p.I = c.inter; p.E = c.n_experts; p.G = c.n_groups; p.tg = c.topk_groups;
-    p.k = c.top_k; p.ns = c.n_shared; p.wbits = c.wbits; p.rsf = c.routed_scaling_factor;
+    p.k = c.top_k; p.ns = c.n_shared; p.wbits = c.wbits; p.rsf = c.routed_scaling_factor; p.topp = c.expert_topp;
     p.x = a.x; p.router_w = a.router_w; p.bias = a.bias; p.routed = a.routed; p.shared = a.shared;
     p.xq = a.xq; p.xd = a.xd; p.logits = a.logits; p.idx = a.idx; p.w = a.w; p.counts = a.counts;
     p.offsets = a.offsets; p.perm = a.perm; p.inv_perm = a.inv_perm; p.active = a.active;

@@ -31,7 +31,7 @@ class MoeError(RuntimeError):
 class MoeConfig(ctypes.Structure):
     _fields_ = [("hidden", _int), ("inter", _int), ("n_experts", _int), ("n_groups", _int),
                 ("topk_groups", _int), ("top_k", _int), ("n_shared", _int),
-                ("routed_scaling_factor", _flt), ("wbits", _int)]
+                ("routed_scaling_factor", _flt), ("wbits", _int), ("expert_topp", _flt)]
 
 
 class MoeExperts(ctypes.Structure):
@@ -114,7 +114,7 @@ def _cuda(t: torch.Tensor, dtype: torch.dtype, name: str) -> torch.Tensor:
 
 def config(shape: synth.LayerShape) -> MoeConfig:
     return MoeConfig(shape.hidden, shape.inter, shape.n_experts, shape.n_groups, shape.topk_groups,
-                     shape.top_k, shape.n_shared, shape.rsf, shape.wbits)
+                     shape.top_k, shape.n_shared, shape.rsf, shape.wbits, shape.topp)
 
 
 # ----------------------------------------------------------------------------

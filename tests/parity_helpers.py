@@ -98,9 +98,14 @@ def check_layer(pair: Pair, x: np.ndarray | None = None, check_intermediates: bo
     np.testing.assert_array_equal(v["offsets"], offsets)
     np.testing.assert_array_equal(v["perm"], perm)
     k, S = s.top_k, s.top_k + s.n_shared
-    # slot p of the GPU holds pair perm[p] = t*k + j; shared slot T*k + t
-    t_of = np.concatenate([perm // k, np.arange(T)]) if s.n_shared else perm // k
-    j_of = np.concatenate([perm % k, np.full(T, k)]) if s.n_shared else perm % k
+    # slot p < n of the GPU holds pair perm[p] = t*k + j (n = routed pairs: the
+    # top-p leaves slots n .. T*k-1 unused); shared slot T*k + t
+    n = int(offsets[-1])
+    live = perm[:n]
+    t_of = np.concatenate([live // k, np.arange(T)]) if s.n_shared else live // k
+    j_of = np.concatenate([live % k, np.full(T, k)]) if s.n_shared else live % k
+    slots = np.concatenate([np.arange(n), T * k + np.arange(T)]) if s.n_shared else np.arange(n)
+    v["hq"], v["y"] = v["hq"][slots], v["y"][slots]
     hq_ref = tr.hq[t_of, j_of]
     dq = np.abs(v["hq"].astype(np.int32) - hq_ref.astype(np.int32))
     assert dq.max() <= 1

@@ -16,7 +16,8 @@ from quantized_routed_expert_group_b200 import moe, synth
 
 pytestmark = pytest.mark.gpu
 
-FULL = ["glm52_decode_int4_t1", "glm52_verify_int4_t4", "glm52_int8_t16_outliers", "glm52_prefill_int4_t512_zipf"]
+FULL = ["glm52_decode_int4_t1", "glm52_verify_int4_t4", "glm52_int8_t16_outliers", "glm52_prefill_int4_t512_zipf",
+        "glm52_decode_int4_t1_topp07"]
 
 
 @pytest.fixture(scope="module", params=FULL)
@@ -41,7 +42,7 @@ def test_full_router_and_bucket(full):
     wl, layer, x, out, v = full
     s = wl.shape
     io, wo, c, gs = orc.router(x, synth.make_router_w(wl), synth.make_bias(wl), s.n_groups, s.topk_groups,
-                               s.top_k, s.rsf, want_scores=True)
+                               s.top_k, s.rsf, want_scores=True, topp=s.topp)
     np.testing.assert_array_equal(v["idx"], io)
     np.testing.assert_allclose(v["w"], wo, rtol=1e-6)
     counts, offsets, perm = orc.bucket(io, s.n_experts)
@@ -55,7 +56,7 @@ def test_full_sampled_outputs(full):
     wl, layer, x, out, v = full
     s = wl.shape
     toks = _sample_tokens(wl.T)
-    need = sorted(set(v["idx"][toks].reshape(-1).tolist()))
+    need = sorted(set(v["idx"][toks].reshape(-1).tolist()) - {-1})  # -1: dropped by the top-p
     routed = {}
     for e in need:
         ex = orc.pack_expert(*host_expert_mats(wl, e), s.wbits)
@@ -73,11 +74,13 @@ def test_full_sampled_outputs(full):
     assert err <= OUT_TOL
     # per-block int32 dots, bit-exact: gate rows on x's codes, down rows on the
     # oracle's own h codes (h itself may round differently by a few ulp)
-    t0, e0 = toks[0], int(v["idx"][toks[0], 0])
+    t0 = toks[0]
+    j0 = int(np.nonzero(v["idx"][t0] >= 0)[0][0])  # the first pick the top-p kept (0 without it)
+    e0 = int(v["idx"][t0, j0])
     ex = routed[e0]
     xq = torch.from_numpy(tr.xq[0:1]).cuda()
     got = moe.block_dots(layer.routed.w_gate[e0], s.hidden, s.wbits, xq).cpu().numpy()
     np.testing.assert_array_equal(got, orc.block_dots(ex.wg, s.hidden, s.wbits, tr.xq[0:1]))
-    hq = np.ascontiguousarray(tr.hq[0, 0:1])
+    hq = np.ascontiguousarray(tr.hq[0, j0:j0 + 1])
     got = moe.block_dots(layer.routed.w_down[e0], s.inter, s.wbits, torch.from_numpy(hq).cuda()).cpu().numpy()
     np.testing.assert_array_equal(got, orc.block_dots(ex.wd, s.inter, s.wbits, hq))

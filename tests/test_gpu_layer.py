@@ -21,6 +21,11 @@ FULLGROUPS = synth.LayerShape(256, 64, 16, 4, 2, 8, 1, 2.5, 4)   # top_k = every
 # groups of 32 experts (one warp per group in the fused selection), as in the GLM-5.2 shape
 GROUP32 = synth.LayerShape(512, 96, 128, 4, 2, 8, 1, 2.5, 4)
 GROUP32_K16 = synth.LayerShape(256, 64, 64, 2, 1, 16, 1, 1.0, 8)   # one kept group, top_k 16 of its 32
+# the adaptive expert top-p: picks past the share prefix that reaches topp are dropped
+MID4_TOPP = synth.LayerShape(1056, 160, 32, 4, 2, 4, 1, 2.5, 4, topp=0.5)
+MID8_TOPP = synth.LayerShape(1056, 160, 32, 4, 2, 4, 1, 1.0, 8, topp=0.7)
+GROUP32_TOPP = synth.LayerShape(512, 96, 128, 4, 2, 8, 1, 2.5, 4, topp=0.7)
+GROUP32_K16_TOPP = synth.LayerShape(256, 64, 64, 2, 1, 16, 1, 1.0, 8, topp=0.6)
 
 
 @pytest.fixture(scope="module")
@@ -80,12 +85,20 @@ def test_tiny_host_entry_point(tiny):
     (GROUP32, 1, 24, "normal"), (GROUP32, 2, 25, "normal"), (GROUP32, 3, 26, "normal"),
     (GROUP32, 4, 27, "correlated"), (GROUP32_K16, 1, 28, "normal"), (GROUP32_K16, 4, 29, "normal"),
     (GROUP32, 6, 30, "normal"),
+    # adaptive expert top-p: multi-kernel path, then the fused path (general
+    # selection, groups-of-32 selection, and the bucketing of more than 32 pairs)
+    (MID4_TOPP, 37, 31, "normal"), (GROUP32_TOPP, 6, 32, "normal"),
+    (MID4_TOPP, 3, 33, "normal"), (MID8_TOPP, 1, 34, "normal"), (GROUP32_TOPP, 1, 35, "normal"),
+    (GROUP32_TOPP, 2, 36, "normal"), (GROUP32_TOPP, 4, 37, "correlated"), (GROUP32_K16_TOPP, 4, 38, "normal"),
 ])
 def test_mid_layers(shape, T, seed, x_kind):
     wl = make_workload(f"mid_{shape.wbits}_{T}", shape, T, seed, x_kind=x_kind)
     p = build_pair(wl)
     check_banks_equal(p)
     st = check_layer(p)
+    if 0 < shape.topp < 1:  # the top-p must actually drop pairs in these cases
+        st["dropped"] = int((p.layer.view(T)["idx"] < 0).sum().item())
+        assert st["dropped"] > 0
     print(wl.name, st)
     del p
     torch.cuda.empty_cache()

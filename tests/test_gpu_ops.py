@@ -73,14 +73,16 @@ def _router_case(name, T):
 
 @pytest.mark.parametrize("name,T", [("tiny_h256_e16_int8_t4", 4), ("tiny_h256_e16_int8_t4", 133),
                                     ("glm52_decode_int4_t1", 1), ("glm52_verify_int4_t4", 4),
-                                    ("glm52_int8_t16_outliers", 16), ("glm52_prefill_int4_t512_zipf", 512)])
+                                    ("glm52_int8_t16_outliers", 16), ("glm52_prefill_int4_t512_zipf", 512),
+                                    ("glm52_decode_int4_t1_topp07", 1), ("glm52_decode_int4_t1_topp07", 64)])
 def test_router_bitexact(name, T):
     wl, x, Wr, bias = _router_case(name, T)
     s = wl.shape
     cfg = moe.config(s)
     idx, w = moe.router_select(cfg, torch.from_numpy(x).cuda(), torch.from_numpy(Wr).cuda(),
                                torch.from_numpy(bias).cuda())
-    io, wo, c, gs = orc.router(x, Wr, bias, s.n_groups, s.topk_groups, s.top_k, s.rsf, want_scores=True)
+    io, wo, c, gs = orc.router(x, Wr, bias, s.n_groups, s.topk_groups, s.top_k, s.rsf, want_scores=True,
+                               topp=s.topp)
     got = idx.cpu().numpy()
     # The logits are summed in different orders on the two sides (oracle: fp64;
     # GPU: compensated fp32 pairs, ~2^-48 relative); only candidates closer than
@@ -88,17 +90,26 @@ def test_router_bitexact(name, T):
     top = -np.sort(-c, axis=1)[:, : s.top_k + 1]
     gtop = -np.sort(-gs, axis=1)[:, : s.topk_groups + 1]
     margin = min(np.abs(np.diff(top, axis=1)).min(), np.abs(np.diff(gtop, axis=1)).min())
+    if 0 < s.topp < 1:  # the top-p's decision: the running shares against topp
+        i0, _ = orc.router(x, Wr, bias, s.n_groups, s.topk_groups, s.top_k, s.rsf)
+        sig = 1.0 / (1.0 + np.exp(-(x.astype(np.float64) @ Wr.astype(np.float64).T)))
+        for t in range(T):
+            q = np.sort(sig[t, i0[t]])[::-1] / sig[t, i0[t]].sum()
+            margin = min(margin, np.abs(np.cumsum(q) - s.topp).min())
     if margin < 1e-10:
         pytest.skip(f"degenerate seed: selection margin {margin:.3g}")
     np.testing.assert_array_equal(got, io)
     np.testing.assert_allclose(w.cpu().numpy(), wo, rtol=1e-6)
 
 
-@pytest.mark.parametrize("T,k,E", [(1, 8, 256), (4, 2, 16), (37, 8, 256), (512, 8, 256), (3000, 8, 256), (0, 8, 256)])
-def test_bucket_bitexact(T, k, E):
+@pytest.mark.parametrize("T,k,E,drop", [(1, 8, 256, 0.0), (4, 2, 16, 0.0), (37, 8, 256, 0.0), (512, 8, 256, 0.0),
+                                        (3000, 8, 256, 0.0), (0, 8, 256, 0.0), (37, 8, 256, 0.3), (5, 4, 16, 0.5)])
+def test_bucket_bitexact(T, k, E, drop):
     rng = np.random.default_rng(T + E)
     rows = [rng.choice(E, size=k, replace=False) for _ in range(T)]
     idx = (np.stack(rows) if rows else np.zeros((0, k))).astype(np.int32).reshape(T, k)
+    if drop:  # pairs the adaptive top-p dropped
+        idx[rng.random(idx.shape) < drop] = -1
     shape = synth.LayerShape(256, 128, E, 8 if E >= 16 else 2, 4 if E >= 16 else 1, k, 1, 1.0, 4)
     cfg = moe.config(shape)
     counts, offsets, perm = moe.bucket_tokens(cfg, torch.from_numpy(idx).cuda() if T else
