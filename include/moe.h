@@ -57,7 +57,8 @@ typedef enum {
  * Supported: hidden and inter multiples of 32 (up to 16384); n_experts <= 1024
  * and a multiple of n_groups; 2 <= n_experts/n_groups; 1 <= topk_groups <=
  * n_groups <= 32; 1 <= top_k <= min(32, topk_groups * n_experts / n_groups);
- * n_shared 0 or 1; wbits 8 or 4.
+ * n_shared 0 or 1; wbits 8, 4 or 2 (int2 runs the fused small-batch kernel
+ * when hidden and inter are multiples of 64, else the multi-kernel path).
  * expert_topp: the adaptive expert top-p ([GN] §모델 다운로드와 실행, option
  * list: "--topp", an adaptive expert top-p that reads 30-40% fewer experts;
  * the pages give no rule, this library reads it as nucleus selection over the
@@ -82,7 +83,8 @@ typedef struct {
  *   w_down       : [n][hidden][inter * wbits / 8] bytes
  *   s_gate, s_up : [n][inter] fp32 row scales;  s_down : [n][hidden]
  * Codes are two's complement; int4 packs element 2j in the low nibble and
- * 2j+1 in the high nibble of byte j ([GN] quantisation-kernel bullet: int8 /
+ * 2j+1 in the high nibble of byte j, int2 packs element 4j+m in bits
+ * 2m..2m+1 of byte j ([GN] quantisation-kernel bullet: int8 /
  * packed int4 / packed int2 with per-row scales; the bit layout is this
  * library's).  Weight pointers must be 16-byte aligned, scale pointers
  * 4-byte aligned. */

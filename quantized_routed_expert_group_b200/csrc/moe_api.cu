@@ -80,7 +80,7 @@ static int check_config(const moe_config* c) {
     if (c->n_experts > 1024 || c->n_groups > 32 || c->n_experts / c->n_groups < 2 || c->top_k > 32 ||
         c->n_shared > 1)
         return MOE_EUNSUPPORTED;
-    if (c->wbits != 4 && c->wbits != 8) return MOE_EUNSUPPORTED;
+    if (c->wbits != 4 && c->wbits != 8 && c->wbits != 2) return MOE_EUNSUPPORTED;
     return MOE_OK;
 }
 
@@ -374,7 +374,7 @@ MOE_API int moe_workspace_view(const moe_config* cfg, int T, void* workspace, si
 MOE_API int moe_block_dots(const uint8_t* packed, int64_t rows, int cols, int wbits, const int8_t* q, int n,
                            int32_t* out, void* stream) {
     if (rows < 0 || n < 0 || cols <= 0 || cols % 32) return MOE_EINVAL;
-    if (wbits != 4 && wbits != 8) return MOE_EUNSUPPORTED;
+    if (wbits != 4 && wbits != 8 && wbits != 2) return MOE_EUNSUPPORTED;
     if (rows == 0 || n == 0) return MOE_OK;
     if (!packed || !q || !out || !aligned(packed, 16) || !aligned(q, 16) || !aligned(out, 4)) return MOE_EINVAL;
     return status_of(launch_block_dots(packed, rows, cols, wbits, q, n, out, (cudaStream_t)stream));

@@ -34,6 +34,12 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
     return r;
 }
 
+__device__ __forceinline__ uint2 ld_stream_v2(const void* p) {
+    uint2 r;
+    asm("ld.global.nc.L1::no_allocate.L2::256B.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+    return r;
+}
+
 __device__ __forceinline__ float4 ld_stream_f4(const float4* p) {
     float4 r;
     asm("ld.global.nc.L1::no_allocate.L2::256B.v4.f32 {%0, %1, %2, %3}, [%4];"
@@ -50,7 +56,8 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
 // Activation block of 32 int8 codes, kept in the order the weight format wants:
 // for int8 weights the natural order (8 words of 4 codes), for int4 weights the
 // even and odd elements of each group of 8 split apart, matching the low and
-// high nibbles of one packed 32-bit weight word.
+// high nibbles of one packed 32-bit weight word, for int2 weights the elements
+// of each half block (16) grouped by their 2-bit field position m.
 struct ActBlock {
     uint32_t v[8];
 };
@@ -73,6 +80,41 @@ __device__ __forceinline__ ActBlock act_nibble_order(uint4 lo, uint4 hi) {
         a.v[2 * k + 1] = __byte_perm(n[2 * k], n[2 * k + 1], 0x7531);
     }
     return a;
+}
+
+// Natural -> crumb order: for each half block h (elements 16h..16h+15, four
+// natural words n[4h..4h+3]) word 4h + m holds elements 16h + 4j + m, j = 0..3
+// (a 4 x 4 byte transpose), matching field m of the 4 bytes of one packed-int2
+// weight word.
+__device__ __forceinline__ ActBlock act_crumb_order(uint4 lo, uint4 hi) {
+    const uint32_t n[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+    ActBlock a;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t t0 = __byte_perm(n[4 * h], n[4 * h + 1], 0x5140);      // b0 b0' b1 b1'
+        const uint32_t t1 = __byte_perm(n[4 * h + 2], n[4 * h + 3], 0x5140);
+        const uint32_t u0 = __byte_perm(n[4 * h], n[4 * h + 1], 0x7362);      // b2 b2' b3 b3'
+        const uint32_t u1 = __byte_perm(n[4 * h + 2], n[4 * h + 3], 0x7362);
+        a.v[4 * h + 0] = __byte_perm(t0, t1, 0x5410);
+        a.v[4 * h + 1] = __byte_perm(t0, t1, 0x7632);
+        a.v[4 * h + 2] = __byte_perm(u0, u1, 0x5410);
+        a.v[4 * h + 3] = __byte_perm(u0, u1, 0x7632);
+    }
+    return a;
+}
+
+// 64 * the exact dot of one packed-int2 block (8 bytes = 32 codes, element
+// 4j + m in bits 2m..2m+1 of byte j) with a crumb-ordered activation block:
+// shifting field m to the top two bits of its byte makes the byte 64 * code as
+// a signed int8, so each field position is one dp4a; |64 * dot| <= 520192.
+__device__ __forceinline__ int dot_block_i2_x64(uint32_t w0, uint32_t w1, const ActBlock& a) {
+    int acc = 0;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        acc = __dp4a(static_cast<int>((w0 << (6 - 2 * m)) & 0xC0C0C0C0u), static_cast<int>(a.v[m]), acc);
+        acc = __dp4a(static_cast<int>((w1 << (6 - 2 * m)) & 0xC0C0C0C0u), static_cast<int>(a.v[4 + m]), acc);
+    }
+    return acc;
 }
 
 // Exact int32 dot of one packed-int4 block (16 bytes = 32 codes, element 2j in
@@ -151,10 +193,12 @@ __device__ __forceinline__ ActBlock load_act_block(const int8_t* q) {
     const uint4 lo = ld_nc_v4(q);
     const uint4 hi = ld_nc_v4(q + 16);
     if constexpr (WBITS == 4) return act_nibble_order(lo, hi);
+    else if constexpr (WBITS == 2) return act_crumb_order(lo, hi);
     else return act_natural(lo, hi);
 }
 
-// One weight block of a row: 32 codes = 16 bytes (int4) or 32 bytes (int8).
+// One weight block of a row: 32 codes = 8 bytes (int2, in a.x, a.y), 16 bytes
+// (int4) or 32 bytes (int8).
 template <int WBITS>
 struct WBlock {
     uint4 a, b;
@@ -166,6 +210,10 @@ __device__ __forceinline__ WBlock<WBITS> load_w_block(const uint8_t* row, int bl
     if constexpr (WBITS == 4) {
         w.a = ld_stream_v4(row + 16 * blk);
         w.b = make_uint4(0, 0, 0, 0);
+    } else if constexpr (WBITS == 2) {
+        const uint2 v = ld_stream_v2(row + 8 * blk);
+        w.a = make_uint4(v.x, v.y, 0, 0);
+        w.b = make_uint4(0, 0, 0, 0);
     } else {
         w.a = ld_stream_v4(row + 32 * blk);
         w.b = ld_stream_v4(row + 32 * blk + 16);
@@ -176,22 +224,24 @@ __device__ __forceinline__ WBlock<WBITS> load_w_block(const uint8_t* row, int bl
 template <int WBITS>
 __device__ __forceinline__ int dot_block(const WBlock<WBITS>& w, const ActBlock& a) {
     if constexpr (WBITS == 4) return dot_block_i4(w.a, a);
+    else if constexpr (WBITS == 2) return dot_block_i2_x64(w.a.x, w.a.y, a) >> 6;
     else return dot_block_i8(w.a, w.b, a);
 }
 
-// The block dot times the factor dot_scale<WBITS>() (16 for int4, 1 for
-// int8) as an exact integer (below 2^24, so exact as a float too); corr is
-// act_corr<WBITS>(a).
+// The block dot times the factor dot_scale<WBITS>() (64 for int2, 16 for
+// int4, 1 for int8) as an exact integer (below 2^24, so exact as a float too);
+// corr is act_corr<WBITS>(a).
 template <int WBITS>
 __device__ __forceinline__ int dot_block_scaled(const WBlock<WBITS>& w, const ActBlock& a, int corr) {
     if constexpr (WBITS == 4) return dot_block_i4_x16(w.a, a, corr);
+    else if constexpr (WBITS == 2) return dot_block_i2_x64(w.a.x, w.a.y, a);
     else return dot_block_i8(w.a, w.b, a);
 }
 
 // 1 / that factor (a power of two: scaling by it is exact).
 template <int WBITS>
 __device__ __forceinline__ float dot_unscale() {
-    return WBITS == 4 ? 0.0625f : 1.0f;
+    return WBITS == 4 ? 0.0625f : WBITS == 2 ? 0.015625f : 1.0f;
 }
 
 template <int WBITS>

@@ -257,6 +257,11 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t s, cudaEvent_t cons
         if (tch == 2) return launch_experts_t<4, 2>(p, s, ev);
         return launch_experts_t<4, 4>(p, s, ev);
     }
+    if (c.wbits == 2) {
+        if (tch == 1) return launch_experts_t<2, 1>(p, s, ev);
+        if (tch == 2) return launch_experts_t<2, 2>(p, s, ev);
+        return launch_experts_t<2, 4>(p, s, ev);
+    }
     if (tch == 1) return launch_experts_t<8, 1>(p, s, ev);
     if (tch == 2) return launch_experts_t<8, 2>(p, s, ev);
     return launch_experts_t<8, 4>(p, s, ev);
@@ -287,6 +292,7 @@ cudaError_t launch_block_dots(const uint8_t* packed, int64_t rows, int cols, int
     const int64_t grid = (warps + 7) / 8;
     if (grid > 0x7fffffff) return cudaErrorInvalidValue;
     if (wbits == 4) k_block_dots<4><<<(unsigned)grid, 256, 0, s>>>(packed, rows, cols, q, n, out);
+    else if (wbits == 2) k_block_dots<2><<<(unsigned)grid, 256, 0, s>>>(packed, rows, cols, q, n, out);
     else k_block_dots<8><<<(unsigned)grid, 256, 0, s>>>(packed, rows, cols, q, n, out);
     return cudaGetLastError();
 }

@@ -245,6 +245,9 @@ static int select_scratch_bytes(int T, int E) { return 3 * T * E * 8 + 4 * 32 * 
 bool small_path_supported(const moe_config& c, int T) {
     if (T < 1 || T > 4) return false;
     if (c.hidden > 6144 || c.n_experts > 256 || c.n_groups > 32 || c.top_k > 32) return false;
+    // bulk copies of whole weight rows start on 16-byte boundaries (int2 rows
+    // of a hidden or inter size that is not a multiple of 64 do not)
+    if ((c.hidden * c.wbits / 8) % 16 || (c.inter * c.wbits / 8) % 16) return false;
     const SmallGeom g = small_geometry(c, T, device_info().sm_count);
     if (g.rg < 4) return false;  // at least one gate/up row per row group
     if (c.hidden / 32 > kColThreads * kMaxGuBlocks || c.inter / 32 > kColThreads * kMaxDownBlocks) return false;
@@ -1020,6 +1023,10 @@ __device__ __forceinline__ WBlock<WBITS> load_block_smem(const uint8_t* row, int
     if constexpr (WBITS == 4) {
         w.a = *reinterpret_cast<const uint4*>(row + 16 * b);
         w.b = make_uint4(0, 0, 0, 0);
+    } else if constexpr (WBITS == 2) {
+        const uint2 v = *reinterpret_cast<const uint2*>(row + 8 * b);
+        w.a = make_uint4(v.x, v.y, 0, 0);
+        w.b = make_uint4(0, 0, 0, 0);
     } else {
         w.a = *reinterpret_cast<const uint4*>(row + 32 * b);
         w.b = *reinterpret_cast<const uint4*>(row + 32 * b + 16);
@@ -1167,6 +1174,7 @@ __device__ __forceinline__ void down_act(const uint8_t* act, const float* hdv, i
         const uint4 lo = *reinterpret_cast<const uint4*>(act + (size_t)ii * I + 32 * b);
         const uint4 hi = *reinterpret_cast<const uint4*>(act + (size_t)ii * I + 32 * b + 16);
         if constexpr (WBITS == 4) a[i] = act_nibble_order(lo, hi);
+        else if constexpr (WBITS == 2) a[i] = act_crumb_order(lo, hi);
         else a[i] = act_natural(lo, hi);
         dh[i] = okb ? hdv[ii * nbI + b] * dot_unscale<WBITS>() : 0.0f;
         cr[i] = act_corr<WBITS>(a[i]);
@@ -1399,7 +1407,9 @@ __global__ void __launch_bounds__(kSmallThreads, 1) k_moe_small(const __grid_con
             const int t = job / nb, b = job % nb;
             const uint4 lo = __ldcg(reinterpret_cast<const uint4*>(p.xq + (int64_t)t * p.H + b * 32));
             const uint4 hi = __ldcg(reinterpret_cast<const uint4*>(p.xq + (int64_t)t * p.H + b * 32 + 16));
-            const ActBlock a = WBITS == 4 ? act_nibble_order(lo, hi) : act_natural(lo, hi);
+            const ActBlock a = WBITS == 4 ? act_nibble_order(lo, hi)
+                             : WBITS == 2 ? act_crumb_order(lo, hi)
+                                          : act_natural(lo, hi);
             *reinterpret_cast<uint4*>(s.xq + ((size_t)(t * 2 + 0) * nb + b) * 16) = make_uint4(a.v[0], a.v[1], a.v[2], a.v[3]);
             *reinterpret_cast<uint4*>(s.xq + ((size_t)(t * 2 + 1) * nb + b) * 16) = make_uint4(a.v[4], a.v[5], a.v[6], a.v[7]);
         }
@@ -1493,6 +1503,11 @@ cudaError_t launch_small(const SmallArgs& a, cudaStream_t st) {
         if (tm == 1) return launch_small_t<4, 1>(p, st);
         if (tm == 2) return launch_small_t<4, 2>(p, st);
         return launch_small_t<4, 4>(p, st);
+    }
+    if (c.wbits == 2) {
+        if (tm == 1) return launch_small_t<2, 1>(p, st);
+        if (tm == 2) return launch_small_t<2, 2>(p, st);
+        return launch_small_t<2, 4>(p, st);
     }
     if (tm == 1) return launch_small_t<8, 1>(p, st);
     if (tm == 2) return launch_small_t<8, 2>(p, st);

@@ -160,6 +160,7 @@ class Workload:
 
 GLM_INT4 = LayerShape(6144, 2048, 256, 8, 4, 8, 1, 2.5, 4)
 GLM_INT8 = replace(GLM_INT4, wbits=8)
+GLM_INT2 = replace(GLM_INT4, wbits=2)
 TINY = LayerShape(256, 128, 16, 4, 2, 2, 1, 2.5, 8)
 
 WORKLOADS = {
@@ -172,6 +173,9 @@ WORKLOADS = {
     "glm52_decode_int4_t1_topp07": Workload(
         "glm52_decode_int4_t1_topp07", replace(GLM_INT4, topp=0.7), 1, 1,
         description="glm52_decode_int4_t1 with the adaptive expert top-p at 0.7 (the kept picks' shares reach 0.7)"),
+    "glm52_decode_int2_t1": Workload(
+        "glm52_decode_int2_t1", GLM_INT2, 1, 1,
+        description="glm52_decode_int4_t1 with packed int2 experts (codes -2..1, per-row scale amax/1): 9.46 MB per expert"),
     "glm52_verify_int4_t4": Workload(
         "glm52_verify_int4_t4", GLM_INT4, 4, 2, x_kind="correlated",
         description="GLM-5.2 shape, int4, 4 tokens (1 + 3 drafts) with 0.8-correlated activations"),

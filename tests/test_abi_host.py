@@ -62,10 +62,11 @@ def _cfg(L, **kw):
 
 
 @pytest.mark.parametrize("kw,status", [
-    ({"hidden": 6000}, -2), ({"inter": 100}, -2), ({"wbits": 3}, -2), ({"wbits": 2}, -2),
+    ({"hidden": 6000}, -2), ({"inter": 100}, -2), ({"wbits": 3}, -2), ({"wbits": 1}, -2),
     ({"n_groups": 7}, -1), ({"topk_groups": 9}, -1), ({"top_k": 129}, -1), ({"top_k": 33, "topk_groups": 8}, -2),
     ({"n_experts": 2048, "n_groups": 16}, -2), ({"n_shared": 2}, -2), ({"n_experts": 8, "n_groups": 8, "top_k": 2}, -2),
     ({"top_k": 0}, -1), ({"routed_scaling_factor": float("nan")}, -1),
+    ({"expert_topp": float("nan")}, -1), ({"expert_topp": -0.5}, -1), ({"expert_topp": float("inf")}, -1),
 ])
 def test_config_validation(L, kw, status):
     c = _cfg(L, **kw)
@@ -121,7 +122,7 @@ def test_other_entry_point_errors(L):
     assert lib.moe_pack_weights(0x1000, 4, 64, 3, 0x1000, 0x1000, None) == -2
     assert lib.moe_pack_weights(0x1004, 4, 64, 4, 0x1000, 0x1000, None) == -1
     assert lib.moe_block_dots(0x1000, 4, 48, 4, 0x1000, 1, 0x1000, None) == -1
-    assert lib.moe_block_dots(0x1000, 4, 64, 2, 0x1000, 1, 0x1000, None) == -2
+    assert lib.moe_block_dots(0x1000, 4, 64, 3, 0x1000, 1, 0x1000, None) == -2
     assert lib.moe_router_select(ctypes.byref(c), 0x1000, 4, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 16, None) == -3
     assert lib.moe_router_workspace_bytes(ctypes.byref(c), 4) >= 4 * 256 * 8
     assert lib.moe_synth_normal(1, 2, -1, 4, 1.0, 0x1000, None) == -1

@@ -17,7 +17,7 @@ from quantized_routed_expert_group_b200 import moe, synth
 pytestmark = pytest.mark.gpu
 
 FULL = ["glm52_decode_int4_t1", "glm52_verify_int4_t4", "glm52_int8_t16_outliers", "glm52_prefill_int4_t512_zipf",
-        "glm52_decode_int4_t1_topp07"]
+        "glm52_decode_int4_t1_topp07", "glm52_decode_int2_t1"]
 
 
 @pytest.fixture(scope="module", params=FULL)

@@ -21,6 +21,11 @@ FULLGROUPS = synth.LayerShape(256, 64, 16, 4, 2, 8, 1, 2.5, 4)   # top_k = every
 # groups of 32 experts (one warp per group in the fused selection), as in the GLM-5.2 shape
 GROUP32 = synth.LayerShape(512, 96, 128, 4, 2, 8, 1, 2.5, 4)
 GROUP32_K16 = synth.LayerShape(256, 64, 64, 2, 1, 16, 1, 1.0, 8)   # one kept group, top_k 16 of its 32
+# packed int2 experts: rows of 264 / 40 bytes (not 16-byte multiples) run the
+# multi-kernel path at every T; 1088 / 192 and 512 / 128 run the fused path
+MID2 = synth.LayerShape(1056, 160, 32, 4, 2, 4, 1, 2.5, 2)
+MID2F = synth.LayerShape(1088, 192, 32, 4, 2, 4, 1, 2.5, 2)
+GROUP32_INT2 = synth.LayerShape(512, 128, 128, 4, 2, 8, 1, 2.5, 2)
 # the adaptive expert top-p: picks past the share prefix that reaches topp are dropped
 MID4_TOPP = synth.LayerShape(1056, 160, 32, 4, 2, 4, 1, 2.5, 4, topp=0.5)
 MID8_TOPP = synth.LayerShape(1056, 160, 32, 4, 2, 4, 1, 1.0, 8, topp=0.7)
@@ -90,6 +95,10 @@ def test_tiny_host_entry_point(tiny):
     (MID4_TOPP, 37, 31, "normal"), (GROUP32_TOPP, 6, 32, "normal"),
     (MID4_TOPP, 3, 33, "normal"), (MID8_TOPP, 1, 34, "normal"), (GROUP32_TOPP, 1, 35, "normal"),
     (GROUP32_TOPP, 2, 36, "normal"), (GROUP32_TOPP, 4, 37, "correlated"), (GROUP32_K16_TOPP, 4, 38, "normal"),
+    # packed int2: multi-kernel path, then the fused path
+    (MID2, 37, 39, "normal"), (MID2, 3, 40, "normal"), (MID2F, 9, 41, "normal"),
+    (MID2F, 1, 42, "normal"), (MID2F, 2, 43, "normal"), (MID2F, 4, 44, "correlated"),
+    (GROUP32_INT2, 1, 45, "normal"), (GROUP32_INT2, 4, 46, "correlated"),
 ])
 def test_mid_layers(shape, T, seed, x_kind):
     wl = make_workload(f"mid_{shape.wbits}_{T}", shape, T, seed, x_kind=x_kind)

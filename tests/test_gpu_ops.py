@@ -53,7 +53,7 @@ def test_pack_weights_bitexact(wbits, rows, cols):
     np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
 
 
-@pytest.mark.parametrize("wbits", [8, 4])
+@pytest.mark.parametrize("wbits", [8, 4, 2])
 @pytest.mark.parametrize("rows,cols,n", [(64, 6144, 1), (33, 1056, 5), (200, 2048, 3)])
 def test_block_dots_bitexact(wbits, rows, cols, n):
     rng = np.random.default_rng(rows + cols + wbits)

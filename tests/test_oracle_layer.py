@@ -39,7 +39,7 @@ def test_block_dots_bruteforce(orc, wbits):
     np.testing.assert_array_equal(got, ref)
 
 
-@pytest.mark.parametrize("wbits", [8, 4])
+@pytest.mark.parametrize("wbits", [8, 4, 2])
 def test_qmatvec_is_dequantised_dot(orc, wbits):
     """s * sum_b d_b * isum_b equals sum_i (s q_w,i)(d_b q_x,i) (fp64), rounded once to fp32."""
     rng = np.random.default_rng(20 + wbits)
