@@ -237,7 +237,7 @@ int moe_workspace_view(const moe_config *cfg, int T, void *workspace, size_t ws_
 /* Per-block int32 dot products of one packed matrix with Q8_0 codes, computed
  * by the same device routine as the expert kernels ([GN] integer-dot kernel):
  * out[t][r][b] = sum_{i<32} code(W[r, 32b+i]) * q[t, 32b+i] for W packed
- * [rows][cols * wbits / 8] (wbits 8 or 4) and q [n][cols] int8. */
+ * [rows][cols * wbits / 8] (wbits 8, 4 or 2) and q [n][cols] int8. */
 int moe_block_dots(const uint8_t *packed, int64_t rows, int cols, int wbits, const int8_t *q, int n,
                    int32_t *out, void *stream);
 
