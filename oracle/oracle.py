@@ -68,6 +68,8 @@ def lib():
             "orc_layer_forward_topp": [_int, _int, _int, _int, _int, _int, _int, _flt, _int, _flt,
                                        _vp, _int, _vp, _vp, ctypes.POINTER(_OrcExpert),
                                        ctypes.POINTER(_OrcExpert), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
+            "orc_fp8_e4m3_decode": [_vp, _i64, _vp],
+            "orc_requant_fp8": [_vp, _vp, _i64, _i64, _int, _int, _vp, _vp],
             "orc_num_threads": [],
             "orc_set_num_threads": [_int],
         }
@@ -181,6 +183,26 @@ def bucket(idx, n_experts: int):
     perm = np.empty(T * k, np.int32)
     _check(lib().orc_bucket(_p(idx), T, k, n_experts, _p(counts), _p(offsets), _p(perm)), "bucket")
     return counts, offsets, perm
+
+
+def fp8_e4m3_decode(codes):
+    codes = _c(codes, np.uint8)
+    out = np.empty(codes.shape, np.float32)
+    _check(lib().orc_fp8_e4m3_decode(_p(codes), codes.size, _p(out)), "fp8_e4m3_decode")
+    return out
+
+
+def requant_fp8(w8, block_scales, block: int, wbits: int):
+    """FP8 E4M3 [rows][cols] with [ceil(rows/block)][ceil(cols/block)] fp32
+    scales -> (packed [rows][cols*wbits/8], row scales [rows])."""
+    w8 = _c(w8, np.uint8)
+    block_scales = _c(block_scales, np.float32)
+    rows, cols = w8.shape
+    packed = np.empty((rows, cols * wbits // 8), np.uint8)
+    scales = np.empty(rows, np.float32)
+    _check(lib().orc_requant_fp8(_p(w8), _p(block_scales), rows, cols, block, wbits, _p(packed), _p(scales)),
+           "requant_fp8")
+    return packed, scales
 
 
 @dataclass
