@@ -21,6 +21,12 @@ ranks' times are max-reduced and value = tokens of all ranks / that time.
 
 --impl reference times the CPU oracle (plain C, fp64) on the host cores on a
 bounded sample of the same workload; on N > 1 only rank 0 runs it.
+
+Other workloads of the same layer: glm52_decode_int4_t1_topp07 (adaptive
+expert top-p 0.7), glm52_decode_int2_t1 (packed int2 experts),
+glm52_verify_int4_t4, glm52_int8_t16_outliers, glm52_prefill_int4_t512_zipf.
+--requant times the FP8 -> int4 requantiser (the converter step) on 16
+experts of the GLM-5.2 shape instead, and prints its own JSON line (GB/s).
 """
 from __future__ import annotations
 
@@ -87,11 +93,19 @@ def gateup_bytes(shape) -> int:
     return 2 * shape.matrix_bytes(shape.inter, shape.hidden) + 2 * 4 * shape.inter
 
 
-def kernel_sources_sha() -> str:
+# The files each measured kernel's device code is compiled from: a committed
+# ncu traffic record of that kernel stays valid while these are unchanged.
+KERNEL_SOURCES = {
+    "k_moe_small": ["moe_small.cu", "moe_device.cuh", "moe_ptx.cuh"],
+    "k_gateup": ["moe_expert.cu", "moe_device.cuh", "moe_ptx.cuh"],
+}
+
+
+def kernel_sources_sha(kernel: str = "k_moe_small") -> str:
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "quantized_routed_expert_group_b200", "csrc", "*"))):
-        with open(f, "rb") as fh:
-            h.update(os.path.basename(f).encode())
+    for name in sorted(KERNEL_SOURCES[kernel]):
+        with open(os.path.join(ROOT, "quantized_routed_expert_group_b200", "csrc", name), "rb") as fh:
+            h.update(name.encode())
             h.update(fh.read())
     return h.hexdigest()[:16]
 
@@ -107,7 +121,7 @@ def ncu_traffic(kernel: str, workload: str) -> float | None:
         return None
     for row in doc.get("kernels", []):
         if row.get("kernel") == kernel and row.get("workload") == workload and \
-                row.get("sources_sha") == kernel_sources_sha():
+                row.get("sources_sha") == kernel_sources_sha(kernel):
             return float(row["dram_bytes_per_launch"])
     return None
 
@@ -157,6 +171,9 @@ def parse_clock_samples(text: str) -> dict | None:
 # ----------------------------------------------------------------------------
 # our implementation
 # ----------------------------------------------------------------------------
+REQUANT_EXPERTS = 16
+
+
 def run_ours(args) -> dict | None:
     import torch
     import torch.distributed as dist
@@ -372,6 +389,95 @@ def run_reference(args) -> dict | None:
     }
 
 
+def run_requant(args) -> dict:
+    """The converter step on the GPU: FP8 E4M3 expert weights with 128 x 128
+    block scales (seeded, resident in HBM, more than L2) requantised into the
+    engine's packed int4 per-row container.  One step = the gate/up rows of
+    REQUANT_EXPERTS experts of the GLM-5.2 shape, then their down rows (two
+    launches).  Reports the bytes the step must move (FP8 codes and block
+    scales in, packed codes and row scales out) per second."""
+    import torch
+    from quantized_routed_expert_group_b200 import moe, synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    s, block, wbits, n_exp = synth.GLM_INT4, 128, 4, REQUANT_EXPERTS
+    gen = torch.Generator(device=dev).manual_seed(2026)
+
+    def fp8_codes(rows, cols):
+        c = torch.randint(0, 256, (rows, cols), dtype=torch.uint8, device=dev, generator=gen)
+        c[(c & 0x7F) == 0x7F] = 0x3A  # no NaN codes
+        return c
+
+    def block_scales(rows, cols):
+        nb = (-(-rows // block), -(-cols // block))
+        return torch.rand(nb, device=dev, generator=gen) * 1e-3 + 1e-4
+
+    mats = [(fp8_codes(n_exp * 2 * s.inter, s.hidden), None), (fp8_codes(n_exp * s.hidden, s.inter), None)]
+    mats = [(w8, block_scales(*w8.shape)) for w8, _ in mats]
+    outs = [(torch.empty((w8.shape[0], w8.shape[1] * wbits // 8), dtype=torch.uint8, device=dev),
+             torch.empty(w8.shape[0], dtype=torch.float32, device=dev)) for w8, _ in mats]
+    step_bytes = sum(w8.numel() + bs.numel() * 4 + p.numel() + sc.numel() * 4
+                     for (w8, bs), (p, sc) in zip(mats, outs))
+
+    def step():
+        for (w8, bs), (p, sc) in zip(mats, outs):
+            moe.requant_fp8(w8, bs, block, wbits, p, sc)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    K = min(args.steps, 200)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    gpu_uuid = None
+    try:
+        gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        if not gpu_uuid.startswith("GPU-"):
+            gpu_uuid = "GPU-" + gpu_uuid
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_uuid)
+    time.sleep(0.15)
+    for a, b in ev:
+        a.record()
+        step()
+        b.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    gbs = step_bytes / (ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peak_hbm()
+    res = {
+        "metric": "FP8 E4M3 (128x128 block scales) -> packed int4 per-row requantisation, bytes moved per second",
+        "value": round(gbs, 1), "unit": "GB/s", "n_gpus": 1, "steps": K, "warmup": args.warmup,
+        "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8-e4m3 -> int4", "data": "synthetic (seeded FP8 codes and block scales)",
+        "config": {"workload": f"requant_fp8_int4_glm52_{n_exp}experts", "experts": n_exp, "hidden": s.hidden,
+                   "inter": s.inter, "block": block, "bytes_per_step": step_bytes,
+                   "l2": "not flushed: each step moves more than L2"},
+        "roofline": {"kernel": "k_pack_rows<4,RowsFp8Block>", "bound": "hbm", "achieved": round(gbs, 1),
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(gbs / peak, 4),
+                     "algorithmic_bytes_per_launch": step_bytes // 2, "traffic": None},
+        "gpu_launches": 2 * K,
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline:
+        from oracle import oracle as orc
+        import numpy as np
+        rows = 512
+        w8 = mats[0][0][:rows].cpu().numpy()
+        bs = mats[0][1][: -(-rows // block)].cpu().numpy()
+        t0 = time.perf_counter()
+        n = 0
+        while time.perf_counter() - t0 < 5.0:
+            orc.requant_fp8(w8, bs, block, wbits)
+            n += 1
+        dt = time.perf_counter() - t0
+        moved = n * (w8.size + bs.size * 4 + w8.size * wbits // 8 + rows * 4)
+        res["cpu_baseline"] = {"value": round(moved / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                               "sample": f"{n} x {rows} gate rows (6144 FP8 codes each) of the same input, {dt:.1f} s"}
+    return res
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -381,9 +487,14 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--flush-l2", action="store_true", help="write 2x L2 before every timed step")
+    ap.add_argument("--requant", action="store_true",
+                    help="time the FP8 -> int4 requantiser (the converter step) instead of the layer")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.requant:
+        print(json.dumps(run_requant(args)), flush=True)
+        return
     if args.impl == "reference":
         res = run_reference(args)
     else:

@@ -115,6 +115,21 @@ int moe_quantize_act_q8_0(const float *x, int64_t n_rows, int cols, int8_t *q, f
 int moe_pack_weights(const float *w, int64_t rows, int cols, int wbits, uint8_t *packed, float *scales,
                      void *stream);
 
+/* FP8 checkpoint requantiser (the offline converter's step: [GN] §구현된 주요
+ * 기능, offline converter bullet; [WP] converter list: the FP8 checkpoint is
+ * dequantised with its 128 x 128 block scales and requantised into the
+ * engine's per-row container).  w_fp8 [rows][cols] holds FP8 E4M3 codes (1
+ * sign, 4 exponent bits with bias 7, 3 mantissa bits; exponent 0 subnormal;
+ * S.1111.111 NaN; no infinities), block_scales [ceil(rows/block)]
+ * [ceil(cols/block)] fp32 row-major; each value is code * scale of its block
+ * (one fp32 multiply), and the dequantised rows are quantised and packed
+ * exactly as moe_pack_weights does.  cols a multiple of 32, block a multiple
+ * of 32 (128 in the checkpoint); w_fp8 and scale pointers 4-byte aligned,
+ * packed 16-byte aligned.  NaN codes give unspecified codes for their row.
+ * Device pointers; asynchronous on stream. */
+int moe_requant_fp8(const uint8_t *w_fp8, const float *block_scales, int64_t rows, int cols, int block, int wbits,
+                    uint8_t *packed, float *scales, void *stream);
+
 /* Bytes of device workspace that moe_router_select needs for T tokens. */
 size_t moe_router_workspace_bytes(const moe_config *cfg, int T);
 

@@ -228,6 +228,18 @@ MOE_API int moe_pack_weights(const float* w, int64_t rows, int cols, int wbits, 
     return status_of(launch_pack_weights(w, rows, cols, wbits, packed, scales, (cudaStream_t)stream));
 }
 
+MOE_API int moe_requant_fp8(const uint8_t* w_fp8, const float* block_scales, int64_t rows, int cols, int block,
+                            int wbits, uint8_t* packed, float* scales, void* stream) {
+    if (rows < 0 || cols <= 0 || cols % 32 || block <= 0 || block % 32) return MOE_EINVAL;
+    if (wbits != 8 && wbits != 4 && wbits != 2) return MOE_EUNSUPPORTED;
+    if (rows == 0) return MOE_OK;
+    if (!w_fp8 || !block_scales || !packed || !scales || !aligned(w_fp8, 4) || !aligned(block_scales, 4) ||
+        !aligned(packed, 16) || !aligned(scales, 4))
+        return MOE_EINVAL;
+    return status_of(
+        launch_requant_fp8(w_fp8, block_scales, rows, cols, block, wbits, packed, scales, (cudaStream_t)stream));
+}
+
 MOE_API size_t moe_router_workspace_bytes(const moe_config* cfg, int T) {
     if (check_config(cfg) != MOE_OK || T < 0) return 0;
     return align256((size_t)T * (size_t)cfg->n_experts * sizeof(double));

@@ -47,6 +47,8 @@ cudaError_t launch_quantize_q8_0(const float* x, int64_t n_rows, int cols, int8_
                                  cudaStream_t s);
 cudaError_t launch_pack_weights(const float* w, int64_t rows, int cols, int wbits, uint8_t* packed,
                                 float* scales, cudaStream_t s);
+cudaError_t launch_requant_fp8(const uint8_t* w8, const float* block_scales, int64_t rows, int cols, int block,
+                               int wbits, uint8_t* packed, float* scales, cudaStream_t s);
 cudaError_t launch_router(const moe_config& c, const float* x, int T, const float* router_w,
                           const float* bias, double* logits, int32_t* idx, float* w, cudaStream_t s);
 cudaError_t launch_bucket(const moe_config& c, const int32_t* idx, int T, int32_t* counts,

@@ -4,7 +4,9 @@
 // (integer-dot kernel with Q8_0-style int8 activations); wpnews.pro "Colibri —
 // รัน GLM-5.2 ...", kernel table.  Weight quantiser: same page, quantisation
 // kernel bullet (int8 / packed int4 / packed int2, per-row scales) and the
-// offline converter that requantises the FP8 checkpoint.
+// offline converter that dequantises the FP8 checkpoint with its 128 x 128
+// block scales and requantises it per row (same bullet list; wpnews.pro
+// converter list).
 #include "moe_device.cuh"
 #include "moe_internal.h"
 
@@ -34,11 +36,44 @@ cudaError_t launch_quantize_q8_0(const float* x, int64_t n_rows, int cols, int8_
     return cudaGetLastError();
 }
 
+// Row sources of the per-row quantiser: get(r, i) returns the fp32 values of
+// row r at columns i .. i+3 (i a multiple of 4).
+struct RowsF32 {  // plain fp32 rows [rows][cols]
+    const float* w;
+    int cols;
+    __device__ __forceinline__ float4 get(int64_t r, int i) const {
+        return *reinterpret_cast<const float4*>(w + r * cols + i);
+    }
+};
+
+// FP8 E4M3 value of one code, from the format: 1 sign bit, 4 exponent bits
+// with bias 7, 3 mantissa bits; exponent 0 is subnormal (m * 2^-9); S.1111.111
+// is NaN; there are no infinities.  A normal code maps to the fp32 with
+// exponent e - 7 + 127 and the 3 mantissa bits on top of its mantissa.
+__device__ __forceinline__ float fp8_e4m3_value(uint32_t b) {
+    const uint32_t e = (b >> 3) & 0xFu, m = b & 7u, sign = (b & 0x80u) << 24;
+    if (e == 15u && m == 7u) return __uint_as_float(0x7FC00000u);
+    if (e == 0u) return __uint_as_float(sign | __float_as_uint((float)m * 0.001953125f));
+    return __uint_as_float(sign | ((e + 120u) << 23) | (m << 20));
+}
+
+struct RowsFp8Block {  // FP8 E4M3 rows [rows][cols] times their block scales
+    const uint8_t* w8;
+    const float* bs;  // [ceil(rows/block)][nbc]
+    int cols, block, nbc;
+    __device__ __forceinline__ float4 get(int64_t r, int i) const {
+        const uint32_t b4 = *reinterpret_cast<const uint32_t*>(w8 + r * cols + i);
+        const float sc = bs[(r / block) * nbc + i / block];  // block % 4 == 0: one block for the four
+        return make_float4(__fmul_rn(fp8_e4m3_value(b4 & 0xFFu), sc), __fmul_rn(fp8_e4m3_value((b4 >> 8) & 0xFFu), sc),
+                           __fmul_rn(fp8_e4m3_value((b4 >> 16) & 0xFFu), sc), __fmul_rn(fp8_e4m3_value(b4 >> 24), sc));
+    }
+};
+
 // Per-row quantiser: one CTA per row.  s = amax / qmax, code =
 // round-half-away(w * (1/s)) clamped to [-2^(b-1), qmax], packed two's
 // complement with the lowest element in the lowest bits.
-template <int WBITS>
-__global__ void __launch_bounds__(256) k_pack_rows(const float* __restrict__ w, int64_t rows, int cols,
+template <int WBITS, class Rows>
+__global__ void __launch_bounds__(256) k_pack_rows(const Rows src, int64_t rows, int cols,
                                                    uint8_t* __restrict__ packed, float* __restrict__ scales) {
     constexpr int qmax = WBITS == 8 ? 127 : WBITS == 4 ? 7 : 1;
     constexpr float qminf = -(float)(1 << (WBITS - 1));
@@ -46,10 +81,9 @@ __global__ void __launch_bounds__(256) k_pack_rows(const float* __restrict__ w, 
     __shared__ float s_is[2];
     const int64_t row_bytes = (int64_t)cols * WBITS / 8;
     for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-        const float* wr = w + r * cols;
         float a = 0.0f;
         for (int i = threadIdx.x * 4; i < cols; i += blockDim.x * 4) {
-            const float4 v = *reinterpret_cast<const float4*>(wr + i);
+            const float4 v = src.get(r, i);
             a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
         }
 #pragma unroll
@@ -76,7 +110,7 @@ __global__ void __launch_bounds__(256) k_pack_rows(const float* __restrict__ w, 
             int codes[32];
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
-                const float4 v = *reinterpret_cast<const float4*>(wr + 32 * g + i);
+                const float4 v = src.get(r, 32 * g + i);
                 const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
@@ -124,9 +158,21 @@ cudaError_t launch_pack_weights(const float* w, int64_t rows, int cols, int wbit
                                 float* scales, cudaStream_t s) {
     if (rows == 0) return cudaSuccess;
     const int grid = (int)(rows < 1048576 ? rows : 1048576);
-    if (wbits == 8) k_pack_rows<8><<<grid, 256, 0, s>>>(w, rows, cols, packed, scales);
-    else if (wbits == 4) k_pack_rows<4><<<grid, 256, 0, s>>>(w, rows, cols, packed, scales);
-    else k_pack_rows<2><<<grid, 256, 0, s>>>(w, rows, cols, packed, scales);
+    const RowsF32 src{w, cols};
+    if (wbits == 8) k_pack_rows<8><<<grid, 256, 0, s>>>(src, rows, cols, packed, scales);
+    else if (wbits == 4) k_pack_rows<4><<<grid, 256, 0, s>>>(src, rows, cols, packed, scales);
+    else k_pack_rows<2><<<grid, 256, 0, s>>>(src, rows, cols, packed, scales);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_requant_fp8(const uint8_t* w8, const float* block_scales, int64_t rows, int cols, int block,
+                               int wbits, uint8_t* packed, float* scales, cudaStream_t s) {
+    if (rows == 0) return cudaSuccess;
+    const int grid = (int)(rows < 1048576 ? rows : 1048576);
+    const RowsFp8Block src{w8, block_scales, cols, block, (cols + block - 1) / block};
+    if (wbits == 8) k_pack_rows<8><<<grid, 256, 0, s>>>(src, rows, cols, packed, scales);
+    else if (wbits == 4) k_pack_rows<4><<<grid, 256, 0, s>>>(src, rows, cols, packed, scales);
+    else k_pack_rows<2><<<grid, 256, 0, s>>>(src, rows, cols, packed, scales);
     return cudaGetLastError();
 }
 

@@ -46,6 +46,7 @@ class MoeWorkspaceLayout(ctypes.Structure):
 _SIGS = {
     "moe_quantize_act_q8_0": ([_vp, _i64, _int, _vp, _vp, _vp], _int),
     "moe_pack_weights": ([_vp, _i64, _int, _int, _vp, _vp, _vp], _int),
+    "moe_requant_fp8": ([_vp, _vp, _i64, _int, _int, _int, _vp, _vp, _vp], _int),
     "moe_router_workspace_bytes": ([ctypes.POINTER(MoeConfig), _int], _sz),
     "moe_router_select": ([ctypes.POINTER(MoeConfig), _vp, _int, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _int),
     "moe_bucket_tokens": ([ctypes.POINTER(MoeConfig), _vp, _int, _vp, _vp, _vp, _vp], _int),
@@ -140,6 +141,22 @@ def pack_weights(w: torch.Tensor, wbits: int, packed: torch.Tensor | None = None
         scales = torch.empty(rows, dtype=torch.float32, device=w.device)
     _check(lib().moe_pack_weights(_ptr(w), rows, cols, wbits, _ptr(packed), _ptr(scales), _stream(stream)),
            "pack_weights")
+    return packed, scales
+
+
+def requant_fp8(w8: torch.Tensor, block_scales: torch.Tensor, block: int, wbits: int,
+                packed: torch.Tensor | None = None, scales: torch.Tensor | None = None, stream=None):
+    """FP8 E4M3 codes [rows][cols] (uint8) with fp32 block scales -> packed
+    codes [rows][cols*wbits/8] and fp32 row scales [rows]."""
+    _cuda(w8, torch.uint8, "w8")
+    _cuda(block_scales, torch.float32, "block_scales")
+    rows, cols = w8.shape
+    if packed is None:
+        packed = torch.empty((rows, cols * wbits // 8), dtype=torch.uint8, device=w8.device)
+    if scales is None:
+        scales = torch.empty(rows, dtype=torch.float32, device=w8.device)
+    _check(lib().moe_requant_fp8(_ptr(w8), _ptr(block_scales), rows, cols, block, wbits, _ptr(packed), _ptr(scales),
+                                 _stream(stream)), "requant_fp8")
     return packed, scales
 
 

@@ -123,6 +123,12 @@ def test_other_entry_point_errors(L):
     assert lib.moe_pack_weights(0x1004, 4, 64, 4, 0x1000, 0x1000, None) == -1
     assert lib.moe_block_dots(0x1000, 4, 48, 4, 0x1000, 1, 0x1000, None) == -1
     assert lib.moe_block_dots(0x1000, 4, 64, 3, 0x1000, 1, 0x1000, None) == -2
+    assert lib.moe_requant_fp8(0x1000, 0x1000, 4, 48, 128, 4, 0x1000, 0x1000, None) == -1   # cols % 32
+    assert lib.moe_requant_fp8(0x1000, 0x1000, 4, 64, 100, 4, 0x1000, 0x1000, None) == -1   # block % 32
+    assert lib.moe_requant_fp8(0x1000, 0x1000, 4, 64, 128, 3, 0x1000, 0x1000, None) == -2   # wbits
+    assert lib.moe_requant_fp8(0x1000, 0x1000, 0, 64, 128, 4, 0x1000, 0x1000, None) == 0    # nothing to do
+    assert lib.moe_requant_fp8(0x1000, 0x1000, 4, 64, 128, 4, 0x1004, 0x1000, None) == -1   # packed alignment
+    assert lib.moe_requant_fp8(None, 0x1000, 4, 64, 128, 4, 0x1000, 0x1000, None) == -1
     assert lib.moe_router_select(ctypes.byref(c), 0x1000, 4, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 16, None) == -3
     assert lib.moe_router_workspace_bytes(ctypes.byref(c), 4) >= 4 * 256 * 8
     assert lib.moe_synth_normal(1, 2, -1, 4, 1.0, 0x1000, None) == -1

@@ -118,3 +118,39 @@ def test_bucket_bitexact(T, k, E, drop):
     np.testing.assert_array_equal(counts.cpu().numpy(), co)
     np.testing.assert_array_equal(offsets.cpu().numpy(), oo)
     np.testing.assert_array_equal(perm.cpu().numpy(), po)
+
+
+def _fp8_case(rng, rows, cols, block):
+    w8 = rng.integers(0, 256, size=(rows, cols), dtype=np.uint8)
+    w8[(w8 & 0x7F) == 0x7F] = 0x3A  # no NaN codes
+    nb = (-(-rows // block), -(-cols // block))
+    bs = (np.exp2(rng.uniform(-12, -4, size=nb)) * rng.uniform(0.5, 1.0, size=nb)).astype(np.float32)
+    return w8, bs
+
+
+@pytest.mark.parametrize("wbits", [8, 4, 2])
+@pytest.mark.parametrize("rows,cols,block", [(2048, 6144, 128), (6144, 2048, 128), (200, 1056, 128), (37, 96, 32)])
+def test_requant_fp8_bitexact(wbits, rows, cols, block):
+    """The converter step: FP8 E4M3 with block scales -> packed codes and row
+    scales, bit-exact against the oracle (a full GLM-5.2 gate/up and down
+    matrix, a ragged last block, a block smaller than the checkpoint's)."""
+    rng = np.random.default_rng(rows + cols + wbits + block)
+    w8, bs = _fp8_case(rng, rows, cols, block)
+    packed, scales = moe.requant_fp8(torch.from_numpy(w8).cuda(), torch.from_numpy(bs).cuda(), block, wbits)
+    po, so = orc.requant_fp8(w8, bs, block, wbits)
+    np.testing.assert_array_equal(packed.cpu().numpy(), po)
+    np.testing.assert_array_equal(scales.cpu().numpy().view(np.uint32), so.view(np.uint32))
+
+
+def test_requant_fp8_every_code():
+    """Each of the 254 finite codes, one row per block scale of 1.0 and 2^-7:
+    the row scales and int8 codes agree with the oracle bit for bit."""
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
+    row = np.zeros(256, np.uint8)
+    row[: len(codes)] = codes
+    w8 = np.tile(row, (256, 1))  # rows 0..127 in block row 0, rows 128..255 in block row 1
+    bs = np.array([[1.0, 1.0], [2.0 ** -7, 2.0 ** -7]], np.float32)
+    packed, scales = moe.requant_fp8(torch.from_numpy(np.ascontiguousarray(w8)).cuda(), torch.from_numpy(bs).cuda(), 128, 8)
+    po, so = orc.requant_fp8(w8, bs, 128, 8)
+    np.testing.assert_array_equal(packed.cpu().numpy(), po)
+    np.testing.assert_array_equal(scales.cpu().numpy().view(np.uint32), so.view(np.uint32))
