@@ -65,9 +65,11 @@ def _silu(v):
     return v / (1.0 + np.exp(-v))
 
 
-@pytest.mark.parametrize("name", ["tiny_h256_e16_int8_t4"])
-def test_expert_ffn_dequantised_fp64(orc, name):
-    wl = synth.WORKLOADS[name]
+@pytest.mark.parametrize("wbits", [8, 4, 2])
+def test_expert_ffn_dequantised_fp64(orc, wbits):
+    from dataclasses import replace
+    base = synth.WORKLOADS["tiny_h256_e16_int8_t4"]
+    wl = replace(base, shape=replace(base.shape, wbits=wbits))
     s = wl.shape
     x = synth.make_x(wl)
     (_, ex) = _tiny_expert(orc, wl, 3)
