@@ -4,6 +4,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "moe_internal.h"
 
 #define MOE_API extern "C" __attribute__((visibility("default")))
@@ -94,6 +96,16 @@ static int check_experts(const moe_experts* ex) {
 
 static int status_of(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ECUDA; }
 
+// NVTX range around the launches of one forward phase, so that a profiler
+// can select a phase's kernels (ncu --nvtx --nvtx-include "moe/fused/").
+// Without an attached tool the calls return at once.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 // Per-thread tracing events (see moe_profile_events).
 static thread_local cudaEvent_t g_trace[MOE_PROFILE_MAX_EVENTS];
 static thread_local bool g_trace_on = false;
@@ -125,6 +137,7 @@ static int forward_device(const moe_config& c, const float* x, int T, const floa
     int32_t* inv_perm = reinterpret_cast<int32_t*>(ws + L.inv_perm);
     int32_t* active = reinterpret_cast<int32_t*>(ws + L.active);
     if (small_path_supported(c, T)) {
+        const NvtxRange range("moe/fused");
         SmallArgs a;
         a.cfg = &c;
         a.T = T;
@@ -155,6 +168,7 @@ static int forward_device(const moe_config& c, const float* x, int T, const floa
         if (!st2) st2 = status_of(trace(1, s));
         return st2;
     }
+    const NvtxRange range("moe/multi_kernel");
     if (trace(0, s) != cudaSuccess) return MOE_ECUDA;
     if (cudaMemsetAsync(err, 0, 64, s) != cudaSuccess) return MOE_ECUDA;
     int st = status_of(launch_quantize_q8_0(x, T, c.hidden, xq, xd, s));
