@@ -147,3 +147,20 @@ def test_forward_paths_and_phases(L):
     big = _cfg(L, n_experts=512, n_groups=16)   # beyond the fused path's 256 experts
     assert L.forward_phases(big, 1) == ["route", "bucket", "gate_up", "down", "combine"]
     assert L.lib().moe_profile_events(None, 3) == -1
+
+
+@pytest.mark.parametrize("shape,T,fused", [
+    (synth.GLM_INT4, 1, True), (synth.GLM_INT4, 4, True), (synth.GLM_INT4, 5, False),
+    (synth.GLM_INT8, 4, True), (synth.GLM_INT2, 1, True),
+    # int2 rows of 264 / 40 bytes are not 16-byte multiples: the multi-kernel path
+    (synth.LayerShape(1056, 160, 32, 4, 2, 4, 1, 2.5, 2), 3, False),
+    (synth.LayerShape(1088, 192, 32, 4, 2, 4, 1, 2.5, 2), 4, True),
+    (synth.LayerShape(1056, 160, 32, 4, 2, 4, 1, 2.5, 4), 4, True),
+])
+def test_path_selection(L, shape, T, fused):
+    """Which path a forward takes (host logic, the device's sizes defaulting to
+    a B200's 148 SMs and 227 KB of shared memory per block without a GPU)."""
+    c = L.config(shape)
+    phases = L.forward_phases(c, T)
+    assert (phases == ["fused"]) == fused, phases
+    assert L.forward_launches(c, T) == (2 if fused else 7)
