@@ -5,15 +5,18 @@
 
 A step is one forward of the whole layer (Q8_0 of x, router, bucketing, expert
 gate/up + SiLU + Q8_0 of h, expert down, combine) over one batch of the
-workload's tokens, with all weights resident in HBM.  Every step streams the
-selected experts' weights (170 MB at one token, more at more tokens) with
-evict-first L2 hints, more than the 126 MB L2 holds, so each step reads them
-from HBM without an explicit flush; --flush-l2 also writes twice the L2 size
-before every step (this evicts the kernel's own instructions as well), and the
-JSON line carries that variant's step time too.  Each step is timed on the
-device with CUDA events recorded by the library at its phase boundaries; the
-phase events also give the live duration of the dominant kernel for the
-roofline.
+workload's tokens, with all weights resident in HBM.  The timed steps cycle
+through seeded token batches (64 for decode-sized batches, 8 for larger ones),
+so consecutive steps select different experts and every step streams its
+experts' weights (170 MB at one token, more at more tokens: more than the
+126 MB L2) from HBM.  The JSON line also reports the same batch repeated
+(fixed_batch) and the same batch with L2 flushed before every step
+(l2_flushed: 2x L2 written; this evicts the kernels' instructions too).  Each
+step is timed on the device with CUDA events recorded by the library at its
+phase boundaries; the phase events also give the live duration of the
+dominant kernel for the roofline (the fused kernel at T <= 4, the gate/up
+GEMV at 5 <= T < 64, the gate/up tensor-core GEMM at T >= 64, for which the
+int8 tensor utilisation is reported as well).
 
 N > 1: one process per GPU (torchrun); each rank runs an independent replica of
 the layer on its own tokens (the layer forward has no exchange step), the
@@ -98,6 +101,7 @@ def gateup_bytes(shape) -> int:
 KERNEL_SOURCES = {
     "k_moe_small": ["moe_small.cu", "moe_device.cuh", "moe_ptx.cuh"],
     "k_gateup": ["moe_expert.cu", "moe_device.cuh", "moe_ptx.cuh"],
+    "k_tc_gemm": ["moe_tc.cu", "moe_tc.cuh", "moe_device.cuh", "moe_ptx.cuh"],
 }
 
 
@@ -174,6 +178,34 @@ def parse_clock_samples(text: str) -> dict | None:
 REQUANT_EXPERTS = 16
 
 
+ROTATIONS_SMALL, ROTATIONS_LARGE = 64, 8  # seeded token batches the timed steps cycle through
+TENSOR_I8_NOMINAL_RATIO = 2.0             # dense int8 / dense bf16 tensor throughput (nominal)
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def measured_peak_bf16() -> tuple[float, str]:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            v = float(json.load(f)["bf16_tflops"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def rotating_workloads(wl, rank: int, n: int):
+    """n seeded token batches of the workload (same shapes and value recipe,
+    different seeds); rank r of a multi-GPU run gets its own."""
+    from quantized_routed_expert_group_b200 import synth
+    return [synth.Workload(wl.name, wl.shape, wl.T, wl.seed + 7919 * rank + 104729 * (i + 1), wl.x_kind,
+                           wl.bias_kind) for i in range(n)]
+
+
+def step_stats(ms: list[float]) -> dict:
+    return {"median": round(statistics.median(ms), 5), "mean": round(statistics.mean(ms), 5),
+            "min": round(min(ms), 5), "max": round(max(ms), 5)}
+
+
 def run_ours(args) -> dict | None:
     import torch
     import torch.distributed as dist
@@ -188,22 +220,20 @@ def run_ours(args) -> dict | None:
     dev = torch.device("cuda", local)
     wl = synth.WORKLOADS[args.workload]
     s = wl.shape
-    # replicas: same weights, each rank its own tokens
-    wl_x = synth.Workload(wl.name, s, wl.T, wl.seed + 7919 * rank, wl.x_kind, wl.bias_kind)
+    # replicas: same weights, each rank its own tokens; the timed steps cycle
+    # through R seeded batches so that no step finds the previous step's
+    # experts in L2 (every step streams more weight bytes than L2 holds)
+    R = ROTATIONS_SMALL if wl.T <= 16 else ROTATIONS_LARGE
     layer = moe.synth_layer(wl, dev)
-    x = torch.from_numpy(synth.make_x(wl_x)).to(dev)
-    out = torch.empty_like(x)
+    xs = [torch.from_numpy(synth.make_x(w)).to(dev) for w in rotating_workloads(wl, rank, R)]
+    out = torch.empty_like(xs[0])
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
 
-    # warm-up
     for i in range(args.warmup):
-        if args.flush_l2:
-            flush.fill_(i & 0xFF)
-        layer.forward(x, out)
+        layer.forward(xs[i % R], out)
     torch.cuda.synchronize()
     assert layer.device_error() == 0
-    n_active = int((layer.view(wl.T)["counts"] > 0).sum().item())
 
     K = args.steps
     phases = moe.forward_phases(layer.cfg, wl.T)
@@ -225,67 +255,90 @@ def run_ours(args) -> dict | None:
     sampler = ClockSampler(gpu_uuid)
     time.sleep(0.15)
     for i in range(K):
-        if args.flush_l2:
-            flush.fill_(i & 0xFF)
         moe.profile_events(evs[i])
-        layer.forward(x, out)
+        layer.forward(xs[i % R], out)
     moe.profile_events(None)
     torch.cuda.synchronize()
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
     step_ms = [evs[i][0].elapsed_time(evs[i][P]) for i in range(K)]
-    # the same steps with L2 flushed before each (reported alongside)
-    K_fl = min(K, 200)
-    evf = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_fl)]
-    for row in evf:
-        for ev in row:
-            ev.record()
-    torch.cuda.synchronize()
-    for i in range(K_fl):
-        flush.fill_(i & 0xFF)
-        evf[i][0].record()
-        layer.forward(x, out)
-        evf[i][1].record()
-    torch.cuda.synchronize()
-    flushed_ms = statistics.mean(evf[i][0].elapsed_time(evf[i][1]) for i in range(K_fl))
     phase_ms = [[evs[i][p].elapsed_time(evs[i][p + 1]) for i in range(K)] for p in range(P)]
     total_ms = sum(step_ms)
     max_total = reduce_max(total_ms, dev)
     value = throughput(wl.T, K, world, max_total)
+    # active experts of each rotation (the bytes a step streams)
+    n_active = []
+    for i in range(R):
+        layer.forward(xs[i], out)
+        n_active.append(int((layer.view(wl.T)["counts"] > 0).sum().item()))
+    torch.cuda.synchronize()
+
+    # variants, reported alongside: the same batch every step (no flush), and
+    # the same batch with L2 flushed (2x its size written) before every step
+    K_v = min(K, 200)
+
+    def timed(flush_l2: bool) -> list[float]:
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_v)]
+        for row in ev:
+            for e in row:
+                e.record()
+        torch.cuda.synchronize()
+        for i in range(K_v):
+            if flush_l2:
+                flush.fill_(i & 0xFF)
+            ev[i][0].record()
+            layer.forward(xs[0], out)
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        return [ev[i][0].elapsed_time(ev[i][1]) for i in range(K_v)]
+
+    fixed_ms = timed(False)
+    flushed_ms = timed(True)
 
     # end to end through the host-buffer entry point (pinned host x / out)
     K_e2e = max(1, min(K, 200))
-    xh = x.cpu().pin_memory()
-    oh = torch.empty_like(xh).pin_memory()
+    xh = [x.cpu().pin_memory() for x in xs]
+    oh = torch.empty_like(xh[0]).pin_memory()
     e2e_s = 0.0
     for i in range(K_e2e):
-        if args.flush_l2:
-            flush.fill_(i & 0xFF)
         torch.cuda.synchronize()
         t0 = time.perf_counter()
-        layer.forward_host(xh, oh)
+        layer.forward_host(xh[i % R], oh)
         e2e_s += time.perf_counter() - t0
     e2e_max = reduce_max(e2e_s * 1e3, dev)
     e2e_value = throughput(wl.T, K_e2e, world, e2e_max)
 
-    # roofline of the dominant phase's kernel: the fused kernel (whole layer)
-    # on the small-batch path, the gate/up GEMV on the multi-kernel path
     peak, peak_kind = measured_peak_hbm()
     router_bytes = s.n_experts * s.hidden * 4
-    layer_bytes = (n_active + s.n_shared) * expert_bytes(s)
+    mean_active = statistics.mean(n_active)
+    layer_bytes = (mean_active + s.n_shared) * expert_bytes(s)
+    ms_step = statistics.mean(step_ms)
+    layer_gbs = layer_bytes / (ms_step * 1e-3) / 1e9
+    tensor = None
     if phases == ["fused"]:
         # the fused phase: the prologue (Q8_0 of x, router logits over the
-        # router weights) and the persistent kernel (the experts), which run
-        # overlapped; bytes and ncu traffic cover both
+        # router weights) and the persistent kernel (the experts); bytes and
+        # ncu traffic cover both
         dom_kernel, dom_ms = "k_moe_small", statistics.mean(phase_ms[0])
         dom_bytes = layer_bytes + router_bytes
     else:
-        dom_kernel, dom_ms = "k_gateup", statistics.mean(phase_ms[phases.index("gate_up")])
-        dom_bytes = (n_active + s.n_shared) * gateup_bytes(s)
+        gu_ms = statistics.mean(phase_ms[phases.index("gate_up")])
+        dom_bytes = (mean_active + s.n_shared) * gateup_bytes(s)
+        dom_ms = gu_ms
+        if moe.forward_launches(layer.cfg, wl.T) == moe.TC_LAUNCHES:
+            dom_kernel = "k_tc_gemm"
+            # int8 tensor work of the gate/up GEMM: 2 ops per MAC, gate and up
+            ops = 2.0 * 2.0 * (wl.T * s.top_k + wl.T * s.n_shared) * s.hidden * s.inter
+            bf16, bf16_kind = measured_peak_bf16()
+            i8_peak = bf16 * TENSOR_I8_NOMINAL_RATIO
+            tops = ops / (gu_ms * 1e-3) / 1e12
+            tensor = {"kernel": "k_tc_gemm (gate/up)", "int8_ops": ops, "achieved_tops": round(tops, 1),
+                      "peak_tops": i8_peak, "peak_kind": f"{bf16_kind} bf16 x {TENSOR_I8_NOMINAL_RATIO:g} (nominal int8/bf16)",
+                      "frac": round(tops / i8_peak, 4)}
+        else:
+            dom_kernel = "k_gateup"
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
-    ms_step = statistics.mean(step_ms)
-    layer_gbs = layer_bytes / (ms_step * 1e-3) / 1e9
     if rank != 0:
         return None
     res = {
@@ -294,24 +347,29 @@ def run_ours(args) -> dict | None:
         "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded; random-init weights of the layer's shape)",
         "config": {"workload": wl.name, "tokens": wl.T, "hidden": s.hidden, "inter": s.inter,
                    "experts": s.n_experts, "top_k": s.top_k, "shared": s.n_shared, "weights": f"int{s.wbits}",
-                   "activations": "Q8_0 int8", "unique_experts_per_step": n_active,
-                   "l2": ("flushed before every step (write of 2x L2)" if args.flush_l2 else
-                          "not flushed: each step streams the selected experts' weights (> L2) with evict-first hints"),
+                   "activations": "Q8_0 int8", "unique_experts_per_step": round(mean_active, 2),
+                   "token_batches": f"{R} seeded batches, step i uses batch i mod {R}",
+                   "l2": ("not flushed: every step streams its selected experts' weights, more than L2 holds, "
+                          "and consecutive steps select different experts"),
                    "parallelism": f"replicas x{world}"},
-        "layer_hbm": {"algorithmic_bytes": layer_bytes, "gbs": round(layer_gbs, 1),
+        "step_ms": step_stats(step_ms),
+        "layer_hbm": {"algorithmic_bytes": int(layer_bytes), "gbs": round(layer_gbs, 1),
                       "frac_measured": round(layer_gbs / peak, 4), "frac_spec_8tbs": round(layer_gbs / SPEC_HBM_GBS, 4)},
         "phases_ms": {n: round(statistics.mean(v), 5) for n, v in zip(phases, phase_ms)},
-        "l2_flushed": {"steps": K_fl, "ms_per_step": round(flushed_ms, 5),
-                       "value": round(throughput(wl.T, K_fl, 1, flushed_ms * K_fl), 3), "unit": "tokens/s"},
+        "fixed_batch": {"steps": K_v, "step_ms": step_stats(fixed_ms)},
+        "l2_flushed": {"steps": K_v, "step_ms": step_stats(flushed_ms),
+                       "value": round(throughput(wl.T, K_v, 1, sum(flushed_ms)), 3), "unit": "tokens/s"},
         "roofline": {"kernel": dom_kernel, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "algorithmic_bytes_per_launch": dom_bytes,
+                     "algorithmic_bytes_per_launch": int(dom_bytes),
                      "traffic": ncu_traffic(dom_kernel, wl.name)},
-        "e2e": {"value": round(e2e_value, 3), "unit": "tokens/s", "h2d_bytes_per_step": x.numel() * 4,
+        "e2e": {"value": round(e2e_value, 3), "unit": "tokens/s", "h2d_bytes_per_step": xs[0].numel() * 4,
                 "d2h_bytes_per_step": out.numel() * 4, "steps": K_e2e},
         "gpu_launches": K * moe.forward_launches(layer.cfg, wl.T),
         "clocks": clocks,
     }
+    if tensor is not None:
+        res["roofline"]["tensor"] = tensor
     return res
 
 
@@ -486,7 +544,6 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--flush-l2", action="store_true", help="write 2x L2 before every timed step")
     ap.add_argument("--requant", action="store_true",
                     help="time the FP8 -> int4 requantiser (the converter step) instead of the layer")
     args = ap.parse_args(argv)

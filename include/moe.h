@@ -31,7 +31,9 @@
  *  - Floating point: fp32 inputs and outputs; no fast-math anywhere.
  *  - Non-finite activations or weights give undefined (but memory-safe)
  *    results; the CPU test oracle rejects them.
- *  - Concurrent calls are safe as long as each has its own workspace.
+ *  - Concurrent calls are safe as long as each has its own workspace (the
+ *    fused small-batch kernel is a cooperative grid of one CTA per SM, so two
+ *    of them on different streams run one after the other).
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -160,8 +162,12 @@ int moe_router_select(const moe_config *cfg, const float *x, int T, const float 
  * sums, offsets[n_experts] = the number n of routed pairs, T*top_k unless
  * the top-p dropped some) and perm [T*top_k], where perm lists t*top_k + j
  * for expert 0's pairs in increasing t, then expert 1's, etc., and ends with
- * -1 for each dropped pair.  idx = -1 marks a dropped pair; any other value
- * outside [0, n_experts) records MOE_EDEVICE's index fault.
+ * -1 for each dropped pair.  idx = -1 marks a dropped pair.  This entry
+ * point has no error word, so it does not detect invalid input: an index
+ * outside [-1, n_experts) is treated like a dropped pair, and a token that
+ * lists the same expert twice gives colliding perm entries (moe_layer_forward
+ * never produces either; its own bucketing records the index fault in its
+ * workspace's error word).
  * Supports n_experts * ceil(T/32) <= 24576 (T <= 3072 at 256 experts). */
 int moe_bucket_tokens(const moe_config *cfg, const int32_t *idx, int T, int32_t *counts, int32_t *offsets,
                       int32_t *perm, void *stream);
@@ -221,10 +227,20 @@ int moe_layer_forward_host(const moe_config *cfg, const float *x_host, int T, co
  * contents; each call clears what must start at zero.  Calls whose executions
  * overlap on the GPU (different streams, or different host threads) race on
  * the array and give wrong results: serialise them.  The intermediates are not
- * reachable through moe_workspace_view or moe_get_device_error. */
+ * reachable through moe_workspace_view; the error word is read with
+ * moe_noalloc_device_error.  The looked-up address belongs to the device's
+ * context as it was at that first call: do not use this entry point after
+ * cudaDeviceReset (or anything else that re-creates the primary context) in
+ * the same process. */
 int moe_layer_forward_noalloc(const moe_config *cfg, const float *x, int T, const float *router_w,
                               const float *router_bias, const moe_experts *routed, const moe_experts *shared,
                               float *out, void *stream);
+
+/* moe_get_device_error for the allocation-free forward: synchronises `stream`
+ * and reads the error word that the last moe_layer_forward_noalloc on the
+ * current device left in the library's fixed scratch (codes as for
+ * moe_get_device_error; a later noalloc call on the device resets it). */
+int moe_noalloc_device_error(void *stream, int32_t *code);
 
 /* Device pointers to the intermediates a moe_layer_forward call leaves in its
  * workspace (valid after the call completes, until the next call on the same
@@ -256,11 +272,54 @@ int moe_workspace_view(const moe_config *cfg, int T, void *workspace, size_t ws_
 int moe_block_dots(const uint8_t *packed, int64_t rows, int cols, int wbits, const int8_t *q, int n,
                    int32_t *out, void *stream);
 
+/* The device routines that compute a block dot on the forward path; each
+ * kernel calls exactly one of them ([GN] integer-dot kernel bullet).
+ *  MOE_DOTS_MULTI_KERNEL: the multi-kernel path's k_gateup / k_down routine
+ *    (int8 dp4a; int4 nibbles shifted to the top of their byte, sum >> 4;
+ *    int2 fields shifted to the top over crumb-ordered codes, sum >> 6).
+ *    out = the dot.
+ *  MOE_DOTS_FUSED: the fused small-batch kernel's routine (int4: low nibbles
+ *    in excess-8 form with the excess removed through the starting value,
+ *    high nibbles as 16 * code; int2 as above without the final shift).
+ *    out = the dot times 16 (int4), 64 (int2) or 1 (int8), exactly: the
+ *    kernel folds that power of two into the activation scale.
+ *  MOE_DOTS_TENSOR: the batched path's tensor-core routine: the packed rows
+ *    widened to int8 in shared memory, one tcgen05.mma kind::i8 (K = 32, one
+ *    Q8_0 block) per block into a TMEM accumulator, read back as int32.
+ *    out = the dot.  Needs n <= 64 and rows of a multiple of 16 bytes
+ *    (cols * wbits / 8), else MOE_EUNSUPPORTED. */
+enum { MOE_DOTS_MULTI_KERNEL = 0, MOE_DOTS_FUSED = 1, MOE_DOTS_TENSOR = 2 };
+
+/* moe_block_dots through the routine `routine` (one of MOE_DOTS_*; anything
+ * else returns MOE_EUNSUPPORTED).  Same arguments and layouts as
+ * moe_block_dots; every packed byte value (all 16 nibbles, all 4 int2 fields)
+ * and every int8 code is accepted. */
+int moe_block_dots_routine(const uint8_t *packed, int64_t rows, int cols, int wbits, const int8_t *q, int n,
+                           int routine, int32_t *out, void *stream);
+
 /* Synchronises `stream` and reads the workspace's device error word into
  * *code (0 = none).  Returns MOE_OK when it is 0, MOE_EDEVICE otherwise.
  * Codes: 1 = an index out of range reached a kernel, 2 = a device-side wait
- * ran out of iterations. */
+ * ran out of time.  Every wait inside a kernel is bounded by the GPU's
+ * global timer: a wait for a free pipeline slot or for another CTA's
+ * results gives up after 25 ms, a wait that can span one of those after
+ * 100 ms; the kernel then records code 2 and returns, leaving the call's
+ * outputs unspecified. */
 int moe_get_device_error(void *workspace, void *stream, int32_t *code);
+
+/* Test hook of the failure-detection tests (the pages have no counterpart).
+ * With withhold_entry >= 0, every following fused small-batch forward
+ * (T <= 4) issued by this process skips the publication of the h codes of
+ * gate/up unit 0 of entry withhold_entry (0 = the shared expert, 1 + a = the
+ * a-th selected routed expert in ascending id order), so the down projection's
+ * wait for them runs out: the forward still returns MOE_OK, its error word
+ * reads 2 and its output is unspecified.  wait_budget_ns > 0 replaces the
+ * 25 ms bound of the producer's waits (the longer waits scale with it);
+ * 0 restores it.  withhold_entry = -1 switches the fault off.  The setting is
+ * process-wide; set it only while no forward is being issued from another
+ * thread.  Returns MOE_EINVAL for withhold_entry < -1 or a budget outside
+ * [0, 10 s]. */
+int moe_debug_fault_injection(int withhold_entry, int64_t wait_budget_ns);
 
 /* Device copy of the seeded input generator (SplitMix64, counter-based; see
  * the package's synth module): out[i] = sigma * z(seed, tid, offset + i) with z

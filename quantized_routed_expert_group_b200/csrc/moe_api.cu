@@ -30,7 +30,7 @@ Layout make_layout(const moe_config& c, int T) {
     L.outbuf = take(t * H * 4);
     L.xq = take(t * H);
     L.xd = take(t * (H / 32) * 4);
-    L.logits = take(t * E * 8);
+    L.logits = take(router_ws_bytes(c, T));
     L.idx = take(t * k * 4);
     L.w = take(t * k * 4);
     L.counts = take(E * 4);
@@ -43,6 +43,23 @@ Layout make_layout(const moe_config& c, int T) {
     L.hq = take(slots * I);
     L.hd = take(slots * (I / 32) * 4);
     L.y = take(slots * H * 4);
+    if (tc_path_supported(c, T)) {
+        const TcSizes z = tc_sizes(c, T);
+        const size_t pr = (size_t)z.prows_cap;
+        L.tc_xg = take(pr * H);
+        L.tc_xdT = take((H / 32) * pr * 8);
+        L.tc_gu = take(2 * pr * I * 4);
+        L.tc_hg = take(pr * I);
+        L.tc_hdT = take((I / 32) * pr * 8);
+        L.tc_row_tok = take(pr * 4);
+        L.tc_row_slot = take(pr * 4);
+        L.tc_units_gu = take((size_t)z.units_gu_cap * kTcUnitBytes);
+        L.tc_units_dn = take((size_t)z.units_dn_cap * kTcUnitBytes);
+        L.tc_ctrl = take(64);
+    } else {
+        L.tc_xg = L.tc_xdT = L.tc_gu = L.tc_hg = L.tc_hdT = L.tc_row_tok = L.tc_row_slot = 0;
+        L.tc_units_gu = L.tc_units_dn = L.tc_ctrl = 0;
+    }
     L.total = off;
     return L;
 }
@@ -177,8 +194,22 @@ static int forward_device(const moe_config& c, const float* x, int T, const floa
     if (!st) st = status_of(trace(1, s));
     if (st) return st;
     st = status_of(launch_bucket(c, idx, T, counts, offsets, perm, inv_perm, active, err, s));
-    if (!st) st = status_of(trace(2, s));
     if (st) return st;
+    const bool tc = tc_path_supported(c, T);
+    TcArgs ta{};
+    if (tc) {
+        ta.xg = reinterpret_cast<int8_t*>(ws + L.tc_xg);
+        ta.xdT = reinterpret_cast<double*>(ws + L.tc_xdT);
+        ta.gu = reinterpret_cast<float*>(ws + L.tc_gu);
+        ta.hg = reinterpret_cast<int8_t*>(ws + L.tc_hg);
+        ta.hdT = reinterpret_cast<double*>(ws + L.tc_hdT);
+        ta.row_tok = reinterpret_cast<int32_t*>(ws + L.tc_row_tok);
+        ta.row_slot = reinterpret_cast<int32_t*>(ws + L.tc_row_slot);
+        ta.units_gu = ws + L.tc_units_gu;
+        ta.units_dn = ws + L.tc_units_dn;
+        ta.ctrl = reinterpret_cast<int32_t*>(ws + L.tc_ctrl);
+        ta.sz = tc_sizes(c, T);
+    }
     ExpertArgs a;
     a.cfg = &c;
     a.T = T;
@@ -196,6 +227,14 @@ static int forward_device(const moe_config& c, const float* x, int T, const floa
     a.y = reinterpret_cast<float*>(ws + L.y);
     a.out = out;
     a.err = err;
+    if (tc) {
+        ta.ex = a;
+        st = status_of(launch_tc_prepare(ta, s));
+        if (!st) st = status_of(trace(2, s));
+        if (st) return st;
+        return status_of(launch_tc_experts(ta, s, g_trace_on ? &g_trace[3] : nullptr));
+    }
+    if (trace(2, s) != cudaSuccess) return MOE_ECUDA;
     return status_of(launch_experts(a, s, g_trace_on ? &g_trace[3] : nullptr));
 }
 
@@ -255,8 +294,8 @@ MOE_API int moe_requant_fp8(const uint8_t* w_fp8, const float* block_scales, int
 }
 
 MOE_API size_t moe_router_workspace_bytes(const moe_config* cfg, int T) {
-    if (check_config(cfg) != MOE_OK || T < 0) return 0;
-    return align256((size_t)T * (size_t)cfg->n_experts * sizeof(double));
+    if (check_config(cfg) != MOE_OK || T < 0 || T > (1 << 20)) return 0;
+    return align256(router_ws_bytes(*cfg, T));
 }
 
 MOE_API int moe_router_select(const moe_config* cfg, const float* x, int T, const float* router_w,
@@ -288,6 +327,7 @@ MOE_API int moe_bucket_tokens(const moe_config* cfg, const int32_t* idx, int T, 
 
 MOE_API size_t moe_workspace_bytes(const moe_config* cfg, int T_max) {
     if (check_config(cfg) != MOE_OK || T_max < 0) return 0;
+    if (check_bucket_fits(*cfg, T_max) != MOE_OK) return 0;  // no forward runs that many tokens
     return make_layout(*cfg, T_max).total;
 }
 
@@ -330,6 +370,8 @@ MOE_API int moe_layer_forward_host(const moe_config* cfg, const float* x_host, i
 // array, so its device address is looked up with cudaGetSymbolAddress, once
 // per device, with that device current, and passed to the kernels.
 // ---------------------------------------------------------------------------
+MOE_API int moe_get_device_error(void* workspace, void* stream, int32_t* code);
+
 constexpr size_t kNoallocScratchBytes = (size_t)8 << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
@@ -362,6 +404,8 @@ MOE_API int moe_layer_forward_noalloc(const moe_config* cfg, const float* x, int
     int st = check_config(cfg);
     if (st) return st;
     if (T < 0) return MOE_EINVAL;
+    st = check_bucket_fits(*cfg, T);  // also keeps the layout arithmetic below in range
+    if (st) return st;
     if (make_layout(*cfg, T).total > kNoallocScratchBytes) return MOE_EWORKSPACE;
     void* scratch = noalloc_scratch_address(&st);
     if (st) return st;
@@ -375,11 +419,22 @@ MOE_API int moe_layer_forward_noalloc(const moe_config* cfg, const float* x, int
                           static_cast<char*>(scratch), L, (cudaStream_t)stream);
 }
 
+MOE_API int moe_noalloc_device_error(void* stream, int32_t* code) {
+    if (!code) return MOE_EINVAL;
+    int st = MOE_OK;
+    void* scratch = noalloc_scratch_address(&st);
+    if (st) return st;
+    // the error word is the first word of the layout, whatever the config
+    return moe_get_device_error(scratch, stream, code);
+}
+
 MOE_API int moe_workspace_view(const moe_config* cfg, int T, void* workspace, size_t ws_bytes,
                                moe_workspace_layout* view) {
     int st = check_config(cfg);
     if (st) return st;
     if (T < 0 || !workspace || !view) return MOE_EINVAL;
+    st = check_bucket_fits(*cfg, T);
+    if (st) return st;
     const Layout L = make_layout(*cfg, T);
     if (ws_bytes < L.total) return MOE_EWORKSPACE;
     char* ws = static_cast<char*>(workspace);
@@ -403,7 +458,23 @@ MOE_API int moe_block_dots(const uint8_t* packed, int64_t rows, int cols, int wb
     if (wbits != 4 && wbits != 8 && wbits != 2) return MOE_EUNSUPPORTED;
     if (rows == 0 || n == 0) return MOE_OK;
     if (!packed || !q || !out || !aligned(packed, 16) || !aligned(q, 16) || !aligned(out, 4)) return MOE_EINVAL;
-    return status_of(launch_block_dots(packed, rows, cols, wbits, q, n, out, (cudaStream_t)stream));
+    return status_of(launch_block_dots(packed, rows, cols, wbits, q, n, out, (cudaStream_t)stream,
+                                       MOE_DOTS_MULTI_KERNEL));
+}
+
+MOE_API int moe_block_dots_routine(const uint8_t* packed, int64_t rows, int cols, int wbits, const int8_t* q, int n,
+                                   int routine, int32_t* out, void* stream) {
+    if (routine != MOE_DOTS_MULTI_KERNEL && routine != MOE_DOTS_FUSED && routine != MOE_DOTS_TENSOR)
+        return MOE_EUNSUPPORTED;
+    if (rows < 0 || n < 0 || cols <= 0 || cols % 32) return MOE_EINVAL;
+    if (wbits != 4 && wbits != 8 && wbits != 2) return MOE_EUNSUPPORTED;
+    if (routine == MOE_DOTS_TENSOR && (n > 64 || ((int64_t)cols * wbits / 8) % 16 || rows > 0x7FFFFFFF))
+        return MOE_EUNSUPPORTED;
+    if (rows == 0 || n == 0) return MOE_OK;
+    if (!packed || !q || !out || !aligned(packed, 16) || !aligned(q, 16) || !aligned(out, 4)) return MOE_EINVAL;
+    if (routine == MOE_DOTS_TENSOR)
+        return status_of(launch_tc_block_dots(packed, rows, cols, wbits, q, n, out, (cudaStream_t)stream));
+    return status_of(launch_block_dots(packed, rows, cols, wbits, q, n, out, (cudaStream_t)stream, routine));
 }
 
 MOE_API int moe_get_device_error(void* workspace, void* stream, int32_t* code) {
@@ -414,6 +485,13 @@ MOE_API int moe_get_device_error(void* workspace, void* stream, int32_t* code) {
     if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ECUDA;
     *code = v;
     return v == 0 ? MOE_OK : MOE_EDEVICE;
+}
+
+MOE_API int moe_debug_fault_injection(int withhold_entry, int64_t wait_budget_ns) {
+    if (withhold_entry < -1 || wait_budget_ns < 0 || wait_budget_ns > (int64_t)10 * 1000 * 1000 * 1000)
+        return MOE_EINVAL;
+    set_fault_injection(withhold_entry, wait_budget_ns);
+    return MOE_OK;
 }
 
 MOE_API int moe_synth_normal(uint64_t seed, uint64_t tid, int64_t offset, int64_t n, float sigma, float* out,
@@ -444,7 +522,7 @@ MOE_API int moe_forward_launches(const moe_config* cfg, int T) {
     if (st) return st;
     if (T < 0) return MOE_EINVAL;
     if (T == 0) return 0;
-    return small_path_supported(*cfg, T) ? kSmallLaunches : kForwardLaunches;
+    return small_path_supported(*cfg, T) ? kSmallLaunches : tc_path_supported(*cfg, T) ? kTcLaunches : kForwardLaunches;
 }
 
 MOE_API int moe_forward_phases(const moe_config* cfg, int T) {

@@ -195,20 +195,22 @@ __global__ void __launch_bounds__(256) k_down(ExpertParams p) {
     }
 }
 
-// out[t][c] = sum_j w[t][j] * y[slot(t,j)][c] + y[T*k + t][c]  (fp32, in
-// slot order, then the shared expert).
+// out[t][c] = sum_j w[t][j] * y[slot(t,j)][c] + y[T*k + t][c], summed in
+// fp64 in slot order, then the shared expert, and rounded to fp32 (each
+// fp32 x fp32 product is exact in fp64, so every step rounds once, as the
+// definition's fp64 sum does).
 __global__ void k_combine(ExpertParams p) {
     const int64_t n = (int64_t)p.T * p.H;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
         const int t = (int)(i / p.H), c = (int)(i % p.H);
-        float acc = 0.0f;
+        double acc = 0.0;
         for (int j = 0; j < p.k; ++j) {
             const int slot = p.inv_perm[t * p.k + j];
             if (slot < 0) continue;  // dropped by the adaptive top-p
-            acc = fmaf(p.w[t * p.k + j], p.y[(int64_t)slot * p.H + c], acc);
+            acc = __fma_rn((double)p.w[t * p.k + j], (double)p.y[(int64_t)slot * p.H + c], acc);
         }
-        if (p.ns) acc += p.y[((int64_t)p.T * p.k + t) * p.H + c];
-        p.out[i] = acc;
+        if (p.ns) acc = __dadd_rn(acc, (double)p.y[((int64_t)p.T * p.k + t) * p.H + c]);
+        p.out[i] = __double2float_rn(acc);
     }
 }
 
@@ -242,6 +244,25 @@ static cudaError_t launch_experts_t(const ExpertParams& p, cudaStream_t s, cudaE
     e = cudaGetLastError();
     if (e == cudaSuccess && ev) e = cudaEventRecord(ev[2], s);
     return e;
+}
+
+static ExpertParams expert_params(const ExpertArgs& a) {
+    const moe_config& c = *a.cfg;
+    ExpertParams p;
+    p.T = a.T; p.H = c.hidden; p.I = c.inter; p.E = c.n_experts; p.k = c.top_k; p.ns = c.n_shared;
+    p.xq = a.xq; p.xd = a.xd; p.w = a.w; p.offsets = a.offsets; p.perm = a.perm; p.inv_perm = a.inv_perm;
+    p.active = a.active; p.routed = a.routed; p.shared = a.shared;
+    p.hq = a.hq; p.hd = a.hd; p.y = a.y; p.out = a.out; p.err = a.err;
+    return p;
+}
+
+cudaError_t launch_combine(const ExpertArgs& a, cudaStream_t s) {
+    const ExpertParams p = expert_params(a);
+    const int64_t n = (int64_t)p.T * p.H;
+    const int64_t want = (n + 255) / 256, cap = (int64_t)device_info().sm_count * 8;
+    const int grid = (int)(want < cap ? want : cap);
+    k_combine<<<max(1, grid), 256, 0, s>>>(p);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t s, cudaEvent_t const* ev) {
@@ -285,12 +306,44 @@ __global__ void __launch_bounds__(256) k_block_dots(const uint8_t* __restrict__ 
     }
 }
 
+// The fused small-batch kernel's routine: the activation block is put in the
+// weights' order by the same reordering (act_nibble_order / act_crumb_order),
+// its correction term taken by act_corr, and the block dotted by
+// dot_block_scaled, which returns the dot times dot_scale (16 for int4, 64 for
+// int2, 1 for int8) exactly; that scaled value is what is stored.
+template <int WBITS>
+__global__ void __launch_bounds__(256) k_block_dots_fused(const uint8_t* __restrict__ packed, int64_t rows, int cols,
+                                                          const int8_t* __restrict__ q, int n,
+                                                          int32_t* __restrict__ out) {
+    const int lane = threadIdx.x & 31;
+    const int64_t wid = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (wid >= rows * n) return;
+    const int64_t r = wid % rows, t = wid / rows;
+    const int nb = cols / kQBlock;
+    const uint8_t* row = packed + r * ((int64_t)cols * WBITS / 8);
+    for (int b = lane; b < nb; b += 32) {
+        const uint4 lo = ld_nc_v4(q + t * cols + b * kQBlock);
+        const uint4 hi = ld_nc_v4(q + t * cols + b * kQBlock + 16);
+        ActBlock a;
+        if constexpr (WBITS == 4) a = act_nibble_order(lo, hi);
+        else if constexpr (WBITS == 2) a = act_crumb_order(lo, hi);
+        else a = act_natural(lo, hi);
+        out[(t * rows + r) * nb + b] = dot_block_scaled<WBITS>(load_w_block<WBITS>(row, b), a, act_corr<WBITS>(a));
+    }
+}
+
 cudaError_t launch_block_dots(const uint8_t* packed, int64_t rows, int cols, int wbits, const int8_t* q, int n,
-                              int32_t* out, cudaStream_t s) {
+                              int32_t* out, cudaStream_t s, int routine) {
     const int64_t warps = rows * n;
     if (warps == 0) return cudaSuccess;
     const int64_t grid = (warps + 7) / 8;
     if (grid > 0x7fffffff) return cudaErrorInvalidValue;
+    if (routine == MOE_DOTS_FUSED) {
+        if (wbits == 4) k_block_dots_fused<4><<<(unsigned)grid, 256, 0, s>>>(packed, rows, cols, q, n, out);
+        else if (wbits == 2) k_block_dots_fused<2><<<(unsigned)grid, 256, 0, s>>>(packed, rows, cols, q, n, out);
+        else k_block_dots_fused<8><<<(unsigned)grid, 256, 0, s>>>(packed, rows, cols, q, n, out);
+        return cudaGetLastError();
+    }
     if (wbits == 4) k_block_dots<4><<<(unsigned)grid, 256, 0, s>>>(packed, rows, cols, q, n, out);
     else if (wbits == 2) k_block_dots<2><<<(unsigned)grid, 256, 0, s>>>(packed, rows, cols, q, n, out);
     else k_block_dots<8><<<(unsigned)grid, 256, 0, s>>>(packed, rows, cols, q, n, out);

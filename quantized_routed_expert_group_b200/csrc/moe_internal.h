@@ -31,6 +31,8 @@ struct Layout {
     size_t hq;         // int8 [slots][I]
     size_t hd;         // fp32 [slots][I/32]
     size_t y;          // fp32 [slots][H]
+    // batched tensor-core path only (0 bytes otherwise)
+    size_t tc_xg, tc_xdT, tc_gu, tc_hg, tc_hdT, tc_row_tok, tc_row_slot, tc_units_gu, tc_units_dn, tc_ctrl;
     size_t total;
 };
 
@@ -49,6 +51,10 @@ cudaError_t launch_pack_weights(const float* w, int64_t rows, int cols, int wbit
                                 float* scales, cudaStream_t s);
 cudaError_t launch_requant_fp8(const uint8_t* w8, const float* block_scales, int64_t rows, int cols, int block,
                                int wbits, uint8_t* packed, float* scales, cudaStream_t s);
+// The router's workspace: logits [T][E] fp64, then (T >= kRouterTiledMinTokens)
+// the tiled kernel's K-split partial sums.
+constexpr int kRouterTiledMinTokens = 64;
+size_t router_ws_bytes(const moe_config& c, int T);
 cudaError_t launch_router(const moe_config& c, const float* x, int T, const float* router_w,
                           const float* bias, double* logits, int32_t* idx, float* w, cudaStream_t s);
 cudaError_t launch_bucket(const moe_config& c, const int32_t* idx, int T, int32_t* counts,
@@ -77,6 +83,37 @@ struct ExpertArgs {
 // ev (optional, 3 events): recorded after gate/up, down and combine.
 cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t s, cudaEvent_t const* ev);
 constexpr int kForwardLaunches = 7;  // quantise, logits, select, bucket, gate/up, down, combine
+cudaError_t launch_combine(const ExpertArgs& a, cudaStream_t s);
+
+// Batched path on the tensor cores (moe_tc.cu), for T >= kTcMinTokens.
+constexpr int kTcMinTokens = 64;
+constexpr int kTcLaunches = 10;  // quantise, logits, select, bucket, plan, gather, gate/up, SwiGLU, down, combine
+bool tc_path_supported(const moe_config& c, int T);
+struct TcSizes {
+    int prows_cap;     // rows of the padded row space
+    int units_gu_cap;  // work units of the gate/up GEMM
+    int units_dn_cap;  // work units of the down GEMM
+};
+TcSizes tc_sizes(const moe_config& c, int T);
+struct TcArgs {
+    ExpertArgs ex;
+    int8_t* xg;         // [prows_cap][hidden]
+    double* xdT;        // [hidden/32][prows_cap]
+    float* gu;          // [2][prows_cap][inter]  g and u row values
+    int8_t* hg;         // [prows_cap][inter]
+    double* hdT;        // [inter/32][prows_cap]
+    int32_t* row_tok;   // [prows_cap]
+    int32_t* row_slot;  // [prows_cap]
+    void* units_gu;     // TcUnit [units_gu_cap]
+    void* units_dn;     // TcUnit [units_dn_cap]
+    int32_t* ctrl;      // [8]
+    TcSizes sz;
+};
+constexpr size_t kTcUnitBytes = 16;
+// plan + gather (the end of the bucketing phase)
+cudaError_t launch_tc_prepare(const TcArgs& a, cudaStream_t s);
+// gate/up GEMM, down GEMM, combine; ev (optional, 3 events) after each
+cudaError_t launch_tc_experts(const TcArgs& a, cudaStream_t s, cudaEvent_t const* ev);
 // Fused small-batch forward (T <= 4), moe_small.cu.
 struct SmallArgs {
     const moe_config* cfg;
@@ -108,9 +145,16 @@ bool small_path_supported(const moe_config& c, int T);
 size_t small_ctrl_bytes(const moe_config& c, int T);
 cudaError_t launch_small(const SmallArgs& a, cudaStream_t s);
 constexpr int kSmallLaunches = 2;  // prologue + persistent kernel
+// Test hook (moe_debug_fault_injection): withhold one entry's first h
+// publication in the fused kernel, and bound its producer waits by wait_ns
+// (<= 0: the default).
+void set_fault_injection(int withhold_entry, int64_t wait_ns);
 
 cudaError_t launch_block_dots(const uint8_t* packed, int64_t rows, int cols, int wbits, const int8_t* q,
-                              int n, int32_t* out, cudaStream_t s);
+                              int n, int32_t* out, cudaStream_t s, int routine);
+// Tensor-core per-block dots (moe_tc.cu): n <= 64 token rows of q.
+cudaError_t launch_tc_block_dots(const uint8_t* packed, int64_t rows, int cols, int wbits, const int8_t* q, int n,
+                                 int32_t* out, cudaStream_t s);
 cudaError_t launch_synth_normal(uint64_t seed, uint64_t tid, int64_t offset, int64_t n, float sigma,
                                 float* out, cudaStream_t s);
 

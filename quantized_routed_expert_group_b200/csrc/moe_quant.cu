@@ -7,6 +7,8 @@
 // offline converter that dequantises the FP8 checkpoint with its 128 x 128
 // block scales and requantises it per row (same bullet list; wpnews.pro
 // converter list).
+#include <cuda_fp16.h>
+
 #include "moe_device.cuh"
 #include "moe_internal.h"
 
@@ -165,9 +167,139 @@ cudaError_t launch_pack_weights(const float* w, int64_t rows, int cols, int wbit
     return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// FP8 requantiser, one warp per row with the row's codes in registers.
+//
+// Lane l holds 16-code chunks l, l + 32, ... (16-byte loads, coalesced).
+// The row's amax needs no decoding of most codes: for E4M3 the magnitude
+// order of the non-NaN codes is the integer order of their low 7 bits, and
+// within a block every value is code * the block's scale (rounding is
+// monotone), so amax = max over blocks of |value(largest code) * scale|,
+// exactly the maximum of |value * scale| over the row.  The codes are then
+// decoded once each (E4M3 -> f16 is exact, f16 -> fp32 is exact), scaled
+// by their block's scale (one fp32 multiply, as the definition), quantised
+// and packed.  Rows up to kRequantMaxCols codes; NaN codes are unspecified.
+// ---------------------------------------------------------------------------
+constexpr int kRequantMaxChunks = 16;  // per lane: 16 x 16 codes
+constexpr int kRequantMaxCols = 32 * 16 * kRequantMaxChunks;
+
+// Two E4M3 codes (low and high byte of v) -> two fp32 values, exactly.
+__device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t v) {
+    uint32_t h2;
+    asm("{\n\t.reg .b16 lo;\n\tcvt.u16.u32 lo, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}" : "=r"(h2) : "r"(v));
+    return __half22float2(*reinterpret_cast<const __half2*>(&h2));
+}
+
+// Largest 7-bit magnitude field of the 16 codes of a chunk.
+__device__ __forceinline__ uint32_t chunk_max_mag(uint4 w) {
+    const uint32_t m = __vmaxu4(__vmaxu4(w.x & 0x7F7F7F7Fu, w.y & 0x7F7F7F7Fu), __vmaxu4(w.z & 0x7F7F7F7Fu, w.w & 0x7F7F7F7Fu));
+    return max(max(m & 0xFFu, (m >> 8) & 0xFFu), max((m >> 16) & 0xFFu, m >> 24));
+}
+
+template <int WBITS, int NCH>
+__global__ void __launch_bounds__(256) k_requant_fp8_rows(const uint8_t* __restrict__ w8, const float* __restrict__ bs,
+                                                          int64_t rows, int cols, int block, int nbc,
+                                                          uint8_t* __restrict__ packed, float* __restrict__ scales) {
+    constexpr int qmax = WBITS == 8 ? 127 : WBITS == 4 ? 7 : 1;
+    constexpr float qminf = -(float)(1 << (WBITS - 1));
+    const int lane = threadIdx.x & 31;
+    const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (r >= rows) return;
+    const int nch = cols / 16;
+    const uint4* src = reinterpret_cast<const uint4*>(w8 + r * cols);
+    const float* bsr = bs + (r / block) * nbc;
+    uint4 w[NCH];
+#pragma unroll
+    for (int j = 0; j < NCH; ++j) {
+        const int c = lane + 32 * j;
+        w[j] = c < nch ? ld_stream_v4(src + c) : make_uint4(0, 0, 0, 0);
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < NCH; ++j) {
+        const int c = lane + 32 * j;
+        if (c < nch) {
+            const float top = e4m3x2_to_f32(chunk_max_mag(w[j])).x;
+            amax = fmaxf(amax, fabsf(__fmul_rn(top, __ldg(bsr + (16 * c) / block))));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
+    float sc = 0.0f, is = 0.0f;
+    if (amax >= FLT_MIN) {
+        sc = __fdiv_rn(amax, (float)qmax);
+        is = __fdiv_rn(1.0f, sc);
+    }
+    const bool zero = !(sc > 0.0f);
+    if (lane == 0) scales[r] = sc;
+    uint8_t* dst = packed + r * ((int64_t)cols * WBITS / 8);
+#pragma unroll
+    for (int j = 0; j < NCH; ++j) {
+        const int c = lane + 32 * j;
+        if (c >= nch) continue;
+        const float bsc = __ldg(bsr + (16 * c) / block);
+        const uint32_t ww[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
+        int code[16];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 a = e4m3x2_to_f32(ww[k] & 0xFFFFu), b = e4m3x2_to_f32(ww[k] >> 16);
+            const float v[4] = {a.x, a.y, b.x, b.y};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float q = roundf(__fmul_rn(__fmul_rn(v[i], bsc), is));
+                q = fminf(fmaxf(q, qminf), (float)qmax);
+                code[4 * k + i] = zero ? 0 : (int)q;
+            }
+        }
+        if constexpr (WBITS == 8) {
+            uint32_t o[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                o[k] = (uint32_t)(code[4 * k] & 0xFF) | ((uint32_t)(code[4 * k + 1] & 0xFF) << 8) |
+                       ((uint32_t)(code[4 * k + 2] & 0xFF) << 16) | ((uint32_t)(code[4 * k + 3] & 0xFF) << 24);
+            reinterpret_cast<uint4*>(dst)[c] = make_uint4(o[0], o[1], o[2], o[3]);
+        } else if constexpr (WBITS == 4) {
+            uint32_t o[2] = {0u, 0u};
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[i >> 3] |= (uint32_t)(code[i] & 0xF) << (4 * (i & 7));
+            reinterpret_cast<uint2*>(dst)[c] = make_uint2(o[0], o[1]);
+        } else {
+            uint32_t o = 0u;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o |= (uint32_t)(code[i] & 0x3) << (2 * i);
+            reinterpret_cast<uint32_t*>(dst)[c] = o;
+        }
+    }
+}
+
+template <int WBITS>
+static cudaError_t launch_requant_rows(const uint8_t* w8, const float* bs, int64_t rows, int cols, int block,
+                                       uint8_t* packed, float* scales, cudaStream_t s) {
+    const int nbc = (cols + block - 1) / block;
+    const int64_t grid = (rows + 7) / 8;
+    if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    const int per_lane = (cols / 16 + 31) / 32;
+    if (per_lane <= 4)
+        k_requant_fp8_rows<WBITS, 4><<<(unsigned)grid, 256, 0, s>>>(w8, bs, rows, cols, block, nbc, packed, scales);
+    else if (per_lane <= 8)
+        k_requant_fp8_rows<WBITS, 8><<<(unsigned)grid, 256, 0, s>>>(w8, bs, rows, cols, block, nbc, packed, scales);
+    else if (per_lane <= 12)
+        k_requant_fp8_rows<WBITS, 12><<<(unsigned)grid, 256, 0, s>>>(w8, bs, rows, cols, block, nbc, packed, scales);
+    else
+        k_requant_fp8_rows<WBITS, 16><<<(unsigned)grid, 256, 0, s>>>(w8, bs, rows, cols, block, nbc, packed, scales);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_requant_fp8(const uint8_t* w8, const float* block_scales, int64_t rows, int cols, int block,
                                int wbits, uint8_t* packed, float* scales, cudaStream_t s) {
     if (rows == 0) return cudaSuccess;
+    // the warp-per-row kernel: 16-byte aligned rows of at most kRequantMaxCols codes
+    if (cols <= kRequantMaxCols && cols % 16 == 0 && reinterpret_cast<uintptr_t>(w8) % 16 == 0 &&
+        (int64_t)cols * wbits / 8 % 4 == 0) {
+        if (wbits == 8) return launch_requant_rows<8>(w8, block_scales, rows, cols, block, packed, scales, s);
+        if (wbits == 4) return launch_requant_rows<4>(w8, block_scales, rows, cols, block, packed, scales, s);
+        return launch_requant_rows<2>(w8, block_scales, rows, cols, block, packed, scales, s);
+    }
     const int grid = (int)(rows < 1048576 ? rows : 1048576);
     const RowsFp8Block src{w8, block_scales, cols, block, (cols + block - 1) / block};
     if (wbits == 8) k_pack_rows<8><<<grid, 256, 0, s>>>(src, rows, cols, packed, scales);

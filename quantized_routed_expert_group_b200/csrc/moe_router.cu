@@ -71,6 +71,94 @@ __global__ void __launch_bounds__(256) k_router_logits(const float* __restrict__
     }
 }
 
+// Batched logits (T >= kRouterTiledMinTokens): a tiled fp64 GEMM on the CUDA
+// cores.  CTA = 64 tokens x 64 experts x one K split; each thread keeps a
+// 4 x 4 tile of fp64 sums; x and the router rows are staged per 32-column
+// chunk in shared memory, widened to fp64 (every fp32 product is then exact
+// and every sum rounds in fp64, as the definition's).  The K splits' partial
+// sums go to parts [S][T][E] and are added in split order by
+// k_router_reduce, so the logits do not depend on the launch.
+constexpr int kRtT = 64, kRtE = 64, kRtK = 32, kRtPad = 2;
+
+int router_splits(const moe_config& c, int T) {
+    if (T < kRouterTiledMinTokens || c.hidden % kRtK) return 0;
+    const int tiles = ((T + kRtT - 1) / kRtT) * ((c.n_experts + kRtE - 1) / kRtE);
+    const int want = tiles <= 16 ? 16 : tiles <= 64 ? 8 : 4;
+    const int chunks = c.hidden / kRtK;
+    return want < chunks ? want : chunks;
+}
+
+__global__ void __launch_bounds__(256) k_router_logits_f64(const float* __restrict__ x, int T, int H,
+                                                           const float* __restrict__ Wr, int E, int chunks_per_split,
+                                                           double* __restrict__ parts) {
+    __shared__ __align__(16) double xs[kRtK][kRtT + kRtPad];
+    __shared__ __align__(16) double ws[kRtK][kRtE + kRtPad];
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    const int t0 = blockIdx.y * kRtT, e0 = blockIdx.x * kRtE, split = blockIdx.z;
+    const int nchunks = H / kRtK;
+    const int kc0 = split * chunks_per_split;
+    const int kc1 = min(nchunks, kc0 + chunks_per_split);
+    double acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+    for (int kc = kc0; kc < kc1; ++kc) {
+        // 64 rows x 32 columns of x and of the router rows: 512 float4 each
+#pragma unroll
+        for (int i = tid; i < 512; i += 256) {
+            const int r = i >> 3, k4 = i & 7;
+            const int t = t0 + r, e = e0 + r;
+            const float4 xv = t < T ? __ldg(reinterpret_cast<const float4*>(x + (int64_t)t * H + kc * kRtK) + k4)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 wv = e < E ? __ldg(reinterpret_cast<const float4*>(Wr + (int64_t)e * H + kc * kRtK) + k4)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            xs[4 * k4 + 0][r] = (double)xv.x;
+            xs[4 * k4 + 1][r] = (double)xv.y;
+            xs[4 * k4 + 2][r] = (double)xv.z;
+            xs[4 * k4 + 3][r] = (double)xv.w;
+            ws[4 * k4 + 0][r] = (double)wv.x;
+            ws[4 * k4 + 1][r] = (double)wv.y;
+            ws[4 * k4 + 2][r] = (double)wv.z;
+            ws[4 * k4 + 3][r] = (double)wv.w;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int k = 0; k < kRtK; ++k) {
+            const double2 a01 = *reinterpret_cast<const double2*>(&xs[k][4 * ty]);
+            const double2 a23 = *reinterpret_cast<const double2*>(&xs[k][4 * ty + 2]);
+            const double2 b01 = *reinterpret_cast<const double2*>(&ws[k][4 * tx]);
+            const double2 b23 = *reinterpret_cast<const double2*>(&ws[k][4 * tx + 2]);
+            const double a[4] = {a01.x, a01.y, a23.x, a23.y};
+            const double b[4] = {b01.x, b01.y, b23.x, b23.y};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = __fma_rn(a[i], b[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int t = t0 + 4 * ty + i;
+        if (t >= T) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int e = e0 + 4 * tx + j;
+            if (e < E) parts[((int64_t)split * T + t) * E + e] = acc[i][j];
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256) k_router_reduce(const double* __restrict__ parts, int S, int64_t n,
+                                                       double* __restrict__ logits) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        double v = parts[i];
+        for (int sp = 1; sp < S; ++sp) v = __dadd_rn(v, parts[(int64_t)sp * n + i]);
+        logits[i] = v;
+    }
+}
+
 // Selection: one warp per token.  s = sigmoid(logit), c = s + bias; group
 // score = sum of the two largest c (first the maximum, then the largest of the
 // rest, ties to the lower index); keep the topk_groups best groups; take the
@@ -151,13 +239,35 @@ __global__ void __launch_bounds__(128) k_router_select(const double* __restrict_
     }
 }
 
+size_t router_ws_bytes(const moe_config& c, int T) {
+    const size_t logits = ((size_t)T * c.n_experts * sizeof(double) + 255) & ~(size_t)255;
+    const int S = router_splits(c, T);
+    return logits + (size_t)S * T * c.n_experts * sizeof(double);
+}
+
 cudaError_t launch_router(const moe_config& c, const float* x, int T, const float* router_w,
                           const float* bias, double* logits, int32_t* idx, float* w, cudaStream_t s) {
     if (T == 0) return cudaSuccess;
-    dim3 g1((c.n_experts + kRouterExpertsPerCta - 1) / kRouterExpertsPerCta,
-            (T + kRouterTokens - 1) / kRouterTokens);
-    k_router_logits<<<g1, 256, 0, s>>>(x, T, c.hidden, router_w, c.n_experts, logits);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e;
+    const int S = router_splits(c, T);
+    if (S > 0) {
+        // the partial sums follow the logits in the router's workspace
+        double* parts = logits + (((size_t)T * c.n_experts * sizeof(double) + 255) & ~(size_t)255) / sizeof(double);
+        const int chunks = c.hidden / kRtK;
+        const int per = (chunks + S - 1) / S;
+        dim3 g0((c.n_experts + kRtE - 1) / kRtE, (T + kRtT - 1) / kRtT, S);
+        k_router_logits_f64<<<g0, 256, 0, s>>>(x, T, c.hidden, router_w, c.n_experts, per, parts);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        const int64_t n = (int64_t)T * c.n_experts;
+        const int64_t want = (n + 255) / 256, cap = (int64_t)device_info().sm_count * 8;
+        k_router_reduce<<<(int)(want < cap ? want : cap), 256, 0, s>>>(parts, S, n, logits);
+    } else {
+        dim3 g1((c.n_experts + kRouterExpertsPerCta - 1) / kRouterExpertsPerCta,
+                (T + kRouterTokens - 1) / kRouterTokens);
+        k_router_logits<<<g1, 256, 0, s>>>(x, T, c.hidden, router_w, c.n_experts, logits);
+    }
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const size_t smem = (size_t)4 * 2 * c.n_experts * sizeof(double);
     if (smem > 48 * 1024) {

@@ -38,6 +38,7 @@
 // * A tiny prologue kernel (Q8_0 of x, control-block reset) runs first; the
 //   main kernel is its programmatic dependent and issues its router rows
 //   before waiting for it.
+#include <atomic>
 #include <cmath>
 
 #include "moe_device.cuh"
@@ -46,11 +47,19 @@
 
 namespace moe {
 
-constexpr int kConsumerWarps = 8;
+constexpr int kConsumerWarps = 8;  // warps of one consumer group
 constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kProducerWarp = kConsumerWarps;      // streams the items
-constexpr int kFinisherWarp = kConsumerWarps + 1;  // finishes gate/up units
-constexpr int kSmallThreads = kConsumers + 64;
+// Warp roles: kGroups groups of consumer warps (two at one token, where the
+// consumers' latency sets the pace: the groups work on alternate ring slots),
+// then the producer warp (streams the items) and the finisher warp (finishes
+// gate/up units).
+template <int TM>
+struct Roles {
+    static constexpr int kGroups = TM == 1 ? 2 : 1;
+    static constexpr int kProducerWarp = kGroups * kConsumerWarps;
+    static constexpr int kFinisherWarp = kProducerWarp + 1;
+    static constexpr int kThreads = (kFinisherWarp + 1) * 32;
+};
 constexpr int kSlotWeightBytes = 48 * 1024;
 constexpr int kMaxSlots = 4;
 constexpr int kUnit = 32;          // gate/up rows per unit: one Q8_0 block of h
@@ -68,22 +77,24 @@ constexpr int kRowBatch = 4;       // rows reduced together
 constexpr int kMaxGuBlocks = 3;    // hidden / 32 <= 192 blocks over 64 column threads
 constexpr int kMaxDownBlocks = 8;  // inter / 32 <= 512
 
-// Bounds of every wait (legitimate waits last microseconds): mbarrier
-// try_wait iterations, and polls of a global word with a short sleep each.
-constexpr uint32_t kWaitLimit = 1u << 20;
-constexpr uint32_t kSpinLimit = 1u << 21;
-// Consumers only ever wait for their producer, whose own waits are bounded
-// and end in a DONE marker, so their bound is far larger and never reached
-// unless the device misbehaves; the producer's wait for the consumers'
-// routing uses the same bound.
-constexpr uint32_t kConsumerWaitLimit = 1u << 24;
+// Bounds of every wait, in nanoseconds of the global timer (legitimate waits
+// last microseconds).  The producer's waits (a free ring slot, another CTA's
+// h codes) give up after wait_ns (kWaitNs unless a test shortens it) and end
+// the CTA's schedule with a DONE marker; every other wait (consumers on their
+// producer, the producer on the consumers' routing, the finisher on the
+// consumers) spans at most one producer wait plus that hand-over, so its
+// bound is kSlackWaits times as long.  A wait that runs out records
+// kErrTimeout in the error word; the kernel then returns.
+constexpr uint64_t kWaitNs = 25ull * 1000 * 1000;
+constexpr uint64_t kSlackWaits = 4;
 
 enum ItemKind : int {
     kItemSelect = 2,
     kItemGateUp = 3,
     kItemDown = 4,
     kItemCombine = 5,
-    kItemDone = 6
+    kItemDone = 6,
+    kItemSync = 7  // two groups: the other group's down outputs are complete
 };
 
 // Control block (int32 words, zeroed by the prologue on every call):
@@ -155,6 +166,8 @@ struct SmallParams {
     float* out;
     int* ctrl;
     int32_t* err;
+    uint64_t wait_ns;  // bound of the producer's waits (see kWaitNs)
+    int fault_entry;   // test hook: the entry whose first unit's h codes are never published (-1: none)
     SmallGeom g;
 };
 
@@ -170,6 +183,7 @@ struct SlotMeta {
     int last;    // gate/up: last chunk of its unit
     int off_a;   // byte offset in the slot: gate scales / h scales
     int off_b;   // byte offset in the slot: up scales / down row scales
+    int uc;      // gate/up: the unit's ordinal in this CTA; DONE: the CTA's unit count
     int tok[4];
 };
 
@@ -210,7 +224,7 @@ SmallGeom small_geometry(const moe_config& c, int T, int grid) {
     g.o_xd = o;
     o += round_up(g.tmax * (H / 32) * 4, 128);
     g.o_bar = o;
-    o += 128;  // full[4], empty[4], routing, ufull[2], ufree[2]
+    o += 128;  // full[4], empty[4], routing, ufull[2], ufree[2], gsync, gexit
     g.o_meta = o;
     o += round_up((int)sizeof(SlotMeta) * kMaxSlots, 128);
     g.o_urec = o;
@@ -232,6 +246,8 @@ SmallGeom small_geometry(const moe_config& c, int T, int grid) {
     // as many ring slots (up to four) as the shared memory holds
     const int smem_max = device_info().max_smem_optin;
     while (g.nslot > 2 && o + g.nslot * g.slot_bytes > smem_max) --g.nslot;
+    // two consumer groups (one token) take alternate slots: an even ring
+    if (g.tmax == 1 && (g.nslot & 1)) --g.nslot;
     const int ring = g.nslot * g.slot_bytes;
     g.o_xq += ring; g.o_xd += ring; g.o_bar += ring; g.o_meta += ring; g.o_urec += ring; g.o_gpart += ring;
     g.o_usc += ring; g.o_ent += ring; g.o_selw += ring; g.o_inv += ring; g.o_ys += ring; g.o_misc += ring;
@@ -264,13 +280,14 @@ size_t small_ctrl_bytes(const moe_config& c, int T) {
 
 // ---------------------------------------------------------------------------
 // Prologue: reset the control block, quantise x and compute the router
-// logits.  It launches its dependent (the main kernel) right away; its blocks
-// need no shared memory and few registers, so they run beside the main
-// kernel's persistent CTAs, which meanwhile stream the shared expert.  The
-// main kernel reads the logits after waiting for this grid.
+// logits.  It launches its dependent (the main kernel) at once; the main
+// kernel's CTAs, which need most of an SM's shared memory, start as the
+// prologue's blocks on their SM exit, and read the logits after waiting for
+// this grid.
 //
 // Router logits (the router row of expert e dotted with x, per token): block
-// b takes experts b, b + grid, ...; warp w takes eighth w of the hidden
+// b takes experts b, b + grid, ... (one row per block: the grid has a block
+// per expert, at least one per SM); warp w takes eighth w of the hidden
 // dimension, each lane holds its weights (float4) in registers and keeps four
 // compensated fp32 sums per token (one per float4 component, about 2^-48
 // relative each), folded into fp64; the eighths are added in fp64 in a fixed
@@ -366,6 +383,8 @@ struct SmemPtrs {
     uint64_t* routing;  // consumers -> producer: the routing tables are ready
     uint64_t* ufull;    // [2] every consumer warp has written its partials of a unit
     uint64_t* ufree;    // [2] the finisher warp has read them
+    uint64_t* gsync;    // the syncing group's warps: their down outputs are in ys
+    uint64_t* gexit;    // every consumer warp has left its loop
     UnitRec* urec;      // [2] the unit to finish
     SlotMeta* meta;
     float* gpart;    // [2][32][2][2][4] gate/up partial dots of a unit: [buffer][pair][gate/up][half][token]
@@ -387,6 +406,8 @@ __device__ __forceinline__ SmemPtrs carve(uint8_t* base, const SmallGeom& g) {
     s.routing = s.empty + kMaxSlots;
     s.ufull = s.routing + 1;
     s.ufree = s.ufull + 2;
+    s.gsync = s.ufree + 2;
+    s.gexit = s.gsync + 1;
     s.meta = reinterpret_cast<SlotMeta*>(base + g.o_meta);
     s.urec = reinterpret_cast<UnitRec*>(base + g.o_urec);
     s.gpart = reinterpret_cast<float*>(base + g.o_gpart);
@@ -427,16 +448,18 @@ struct Producer {
     const SmallParams& p;
     const SmemPtrs& s;
     const int lane;
+    const int groups;  // consumer groups (each takes every groups-th ring slot)
     uint64_t pol;
     int slot = 0;
+    int units = 0;     // gate/up units issued (their ordinals stamp the items)
     uint32_t pe = 1;  // parity to wait on the empty barriers (fresh ring: all empty)
     bool aborted = false;
     bool need_proxy_fence = false;  // set after acquiring data that later copies read
     uint32_t issued_mask = 0, issued_par = 0;
     uint32_t rdy0 = 0, rdy1 = 0, rdy2 = 0, rdy3 = 0, rdy4 = 0;  // entries whose h codes are all published
 
-    __forceinline__ __device__ Producer(const SmallParams& p_, const SmemPtrs& s_, int lane_)
-        : p(p_), s(s_), lane(lane_) {
+    __forceinline__ __device__ Producer(const SmallParams& p_, const SmemPtrs& s_, int lane_, int groups_)
+        : p(p_), s(s_), lane(lane_), groups(groups_) {
         pol = l2_evict_first_policy();
     }
 
@@ -458,6 +481,7 @@ struct Producer {
         m.last = 0;
         m.off_a = 0;
         m.off_b = 0;
+        m.uc = 0;
         for (int i = 0; i < 4; ++i) m.tok[i] = 0;
         return m;
     }
@@ -476,7 +500,7 @@ struct Producer {
                                          const Copy& c3) {
         if (aborted) return false;
         int ok = 1;
-        if (lane == 0) ok = mbar_wait(&s.empty[slot], pe, kWaitLimit) ? 1 : 0;
+        if (lane == 0) ok = mbar_wait_ns(&s.empty[slot], pe, p.wait_ns) ? 1 : 0;
         ok = __shfl_sync(kFull, ok, 0);
         __syncwarp();
         if (!ok) {
@@ -537,6 +561,8 @@ struct Producer {
         const Copy c3 = window(ex.s_up + r, g.rg, kSlotWeightBytes + kScaleWin);
         m.off_a = c2.first;
         m.off_b = c3.first;
+        m.uc = units;
+        if (m.last) ++units;
         return push(m, c0, c1, c2, c3);
     }
 
@@ -579,7 +605,8 @@ struct Producer {
     __forceinline__ __device__ bool wait_entry(int e, int U) {
         if (is_ready(e)) return true;
         need_proxy_fence = true;
-        for (uint32_t it = 0; it < kSpinLimit; ++it) {
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 <= p.wait_ns) {
             const bool f0 = entry_done(lane, U), f1 = entry_done(lane + 32, U), f2 = entry_done(lane + 64, U);
             const bool f3 = entry_done(lane + 96, U), f4 = entry_done(lane + 128, U);
             rdy0 = __ballot_sync(kFull, f0);
@@ -597,19 +624,30 @@ struct Producer {
         return false;
     }
 
-    // After a timeout: hand the consumers a DONE marker if a slot frees up in
-    // time (otherwise they time out on their own).
+    // One DONE marker per consumer group (consecutive slots belong to
+    // different groups), carrying the CTA's unit count.  After a timeout this
+    // runs with `aborted` set: each marker is handed over if a slot frees up in
+    // time (otherwise that group times out on its own).
     __forceinline__ __device__ void finish() {
-        int ok = 0;
-        if (lane == 0 && mbar_wait(&s.empty[slot], pe, kWaitLimit)) {
-            s.meta[slot].kind = kItemDone;
-            mbar_arrive(&s.full[slot]);
-            ok = 1;
-        }
-        ok = __shfl_sync(kFull, ok, 0);
-        if (ok) {
+        for (int gi = 0; gi < groups; ++gi) {
+            int ok = 0;
+            if (lane == 0 && mbar_wait_ns(&s.empty[slot], pe, p.wait_ns)) {
+                s.meta[slot].kind = kItemDone;
+                s.meta[slot].uc = units;
+                mbar_arrive(&s.full[slot]);
+                ok = 1;
+            }
+            ok = __shfl_sync(kFull, ok, 0);
+            if (!ok) {
+                if (lane == 0) set_error(p.err, kErrTimeout);
+                return;
+            }
             issued_mask |= 1u << slot;
             issued_par = (issued_par & ~(1u << slot)) | ((pe ^ 1u) << slot);
+            if (++slot == p.g.nslot) {
+                slot = 0;
+                pe ^= 1u;
+            }
         }
     }
 
@@ -617,14 +655,16 @@ struct Producer {
     __forceinline__ __device__ void drain() {
         if (lane != 0) return;
         for (int i = 0; i < p.g.nslot; ++i)
-            if ((issued_mask >> i) & 1u) mbar_wait(&s.full[i], (issued_par >> i) & 1u, kWaitLimit);
+            if ((issued_mask >> i) & 1u) mbar_wait_ns(&s.full[i], (issued_par >> i) & 1u, p.wait_ns);
     }
 };
 
 // ---------------------------------------------------------------------------
 // Consumer items
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void consumers_sync() { named_barrier(1, kConsumers); }
+// Barrier of one consumer group's warps (group 0 runs the selection).
+__device__ __forceinline__ void group_sync(int group) { named_barrier(1 + group, kConsumers); }
+__device__ __forceinline__ void consumers_sync() { group_sync(0); }
 
 // (ka, ia) ranks before (kb, ib): larger key, ties to the lower index.
 // Branch-free, so that unrolled compare loops pipeline their loads.
@@ -1039,8 +1079,9 @@ __device__ __forceinline__ WBlock<WBITS> load_block_smem(const uint8_t* row, int
 // publishes it ----
 template <int WBITS, int TM>
 __device__ __forceinline__ void do_gateup(const SmallParams& p, const SmemPtrs& s, const SlotMeta& m,
-                                          const uint8_t* slot, int tid, uint64_t* empty, int uc) {
+                                          const uint8_t* slot, int tid, uint64_t* empty) {
     constexpr int V = kRowBatch * TM;
+    const int uc = m.uc;  // the unit's ordinal in this CTA
     const int buf = uc & 1;
     constexpr int SHIFT = 5 - Log2<V>::value;
     const int warp = tid >> 5, lane = tid & 31;
@@ -1053,8 +1094,9 @@ __device__ __forceinline__ void do_gateup(const SmallParams& p, const SmemPtrs& 
     const int first = m.row0 - m.blk * kUnit;  // first pair of the chunk inside its unit
     const float* sg = reinterpret_cast<const float*>(slot + m.off_a);
     const float* su = reinterpret_cast<const float*>(slot + m.off_b);
-    // the partials buffer of this unit was last read by the finisher of unit uc - 2
-    if (first == 0 && uc >= 2 && !mbar_wait(&s.ufree[buf], ((uc >> 1) - 1) & 1, kConsumerWaitLimit))
+    // the partials buffer of this unit was last read by the finisher of unit
+    // uc - 2 (every chunk checks: with two groups a unit's chunks are split)
+    if (uc >= 2 && !mbar_wait_ns(&s.ufree[buf], ((uc >> 1) - 1) & 1, kSlackWaits * p.wait_ns))
         set_error(p.err, kErrTimeout);
     // Branch-free inner loops (so that the independent dots interleave):
     // out-of-range blocks are clamped and get a zero scale, out-of-range rows
@@ -1112,10 +1154,10 @@ __device__ __forceinline__ void do_gateup(const SmallParams& p, const SmemPtrs& 
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty);
-    if (!m.last) return;
-    // Unit end: every warp reports its partials and goes on; the finisher
-    // warp turns them into h codes and publishes them
-    if (warp == 0 && lane == 0) s.urec[buf] = UnitRec{m.entry, m.blk, m.slot0, m.n};
+    // Every warp reports each chunk's partials and goes on (the unit's first
+    // chunk also leaves the unit's record); once all chunks of the unit are
+    // in, the finisher warp turns them into h codes and publishes them
+    if (first == 0 && warp == 0 && lane == 0) s.urec[buf] = UnitRec{m.entry, m.blk, m.slot0, m.n};
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.ufull[buf]);
 }
@@ -1130,7 +1172,7 @@ __device__ __forceinline__ void finisher(const SmallParams& p, const SmemPtrs& s
 #pragma unroll 1
     for (int k = 0;; ++k) {
         const int buf = k & 1;
-        if (!mbar_wait(&s.ufull[buf], (k >> 1) & 1, kConsumerWaitLimit)) {
+        if (!mbar_wait_ns(&s.ufull[buf], (k >> 1) & 1, kSlackWaits * p.wait_ns)) {
             if (lane == 0) set_error(p.err, kErrTimeout);
             return;
         }
@@ -1155,7 +1197,7 @@ __device__ __forceinline__ void finisher(const SmallParams& p, const SmemPtrs& s
         if (lane == 0) {
             mbar_arrive(&s.ufree[buf]);
             fence_acq_rel_gpu();  // the warp's h codes before the count (release pattern)
-            red_add_relaxed_gpu(p.ctrl + kCHeader + r.entry, n);
+            if (r.entry != p.fault_entry || r.blk != 0) red_add_relaxed_gpu(p.ctrl + kCHeader + r.entry, n);
         }
         __syncwarp();
     }
@@ -1262,9 +1304,25 @@ __device__ __forceinline__ void do_down(const SmallParams& p, const SmemPtrs& s,
 
 // ---- COMBINE: the CTA's output rows from its per-slot down outputs (the
 // two column halves of each row are added here, half 0 + half 1) ----
+// ---- SYNC (two groups): this group's down outputs are all in ys (its
+// items are processed in order); the other group's COMBINE waits for it ----
+__device__ __forceinline__ void do_sync(const SmemPtrs& s, int tid, uint64_t* empty) {
+    __syncwarp();
+    if ((tid & 31) == 0) {
+        mbar_arrive(s.gsync);
+        mbar_arrive(empty);
+    }
+}
+
 __device__ __forceinline__ void do_combine(const SmallParams& p, const SmemPtrs& s, const SlotMeta& m, int tid,
-                                           uint64_t* empty) {
-    consumers_sync();  // every warp's down outputs are in ys
+                                           uint64_t* empty, int group, int groups) {
+    group_sync(group);  // every warp of this group has its down outputs in ys
+    if (groups > 1 && !mbar_wait_ns(s.gsync, 0, kSlackWaits * p.wait_ns)) {  // and the other group's
+        set_error(p.err, kErrTimeout);
+        __syncwarp();
+        if ((tid & 31) == 0) mbar_arrive(empty);
+        return;
+    }
     const int rows = m.nrows, T = p.T, k = p.k, rpc = p.g.rpc;
     const float2* ys = reinterpret_cast<const float2*>(s.ys);
     for (int idx = tid; idx < T * rows; idx += kConsumers) {
@@ -1296,7 +1354,9 @@ __device__ __forceinline__ void do_combine(const SmallParams& p, const SmemPtrs&
 // Main kernel
 // ---------------------------------------------------------------------------
 template <int WBITS, int TM>
-__global__ void __launch_bounds__(kSmallThreads, 1) k_moe_small(const __grid_constant__ SmallParams p) {
+__global__ void __launch_bounds__(Roles<TM>::kThreads, 1) k_moe_small(const __grid_constant__ SmallParams p) {
+    using R = Roles<TM>;
+    constexpr int G = R::kGroups;
     extern __shared__ __align__(128) uint8_t smem_raw[];
     const SmemPtrs s = carve(smem_raw, p.g);
     const SmallGeom& g = p.g;
@@ -1311,20 +1371,22 @@ __global__ void __launch_bounds__(kSmallThreads, 1) k_moe_small(const __grid_con
         }
         mbar_init(s.routing, 1);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&s.ufull[i], kConsumerWarps);
+            mbar_init(&s.ufull[i], kConsumerWarps * g.cpu);  // every warp, every chunk of a unit
             mbar_init(&s.ufree[i], 1);
         }
+        mbar_init(s.gsync, kConsumerWarps);
+        mbar_init(s.gexit, G * kConsumerWarps);
         fence_barrier_init();
     }
     __syncthreads();
 
-    if (warp == kFinisherWarp) {
+    if (warp == R::kFinisherWarp) {
         finisher(p, s, lane);
         return;
     }
-    if (warp == kProducerWarp) {
+    if (warp == R::kProducerWarp) {
         // ------------------------- producer -------------------------
-        Producer pr(p, s, lane);
+        Producer pr(p, s, lane, G);
         const int64_t rowI = (int64_t)p.I * p.wbits / 8;
         if (p.ns && lane == 0 && r1 > r0)
             bulk_prefetch_l2(p.shared.w_down + (int64_t)r0 * rowI, (uint32_t)((r1 - r0) * rowI));
@@ -1342,7 +1404,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1) k_moe_small(const __grid_con
         // (and the control block the prologue reset)
         pdl_wait();
         int ok = 1;
-        if (lane == 0) ok = mbar_wait(s.routing, 0, kConsumerWaitLimit) ? 1 : 0;
+        if (lane == 0) ok = mbar_wait_ns(s.routing, 0, kSlackWaits * p.wait_ns) ? 1 : 0;
         ok = __shfl_sync(kFull, ok, 0);
         __syncwarp();  // lane 0's acquire of the tables orders the other lanes' reads
         if (!ok) pr.fail();
@@ -1386,24 +1448,28 @@ __global__ void __launch_bounds__(kSmallThreads, 1) k_moe_small(const __grid_con
             }
         }
         if (!pr.aborted) {
+            // two groups: the SYNC marker goes to one group, the COMBINE
+            // marker (the next slot) to the other, which waits for it
+            if (G > 1) pr.marker(kItemSync);
             SlotMeta m = pr.blank(kItemCombine);
             m.row0 = r0;
             m.nrows = r1 - r0;
             pr.push(m, no_copy(), no_copy(), no_copy(), no_copy());
         }
-        if (!pr.aborted) pr.marker(kItemDone);
-        if (pr.aborted) pr.finish();
+        pr.finish();  // a DONE marker per group
         pr.drain();
         return;
     }
 
     // ------------------------- consumers -------------------------
+    const int group = warp / kConsumerWarps;     // consumer group
+    const int gtid = tid - group * kConsumers;   // thread index inside the group
     pdl_wait();
     {
         // Q8_0 activations of all tokens into shared memory, each 32-code
         // block split in 16-byte halves so that lanes read consecutive words
         const int nb = p.H / 32;
-        for (int job = tid; job < p.T * nb; job += kConsumers) {
+        for (int job = tid; job < p.T * nb; job += G * kConsumers) {
             const int t = job / nb, b = job % nb;
             const uint4 lo = __ldcg(reinterpret_cast<const uint4*>(p.xq + (int64_t)t * p.H + b * 32));
             const uint4 hi = __ldcg(reinterpret_cast<const uint4*>(p.xq + (int64_t)t * p.H + b * 32 + 16));
@@ -1413,14 +1479,15 @@ __global__ void __launch_bounds__(kSmallThreads, 1) k_moe_small(const __grid_con
             *reinterpret_cast<uint4*>(s.xq + ((size_t)(t * 2 + 0) * nb + b) * 16) = make_uint4(a.v[0], a.v[1], a.v[2], a.v[3]);
             *reinterpret_cast<uint4*>(s.xq + ((size_t)(t * 2 + 1) * nb + b) * 16) = make_uint4(a.v[4], a.v[5], a.v[6], a.v[7]);
         }
-        for (int job = tid; job < p.T * nb; job += kConsumers) s.xd[job] = __ldcg(p.xd + job);
+        for (int job = tid; job < p.T * nb; job += G * kConsumers) s.xd[job] = __ldcg(p.xd + job);
     }
-    consumers_sync();
-    int slot = 0;
+    named_barrier(3, G * kConsumers);  // every consumer warp, before any item
+    // group g takes ring slots g, g + G, ... in order
+    int slot = group;
     uint32_t pf = 0;
-    int uc = 0;  // gate/up units started by this CTA
+    int units = 0;  // the CTA's gate/up units, from the DONE marker (or the last unit seen)
     while (true) {
-        if (!mbar_wait(&s.full[slot], pf, kConsumerWaitLimit)) {
+        if (!mbar_wait_ns(&s.full[slot], pf, kSlackWaits * p.wait_ns)) {
             set_error(p.err, kErrTimeout);
             break;
         }
@@ -1428,36 +1495,54 @@ __global__ void __launch_bounds__(kSmallThreads, 1) k_moe_small(const __grid_con
         uint8_t* data = s.slots + (size_t)slot * g.slot_bytes;
         uint64_t* empty = &s.empty[slot];
         if (m.kind == kItemGateUp) {
-            do_gateup<WBITS, TM>(p, s, m, data, tid, empty, uc);
-            if (m.last) ++uc;
+            do_gateup<WBITS, TM>(p, s, m, data, gtid, empty);
+            units = max(units, m.uc + 1);
         } else if (m.kind == kItemDown) {
-            do_down<WBITS, TM>(p, s, m, data, tid, empty);
+            do_down<WBITS, TM>(p, s, m, data, gtid, empty);
         } else if (m.kind == kItemSelect) {
-            do_select(p, s, data, tid);
+            do_select(p, s, data, gtid);  // always group 0's: the first item
             __syncwarp();
             if (lane == 0) mbar_arrive(empty);  // the slot was the scratch
+        } else if (m.kind == kItemSync) {
+            do_sync(s, gtid, empty);
         } else if (m.kind == kItemCombine) {
-            do_combine(p, s, m, tid, empty);
+            do_combine(p, s, m, gtid, empty, group, G);
         } else {
+            if (m.kind == kItemDone) units = m.uc;
             break;  // DONE (or an unknown marker)
         }
-        if (++slot == g.nslot) {
-            slot = 0;
+        slot += G;
+        if (slot >= g.nslot) {
+            slot = group;
             pf ^= 1u;
         }
     }
-    // no more units: hand the finisher a terminal record (its buffer was last
-    // used by unit uc - 2, which the finisher must have read first)
-    const int buf = uc & 1;
-    if (uc >= 2 && !mbar_wait(&s.ufree[buf], ((uc >> 1) - 1) & 1, kConsumerWaitLimit)) set_error(p.err, kErrTimeout);
-    if (warp == 0 && lane == 0) s.urec[buf] = UnitRec{-1, 0, 0, 0};
+    // No more units: once every consumer warp has left its loop, hand the
+    // finisher a terminal record with the full arrival count (its buffer was
+    // last used by unit units - 2, which the finisher must have read first).
+    if (gtid == 0) s.misc[4 + group] = units;
     __syncwarp();
-    if (lane == 0) mbar_arrive(&s.ufull[buf]);
+    if (lane == 0) mbar_arrive(s.gexit);
+    if (tid == 0) {
+        bool ok = mbar_wait_ns(s.gexit, 0, kSlackWaits * p.wait_ns);
+        int n = s.misc[4];
+        for (int gi = 1; gi < G; ++gi) n = max(n, s.misc[4 + gi]);
+        const int buf = n & 1;
+        if (ok && n >= 2) ok = mbar_wait_ns(&s.ufree[buf], ((n >> 1) - 1) & 1, kSlackWaits * p.wait_ns);
+        if (!ok) set_error(p.err, kErrTimeout);
+        s.urec[buf] = UnitRec{-1, 0, 0, 0};
+        mbar_arrive_count(&s.ufull[buf], (uint32_t)(kConsumerWarps * g.cpu));
+    }
 }
 
 // ---------------------------------------------------------------------------
 // Host launcher
 // ---------------------------------------------------------------------------
+// The persistent kernel's CTAs wait for one another (the down chunks wait for
+// other CTAs' h codes), so the grid must be resident all at once: it is
+// launched as a cooperative grid (one CTA per SM), which the runtime only
+// starts when every CTA can run, also beside another forward on another
+// stream.  It is also the prologue's programmatic dependent.
 template <int WBITS, int TM>
 static cudaError_t launch_small_t(const SmallParams& prm, cudaStream_t st) {
     static bool attr_done[64];
@@ -1468,19 +1553,35 @@ static cudaError_t launch_small_t(const SmallParams& prm, cudaStream_t st) {
         cudaError_t e = cudaFuncSetAttribute(k_moe_small<WBITS, TM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              device_info().max_smem_optin);
         if (e != cudaSuccess) return e;
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_moe_small<WBITS, TM>, Roles<TM>::kThreads,
+                                                          prm.g.smem_bytes);
+        if (e != cudaSuccess) return e;
+        if (per_sm < 1) return cudaErrorInvalidConfiguration;
         attr_done[dev] = true;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(prm.g.grid);
-    cfg.blockDim = dim3(kSmallThreads);
+    cfg.blockDim = dim3(Roles<TM>::kThreads);
     cfg.dynamicSmemBytes = prm.g.smem_bytes;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeCooperative;
+    attr[1].val.cooperative = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, k_moe_small<WBITS, TM>, prm);
+}
+
+// Test hook state (moe_debug_fault_injection): read by every launch.
+static std::atomic<int> g_fault_entry{-1};
+static std::atomic<long long> g_wait_ns{(long long)kWaitNs};
+
+void set_fault_injection(int withhold_entry, int64_t wait_ns) {
+    g_fault_entry.store(withhold_entry < 0 ? -1 : withhold_entry);
+    g_wait_ns.store(wait_ns > 0 ? (long long)wait_ns : (long long)kWaitNs);
 }
 
 cudaError_t launch_small(const SmallArgs& a, cudaStream_t st) {
@@ -1492,9 +1593,14 @@ cudaError_t launch_small(const SmallArgs& a, cudaStream_t st) {
     p.xq = a.xq; p.xd = a.xd; p.logits = a.logits; p.idx = a.idx; p.w = a.w; p.counts = a.counts;
     p.offsets = a.offsets; p.perm = a.perm; p.inv_perm = a.inv_perm; p.active = a.active;
     p.hq = a.hq; p.hd = a.hd; p.y = a.y; p.out = a.out; p.ctrl = a.ctrl; p.err = a.err;
+    p.wait_ns = (uint64_t)g_wait_ns.load();
+    p.fault_entry = g_fault_entry.load();
     p.g = small_geometry(c, a.T, device_info().sm_count);
     if (p.g.smem_bytes > device_info().max_smem_optin) return cudaErrorInvalidConfiguration;
-    k_small_prologue<<<p.g.grid, kPrologueThreads, 0, st>>>(a.x, a.T, c.hidden, c.n_experts, a.router_w, a.logits,
+    // one prologue block per router row (at least one per SM): every row's
+    // loads are issued at once, so the logits take one DRAM round trip
+    const int pro_grid = c.n_experts > p.g.grid ? c.n_experts : p.g.grid;
+    k_small_prologue<<<pro_grid, kPrologueThreads, 0, st>>>(a.x, a.T, c.hidden, c.n_experts, a.router_w, a.logits,
                                                             a.xq, a.xd, a.ctrl, p.g.ctrl_words, a.err);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

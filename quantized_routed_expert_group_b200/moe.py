@@ -59,8 +59,11 @@ _SIGS = {
                                    ctypes.POINTER(MoeExperts), _vp, _vp], _int),
     "moe_workspace_view": ([ctypes.POINTER(MoeConfig), _int, _vp, _sz, ctypes.POINTER(MoeWorkspaceLayout)], _int),
     "moe_block_dots": ([_vp, _i64, _int, _int, _vp, _int, _vp, _vp], _int),
+    "moe_block_dots_routine": ([_vp, _i64, _int, _int, _vp, _int, _int, _vp, _vp], _int),
     "moe_get_device_error": ([_vp, _vp, ctypes.POINTER(ctypes.c_int32)], _int),
+    "moe_noalloc_device_error": ([_vp, ctypes.POINTER(ctypes.c_int32)], _int),
     "moe_synth_normal": ([_u64, _u64, _i64, _i64, _flt, _vp, _vp], _int),
+    "moe_debug_fault_injection": ([_int, _i64], _int),
     "moe_profile_events": ([ctypes.POINTER(_vp), _int], _int),
     "moe_forward_launches": ([ctypes.POINTER(MoeConfig), _int], _int),
     "moe_forward_phases": ([ctypes.POINTER(MoeConfig), _int], _int),
@@ -69,6 +72,9 @@ _SIGS = {
 }
 
 PROFILE_MAX_EVENTS = 8
+# launches of one forward on each path (moe_forward_launches): fused small
+# batch, multi-kernel, batched tensor-core
+SMALL_LAUNCHES, MULTI_KERNEL_LAUNCHES, TC_LAUNCHES = 2, 7, 10
 
 _LIB = None
 
@@ -181,13 +187,27 @@ def bucket_tokens(cfg: MoeConfig, idx: torch.Tensor, stream=None):
     return counts, offsets, perm[: T * cfg.top_k]
 
 
-def block_dots(packed: torch.Tensor, cols: int, wbits: int, q: torch.Tensor, stream=None):
+DOTS_MULTI_KERNEL, DOTS_FUSED, DOTS_TENSOR = 0, 1, 2
+
+
+def block_dots(packed: torch.Tensor, cols: int, wbits: int, q: torch.Tensor, stream=None, routine: int | None = None):
+    """Per-block int32 dots [n][rows][cols/32]; routine None is moe_block_dots,
+    otherwise moe_block_dots_routine with that routine (DOTS_*)."""
     rows = packed.shape[0]
     q2 = q.reshape(-1, cols)
     out = torch.empty((q2.shape[0], rows, cols // 32), dtype=torch.int32, device=packed.device)
-    _check(lib().moe_block_dots(_ptr(packed), rows, cols, wbits, _ptr(q2), q2.shape[0], _ptr(out), _stream(stream)),
-           "block_dots")
+    if routine is None:
+        st = lib().moe_block_dots(_ptr(packed), rows, cols, wbits, _ptr(q2), q2.shape[0], _ptr(out), _stream(stream))
+    else:
+        st = lib().moe_block_dots_routine(_ptr(packed), rows, cols, wbits, _ptr(q2), q2.shape[0], routine, _ptr(out),
+                                          _stream(stream))
+    _check(st, "block_dots")
     return out
+
+
+def debug_fault_injection(withhold_entry: int, wait_budget_ns: int = 0) -> None:
+    """Test hook (see moe_debug_fault_injection): -1 switches it off."""
+    _check(lib().moe_debug_fault_injection(withhold_entry, wait_budget_ns), "debug_fault_injection")
 
 
 def synth_normal(seed: int, tid: int, n: int, sigma: float, offset: int = 0, out: torch.Tensor | None = None,

@@ -123,6 +123,9 @@ def test_other_entry_point_errors(L):
     assert lib.moe_pack_weights(0x1004, 4, 64, 4, 0x1000, 0x1000, None) == -1
     assert lib.moe_block_dots(0x1000, 4, 48, 4, 0x1000, 1, 0x1000, None) == -1
     assert lib.moe_block_dots(0x1000, 4, 64, 3, 0x1000, 1, 0x1000, None) == -2
+    assert lib.moe_block_dots_routine(0x1000, 4, 64, 4, 0x1000, 1, 7, 0x1000, None) == -2   # unknown routine
+    assert lib.moe_block_dots_routine(0x1000, 4, 48, 4, 0x1000, 1, 1, 0x1000, None) == -1   # cols % 32
+    assert lib.moe_block_dots_routine(0x1000, 0, 64, 4, 0x1000, 1, 1, 0x1000, None) == 0    # nothing to do
     assert lib.moe_requant_fp8(0x1000, 0x1000, 4, 48, 128, 4, 0x1000, 0x1000, None) == -1   # cols % 32
     assert lib.moe_requant_fp8(0x1000, 0x1000, 4, 64, 100, 4, 0x1000, 0x1000, None) == -1   # block % 32
     assert lib.moe_requant_fp8(0x1000, 0x1000, 4, 64, 128, 3, 0x1000, 0x1000, None) == -2   # wbits

@@ -35,7 +35,11 @@ def full(request):
 
 
 def _sample_tokens(T):
-    return sorted(set([0, T - 1, T // 2]))[: 3 if T > 64 else 2]
+    """Every token of a batch of at most 16, else 16 spread over the batch
+    (first and last included)."""
+    if T <= 16:
+        return list(range(T))
+    return sorted(set(np.linspace(0, T - 1, 16).round().astype(int).tolist()))
 
 
 def test_full_router_and_bucket(full):
@@ -79,8 +83,45 @@ def test_full_sampled_outputs(full):
     e0 = int(v["idx"][t0, j0])
     ex = routed[e0]
     xq = torch.from_numpy(tr.xq[0:1]).cuda()
-    got = moe.block_dots(layer.routed.w_gate[e0], s.hidden, s.wbits, xq).cpu().numpy()
-    np.testing.assert_array_equal(got, orc.block_dots(ex.wg, s.hidden, s.wbits, tr.xq[0:1]))
+    ref_g = orc.block_dots(ex.wg, s.hidden, s.wbits, tr.xq[0:1])
     hq = np.ascontiguousarray(tr.hq[0, j0:j0 + 1])
-    got = moe.block_dots(layer.routed.w_down[e0], s.inter, s.wbits, torch.from_numpy(hq).cuda()).cpu().numpy()
-    np.testing.assert_array_equal(got, orc.block_dots(ex.wd, s.inter, s.wbits, hq))
+    ref_d = orc.block_dots(ex.wd, s.inter, s.wbits, hq)
+    factor = {8: 1, 4: 16, 2: 64}[s.wbits]
+    for routine, f in ((None, 1), (moe.DOTS_FUSED, factor)):
+        got = moe.block_dots(layer.routed.w_gate[e0], s.hidden, s.wbits, xq, routine=routine).cpu().numpy()
+        np.testing.assert_array_equal(got.astype(np.int64), f * ref_g.astype(np.int64))
+        got = moe.block_dots(layer.routed.w_down[e0], s.inter, s.wbits, torch.from_numpy(hq).cuda(),
+                             routine=routine).cpu().numpy()
+        np.testing.assert_array_equal(got.astype(np.int64), f * ref_d.astype(np.int64))
+
+
+def test_full_hot_expert_slots(full):
+    """Per-slot expert outputs y (before the combine) of EVERY token routed to
+    the two most loaded experts, and of the shared expert on every token,
+    against the oracle's expert FFN on the oracle's own Q8_0 codes of x."""
+    wl, layer, x, out, v = full
+    s = wl.shape
+    if wl.T < 2:
+        pytest.skip("one token: the sampled-output test covers every slot")
+    counts, offsets, perm = v["counts"], v["offsets"], v["perm"]
+    hot = [int(e) for e in np.argsort(-counts, kind="stable")[:2] if counts[e] > 0]
+    xq, xd = orc.q8_0_quantize(x)
+    checked = 0
+    for e in hot:
+        ex = orc.pack_expert(*host_expert_mats(wl, e), s.wbits)
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        toks = perm[lo:hi] // s.top_k
+        ref = np.stack([orc.expert_ffn(ex, s.hidden, s.inter, s.wbits, xq[t], xd[t])[0] for t in toks])
+        err = rel_rms_err(v["y"][lo:hi], ref)
+        print(wl.name, "expert", e, "tokens", hi - lo, "y err / rms =", err)
+        assert err <= OUT_TOL
+        checked += hi - lo
+    if s.n_shared:
+        sh = orc.pack_expert(*host_expert_mats(wl, 0, shared=True), s.wbits)
+        base = wl.T * s.top_k
+        ref = np.stack([orc.expert_ffn(sh, s.hidden, s.inter, s.wbits, xq[t], xd[t])[0] for t in range(wl.T)])
+        err = rel_rms_err(v["y"][base:base + wl.T], ref)
+        print(wl.name, "shared expert y err / rms =", err)
+        assert err <= OUT_TOL
+        checked += wl.T
+    assert checked >= min(wl.T, 16)

@@ -66,6 +66,78 @@ def test_block_dots_bitexact(wbits, rows, cols, n):
     np.testing.assert_array_equal(got.cpu().numpy(), orc.block_dots(po, cols, wbits, q))
 
 
+# The factor each routine's stored value carries (see moe_block_dots_routine).
+DOT_FACTOR = {(moe.DOTS_MULTI_KERNEL, 8): 1, (moe.DOTS_MULTI_KERNEL, 4): 1, (moe.DOTS_MULTI_KERNEL, 2): 1,
+              (moe.DOTS_FUSED, 8): 1, (moe.DOTS_FUSED, 4): 16, (moe.DOTS_FUSED, 2): 64,
+              (moe.DOTS_TENSOR, 8): 1, (moe.DOTS_TENSOR, 4): 1, (moe.DOTS_TENSOR, 2): 1}
+
+
+def _random_dot_inputs(wbits, rows, cols, n, seed):
+    """Random packed bytes (every nibble / 2-bit field, including the codes -8
+    and -2 that the quantiser never writes) and int8 codes in [-127, 127] with
+    saturated blocks: rows 0-1 all -8 / -2 codes, row 2 all +7 / +1, block 0 of
+    token 0 all +127, the last block of the last token all -127, one block
+    alternating +-127."""
+    rng = np.random.default_rng(seed)
+    packed = rng.integers(0, 256, size=(rows, cols * wbits // 8), dtype=np.uint8)
+    lowest = {8: 0x80, 4: 0x88, 2: 0xAA}[wbits]
+    highest = {8: 0x7F, 4: 0x77, 2: 0x55}[wbits]
+    packed[0] = lowest
+    packed[1 % rows] = lowest
+    packed[2 % rows] = highest
+    q = rng.integers(-127, 128, size=(n, cols)).astype(np.int8)
+    q[0, :32] = 127
+    q[-1, -32:] = -127
+    if cols >= 96:
+        q[0, 64:96] = np.where(np.arange(32) % 2 == 0, 127, -127)
+    return packed, q
+
+
+@pytest.mark.parametrize("routine", [moe.DOTS_MULTI_KERNEL, moe.DOTS_FUSED])
+@pytest.mark.parametrize("wbits", [8, 4, 2])
+@pytest.mark.parametrize("rows,cols,n", [(48, 6144, 2), (37, 2048, 4), (5, 96, 3)])
+def test_dot_routines_random_bytes(routine, wbits, rows, cols, n):
+    """Each device dot routine the kernels call, bit-exact against the oracle's
+    brute-force block dots on arbitrary packed bytes; the fused routine's
+    scaled value is checked as the exact product first."""
+    packed, q = _random_dot_inputs(wbits, rows, cols, n, seed=rows * 7 + cols + wbits + 100 * routine)
+    ref = orc.block_dots(packed, cols, wbits, q).astype(np.int64)
+    got = moe.block_dots(torch.from_numpy(packed).cuda(), cols, wbits, torch.from_numpy(q).cuda(),
+                         routine=routine).cpu().numpy().astype(np.int64)
+    f = DOT_FACTOR[(routine, wbits)]
+    np.testing.assert_array_equal(got, f * ref)
+    np.testing.assert_array_equal(got // f, ref)
+    # the saturated rows reach the extremes the routines must carry exactly
+    assert np.abs(ref).max() >= 32 * 127 * {8: 128, 4: 8, 2: 2}[wbits] // 2
+
+
+@pytest.mark.parametrize("wbits", [8, 4, 2])
+@pytest.mark.parametrize("rows,cols,n", [(128, 128, 16), (300, 6144, 64), (77, 2048, 17), (200, 192, 1),
+                                         (129, 320, 48)])
+def test_tensor_dot_routine_random_bytes(wbits, rows, cols, n):
+    """The tensor-core routine (widening in shared memory, one kind::i8 MMA per
+    Q8_0 block, int32 read back from TMEM), bit-exact against the oracle on
+    arbitrary packed bytes: ragged row tiles (77, 129, 300 rows), partial
+    last stages (192, 320 codes), token counts that are not multiples of 16."""
+    if (cols * wbits // 8) % 16:
+        pytest.skip("rows of the tensor routine are multiples of 16 bytes")
+    packed, q = _random_dot_inputs(wbits, rows, cols, n, seed=rows * 11 + cols + wbits + n)
+    ref = orc.block_dots(packed, cols, wbits, q)
+    got = moe.block_dots(torch.from_numpy(packed).cuda(), cols, wbits, torch.from_numpy(q).cuda(),
+                         routine=moe.DOTS_TENSOR).cpu().numpy()
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_tensor_dot_routine_limits():
+    p = torch.zeros((4, 64), dtype=torch.uint8, device="cuda")
+    q = torch.zeros((65, 128), dtype=torch.int8, device="cuda")
+    with pytest.raises(moe.MoeError):
+        moe.block_dots(p, 128, 4, q, routine=moe.DOTS_TENSOR)  # more than 64 tokens
+    p2 = torch.zeros((4, 8), dtype=torch.uint8, device="cuda")
+    with pytest.raises(moe.MoeError):
+        moe.block_dots(p2, 32, 2, q[:1, :32].contiguous(), routine=moe.DOTS_TENSOR)  # 8-byte rows
+
+
 def _router_case(name, T):
     wl = synth.WORKLOADS[name].with_tokens(T)
     return wl, synth.make_x(wl), synth.make_router_w(wl), synth.make_bias(wl)

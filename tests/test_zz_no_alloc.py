@@ -47,8 +47,14 @@ def test_noalloc_matches_workspace_forward_twice(shape, T):
         out = torch.full_like(x, float("nan"))
         assert _call(layer, x, out) == moe.MOE_OK
         torch.cuda.synchronize()
+        code = ctypes.c_int32(-1)
+        assert moe.lib().moe_noalloc_device_error(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream),
+                                                  ctypes.byref(code)) == moe.MOE_OK
+        assert code.value == 0
         assert torch.isfinite(out).all()
         assert rel_rms_err(out.cpu().numpy(), ref.cpu().numpy()) <= OUT_TOL
+        # the same deterministic kernels on the same inputs: bit-identical
+        assert torch.equal(out, ref)
 
 
 def test_noalloc_rejects_batches_beyond_its_scratch():
