@@ -195,6 +195,28 @@ int moe_layer_forward(const moe_config *cfg, const float *x, int T, const float 
                       const float *router_bias, const moe_experts *routed, const moe_experts *shared,
                       float *out, void *workspace, size_t ws_bytes, void *stream);
 
+/* Expert-parallel share of moe_layer_forward (the pages' multi-GPU expert
+ * tier, [WP] "Multi-GPU expert tier": experts spread over GPUs).  Every rank
+ * routes all tokens exactly as moe_layer_forward does, then computes only the
+ * picks whose expert lies in [expert_lo, expert_hi), and the shared expert
+ * when with_shared is 1:
+ *   out[t] = sum over those picks j of w[t,j] * y_{idx[t,j]}(t)
+ *            (+ y_shared(t) when with_shared)
+ * so the layer's output is the sum of the ranks' outputs when their ranges
+ * cover [0, n_experts) without overlap and exactly one rank adds the shared
+ * expert (each rank's sum is rounded to fp32 before that cross-rank sum).
+ * Only the experts of the range (and the shared expert when with_shared) are
+ * read: `routed` may point at a bank of which only those experts exist, as
+ * long as expert e's data sits where it would in a full bank.  Arguments,
+ * workspace (the full layer's: moe_workspace_bytes(cfg, T)) and errors as
+ * for moe_layer_forward; 0 <= expert_lo <= expert_hi <= n_experts and
+ * with_shared 0 or 1, else MOE_EINVAL.  The workspace view then describes
+ * this call: idx / w the full routing, the buckets only the range's picks. */
+int moe_layer_forward_partial(const moe_config *cfg, const float *x, int T, const float *router_w,
+                              const float *router_bias, const moe_experts *routed, const moe_experts *shared,
+                              int expert_lo, int expert_hi, int with_shared, float *out, void *workspace,
+                              size_t ws_bytes, void *stream);
+
 /* moe_layer_forward with HOST activations: copies x_host [T][hidden] to the
  * workspace, runs the forward, copies the result to out_host [T][hidden] and
  * synchronises `stream`.  Host buffers should be pinned (cudaHostAlloc) for

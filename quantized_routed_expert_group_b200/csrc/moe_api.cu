@@ -32,6 +32,7 @@ Layout make_layout(const moe_config& c, int T) {
     L.xd = take(t * (H / 32) * 4);
     L.logits = take(router_ws_bytes(c, T));
     L.idx = take(t * k * 4);
+    L.idx_ep = take(t * k * 4);
     L.w = take(t * k * 4);
     L.counts = take(E * 4);
     L.offsets = take((E + 1) * 4);
@@ -140,9 +141,11 @@ static int check_bucket_fits(const moe_config& c, int T) {
 }
 
 // The forward on a device-resident x; used by both public forwards.
+// ep_lo, ep_hi: the routed experts this call computes (all: 0, n_experts);
+// the picks outside the range are routed as usual but left to another call.
 static int forward_device(const moe_config& c, const float* x, int T, const float* router_w,
                           const float* router_bias, const moe_experts& routed, const moe_experts* shared,
-                          float* out, char* ws, const Layout& L, cudaStream_t s) {
+                          float* out, char* ws, const Layout& L, cudaStream_t s, int ep_lo, int ep_hi) {
     int32_t* err = reinterpret_cast<int32_t*>(ws + L.err);
     int8_t* xq = reinterpret_cast<int8_t*>(ws + L.xq);
     float* xd = reinterpret_cast<float*>(ws + L.xd);
@@ -180,6 +183,8 @@ static int forward_device(const moe_config& c, const float* x, int T, const floa
         a.out = out;
         a.ctrl = reinterpret_cast<int*>(ws + L.ctrl);
         a.err = err;
+        a.ep_lo = ep_lo;
+        a.ep_hi = ep_hi;
         int st2 = status_of(trace(0, s));
         if (!st2) st2 = status_of(launch_small(a, s));
         if (!st2) st2 = status_of(trace(1, s));
@@ -193,7 +198,14 @@ static int forward_device(const moe_config& c, const float* x, int T, const floa
     st = status_of(launch_router(c, x, T, router_w, router_bias, reinterpret_cast<double*>(ws + L.logits), idx, w, s));
     if (!st) st = status_of(trace(1, s));
     if (st) return st;
-    st = status_of(launch_bucket(c, idx, T, counts, offsets, perm, inv_perm, active, err, s));
+    const int32_t* bidx = idx;  // the picks this call computes
+    if (ep_lo > 0 || ep_hi < c.n_experts) {
+        int32_t* idx_ep = reinterpret_cast<int32_t*>(ws + L.idx_ep);
+        st = status_of(launch_ep_mask(idx, (int64_t)T * c.top_k, ep_lo, ep_hi, idx_ep, s));
+        if (st) return st;
+        bidx = idx_ep;
+    }
+    st = status_of(launch_bucket(c, bidx, T, counts, offsets, perm, inv_perm, active, err, s));
     if (st) return st;
     const bool tc = tc_path_supported(c, T);
     TcArgs ta{};
@@ -340,7 +352,30 @@ MOE_API int moe_layer_forward(const moe_config* cfg, const float* x, int T, cons
     if (T == 0) return MOE_OK;
     if (!aligned(x, 16) || !aligned(out, 4)) return MOE_EINVAL;
     return forward_device(*cfg, x, T, router_w, router_bias, *routed, cfg->n_shared ? shared : nullptr, out,
-                          static_cast<char*>(workspace), L, (cudaStream_t)stream);
+                          static_cast<char*>(workspace), L, (cudaStream_t)stream, 0, cfg->n_experts);
+}
+
+MOE_API int moe_layer_forward_partial(const moe_config* cfg, const float* x, int T, const float* router_w,
+                                      const float* router_bias, const moe_experts* routed, const moe_experts* shared,
+                                      int expert_lo, int expert_hi, int with_shared, float* out, void* workspace,
+                                      size_t ws_bytes, void* stream) {
+    int st = check_config(cfg);
+    if (st) return st;
+    if (expert_lo < 0 || expert_hi < expert_lo || expert_hi > cfg->n_experts) return MOE_EINVAL;
+    if (with_shared != 0 && with_shared != 1) return MOE_EINVAL;
+    moe_config c = *cfg;  // the shared expert only where this call adds it
+    if (!with_shared) c.n_shared = 0;
+    // the workspace is the full layer's (it is at least this call's)
+    Layout L;
+    st = check_forward_args(cfg, x, T, router_w, router_bias, routed, with_shared ? shared : routed, out, workspace,
+                            ws_bytes, &L);
+    if (st) return st;
+    if (T == 0) return MOE_OK;
+    if (!aligned(x, 16) || !aligned(out, 4)) return MOE_EINVAL;
+    // the full layer's layout (every region is at least this call's), so
+    // moe_workspace_view(cfg, T) describes this call's intermediates too
+    return forward_device(c, x, T, router_w, router_bias, *routed, c.n_shared ? shared : nullptr, out,
+                          static_cast<char*>(workspace), L, (cudaStream_t)stream, expert_lo, expert_hi);
 }
 
 MOE_API int moe_layer_forward_host(const moe_config* cfg, const float* x_host, int T, const float* router_w,
@@ -358,7 +393,7 @@ MOE_API int moe_layer_forward_host(const moe_config* cfg, const float* x_host, i
     float* odev = reinterpret_cast<float*>(ws + L.outbuf);
     if (cudaMemcpyAsync(xdev, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return MOE_ECUDA;
     st = forward_device(*cfg, xdev, T, router_w, router_bias, *routed, cfg->n_shared ? shared : nullptr, odev, ws, L,
-                        s);
+                        s, 0, cfg->n_experts);
     if (st) return st;
     if (cudaMemcpyAsync(out_host, odev, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ECUDA;
     return status_of(cudaStreamSynchronize(s));
@@ -416,7 +451,7 @@ MOE_API int moe_layer_forward_noalloc(const moe_config* cfg, const float* x, int
     if (T == 0) return MOE_OK;
     if (!aligned(x, 16) || !aligned(out, 4)) return MOE_EINVAL;
     return forward_device(*cfg, x, T, router_w, router_bias, *routed, cfg->n_shared ? shared : nullptr, out,
-                          static_cast<char*>(scratch), L, (cudaStream_t)stream);
+                          static_cast<char*>(scratch), L, (cudaStream_t)stream, 0, cfg->n_experts);
 }
 
 MOE_API int moe_noalloc_device_error(void* stream, int32_t* code) {

@@ -129,4 +129,18 @@ cudaError_t launch_bucket(const moe_config& c, const int32_t* idx, int T, int32_
     return cudaGetLastError();
 }
 
+__global__ void k_ep_mask(const int32_t* __restrict__ idx, int64_t n, int lo, int hi, int32_t* __restrict__ out) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int e = idx[i];
+        out[i] = (e >= lo && e < hi) ? e : -1;
+    }
+}
+
+cudaError_t launch_ep_mask(const int32_t* idx, int64_t n, int lo, int hi, int32_t* idx_ep, cudaStream_t s) {
+    if (n == 0) return cudaSuccess;
+    const int64_t want = (n + 255) / 256;
+    k_ep_mask<<<(int)(want < 1024 ? want : 1024), 256, 0, s>>>(idx, n, lo, hi, idx_ep);
+    return cudaGetLastError();
+}
+
 }  // namespace moe

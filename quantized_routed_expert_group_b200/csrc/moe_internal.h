@@ -20,6 +20,7 @@ struct Layout {
     size_t xd;         // fp32 [T][H/32]
     size_t logits;     // fp64 [T][E]
     size_t idx;        // int32 [T][k]
+    size_t idx_ep;     // int32 [T][k]  idx with the picks outside this call's expert range as -1
     size_t w;          // fp32 [T][k]
     size_t counts;     // int32 [E]
     size_t offsets;    // int32 [E+1]
@@ -57,6 +58,8 @@ constexpr int kRouterTiledMinTokens = 64;
 size_t router_ws_bytes(const moe_config& c, int T);
 cudaError_t launch_router(const moe_config& c, const float* x, int T, const float* router_w,
                           const float* bias, double* logits, int32_t* idx, float* w, cudaStream_t s);
+// idx_ep = idx with every pick outside [lo, hi) replaced by -1.
+cudaError_t launch_ep_mask(const int32_t* idx, int64_t n, int lo, int hi, int32_t* idx_ep, cudaStream_t s);
 cudaError_t launch_bucket(const moe_config& c, const int32_t* idx, int T, int32_t* counts,
                           int32_t* offsets, int32_t* perm, int32_t* inv_perm, int32_t* active,
                           int32_t* err, cudaStream_t s);
@@ -140,6 +143,7 @@ struct SmallArgs {
     float* out;
     int* ctrl;
     int32_t* err;
+    int ep_lo, ep_hi;  // routed experts computed by this call: [ep_lo, ep_hi)
 };
 bool small_path_supported(const moe_config& c, int T);
 size_t small_ctrl_bytes(const moe_config& c, int T);

@@ -145,6 +145,7 @@ struct SmallParams {
     int T, H, I, E, G, tg, k, ns, wbits;
     float rsf;
     float topp;  // adaptive expert top-p; outside (0, 1): keep every pick
+    int ep_lo, ep_hi;  // routed experts this call computes (expert parallelism): [ep_lo, ep_hi)
     const float* x;
     const float* router_w;
     const float* bias;
@@ -877,6 +878,30 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
         }
         consumers_sync();
     }
+    // 4c. expert parallelism: the picks outside [ep_lo, ep_hi) are computed by
+    // another call; the routing and the weights are published as they are,
+    // then those picks leave sel as -1 (in no bucket, skipped by the combine)
+    const bool ep_on = p.ep_lo > 0 || p.ep_hi < E;
+    if (ep_on) {
+        if (!topp_on && warp < T && lane < k) {
+            const int t = warp;
+            double ssum = 0.0;
+            for (int j = 0; j < k; ++j) ssum += ss[(size_t)t * E + sel[t * 32 + j]];
+            const int e = sel[t * 32 + lane];
+            const float wv = (float)(ss[(size_t)t * E + e] / ssum * (double)p.rsf);
+            s.selw[t * k + lane] = wv;
+            if (publish) {
+                p.idx[(int64_t)t * k + lane] = e;
+                p.w[(int64_t)t * k + lane] = wv;
+            }
+        }
+        consumers_sync();
+        if (warp < T && lane < k) {
+            const int e = sel[warp * 32 + lane];
+            if (e >= 0 && (e < p.ep_lo || e >= p.ep_hi)) sel[warp * 32 + lane] = -1;
+        }
+        consumers_sync();
+    }
     // 5. bucketing (a dropped pick, sel -1, is in no bucket: inv -1)
     const int n = T * k;
     if (n <= 32) {
@@ -1037,7 +1062,7 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
     }
     // routing weights from the unbiased sigmoid, summed in pick order (with the
     // top-p they were written before the bucketing)
-    if (!topp_on && warp < T && lane < k) {
+    if (!topp_on && !ep_on && warp < T && lane < k) {
         const int t = warp;
         double ssum = 0.0;
 #pragma unroll 8
@@ -1589,6 +1614,7 @@ cudaError_t launch_small(const SmallArgs& a, cudaStream_t st) {
     SmallParams p;
     p.T = a.T; p.H = c.hidden; p.I = c.inter; p.E = c.n_experts; p.G = c.n_groups; p.tg = c.topk_groups;
     p.k = c.top_k; p.ns = c.n_shared; p.wbits = c.wbits; p.rsf = c.routed_scaling_factor; p.topp = c.expert_topp;
+    p.ep_lo = a.ep_lo; p.ep_hi = a.ep_hi;
     p.x = a.x; p.router_w = a.router_w; p.bias = a.bias; p.routed = a.routed; p.shared = a.shared;
     p.xq = a.xq; p.xd = a.xd; p.logits = a.logits; p.idx = a.idx; p.w = a.w; p.counts = a.counts;
     p.offsets = a.offsets; p.perm = a.perm; p.inv_perm = a.inv_perm; p.active = a.active;

@@ -53,6 +53,8 @@ _SIGS = {
     "moe_workspace_bytes": ([ctypes.POINTER(MoeConfig), _int], _sz),
     "moe_layer_forward": ([ctypes.POINTER(MoeConfig), _vp, _int, _vp, _vp, ctypes.POINTER(MoeExperts),
                            ctypes.POINTER(MoeExperts), _vp, _vp, _sz, _vp], _int),
+    "moe_layer_forward_partial": ([ctypes.POINTER(MoeConfig), _vp, _int, _vp, _vp, ctypes.POINTER(MoeExperts),
+                                   ctypes.POINTER(MoeExperts), _int, _int, _int, _vp, _vp, _sz, _vp], _int),
     "moe_layer_forward_host": ([ctypes.POINTER(MoeConfig), _vp, _int, _vp, _vp, ctypes.POINTER(MoeExperts),
                                 ctypes.POINTER(MoeExperts), _vp, _vp, _sz, _vp], _int),
     "moe_layer_forward_noalloc": ([ctypes.POINTER(MoeConfig), _vp, _int, _vp, _vp, ctypes.POINTER(MoeExperts),
@@ -358,6 +360,24 @@ class MoeLayer:
                                        ctypes.byref(self._routed_s), ctypes.byref(self._shared_s), _ptr(out),
                                        _ptr(self.workspace), self.workspace.numel(), _stream(stream)),
                "layer_forward")
+        return out
+
+    def forward_partial(self, x: torch.Tensor, expert_lo: int, expert_hi: int, with_shared: bool,
+                        out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """The share of the layer output of the routed experts in
+        [expert_lo, expert_hi) (+ the shared expert when with_shared), see
+        moe_layer_forward_partial."""
+        _cuda(x, torch.float32, "x")
+        T = x.shape[0]
+        if T > self.T_max:
+            raise ValueError(f"T={T} exceeds the workspace's T_max={self.T_max}")
+        if out is None:
+            out = torch.empty_like(x)
+        _check(lib().moe_layer_forward_partial(ctypes.byref(self.cfg), _ptr(x), T, _ptr(self.router_w),
+                                               _ptr(self.bias), ctypes.byref(self._routed_s),
+                                               ctypes.byref(self._shared_s), expert_lo, expert_hi,
+                                               1 if with_shared else 0, _ptr(out), _ptr(self.workspace),
+                                               self.workspace.numel(), _stream(stream)), "layer_forward_partial")
         return out
 
     def forward_noalloc(self, x: torch.Tensor, out: torch.Tensor, stream=None) -> torch.Tensor:

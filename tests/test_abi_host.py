@@ -123,6 +123,13 @@ def test_other_entry_point_errors(L):
     assert lib.moe_pack_weights(0x1004, 4, 64, 4, 0x1000, 0x1000, None) == -1
     assert lib.moe_block_dots(0x1000, 4, 48, 4, 0x1000, 1, 0x1000, None) == -1
     assert lib.moe_block_dots(0x1000, 4, 64, 3, 0x1000, 1, 0x1000, None) == -2
+    ex = L.MoeExperts(*([0x1000] * 6))
+    big = 1 << 40
+    for lo, hi, sh in ((-1, 3, 1), (4, 3, 1), (0, c.n_experts + 1, 1), (0, 3, 2)):
+        assert lib.moe_layer_forward_partial(ctypes.byref(c), 0x1000, 1, 0x1000, 0x1000, ctypes.byref(ex),
+                                             ctypes.byref(ex), lo, hi, sh, 0x1000, 0x1000, big, None) == -1
+    assert lib.moe_layer_forward_partial(ctypes.byref(c), 0x1000, 0, 0x1000, 0x1000, ctypes.byref(ex),
+                                         ctypes.byref(ex), 0, 3, 0, 0x1000, 0x1000, big, None) == 0  # T = 0
     assert lib.moe_block_dots_routine(0x1000, 4, 64, 4, 0x1000, 1, 7, 0x1000, None) == -2   # unknown routine
     assert lib.moe_block_dots_routine(0x1000, 4, 48, 4, 0x1000, 1, 1, 0x1000, None) == -1   # cols % 32
     assert lib.moe_block_dots_routine(0x1000, 0, 64, 4, 0x1000, 1, 1, 0x1000, None) == 0    # nothing to do
