@@ -206,6 +206,28 @@ def step_stats(ms: list[float]) -> dict:
             "min": round(min(ms), 5), "max": round(max(ms), 5)}
 
 
+def capture_graphs(torch, layer, xs, out):
+    """One CUDA graph per token batch (the layer's forward on it), or [] if
+    the capture fails (the steps then run eagerly)."""
+    graphs = []
+    try:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for x in xs:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=side):
+                    layer.forward(x, out)
+                graphs.append(g)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+    except Exception as exc:  # noqa: BLE001
+        print(f"graph capture unavailable ({exc}); timing eager steps", file=sys.stderr)
+        torch.cuda.synchronize()
+        return []
+    return graphs
+
+
 def run_ours(args) -> dict | None:
     import torch
     import torch.distributed as dist
@@ -235,13 +257,21 @@ def run_ours(args) -> dict | None:
     torch.cuda.synchronize()
     assert layer.device_error() == 0
 
+    # one CUDA graph per token batch: a timed step is one graph replay, so the
+    # device runs the step's launches back to back whatever the host's pace
+    graphs = capture_graphs(torch, layer, xs, out)
+    for i in range(args.warmup):
+        if graphs:
+            graphs[i % R].replay()
+        else:
+            layer.forward(xs[i % R], out)
+    torch.cuda.synchronize()
+
     K = args.steps
     phases = moe.forward_phases(layer.cfg, wl.T)
     P = len(phases)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.PROFILE_MAX_EVENTS)] for _ in range(K)]
-    for row in evs:  # torch creates the CUDA event on first record
-        for ev in row:
-            ev.record()
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     gpu_uuid = None
     try:
         gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
@@ -255,16 +285,32 @@ def run_ours(args) -> dict | None:
     sampler = ClockSampler(gpu_uuid)
     time.sleep(0.15)
     for i in range(K):
-        moe.profile_events(evs[i])
-        layer.forward(xs[i % R], out)
-    moe.profile_events(None)
+        ev_s[i].record()
+        if graphs:
+            graphs[i % R].replay()
+        else:
+            layer.forward(xs[i % R], out)
+        ev_e[i].record()
     torch.cuda.synchronize()
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
-    step_ms = [evs[i][0].elapsed_time(evs[i][P]) for i in range(K)]
-    phase_ms = [[evs[i][p].elapsed_time(evs[i][p + 1]) for i in range(K)] for p in range(P)]
+    step_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(K)]
     total_ms = sum(step_ms)
+    assert layer.device_error() == 0
+    # the phases (library events at the phase boundaries), from eager steps
+    K_p = min(K, 200)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.PROFILE_MAX_EVENTS)] for _ in range(K_p)]
+    for row in evs:  # torch creates the CUDA event on first record
+        for ev in row:
+            ev.record()
+    torch.cuda.synchronize()
+    for i in range(K_p):
+        moe.profile_events(evs[i])
+        layer.forward(xs[i % R], out)
+    moe.profile_events(None)
+    torch.cuda.synchronize()
+    phase_ms = [[evs[i][p].elapsed_time(evs[i][p + 1]) for i in range(K_p)] for p in range(P)]
     max_total = reduce_max(total_ms, dev)
     value = throughput(wl.T, K, world, max_total)
     # active experts of each rotation (the bytes a step streams)
@@ -288,7 +334,10 @@ def run_ours(args) -> dict | None:
             if flush_l2:
                 flush.fill_(i & 0xFF)
             ev[i][0].record()
-            layer.forward(xs[0], out)
+            if graphs:
+                graphs[0].replay()
+            else:
+                layer.forward(xs[0], out)
             ev[i][1].record()
         torch.cuda.synchronize()
         return [ev[i][0].elapsed_time(ev[i][1]) for i in range(K_v)]
@@ -318,9 +367,9 @@ def run_ours(args) -> dict | None:
     tensor = None
     if phases == ["fused"]:
         # the fused phase: the prologue (Q8_0 of x, router logits over the
-        # router weights) and the persistent kernel (the experts); bytes and
-        # ncu traffic cover both
-        dom_kernel, dom_ms = "k_moe_small", statistics.mean(phase_ms[0])
+        # router weights) and the persistent kernel (the experts) are the whole
+        # step, timed as graph replays; bytes and ncu traffic cover both
+        dom_kernel, dom_ms = "k_moe_small", ms_step
         dom_bytes = layer_bytes + router_bytes
     else:
         gu_ms = statistics.mean(phase_ms[phases.index("gate_up")])
@@ -349,6 +398,8 @@ def run_ours(args) -> dict | None:
                    "experts": s.n_experts, "top_k": s.top_k, "shared": s.n_shared, "weights": f"int{s.wbits}",
                    "activations": "Q8_0 int8", "unique_experts_per_step": round(mean_active, 2),
                    "token_batches": f"{R} seeded batches, step i uses batch i mod {R}",
+                   "timing": ("CUDA-event pair around each step's CUDA-graph replay" if graphs else
+                              "CUDA-event pair around each step (graph capture unavailable)"),
                    "l2": ("not flushed: every step streams its selected experts' weights, more than L2 holds, "
                           "and consecutive steps select different experts"),
                    "parallelism": f"replicas x{world}"},

@@ -358,9 +358,10 @@ int moe_synth_normal(uint64_t seed, uint64_t tid, int64_t offset, int64_t n, flo
  * from that thread records events[0] on its stream before its first launch
  * and events[i] after phase i, for i = 1 .. moe_forward_phases(cfg, T).  The
  * phases depend on the path the forward takes: the fused small-batch path
- * (T <= 4) has one phase, "fused" (both of its kernels); the multi-kernel path
- * has five: "route" (Q8_0 of x, logits, selection), "bucket", "gate_up",
- * "down", "combine".  The caller keeps the events alive until they have
+ * (T <= 4) has one phase, "fused" (both of its kernels); the other paths have
+ * five: "route" (Q8_0 of x, logits, selection), "bucket" (with, at T >= 64,
+ * the tensor-core path's plan and gather), "gate_up" (the gate/up kernel),
+ * "down" (at T >= 64 SwiGLU and the down GEMM), "combine".  The caller keeps the events alive until they have
  * completed. */
 #define MOE_PROFILE_MAX_EVENTS 8
 int moe_profile_events(void *const *events, int n_events);

@@ -47,6 +47,19 @@
 
 namespace moe {
 
+// Build options of the one-token schedule (tuning knobs; the defaults are
+// the measured best): consumer groups, cooperative launch, one prologue block
+// per router row.
+#ifndef MOE_SMALL_GROUPS
+#define MOE_SMALL_GROUPS 2
+#endif
+#ifndef MOE_SMALL_COOPERATIVE
+#define MOE_SMALL_COOPERATIVE 1
+#endif
+#ifndef MOE_PROLOGUE_ROW_BLOCKS
+#define MOE_PROLOGUE_ROW_BLOCKS 1
+#endif
+
 constexpr int kConsumerWarps = 8;  // warps of one consumer group
 constexpr int kConsumers = kConsumerWarps * 32;
 // Warp roles: kGroups groups of consumer warps (two at one token, where the
@@ -55,7 +68,7 @@ constexpr int kConsumers = kConsumerWarps * 32;
 // gate/up units).
 template <int TM>
 struct Roles {
-    static constexpr int kGroups = TM == 1 ? 2 : 1;
+    static constexpr int kGroups = TM == 1 ? MOE_SMALL_GROUPS : 1;
     static constexpr int kProducerWarp = kGroups * kConsumerWarps;
     static constexpr int kFinisherWarp = kProducerWarp + 1;
     static constexpr int kThreads = (kFinisherWarp + 1) * 32;
@@ -1596,7 +1609,7 @@ static cudaError_t launch_small_t(const SmallParams& prm, cudaStream_t st) {
     attr[1].id = cudaLaunchAttributeCooperative;
     attr[1].val.cooperative = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 2;
+    cfg.numAttrs = MOE_SMALL_COOPERATIVE ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, k_moe_small<WBITS, TM>, prm);
 }
 
@@ -1625,7 +1638,7 @@ cudaError_t launch_small(const SmallArgs& a, cudaStream_t st) {
     if (p.g.smem_bytes > device_info().max_smem_optin) return cudaErrorInvalidConfiguration;
     // one prologue block per router row (at least one per SM): every row's
     // loads are issued at once, so the logits take one DRAM round trip
-    const int pro_grid = c.n_experts > p.g.grid ? c.n_experts : p.g.grid;
+    const int pro_grid = (MOE_PROLOGUE_ROW_BLOCKS && c.n_experts > p.g.grid) ? c.n_experts : p.g.grid;
     k_small_prologue<<<pro_grid, kPrologueThreads, 0, st>>>(a.x, a.T, c.hidden, c.n_experts, a.router_w, a.logits,
                                                             a.xq, a.xd, a.ctrl, p.g.ctrl_words, a.err);
     cudaError_t e = cudaGetLastError();

@@ -43,11 +43,15 @@ def make_workload(name: str, shape: synth.LayerShape, T: int, seed: int, **kw) -
     return synth.Workload(name, shape, T, seed, **kw)
 
 
-def build_pair(wl: synth.Workload, T_max: int | None = None, device="cuda") -> Pair:
+def build_pair(wl: synth.Workload, T_max: int | None = None, device="cuda", mutate=None) -> Pair:
+    """mutate(mats, shared_mats), if given, edits the fp32 matrices (tuples
+    of gate, up, down arrays) in place before either side packs them."""
     s = wl.shape
     x, Wr, bias = synth.make_x(wl), synth.make_router_w(wl), synth.make_bias(wl)
     mats = {e: tuple(synth.make_expert_matrix(wl, e, m) for m in range(3)) for e in range(s.n_experts)}
     shm = tuple(synth.make_expert_matrix(wl, 0, m, shared=True) for m in range(3)) if s.n_shared else None
+    if mutate is not None:
+        mutate(mats, shm)
     orc_routed = {e: orc.pack_expert(*mats[e], s.wbits) for e in range(s.n_experts)}
     orc_shared = orc.pack_expert(*shm, s.wbits) if shm else None
     routed = moe.bank_from_host_matrices(s, [mats[e] for e in range(s.n_experts)], device)

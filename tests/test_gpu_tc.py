@@ -78,3 +78,21 @@ def test_tc_then_small_batches_share_a_workspace():
     for T in (300, 3, 17, 64):
         x = synth.make_x(make_workload("tc_mixed", TC4, T, 500 + T))
         check_layer(pair, x)
+
+
+def test_tc_wide_block_scales_take_the_fp64_epilogue():
+    """Tokens whose block scales span more than 2^7 cannot use the integer
+    epilogue (m' would not fit 31 bits) and take the fp64 one: x with some
+    blocks scaled by 2^-12 on every third token (gate/up side), and a shared
+    expert whose first 32 up rows are scaled by 1e-4, so that h's first block
+    is tiny on every token (down side).  Still bit-identical."""
+    def mutate(mats, shm):
+        shm[1][:32] *= np.float32(1e-4)
+
+    T = 80
+    pair = build_pair(make_workload("tc_wide", TC4, T, 123), T_max=T, mutate=mutate)
+    x = pair.x.copy()
+    for t in range(0, T, 3):
+        for b in range(0, TC4.hidden // 32, 5):
+            x[t, 32 * b:32 * (b + 1)] *= np.float32(2.0 ** -12)
+    _strict(pair, x)
