@@ -206,26 +206,49 @@ def step_stats(ms: list[float]) -> dict:
             "min": round(min(ms), 5), "max": round(max(ms), 5)}
 
 
-def capture_graphs(torch, layer, xs, out):
-    """One CUDA graph per token batch (the layer's forward on it), or [] if
-    the capture fails (the steps then run eagerly)."""
-    graphs = []
+def capture_steps(torch, moe, layer, batches, out, flush=None):
+    """One CUDA graph of len(batches) consecutive forwards, each bracketed by
+    the library's phase events (moe_profile_events), with an L2 flush before
+    each when `flush` is given.  Returns (graph, events), or (None, events)
+    if the capture fails (the caller then runs the steps eagerly)."""
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.PROFILE_MAX_EVENTS)] for _ in batches]
+    for row in evs:  # torch creates the CUDA event on first record
+        for ev in row:
+            ev.record()
+    torch.cuda.synchronize()
     try:
+        g = torch.cuda.CUDAGraph()
         side = torch.cuda.Stream()
         side.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(side):
-            for x in xs:
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=side):
+            with torch.cuda.graph(g, stream=side):
+                for i, x in enumerate(batches):
+                    if flush is not None:
+                        flush.fill_(i & 0xFF)
+                    moe.profile_events(evs[i])
                     layer.forward(x, out)
-                graphs.append(g)
+                moe.profile_events(None)
         torch.cuda.current_stream().wait_stream(side)
         torch.cuda.synchronize()
+        return g, evs
     except Exception as exc:  # noqa: BLE001
+        moe.profile_events(None)
         print(f"graph capture unavailable ({exc}); timing eager steps", file=sys.stderr)
         torch.cuda.synchronize()
-        return []
-    return graphs
+        return None, evs
+
+
+def run_steps(torch, moe, layer, batches, out, graph, evs, flush=None):
+    """Run the captured steps (or the same steps eagerly)."""
+    if graph is not None:
+        graph.replay()
+        return
+    for i, x in enumerate(batches):
+        if flush is not None:
+            flush.fill_(i & 0xFF)
+        moe.profile_events(evs[i])
+        layer.forward(x, out)
+    moe.profile_events(None)
 
 
 def run_ours(args) -> dict | None:
@@ -257,21 +280,17 @@ def run_ours(args) -> dict | None:
     torch.cuda.synchronize()
     assert layer.device_error() == 0
 
-    # one CUDA graph per token batch: a timed step is one graph replay, so the
-    # device runs the step's launches back to back whatever the host's pace
-    graphs = capture_graphs(torch, layer, xs, out)
-    for i in range(args.warmup):
-        if graphs:
-            graphs[i % R].replay()
-        else:
-            layer.forward(xs[i % R], out)
-    torch.cuda.synchronize()
-
     K = args.steps
     phases = moe.forward_phases(layer.cfg, wl.T)
     P = len(phases)
-    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    # the K timed steps as one CUDA graph: the device runs them back to back
+    # whatever the host's pace, and each step is timed by the library's own
+    # events at its phase boundaries inside the graph
+    batches = [xs[i % R] for i in range(K)]
+    graph, evs = capture_steps(torch, moe, layer, batches, out)
+    run_steps(torch, moe, layer, batches[: min(K, args.warmup)], out, None,
+              evs[: min(K, args.warmup)])  # untimed eager steps after the capture
+    torch.cuda.synchronize()
     gpu_uuid = None
     try:
         gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
@@ -284,33 +303,17 @@ def run_ours(args) -> dict | None:
     torch.cuda.synchronize()
     sampler = ClockSampler(gpu_uuid)
     time.sleep(0.15)
-    for i in range(K):
-        ev_s[i].record()
-        if graphs:
-            graphs[i % R].replay()
-        else:
-            layer.forward(xs[i % R], out)
-        ev_e[i].record()
+    run_steps(torch, moe, layer, batches, out, graph, evs)
     torch.cuda.synchronize()
     clocks = sampler.stop()
+    graph_used = graph is not None
     if world > 1:
         dist.barrier()
-    step_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(K)]
-    total_ms = sum(step_ms)
+    step_ms = [evs[i][0].elapsed_time(evs[i][P]) for i in range(K)]
+    phase_ms = [[evs[i][p].elapsed_time(evs[i][p + 1]) for i in range(K)] for p in range(P)]
     assert layer.device_error() == 0
-    # the phases (library events at the phase boundaries), from eager steps
-    K_p = min(K, 200)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.PROFILE_MAX_EVENTS)] for _ in range(K_p)]
-    for row in evs:  # torch creates the CUDA event on first record
-        for ev in row:
-            ev.record()
-    torch.cuda.synchronize()
-    for i in range(K_p):
-        moe.profile_events(evs[i])
-        layer.forward(xs[i % R], out)
-    moe.profile_events(None)
-    torch.cuda.synchronize()
-    phase_ms = [[evs[i][p].elapsed_time(evs[i][p + 1]) for i in range(K_p)] for p in range(P)]
+    del graph
+    total_ms = sum(step_ms)
     max_total = reduce_max(total_ms, dev)
     value = throughput(wl.T, K, world, max_total)
     # active experts of each rotation (the bytes a step streams)
@@ -325,22 +328,11 @@ def run_ours(args) -> dict | None:
     K_v = min(K, 200)
 
     def timed(flush_l2: bool) -> list[float]:
-        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_v)]
-        for row in ev:
-            for e in row:
-                e.record()
+        same = [xs[0]] * K_v
+        g, ev = capture_steps(torch, moe, layer, same, out, flush if flush_l2 else None)
+        run_steps(torch, moe, layer, same, out, g, ev, flush if flush_l2 else None)
         torch.cuda.synchronize()
-        for i in range(K_v):
-            if flush_l2:
-                flush.fill_(i & 0xFF)
-            ev[i][0].record()
-            if graphs:
-                graphs[0].replay()
-            else:
-                layer.forward(xs[0], out)
-            ev[i][1].record()
-        torch.cuda.synchronize()
-        return [ev[i][0].elapsed_time(ev[i][1]) for i in range(K_v)]
+        return [ev[i][0].elapsed_time(ev[i][P]) for i in range(K_v)]
 
     fixed_ms = timed(False)
     flushed_ms = timed(True)
@@ -398,8 +390,9 @@ def run_ours(args) -> dict | None:
                    "experts": s.n_experts, "top_k": s.top_k, "shared": s.n_shared, "weights": f"int{s.wbits}",
                    "activations": "Q8_0 int8", "unique_experts_per_step": round(mean_active, 2),
                    "token_batches": f"{R} seeded batches, step i uses batch i mod {R}",
-                   "timing": ("CUDA-event pair around each step's CUDA-graph replay" if graphs else
-                              "CUDA-event pair around each step (graph capture unavailable)"),
+                   "timing": ("the K steps as one CUDA graph, each step timed by the library's events at its "
+                              "first launch and after its last" if graph_used else
+                              "eager steps timed by the library's events (graph capture unavailable)"),
                    "l2": ("not flushed: every step streams its selected experts' weights, more than L2 holds, "
                           "and consecutive steps select different experts"),
                    "parallelism": f"replicas x{world}"},

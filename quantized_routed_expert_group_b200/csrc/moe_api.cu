@@ -48,24 +48,17 @@ Layout make_layout(const moe_config& c, int T) {
         const TcSizes z = tc_sizes(c, T);
         const size_t pr = (size_t)z.prows_cap;
         L.tc_xg = take(pr * H);
-        L.tc_xm = take((H / 32) * pr * 4);
-        L.tc_xd = take((H / 32) * pr * 4);
-        L.tc_xe = take(pr * 4);
-        L.tc_xok = take(pr * 4);
+        L.tc_xdT = take((H / 32) * pr * 8);
         L.tc_gu = take(2 * pr * I * 4);
         L.tc_hg = take(pr * I);
-        L.tc_hm = take((I / 32) * pr * 4);
-        L.tc_hd = take((I / 32) * pr * 4);
-        L.tc_he = take(pr * 4);
-        L.tc_hok = take(pr * 4);
+        L.tc_hdT = take((I / 32) * pr * 8);
         L.tc_row_tok = take(pr * 4);
         L.tc_row_slot = take(pr * 4);
         L.tc_units_gu = take((size_t)z.units_gu_cap * kTcUnitBytes);
         L.tc_units_dn = take((size_t)z.units_dn_cap * kTcUnitBytes);
         L.tc_ctrl = take(64);
     } else {
-        L.tc_xg = L.tc_xm = L.tc_xd = L.tc_xe = L.tc_xok = L.tc_gu = 0;
-        L.tc_hg = L.tc_hm = L.tc_hd = L.tc_he = L.tc_hok = L.tc_row_tok = L.tc_row_slot = 0;
+        L.tc_xg = L.tc_xdT = L.tc_gu = L.tc_hg = L.tc_hdT = L.tc_row_tok = L.tc_row_slot = 0;
         L.tc_units_gu = L.tc_units_dn = L.tc_ctrl = 0;
     }
     L.total = off;
@@ -136,7 +129,7 @@ static thread_local cudaEvent_t g_trace[MOE_PROFILE_MAX_EVENTS];
 static thread_local bool g_trace_on = false;
 
 static cudaError_t trace(int i, cudaStream_t s) {
-    return g_trace_on ? cudaEventRecord(g_trace[i], s) : cudaSuccess;
+    return g_trace_on ? record_event(g_trace[i], s) : cudaSuccess;
 }
 
 static int check_bucket_fits(const moe_config& c, int T) {
@@ -218,12 +211,10 @@ static int forward_device(const moe_config& c, const float* x, int T, const floa
     TcArgs ta{};
     if (tc) {
         ta.xg = reinterpret_cast<int8_t*>(ws + L.tc_xg);
-        ta.xs = RowScales{reinterpret_cast<int32_t*>(ws + L.tc_xm), reinterpret_cast<float*>(ws + L.tc_xd),
-                          reinterpret_cast<int32_t*>(ws + L.tc_xe), reinterpret_cast<int32_t*>(ws + L.tc_xok)};
+        ta.xdT = reinterpret_cast<double*>(ws + L.tc_xdT);
         ta.gu = reinterpret_cast<float*>(ws + L.tc_gu);
         ta.hg = reinterpret_cast<int8_t*>(ws + L.tc_hg);
-        ta.hs = RowScales{reinterpret_cast<int32_t*>(ws + L.tc_hm), reinterpret_cast<float*>(ws + L.tc_hd),
-                          reinterpret_cast<int32_t*>(ws + L.tc_he), reinterpret_cast<int32_t*>(ws + L.tc_hok)};
+        ta.hdT = reinterpret_cast<double*>(ws + L.tc_hdT);
         ta.row_tok = reinterpret_cast<int32_t*>(ws + L.tc_row_tok);
         ta.row_slot = reinterpret_cast<int32_t*>(ws + L.tc_row_slot);
         ta.units_gu = ws + L.tc_units_gu;

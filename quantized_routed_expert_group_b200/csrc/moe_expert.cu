@@ -198,20 +198,45 @@ __global__ void __launch_bounds__(256) k_down(ExpertParams p) {
 // out[t][c] = sum_j w[t][j] * y[slot(t,j)][c] + y[T*k + t][c], summed in
 // fp64 in slot order, then the shared expert, and rounded to fp32 (each
 // fp32 x fp32 product is exact in fp64, so every step rounds once, as the
-// definition's fp64 sum does).
-__global__ void k_combine(ExpertParams p) {
-    const int64_t n = (int64_t)p.T * p.H;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-        const int t = (int)(i / p.H), c = (int)(i % p.H);
-        double acc = 0.0;
-        for (int j = 0; j < p.k; ++j) {
-            const int slot = p.inv_perm[t * p.k + j];
-            if (slot < 0) continue;  // dropped by the adaptive top-p
-            acc = __fma_rn((double)p.w[t * p.k + j], (double)p.y[(int64_t)slot * p.H + c], acc);
-        }
-        if (p.ns) acc = __dadd_rn(acc, (double)p.y[((int64_t)p.T * p.k + t) * p.H + c]);
-        p.out[i] = __double2float_rn(acc);
+// definition's fp64 sum does).  CTA = one token x kCombineCols columns: the
+// token's slots and weights are read once into shared memory, each thread
+// then streams four columns of every slot's row (128-bit loads).
+constexpr int kCombineCols = 1024;
+__global__ void __launch_bounds__(256) k_combine(ExpertParams p) {
+    __shared__ int s_slot[33];
+    __shared__ double s_w[33];
+    const int t = blockIdx.y;
+    const int k = p.k;
+    if ((int)threadIdx.x < k) {
+        s_slot[threadIdx.x] = p.inv_perm[t * k + threadIdx.x];  // < 0: dropped by the adaptive top-p
+        s_w[threadIdx.x] = (double)p.w[t * k + threadIdx.x];
     }
+    __syncthreads();
+    const int c = blockIdx.x * kCombineCols + 4 * threadIdx.x;
+    if (c >= p.H) return;
+    double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+    for (int j = 0; j < k; ++j) {
+        const int slot = s_slot[j];
+        if (slot < 0) continue;
+        const float4 y = __ldcs(reinterpret_cast<const float4*>(p.y + (int64_t)slot * p.H + c));
+        const double w = s_w[j];
+        a0 = __fma_rn(w, (double)y.x, a0);
+        a1 = __fma_rn(w, (double)y.y, a1);
+        a2 = __fma_rn(w, (double)y.z, a2);
+        a3 = __fma_rn(w, (double)y.w, a3);
+    }
+    if (p.ns) {
+        const float4 y = __ldcs(reinterpret_cast<const float4*>(p.y + ((int64_t)p.T * k + t) * p.H + c));
+        a0 = __dadd_rn(a0, (double)y.x);
+        a1 = __dadd_rn(a1, (double)y.y);
+        a2 = __dadd_rn(a2, (double)y.z);
+        a3 = __dadd_rn(a3, (double)y.w);
+    }
+    float* o = p.out + (int64_t)t * p.H + c;  // out is only 4-byte aligned
+    o[0] = __double2float_rn(a0);
+    o[1] = __double2float_rn(a1);
+    o[2] = __double2float_rn(a2);
+    o[3] = __double2float_rn(a3);
 }
 
 template <typename K>
@@ -231,18 +256,15 @@ static cudaError_t launch_experts_t(const ExpertParams& p, cudaStream_t s, cudaE
     const int items_dn = max_entries * ((p.H + 63) / 64);
     k_gateup<WBITS, TCH><<<max(1, min(items_gu, di.sm_count * occ_gu)), 256, 0, s>>>(p);
     cudaError_t e = cudaGetLastError();
-    if (e == cudaSuccess && ev) e = cudaEventRecord(ev[0], s);
+    if (e == cudaSuccess && ev) e = record_event(ev[0], s);
     if (e != cudaSuccess) return e;
     k_down<WBITS, TCH><<<max(1, min(items_dn, di.sm_count * occ_dn)), 256, 0, s>>>(p);
     e = cudaGetLastError();
-    if (e == cudaSuccess && ev) e = cudaEventRecord(ev[1], s);
+    if (e == cudaSuccess && ev) e = record_event(ev[1], s);
     if (e != cudaSuccess) return e;
-    const int64_t n = (int64_t)p.T * p.H;
-    const int64_t want = (n + 255) / 256, cap = (int64_t)di.sm_count * 8;
-    const int grid = (int)(want < cap ? want : cap);
-    k_combine<<<max(1, grid), 256, 0, s>>>(p);
+    k_combine<<<dim3((p.H + kCombineCols - 1) / kCombineCols, p.T), 256, 0, s>>>(p);
     e = cudaGetLastError();
-    if (e == cudaSuccess && ev) e = cudaEventRecord(ev[2], s);
+    if (e == cudaSuccess && ev) e = record_event(ev[2], s);
     return e;
 }
 
@@ -258,10 +280,9 @@ static ExpertParams expert_params(const ExpertArgs& a) {
 
 cudaError_t launch_combine(const ExpertArgs& a, cudaStream_t s) {
     const ExpertParams p = expert_params(a);
-    const int64_t n = (int64_t)p.T * p.H;
-    const int64_t want = (n + 255) / 256, cap = (int64_t)device_info().sm_count * 8;
-    const int grid = (int)(want < cap ? want : cap);
-    k_combine<<<max(1, grid), 256, 0, s>>>(p);
+    if (p.T == 0) return cudaSuccess;
+    const dim3 grid((p.H + kCombineCols - 1) / kCombineCols, p.T);
+    k_combine<<<grid, 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 

@@ -33,12 +33,22 @@ struct Layout {
     size_t hd;         // fp32 [slots][I/32]
     size_t y;          // fp32 [slots][H]
     // batched tensor-core path only (0 bytes otherwise)
-    size_t tc_xg, tc_xm, tc_xd, tc_xe, tc_xok, tc_gu, tc_hg, tc_hm, tc_hd, tc_he, tc_hok;
-    size_t tc_row_tok, tc_row_slot, tc_units_gu, tc_units_dn, tc_ctrl;
+    size_t tc_xg, tc_xdT, tc_gu, tc_hg, tc_hdT, tc_row_tok, tc_row_slot, tc_units_gu, tc_units_dn, tc_ctrl;
     size_t total;
 };
 
 Layout make_layout(const moe_config& c, int T);
+
+// Record a tracing event on s.  Inside a stream capture a plain record only
+// orders the graph; an external record makes the graph record the event when
+// it runs, so the phase events time captured forwards too.
+inline cudaError_t record_event(cudaEvent_t ev, cudaStream_t s) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    const cudaError_t e = cudaStreamIsCapturing(s, &cs);
+    if (e != cudaSuccess) return e;
+    return cs == cudaStreamCaptureStatusActive ? cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal)
+                                               : cudaEventRecord(ev, s);
+}
 
 struct DeviceInfo {
     int sm_count;
@@ -99,23 +109,13 @@ struct TcSizes {
     int units_dn_cap;  // work units of the down GEMM
 };
 TcSizes tc_sizes(const moe_config& c, int T);
-// Block scales of the padded rows of one GEMM's tokens, for the epilogue:
-// the scales as integers over a common power of two per row (m' = m << (ex -
-// e) of d = m * 2^ex, see moe_tc.cu), the scales themselves, the row's
-// exponent e and whether the row takes the integer epilogue.
-struct RowScales {
-    int32_t* mT;  // [nb][prows_cap]
-    float* dT;    // [nb][prows_cap]
-    int32_t* e;   // [prows_cap]
-    int32_t* ok;  // [prows_cap]
-};
 struct TcArgs {
     ExpertArgs ex;
     int8_t* xg;         // [prows_cap][hidden]
-    RowScales xs;       // of x's blocks (nb = hidden/32)
+    double* xdT;        // [hidden/32][prows_cap]
     float* gu;          // [2][prows_cap][inter]  g and u row values
     int8_t* hg;         // [prows_cap][inter]
-    RowScales hs;       // of h's blocks (nb = inter/32)
+    double* hdT;        // [inter/32][prows_cap]
     int32_t* row_tok;   // [prows_cap]
     int32_t* row_slot;  // [prows_cap]
     void* units_gu;     // TcUnit [units_gu_cap]

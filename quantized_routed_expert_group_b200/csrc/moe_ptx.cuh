@@ -54,13 +54,30 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
+// try_wait that lets the hardware suspend the thread for up to hint_ns (it
+// resumes as soon as the phase completes), so that waiting warps do not spin
+// on the issue slots the working warps need.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait on a barrier phase: gives up (returns false) once budget_ns
-// nanoseconds of the global timer have passed since the call.
+// nanoseconds of the global timer have passed since the call.  The thread
+// sleeps in slices of at most 20 us between checks of the timer.
 __device__ __forceinline__ bool mbar_wait_ns(uint64_t* bar, uint32_t parity, uint64_t budget_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
+    const uint32_t slice = budget_ns < 20000u ? (uint32_t)budget_ns : 20000u;
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, slice)) return true;
         if (global_timer_ns() - t0 > budget_ns) return false;
     }
 }

@@ -207,27 +207,23 @@ cudaError_t launch_tc_block_dots(const uint8_t* packed, int64_t rows, int cols, 
 //                 units (entry, 128-row weight tile, matrix, chunk of <= 64
 //                 tokens), heaviest entries first
 //   k_tc_gather   the entries' Q8_0 codes of x into the padded row space
-//                 (xg [prows][hidden]) and their block scales (RowScales,
-//                 transposed [hidden/32][prows]), so that every unit's tokens
-//                 are one TMA box
+//                 (xg [prows][hidden]) and their block scales, transposed and
+//                 widened to fp64 (xdT [hidden/32][prows]), so that every
+//                 unit's tokens are one TMA box
 //   k_tc_gemm     gate/up: g and u row values per padded row (gu [2][prows][inter])
-//   k_tc_swiglu   h = silu(g) * u and Q8_0 of h -> hg and its RowScales
-//                 (padded rows, for the down GEMM) and hq / hd (per slot)
+//   k_tc_swiglu   h = silu(g) * u and Q8_0 of h -> hg / hdT (padded rows, for
+//                 the down GEMM) and hq / hd (per slot)
 //   k_tc_gemm     down: y per slot
 //   k_combine     (the multi-kernel path's)
 //
 // Arithmetic: a row value is s_row * sum_b d_b * dot_b with the int32 block
-// dots from the tensor core.  A block scale is d_b = m_b * 2^e_b with m_b an
-// integer below 2^24; with e = the token's smallest e_b, d_b = m'_b * 2^e for
-// the integer m'_b = m_b << (e_b - e).  When every m'_b of the token is below
-// 2^31 (the scales span at most 2^7), the epilogue sums m'_b * dot_b exactly
-// in int64 (one 32 x 32 -> 64-bit multiply-add per block), and the row value
-// is s_row * (sum * 2^e) in fp64, rounded to fp32: the exact sum where the
-// definition rounds each fp64 addition (a relative difference near 2^-50,
-// far below an fp32 rounding step).  Other tokens take an fp64 epilogue
-// (d_b * dot_b added in fp64 in block order).  SwiGLU is evaluated in fp64
-// and rounded to fp32 before Q8_0, as the definition does, so the h codes do
-// not depend on a summation order.
+// dots from the tensor core; the epilogue adds d_b * dot_b in fp64 in block
+// order (each product is exact in fp64), multiplies by s_row in fp64 and
+// rounds to fp32, and SwiGLU is evaluated in fp64 and rounded to fp32 before
+// Q8_0 -- the same operations in the same order as the definition, so the h
+// codes do not depend on a summation order.  (fp64 on the B200's CUDA cores
+// runs at half the fp32 rate; a 32 x 32 -> 64-bit integer multiply-add, the
+// alternative for exact sums, at a sixth.)
 namespace tc {
 
 struct PlanParams {
@@ -346,31 +342,41 @@ __global__ void __launch_bounds__(kPlanThreads) k_tc_plan(PlanParams p) {
         return;
     }
     // work units: per entry (in schedule order) by weight tile, then matrix,
-    // then token chunk, so that the chunks of one weight tile follow each other
-    for (int r = tid; r < ne; r += kPlanThreads) {
-        const int i = s_sched[r];
+    // then token chunk, so that the chunks of one weight tile follow each
+    // other; every thread writes units, each finding its entry by a binary
+    // search over the entries' first unit
+    auto entry_of = [&](const int* first, int u) {
+        int lo = 0, hi = ne - 1;
+        while (lo < hi) {  // last entry (schedule rank) whose first unit is <= u
+            const int mid = (lo + hi + 1) >> 1;
+            if (first[mid] <= u) lo = mid;
+            else hi = mid - 1;
+        }
+        return lo;
+    };
+    for (int u = tid; u < rgu; u += kPlanThreads) {
+        const int r = entry_of(s_ugu0, u), i = s_sched[r];
         const int n = s_n[i], nch = (n + kMaxN - 1) / kMaxN;
+        const int l = u - s_ugu0[r], c = l % nch, tm = l / nch, m = tm & 1, t = tm >> 1;
         const bool shared = i >= U;
-        const int expert = shared ? 0 : p.active[1 + i];
-        for (int t = 0; t < tiles_gu; ++t)
-            for (int m = 0; m < 2; ++m)
-                for (int c = 0; c < nch; ++c) {
-                    TcUnit u;
-                    u.prow0 = s_prow0[i] + c * kMaxN;
-                    u.ntok = min(kMaxN, n - c * kMaxN);
-                    u.wrow0 = expert * p.I + t * kTileRows;
-                    u.info = t | (shared ? kUnitShared : 0) | (m ? kUnitUp : 0);
-                    p.units_gu[s_ugu0[r] + (t * 2 + m) * nch + c] = u;
-                }
-        for (int t = 0; t < tiles_dn; ++t)
-            for (int c = 0; c < nch; ++c) {
-                TcUnit u;
-                u.prow0 = s_prow0[i] + c * kMaxN;
-                u.ntok = min(kMaxN, n - c * kMaxN);
-                u.wrow0 = expert * p.H + t * kTileRows;
-                u.info = t | (shared ? kUnitShared : 0);
-                p.units_dn[s_udn0[r] + t * nch + c] = u;
-            }
+        TcUnit w;
+        w.prow0 = s_prow0[i] + c * kMaxN;
+        w.ntok = min(kMaxN, n - c * kMaxN);
+        w.wrow0 = (shared ? 0 : p.active[1 + i]) * p.I + t * kTileRows;
+        w.info = t | (shared ? kUnitShared : 0) | (m ? kUnitUp : 0);
+        p.units_gu[u] = w;
+    }
+    for (int u = tid; u < rdn; u += kPlanThreads) {
+        const int r = entry_of(s_udn0, u), i = s_sched[r];
+        const int n = s_n[i], nch = (n + kMaxN - 1) / kMaxN;
+        const int l = u - s_udn0[r], c = l % nch, t = l / nch;
+        const bool shared = i >= U;
+        TcUnit w;
+        w.prow0 = s_prow0[i] + c * kMaxN;
+        w.ntok = min(kMaxN, n - c * kMaxN);
+        w.wrow0 = (shared ? 0 : p.active[1 + i]) * p.H + t * kTileRows;
+        w.info = t | (shared ? kUnitShared : 0);
+        p.units_dn[u] = w;
     }
     // padded row -> token and slot (-1 for the padding rows)
     for (int q = tid; q < prows; q += kPlanThreads) {
@@ -398,58 +404,12 @@ __global__ void __launch_bounds__(kPlanThreads) k_tc_plan(PlanParams p) {
     }
 }
 
-// An fp32 block scale d >= 0 as m * 2^ex with m an integer below 2^24
-// (m = 0 for d = 0).
-__device__ __forceinline__ void scale_parts(float d, uint32_t& m, int& ex) {
-    const uint32_t bits = __float_as_uint(d) & 0x7FFFFFFFu;
-    const uint32_t e = bits >> 23, mant = bits & 0x7FFFFFu;
-    m = e ? (mant | 0x800000u) : mant;
-    ex = e ? (int)e - 150 : -149;
-}
-
-// The warp's row: its nb block scales d_b (d_of(b)) -> m'_b into mT[b][q]
-// (transposed), d_b into dT[b][q], the row's exponent into e[q] and whether
-// it takes the integer epilogue into ok[q] (all m'_b below 2^31).
-template <class DOf>
-__device__ __forceinline__ void row_scales(DOf d_of, int nb, int q, int prows_cap, const RowScales& rs, int lane) {
-    int emin = 1 << 30, emax = -(1 << 30);
-    for (int b = lane; b < nb; b += 32) {
-        uint32_t m;
-        int ex;
-        scale_parts(d_of(b), m, ex);
-        if (m) {
-            emin = min(emin, ex);
-            emax = max(emax, ex);
-        }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        emin = min(emin, __shfl_xor_sync(kFull, emin, o));
-        emax = max(emax, __shfl_xor_sync(kFull, emax, o));
-    }
-    const bool any = emax >= emin;
-    const bool ok = !any || emax - emin <= 7;  // m' < 2^24 * 2^7 = 2^31
-    const int e = any ? emin : 0;
-    for (int b = lane; b < nb; b += 32) {
-        const float d = d_of(b);
-        uint32_t m;
-        int ex;
-        scale_parts(d, m, ex);
-        rs.mT[(int64_t)b * prows_cap + q] = (ok && m) ? (int32_t)(m << (ex - e)) : 0;
-        rs.dT[(int64_t)b * prows_cap + q] = d;
-    }
-    if (lane == 0) {
-        rs.e[q] = e;
-        rs.ok[q] = ok ? 1 : 0;
-    }
-}
-
 // One warp per padded row: the token's Q8_0 codes (zeros for a padding row)
-// and its block scales.
+// and its block scales, transposed, as fp64.
 __global__ void __launch_bounds__(256) k_tc_gather(const int8_t* __restrict__ xq, const float* __restrict__ xd,
                                                    int H, int prows_cap, const int32_t* __restrict__ row_tok,
                                                    const int32_t* __restrict__ ctrl, int8_t* __restrict__ xg,
-                                                   RowScales rs) {
+                                                   double* __restrict__ xdT) {
     const int lane = threadIdx.x & 31;
     const int q = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (q >= ctrl[2]) return;
@@ -458,8 +418,8 @@ __global__ void __launch_bounds__(256) k_tc_gather(const int8_t* __restrict__ xq
     uint4* dst = reinterpret_cast<uint4*>(xg + (int64_t)q * H);
     const uint4* src = reinterpret_cast<const uint4*>(xq + (int64_t)(tok < 0 ? 0 : tok) * H);
     for (int i = lane; i < n16; i += 32) dst[i] = tok >= 0 ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
-    const float* xdr = xd + (int64_t)(tok < 0 ? 0 : tok) * nb;
-    row_scales([&](int b) { return tok >= 0 ? __ldg(xdr + b) : 0.0f; }, nb, q, prows_cap, rs, lane);
+    for (int b = lane; b < nb; b += 32)
+        xdT[(int64_t)b * prows_cap + q] = tok >= 0 ? (double)__ldg(xd + (int64_t)tok * nb + b) : 0.0;
 }
 
 // ---------------------------------------------------------------------------
@@ -467,10 +427,9 @@ __global__ void __launch_bounds__(256) k_tc_gather(const int8_t* __restrict__ xq
 // ---------------------------------------------------------------------------
 // warps 0-15  epilogue: warp w reads TMEM lanes 32 (w % 4) .. (its 32 weight
 //             rows) and columns 16 (w / 4) .. (its 16 tokens); per Q8_0 block
-//             it accumulates m'_token * dot in int64 (or, for a token whose
-//             scales span more than 2^7, d_token * dot in fp64); at a unit's
-//             end it applies 2^e and the row scale (fp64, rounded to fp32)
-//             and writes g / u (gate/up) or y (down)
+//             it converts the int32 dots exactly to fp64 and accumulates
+//             d_token * dot in fp64; at a unit's end it applies the row scale
+//             (fp64, rounded to fp32) and writes g / u (gate/up) or y (down)
 // warps 16-17 widening: packed int4 / int2 staging rows -> int8 MMA tiles
 // warp 18     producer: takes units from a global counter, TMA of the packed
 //             weight rows, the token codes and their block scales per stage
@@ -491,14 +450,14 @@ struct GemmSmem {
     static constexpr int kA = 0;                       // widened tile (int8: the TMA target)
     static constexpr int kX = kTileBytes;              // token codes [64][128]
     static constexpr int kRaw = kX + kMaxN * kStageK;  // packed staging tile
-    static constexpr int kD = kRaw + kRawTile;         // integer block scales m' [4][64]
-    static constexpr int kStageBytes = (kD + kBlocksPerStage * kMaxN * 4 + 1023) & ~1023;
+    static constexpr int kD = kRaw + kRawTile;         // block scales [4][64] fp64
+    static constexpr int kStageBytes = (kD + kBlocksPerStage * kMaxN * 8 + 1023) & ~1023;
     static constexpr int kCtrl = 1024;
     static constexpr int kStagesFit = (220 * 1024 - kCtrl - 1024) / kStageBytes;
     static constexpr int kStages = kStagesFit < 6 ? kStagesFit : 6;
     static constexpr int kBytes = kStages * kStageBytes + kCtrl + 1024;  // + alignment slack
     static constexpr uint32_t kTxBytes =
-        (uint32_t)(kTileRows * raw_row_bytes<WBITS>() + kMaxN * kStageK + kBlocksPerStage * kMaxN * 4);
+        (uint32_t)(kTileRows * raw_row_bytes<WBITS>() + kMaxN * kStageK + kBlocksPerStage * kMaxN * 8);
     static constexpr int kTmemCols = kNAcc * kMaxN;
 };
 
@@ -516,9 +475,8 @@ struct GemmParams {
     const float* s_r1;
     const float* s_s0;
     const float* s_s1;
-    RowScales rs;  // the tokens' block scales (exponent, integer-path flag, fp32 scales)
-    float* gu;     // gate/up: [2][prows_cap][I]
-    float* y;      // down: [slots][H]
+    float* gu;  // gate/up: [2][prows_cap][I]
+    float* y;   // down: [slots][H]
     int32_t* err;
 };
 
@@ -699,10 +657,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int s = 0, a = 0;
         uint32_t ph = 0, aph = 0;
         TcUnit u{0, 0, 0, 0};
-        long long acc[16];  // int64 sums, or the bits of fp64 sums on the fp64 path
-        bool fp64_path = false;
+        double acc[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) acc[c] = 0;
+        for (int c = 0; c < 16; ++c) acc[c] = 0.0;
         bool ok = true;
         while (ok) {
             if (!mbar_wait_ns(&full[s], ph, kGemmWaitNs)) {
@@ -715,15 +672,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (kstep == 0) {
                 u = p.units[unit];
 #pragma unroll
-                for (int c = 0; c < 16; ++c) acc[c] = 0;
-                // the integer path unless one of the warp's tokens needs fp64
-                int need = 0;
-                for (int c = 0; c < 16; ++c)
-                    if (16 * qt + c < u.ntok) need |= p.rs.ok[u.prow0 + 16 * qt + c] ? 0 : 1;
-                fp64_path = need != 0;
+                for (int c = 0; c < 16; ++c) acc[c] = 0.0;
             }
             const bool active = 16 * qt < u.ntok;  // the same in the whole warp
-            const int32_t* mt = reinterpret_cast<const int32_t*>(stage(s) + L::kD);
+            const double* dt = reinterpret_cast<const double*>(stage(s) + L::kD);
 #pragma unroll 1
             for (int j = 0; j < kBlocksPerStage; ++j) {
                 if (kstep * kBlocksPerStage + j >= p.nbK) break;
@@ -740,23 +692,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tc_fence_before_sync();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&acce[a]);
-                    if (!fp64_path) {
-                        const int4* m4 = reinterpret_cast<const int4*>(mt + j * kMaxN + 16 * qt);
+                    const double2* d2 = reinterpret_cast<const double2*>(dt + j * kMaxN + 16 * qt);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int4 mm = m4[i];
-                            acc[4 * i] += (long long)mm.x * (long long)(int)v[4 * i];
-                            acc[4 * i + 1] += (long long)mm.y * (long long)(int)v[4 * i + 1];
-                            acc[4 * i + 2] += (long long)mm.z * (long long)(int)v[4 * i + 2];
-                            acc[4 * i + 3] += (long long)mm.w * (long long)(int)v[4 * i + 3];
-                        }
-                    } else {
-                        const int b = kstep * kBlocksPerStage + j;
-                        const float* db = p.rs.dT + (int64_t)b * p.prows_cap + u.prow0 + 16 * qt;
-#pragma unroll
-                        for (int c = 0; c < 16; ++c)
-                            acc[c] = __double_as_longlong(
-                                __fma_rn((double)__ldg(db + c), exact_i2d(v[c]), __longlong_as_double(acc[c])));
+                    for (int i = 0; i < 8; ++i) {
+                        const double2 dd = d2[i];
+                        acc[2 * i] = __fma_rn(dd.x, exact_i2d(v[2 * i]), acc[2 * i]);
+                        acc[2 * i + 1] = __fma_rn(dd.y, exact_i2d(v[2 * i + 1]), acc[2 * i + 1]);
                     }
                 } else {
                     tc_fence_before_sync();
@@ -782,10 +723,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const int col = 16 * qt + c;
                     if (col >= u.ntok) continue;
                     const int prow = u.prow0 + col;
-                    // the exact int64 sum (rounded once to fp64) times 2^e, or the fp64 sum
-                    const double sum = fp64_path ? __longlong_as_double(acc[c])
-                                                 : ldexp(__ll2double_rn(acc[c]), p.rs.e[prow]);
-                    const float v = __double2float_rn(__dmul_rn(sr, sum));
+                    const float v = __double2float_rn(__dmul_rn(sr, acc[c]));
                     if (p.mode == 0) {
                         p.gu[((int64_t)(up ? p.prows_cap : 0) + prow) * p.I + r] = v;
                     } else {
@@ -806,38 +744,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (warp == kMmaWarp) tmem_dealloc(tmem, L::kTmemCols);
 }
 
-// SwiGLU and Q8_0 of h, one warp per padded row (lane = h value of a block):
-// h = silu(g) * u evaluated in fp64 and rounded to fp32, then Q8_0; then the
-// row's block scales for the down GEMM.
+// SwiGLU and Q8_0 of h, one warp per (padded row, block of 32 h values):
+// h = silu(g) * u evaluated in fp64 and rounded to fp32, then Q8_0.
 __global__ void __launch_bounds__(256) k_tc_swiglu(const float* __restrict__ gu, int I, int prows_cap,
                                                    const int32_t* __restrict__ row_slot,
                                                    const int32_t* __restrict__ ctrl, int8_t* __restrict__ hg,
-                                                   RowScales hs, int8_t* __restrict__ hq, float* __restrict__ hd) {
+                                                   double* __restrict__ hdT, int8_t* __restrict__ hq,
+                                                   float* __restrict__ hd) {
     const int lane = threadIdx.x & 31;
     const int nbI = I / 32;
-    const int prows = ctrl[2];
-    for (int q = blockIdx.x * 8 + (threadIdx.x >> 5); q < prows; q += gridDim.x * 8) {
-        const int slot = row_slot[q];  // -1: a padding row (the same in the whole warp)
-        if (slot >= 0) {
-            for (int b = 0; b < nbI; ++b) {
-                const int i = 32 * b + lane;
-                const double g = (double)gu[(int64_t)q * I + i];
-                const double uu = (double)gu[((int64_t)prows_cap + q) * I + i];
-                const float h = __double2float_rn(__dmul_rn(__ddiv_rn(g, __dadd_rn(1.0, exp(-g))), uu));
-                int8_t qv;
-                float d;
-                q8_0_warp(h, qv, d);
-                hg[(int64_t)q * I + i] = qv;
-                hq[(int64_t)slot * I + i] = qv;
-                if (lane == 0) {
-                    hd[(int64_t)slot * nbI + b] = d;
-                    hs.dT[(int64_t)b * prows_cap + q] = d;
-                }
-            }
-            __syncwarp();  // lane 0's scales, for the whole warp
-            row_scales([&](int b) { return hs.dT[(int64_t)b * prows_cap + q]; }, nbI, q, prows_cap, hs, lane);
-        } else {
-            row_scales([&](int) { return 0.0f; }, nbI, q, prows_cap, hs, lane);
+    const int64_t n_jobs = (int64_t)ctrl[2] * nbI;
+    for (int64_t job = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); job < n_jobs; job += (int64_t)gridDim.x * 8) {
+        const int q = (int)(job / nbI), b = (int)(job % nbI);
+        const int slot = row_slot[q];
+        if (slot < 0) {  // a padding row (the same in the whole warp): zero scale
+            if (lane == 0) hdT[(int64_t)b * prows_cap + q] = 0.0;
+            continue;
+        }
+        const int i = 32 * b + lane;
+        const double g = (double)gu[(int64_t)q * I + i];
+        const double uu = (double)gu[((int64_t)prows_cap + q) * I + i];
+        const float h = __double2float_rn(__dmul_rn(__ddiv_rn(g, __dadd_rn(1.0, exp(-g))), uu));
+        int8_t qv;
+        float d;
+        q8_0_warp(h, qv, d);
+        hg[(int64_t)q * I + i] = qv;
+        hq[(int64_t)slot * I + i] = qv;
+        if (lane == 0) {
+            hdT[(int64_t)b * prows_cap + q] = (double)d;
+            hd[(int64_t)slot * nbI + b] = d;
         }
     }
 }
@@ -878,7 +813,7 @@ cudaError_t launch_tc_prepare(const TcArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     const int grid = (a.sz.prows_cap + 7) / 8;
     tc::k_tc_gather<<<grid, 256, 0, s>>>(a.ex.xq, a.ex.xd, c.hidden, a.sz.prows_cap, a.row_tok, a.ctrl, a.xg,
-                                         a.xs);
+                                         a.xdT);
     return cudaGetLastError();
 }
 
@@ -908,15 +843,15 @@ static cudaError_t launch_gemm(int wbits, const CUtensorMap (&m)[6], const GemmP
     return launch_gemm_t<8>(m, gp, s);
 }
 
-// Token-side maps of a GEMM: codes [prows_cap][K] (128-byte swizzle) and the
-// integer block scales m' [K/32][prows_cap].
-static cudaError_t encode_tokens(CUtensorMap* codes, CUtensorMap* scales, const void* q, const int32_t* mT, int K,
+// Token-side maps of a GEMM: codes [prows_cap][K] (128-byte swizzle) and block
+// scales [K/32][prows_cap] fp64.
+static cudaError_t encode_tokens(CUtensorMap* codes, CUtensorMap* scales, const void* q, const double* dT, int K,
                                  int prows_cap) {
     cudaError_t e = encode_2d(codes, q, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)K, (uint64_t)prows_cap,
                               (uint64_t)K, kStageK, kMaxN, CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess) return e;
-    return encode_2d(scales, mT, CU_TENSOR_MAP_DATA_TYPE_INT32, (uint64_t)prows_cap, (uint64_t)(K / 32),
-                     (uint64_t)prows_cap * 4, kMaxN, kBlocksPerStage, CU_TENSOR_MAP_SWIZZLE_NONE);
+    return encode_2d(scales, dT, CU_TENSOR_MAP_DATA_TYPE_FLOAT64, (uint64_t)prows_cap, (uint64_t)(K / 32),
+                     (uint64_t)prows_cap * 8, kMaxN, kBlocksPerStage, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 }  // namespace tc
@@ -936,18 +871,18 @@ cudaError_t launch_tc_experts(const TcArgs& a, cudaStream_t s, cudaEvent_t const
         if ((e = encode_weights(&m[1], R.w_up, (int64_t)E * I, H, wb)) != cudaSuccess) return e;
         if ((e = encode_weights(&m[2], Sh.w_gate, sh_rows_gu, H, wb)) != cudaSuccess) return e;
         if ((e = encode_weights(&m[3], Sh.w_up, sh_rows_gu, H, wb)) != cudaSuccess) return e;
-        if ((e = encode_tokens(&m[4], &m[5], a.xg, a.xs.mT, H, a.sz.prows_cap)) != cudaSuccess) return e;
+        if ((e = encode_tokens(&m[4], &m[5], a.xg, a.xdT, H, a.sz.prows_cap)) != cudaSuccess) return e;
         GemmParams gp{};
         gp.mode = 0; gp.K = H; gp.nbK = H / 32; gp.nstage = (H + kStageK - 1) / kStageK; gp.H = H; gp.I = I;
         gp.prows_cap = a.sz.prows_cap; gp.units = static_cast<const TcUnit*>(a.units_gu); gp.ctrl = a.ctrl;
         gp.n_units_idx = 0; gp.counter = a.ctrl + 3; gp.row_slot = a.row_slot;
         gp.s_r0 = R.s_gate; gp.s_r1 = R.s_up; gp.s_s0 = Sh.s_gate; gp.s_s1 = Sh.s_up;
-        gp.rs = a.xs; gp.gu = a.gu; gp.y = a.ex.y; gp.err = a.ex.err;
+        gp.gu = a.gu; gp.y = a.ex.y; gp.err = a.ex.err;
         if ((e = launch_gemm(wb, m, gp, s)) != cudaSuccess) return e;
         // the "gate_up" phase ends with the GEMM; SwiGLU opens the "down" phase
-        if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return e;
+        if (ev && (e = record_event(ev[0], s)) != cudaSuccess) return e;
         const int grid = device_info().sm_count * 8;
-        k_tc_swiglu<<<grid, 256, 0, s>>>(a.gu, I, a.sz.prows_cap, a.row_slot, a.ctrl, a.hg, a.hs, a.ex.hq, a.ex.hd);
+        k_tc_swiglu<<<grid, 256, 0, s>>>(a.gu, I, a.sz.prows_cap, a.row_slot, a.ctrl, a.hg, a.hdT, a.ex.hq, a.ex.hd);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     // down: weights [E * H][I], h codes hg / hdT -> y per slot
@@ -957,18 +892,18 @@ cudaError_t launch_tc_experts(const TcArgs& a, cudaStream_t s, cudaEvent_t const
         m[1] = m[0];
         if ((e = encode_weights(&m[2], Sh.w_down, sh_rows_dn, I, wb)) != cudaSuccess) return e;
         m[3] = m[2];
-        if ((e = encode_tokens(&m[4], &m[5], a.hg, a.hs.mT, I, a.sz.prows_cap)) != cudaSuccess) return e;
+        if ((e = encode_tokens(&m[4], &m[5], a.hg, a.hdT, I, a.sz.prows_cap)) != cudaSuccess) return e;
         GemmParams gp{};
         gp.mode = 1; gp.K = I; gp.nbK = I / 32; gp.nstage = (I + kStageK - 1) / kStageK; gp.H = H; gp.I = I;
         gp.prows_cap = a.sz.prows_cap; gp.units = static_cast<const TcUnit*>(a.units_dn); gp.ctrl = a.ctrl;
         gp.n_units_idx = 1; gp.counter = a.ctrl + 4; gp.row_slot = a.row_slot;
         gp.s_r0 = R.s_down; gp.s_r1 = R.s_down; gp.s_s0 = Sh.s_down; gp.s_s1 = Sh.s_down;
-        gp.rs = a.hs; gp.gu = a.gu; gp.y = a.ex.y; gp.err = a.ex.err;
+        gp.gu = a.gu; gp.y = a.ex.y; gp.err = a.ex.err;
         if ((e = launch_gemm(wb, m, gp, s)) != cudaSuccess) return e;
-        if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return e;
+        if (ev && (e = record_event(ev[1], s)) != cudaSuccess) return e;
     }
     if ((e = launch_combine(a.ex, s)) != cudaSuccess) return e;
-    if (ev && (e = cudaEventRecord(ev[2], s)) != cudaSuccess) return e;
+    if (ev && (e = record_event(ev[2], s)) != cudaSuccess) return e;
     return cudaSuccess;
 }
 
