@@ -176,6 +176,18 @@ int moe_bucket_tokens(const moe_config *cfg, const int32_t *idx, int T, int32_t 
  * tokens (0 on an invalid config). */
 size_t moe_workspace_bytes(const moe_config *cfg, int T_max);
 
+/* Initialises the part of a workspace that the fused small-batch path
+ * (T <= 4) keeps from one call to the next: 1 KiB at a fixed offset holding
+ * the grid-wide counters of its persistent kernel (never reset between
+ * calls; each call counts from the values it finds) and a marker.  The
+ * forward entry points do this themselves the first time this process passes
+ * them a given workspace pointer on a given device; call it when the memory
+ * behind a pointer already used with them was written by anything else since
+ * (a fused forward on such a workspace records error code 3 and computes
+ * nothing when the marker is gone).  Enqueued on `stream`.  workspace: >=
+ * moe_workspace_bytes(cfg, T_max) bytes. */
+int moe_workspace_init(const moe_config *cfg, int T_max, void *workspace, size_t ws_bytes, void *stream);
+
 /* One MoE layer forward ([GN] §구현된 주요 기능; [WP] spec table, kernel table,
  * "Batch-Union MoE"):
  *   route (as moe_router_select), bucket (as moe_bucket_tokens), then for every
@@ -189,7 +201,8 @@ size_t moe_workspace_bytes(const moe_config *cfg, int T_max);
  * x [T][hidden] fp32 (16-byte aligned), out [T][hidden] fp32.  routed holds
  * n_experts experts, shared n_shared (ignored when n_shared == 0).
  * workspace: >= moe_workspace_bytes(cfg, T) bytes, 256-byte aligned; it holds
- * every intermediate of the call (see moe_workspace_view) and its error word.
+ * every intermediate of the call (see moe_workspace_view), its error word and
+ * the fused path's control region (see moe_workspace_init).
  * 0 <= T; T = 0 returns MOE_OK without launching. */
 int moe_layer_forward(const moe_config *cfg, const float *x, int T, const float *router_w,
                       const float *router_bias, const moe_experts *routed, const moe_experts *shared,
@@ -322,7 +335,8 @@ int moe_block_dots_routine(const uint8_t *packed, int64_t rows, int cols, int wb
 /* Synchronises `stream` and reads the workspace's device error word into
  * *code (0 = none).  Returns MOE_OK when it is 0, MOE_EDEVICE otherwise.
  * Codes: 1 = an index out of range reached a kernel, 2 = a device-side wait
- * ran out of time.  Every wait inside a kernel is bounded by the GPU's
+ * ran out of time, 3 = the fused path found the workspace's control region
+ * uninitialised (see moe_workspace_init).  Every wait inside a kernel is bounded by the GPU's
  * global timer: a wait for a free pipeline slot or for another CTA's
  * results gives up after 25 ms, a wait that can span one of those after
  * 100 ms; the kernel then records code 2 and returns, leaving the call's

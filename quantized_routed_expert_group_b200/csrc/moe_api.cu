@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <unordered_set>
 
 #include <nvtx3/nvToolsExt.h>
 
@@ -26,6 +27,7 @@ Layout make_layout(const moe_config& c, int T) {
                  k = (size_t)c.top_k;
     const size_t slots = t * k + t * (size_t)c.n_shared;
     L.err = take(64);
+    L.ctrl = take(kFusedCtrlBytes);  // fixed offset: the fused path keeps it across calls
     L.xin = take(t * H * 4);
     L.outbuf = take(t * H * 4);
     L.xq = take(t * H);
@@ -39,7 +41,6 @@ Layout make_layout(const moe_config& c, int T) {
     L.perm = take(t * k * 4);
     L.inv_perm = take(t * k * 4);
     L.active = take((E + 2) * 4);
-    L.ctrl = take(small_ctrl_bytes(c, T));
     L.hbuf = take(slots * I * 4);
     L.hq = take(slots * I);
     L.hd = take(slots * (I / 32) * 4);
@@ -143,6 +144,25 @@ static int check_bucket_fits(const moe_config& c, int T) {
 // The forward on a device-resident x; used by both public forwards.
 // ep_lo, ep_hi: the routed experts this call computes (all: 0, n_experts);
 // the picks outside the range are routed as usual but left to another call.
+// The fused path's control region of a workspace is initialised on the
+// first fused forward this process issues with it (or by moe_workspace_init);
+// the process remembers the regions it has initialised.  Initialising again
+// is always correct: no call uses the region meanwhile (calls that share a
+// workspace are ordered on one stream).
+static int ensure_fused_ctrl(int* ctrl, cudaStream_t s, bool force) {
+    static std::mutex mu;
+    static std::unordered_set<uint64_t> seen;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ECUDA;
+    const uint64_t key = ((uint64_t)(uint32_t)dev << 56) ^ (uint64_t)reinterpret_cast<uintptr_t>(ctrl);
+    std::lock_guard<std::mutex> lock(mu);
+    if (!force && seen.count(key)) return MOE_OK;
+    if (launch_fused_ctrl_init(ctrl, s) != cudaSuccess) return MOE_ECUDA;
+    if (seen.size() >= 4096) seen.clear();
+    seen.insert(key);
+    return MOE_OK;
+}
+
 static int forward_device(const moe_config& c, const float* x, int T, const float* router_w,
                           const float* router_bias, const moe_experts& routed, const moe_experts* shared,
                           float* out, char* ws, const Layout& L, cudaStream_t s, int ep_lo, int ep_hi) {
@@ -185,7 +205,8 @@ static int forward_device(const moe_config& c, const float* x, int T, const floa
         a.err = err;
         a.ep_lo = ep_lo;
         a.ep_hi = ep_hi;
-        int st2 = status_of(trace(0, s));
+        int st2 = ensure_fused_ctrl(a.ctrl, s, false);
+        if (!st2) st2 = status_of(trace(0, s));
         if (!st2) st2 = status_of(launch_small(a, s));
         if (!st2) st2 = status_of(trace(1, s));
         return st2;
@@ -341,6 +362,16 @@ MOE_API size_t moe_workspace_bytes(const moe_config* cfg, int T_max) {
     if (check_config(cfg) != MOE_OK || T_max < 0) return 0;
     if (check_bucket_fits(*cfg, T_max) != MOE_OK) return 0;  // no forward runs that many tokens
     return make_layout(*cfg, T_max).total;
+}
+
+MOE_API int moe_workspace_init(const moe_config* cfg, int T_max, void* workspace, size_t ws_bytes, void* stream) {
+    int st = check_config(cfg);
+    if (st) return st;
+    if (T_max < 0 || !workspace) return MOE_EINVAL;
+    const Layout L = make_layout(*cfg, T_max);
+    if (ws_bytes < L.total) return MOE_EWORKSPACE;
+    return ensure_fused_ctrl(reinterpret_cast<int*>(static_cast<char*>(workspace) + L.ctrl), (cudaStream_t)stream,
+                             true);
 }
 
 MOE_API int moe_layer_forward(const moe_config* cfg, const float* x, int T, const float* router_w,

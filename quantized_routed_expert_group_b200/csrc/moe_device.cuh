@@ -19,6 +19,7 @@ constexpr unsigned kFull = 0xffffffffu;
 // Error codes written to the workspace error word.
 constexpr int kErrIndex = 1;
 constexpr int kErrTimeout = 2;
+constexpr int kErrWorkspace = 3;  // the fused path's control region is not initialised
 
 __device__ __forceinline__ void set_error(int32_t* err, int code) {
     if (err) atomicCAS(reinterpret_cast<int*>(err), 0, code);

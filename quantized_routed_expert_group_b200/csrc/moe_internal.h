@@ -157,9 +157,13 @@ struct SmallArgs {
     int ep_lo, ep_hi;  // routed experts computed by this call: [ep_lo, ep_hi)
 };
 bool small_path_supported(const moe_config& c, int T);
-size_t small_ctrl_bytes(const moe_config& c, int T);
+// The fused path's control region: at a fixed workspace offset (the same
+// for every T), kept from one call to the next; launch_fused_ctrl_init
+// initialises it (zeros and a marker) before the first fused forward.
+constexpr size_t kFusedCtrlBytes = 1024;
+cudaError_t launch_fused_ctrl_init(int* ctrl, cudaStream_t s);
 cudaError_t launch_small(const SmallArgs& a, cudaStream_t s);
-constexpr int kSmallLaunches = 2;  // prologue + persistent kernel
+constexpr int kSmallLaunches = 1;  // the persistent kernel
 // Test hook (moe_debug_fault_injection): withhold one entry's first h
 // publication in the fused kernel, and bound its producer waits by wait_ns
 // (<= 0: the default).

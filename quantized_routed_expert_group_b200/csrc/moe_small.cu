@@ -28,16 +28,18 @@
 //   - down + combine: CTA c owns output rows [H c / grid, H (c+1) / grid) of
 //     every expert and combines them itself at the end, so no partial output
 //     crosses CTAs: no float atomics, bit-reproducible results.
-// * The only waits: the selection waits for every router item, and each
-//   down chunk waits for its expert's h (the producer polls, then copies the
-//   h codes into the slot with the weights).  Every wait is bounded and
-//   records a timeout in the error word.
-// * Weights known before the routing (the shared expert's) are issued first,
-//   and the CTA's shared-expert down rows are prefetched into L2 while the
-//   routing is computed.
-// * A tiny prologue kernel (Q8_0 of x, control-block reset) runs first; the
-//   main kernel is its programmatic dependent and issues its router rows
-//   before waiting for it.
+// * The only waits: the selection waits for every CTA's router logits (one
+//   grid-wide barrier), and each down chunk waits for its expert's h (the
+//   producer polls, then copies the h codes into the slot with the
+//   weights).  Every wait is bounded and records a timeout in the error word.
+// * Weights known before the routing (the shared expert's) are issued at the
+//   kernel's first instruction, and the CTA's shared-expert down rows are
+//   prefetched into L2 while the routing is computed.
+// * One launch: the consumer warps quantise x and compute the CTA's router
+//   logits themselves, so the weights start to stream as the kernel starts.
+//   The control words it shares between CTAs are never reset (see
+//   kFcMarker): each CTA reads their values before its router arrival and
+//   counts from there.
 #include <atomic>
 #include <cmath>
 
@@ -47,17 +49,15 @@
 
 namespace moe {
 
-// Build options of the one-token schedule (tuning knobs; the defaults are
-// the measured best): consumer groups, cooperative launch, one prologue block
-// per router row.
+// Build options of the schedule (tuning knobs; the defaults are the measured
+// best): consumer groups at one token; the producer holds the first weight
+// copies back until every consumer warp has its router row (so that the
+// router reads, which the selection waits for, do not queue behind them).
 #ifndef MOE_SMALL_GROUPS
 #define MOE_SMALL_GROUPS 2
 #endif
-#ifndef MOE_SMALL_COOPERATIVE
-#define MOE_SMALL_COOPERATIVE 1
-#endif
-#ifndef MOE_PROLOGUE_ROW_BLOCKS
-#define MOE_PROLOGUE_ROW_BLOCKS 1
+#ifndef MOE_SMALL_ROUTER_FIRST
+#define MOE_SMALL_ROUTER_FIRST 1
 #endif
 
 constexpr int kConsumerWarps = 8;  // warps of one consumer group
@@ -79,6 +79,8 @@ constexpr int kUnit = 32;          // gate/up rows per unit: one Q8_0 block of h
 constexpr int kMaxOwnedRows = 64;  // output rows one CTA owns
 constexpr int kScaleWin = 160;     // 16-byte aligned window over <= 32 fp32 scales
 constexpr int kMaxEntryWords = 5;  // ready bitmask words (entries <= 160)
+constexpr int kRouterRound = 4;    // router rows a CTA computes at a time
+constexpr uint64_t kFcMarkerValue = 0x3130646573756646ull;
 // Thread layout of the gate/up and down chunks: the 64 threads of a warp
 // pair (w, w+1) split the columns (K blocks c, c + 64, ...), the 4 warp pairs
 // split the rows.  Each thread loads its activation blocks once per chunk and
@@ -110,11 +112,19 @@ enum ItemKind : int {
     kItemSync = 7  // two groups: the other group's down outputs are complete
 };
 
-// Control block (int32 words, zeroed by the prologue on every call):
-// [units, -, -, -, gu_done[nent]]; units counts the routed gate/up units
-// taken; gu_done[e] counts (unit, token) pairs of entry e whose h codes are
-// published.
-enum : int { kCUnits = 0, kCHeader = 4 };
+// Control region of the fused path (int32 words at a fixed workspace offset,
+// the only workspace state kept from one call to the next):
+//   [0, 1]  a 64-bit marker that moe_workspace_init writes; a call that does
+//           not find it records kErrWorkspace and computes nothing;
+//   [2]     the router barrier: each CTA adds 1, CTA 0 adds 2^31 - (grid - 1),
+//           so that bit 31 flips when the last CTA arrives and the low 31
+//           bits are zero again (zero after the initialisation);
+//   [3]     routed gate/up units taken (T > 1);
+//   [4 + e] (unit, token) pairs of entry e whose h codes are published.
+// The counters are never reset: every CTA reads them before its router
+// arrival, and nobody adds to them before the barrier completes, so every
+// CTA counts from the same values (differences modulo 2^32).
+enum : int { kFcMarker = 0, kFcBarrier = 2, kFcUnits = 3, kFcDone = 4 };
 
 // One expert of the batch union: entry 0 is the shared expert, entry 1 + a
 // the a-th routed expert in ascending id order.
@@ -149,8 +159,7 @@ struct SmallGeom {
     int a_sd;  // act-area offset of the row-scale window (down chunks)
     int act_bytes;
     int slot_bytes;
-    int ctrl_words;
-    int o_xq, o_xd, o_bar, o_meta, o_urec, o_gpart, o_usc, o_ent, o_selw, o_inv, o_ys, o_misc;
+    int o_xq, o_xd, o_bar, o_meta, o_urec, o_gpart, o_usc, o_ent, o_selw, o_inv, o_ys, o_misc, o_base, o_part, o_bias;
     int smem_bytes;
 };
 
@@ -178,7 +187,7 @@ struct SmallParams {
     float* hd;
     float* y;
     float* out;
-    int* ctrl;
+    int* ctrl;  // the control region (kFc*)
     int32_t* err;
     uint64_t wait_ns;  // bound of the producer's waits (see kWaitNs)
     int fault_entry;   // test hook: the entry whose first unit's h codes are never published (-1: none)
@@ -221,6 +230,9 @@ SmallGeom small_geometry(const moe_config& c, int T, int grid) {
     g.cpu = g.rg > 0 ? kUnit / g.rg : 0;
     g.nu = I / kUnit;
     g.rpc = (H + grid - 1) / grid;
+    // one token: the rows are split so that every CTA streams the same bytes
+    // (see owned_rows), up to twice the even share
+    if (g.tmax == 1) g.rpc = min(2 * g.rpc, kMaxOwnedRows);
     const int rd = kSlotWeightBytes / rowI;
     g.rd = rd > kMaxOwnedRows ? kMaxOwnedRows : rd;
     g.nys = T * c.top_k + T * c.n_shared;
@@ -231,14 +243,13 @@ SmallGeom small_geometry(const moe_config& c, int T, int grid) {
     g.act_bytes = round_up(g.a_sd + kMaxOwnedRows * 4 + 32, 128);
     if (g.act_bytes < 2 * kScaleWin) g.act_bytes = round_up(2 * kScaleWin, 128);
     g.slot_bytes = kSlotWeightBytes + g.act_bytes;
-    g.ctrl_words = round_up(kCHeader + g.nent, 4);
     int o = 0;
     g.o_xq = o;
     o += round_up(g.tmax * H, 128);
     g.o_xd = o;
     o += round_up(g.tmax * (H / 32) * 4, 128);
     g.o_bar = o;
-    o += 128;  // full[4], empty[4], routing, ufull[2], ufree[2], gsync, gexit
+    o += 128;  // full[4], empty[4], routing, ufull[2], ufree[2], gsync, gexit, rowsin
     g.o_meta = o;
     o += round_up((int)sizeof(SlotMeta) * kMaxSlots, 128);
     g.o_urec = o;
@@ -257,6 +268,12 @@ SmallGeom small_geometry(const moe_config& c, int T, int grid) {
     o += round_up(g.nys * g.rpc * 8, 128);
     g.o_misc = o;
     o += 128;
+    g.o_base = o;  // the control counters at the CTA's start: [units, done[nent]]
+    o += round_up((1 + g.nent) * 4, 128);
+    g.o_part = o;  // router logits: [expert of the round][eighth][token] fp64
+    o += kRouterRound * 8 * 4 * 8;
+    g.o_bias = o;  // router correction bias [E]
+    o += round_up(E * 4, 128);
     // as many ring slots (up to four) as the shared memory holds
     const int smem_max = device_info().max_smem_optin;
     while (g.nslot > 2 && o + g.nslot * g.slot_bytes > smem_max) --g.nslot;
@@ -265,6 +282,7 @@ SmallGeom small_geometry(const moe_config& c, int T, int grid) {
     const int ring = g.nslot * g.slot_bytes;
     g.o_xq += ring; g.o_xd += ring; g.o_bar += ring; g.o_meta += ring; g.o_urec += ring; g.o_gpart += ring;
     g.o_usc += ring; g.o_ent += ring; g.o_selw += ring; g.o_inv += ring; g.o_ys += ring; g.o_misc += ring;
+    g.o_base += ring; g.o_part += ring; g.o_bias += ring;
     g.smem_bytes = o + ring;
     return g;
 }
@@ -281,33 +299,36 @@ bool small_path_supported(const moe_config& c, int T) {
     const SmallGeom g = small_geometry(c, T, device_info().sm_count);
     if (g.rg < 4) return false;  // at least one gate/up row per row group
     if (c.hidden / 32 > kColThreads * kMaxGuBlocks || c.inter / 32 > kColThreads * kMaxDownBlocks) return false;
-    if (g.rd < 1 || g.rpc > kMaxOwnedRows) return false;
+    if (g.rd < 1 || g.rpc > kMaxOwnedRows || (c.hidden + g.grid - 1) / g.grid > g.rpc) return false;
     if (g.nent > 32 * kMaxEntryWords) return false;
     if (select_scratch_bytes(T, c.n_experts) > g.slot_bytes) return false;
     return g.smem_bytes <= device_info().max_smem_optin;
 }
 
-size_t small_ctrl_bytes(const moe_config& c, int T) {
-    const SmallGeom g = small_geometry(c, T > 0 ? T : 1, device_info().sm_count);
-    return (size_t)g.ctrl_words * 4;
+static_assert(kFcDone + 32 * kMaxEntryWords <= (int)(kFusedCtrlBytes / 4), "fused control region");
+
+__global__ void k_fused_ctrl_init(int* ctrl) {
+    for (int i = threadIdx.x; i < (int)(kFusedCtrlBytes / 4); i += blockDim.x) ctrl[i] = 0;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        ctrl[kFcMarker] = (int)(uint32_t)kFcMarkerValue;
+        ctrl[kFcMarker + 1] = (int)(uint32_t)(kFcMarkerValue >> 32);
+    }
+}
+
+cudaError_t launch_fused_ctrl_init(int* ctrl, cudaStream_t s) {
+    k_fused_ctrl_init<<<1, 256, 0, s>>>(ctrl);
+    return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
-// Prologue: reset the control block, quantise x and compute the router
-// logits.  It launches its dependent (the main kernel) at once; the main
-// kernel's CTAs, which need most of an SM's shared memory, start as the
-// prologue's blocks on their SM exit, and read the logits after waiting for
-// this grid.
-//
-// Router logits (the router row of expert e dotted with x, per token): block
-// b takes experts b, b + grid, ... (one row per block: the grid has a block
-// per expert, at least one per SM); warp w takes eighth w of the hidden
-// dimension, each lane holds its weights (float4) in registers and keeps four
-// compensated fp32 sums per token (one per float4 component, about 2^-48
-// relative each), folded into fp64; the eighths are added in fp64 in a fixed
-// order.
+// Router logits (the router row of expert e dotted with x, per token): CTA c
+// computes experts c, c + grid, ...; a warp takes eighth w of the hidden
+// dimension of one row, each lane holds its weights (float4) in registers
+// and keeps four compensated fp32 sums per token (one per float4 component,
+// about 2^-48 relative each), folded into fp64; the eighths are added in fp64
+// in a fixed order.
 // ---------------------------------------------------------------------------
-constexpr int kPrologueThreads = 256;
 constexpr int kRouterVec = 6;  // float4 of one router row per lane: hidden / 8 / 4 / 32 <= 6
 
 __device__ __forceinline__ void dfacc4_add(DFAcc (&acc)[4], float4 x, float4 w) {
@@ -328,63 +349,6 @@ __device__ __forceinline__ void load_router_row(const float* router_w, int e, in
     }
 }
 
-__global__ void __launch_bounds__(kPrologueThreads) k_small_prologue(const float* __restrict__ x, int T, int H, int E,
-                                                                     const float* __restrict__ router_w,
-                                                                     double* __restrict__ logits,
-                                                                     int8_t* __restrict__ xq, float* __restrict__ xd,
-                                                                     int* ctrl, int ctrl_words, int32_t* err) {
-    pdl_launch_dependents();
-    __shared__ double part[8][4];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // the block's first router row is requested first (its latency covers
-    // the rest of the setup), its later rows go to L2 meanwhile
-    float4 w[kRouterVec];
-    load_router_row(router_w, blockIdx.x, E, H, warp, lane, w);
-    if (threadIdx.x == 0)
-        for (int e = blockIdx.x + gridDim.x; e < E; e += gridDim.x)
-            bulk_prefetch_l2(router_w + (int64_t)e * H, (uint32_t)(H * 4));
-    const int gtid = blockIdx.x * blockDim.x + threadIdx.x;
-    for (int i = gtid; i < ctrl_words; i += gridDim.x * blockDim.x) ctrl[i] = 0;
-    if (gtid == 0) *err = 0;
-    // Q8_0 of x, one block of 32 per warp
-    const int64_t nblk = (int64_t)T * (H / 32);
-    for (int64_t b = (int64_t)blockIdx.x * 8 + warp; b < nblk; b += (int64_t)gridDim.x * 8) {
-        int8_t q;
-        float d;
-        q8_0_warp(x[b * kQBlock + lane], q, d);
-        xq[b * kQBlock + lane] = q;
-        if (lane == 0) xd[b] = d;
-    }
-    // router logits
-    const int n8 = H / 32;  // float4 per eighth
-#pragma unroll 1
-    for (int e = blockIdx.x; e < E; e += gridDim.x) {
-        if (e != (int)blockIdx.x) load_router_row(router_w, e, E, H, warp, lane, w);
-#pragma unroll 1
-        for (int t = 0; t < T; ++t) {
-            const float4* xr = reinterpret_cast<const float4*>(x + (int64_t)t * H) + warp * n8;
-            DFAcc acc[4];
-#pragma unroll
-            for (int u = 0; u < kRouterVec; ++u) {
-                const int j = lane + 32 * u;
-                dfacc4_add(acc, j < n8 ? __ldg(xr + j) : make_float4(0.f, 0.f, 0.f, 0.f), w[u]);
-            }
-            double v = (acc[0].value() + acc[1].value()) + (acc[2].value() + acc[3].value());
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
-            if (lane == 0) part[warp][t] = v;
-        }
-        __syncthreads();
-        if ((int)threadIdx.x < T) {
-            double v = 0.0;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) v += part[k][threadIdx.x];
-            logits[(int64_t)threadIdx.x * E + e] = v;
-        }
-        __syncthreads();
-    }
-}
-
 // ---------------------------------------------------------------------------
 // Shared-memory layout of the main kernel
 // ---------------------------------------------------------------------------
@@ -399,6 +363,7 @@ struct SmemPtrs {
     uint64_t* ufree;    // [2] the finisher warp has read them
     uint64_t* gsync;    // the syncing group's warps: their down outputs are in ys
     uint64_t* gexit;    // every consumer warp has left its loop
+    uint64_t* rowsin;   // every consumer warp holds its first router row
     UnitRec* urec;      // [2] the unit to finish
     SlotMeta* meta;
     float* gpart;    // [2][32][2][2][4] gate/up partial dots of a unit: [buffer][pair][gate/up][half][token]
@@ -407,7 +372,12 @@ struct SmemPtrs {
     float* selw;     // [T*k] routing weights
     int* inv;        // [T*k] slot of pair (t, j)
     float* ys;       // [nys][rpc][2] down outputs of the CTA's rows, per column half
-    int* misc;       // [0] = routed entries U
+    int* misc;       // [0] = routed entries U, [1] routed pairs, [4 + group] units seen,
+                     // [8] bit 31 of the router barrier before this call's arrivals,
+                     // [9] the control region is initialised
+    uint32_t* base;  // [1 + nent] the control counters at the CTA's start: units, done[e]
+    double* part;    // [kRouterRound][8][4] router logits per eighth of the hidden dimension
+    float* bias;     // [E] router correction bias
 };
 
 __device__ __forceinline__ SmemPtrs carve(uint8_t* base, const SmallGeom& g) {
@@ -422,6 +392,7 @@ __device__ __forceinline__ SmemPtrs carve(uint8_t* base, const SmallGeom& g) {
     s.ufree = s.ufull + 2;
     s.gsync = s.ufree + 2;
     s.gexit = s.gsync + 1;
+    s.rowsin = s.gexit + 1;
     s.meta = reinterpret_cast<SlotMeta*>(base + g.o_meta);
     s.urec = reinterpret_cast<UnitRec*>(base + g.o_urec);
     s.gpart = reinterpret_cast<float*>(base + g.o_gpart);
@@ -431,7 +402,159 @@ __device__ __forceinline__ SmemPtrs carve(uint8_t* base, const SmallGeom& g) {
     s.inv = reinterpret_cast<int*>(base + g.o_inv);
     s.ys = reinterpret_cast<float*>(base + g.o_ys);
     s.misc = reinterpret_cast<int*>(base + g.o_misc);
+    s.base = reinterpret_cast<uint32_t*>(base + g.o_base);
+    s.part = reinterpret_cast<double*>(base + g.o_part);
+    s.bias = reinterpret_cast<float*>(base + g.o_bias);
     return s;
+}
+
+// Wait (bounded) until the router barrier has flipped past this call's
+// value: every CTA has published its logits.  One thread polls.
+__device__ __forceinline__ bool router_barrier_wait(const SmallParams& p, const SmemPtrs& s, uint64_t budget_ns) {
+    const uint32_t b0 = (uint32_t)s.misc[8] >> 31;
+    const uint64_t t0 = global_timer_ns();
+    while (((uint32_t)ld_acquire_gpu(p.ctrl + kFcBarrier) >> 31) == b0) {
+        if (global_timer_ns() - t0 > budget_ns) return false;
+        __nanosleep(64);
+    }
+    return true;
+}
+
+// Q8_0 of one block of 32 activations held as a float4 by each of 8
+// consecutive lanes (the same arithmetic as q8_0_warp): the 4 codes packed
+// little-endian into one word, the block scale in d.
+__device__ __forceinline__ uint32_t q8_0_octet(float4 v, float& d) {
+    float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, o));
+    if (!(a >= FLT_MIN)) {
+        d = 0.0f;
+        return 0u;
+    }
+    d = __fdiv_rn(a, 127.0f);
+    const float id = __fdiv_rn(1.0f, d);
+    const float f[4] = {v.x, v.y, v.z, v.w};
+    uint32_t w = 0u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float r = roundf(__fmul_rn(f[i], id));
+        r = fminf(fmaxf(r, -127.0f), 127.0f);
+        w |= ((uint32_t)(int)r & 0xFFu) << (8 * i);
+    }
+    return w;
+}
+
+// The consumers' start (all G consumer groups, nthr threads, tid < nthr):
+// the CTA's router logits, published to the workspace, and the Q8_0 of x
+// (codes staged in natural order in `stage`, ring slot 0, which only the
+// selection uses later; then put in the weights' order in s.xq; CTA 0 also
+// publishes xq and xd).  Ends with the CTA's arrival on the router barrier.
+template <int WBITS>
+__device__ __forceinline__ void consumers_start(const SmallParams& p, const SmemPtrs& s, uint8_t* stage, int tid,
+                                                int nthr) {
+    const int warp = tid >> 5, lane = tid & 31, nw = nthr >> 5;
+    const int c = blockIdx.x, grid = gridDim.x;
+    const int T = p.T, H = p.H, E = p.E, nb = H / 32;
+    const int n_mine = c < E ? (E - 1 - c) / grid + 1 : 0;  // router rows of this CTA
+    // the first router row of the warp is requested first: its latency (HBM)
+    // covers the quantisation of x
+    float4 w[kRouterVec];
+    load_router_row(p.router_w, warp / 8 < n_mine ? c + grid * (warp / 8) : E, E, H, warp & 7, lane, w);
+    for (int e = tid; e < E; e += nthr) s.bias[e] = __ldg(p.bias + e);  // read by the selection
+    // Q8_0 of x: a warp takes 4 blocks at a time (8 lanes, a float4 each);
+    // the loads of up to 8 steps are issued before any is used
+    {
+        uint32_t* nat = reinterpret_cast<uint32_t*>(stage);  // [T][H] codes
+        const int nblk = T * nb, nstep = (nblk + 3) / 4;
+        for (int s0 = warp; s0 < nstep; s0 += 8 * nw) {
+            float4 v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int blk = 4 * (s0 + j * nw) + (lane >> 3);
+                v[j] = blk < nblk ? __ldg(reinterpret_cast<const float4*>(p.x) + (int64_t)blk * 8 + (lane & 7))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int st = s0 + j * nw;
+                if (st >= nstep) break;  // the same for the whole warp
+                const int blk = 4 * st + (lane >> 3);
+                float d;
+                const uint32_t q = q8_0_octet(v[j], d);
+                if (blk < nblk) {
+                    nat[(int64_t)blk * 8 + (lane & 7)] = q;
+                    if ((lane & 7) == 0) s.xd[blk] = d;
+                }
+            }
+        }
+    }
+    // router logits, kRouterRound rows at a time: job = (row of the round,
+    // eighth of the hidden dimension); each warp reports (rowsin) once its
+    // first row has arrived, i.e. after that row's dot
+    const int n8 = H / 32;
+    bool rows_in = false;
+    for (int r0 = 0; r0 < n_mine; r0 += kRouterRound) {
+        const int nr = min(kRouterRound, n_mine - r0);
+        for (int job = warp; job < nr * 8; job += nw) {
+            const int i = job >> 3, w8 = job & 7, e = c + grid * (r0 + i);
+            if (!(r0 == 0 && job == warp)) load_router_row(p.router_w, e, E, H, w8, lane, w);
+#pragma unroll 1
+            for (int t = 0; t < T; ++t) {
+                const float4* xr = reinterpret_cast<const float4*>(p.x + (int64_t)t * H) + w8 * n8;
+                DFAcc acc[4];
+#pragma unroll
+                for (int u = 0; u < kRouterVec; ++u) {
+                    const int j = lane + 32 * u;
+                    dfacc4_add(acc, j < n8 ? __ldg(xr + j) : make_float4(0.f, 0.f, 0.f, 0.f), w[u]);
+                }
+                double v = (acc[0].value() + acc[1].value()) + (acc[2].value() + acc[3].value());
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+                if (lane == 0) s.part[(i * 8 + w8) * 4 + t] = v;
+            }
+            if (!rows_in) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(s.rowsin);
+                rows_in = true;
+            }
+        }
+        named_barrier(3, nthr);
+        if (tid < nr * T) {
+            const int i = tid / T, t = tid - i * T;
+            double v = 0.0;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v += s.part[(i * 8 + k) * 4 + t];
+            p.logits[(int64_t)t * E + c + grid * (r0 + i)] = v;
+        }
+        named_barrier(3, nthr);
+    }
+    if (!rows_in && lane == 0) mbar_arrive(s.rowsin);
+    // the staged codes in the weights' order, each 32-code block split in
+    // 16-byte halves so that lanes read consecutive words (after every
+    // warp's staging: a CTA without router rows has had no barrier yet)
+    named_barrier(3, nthr);
+    for (int job = tid; job < T * nb; job += nthr) {
+        const int t = job / nb, b = job - t * nb;
+        const uint4 lo = *reinterpret_cast<const uint4*>(stage + (size_t)job * 32);
+        const uint4 hi = *reinterpret_cast<const uint4*>(stage + (size_t)job * 32 + 16);
+        const ActBlock a = WBITS == 4 ? act_nibble_order(lo, hi)
+                         : WBITS == 2 ? act_crumb_order(lo, hi)
+                                      : act_natural(lo, hi);
+        *reinterpret_cast<uint4*>(s.xq + ((size_t)(t * 2 + 0) * nb + b) * 16) = make_uint4(a.v[0], a.v[1], a.v[2], a.v[3]);
+        *reinterpret_cast<uint4*>(s.xq + ((size_t)(t * 2 + 1) * nb + b) * 16) = make_uint4(a.v[4], a.v[5], a.v[6], a.v[7]);
+        if (c == 0) {
+            *reinterpret_cast<uint4*>(p.xq + (size_t)job * 32) = lo;
+            *reinterpret_cast<uint4*>(p.xq + (size_t)job * 32 + 16) = hi;
+            p.xd[job] = s.xd[job];
+        }
+    }
+    // every consumer thread's logits are written: the CTA's arrival (CTA 0
+    // adds 2^31 - (grid - 1), the others 1: bit 31 flips at the last one)
+    named_barrier(3, nthr);
+    if (tid == 0) {
+        const int add = c == 0 ? (int)(0x80000000u - (uint32_t)(grid - 1)) : 1;
+        red_add_release_gpu(p.ctrl + kFcBarrier, add);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -611,7 +734,7 @@ struct Producer {
     }
 
     __forceinline__ __device__ bool entry_done(int i, int U) const {
-        return i <= U && ld_acquire_gpu(p.ctrl + kCHeader + i) >= p.g.nu * s.ent[i].n;
+        return i <= U && (uint32_t)ld_acquire_gpu(p.ctrl + kFcDone + i) - s.base[1 + i] >= (uint32_t)(p.g.nu * s.ent[i].n);
     }
 
     // Wait until every unit of entry e has published its h codes.  Each poll
@@ -755,13 +878,13 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
     unsigned long long* lkey = reinterpret_cast<unsigned long long*>(wsum + 16);  // [T][tg*kk] listed keys
     int* lid = reinterpret_cast<int*>(lkey + T * p.tg * min(k, per));            // [T][tg*kk] listed ids
     const int warp = tid >> 5, lane = tid & 31;
-    // the logits are the prologue's: the consumers waited for its grid
+    // the logits are every CTA's: the router barrier has completed
     // 1. s, c and keys
 #pragma unroll 1
     for (int i = tid; i < TE; i += kConsumers) {
         const double l = __ldcg(p.logits + i);
         const double sv = 1.0 / (1.0 + exp(-l));
-        const double cv = sv + (double)__ldg(p.bias + i % E);
+        const double cv = sv + (double)s.bias[i % E];
         ss[i] = sv;
         sc[i] = cv;
         key[i] = order_key(cv);
@@ -1206,7 +1329,8 @@ __device__ __forceinline__ void do_gateup(const SmallParams& p, const SmemPtrs& 
 // release of the codes to the other CTAs; the consumer warps never wait for
 // this (nor for the release fence) ----
 __device__ __forceinline__ void finisher(const SmallParams& p, const SmemPtrs& s, int lane) {
-    pdl_wait();  // the control block was reset by the prologue
+    bool open = false;  // the router barrier has completed (every CTA has read its counters)
+    bool gave_up = false;
 #pragma unroll 1
     for (int k = 0;; ++k) {
         const int buf = k & 1;
@@ -1234,9 +1358,15 @@ __device__ __forceinline__ void finisher(const SmallParams& p, const SmemPtrs& s
         __syncwarp();
         if (lane == 0) {
             mbar_arrive(&s.ufree[buf]);
+            if (!open && !gave_up) {
+                open = router_barrier_wait(p, s, kSlackWaits * p.wait_ns);
+                gave_up = !open;
+                if (gave_up) set_error(p.err, kErrTimeout);
+            }
             fence_acq_rel_gpu();  // the warp's h codes before the count (release pattern)
-            if (r.entry != p.fault_entry || r.blk != 0) red_add_relaxed_gpu(p.ctrl + kCHeader + r.entry, n);
+            if (open && (r.entry != p.fault_entry || r.blk != 0)) red_add_relaxed_gpu(p.ctrl + kFcDone + r.entry, n);
         }
+        open = __shfl_sync(kFull, open, 0);
         __syncwarp();
     }
 }
@@ -1388,6 +1518,42 @@ __device__ __forceinline__ void do_combine(const SmallParams& p, const SmemPtrs&
     if ((tid & 31) == 0) mbar_arrive(empty);
 }
 
+// Output rows [r0, r1) that CTA c owns in the down projection and combine.
+// More than one token: an even split.  One token: the gate/up units go round
+// robin (unit u to CTA u mod grid), so the first n1 = units mod grid CTAs
+// stream one unit more; they own fewer rows, so that every CTA streams the
+// same bytes (gate/up units + its rows of every entry's down matrix), as far
+// as the row cap allows.  Every CTA computes the same split.
+__device__ __forceinline__ void owned_rows(const SmallParams& p, int n_entries, int c, int grid, int& r0, int& r1) {
+    const int H = p.H;
+    if (p.T > 1 || n_entries <= 0) {
+        r0 = (int)((int64_t)H * c / grid);
+        r1 = (int)((int64_t)H * (c + 1) / grid);
+        return;
+    }
+    const int n_units = n_entries * p.g.nu;
+    const int n1 = n_units % grid;
+    // a unit's bytes in rows of every entry's down matrix
+    const double unit_rows = (double)(2 * kUnit * p.H) / (double)(n_entries * p.I);
+    double a = ((double)H - (double)(grid - n1) * unit_rows) / (double)grid;  // rows of a CTA with one more unit
+    a = fmax(a, 0.0);
+    double b = n1 < grid ? ((double)H - (double)n1 * a) / (double)(grid - n1) : a;
+    const double cap = (double)p.g.rpc;
+    if (b > cap) {  // the cap binds: even split instead
+        r0 = (int)((int64_t)H * c / grid);
+        r1 = (int)((int64_t)H * (c + 1) / grid);
+        return;
+    }
+    auto start = [&](int cc) -> int {
+        if (cc >= grid) return H;
+        const double v = cc <= n1 ? cc * a : n1 * a + (cc - n1) * b;
+        const int r = (int)floor(v + 1e-6);
+        return r < H ? r : H;
+    };
+    r0 = start(c);
+    r1 = start(c + 1);
+}
+
 // ---------------------------------------------------------------------------
 // Main kernel
 // ---------------------------------------------------------------------------
@@ -1401,7 +1567,6 @@ __global__ void __launch_bounds__(Roles<TM>::kThreads, 1) k_moe_small(const __gr
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x, grid = gridDim.x;
-    const int r0 = (int)((int64_t)p.H * c / grid), r1 = (int)((int64_t)p.H * (c + 1) / grid);
     if (tid == 0) {
         for (int i = 0; i < g.nslot; ++i) {
             mbar_init(&s.full[i], 1);
@@ -1414,9 +1579,28 @@ __global__ void __launch_bounds__(Roles<TM>::kThreads, 1) k_moe_small(const __gr
         }
         mbar_init(s.gsync, kConsumerWarps);
         mbar_init(s.gexit, G * kConsumerWarps);
+        mbar_init(s.rowsin, G * kConsumerWarps);
         fence_barrier_init();
     }
+    if (warp == 0) {
+        // the control region: its marker, and the counters as this CTA finds
+        // them (read before its router arrival; see kFcMarker).  Plain loads
+        // issued together: what earlier kernels wrote is visible at launch,
+        // and this call's additions come only after every CTA's arrival.
+        const volatile int* cv = p.ctrl;
+        for (int i = lane; i < 1 + g.nent; i += 32)
+            s.base[i] = (uint32_t)(i == 0 ? cv[kFcUnits] : cv[kFcDone + i - 1]);
+        if (lane == 0) {
+            const uint32_t m0 = (uint32_t)cv[kFcMarker], m1 = (uint32_t)cv[kFcMarker + 1];
+            const bool init = (((uint64_t)m1 << 32) | m0) == kFcMarkerValue;
+            s.misc[9] = init ? 1 : 0;
+            s.misc[8] = cv[kFcBarrier];
+            if (c == 0) *p.err = 0;  // before CTA 0's router arrival: no CTA records an error before it
+            if (!init) set_error(p.err, kErrWorkspace);
+        }
+    }
     __syncthreads();
+    if (!s.misc[9]) return;  // the same in every CTA
 
     if (warp == R::kFinisherWarp) {
         finisher(p, s, lane);
@@ -1426,9 +1610,20 @@ __global__ void __launch_bounds__(Roles<TM>::kThreads, 1) k_moe_small(const __gr
         // ------------------------- producer -------------------------
         Producer pr(p, s, lane, G);
         const int64_t rowI = (int64_t)p.I * p.wbits / 8;
-        if (p.ns && lane == 0 && r1 > r0)
-            bulk_prefetch_l2(p.shared.w_down + (int64_t)r0 * rowI, (uint32_t)((r1 - r0) * rowI));
         pr.marker(kItemSelect);
+        if (MOE_SMALL_ROUTER_FIRST) {
+            int okr = 1;
+            if (lane == 0) okr = mbar_wait_ns(s.rowsin, 0, p.wait_ns) ? 1 : 0;
+            okr = __shfl_sync(kFull, okr, 0);
+            if (!okr) pr.fail();
+        }
+        {
+            // the shared expert's down rows this CTA will probably own
+            int q0, q1;
+            owned_rows(p, p.k + (p.ns ? 1 : 0), c, grid, q0, q1);
+            if (p.ns && lane == 0 && q1 > q0)
+                bulk_prefetch_l2(p.shared.w_down + (int64_t)q0 * rowI, (uint32_t)((q1 - q0) * rowI));
+        }
         // the shared expert's gate/up units need no routing
         EntryInfo e0;
         e0.expert = -1;
@@ -1439,8 +1634,6 @@ __global__ void __launch_bounds__(Roles<TM>::kThreads, 1) k_moe_small(const __gr
         for (int u = c; u < n_pre; u += grid)
             for (int ch = 0; ch < g.cpu; ++ch) pr.gateup(0, e0, u, ch);
         // the routed part of the schedule needs this CTA's routing tables
-        // (and the control block the prologue reset)
-        pdl_wait();
         int ok = 1;
         if (lane == 0) ok = mbar_wait_ns(s.routing, 0, kSlackWaits * p.wait_ns) ? 1 : 0;
         ok = __shfl_sync(kFull, ok, 0);
@@ -1457,11 +1650,11 @@ __global__ void __launch_bounds__(Roles<TM>::kThreads, 1) k_moe_small(const __gr
             // take more, so every CTA reaches its down chunks at about the
             // same time
             int next = 0;
-            if (lane == 0) next = atom_add_relaxed_gpu(p.ctrl + kCUnits, 1);
+            if (lane == 0) next = (int)((uint32_t)atom_add_relaxed_gpu(p.ctrl + kFcUnits, 1) - s.base[0]);
             next = __shfl_sync(kFull, next, 0);
             while (next < n_routed && !pr.aborted) {
                 const int r = next;
-                if (lane == 0) next = atom_add_relaxed_gpu(p.ctrl + kCUnits, 1);
+                if (lane == 0) next = (int)((uint32_t)atom_add_relaxed_gpu(p.ctrl + kFcUnits, 1) - s.base[0]);
                 const int entry = 1 + r / g.nu, blk = r % g.nu;
                 const EntryInfo ei = s.ent[entry];
                 for (int ch = 0; ch < g.cpu; ++ch) pr.gateup(entry, ei, blk, ch);
@@ -1478,6 +1671,8 @@ __global__ void __launch_bounds__(Roles<TM>::kThreads, 1) k_moe_small(const __gr
                 for (int ch = 0; ch < g.cpu; ++ch) pr.gateup(entry, ei, blk, ch);
             }
         }
+        int r0, r1;
+        owned_rows(p, U + (p.ns ? 1 : 0), c, grid, r0, r1);
         for (int entry = first; entry <= U && !pr.aborted; ++entry) {
             const EntryInfo ei = s.ent[entry];
             for (int rr = r0; rr < r1; rr += g.rd) {
@@ -1502,24 +1697,7 @@ __global__ void __launch_bounds__(Roles<TM>::kThreads, 1) k_moe_small(const __gr
     // ------------------------- consumers -------------------------
     const int group = warp / kConsumerWarps;     // consumer group
     const int gtid = tid - group * kConsumers;   // thread index inside the group
-    pdl_wait();
-    {
-        // Q8_0 activations of all tokens into shared memory, each 32-code
-        // block split in 16-byte halves so that lanes read consecutive words
-        const int nb = p.H / 32;
-        for (int job = tid; job < p.T * nb; job += G * kConsumers) {
-            const int t = job / nb, b = job % nb;
-            const uint4 lo = __ldcg(reinterpret_cast<const uint4*>(p.xq + (int64_t)t * p.H + b * 32));
-            const uint4 hi = __ldcg(reinterpret_cast<const uint4*>(p.xq + (int64_t)t * p.H + b * 32 + 16));
-            const ActBlock a = WBITS == 4 ? act_nibble_order(lo, hi)
-                             : WBITS == 2 ? act_crumb_order(lo, hi)
-                                          : act_natural(lo, hi);
-            *reinterpret_cast<uint4*>(s.xq + ((size_t)(t * 2 + 0) * nb + b) * 16) = make_uint4(a.v[0], a.v[1], a.v[2], a.v[3]);
-            *reinterpret_cast<uint4*>(s.xq + ((size_t)(t * 2 + 1) * nb + b) * 16) = make_uint4(a.v[4], a.v[5], a.v[6], a.v[7]);
-        }
-        for (int job = tid; job < p.T * nb; job += G * kConsumers) s.xd[job] = __ldcg(p.xd + job);
-    }
-    named_barrier(3, G * kConsumers);  // every consumer warp, before any item
+    consumers_start<WBITS>(p, s, s.slots, tid, G * kConsumers);
     // group g takes ring slots g, g + G, ... in order
     int slot = group;
     uint32_t pf = 0;
@@ -1538,7 +1716,10 @@ __global__ void __launch_bounds__(Roles<TM>::kThreads, 1) k_moe_small(const __gr
         } else if (m.kind == kItemDown) {
             do_down<WBITS, TM>(p, s, m, data, gtid, empty);
         } else if (m.kind == kItemSelect) {
-            do_select(p, s, data, gtid);  // always group 0's: the first item
+            // always group 0's: the first item; every CTA's logits first
+            if (gtid == 0 && !router_barrier_wait(p, s, kSlackWaits * p.wait_ns)) set_error(p.err, kErrTimeout);
+            consumers_sync();
+            do_select(p, s, data, gtid);
             __syncwarp();
             if (lane == 0) mbar_arrive(empty);  // the slot was the scratch
         } else if (m.kind == kItemSync) {
@@ -1580,7 +1761,7 @@ __global__ void __launch_bounds__(Roles<TM>::kThreads, 1) k_moe_small(const __gr
 // other CTAs' h codes), so the grid must be resident all at once: it is
 // launched as a cooperative grid (one CTA per SM), which the runtime only
 // starts when every CTA can run, also beside another forward on another
-// stream.  It is also the prologue's programmatic dependent.
+// stream.
 template <int WBITS, int TM>
 static cudaError_t launch_small_t(const SmallParams& prm, cudaStream_t st) {
     static bool attr_done[64];
@@ -1603,13 +1784,11 @@ static cudaError_t launch_small_t(const SmallParams& prm, cudaStream_t st) {
     cfg.blockDim = dim3(Roles<TM>::kThreads);
     cfg.dynamicSmemBytes = prm.g.smem_bytes;
     cfg.stream = st;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    attr[1].id = cudaLaunchAttributeCooperative;
-    attr[1].val.cooperative = 1;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = MOE_SMALL_COOPERATIVE ? 2 : 1;
+    cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, k_moe_small<WBITS, TM>, prm);
 }
 
@@ -1636,13 +1815,6 @@ cudaError_t launch_small(const SmallArgs& a, cudaStream_t st) {
     p.fault_entry = g_fault_entry.load();
     p.g = small_geometry(c, a.T, device_info().sm_count);
     if (p.g.smem_bytes > device_info().max_smem_optin) return cudaErrorInvalidConfiguration;
-    // one prologue block per router row (at least one per SM): every row's
-    // loads are issued at once, so the logits take one DRAM round trip
-    const int pro_grid = (MOE_PROLOGUE_ROW_BLOCKS && c.n_experts > p.g.grid) ? c.n_experts : p.g.grid;
-    k_small_prologue<<<pro_grid, kPrologueThreads, 0, st>>>(a.x, a.T, c.hidden, c.n_experts, a.router_w, a.logits,
-                                                            a.xq, a.xd, a.ctrl, p.g.ctrl_words, a.err);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
     const int tm = p.g.tmax;
     if (c.wbits == 4) {
         if (tm == 1) return launch_small_t<4, 1>(p, st);

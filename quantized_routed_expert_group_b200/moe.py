@@ -51,6 +51,7 @@ _SIGS = {
     "moe_router_select": ([ctypes.POINTER(MoeConfig), _vp, _int, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _int),
     "moe_bucket_tokens": ([ctypes.POINTER(MoeConfig), _vp, _int, _vp, _vp, _vp, _vp], _int),
     "moe_workspace_bytes": ([ctypes.POINTER(MoeConfig), _int], _sz),
+    "moe_workspace_init": ([ctypes.POINTER(MoeConfig), _int, _vp, _sz, _vp], _int),
     "moe_layer_forward": ([ctypes.POINTER(MoeConfig), _vp, _int, _vp, _vp, ctypes.POINTER(MoeExperts),
                            ctypes.POINTER(MoeExperts), _vp, _vp, _sz, _vp], _int),
     "moe_layer_forward_partial": ([ctypes.POINTER(MoeConfig), _vp, _int, _vp, _vp, ctypes.POINTER(MoeExperts),
@@ -76,7 +77,7 @@ _SIGS = {
 PROFILE_MAX_EVENTS = 8
 # launches of one forward on each path (moe_forward_launches): fused small
 # batch, multi-kernel, batched tensor-core
-SMALL_LAUNCHES, MULTI_KERNEL_LAUNCHES, TC_LAUNCHES = 2, 7, 10
+SMALL_LAUNCHES, MULTI_KERNEL_LAUNCHES, TC_LAUNCHES = 1, 7, 10
 
 _LIB = None
 
@@ -348,6 +349,8 @@ class MoeLayer:
         self._shared_s = shared.struct() if shared is not None else MoeExperts()
         self.T_max = T_max
         self.workspace = torch.empty(workspace_bytes(self.cfg, T_max), dtype=torch.uint8, device=router_w.device)
+        _check(lib().moe_workspace_init(ctypes.byref(self.cfg), T_max, _ptr(self.workspace), self.workspace.numel(),
+                                        None), "workspace_init")
 
     def forward(self, x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
         _cuda(x, torch.float32, "x")

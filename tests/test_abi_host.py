@@ -150,7 +150,7 @@ def test_forward_paths_and_phases(L):
     """T <= 4 takes the fused small-batch path (2 launches, one traced phase);
     larger batches the multi-kernel path (7 launches, five phases)."""
     c = _cfg(L)
-    assert L.forward_phases(c, 1) == ["fused"] and L.forward_launches(c, 1) == 2
+    assert L.forward_phases(c, 1) == ["fused"] and L.forward_launches(c, 1) == 1
     assert L.forward_phases(c, 4) == ["fused"]
     assert L.forward_phases(c, 5) == ["route", "bucket", "gate_up", "down", "combine"]
     assert L.forward_launches(c, 16) == 7 and L.forward_launches(c, 0) == 0
@@ -173,4 +173,4 @@ def test_path_selection(L, shape, T, fused):
     c = L.config(shape)
     phases = L.forward_phases(c, T)
     assert (phases == ["fused"]) == fused, phases
-    assert L.forward_launches(c, T) == (2 if fused else 7)
+    assert L.forward_launches(c, T) == (1 if fused else 7)
