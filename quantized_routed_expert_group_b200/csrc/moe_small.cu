@@ -49,15 +49,10 @@
 
 namespace moe {
 
-// Build options of the schedule (tuning knobs; the defaults are the measured
-// best): consumer groups at one token; the producer holds the first weight
-// copies back until every consumer warp has its router row (so that the
-// router reads, which the selection waits for, do not queue behind them).
+// Build option of the one-token schedule (a tuning knob; the default is the
+// measured best): consumer groups.
 #ifndef MOE_SMALL_GROUPS
 #define MOE_SMALL_GROUPS 2
-#endif
-#ifndef MOE_SMALL_ROUTER_FIRST
-#define MOE_SMALL_ROUTER_FIRST 1
 #endif
 
 constexpr int kConsumerWarps = 8;  // warps of one consumer group
@@ -80,6 +75,7 @@ constexpr int kMaxOwnedRows = 64;  // output rows one CTA owns
 constexpr int kScaleWin = 160;     // 16-byte aligned window over <= 32 fp32 scales
 constexpr int kMaxEntryWords = 5;  // ready bitmask words (entries <= 160)
 constexpr int kRouterRound = 4;    // router rows a CTA computes at a time
+constexpr int kMaxKeptFast = 4;    // kept groups of the groups-of-32 selection
 constexpr uint64_t kFcMarkerValue = 0x3130646573756646ull;
 // Thread layout of the gate/up and down chunks: the 64 threads of a warp
 // pair (w, w+1) split the columns (K blocks c, c + 64, ...), the 4 warp pairs
@@ -175,7 +171,7 @@ struct SmallParams {
     moe_experts shared;
     int8_t* xq;
     float* xd;
-    double* logits;
+    double* logits;  // [T][E] router scores s = sigmoid(logit), one row per expert from its CTA
     int32_t* idx;
     float* w;
     int32_t* counts;
@@ -191,6 +187,7 @@ struct SmallParams {
     int32_t* err;
     uint64_t wait_ns;  // bound of the producer's waits (see kWaitNs)
     int fault_entry;   // test hook: the entry whose first unit's h codes are never published (-1: none)
+    int rows_bulk;     // the router matrix is 16-byte aligned: router rows by bulk copy
     SmallGeom g;
 };
 
@@ -249,7 +246,7 @@ SmallGeom small_geometry(const moe_config& c, int T, int grid) {
     g.o_xd = o;
     o += round_up(g.tmax * (H / 32) * 4, 128);
     g.o_bar = o;
-    o += 128;  // full[4], empty[4], routing, ufull[2], ufree[2], gsync, gexit, rowsin
+    o += 256;  // full[4], empty[4], routing, ufull[2], ufree[2], gsync, gexit, rowsin, ctrl
     g.o_meta = o;
     o += round_up((int)sizeof(SlotMeta) * kMaxSlots, 128);
     g.o_urec = o;
@@ -363,7 +360,8 @@ struct SmemPtrs {
     uint64_t* ufree;    // [2] the finisher warp has read them
     uint64_t* gsync;    // the syncing group's warps: their down outputs are in ys
     uint64_t* gexit;    // every consumer warp has left its loop
-    uint64_t* rowsin;   // every consumer warp holds its first router row
+    uint64_t* rowsin;   // the producer's copy of the CTA's router rows into slot 0 has landed
+    uint64_t* ctrl;     // the control snapshot (s.base, misc[8], misc[9]) is in shared memory
     UnitRec* urec;      // [2] the unit to finish
     SlotMeta* meta;
     float* gpart;    // [2][32][2][2][4] gate/up partial dots of a unit: [buffer][pair][gate/up][half][token]
@@ -393,6 +391,7 @@ __device__ __forceinline__ SmemPtrs carve(uint8_t* base, const SmallGeom& g) {
     s.gsync = s.ufree + 2;
     s.gexit = s.gsync + 1;
     s.rowsin = s.gexit + 1;
+    s.ctrl = s.rowsin + 1;
     s.meta = reinterpret_cast<SlotMeta*>(base + g.o_meta);
     s.urec = reinterpret_cast<UnitRec*>(base + g.o_urec);
     s.gpart = reinterpret_cast<float*>(base + g.o_gpart);
@@ -444,34 +443,89 @@ __device__ __forceinline__ uint32_t q8_0_octet(float4 v, float& d) {
     return w;
 }
 
+// Snapshot of the control region that warp 0 takes at the CTA's start: its
+// marker and the counters as this CTA finds them (see kFcMarker).  Plain
+// loads: what earlier kernels wrote is visible at launch, and this call's
+// additions come only after every CTA's router arrival.  Lane l holds the
+// counters of entries l, l + 32, ...
+struct CtrlSnap {
+    uint32_t m0, m1, bar, units;
+    uint32_t done[kMaxEntryWords];
+};
+
+__device__ __forceinline__ CtrlSnap ctrl_load(const SmallParams& p, int lane, int nent) {
+    const volatile int* cv = p.ctrl;
+    CtrlSnap c;
+    c.m0 = (uint32_t)cv[kFcMarker];
+    c.m1 = (uint32_t)cv[kFcMarker + 1];
+    c.bar = (uint32_t)cv[kFcBarrier];
+    c.units = (uint32_t)cv[kFcUnits];
+#pragma unroll
+    for (int j = 0; j < kMaxEntryWords; ++j) {
+        const int i = lane + 32 * j;
+        c.done[j] = i < nent ? (uint32_t)cv[kFcDone + i] : 0u;
+    }
+    return c;
+}
+
+// Warp 0: the snapshot into shared memory (s.base, misc[8], misc[9]); an
+// uninitialised region records kErrWorkspace, and the call then only winds
+// down (no router arrival, no selection, no publication).
+__device__ __forceinline__ void ctrl_store(const SmallParams& p, const SmemPtrs& s, const CtrlSnap& c, int lane,
+                                           int nent) {
+#pragma unroll
+    for (int j = 0; j < kMaxEntryWords; ++j) {
+        const int i = lane + 32 * j;
+        if (i < nent) s.base[1 + i] = c.done[j];
+    }
+    if (lane == 0) {
+        const bool init = (((uint64_t)c.m1 << 32) | c.m0) == kFcMarkerValue;
+        s.base[0] = c.units;
+        s.misc[8] = (int)c.bar;
+        s.misc[9] = init ? 1 : 0;
+        if (blockIdx.x == 0) *p.err = 0;  // before CTA 0's router arrival: no CTA records an error before it
+        if (!init) set_error(p.err, kErrWorkspace);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(s.ctrl);
+}
+
+// Router rows of CTA c that its producer copies into ring slot 0 (ahead of
+// every weight copy) instead of the consumers loading them: the first ones,
+// as many as the slot's weight area holds (needs a 16-byte aligned router
+// matrix; the flag is set on the host).
+__device__ __forceinline__ int router_rows_in_slot(const SmallParams& p, int c, int grid) {
+    if (!p.rows_bulk || c >= p.E) return 0;
+    const int n_mine = (p.E - 1 - c) / grid + 1;
+    const int fit = kSlotWeightBytes / (p.H * 4);
+    return min(min(n_mine, fit), kRouterRound);
+}
+
 // The consumers' start (all G consumer groups, nthr threads, tid < nthr):
-// the CTA's router logits, published to the workspace, and the Q8_0 of x
-// (codes staged in natural order in `stage`, ring slot 0, which only the
-// selection uses later; then put in the weights' order in s.xq; CTA 0 also
-// publishes xq and xd).  Ends with the CTA's arrival on the router barrier.
+// the Q8_0 of x (each block's codes put in the weights' order in registers
+// and stored to s.xq; CTA 0 also publishes xq and xd), then the CTA's router
+// logits, published to the workspace, from the rows the producer copied into
+// `rows` (ring slot 0) and, past those, rows read directly.  Ends with the
+// CTA's arrival on the router barrier.
 template <int WBITS>
-__device__ __forceinline__ void consumers_start(const SmallParams& p, const SmemPtrs& s, uint8_t* stage, int tid,
-                                                int nthr) {
+__device__ __forceinline__ void consumers_start(const SmallParams& p, const SmemPtrs& s, const uint8_t* rows,
+                                                const CtrlSnap& snap, int tid, int nthr) {
     const int warp = tid >> 5, lane = tid & 31, nw = nthr >> 5;
     const int c = blockIdx.x, grid = gridDim.x;
     const int T = p.T, H = p.H, E = p.E, nb = H / 32;
     const int n_mine = c < E ? (E - 1 - c) / grid + 1 : 0;  // router rows of this CTA
-    // the first router row of the warp is requested first: its latency (HBM)
-    // covers the quantisation of x
-    float4 w[kRouterVec];
-    load_router_row(p.router_w, warp / 8 < n_mine ? c + grid * (warp / 8) : E, E, H, warp & 7, lane, w);
-    for (int e = tid; e < E; e += nthr) s.bias[e] = __ldg(p.bias + e);  // read by the selection
+    const int n_slot = router_rows_in_slot(p, c, grid);     // of which the producer copies these
+    const float bias_v = tid < E ? __ldg(p.bias + tid) : 0.f;  // stored below: its load overlaps x's
     // Q8_0 of x: a warp takes 4 blocks at a time (8 lanes, a float4 each);
     // the loads of up to 8 steps are issued before any is used
     {
-        uint32_t* nat = reinterpret_cast<uint32_t*>(stage);  // [T][H] codes
-        const int nblk = T * nb, nstep = (nblk + 3) / 4;
+        const int nblk = T * nb, nstep = (nblk + 3) / 4, l8 = lane & 7;
         for (int s0 = warp; s0 < nstep; s0 += 8 * nw) {
             float4 v[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int blk = 4 * (s0 + j * nw) + (lane >> 3);
-                v[j] = blk < nblk ? __ldg(reinterpret_cast<const float4*>(p.x) + (int64_t)blk * 8 + (lane & 7))
+                v[j] = blk < nblk ? __ldg(reinterpret_cast<const float4*>(p.x) + (int64_t)blk * 8 + l8)
                                   : make_float4(0.f, 0.f, 0.f, 0.f);
             }
 #pragma unroll
@@ -480,24 +534,61 @@ __device__ __forceinline__ void consumers_start(const SmallParams& p, const Smem
                 if (st >= nstep) break;  // the same for the whole warp
                 const int blk = 4 * st + (lane >> 3);
                 float d;
-                const uint32_t q = q8_0_octet(v[j], d);
+                const uint32_t q = q8_0_octet(v[j], d);  // natural codes 4 l8 .. 4 l8 + 3
+                // word l8 of the block in the weights' order (ActBlock layout)
+                uint32_t o;
+                if constexpr (WBITS == 4) {
+                    const uint32_t nb2 = __shfl_xor_sync(kFull, q, 1);
+                    o = (l8 & 1) ? __byte_perm(nb2, q, 0x7531) : __byte_perm(q, nb2, 0x6420);
+                } else if constexpr (WBITS == 2) {
+                    const int qb = lane & ~3;
+                    const uint32_t w0 = __shfl_sync(kFull, q, qb), w1 = __shfl_sync(kFull, q, qb + 1);
+                    const uint32_t w2 = __shfl_sync(kFull, q, qb + 2), w3 = __shfl_sync(kFull, q, qb + 3);
+                    const uint32_t m = (uint32_t)(l8 & 3), sel = m | ((m + 4) << 4);
+                    o = __byte_perm(__byte_perm(w0, w1, sel), __byte_perm(w2, w3, sel), 0x5410);
+                } else {
+                    o = q;
+                }
                 if (blk < nblk) {
-                    nat[(int64_t)blk * 8 + (lane & 7)] = q;
-                    if ((lane & 7) == 0) s.xd[blk] = d;
+                    const int t = blk / nb, b = blk - t * nb;
+                    reinterpret_cast<uint32_t*>(s.xq + ((size_t)(t * 2 + (l8 >> 2)) * nb + b) * 16)[l8 & 3] = o;
+                    if (l8 == 0) s.xd[blk] = d;
+                    if (c == 0) {
+                        reinterpret_cast<uint32_t*>(p.xq)[(int64_t)blk * 8 + l8] = q;
+                        if (l8 == 0) p.xd[blk] = d;
+                    }
                 }
             }
         }
     }
+    if (tid < E) s.bias[tid] = bias_v;  // read by the selection
+    for (int e = tid + nthr; e < E; e += nthr) s.bias[e] = __ldg(p.bias + e);
+    if (warp == 0) ctrl_store(p, s, snap, lane, p.g.nent);
     // router logits, kRouterRound rows at a time: job = (row of the round,
-    // eighth of the hidden dimension); each warp reports (rowsin) once its
-    // first row has arrived, i.e. after that row's dot
+    // eighth of the hidden dimension)
     const int n8 = H / 32;
-    bool rows_in = false;
+    bool rows_waited = n_slot == 0;
     for (int r0 = 0; r0 < n_mine; r0 += kRouterRound) {
         const int nr = min(kRouterRound, n_mine - r0);
         for (int job = warp; job < nr * 8; job += nw) {
             const int i = job >> 3, w8 = job & 7, e = c + grid * (r0 + i);
-            if (!(r0 == 0 && job == warp)) load_router_row(p.router_w, e, E, H, w8, lane, w);
+            float4 w[kRouterVec];
+            if (r0 + i < n_slot) {
+                if (!rows_waited) {
+                    int ok = 1;
+                    if (lane == 0) ok = mbar_wait_ns(s.rowsin, 0, kSlackWaits * p.wait_ns) ? 1 : 0;
+                    if (!__shfl_sync(kFull, ok, 0) && lane == 0) set_error(p.err, kErrTimeout);
+                    rows_waited = true;
+                }
+                const float4* wr = reinterpret_cast<const float4*>(rows + (size_t)(r0 + i) * H * 4) + w8 * n8;
+#pragma unroll
+                for (int u = 0; u < kRouterVec; ++u) {
+                    const int j = lane + 32 * u;
+                    w[u] = j < n8 ? wr[j] : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            } else {
+                load_router_row(p.router_w, e, E, H, w8, lane, w);
+            }
 #pragma unroll 1
             for (int t = 0; t < T; ++t) {
                 const float4* xr = reinterpret_cast<const float4*>(p.x + (int64_t)t * H) + w8 * n8;
@@ -512,11 +603,6 @@ __device__ __forceinline__ void consumers_start(const SmallParams& p, const Smem
                 for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
                 if (lane == 0) s.part[(i * 8 + w8) * 4 + t] = v;
             }
-            if (!rows_in) {
-                __syncwarp();
-                if (lane == 0) mbar_arrive(s.rowsin);
-                rows_in = true;
-            }
         }
         named_barrier(3, nthr);
         if (tid < nr * T) {
@@ -524,34 +610,15 @@ __device__ __forceinline__ void consumers_start(const SmallParams& p, const Smem
             double v = 0.0;
 #pragma unroll
             for (int k = 0; k < 8; ++k) v += s.part[(i * 8 + k) * 4 + t];
-            p.logits[(int64_t)t * E + c + grid * (r0 + i)] = v;
+            // the sigmoid here, off the selection's path
+            p.logits[(int64_t)t * E + c + grid * (r0 + i)] = 1.0 / (1.0 + exp(-v));
         }
         named_barrier(3, nthr);
-    }
-    if (!rows_in && lane == 0) mbar_arrive(s.rowsin);
-    // the staged codes in the weights' order, each 32-code block split in
-    // 16-byte halves so that lanes read consecutive words (after every
-    // warp's staging: a CTA without router rows has had no barrier yet)
-    named_barrier(3, nthr);
-    for (int job = tid; job < T * nb; job += nthr) {
-        const int t = job / nb, b = job - t * nb;
-        const uint4 lo = *reinterpret_cast<const uint4*>(stage + (size_t)job * 32);
-        const uint4 hi = *reinterpret_cast<const uint4*>(stage + (size_t)job * 32 + 16);
-        const ActBlock a = WBITS == 4 ? act_nibble_order(lo, hi)
-                         : WBITS == 2 ? act_crumb_order(lo, hi)
-                                      : act_natural(lo, hi);
-        *reinterpret_cast<uint4*>(s.xq + ((size_t)(t * 2 + 0) * nb + b) * 16) = make_uint4(a.v[0], a.v[1], a.v[2], a.v[3]);
-        *reinterpret_cast<uint4*>(s.xq + ((size_t)(t * 2 + 1) * nb + b) * 16) = make_uint4(a.v[4], a.v[5], a.v[6], a.v[7]);
-        if (c == 0) {
-            *reinterpret_cast<uint4*>(p.xq + (size_t)job * 32) = lo;
-            *reinterpret_cast<uint4*>(p.xq + (size_t)job * 32 + 16) = hi;
-            p.xd[job] = s.xd[job];
-        }
     }
     // every consumer thread's logits are written: the CTA's arrival (CTA 0
     // adds 2^31 - (grid - 1), the others 1: bit 31 flips at the last one)
     named_barrier(3, nthr);
-    if (tid == 0) {
+    if (tid == 0 && s.misc[9]) {
         const int add = c == 0 ? (int)(0x80000000u - (uint32_t)(grid - 1)) : 1;
         red_add_release_gpu(p.ctrl + kFcBarrier, add);
     }
@@ -863,7 +930,7 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
     const int kc = min(max(k, 2), per);  // listed experts per group
     const int kk = min(k, per);          // of which can reach the top_k
     const bool publish = blockIdx.x == 0;
-    const bool fast = per == 32 && G <= kConsumerWarps && tg * kk <= 32;
+    const bool fast = per == 32 && G <= kConsumerWarps && tg <= kMaxKeptFast && tg * kk <= 32;
     double* sc = reinterpret_cast<double*>(scratch);                         // [T][E] c = s + bias
     double* ss = sc + TE;                                                     // [T][E] s
     unsigned long long* key = reinterpret_cast<unsigned long long*>(ss + TE);  // [T][E] order key of c
@@ -882,8 +949,7 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
     // 1. s, c and keys
 #pragma unroll 1
     for (int i = tid; i < TE; i += kConsumers) {
-        const double l = __ldcg(p.logits + i);
-        const double sv = 1.0 / (1.0 + exp(-l));
+        const double sv = __ldcg(p.logits + i);  // s = sigmoid(logit), published by the row's CTA
         const double cv = sv + (double)s.bias[i % E];
         ss[i] = sv;
         sc[i] = cv;
@@ -894,46 +960,58 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
     consumers_sync();
     if (fast) {
         // GLM-like shape: warp g owns group g (32 experts, one per lane).
-        // 2. each (token, group): its experts sorted best first; the best kc
-        // are listed, the best two give the group score
+        // 2. each (token, group): its best two experts by two warp arg-max
+        // rounds (larger key, ties to the lower index) give the group score
         if (warp < G) {
             const int g = warp, e = g * 32 + lane;
 #pragma unroll 1
             for (int t = 0; t < T; ++t) {
-                unsigned long long kv = key[(size_t)t * E + e];
-                int iv = e;
-                warp_sort_desc(kv, iv, lane);
-                if (lane < kc) cand[(t * G + g) * kc + lane] = iv;
-                const int b1 = __shfl_sync(kFull, iv, 0), b2 = __shfl_sync(kFull, iv, 1);
+                const unsigned long long kv = key[(size_t)t * E + e];
+                const int b1 = warp_argmax_u64(kv, e);
+                const int b2 = warp_argmax_u64(e == b1 ? 0ull : kv, e == b1 ? 0x7FFFFFFF : e);
                 if (lane == 0) gkey[t * 32 + g] = order_key(sc[(size_t)t * E + b1] + sc[(size_t)t * E + b2]);
             }
         }
         consumers_sync();
-        // 3. kept groups: each group's rank among the groups of its token
-        if (warp < G && lane < T) {
-            const int g = warp, t = lane;
-            const unsigned long long kgk = gkey[t * 32 + g];
-            int rank = 0;
-#pragma unroll 8
-            for (int g2 = 0; g2 < G; ++g2) rank += beats(gkey[t * 32 + g2], g2, kgk, g) ? 1 : 0;
-            if (rank < tg) kg[t * 32 + rank] = g;
-        }
-        consumers_sync();
-        // 4. one warp per token ranks the listed experts of its kept groups
+        // 3.-4. one warp per token: each group's rank among the token's groups
+        // (kept = rank < topk_groups), then k arg-max rounds over the kept
+        // groups' experts (lane l holds expert l of each kept group); the
+        // picks come out best first
         if (warp < T) {
-            const int t = warp, nl = tg * kk;
-            const bool act = lane < nl;
-            const int q = act ? lane / kk : 0, r = act ? lane - q * kk : 0;
-            const int e = act ? cand[(t * G + kg[t * 32 + q]) * kc + r] : 0x7FFFFFFF;
-            const unsigned long long ke = act ? key[(size_t)t * E + e] : 0ull;
-            int rank = 0;
-#pragma unroll 8
-            for (int j = 0; j < 32; ++j) {  // partly unrolled: the shuffles pipeline
-                const unsigned long long kj = __shfl_sync(kFull, ke, j);
-                const int ej = __shfl_sync(kFull, e, j);
-                rank += beats(kj, ej, ke, e) ? 1 : 0;
+            const int t = warp;
+            const unsigned long long gk = lane < G ? gkey[t * 32 + lane] : 0ull;
+            int grank = 0;
+#pragma unroll 1
+            for (int g2 = 0; g2 < G; ++g2) grank += beats(gkey[t * 32 + g2], g2, gk, lane) ? 1 : 0;
+            uint32_t kept = __ballot_sync(kFull, lane < G && grank < tg);
+            unsigned long long ck[kMaxKeptFast];
+            int ce[kMaxKeptFast];
+#pragma unroll
+            for (int q = 0; q < kMaxKeptFast; ++q) {  // kept groups in index order (the order does not change the picks)
+                const int g = kept ? __ffs(kept) - 1 : -1;
+                kept &= kept - 1;
+                ce[q] = g >= 0 ? g * 32 + lane : 0x7FFFFFFF;
+                ck[q] = g >= 0 ? key[(size_t)t * E + ce[q]] : 0ull;
             }
-            if (act && rank < k) sel[t * 32 + rank] = e;
+#pragma unroll 1
+            for (int j = 0; j < k; ++j) {
+                unsigned long long bk = ck[0];
+                int be = ce[0];
+#pragma unroll
+                for (int q = 1; q < kMaxKeptFast; ++q)
+                    if (beats(ck[q], ce[q], bk, be)) {
+                        bk = ck[q];
+                        be = ce[q];
+                    }
+                const int win = warp_argmax_u64(bk, be);
+#pragma unroll
+                for (int q = 0; q < kMaxKeptFast; ++q)
+                    if (ce[q] == win) {  // taken: out of the later rounds
+                        ck[q] = 0ull;
+                        ce[q] = 0x7FFFFFFF;
+                    }
+                if (lane == 0) sel[t * 32 + j] = win;
+            }
         }
         consumers_sync();
     } else {
@@ -1047,12 +1125,13 @@ __device__ __forceinline__ void do_select(const SmallParams& p, const SmemPtrs& 
             const int e_in = lane < n ? sel[(lane / k) * 32 + lane % k] : -1;
             const bool act = e_in >= 0;
             const int e = act ? e_in : 0x7FFFFFFF;
-            const uint32_t same = __match_any_sync(kFull, e);
+            // one token: the picks are distinct experts
+            const uint32_t same = T == 1 ? (1u << lane) : __match_any_sync(kFull, e);
             const int lead = __ffs(same) - 1;
             const int rank = __popc(same & ((1u << lane) - 1u));  // earlier picks (tokens) of this expert
             int less = 0, dless = 0;  // picks / distinct experts below e
 #pragma unroll 8
-            for (int l2 = 0; l2 < 32; ++l2) {  // partly unrolled: the shuffles pipeline
+            for (int l2 = 0; l2 < n; ++l2) {  // partly unrolled: the shuffles pipeline (lanes >= n hold no pick)
                 const int e2 = __shfl_sync(kFull, e, l2);
                 const int lead2 = __shfl_sync(kFull, lead, l2);
                 less += e2 < e ? 1 : 0;
@@ -1359,9 +1438,9 @@ __device__ __forceinline__ void finisher(const SmallParams& p, const SmemPtrs& s
         if (lane == 0) {
             mbar_arrive(&s.ufree[buf]);
             if (!open && !gave_up) {
-                open = router_barrier_wait(p, s, kSlackWaits * p.wait_ns);
+                open = s.misc[9] && router_barrier_wait(p, s, kSlackWaits * p.wait_ns);
                 gave_up = !open;
-                if (gave_up) set_error(p.err, kErrTimeout);
+                if (gave_up && s.misc[9]) set_error(p.err, kErrTimeout);
             }
             fence_acq_rel_gpu();  // the warp's h codes before the count (release pattern)
             if (open && (r.entry != p.fault_entry || r.blk != 0)) red_add_relaxed_gpu(p.ctrl + kFcDone + r.entry, n);
@@ -1579,28 +1658,15 @@ __global__ void __launch_bounds__(Roles<TM>::kThreads, 1) k_moe_small(const __gr
         }
         mbar_init(s.gsync, kConsumerWarps);
         mbar_init(s.gexit, G * kConsumerWarps);
-        mbar_init(s.rowsin, G * kConsumerWarps);
+        mbar_init(s.rowsin, 1);
+        mbar_init(s.ctrl, 1);
         fence_barrier_init();
     }
-    if (warp == 0) {
-        // the control region: its marker, and the counters as this CTA finds
-        // them (read before its router arrival; see kFcMarker).  Plain loads
-        // issued together: what earlier kernels wrote is visible at launch,
-        // and this call's additions come only after every CTA's arrival.
-        const volatile int* cv = p.ctrl;
-        for (int i = lane; i < 1 + g.nent; i += 32)
-            s.base[i] = (uint32_t)(i == 0 ? cv[kFcUnits] : cv[kFcDone + i - 1]);
-        if (lane == 0) {
-            const uint32_t m0 = (uint32_t)cv[kFcMarker], m1 = (uint32_t)cv[kFcMarker + 1];
-            const bool init = (((uint64_t)m1 << 32) | m0) == kFcMarkerValue;
-            s.misc[9] = init ? 1 : 0;
-            s.misc[8] = cv[kFcBarrier];
-            if (c == 0) *p.err = 0;  // before CTA 0's router arrival: no CTA records an error before it
-            if (!init) set_error(p.err, kErrWorkspace);
-        }
-    }
+    // warp 0 reads the control region now (the values are stored to shared
+    // memory later, by consumers_start, before this CTA's router arrival)
+    CtrlSnap snap{};
+    if (warp == 0) snap = ctrl_load(p, lane, g.nent);
     __syncthreads();
-    if (!s.misc[9]) return;  // the same in every CTA
 
     if (warp == R::kFinisherWarp) {
         finisher(p, s, lane);
@@ -1610,13 +1676,17 @@ __global__ void __launch_bounds__(Roles<TM>::kThreads, 1) k_moe_small(const __gr
         // ------------------------- producer -------------------------
         Producer pr(p, s, lane, G);
         const int64_t rowI = (int64_t)p.I * p.wbits / 8;
-        pr.marker(kItemSelect);
-        if (MOE_SMALL_ROUTER_FIRST) {
-            int okr = 1;
-            if (lane == 0) okr = mbar_wait_ns(s.rowsin, 0, p.wait_ns) ? 1 : 0;
-            okr = __shfl_sync(kFull, okr, 0);
-            if (!okr) pr.fail();
+        // the CTA's router rows first (the selection waits for them), into
+        // slot 0, which the selection's marker holds until it is done
+        const int n_slot = router_rows_in_slot(p, c, grid);
+        if (lane == 0) bulk_prefetch_l2(p.x, (uint32_t)(p.T * p.H * 4));  // x ahead of every copy
+        if (n_slot > 0 && lane == 0) {
+            mbar_arrive_expect_tx(s.rowsin, (uint32_t)(n_slot * p.H * 4));
+            for (int i = 0; i < n_slot; ++i)
+                bulk_g2s_nohint(s.slots + (size_t)i * p.H * 4, p.router_w + (int64_t)(c + grid * i) * p.H,
+                                (uint32_t)(p.H * 4), s.rowsin);
         }
+        pr.marker(kItemSelect);
         {
             // the shared expert's down rows this CTA will probably own
             int q0, q1;
@@ -1639,6 +1709,7 @@ __global__ void __launch_bounds__(Roles<TM>::kThreads, 1) k_moe_small(const __gr
         ok = __shfl_sync(kFull, ok, 0);
         __syncwarp();  // lane 0's acquire of the tables orders the other lanes' reads
         if (!ok) pr.fail();
+        if (!s.misc[9]) pr.aborted = true;  // uninitialised control region: no routed work (error recorded)
         const int umax = g.nent - 1;
         int U = s.misc[0];
         U = U < 0 ? 0 : (U > umax ? umax : U);
@@ -1697,7 +1768,7 @@ __global__ void __launch_bounds__(Roles<TM>::kThreads, 1) k_moe_small(const __gr
     // ------------------------- consumers -------------------------
     const int group = warp / kConsumerWarps;     // consumer group
     const int gtid = tid - group * kConsumers;   // thread index inside the group
-    consumers_start<WBITS>(p, s, s.slots, tid, G * kConsumers);
+    consumers_start<WBITS>(p, s, s.slots, snap, tid, G * kConsumers);
     // group g takes ring slots g, g + G, ... in order
     int slot = group;
     uint32_t pf = 0;
@@ -1717,9 +1788,15 @@ __global__ void __launch_bounds__(Roles<TM>::kThreads, 1) k_moe_small(const __gr
             do_down<WBITS, TM>(p, s, m, data, gtid, empty);
         } else if (m.kind == kItemSelect) {
             // always group 0's: the first item; every CTA's logits first
-            if (gtid == 0 && !router_barrier_wait(p, s, kSlackWaits * p.wait_ns)) set_error(p.err, kErrTimeout);
-            consumers_sync();
-            do_select(p, s, data, gtid);
+            if (s.misc[9]) {
+                if (gtid == 0 && !router_barrier_wait(p, s, kSlackWaits * p.wait_ns)) set_error(p.err, kErrTimeout);
+                consumers_sync();
+                do_select(p, s, data, gtid);
+            } else if (gtid == 0) {  // no routing: the producer winds down
+                s.misc[0] = 0;
+                s.misc[1] = 0;
+                mbar_arrive(s.routing);
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(empty);  // the slot was the scratch
         } else if (m.kind == kItemSync) {
@@ -1813,6 +1890,7 @@ cudaError_t launch_small(const SmallArgs& a, cudaStream_t st) {
     p.hq = a.hq; p.hd = a.hd; p.y = a.y; p.out = a.out; p.ctrl = a.ctrl; p.err = a.err;
     p.wait_ns = (uint64_t)g_wait_ns.load();
     p.fault_entry = g_fault_entry.load();
+    p.rows_bulk = (reinterpret_cast<uintptr_t>(a.router_w) % 16 == 0) ? 1 : 0;
     p.g = small_geometry(c, a.T, device_info().sm_count);
     if (p.g.smem_bytes > device_info().max_smem_optin) return cudaErrorInvalidConfiguration;
     const int tm = p.g.tmax;
