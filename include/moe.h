@@ -294,7 +294,11 @@ typedef struct {
     int8_t *hq;        /* [slots][inter]    Q8_0 codes of h per slot */
     float *hd;         /* [slots][inter/32] Q8_0 scales of h per slot */
     float *y;          /* [slots][hidden]   expert outputs per slot (unweighted) */
-    int32_t *error;    /* device error word (0 = none) */
+    int32_t *error;    /* device error word (0 = none); error[8] and error[9] are set
+                        * by a batched tensor-core forward (T >= 64) whose activations
+                        * (x, resp. h) had a token with block-scale exponents more than 8
+                        * apart, so that its GEMM took the fp64-epilogue form instead of
+                        * the digit planes (see moe_layer_forward) */
 } moe_workspace_layout;
 
 int moe_workspace_view(const moe_config *cfg, int T, void *workspace, size_t ws_bytes,

@@ -53,6 +53,12 @@ Layout make_layout(const moe_config& c, int T) {
         L.tc_gu = take(2 * pr * I * 4);
         L.tc_hg = take(pr * I);
         L.tc_hdT = take((I / 32) * pr * 8);
+        L.tc_xp = take(pr * 5 * H);
+        L.tc_hp = take(pr * 5 * I);
+        L.tc_pex = take(pr * 8);
+        L.tc_peh = take(pr * 8);
+        L.tc_xpt = take(t * 5 * H);
+        L.tc_pet = take(t * 8);
         L.tc_row_tok = take(pr * 4);
         L.tc_row_slot = take(pr * 4);
         L.tc_units_gu = take((size_t)z.units_gu_cap * kTcUnitBytes);
@@ -60,6 +66,7 @@ Layout make_layout(const moe_config& c, int T) {
         L.tc_ctrl = take(64);
     } else {
         L.tc_xg = L.tc_xdT = L.tc_gu = L.tc_hg = L.tc_hdT = L.tc_row_tok = L.tc_row_slot = 0;
+        L.tc_xp = L.tc_hp = L.tc_pex = L.tc_peh = L.tc_xpt = L.tc_pet = 0;
         L.tc_units_gu = L.tc_units_dn = L.tc_ctrl = 0;
     }
     L.total = off;
@@ -213,8 +220,11 @@ static int forward_device(const moe_config& c, const float* x, int T, const floa
     }
     const NvtxRange range("moe/multi_kernel");
     if (trace(0, s) != cudaSuccess) return MOE_ECUDA;
-    if (cudaMemsetAsync(err, 0, 64, s) != cudaSuccess) return MOE_ECUDA;
-    int st = status_of(launch_quantize_q8_0(x, T, c.hidden, xq, xd, s));
+    if (cudaMemsetAsync(err, 0, 64, s) != cudaSuccess) return MOE_ECUDA;  // also the batched path's wide flags
+    const bool tc = tc_path_supported(c, T);
+    int st = tc ? status_of(launch_tc_quantize(x, T, c.hidden, xq, xd, reinterpret_cast<int8_t*>(ws + L.tc_xpt),
+                                               reinterpret_cast<double*>(ws + L.tc_pet), err + 8, s))
+                : status_of(launch_quantize_q8_0(x, T, c.hidden, xq, xd, s));
     if (st) return st;
     st = status_of(launch_router(c, x, T, router_w, router_bias, reinterpret_cast<double*>(ws + L.logits), idx, w, s));
     if (!st) st = status_of(trace(1, s));
@@ -228,7 +238,6 @@ static int forward_device(const moe_config& c, const float* x, int T, const floa
     }
     st = status_of(launch_bucket(c, bidx, T, counts, offsets, perm, inv_perm, active, err, s));
     if (st) return st;
-    const bool tc = tc_path_supported(c, T);
     TcArgs ta{};
     if (tc) {
         ta.xg = reinterpret_cast<int8_t*>(ws + L.tc_xg);
@@ -236,6 +245,14 @@ static int forward_device(const moe_config& c, const float* x, int T, const floa
         ta.gu = reinterpret_cast<float*>(ws + L.tc_gu);
         ta.hg = reinterpret_cast<int8_t*>(ws + L.tc_hg);
         ta.hdT = reinterpret_cast<double*>(ws + L.tc_hdT);
+        ta.xp = reinterpret_cast<int8_t*>(ws + L.tc_xp);
+        ta.hp = reinterpret_cast<int8_t*>(ws + L.tc_hp);
+        ta.pex = reinterpret_cast<double*>(ws + L.tc_pex);
+        ta.peh = reinterpret_cast<double*>(ws + L.tc_peh);
+        ta.xpt = reinterpret_cast<int8_t*>(ws + L.tc_xpt);
+        ta.pet = reinterpret_cast<double*>(ws + L.tc_pet);
+        ta.xwide = err + 8;
+        ta.hwide = err + 9;
         ta.row_tok = reinterpret_cast<int32_t*>(ws + L.tc_row_tok);
         ta.row_slot = reinterpret_cast<int32_t*>(ws + L.tc_row_slot);
         ta.units_gu = ws + L.tc_units_gu;

@@ -34,6 +34,7 @@ struct Layout {
     size_t y;          // fp32 [slots][H]
     // batched tensor-core path only (0 bytes otherwise)
     size_t tc_xg, tc_xdT, tc_gu, tc_hg, tc_hdT, tc_row_tok, tc_row_slot, tc_units_gu, tc_units_dn, tc_ctrl;
+    size_t tc_xp, tc_hp, tc_pex, tc_peh, tc_xpt, tc_pet;
     size_t total;
 };
 
@@ -101,7 +102,9 @@ cudaError_t launch_combine(const ExpertArgs& a, cudaStream_t s);
 
 // Batched path on the tensor cores (moe_tc.cu), for T >= kTcMinTokens.
 constexpr int kTcMinTokens = 64;
-constexpr int kTcLaunches = 10;  // quantise, logits, select, bucket, plan, gather, gate/up, SwiGLU, down, combine
+// quantise, logits, select, bucket, plan, planes; gate/up on the digit planes and its fp64
+// fallback (one of the two returns at once), SwiGLU, down and its fallback, combine
+constexpr int kTcLaunches = 12;
 bool tc_path_supported(const moe_config& c, int T);
 struct TcSizes {
     int prows_cap;     // rows of the padded row space
@@ -116,14 +119,25 @@ struct TcArgs {
     float* gu;          // [2][prows_cap][inter]  g and u row values
     int8_t* hg;         // [prows_cap][inter]
     double* hdT;        // [inter/32][prows_cap]
+    int8_t* xp;         // [prows_cap][5][hidden]  digit planes of the scaled x codes
+    int8_t* hp;         // [prows_cap][5][inter]   digit planes of the scaled h codes
+    double* pex;        // [prows_cap] 2^E of each row's x planes
+    double* peh;        // [prows_cap] 2^E of each row's h planes
+    int8_t* xpt;        // [T][5][hidden] digit planes of each token (k_tc_quantize)
+    double* pet;        // [T] 2^E of each token's planes
+    int* xwide;         // some token's block scales spread too far for the planes (zeroed per call)
+    int* hwide;         // the same for some row of h
     int32_t* row_tok;   // [prows_cap]
     int32_t* row_slot;  // [prows_cap]
     void* units_gu;     // TcUnit [units_gu_cap]
     void* units_dn;     // TcUnit [units_dn_cap]
-    int32_t* ctrl;      // [8]
+    int32_t* ctrl;      // [16]
     TcSizes sz;
 };
 constexpr size_t kTcUnitBytes = 16;
+// Q8_0 of x and each token's digit planes (the batched path's quantiser)
+cudaError_t launch_tc_quantize(const float* x, int T, int H, int8_t* xq, float* xd, int8_t* xpt, double* pet,
+                               int* xwide, cudaStream_t s);
 // plan + gather (the end of the bucketing phase)
 cudaError_t launch_tc_prepare(const TcArgs& a, cudaStream_t s);
 // gate/up GEMM, down GEMM, combine; ev (optional, 3 events) after each

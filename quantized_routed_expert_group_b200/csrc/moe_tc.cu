@@ -322,7 +322,7 @@ __global__ void __launch_bounds__(kPlanThreads) k_tc_plan(PlanParams p) {
     int rgu = 0, rdn = 0;
     for (int base = 0; base < ne; base += kPlanThreads) {
         const int r = base + tid;
-        const int nch = r < ne ? (s_n[s_sched[r]] + kMaxN - 1) / kMaxN : 0;
+        const int nch = r < ne ? (s_n[s_sched[r]] + kChunk - 1) / kChunk : 0;
         int tg, td;
         const int eg = block_excl_scan(2 * nch * tiles_gu, s_ws, &tg);
         const int ed = block_excl_scan(nch * tiles_dn, s_ws, &td);
@@ -356,24 +356,24 @@ __global__ void __launch_bounds__(kPlanThreads) k_tc_plan(PlanParams p) {
     };
     for (int u = tid; u < rgu; u += kPlanThreads) {
         const int r = entry_of(s_ugu0, u), i = s_sched[r];
-        const int n = s_n[i], nch = (n + kMaxN - 1) / kMaxN;
+        const int n = s_n[i], nch = (n + kChunk - 1) / kChunk;
         const int l = u - s_ugu0[r], c = l % nch, tm = l / nch, m = tm & 1, t = tm >> 1;
         const bool shared = i >= U;
         TcUnit w;
-        w.prow0 = s_prow0[i] + c * kMaxN;
-        w.ntok = min(kMaxN, n - c * kMaxN);
+        w.prow0 = s_prow0[i] + c * kChunk;
+        w.ntok = min(kChunk, n - c * kChunk);
         w.wrow0 = (shared ? 0 : p.active[1 + i]) * p.I + t * kTileRows;
         w.info = t | (shared ? kUnitShared : 0) | (m ? kUnitUp : 0);
         p.units_gu[u] = w;
     }
     for (int u = tid; u < rdn; u += kPlanThreads) {
         const int r = entry_of(s_udn0, u), i = s_sched[r];
-        const int n = s_n[i], nch = (n + kMaxN - 1) / kMaxN;
+        const int n = s_n[i], nch = (n + kChunk - 1) / kChunk;
         const int l = u - s_udn0[r], c = l % nch, t = l / nch;
         const bool shared = i >= U;
         TcUnit w;
-        w.prow0 = s_prow0[i] + c * kMaxN;
-        w.ntok = min(kMaxN, n - c * kMaxN);
+        w.prow0 = s_prow0[i] + c * kChunk;
+        w.ntok = min(kChunk, n - c * kChunk);
         w.wrow0 = (shared ? 0 : p.active[1 + i]) * p.H + t * kTileRows;
         w.info = t | (shared ? kUnitShared : 0);
         p.units_dn[u] = w;
@@ -404,16 +404,105 @@ __global__ void __launch_bounds__(kPlanThreads) k_tc_plan(PlanParams p) {
     }
 }
 
-// One warp per padded row: the token's Q8_0 codes (zeros for a padding row)
-// and its block scales, transposed, as fp64.
+// Q8_0 of x, one CTA per token (as k_quantize_q8_0: one warp per block of 32,
+// lane = element), and the token's digit planes [5][hidden] with its 2^E
+// (see kPlanes).  A token whose block-scale exponents spread over more than
+// kMaxSpread sets *wide; the call then takes the fp64-epilogue GEMMs and the
+// planes are not used.
+constexpr int kQuantThreads = 256;
+constexpr int kMaxBlocksPerWarp = 32;  // hidden <= 8 * 32 * 32
+
+__global__ void __launch_bounds__(kQuantThreads) k_tc_quantize(const float* __restrict__ x, int H,
+                                                               int8_t* __restrict__ xq, float* __restrict__ xd,
+                                                               int8_t* __restrict__ xpt, double* __restrict__ pet,
+                                                               int* wide) {
+    __shared__ int s_e[2][kQuantThreads / 32];
+    const int t = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nb = H / 32, nw = kQuantThreads / 32;
+    const float* xt = x + (int64_t)t * H;
+    float v[kMaxBlocksPerWarp];
+#pragma unroll
+    for (int j = 0; j < kMaxBlocksPerWarp; ++j) {
+        const int b = warp + nw * j;
+        v[j] = b < nb ? __ldg(xt + 32 * b + lane) : 0.f;
+    }
+    int qv[kMaxBlocksPerWarp];
+    uint32_t mm[kMaxBlocksPerWarp];
+    int ee[kMaxBlocksPerWarp];
+    int emin = 0x7FFFFFFF, emax = -0x7FFFFFFF;
+#pragma unroll
+    for (int j = 0; j < kMaxBlocksPerWarp; ++j) {
+        const int b = warp + nw * j;
+        qv[j] = 0;
+        mm[j] = 0u;
+        ee[j] = 0;
+        if (b < nb) {  // the same in the whole warp
+            int8_t q;
+            float d;
+            q8_0_warp(v[j], q, d);
+            xq[(int64_t)t * H + 32 * b + lane] = q;
+            if (lane == 0) xd[(int64_t)t * nb + b] = d;
+            qv[j] = q;
+            f32_mant_exp(d, mm[j], ee[j]);
+            if (mm[j]) {
+                emin = min(emin, ee[j]);
+                emax = max(emax, ee[j]);
+            }
+        }
+    }
+    if (lane == 0) {
+        s_e[0][warp] = emin;
+        s_e[1][warp] = emax;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < nw; ++w) {
+        emin = min(emin, s_e[0][w]);
+        emax = max(emax, s_e[1][w]);
+    }
+    const bool any = emin <= emax;  // some block is not zero
+    if (any && emax - emin > kMaxSpread) {
+        if (threadIdx.x == 0) atomicOr(wide, 1);
+        return;
+    }
+    int8_t* dst = xpt + (int64_t)t * kPlanes * H;
+#pragma unroll
+    for (int j = 0; j < kMaxBlocksPerWarp; ++j) {
+        const int b = warp + nw * j;
+        if (b < nb) {
+            const uint32_t m = mm[j] ? mm[j] << (ee[j] - emin) : 0u;
+            int c[kPlanes];
+            digits5(qv[j], m, c);
+#pragma unroll
+            for (int pl = 0; pl < kPlanes; ++pl) dst[(int64_t)pl * H + 32 * b + lane] = (int8_t)c[pl];
+        }
+    }
+    if (threadIdx.x == 0) pet[t] = any ? ldexp(1.0, emin) : 0.0;
+}
+
+// One warp per padded row: its token's digit planes and 2^E (zeros for a
+// padding row); when some token is wide instead the token's Q8_0 codes and
+// its block scales, transposed, as fp64 (for the fp64-epilogue GEMM).
 __global__ void __launch_bounds__(256) k_tc_gather(const int8_t* __restrict__ xq, const float* __restrict__ xd,
-                                                   int H, int prows_cap, const int32_t* __restrict__ row_tok,
+                                                   const int8_t* __restrict__ xpt, const double* __restrict__ pet,
+                                                   const int* __restrict__ wide, int H, int prows_cap,
+                                                   const int32_t* __restrict__ row_tok,
                                                    const int32_t* __restrict__ ctrl, int8_t* __restrict__ xg,
-                                                   double* __restrict__ xdT) {
+                                                   double* __restrict__ xdT, int8_t* __restrict__ xp,
+                                                   double* __restrict__ pex) {
     const int lane = threadIdx.x & 31;
     const int q = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (q >= ctrl[2]) return;
     const int tok = row_tok[q];
+    if (!*wide) {
+        const int n16 = kPlanes * H / 16;
+        uint4* dst = reinterpret_cast<uint4*>(xp + (int64_t)q * kPlanes * H);
+        const uint4* src = reinterpret_cast<const uint4*>(xpt + (int64_t)(tok < 0 ? 0 : tok) * kPlanes * H);
+#pragma unroll 4
+        for (int i = lane; i < n16; i += 32) dst[i] = tok >= 0 ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+        if (lane == 0) pex[q] = tok >= 0 ? pet[tok] : 0.0;
+        return;
+    }
     const int n16 = H / 16, nb = H / 32;
     uint4* dst = reinterpret_cast<uint4*>(xg + (int64_t)q * H);
     const uint4* src = reinterpret_cast<const uint4*>(xq + (int64_t)(tok < 0 ? 0 : tok) * H);
@@ -478,6 +567,8 @@ struct GemmParams {
     float* gu;  // gate/up: [2][prows_cap][I]
     float* y;   // down: [slots][H]
     int32_t* err;
+    const int* wide;   // some row's block scales spread too far for the digit planes
+    const double* pe;  // digit-plane GEMM: 2^E of each padded row
 };
 
 // Exact fp64 of an int32: the 32 bits (offset by 2^31) become the low
@@ -492,6 +583,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               const __grid_constant__ CUtensorMap w_s0, const __grid_constant__ CUtensorMap w_s1,
               const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap dmap,
               const GemmParams p) {
+    if (!*p.wide) return;  // the digit-plane GEMM does this call's work
     using L = GemmSmem<WBITS>;
     constexpr int S = L::kStages;
     extern __shared__ uint8_t smem_raw[];
@@ -744,37 +836,378 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (warp == kMmaWarp) tmem_dealloc(tmem, L::kTmemCols);
 }
 
-// SwiGLU and Q8_0 of h, one warp per (padded row, block of 32 h values):
-// h = silu(g) * u evaluated in fp64 and rounded to fp32, then Q8_0.
-__global__ void __launch_bounds__(256) k_tc_swiglu(const float* __restrict__ gu, int I, int prows_cap,
-                                                   const int32_t* __restrict__ row_slot,
-                                                   const int32_t* __restrict__ ctrl, int8_t* __restrict__ hg,
-                                                   double* __restrict__ hdT, int8_t* __restrict__ hq,
-                                                   float* __restrict__ hd) {
-    const int lane = threadIdx.x & 31;
-    const int nbI = I / 32;
-    const int64_t n_jobs = (int64_t)ctrl[2] * nbI;
-    for (int64_t job = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); job < n_jobs; job += (int64_t)gridDim.x * 8) {
-        const int q = (int)(job / nbI), b = (int)(job % nbI);
-        const int slot = row_slot[q];
-        if (slot < 0) {  // a padding row (the same in the whole warp): zero scale
-            if (lane == 0) hdT[(int64_t)b * prows_cap + q] = 0.0;
-            continue;
+// ---------------------------------------------------------------------------
+// Grouped GEMM on the digit planes (persistent, one CTA per SM)
+// ---------------------------------------------------------------------------
+// Per unit (128 weight rows x a chunk of nt <= kChunk tokens) one kind::i8
+// MMA per 32 codes of K with M = 128 and N = kPlanes * nt16 columns: column
+// 5 c + p is token c's plane p (the plane tensor is [rows][kPlanes][K], so a
+// chunk's planes are kPlanes * nt consecutive rows).  The accumulator sums
+// the whole K in int32; at the unit's end
+//   acc = 2^E_c (D_0 + 2^8 D_1 + 2^16 D_2 + 2^24 D_3 + 2^32 D_4)
+// is formed exactly in int64 (a double while it stays below 2^53), and the
+// output is fp32(s_row * acc) in fp64, as the oracle rounds it.
+// warps 0-3  epilogue (warp w: TMEM lanes 32 w .. 32 w + 31 = its 32 rows)
+// warps 4-5  widening of packed int4 / int2 staging rows
+// warp 6     producer: units from a global counter, TMA per stage of the
+//            weight rows and of the chunk's planes (box of 80, 160 or 240 rows)
+// warp 7     MMA: two accumulators of 256 TMEM columns, alternating units
+// Every wait is bounded by the global timer and records kErrTimeout.
+constexpr int kDpEpiWarps = 4;
+constexpr int kDpConvWarps = 2;
+constexpr int kDpProdWarp = kDpEpiWarps + kDpConvWarps;
+constexpr int kDpMmaWarp = kDpProdWarp + 1;
+constexpr int kDpThreads = (kDpMmaWarp + 1) * 32;
+constexpr int kDpAccCols = 256;
+
+template <int WBITS>
+struct DpSmem {
+    static constexpr int kRawTile = WBITS == 8 ? 0 : kTileRows * raw_row_bytes<WBITS>();
+    static constexpr int kA = 0;                                   // widened tile (int8: the TMA target)
+    static constexpr int kB = kTileBytes;                          // planes [kPlanes * kChunk][128]
+    static constexpr int kRaw = kB + kPlanes * kChunk * kStageK;  // packed staging tile
+    static constexpr int kStageBytes = (kRaw + kRawTile + 1023) & ~1023;
+    static constexpr int kCtrl = 1024;
+    static constexpr int kStagesFit = (224 * 1024 - kCtrl - 1024) / kStageBytes;
+    static constexpr int kStages = kStagesFit < 6 ? kStagesFit : 6;
+    static constexpr int kBytes = kStages * kStageBytes + kCtrl + 1024;  // + alignment slack
+    static constexpr uint32_t kWeightTx = (uint32_t)(kTileRows * raw_row_bytes<WBITS>());
+};
+
+// Unit counter value -> padded-row group of 16 (1..3): which plane map
+__device__ __forceinline__ int nt_groups(int ntok) { return (ntok + 15) >> 4; }
+
+template <int WBITS>
+__global__ void __launch_bounds__(kDpThreads, 1)
+    k_tc_gemm_dp(const __grid_constant__ CUtensorMap w_r0, const __grid_constant__ CUtensorMap w_r1,
+                 const __grid_constant__ CUtensorMap w_s0, const __grid_constant__ CUtensorMap w_s1,
+                 const __grid_constant__ CUtensorMap b16, const __grid_constant__ CUtensorMap b32,
+                 const __grid_constant__ CUtensorMap b48, const GemmParams p) {
+    if (*p.wide) return;  // the fp64-epilogue GEMM does this call's work
+    using L = DpSmem<WBITS>;
+    constexpr int S = L::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* ctl = sm + S * L::kStageBytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(ctl);
+    uint64_t* conv = full + S;
+    uint64_t* empty = conv + S;
+    uint64_t* accf = empty + S;   // [2] the accumulator's unit is complete (MMA commit)
+    uint64_t* acce = accf + 2;    // [2] the epilogue has read the accumulator
+    uint64_t* uready = acce + 2;  // [2] the accumulator's next unit id is in unit_of
+    int* meta = reinterpret_cast<int*>(uready + 2);  // [S][2]: unit (-1: end), stage of the unit
+    int* unit_of = meta + 2 * S;                      // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(unit_of + 2);
+    auto stage = [&](int s) { return sm + s * L::kStageBytes; };
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&conv[s], kDpConvWarps);
+            mbar_init(&empty[s], 1);
         }
-        const int i = 32 * b + lane;
-        const double g = (double)gu[(int64_t)q * I + i];
-        const double uu = (double)gu[((int64_t)prows_cap + q) * I + i];
-        const float h = __double2float_rn(__dmul_rn(__ddiv_rn(g, __dadd_rn(1.0, exp(-g))), uu));
-        int8_t qv;
-        float d;
-        q8_0_warp(h, qv, d);
-        hg[(int64_t)q * I + i] = qv;
-        hq[(int64_t)slot * I + i] = qv;
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&accf[a], 1);
+            mbar_init(&acce[a], kDpEpiWarps);
+            mbar_init(&uready[a], 1);
+        }
+        fence_barrier_init();
+    }
+    if (warp == kDpMmaWarp) {
+        tmem_alloc(tmem_slot, 2 * kDpAccCols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const int n_units = p.ctrl[p.n_units_idx];
+
+    if (warp == kDpProdWarp) {
+        // ---------------- producer ----------------
         if (lane == 0) {
-            hdT[(int64_t)b * prows_cap + q] = (double)d;
-            hd[(int64_t)slot * nbI + b] = d;
+            tma_prefetch_map(&w_r0);
+            tma_prefetch_map(&w_r1);
+            tma_prefetch_map(&w_s0);
+            tma_prefetch_map(&w_s1);
+            tma_prefetch_map(&b16);
+            tma_prefetch_map(&b32);
+            tma_prefetch_map(&b48);
+            int s = 0;
+            uint32_t ph = 0;
+            int unit = atomicAdd(p.counter, 1), kstep = 0;
+            TcUnit u = unit < n_units ? p.units[unit] : TcUnit{0, 0, 0, 0};
+            while (true) {
+                if (!mbar_wait_ns(&empty[s], ph ^ 1u, kGemmWaitNs)) {
+                    set_error(p.err, kErrTimeout);
+                    break;
+                }
+                if (unit >= n_units) {
+                    meta[2 * s] = -1;
+                    meta[2 * s + 1] = 0;
+                    mbar_arrive(&full[s]);
+                    break;
+                }
+                meta[2 * s] = unit;
+                meta[2 * s + 1] = kstep;
+                const int ng = nt_groups(u.ntok);
+                mbar_arrive_expect_tx(&full[s], L::kWeightTx + (uint32_t)(kPlanes * 16 * ng * kStageK));
+                uint8_t* st = stage(s);
+                const bool sh = (u.info & kUnitShared) != 0, up = (u.info & kUnitUp) != 0;
+                const CUtensorMap* wm = sh ? (up ? &w_s1 : &w_s0) : (up ? &w_r1 : &w_r0);
+                tma_load_2d(WBITS == 8 ? st + L::kA : st + L::kRaw, wm, kstep * raw_row_bytes<WBITS>(), u.wrow0,
+                            &full[s]);
+                const CUtensorMap* bm = ng == 1 ? &b16 : ng == 2 ? &b32 : &b48;
+                tma_load_2d(st + L::kB, bm, kstep * kStageK, u.prow0 * kPlanes, &full[s]);
+                if (++kstep == p.nstage) {
+                    kstep = 0;
+                    unit = atomicAdd(p.counter, 1);
+                    if (unit < n_units) u = p.units[unit];
+                }
+                if (++s == S) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == kDpMmaWarp) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            int s = 0, cur = -1, nu = -1;
+            uint32_t ph = 0, idesc = 0, acc = 0;
+            bool ok = true;
+            while (ok) {
+                if (!mbar_wait_ns(&full[s], ph, kGemmWaitNs)) {
+                    set_error(p.err, kErrTimeout);
+                    break;
+                }
+                const int unit = meta[2 * s];
+                const int kstep = meta[2 * s + 1];
+                if (unit < 0 || unit != cur) {
+                    // a new unit (or the end) takes the next accumulator, once
+                    // the epilogue has read that accumulator's previous unit;
+                    // the epilogue learns the unit id through unit_of
+                    ++nu;
+                    const int buf = nu & 1;
+                    if (nu >= 2 && !mbar_wait_ns(&acce[buf], ((nu >> 1) - 1) & 1, kGemmWaitNs)) {
+                        set_error(p.err, kErrTimeout);
+                        break;
+                    }
+                    unit_of[buf] = unit;
+                    mbar_arrive(&uready[buf]);
+                    if (unit < 0) break;
+                    cur = unit;
+                    idesc = idesc_i8(kPlanes * 16 * nt_groups(p.units[unit].ntok));
+                    acc = tmem + (uint32_t)(buf * kDpAccCols);
+                }
+                if (WBITS != 8 && !mbar_wait_ns(&conv[s], ph, kGemmWaitNs)) {
+                    set_error(p.err, kErrTimeout);
+                    break;
+                }
+                tc_fence_after_sync();
+                uint8_t* st = stage(s);
+                const uint64_t bdsc = desc_k128_sw128(st + L::kB);
+                const uint64_t adsc = desc_k128_sw128(st + L::kA);
+#pragma unroll
+                for (int j = 0; j < kBlocksPerStage; ++j)
+                    if (kstep * kBlocksPerStage + j < p.nbK)
+                        mma_i8(acc, adsc + 2 * j, bdsc + 2 * j, idesc, kstep > 0 || j > 0);
+                mma_commit(&empty[s]);
+                if (kstep == p.nstage - 1) mma_commit(&accf[nu & 1]);
+                if (++s == S) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp >= kDpEpiWarps) {
+        // ---------------- widening ----------------
+        if constexpr (WBITS != 8) {
+            const int r0 = threadIdx.x - kDpEpiWarps * 32;  // rows r0 and r0 + 64 of the tile
+            int s = 0;
+            uint32_t ph = 0;
+            while (true) {
+                if (!mbar_wait_ns(&full[s], ph, kGemmWaitNs)) {
+                    set_error(p.err, kErrTimeout);
+                    break;
+                }
+                if (meta[2 * s] < 0) break;
+                uint8_t* st = stage(s);
+                widen_row<WBITS>(st + L::kRaw, st + L::kA, r0);
+                widen_row<WBITS>(st + L::kRaw, st + L::kA, r0 + 64);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&conv[s]);
+                if (++s == S) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+        }
+    } else {
+        // ---------------- epilogue ----------------
+        // the MMA warp hands over each accumulator's unit id (uready), then
+        // its completion (accf)
+        const uint32_t tlane = (uint32_t)(32 * warp) << 16;
+        const int rl = 32 * warp + lane;  // the thread's row in the tile
+        for (int nu = 0;; ++nu) {
+            const int buf = nu & 1;
+            const uint32_t par = (uint32_t)(nu >> 1) & 1u;
+            if (!mbar_wait_ns(&uready[buf], par, kGemmWaitNs)) {
+                set_error(p.err, kErrTimeout);
+                break;
+            }
+            const int unit = unit_of[buf];
+            if (unit < 0) break;
+            if (!mbar_wait_ns(&accf[buf], par, kGemmWaitNs)) {
+                set_error(p.err, kErrTimeout);
+                break;
+            }
+            tc_fence_after_sync();
+            const TcUnit u = p.units[unit];
+            const int tile = u.info & 0xFFFF;
+            const bool sh = (u.info & kUnitShared) != 0, up = (u.info & kUnitUp) != 0;
+            const float* sc = sh ? (up ? p.s_s1 : p.s_s0) : (up ? p.s_r1 : p.s_r0);
+            const double sr = (double)__ldg(sc + u.wrow0 + rl);
+            const int r = tile * kTileRows + rl;  // output row of this thread
+            const int ng = nt_groups(u.ntok);
+            for (int g = 0; g < ng; ++g) {
+                uint32_t v[kPlanes * 16];
+#pragma unroll
+                for (int i = 0; i < kPlanes; ++i) {
+                    uint32_t w16[16];
+                    tmem_ld16(tmem + tlane + (uint32_t)(buf * kDpAccCols + kPlanes * 16 * g + 16 * i), w16);
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) v[16 * i + k] = w16[k];
+                }
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    const int tk = 16 * g + c;
+                    if (tk >= u.ntok) break;
+                    const int prow = u.prow0 + tk;
+                    const int64_t sum = (int64_t)(int)v[kPlanes * c] + ((int64_t)(int)v[kPlanes * c + 1] << 8) +
+                                        ((int64_t)(int)v[kPlanes * c + 2] << 16) +
+                                        ((int64_t)(int)v[kPlanes * c + 3] << 24) +
+                                        ((int64_t)(int)v[kPlanes * c + 4] << 32);
+                    const double accd = __dmul_rn(__ll2double_rn(sum), __ldg(p.pe + prow));
+                    const float val = __double2float_rn(__dmul_rn(sr, accd));
+                    if (p.mode == 0) {
+                        p.gu[((int64_t)(up ? p.prows_cap : 0) + prow) * p.I + r] = val;
+                    } else {
+                        const int slot = p.row_slot[prow];
+                        if (slot >= 0) p.y[(int64_t)slot * p.H + r] = val;
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acce[buf]);
         }
     }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    if (warp == kDpMmaWarp) tmem_dealloc(tmem, 2 * kDpAccCols);
+}
+
+// SwiGLU and Q8_0 of h, one CTA per padded row (warp w takes the row's
+// blocks w, w + 8, ..., lane = element): h = silu(g) * u evaluated in fp64
+// and rounded to fp32, then Q8_0; the codes and scales go to the slot's h
+// (hq, hd), to the row's codes and transposed fp64 scales (hg, hdT: the
+// fp64-epilogue GEMM's operands) and, as in k_tc_quantize, to the row's
+// digit planes [5][inter] with 2^E in peh (a row whose exponents spread over
+// more than kMaxSpread sets *wide instead).  Padding rows: zero planes and
+// scales.
+__global__ void __launch_bounds__(kQuantThreads) k_tc_swiglu(const float* __restrict__ gu, int I, int prows_cap,
+                                                             const int32_t* __restrict__ row_slot,
+                                                             const int32_t* __restrict__ ctrl, int8_t* __restrict__ hg,
+                                                             double* __restrict__ hdT, int8_t* __restrict__ hq,
+                                                             float* __restrict__ hd, int8_t* __restrict__ hp,
+                                                             double* __restrict__ peh, int* wide) {
+    __shared__ int s_e[2][kQuantThreads / 32];
+    const int q = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (q >= ctrl[2]) return;
+    const int nbI = I / 32, nw = kQuantThreads / 32;
+    const int slot = row_slot[q];
+    int8_t* dst = hp + (int64_t)q * kPlanes * I;
+    if (slot < 0) {  // a padding row
+        for (int b = warp; b < nbI; b += nw) {
+            if (lane == 0) hdT[(int64_t)b * prows_cap + q] = 0.0;
+#pragma unroll
+            for (int pl = 0; pl < kPlanes; ++pl) dst[(int64_t)pl * I + 32 * b + lane] = 0;
+        }
+        if (threadIdx.x == 0) peh[q] = 0.0;
+        return;
+    }
+    float g[kMaxBlocksPerWarp], u[kMaxBlocksPerWarp];
+#pragma unroll
+    for (int j = 0; j < kMaxBlocksPerWarp; ++j) {
+        const int b = warp + nw * j;
+        g[j] = b < nbI ? gu[(int64_t)q * I + 32 * b + lane] : 0.f;
+        u[j] = b < nbI ? gu[((int64_t)prows_cap + q) * I + 32 * b + lane] : 0.f;
+    }
+    int qv[kMaxBlocksPerWarp];
+    uint32_t mm[kMaxBlocksPerWarp];
+    int ee[kMaxBlocksPerWarp];
+    int emin = 0x7FFFFFFF, emax = -0x7FFFFFFF;
+#pragma unroll
+    for (int j = 0; j < kMaxBlocksPerWarp; ++j) {
+        const int b = warp + nw * j;
+        qv[j] = 0;
+        mm[j] = 0u;
+        ee[j] = 0;
+        if (b < nbI) {  // the same in the whole warp
+            const int i = 32 * b + lane;
+            const double gd = (double)g[j];
+            const float h = __double2float_rn(__dmul_rn(__ddiv_rn(gd, __dadd_rn(1.0, exp(-gd))), (double)u[j]));
+            int8_t qq;
+            float d;
+            q8_0_warp(h, qq, d);
+            hg[(int64_t)q * I + i] = qq;
+            hq[(int64_t)slot * I + i] = qq;
+            if (lane == 0) {
+                hdT[(int64_t)b * prows_cap + q] = (double)d;
+                hd[(int64_t)slot * nbI + b] = d;
+            }
+            qv[j] = qq;
+            f32_mant_exp(d, mm[j], ee[j]);
+            if (mm[j]) {
+                emin = min(emin, ee[j]);
+                emax = max(emax, ee[j]);
+            }
+        }
+    }
+    if (lane == 0) {
+        s_e[0][warp] = emin;
+        s_e[1][warp] = emax;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < nw; ++w) {
+        emin = min(emin, s_e[0][w]);
+        emax = max(emax, s_e[1][w]);
+    }
+    const bool any = emin <= emax;
+    if (any && emax - emin > kMaxSpread) {
+        if (threadIdx.x == 0) atomicOr(wide, 1);
+        return;
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxBlocksPerWarp; ++j) {
+        const int b = warp + nw * j;
+        if (b < nbI) {
+            const uint32_t m = mm[j] ? mm[j] << (ee[j] - emin) : 0u;
+            int c[kPlanes];
+            digits5(qv[j], m, c);
+#pragma unroll
+            for (int pl = 0; pl < kPlanes; ++pl) dst[(int64_t)pl * I + 32 * b + lane] = (int8_t)c[pl];
+        }
+    }
+    if (threadIdx.x == 0) peh[q] = any ? ldexp(1.0, emin) : 0.0;
 }
 
 }  // namespace tc
@@ -785,6 +1218,9 @@ __global__ void __launch_bounds__(256) k_tc_swiglu(const float* __restrict__ gu,
 bool tc_path_supported(const moe_config& c, int T) {
     if (T < kTcMinTokens) return false;
     if (c.hidden % tc::kTileRows || c.inter % tc::kTileRows) return false;
+    // one CTA of the quantisers holds a row's blocks in registers
+    const int max_cols = tc::kMaxBlocksPerWarp * (tc::kQuantThreads / 32) * 32;
+    if (c.hidden > max_cols || c.inter > max_cols) return false;
     return c.wbits == 8 || c.wbits == 4 || c.wbits == 2;
 }
 
@@ -793,7 +1229,7 @@ TcSizes tc_sizes(const moe_config& c, int T) {
     const int64_t entries = (c.n_experts < pairs ? c.n_experts : pairs) + c.n_shared;
     TcSizes z;
     z.prows_cap = (int)(((slots + 15 * entries) + 63) / 64 * 64 + 64);
-    const int64_t chunks = (slots + tc::kMaxN - 1) / tc::kMaxN + entries;
+    const int64_t chunks = (slots + tc::kChunk - 1) / tc::kChunk + entries;
     z.units_gu_cap = (int)(2 * chunks * (c.inter / tc::kTileRows));
     z.units_dn_cap = (int)(chunks * (c.hidden / tc::kTileRows));
     return z;
@@ -812,8 +1248,15 @@ cudaError_t launch_tc_prepare(const TcArgs& a, cudaStream_t s) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int grid = (a.sz.prows_cap + 7) / 8;
-    tc::k_tc_gather<<<grid, 256, 0, s>>>(a.ex.xq, a.ex.xd, c.hidden, a.sz.prows_cap, a.row_tok, a.ctrl, a.xg,
-                                         a.xdT);
+    tc::k_tc_gather<<<grid, 256, 0, s>>>(a.ex.xq, a.ex.xd, a.xpt, a.pet, a.xwide, c.hidden, a.sz.prows_cap,
+                                         a.row_tok, a.ctrl, a.xg, a.xdT, a.xp, a.pex);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_tc_quantize(const float* x, int T, int H, int8_t* xq, float* xd, int8_t* xpt, double* pet,
+                               int* xwide, cudaStream_t s) {
+    if (T == 0) return cudaSuccess;
+    tc::k_tc_quantize<<<T, tc::kQuantThreads, 0, s>>>(x, H, xq, xd, xpt, pet, xwide);
     return cudaGetLastError();
 }
 
@@ -841,6 +1284,43 @@ static cudaError_t launch_gemm(int wbits, const CUtensorMap (&m)[6], const GemmP
     if (wbits == 4) return launch_gemm_t<4>(m, gp, s);
     if (wbits == 2) return launch_gemm_t<2>(m, gp, s);
     return launch_gemm_t<8>(m, gp, s);
+}
+
+template <int WBITS>
+static cudaError_t launch_gemm_dp_t(const CUtensorMap (&m)[7], const GemmParams& gp, cudaStream_t s) {
+    using L = DpSmem<WBITS>;
+    static_assert(L::kStages >= 2, "at least two pipeline stages");
+    static bool attr_done[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (!attr_done[dev]) {
+        const cudaError_t e =
+            cudaFuncSetAttribute(k_tc_gemm_dp<WBITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+        if (e != cudaSuccess) return e;
+        attr_done[dev] = true;
+    }
+    k_tc_gemm_dp<WBITS><<<device_info().sm_count, kDpThreads, L::kBytes, s>>>(m[0], m[1], m[2], m[3], m[4], m[5],
+                                                                               m[6], gp);
+    return cudaGetLastError();
+}
+
+static cudaError_t launch_gemm_dp(int wbits, const CUtensorMap (&m)[7], const GemmParams& gp, cudaStream_t s) {
+    if (wbits == 4) return launch_gemm_dp_t<4>(m, gp, s);
+    if (wbits == 2) return launch_gemm_dp_t<2>(m, gp, s);
+    return launch_gemm_dp_t<8>(m, gp, s);
+}
+
+// Maps of a plane tensor [prows_cap * kPlanes][K] with boxes of 80, 160 and
+// 240 rows (the chunk's planes at 16, 32 or 48 tokens), 128-byte swizzle.
+static cudaError_t encode_planes(CUtensorMap (&b)[3], const int8_t* planes, int K, int prows_cap) {
+    for (int g = 0; g < 3; ++g) {
+        const cudaError_t e = encode_2d(&b[g], planes, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)K,
+                                        (uint64_t)prows_cap * kPlanes, (uint64_t)K, kStageK,
+                                        (uint32_t)(kPlanes * 16 * (g + 1)), CU_TENSOR_MAP_SWIZZLE_128B);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 // Token-side maps of a GEMM: codes [prows_cap][K] (128-byte swizzle) and block
@@ -878,11 +1358,17 @@ cudaError_t launch_tc_experts(const TcArgs& a, cudaStream_t s, cudaEvent_t const
         gp.n_units_idx = 0; gp.counter = a.ctrl + 3; gp.row_slot = a.row_slot;
         gp.s_r0 = R.s_gate; gp.s_r1 = R.s_up; gp.s_s0 = Sh.s_gate; gp.s_s1 = Sh.s_up;
         gp.gu = a.gu; gp.y = a.ex.y; gp.err = a.ex.err;
+        gp.wide = a.xwide; gp.pe = a.pex;
+        CUtensorMap md[7] = {m[0], m[1], m[2], m[3]};
+        if ((e = encode_planes(*reinterpret_cast<CUtensorMap(*)[3]>(&md[4]), a.xp, H, a.sz.prows_cap)) != cudaSuccess)
+            return e;
+        // the digit-plane GEMM, or (a token too wide for the planes) the fp64 one
+        if ((e = launch_gemm_dp(wb, md, gp, s)) != cudaSuccess) return e;
         if ((e = launch_gemm(wb, m, gp, s)) != cudaSuccess) return e;
         // the "gate_up" phase ends with the GEMM; SwiGLU opens the "down" phase
         if (ev && (e = record_event(ev[0], s)) != cudaSuccess) return e;
-        const int grid = device_info().sm_count * 8;
-        k_tc_swiglu<<<grid, 256, 0, s>>>(a.gu, I, a.sz.prows_cap, a.row_slot, a.ctrl, a.hg, a.hdT, a.ex.hq, a.ex.hd);
+        k_tc_swiglu<<<a.sz.prows_cap, kQuantThreads, 0, s>>>(a.gu, I, a.sz.prows_cap, a.row_slot, a.ctrl, a.hg, a.hdT,
+                                                            a.ex.hq, a.ex.hd, a.hp, a.peh, a.hwide);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     // down: weights [E * H][I], h codes hg / hdT -> y per slot
@@ -899,6 +1385,11 @@ cudaError_t launch_tc_experts(const TcArgs& a, cudaStream_t s, cudaEvent_t const
         gp.n_units_idx = 1; gp.counter = a.ctrl + 4; gp.row_slot = a.row_slot;
         gp.s_r0 = R.s_down; gp.s_r1 = R.s_down; gp.s_s0 = Sh.s_down; gp.s_s1 = Sh.s_down;
         gp.gu = a.gu; gp.y = a.ex.y; gp.err = a.ex.err;
+        gp.wide = a.hwide; gp.pe = a.peh;
+        CUtensorMap md[7] = {m[0], m[1], m[2], m[3]};
+        if ((e = encode_planes(*reinterpret_cast<CUtensorMap(*)[3]>(&md[4]), a.hp, I, a.sz.prows_cap)) != cudaSuccess)
+            return e;
+        if ((e = launch_gemm_dp(wb, md, gp, s)) != cudaSuccess) return e;
         if ((e = launch_gemm(wb, m, gp, s)) != cudaSuccess) return e;
         if (ev && (e = record_event(ev[1], s)) != cudaSuccess) return e;
     }

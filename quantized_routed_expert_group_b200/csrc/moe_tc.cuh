@@ -32,11 +32,47 @@ constexpr int kBlocksPerStage = kStageK / 32;
 constexpr int kMaxN = 64;       // tokens per unit (MMA N, in steps of 16)
 constexpr int kTileBytes = kTileRows * kStageK;  // one widened weight tile of a stage
 
+// Exact digit planes of the block-scaled activations.  A token's Q8_0 block
+// scales d_b = m_b 2^e_b (fp32: m_b < 2^24 an integer) share the exponent
+// E = min_b e_b; with spread = max_b e_b - E <= kMaxSpread, every scaled code
+// q m_b 2^(e_b - E) is an integer below 127 * 2^32 in magnitude and splits
+// exactly into kPlanes signed base-256 digits, each an int8.  So
+//   sum_b d_b dot_b(w, q) = 2^E sum_p 256^p (w . plane_p)
+// and the tensor core accumulates each plane's product in int32 over the
+// whole K (|w . plane_p| <= K * 127 * 128 < 2^31 for K <= 2^17).
+constexpr int kPlanes = 5;
+constexpr int kMaxSpread = 8;
+constexpr int kChunk = 48;  // tokens per unit of the grouped GEMMs (kPlanes * 48 = 240 <= 256 MMA columns)
+
+// Integer mantissa and exponent of a finite fp32 value v >= 0: v = m 2^e with
+// m < 2^24 (m = 0 for v = 0).
+__device__ __forceinline__ void f32_mant_exp(float v, uint32_t& m, int& e) {
+    const uint32_t b = __float_as_uint(v);
+    const uint32_t f = (b >> 23) & 0xFFu;
+    m = f ? ((b & 0x7FFFFFu) | 0x800000u) : (b & 0x7FFFFFu);
+    e = f ? (int)f - 150 : -149;
+}
+
+// The kPlanes signed base-256 digits of q * m (|q| <= 127, m < 2^32): q m =
+// sum_p 256^p c_p with c_p in [-128, 127], lowest first.  q m is split as
+// q (m >> 16) 2^16 + q (m & 0xFFFF), both products below 2^23.
+__device__ __forceinline__ void digits5(int q, uint32_t m, int (&c)[kPlanes]) {
+    const int lo = q * (int)(m & 0xFFFFu), hi = q * (int)(m >> 16);
+    c[0] = (int)(int8_t)lo;
+    int r = (lo - c[0]) >> 8;
+    c[1] = (int)(int8_t)r;
+    r = ((r - c[1]) >> 8) + hi;
+    c[2] = (int)(int8_t)r;
+    r = (r - c[2]) >> 8;
+    c[3] = (int)(int8_t)r;
+    c[4] = (r - c[3]) >> 8;
+}
+
 // A unit of work of the grouped GEMMs: one 128-row tile of one expert's
-// weight matrix applied to a chunk of <= kMaxN of the expert's tokens.
+// weight matrix applied to a chunk of <= kChunk of the expert's tokens.
 struct TcUnit {
     int prow0;  // first row of the chunk in the padded row space
-    int ntok;   // tokens of the chunk (1 .. kMaxN)
+    int ntok;   // tokens of the chunk (1 .. kChunk)
     int wrow0;  // first weight row in the bank's matrix (expert * rows + 128 * tile)
     int info;   // tile index | kUnitShared
 };

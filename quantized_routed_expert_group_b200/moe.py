@@ -77,7 +77,7 @@ _SIGS = {
 PROFILE_MAX_EVENTS = 8
 # launches of one forward on each path (moe_forward_launches): fused small
 # batch, multi-kernel, batched tensor-core
-SMALL_LAUNCHES, MULTI_KERNEL_LAUNCHES, TC_LAUNCHES = 1, 7, 10
+SMALL_LAUNCHES, MULTI_KERNEL_LAUNCHES, TC_LAUNCHES = 1, 7, 12
 
 _LIB = None
 
@@ -434,6 +434,8 @@ class MoeLayer:
             "hq": at(L.hq, torch.int8, (slots, s.inter)),
             "hd": at(L.hd, torch.float32, (slots, s.inter // 32)),
             "y": at(L.y, torch.float32, (slots, s.hidden)),
+            # batched tensor-core path: [x, h] took the fp64-epilogue GEMM
+            "fp64_fallback": at(L.error + 32, torch.int32, (2,)),
         }
 
     def device_error(self, stream=None) -> int:

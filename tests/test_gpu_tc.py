@@ -2,16 +2,21 @@
 the oracle, through the C ABI.
 
 At these batch sizes every selected expert meets several tokens per weight
-row, so the layer runs the grouped int8 GEMMs: the tensor core produces the
-exact int32 block dots, and the epilogue applies the block scales in fp64 in
-block order, the row scale in fp64, SwiGLU in fp64 and the combine in fp64,
-the same operations in the same order as the oracle.  So beyond the 1e-3
-output bound, the h codes, the per-slot expert outputs y and the layer output
-are compared bit for bit.
+row, so the layer runs the grouped int8 GEMMs.  Each token's block-scaled
+Q8_0 activations (and each row's h) are split exactly into five signed int8
+digit planes (block scales as integers over the token's smallest exponent,
+while the exponents lie within 8 of each other), so the tensor core sums
+the whole K in int32 per plane and the epilogue forms the exact sum once per
+output, scales it by the row scale in fp64 and rounds to fp32 -- what the
+oracle computes when its fp64 block sum is exact.  Tokens whose block scales
+spread wider take the fp64-epilogue GEMM (exact int32 block dots, fp64 block
+order).  SwiGLU is fp64, the combine fp64.  So beyond the 1e-3 output bound,
+the h codes, the per-slot expert outputs y and the layer output are compared
+bit for bit, and the test checks which GEMM form ran.
 
 Shapes: hidden and intermediate multiples of 128 (one MMA tile of rows); 1-3
 weight tiles per matrix and 2-5 pipeline stages per unit; token counts that
-leave ragged 16-token groups and 64-token chunks; int8, int4 and int2 weights;
+leave ragged 16-token groups and 48-token chunks; int8, int4 and int2 weights;
 no shared expert; the adaptive top-p dropping picks."""
 import numpy as np
 import pytest
@@ -31,13 +36,15 @@ TC4_TOPP = synth.LayerShape(512, 256, 32, 4, 2, 4, 1, 2.5, 4, topp=0.6)
 TC4_G32 = synth.LayerShape(256, 128, 128, 4, 2, 8, 1, 2.5, 4)   # groups of 32 experts, top-8, as GLM-5.2
 
 
-def _strict(pair, x):
+def _strict(pair, x, fallback=(0, 0)):
     s = pair.wl.shape
     T = x.shape[0]
-    assert moe.forward_launches(pair.layer.cfg, T) == 10, "expected the tensor-core path"
+    assert moe.forward_launches(pair.layer.cfg, T) == moe.TC_LAUNCHES, "expected the tensor-core path"
     out = pair.layer.forward(torch.from_numpy(np.ascontiguousarray(x)).cuda())
     torch.cuda.synchronize()
     assert pair.layer.device_error() == 0
+    # which GEMM form ran: the digit planes (0) or the fp64 epilogue (1), for x and h
+    assert tuple(pair.layer.view(T)["fp64_fallback"].cpu().tolist()) == fallback
     tr = orc.layer_forward(s, x, pair.router_w, pair.bias, pair.orc_routed, pair.orc_shared)
     v = {k: t.cpu().numpy() for k, t in pair.layer.view(T).items()}
     got = out.cpu().numpy()
@@ -81,11 +88,11 @@ def test_tc_then_small_batches_share_a_workspace():
 
 
 def test_tc_wide_block_scales_take_the_fp64_epilogue():
-    """Tokens whose block scales span more than 2^7 cannot use the integer
-    epilogue (m' would not fit 31 bits) and take the fp64 one: x with some
-    blocks scaled by 2^-12 on every third token (gate/up side), and a shared
-    expert whose first 32 up rows are scaled by 1e-4, so that h's first block
-    is tiny on every token (down side).  Still bit-identical."""
+    """Tokens whose block-scale exponents lie more than 8 apart do not fit the
+    five digit planes and take the fp64-epilogue GEMM: x with some blocks
+    scaled by 2^-12 on every third token (gate/up side), and a shared expert
+    whose first 32 up rows are scaled by 1e-4, so that h's first block is tiny
+    on every token (down side).  Still bit-identical."""
     def mutate(mats, shm):
         shm[1][:32] *= np.float32(1e-4)
 
@@ -95,4 +102,4 @@ def test_tc_wide_block_scales_take_the_fp64_epilogue():
     for t in range(0, T, 3):
         for b in range(0, TC4.hidden // 32, 5):
             x[t, 32 * b:32 * (b + 1)] *= np.float32(2.0 ** -12)
-    _strict(pair, x)
+    _strict(pair, x, fallback=(1, 1))
