@@ -848,13 +848,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // is formed exactly in int64 (a double while it stays below 2^53), and the
 // output is fp32(s_row * acc) in fp64, as the oracle rounds it.
 // warps 0-3  epilogue (warp w: TMEM lanes 32 w .. 32 w + 31 = its 32 rows)
-// warps 4-5  widening of packed int4 / int2 staging rows
-// warp 6     producer: units from a global counter, TMA per stage of the
+// warps 4-7  widening of packed int4 / int2 staging rows (one row per thread)
+// warp 8     producer: units from a global counter, TMA per stage of the
 //            weight rows and of the chunk's planes (box of 80, 160 or 240 rows)
-// warp 7     MMA: two accumulators of 256 TMEM columns, alternating units
+// warp 9     MMA: two accumulators of 256 TMEM columns, alternating units
 // Every wait is bounded by the global timer and records kErrTimeout.
 constexpr int kDpEpiWarps = 4;
-constexpr int kDpConvWarps = 2;
+constexpr int kDpConvWarps = 4;
 constexpr int kDpProdWarp = kDpEpiWarps + kDpConvWarps;
 constexpr int kDpMmaWarp = kDpProdWarp + 1;
 constexpr int kDpThreads = (kDpMmaWarp + 1) * 32;
@@ -895,8 +895,8 @@ __global__ void __launch_bounds__(kDpThreads, 1)
     uint64_t* accf = empty + S;   // [2] the accumulator's unit is complete (MMA commit)
     uint64_t* acce = accf + 2;    // [2] the epilogue has read the accumulator
     uint64_t* uready = acce + 2;  // [2] the accumulator's next unit id is in unit_of
-    int* meta = reinterpret_cast<int*>(uready + 2);  // [S][2]: unit (-1: end), stage of the unit
-    int* unit_of = meta + 2 * S;                      // [2]
+    int* meta = reinterpret_cast<int*>(uready + 2);  // [S][3]: unit (-1: end), stage of the unit, its tokens
+    int* unit_of = meta + 3 * S;                      // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(unit_of + 2);
     auto stage = [&](int s) { return sm + s * L::kStageBytes; };
 
@@ -936,21 +936,28 @@ __global__ void __launch_bounds__(kDpThreads, 1)
             tma_prefetch_map(&b48);
             int s = 0;
             uint32_t ph = 0;
+            // units come from the global counter one unit ahead: the next
+            // unit's id and description are requested when the current one
+            // starts, so that neither round trip stalls the stage sequence
             int unit = atomicAdd(p.counter, 1), kstep = 0;
             TcUnit u = unit < n_units ? p.units[unit] : TcUnit{0, 0, 0, 0};
+            int next = unit < n_units ? atomicAdd(p.counter, 1) : n_units;
+            TcUnit nu_ = next < n_units ? p.units[next] : TcUnit{0, 0, 0, 0};
             while (true) {
                 if (!mbar_wait_ns(&empty[s], ph ^ 1u, kGemmWaitNs)) {
                     set_error(p.err, kErrTimeout);
                     break;
                 }
                 if (unit >= n_units) {
-                    meta[2 * s] = -1;
-                    meta[2 * s + 1] = 0;
+                    meta[3 * s] = -1;
+                    meta[3 * s + 1] = 0;
+                    meta[3 * s + 2] = 0;
                     mbar_arrive(&full[s]);
                     break;
                 }
-                meta[2 * s] = unit;
-                meta[2 * s + 1] = kstep;
+                meta[3 * s] = unit;
+                meta[3 * s + 1] = kstep;
+                meta[3 * s + 2] = u.ntok;
                 const int ng = nt_groups(u.ntok);
                 mbar_arrive_expect_tx(&full[s], L::kWeightTx + (uint32_t)(kPlanes * 16 * ng * kStageK));
                 uint8_t* st = stage(s);
@@ -962,8 +969,10 @@ __global__ void __launch_bounds__(kDpThreads, 1)
                 tma_load_2d(st + L::kB, bm, kstep * kStageK, u.prow0 * kPlanes, &full[s]);
                 if (++kstep == p.nstage) {
                     kstep = 0;
-                    unit = atomicAdd(p.counter, 1);
-                    if (unit < n_units) u = p.units[unit];
+                    unit = next;
+                    u = nu_;
+                    next = unit < n_units ? atomicAdd(p.counter, 1) : n_units;
+                    if (next < n_units) nu_ = p.units[next];
                 }
                 if (++s == S) {
                     s = 0;
@@ -983,8 +992,8 @@ __global__ void __launch_bounds__(kDpThreads, 1)
                     set_error(p.err, kErrTimeout);
                     break;
                 }
-                const int unit = meta[2 * s];
-                const int kstep = meta[2 * s + 1];
+                const int unit = meta[3 * s];
+                const int kstep = meta[3 * s + 1];
                 if (unit < 0 || unit != cur) {
                     // a new unit (or the end) takes the next accumulator, once
                     // the epilogue has read that accumulator's previous unit;
@@ -999,7 +1008,7 @@ __global__ void __launch_bounds__(kDpThreads, 1)
                     mbar_arrive(&uready[buf]);
                     if (unit < 0) break;
                     cur = unit;
-                    idesc = idesc_i8(kPlanes * 16 * nt_groups(p.units[unit].ntok));
+                    idesc = idesc_i8(kPlanes * 16 * nt_groups(meta[3 * s + 2]));
                     acc = tmem + (uint32_t)(buf * kDpAccCols);
                 }
                 if (WBITS != 8 && !mbar_wait_ns(&conv[s], ph, kGemmWaitNs)) {
@@ -1026,7 +1035,7 @@ __global__ void __launch_bounds__(kDpThreads, 1)
     } else if (warp >= kDpEpiWarps) {
         // ---------------- widening ----------------
         if constexpr (WBITS != 8) {
-            const int r0 = threadIdx.x - kDpEpiWarps * 32;  // rows r0 and r0 + 64 of the tile
+            const int r0 = threadIdx.x - kDpEpiWarps * 32;  // rows r0, r0 + 32 kDpConvWarps, ... of the tile
             int s = 0;
             uint32_t ph = 0;
             while (true) {
@@ -1034,10 +1043,10 @@ __global__ void __launch_bounds__(kDpThreads, 1)
                     set_error(p.err, kErrTimeout);
                     break;
                 }
-                if (meta[2 * s] < 0) break;
+                if (meta[3 * s] < 0) break;
                 uint8_t* st = stage(s);
-                widen_row<WBITS>(st + L::kRaw, st + L::kA, r0);
-                widen_row<WBITS>(st + L::kRaw, st + L::kA, r0 + 64);
+#pragma unroll
+                for (int r = r0; r < kTileRows; r += 32 * kDpConvWarps) widen_row<WBITS>(st + L::kRaw, st + L::kA, r);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&conv[s]);
@@ -1074,6 +1083,13 @@ __global__ void __launch_bounds__(kDpThreads, 1)
             const double sr = (double)__ldg(sc + u.wrow0 + rl);
             const int r = tile * kTileRows + rl;  // output row of this thread
             const int ng = nt_groups(u.ntok);
+            // the chunk's 2^E and (down) slots, one token per lane (kChunk <= 64),
+            // loaded together and broadcast per token below
+            const bool ina = lane < u.ntok, inb = lane + 32 < u.ntok;
+            const double pea = ina ? __ldg(p.pe + u.prow0 + lane) : 0.0;
+            const double peb = inb ? __ldg(p.pe + u.prow0 + lane + 32) : 0.0;
+            const int sla = (p.mode == 1 && ina) ? __ldg(p.row_slot + u.prow0 + lane) : -1;
+            const int slb = (p.mode == 1 && inb) ? __ldg(p.row_slot + u.prow0 + lane + 32) : -1;
             for (int g = 0; g < ng; ++g) {
                 uint32_t v[kPlanes * 16];
 #pragma unroll
@@ -1087,19 +1103,19 @@ __global__ void __launch_bounds__(kDpThreads, 1)
 #pragma unroll
                 for (int c = 0; c < 16; ++c) {
                     const int tk = 16 * g + c;
-                    if (tk >= u.ntok) break;
-                    const int prow = u.prow0 + tk;
+                    if (tk >= u.ntok) break;  // the same in the whole warp
+                    const double pe = __shfl_sync(kFull, tk < 32 ? pea : peb, tk & 31);
+                    const int slot = __shfl_sync(kFull, tk < 32 ? sla : slb, tk & 31);
                     const int64_t sum = (int64_t)(int)v[kPlanes * c] + ((int64_t)(int)v[kPlanes * c + 1] << 8) +
                                         ((int64_t)(int)v[kPlanes * c + 2] << 16) +
                                         ((int64_t)(int)v[kPlanes * c + 3] << 24) +
                                         ((int64_t)(int)v[kPlanes * c + 4] << 32);
-                    const double accd = __dmul_rn(__ll2double_rn(sum), __ldg(p.pe + prow));
+                    const double accd = __dmul_rn(__ll2double_rn(sum), pe);
                     const float val = __double2float_rn(__dmul_rn(sr, accd));
                     if (p.mode == 0) {
-                        p.gu[((int64_t)(up ? p.prows_cap : 0) + prow) * p.I + r] = val;
-                    } else {
-                        const int slot = p.row_slot[prow];
-                        if (slot >= 0) p.y[(int64_t)slot * p.H + r] = val;
+                        p.gu[((int64_t)(up ? p.prows_cap : 0) + u.prow0 + tk) * p.I + r] = val;
+                    } else if (slot >= 0) {
+                        p.y[(int64_t)slot * p.H + r] = val;
                     }
                 }
             }

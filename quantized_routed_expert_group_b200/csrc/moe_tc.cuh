@@ -43,6 +43,7 @@ constexpr int kTileBytes = kTileRows * kStageK;  // one widened weight tile of a
 constexpr int kPlanes = 5;
 constexpr int kMaxSpread = 8;
 constexpr int kChunk = 48;  // tokens per unit of the grouped GEMMs (kPlanes * 48 = 240 <= 256 MMA columns)
+static_assert(kChunk <= 64, "the epilogue holds a chunk's tokens in two lanes each");
 
 // Integer mantissa and exponent of a finite fp32 value v >= 0: v = m 2^e with
 // m < 2^24 (m = 0 for v = 0).
