@@ -101,7 +101,7 @@ def gateup_bytes(shape) -> int:
 KERNEL_SOURCES = {
     "k_moe_small": ["moe_small.cu", "moe_device.cuh", "moe_ptx.cuh"],
     "k_gateup": ["moe_expert.cu", "moe_device.cuh", "moe_ptx.cuh"],
-    "k_tc_gemm": ["moe_tc.cu", "moe_tc.cuh", "moe_device.cuh", "moe_ptx.cuh"],
+    "k_tc_gemm_dp": ["moe_tc.cu", "moe_tc.cuh", "moe_device.cuh", "moe_ptx.cuh"],
 }
 
 
@@ -206,11 +206,12 @@ def step_stats(ms: list[float]) -> dict:
             "min": round(min(ms), 5), "max": round(max(ms), 5)}
 
 
-def capture_steps(torch, moe, layer, batches, out, flush=None):
+def capture_steps(torch, moe, layer, batches, out, flush=None, phase_events=True):
     """One CUDA graph of len(batches) consecutive forwards, each bracketed by
-    the library's phase events (moe_profile_events), with an L2 flush before
-    each when `flush` is given.  Returns (graph, events), or (None, events)
-    if the capture fails (the caller then runs the steps eagerly)."""
+    the library's phase events (moe_profile_events) unless phase_events is
+    False, with an L2 flush before each when `flush` is given.  Returns
+    (graph, events), or (None, events) if the capture fails (the caller then
+    runs the steps eagerly)."""
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.PROFILE_MAX_EVENTS)] for _ in batches]
     for row in evs:  # torch creates the CUDA event on first record
         for ev in row:
@@ -225,7 +226,8 @@ def capture_steps(torch, moe, layer, batches, out, flush=None):
                 for i, x in enumerate(batches):
                     if flush is not None:
                         flush.fill_(i & 0xFF)
-                    moe.profile_events(evs[i])
+                    if phase_events:
+                        moe.profile_events(evs[i])
                     layer.forward(x, out)
                 moe.profile_events(None)
         torch.cuda.current_stream().wait_stream(side)
@@ -284,10 +286,13 @@ def run_ours(args) -> dict | None:
     phases = moe.forward_phases(layer.cfg, wl.T)
     P = len(phases)
     # the K timed steps as one CUDA graph: the device runs them back to back
-    # whatever the host's pace, and each step is timed by the library's own
-    # events at its phase boundaries inside the graph
+    # whatever the host's pace; the graph is timed by two events around it
+    # (ms_per_step = total / K).  A second graph of the same K steps carries
+    # the library's events at each step's phase boundaries (per-step median,
+    # phase times); those events cost a little time of their own.
     batches = [xs[i % R] for i in range(K)]
     graph, evs = capture_steps(torch, moe, layer, batches, out)
+    graph_plain, _ = capture_steps(torch, moe, layer, batches, out, phase_events=False)
     run_steps(torch, moe, layer, batches[: min(K, args.warmup)], out, None,
               evs[: min(K, args.warmup)])  # untimed eager steps after the capture
     torch.cuda.synchronize()
@@ -303,24 +308,33 @@ def run_ours(args) -> dict | None:
     torch.cuda.synchronize()
     sampler = ClockSampler(gpu_uuid)
     time.sleep(0.15)
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if graph_plain is not None:
+        e_start.record()
+        graph_plain.replay()
+        e_end.record()
     run_steps(torch, moe, layer, batches, out, graph, evs)
     torch.cuda.synchronize()
     clocks = sampler.stop()
-    graph_used = graph is not None
+    graph_used = graph is not None and graph_plain is not None
     if world > 1:
         dist.barrier()
     step_ms = [evs[i][0].elapsed_time(evs[i][P]) for i in range(K)]
     phase_ms = [[evs[i][p].elapsed_time(evs[i][p + 1]) for i in range(K)] for p in range(P)]
     assert layer.device_error() == 0
-    del graph
-    total_ms = sum(step_ms)
+    del graph, graph_plain
+    total_ms = e_start.elapsed_time(e_end) if graph_used else sum(step_ms)
     max_total = reduce_max(total_ms, dev)
     value = throughput(wl.T, K, world, max_total)
     # active experts of each rotation (the bytes a step streams)
     n_active = []
+    tokens_per_entry = []  # of the first batch: routed experts' token counts, then the shared expert's
     for i in range(R):
         layer.forward(xs[i], out)
-        n_active.append(int((layer.view(wl.T)["counts"] > 0).sum().item()))
+        cnt = layer.view(wl.T)["counts"]
+        n_active.append(int((cnt > 0).sum().item()))
+        if i == 0:
+            tokens_per_entry = [int(c) for c in cnt.cpu().tolist() if c > 0] + ([wl.T] * s.n_shared)
     torch.cuda.synchronize()
 
     # variants, reported alongside: the same batch every step (no flush), and
@@ -354,13 +368,13 @@ def run_ours(args) -> dict | None:
     router_bytes = s.n_experts * s.hidden * 4
     mean_active = statistics.mean(n_active)
     layer_bytes = (mean_active + s.n_shared) * expert_bytes(s)
-    ms_step = statistics.mean(step_ms)
+    ms_step = max_total / K
     layer_gbs = layer_bytes / (ms_step * 1e-3) / 1e9
     tensor = None
     if phases == ["fused"]:
-        # the fused phase: the prologue (Q8_0 of x, router logits over the
-        # router weights) and the persistent kernel (the experts) are the whole
-        # step, timed as graph replays; bytes and ncu traffic cover both
+        # the fused path: one persistent kernel is the whole step (Q8_0 of x,
+        # router logits over the router weights, selection, experts,
+        # combine); its bytes are the experts' and the router matrix
         dom_kernel, dom_ms = "k_moe_small", ms_step
         dom_bytes = layer_bytes + router_bytes
     else:
@@ -368,15 +382,24 @@ def run_ours(args) -> dict | None:
         dom_bytes = (mean_active + s.n_shared) * gateup_bytes(s)
         dom_ms = gu_ms
         if moe.forward_launches(layer.cfg, wl.T) == moe.TC_LAUNCHES:
-            dom_kernel = "k_tc_gemm"
+            dom_kernel = "k_tc_gemm_dp"
             # int8 tensor work of the gate/up GEMM: 2 ops per MAC, gate and up
+            # (algorithmic: every (token, pick) once; issued: the five digit
+            # planes of each token over its 48-token chunk padded to 16)
             ops = 2.0 * 2.0 * (wl.T * s.top_k + wl.T * s.n_shared) * s.hidden * s.inter
+            pad_rows = 0
+            for n in tokens_per_entry:
+                full, rem = divmod(int(n), 48)
+                pad_rows += 48 * full + 16 * ((rem + 15) // 16)
+            issued = 2.0 * 2.0 * 5 * pad_rows * s.hidden * s.inter
             bf16, bf16_kind = measured_peak_bf16()
             i8_peak = bf16 * TENSOR_I8_NOMINAL_RATIO
             tops = ops / (gu_ms * 1e-3) / 1e12
-            tensor = {"kernel": "k_tc_gemm (gate/up)", "int8_ops": ops, "achieved_tops": round(tops, 1),
+            itops = issued / (gu_ms * 1e-3) / 1e12
+            tensor = {"kernel": "k_tc_gemm_dp (gate/up)", "int8_ops": ops, "achieved_tops": round(tops, 1),
+                      "issued_int8_ops": issued, "issued_tops": round(itops, 1),
                       "peak_tops": i8_peak, "peak_kind": f"{bf16_kind} bf16 x {TENSOR_I8_NOMINAL_RATIO:g} (nominal int8/bf16)",
-                      "frac": round(tops / i8_peak, 4)}
+                      "frac": round(tops / i8_peak, 4), "issued_frac": round(itops / i8_peak, 4)}
         else:
             dom_kernel = "k_gateup"
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
@@ -390,8 +413,9 @@ def run_ours(args) -> dict | None:
                    "experts": s.n_experts, "top_k": s.top_k, "shared": s.n_shared, "weights": f"int{s.wbits}",
                    "activations": "Q8_0 int8", "unique_experts_per_step": round(mean_active, 2),
                    "token_batches": f"{R} seeded batches, step i uses batch i mod {R}",
-                   "timing": ("the K steps as one CUDA graph, each step timed by the library's events at its "
-                              "first launch and after its last" if graph_used else
+                   "timing": ("the K steps as one CUDA graph timed by two events around it (ms_per_step = total "
+                              "/ K); step_ms and phases_ms from a second graph of the same steps with the library's "
+                              "events at each step's phase boundaries" if graph_used else
                               "eager steps timed by the library's events (graph capture unavailable)"),
                    "l2": ("not flushed: every step streams its selected experts' weights, more than L2 holds, "
                           "and consecutive steps select different experts"),

@@ -605,7 +605,9 @@ MOE_API int moe_forward_launches(const moe_config* cfg, int T) {
     if (st) return st;
     if (T < 0) return MOE_EINVAL;
     if (T == 0) return 0;
-    return small_path_supported(*cfg, T) ? kSmallLaunches : tc_path_supported(*cfg, T) ? kTcLaunches : kForwardLaunches;
+    if (small_path_supported(*cfg, T)) return kSmallLaunches;
+    if (tc_path_supported(*cfg, T)) return kTcLaunches;
+    return kForwardLaunches + (router_splits(*cfg, T) > 0 ? 1 : 0);
 }
 
 MOE_API int moe_forward_phases(const moe_config* cfg, int T) {

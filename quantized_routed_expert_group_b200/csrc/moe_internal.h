@@ -97,14 +97,17 @@ struct ExpertArgs {
 };
 // ev (optional, 3 events): recorded after gate/up, down and combine.
 cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t s, cudaEvent_t const* ev);
+int router_splits(const moe_config& c, int T);
 constexpr int kForwardLaunches = 7;  // quantise, logits, select, bucket, gate/up, down, combine
+// (+1 when the router logits take the split-K form: router_splits > 0)
 cudaError_t launch_combine(const ExpertArgs& a, cudaStream_t s);
 
 // Batched path on the tensor cores (moe_tc.cu), for T >= kTcMinTokens.
 constexpr int kTcMinTokens = 64;
-// quantise, logits, select, bucket, plan, planes; gate/up on the digit planes and its fp64
-// fallback (one of the two returns at once), SwiGLU, down and its fallback, combine
-constexpr int kTcLaunches = 12;
+// quantise (with the digit planes), router logits, their split-K reduce, select,
+// bucket, plan, gather; gate/up on the digit planes and its fp64 fallback (one
+// of the two returns at once), SwiGLU, down and its fallback, combine
+constexpr int kTcLaunches = 13;
 bool tc_path_supported(const moe_config& c, int T);
 struct TcSizes {
     int prows_cap;     // rows of the padded row space

@@ -410,74 +410,82 @@ __global__ void __launch_bounds__(kPlanThreads) k_tc_plan(PlanParams p) {
 // kMaxSpread sets *wide; the call then takes the fp64-epilogue GEMMs and the
 // planes are not used.
 constexpr int kQuantThreads = 256;
-constexpr int kMaxBlocksPerWarp = 32;  // hidden <= 8 * 32 * 32
+constexpr int kMaxQuantCols = 8192;  // hidden and inter of the batched path
 
-__global__ void __launch_bounds__(kQuantThreads) k_tc_quantize(const float* __restrict__ x, int H,
-                                                               int8_t* __restrict__ xq, float* __restrict__ xd,
-                                                               int8_t* __restrict__ xpt, double* __restrict__ pet,
-                                                               int* wide) {
-    __shared__ int s_e[2][kQuantThreads / 32];
-    const int t = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nb = H / 32, nw = kQuantThreads / 32;
-    const float* xt = x + (int64_t)t * H;
-    float v[kMaxBlocksPerWarp];
-#pragma unroll
-    for (int j = 0; j < kMaxBlocksPerWarp; ++j) {
-        const int b = warp + nw * j;
-        v[j] = b < nb ? __ldg(xt + 32 * b + lane) : 0.f;
-    }
-    int qv[kMaxBlocksPerWarp];
-    uint32_t mm[kMaxBlocksPerWarp];
-    int ee[kMaxBlocksPerWarp];
+// The digit planes of one row of n codes (Q8_0 blocks of 32) from its codes
+// and block scales in shared memory: the row's smallest block exponent E
+// and spread (CTA-wide), then each thread's elements split into kPlanes
+// digits written to planes [kPlanes][n]; 2^E to *pe (0 for an all-zero row).
+// A row whose exponents spread over more than kMaxSpread sets *wide and
+// writes no planes.  Every thread of the CTA calls it.
+__device__ __forceinline__ void row_planes(const int8_t* s_q, const uint32_t* s_m, const int* s_e, int n,
+                                           int* s_red, int8_t* __restrict__ planes, double* __restrict__ pe,
+                                           int* wide) {
+    const int nb = n / 32, warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     int emin = 0x7FFFFFFF, emax = -0x7FFFFFFF;
-#pragma unroll
-    for (int j = 0; j < kMaxBlocksPerWarp; ++j) {
-        const int b = warp + nw * j;
-        qv[j] = 0;
-        mm[j] = 0u;
-        ee[j] = 0;
-        if (b < nb) {  // the same in the whole warp
-            int8_t q;
-            float d;
-            q8_0_warp(v[j], q, d);
-            xq[(int64_t)t * H + 32 * b + lane] = q;
-            if (lane == 0) xd[(int64_t)t * nb + b] = d;
-            qv[j] = q;
-            f32_mant_exp(d, mm[j], ee[j]);
-            if (mm[j]) {
-                emin = min(emin, ee[j]);
-                emax = max(emax, ee[j]);
-            }
+    for (int b = threadIdx.x; b < nb; b += blockDim.x)
+        if (s_m[b]) {
+            emin = min(emin, s_e[b]);
+            emax = max(emax, s_e[b]);
         }
-    }
+    emin = __reduce_min_sync(kFull, emin);
+    emax = __reduce_max_sync(kFull, emax);
     if (lane == 0) {
-        s_e[0][warp] = emin;
-        s_e[1][warp] = emax;
+        s_red[warp] = emin;
+        s_red[nw + warp] = emax;
     }
     __syncthreads();
-#pragma unroll
     for (int w = 0; w < nw; ++w) {
-        emin = min(emin, s_e[0][w]);
-        emax = max(emax, s_e[1][w]);
+        emin = min(emin, s_red[w]);
+        emax = max(emax, s_red[nw + w]);
     }
     const bool any = emin <= emax;  // some block is not zero
     if (any && emax - emin > kMaxSpread) {
         if (threadIdx.x == 0) atomicOr(wide, 1);
         return;
     }
-    int8_t* dst = xpt + (int64_t)t * kPlanes * H;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int b = i >> 5;
+        const uint32_t m = s_m[b] ? s_m[b] << (s_e[b] - emin) : 0u;
+        int c[kPlanes];
+        digits5((int)s_q[i], m, c);
 #pragma unroll
-    for (int j = 0; j < kMaxBlocksPerWarp; ++j) {
-        const int b = warp + nw * j;
-        if (b < nb) {
-            const uint32_t m = mm[j] ? mm[j] << (ee[j] - emin) : 0u;
-            int c[kPlanes];
-            digits5(qv[j], m, c);
-#pragma unroll
-            for (int pl = 0; pl < kPlanes; ++pl) dst[(int64_t)pl * H + 32 * b + lane] = (int8_t)c[pl];
-        }
+        for (int pl = 0; pl < kPlanes; ++pl) planes[(int64_t)pl * n + i] = (int8_t)c[pl];
     }
-    if (threadIdx.x == 0) pet[t] = any ? ldexp(1.0, emin) : 0.0;
+    if (threadIdx.x == 0) *pe = any ? ldexp(1.0, emin) : 0.0;
+}
+
+// Q8_0 of x, one CTA per token (as k_quantize_q8_0: one warp per block of 32,
+// lane = element), and the token's digit planes [5][hidden] with its 2^E
+// (see kPlanes); a token too wide for the planes sets *wide (the call then
+// takes the fp64-epilogue GEMMs).
+__global__ void __launch_bounds__(kQuantThreads) k_tc_quantize(const float* __restrict__ x, int H,
+                                                               int8_t* __restrict__ xq, float* __restrict__ xd,
+                                                               int8_t* __restrict__ xpt, double* __restrict__ pet,
+                                                               int* wide) {
+    __shared__ int8_t s_q[kMaxQuantCols];
+    __shared__ uint32_t s_m[kMaxQuantCols / 32];
+    __shared__ int s_e[kMaxQuantCols / 32];
+    __shared__ int s_red[2 * kQuantThreads / 32];
+    const int t = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nb = H / 32, nw = kQuantThreads / 32;
+    const float* xt = x + (int64_t)t * H;
+    float v = warp < nb ? __ldg(xt + 32 * warp + lane) : 0.f;
+    for (int b = warp; b < nb; b += nw) {
+        const float vn = b + nw < nb ? __ldg(xt + 32 * (b + nw) + lane) : 0.f;  // the next block's load in flight
+        int8_t q;
+        float d;
+        q8_0_warp(v, q, d);
+        xq[(int64_t)t * H + 32 * b + lane] = q;
+        s_q[32 * b + lane] = q;
+        if (lane == 0) {
+            xd[(int64_t)t * nb + b] = d;
+            f32_mant_exp(d, s_m[b], s_e[b]);
+        }
+        v = vn;
+    }
+    __syncthreads();
+    row_planes(s_q, s_m, s_e, H, s_red, xpt + (int64_t)t * kPlanes * H, pet + t, wide);
 }
 
 // One warp per padded row: its token's digit planes and 2^E (zeros for a
@@ -1135,95 +1143,55 @@ __global__ void __launch_bounds__(kDpThreads, 1)
 // and rounded to fp32, then Q8_0; the codes and scales go to the slot's h
 // (hq, hd), to the row's codes and transposed fp64 scales (hg, hdT: the
 // fp64-epilogue GEMM's operands) and, as in k_tc_quantize, to the row's
-// digit planes [5][inter] with 2^E in peh (a row whose exponents spread over
-// more than kMaxSpread sets *wide instead).  Padding rows: zero planes and
-// scales.
+// digit planes [5][inter] with 2^E in peh (a row too wide for the planes
+// sets *wide).  Padding rows: zero planes and scales.
 __global__ void __launch_bounds__(kQuantThreads) k_tc_swiglu(const float* __restrict__ gu, int I, int prows_cap,
                                                              const int32_t* __restrict__ row_slot,
                                                              const int32_t* __restrict__ ctrl, int8_t* __restrict__ hg,
                                                              double* __restrict__ hdT, int8_t* __restrict__ hq,
                                                              float* __restrict__ hd, int8_t* __restrict__ hp,
                                                              double* __restrict__ peh, int* wide) {
-    __shared__ int s_e[2][kQuantThreads / 32];
+    __shared__ int8_t s_q[kMaxQuantCols];
+    __shared__ uint32_t s_m[kMaxQuantCols / 32];
+    __shared__ int s_e[kMaxQuantCols / 32];
+    __shared__ int s_red[2 * kQuantThreads / 32];
     const int q = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (q >= ctrl[2]) return;
     const int nbI = I / 32, nw = kQuantThreads / 32;
     const int slot = row_slot[q];
     int8_t* dst = hp + (int64_t)q * kPlanes * I;
     if (slot < 0) {  // a padding row
-        for (int b = warp; b < nbI; b += nw) {
-            if (lane == 0) hdT[(int64_t)b * prows_cap + q] = 0.0;
-#pragma unroll
-            for (int pl = 0; pl < kPlanes; ++pl) dst[(int64_t)pl * I + 32 * b + lane] = 0;
-        }
+        for (int b = threadIdx.x; b < nbI; b += kQuantThreads) hdT[(int64_t)b * prows_cap + q] = 0.0;
+        for (int i = threadIdx.x; i < kPlanes * I; i += kQuantThreads) dst[i] = 0;
         if (threadIdx.x == 0) peh[q] = 0.0;
         return;
     }
-    float g[kMaxBlocksPerWarp], u[kMaxBlocksPerWarp];
-#pragma unroll
-    for (int j = 0; j < kMaxBlocksPerWarp; ++j) {
-        const int b = warp + nw * j;
-        g[j] = b < nbI ? gu[(int64_t)q * I + 32 * b + lane] : 0.f;
-        u[j] = b < nbI ? gu[((int64_t)prows_cap + q) * I + 32 * b + lane] : 0.f;
-    }
-    int qv[kMaxBlocksPerWarp];
-    uint32_t mm[kMaxBlocksPerWarp];
-    int ee[kMaxBlocksPerWarp];
-    int emin = 0x7FFFFFFF, emax = -0x7FFFFFFF;
-#pragma unroll
-    for (int j = 0; j < kMaxBlocksPerWarp; ++j) {
-        const int b = warp + nw * j;
-        qv[j] = 0;
-        mm[j] = 0u;
-        ee[j] = 0;
-        if (b < nbI) {  // the same in the whole warp
-            const int i = 32 * b + lane;
-            const double gd = (double)g[j];
-            const float h = __double2float_rn(__dmul_rn(__ddiv_rn(gd, __dadd_rn(1.0, exp(-gd))), (double)u[j]));
-            int8_t qq;
-            float d;
-            q8_0_warp(h, qq, d);
-            hg[(int64_t)q * I + i] = qq;
-            hq[(int64_t)slot * I + i] = qq;
-            if (lane == 0) {
-                hdT[(int64_t)b * prows_cap + q] = (double)d;
-                hd[(int64_t)slot * nbI + b] = d;
-            }
-            qv[j] = qq;
-            f32_mant_exp(d, mm[j], ee[j]);
-            if (mm[j]) {
-                emin = min(emin, ee[j]);
-                emax = max(emax, ee[j]);
-            }
+    const float* gr = gu + (int64_t)q * I;
+    const float* ur = gu + ((int64_t)prows_cap + q) * I;
+    float g = warp < nbI ? gr[32 * warp + lane] : 0.f, u = warp < nbI ? ur[32 * warp + lane] : 0.f;
+    for (int b = warp; b < nbI; b += nw) {
+        // the next block's loads in flight while this one is computed
+        const bool nx = b + nw < nbI;
+        const float gn = nx ? gr[32 * (b + nw) + lane] : 0.f, un = nx ? ur[32 * (b + nw) + lane] : 0.f;
+        const int i = 32 * b + lane;
+        const double gd = (double)g;
+        const float h = __double2float_rn(__dmul_rn(__ddiv_rn(gd, __dadd_rn(1.0, exp(-gd))), (double)u));
+        int8_t qq;
+        float d;
+        q8_0_warp(h, qq, d);
+        hg[(int64_t)q * I + i] = qq;
+        hq[(int64_t)slot * I + i] = qq;
+        s_q[i] = qq;
+        if (lane == 0) {
+            hdT[(int64_t)b * prows_cap + q] = (double)d;
+            hd[(int64_t)slot * nbI + b] = d;
+            f32_mant_exp(d, s_m[b], s_e[b]);
         }
-    }
-    if (lane == 0) {
-        s_e[0][warp] = emin;
-        s_e[1][warp] = emax;
+        g = gn;
+        u = un;
     }
     __syncthreads();
-#pragma unroll
-    for (int w = 0; w < nw; ++w) {
-        emin = min(emin, s_e[0][w]);
-        emax = max(emax, s_e[1][w]);
-    }
-    const bool any = emin <= emax;
-    if (any && emax - emin > kMaxSpread) {
-        if (threadIdx.x == 0) atomicOr(wide, 1);
-        return;
-    }
-#pragma unroll
-    for (int j = 0; j < kMaxBlocksPerWarp; ++j) {
-        const int b = warp + nw * j;
-        if (b < nbI) {
-            const uint32_t m = mm[j] ? mm[j] << (ee[j] - emin) : 0u;
-            int c[kPlanes];
-            digits5(qv[j], m, c);
-#pragma unroll
-            for (int pl = 0; pl < kPlanes; ++pl) dst[(int64_t)pl * I + 32 * b + lane] = (int8_t)c[pl];
-        }
-    }
-    if (threadIdx.x == 0) peh[q] = any ? ldexp(1.0, emin) : 0.0;
+    row_planes(s_q, s_m, s_e, I, s_red, dst, peh + q, wide);
 }
 
 }  // namespace tc
@@ -1234,9 +1202,8 @@ __global__ void __launch_bounds__(kQuantThreads) k_tc_swiglu(const float* __rest
 bool tc_path_supported(const moe_config& c, int T) {
     if (T < kTcMinTokens) return false;
     if (c.hidden % tc::kTileRows || c.inter % tc::kTileRows) return false;
-    // one CTA of the quantisers holds a row's blocks in registers
-    const int max_cols = tc::kMaxBlocksPerWarp * (tc::kQuantThreads / 32) * 32;
-    if (c.hidden > max_cols || c.inter > max_cols) return false;
+    // the quantisers hold a row's codes in shared memory
+    if (c.hidden > tc::kMaxQuantCols || c.inter > tc::kMaxQuantCols) return false;
     return c.wbits == 8 || c.wbits == 4 || c.wbits == 2;
 }
 

@@ -77,7 +77,7 @@ _SIGS = {
 PROFILE_MAX_EVENTS = 8
 # launches of one forward on each path (moe_forward_launches): fused small
 # batch, multi-kernel, batched tensor-core
-SMALL_LAUNCHES, MULTI_KERNEL_LAUNCHES, TC_LAUNCHES = 1, 7, 12
+SMALL_LAUNCHES, MULTI_KERNEL_LAUNCHES, TC_LAUNCHES = 1, 7, 13
 
 _LIB = None
 
