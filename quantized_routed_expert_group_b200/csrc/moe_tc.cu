@@ -856,7 +856,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // is formed exactly in int64 (a double while it stays below 2^53), and the
 // output is fp32(s_row * acc) in fp64, as the oracle rounds it.
 // warps 0-3  epilogue (warp w: TMEM lanes 32 w .. 32 w + 31 = its 32 rows)
-// warps 4-7  widening of packed int4 / int2 staging rows (one row per thread)
+// warps 4-7  widening of packed int4 / int2 staging rows (one row per thread;
+//            codes at the top of their bytes, see widen_row_top)
 // warp 8     producer: units from a global counter, TMA per stage of the
 //            weight rows and of the chunk's planes (box of 80, 160 or 240 rows)
 // warp 9     MMA: two accumulators of 256 TMEM columns, alternating units
@@ -1054,7 +1055,7 @@ __global__ void __launch_bounds__(kDpThreads, 1)
                 if (meta[3 * s] < 0) break;
                 uint8_t* st = stage(s);
 #pragma unroll
-                for (int r = r0; r < kTileRows; r += 32 * kDpConvWarps) widen_row<WBITS>(st + L::kRaw, st + L::kA, r);
+                for (int r = r0; r < kTileRows; r += 32 * kDpConvWarps) widen_row_top<WBITS>(st + L::kRaw, st + L::kA, r);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&conv[s]);
@@ -1118,7 +1119,9 @@ __global__ void __launch_bounds__(kDpThreads, 1)
                                         ((int64_t)(int)v[kPlanes * c + 2] << 16) +
                                         ((int64_t)(int)v[kPlanes * c + 3] << 24) +
                                         ((int64_t)(int)v[kPlanes * c + 4] << 32);
-                    const double accd = __dmul_rn(__ll2double_rn(sum), pe);
+                    // every plane's dot is 2^kWidenShift times the exact one (the weights
+                    // were widened to the top of their bytes): an exact shift, then 2^E
+                    const double accd = __dmul_rn(__ll2double_rn(sum >> kWidenShift<WBITS>), pe);
                     const float val = __double2float_rn(__dmul_rn(sr, accd));
                     if (p.mode == 0) {
                         p.gu[((int64_t)(up ? p.prows_cap : 0) + u.prow0 + tk) * p.I + r] = val;
