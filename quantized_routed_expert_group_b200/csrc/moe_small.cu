@@ -76,6 +76,7 @@ constexpr int kScaleWin = 160;     // 16-byte aligned window over <= 32 fp32 sca
 constexpr int kMaxEntryWords = 5;  // ready bitmask words (entries <= 160)
 constexpr int kRouterRound = 4;    // router rows a CTA computes at a time
 constexpr int kMaxKeptFast = 4;    // kept groups of the groups-of-32 selection
+constexpr double kDownCost = 1.5;  // one token: time of a down byte over a gate/up byte (see owned_rows)
 constexpr uint64_t kFcMarkerValue = 0x3130646573756646ull;
 // Thread layout of the gate/up and down chunks: the 64 threads of a warp
 // pair (w, w+1) split the columns (K blocks c, c + 64, ...), the 4 warp pairs
@@ -1600,9 +1601,12 @@ __device__ __forceinline__ void do_combine(const SmallParams& p, const SmemPtrs&
 // Output rows [r0, r1) that CTA c owns in the down projection and combine.
 // More than one token: an even split.  One token: the gate/up units go round
 // robin (unit u to CTA u mod grid), so the first n1 = units mod grid CTAs
-// stream one unit more; they own fewer rows, so that every CTA streams the
-// same bytes (gate/up units + its rows of every entry's down matrix), as far
-// as the row cap allows.  Every CTA computes the same split.
+// stream one unit more; they own fewer rows, so that every CTA spends about
+// the same time (gate/up units + its rows of every entry's down matrix), as
+// far as the row cap allows.  A down byte counts kDownCost times a gate/up
+// byte: measured per SM, down chunks stream at about two thirds of the
+// gate/up chunks' rate (~37 vs ~54 GB/s at one token).  Every CTA computes
+// the same split.
 __device__ __forceinline__ void owned_rows(const SmallParams& p, int n_entries, int c, int grid, int& r0, int& r1) {
     const int H = p.H;
     if (p.T > 1 || n_entries <= 0) {
@@ -1612,13 +1616,19 @@ __device__ __forceinline__ void owned_rows(const SmallParams& p, int n_entries, 
     }
     const int n_units = n_entries * p.g.nu;
     const int n1 = n_units % grid;
-    // a unit's bytes in rows of every entry's down matrix
-    const double unit_rows = (double)(2 * kUnit * p.H) / (double)(n_entries * p.I);
+    // a unit's time in rows of every entry's down matrix
+    const double unit_rows = (double)(2 * kUnit * p.H) / (double)(n_entries * p.I) / kDownCost;
     double a = ((double)H - (double)(grid - n1) * unit_rows) / (double)grid;  // rows of a CTA with one more unit
     a = fmax(a, 0.0);
     double b = n1 < grid ? ((double)H - (double)n1 * a) / (double)(grid - n1) : a;
-    const double cap = (double)p.g.rpc;
-    if (b > cap) {  // the cap binds: even split instead
+    // at most one down chunk per entry (a second, short chunk costs more
+    // than its rows): the CTAs with fewer units take at most rd rows
+    const double cap = (double)min(p.g.rpc, p.g.rd);
+    if (b > cap && n1 > 0) {
+        b = cap;
+        a = ((double)H - (double)(grid - n1) * b) / (double)n1;
+    }
+    if (a > cap || b > cap) {  // the cap binds on both: even split instead
         r0 = (int)((int64_t)H * c / grid);
         r1 = (int)((int64_t)H * (c + 1) / grid);
         return;
