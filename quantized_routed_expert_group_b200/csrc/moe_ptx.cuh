@@ -82,6 +82,25 @@ __device__ __forceinline__ bool mbar_wait_ns(uint64_t* bar, uint32_t parity, uin
     }
 }
 
+// Bounded wait for a phase that is due within a few hundred cycles (a
+// pipeline stage): each try_wait lets the thread be suspended for at most
+// 32 ns, so that it resumes promptly once the phase completes; the global
+// timer is read every 256 tries.
+__device__ __forceinline__ bool mbar_wait_short(uint64_t* bar, uint32_t parity, uint64_t budget_ns) {
+    uint64_t t0 = 0;
+    for (uint32_t i = 0;; ++i) {
+        if (mbar_try_wait_sleep(bar, parity, 32u)) return true;
+        if ((i & 255u) == 0) {
+            const uint64_t t = global_timer_ns();
+            if (i == 0) {
+                t0 = t;
+            } else if (t - t0 > budget_ns) {
+                return false;
+            }
+        }
+    }
+}
+
 // L2 policy for data read once per call (expert weights): evict first.
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
     uint64_t pol;

@@ -856,14 +856,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // is formed exactly in int64 (a double while it stays below 2^53), and the
 // output is fp32(s_row * acc) in fp64, as the oracle rounds it.
 // warps 0-3  epilogue (warp w: TMEM lanes 32 w .. 32 w + 31 = its 32 rows)
-// warps 4-7  widening of packed int4 / int2 staging rows (one row per thread;
-//            codes at the top of their bytes, see widen_row_top)
-// warp 8     producer: units from a global counter, TMA per stage of the
-//            weight rows and of the chunk's planes (box of 80, 160 or 240 rows)
-// warp 9     MMA: two accumulators of 256 TMEM columns, alternating units
+// warps 4-7  widening of the packed int4 / int2 staging rows (one row per
+//            thread; codes at the top of their bytes, see widen_row_top)
+// warp 8     producer: TMA per stage of the weight rows and of the chunk's
+//            planes (box of 80, 160 or 240 rows)
+// warp 9     MMA: two accumulators of 256 TMEM columns, alternating units;
+//            its stage waits suspend for at most 32 ns at a time
+//            (mbar_wait_short): with the default suspend the tensor pipe sat
+//            idle long after a stage's operands had landed
 // Every wait is bounded by the global timer and records kErrTimeout.
 constexpr int kDpEpiWarps = 4;
 constexpr int kDpConvWarps = 4;
+constexpr int kDpWidenParts = kDpConvWarps * 32 / kTileRows;  // threads per widened row
+static_assert(kDpWidenParts * kTileRows == kDpConvWarps * 32, "whole rows per widening pass");
 constexpr int kDpProdWarp = kDpEpiWarps + kDpConvWarps;
 constexpr int kDpMmaWarp = kDpProdWarp + 1;
 constexpr int kDpThreads = (kDpMmaWarp + 1) * 32;
@@ -883,7 +888,7 @@ struct DpSmem {
     static constexpr uint32_t kWeightTx = (uint32_t)(kTileRows * raw_row_bytes<WBITS>());
 };
 
-// Unit counter value -> padded-row group of 16 (1..3): which plane map
+// Tokens of a unit -> groups of 16 (1..3): which plane map, and N / 80
 __device__ __forceinline__ int nt_groups(int ntok) { return (ntok + 15) >> 4; }
 
 template <int WBITS>
@@ -901,12 +906,9 @@ __global__ void __launch_bounds__(kDpThreads, 1)
     uint64_t* full = reinterpret_cast<uint64_t*>(ctl);
     uint64_t* conv = full + S;
     uint64_t* empty = conv + S;
-    uint64_t* accf = empty + S;   // [2] the accumulator's unit is complete (MMA commit)
-    uint64_t* acce = accf + 2;    // [2] the epilogue has read the accumulator
-    uint64_t* uready = acce + 2;  // [2] the accumulator's next unit id is in unit_of
-    int* meta = reinterpret_cast<int*>(uready + 2);  // [S][3]: unit (-1: end), stage of the unit, its tokens
-    int* unit_of = meta + 3 * S;                      // [2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(unit_of + 2);
+    uint64_t* accf = empty + S;  // [2] the accumulator's unit is complete (MMA commit)
+    uint64_t* acce = accf + 2;   // [2] the epilogue has read the accumulator
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
     auto stage = [&](int s) { return sm + s * L::kStageBytes; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -919,7 +921,6 @@ __global__ void __launch_bounds__(kDpThreads, 1)
         for (int a = 0; a < 2; ++a) {
             mbar_init(&accf[a], 1);
             mbar_init(&acce[a], kDpEpiWarps);
-            mbar_init(&uready[a], 1);
         }
         fence_barrier_init();
     }
@@ -931,11 +932,17 @@ __global__ void __launch_bounds__(kDpThreads, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    // Units are dealt round-robin: this CTA's are blockIdx.x, + gridDim.x, ...
+    // Every unit is nstage stages of the same work, so the deal is as even as
+    // a counter's, and each role walks the sequence on its own (no hand-over
+    // of unit ids, no atomics).
     const int n_units = p.ctrl[p.n_units_idx];
+    const int u0 = blockIdx.x, du = gridDim.x;
+    const int my_units = u0 < n_units ? (n_units - 1 - u0) / du + 1 : 0;
 
     if (warp == kDpProdWarp) {
         // ---------------- producer ----------------
-        if (lane == 0) {
+        if (lane == 0 && my_units > 0) {
             tma_prefetch_map(&w_r0);
             tma_prefetch_map(&w_r1);
             tma_prefetch_map(&w_s0);
@@ -945,117 +952,97 @@ __global__ void __launch_bounds__(kDpThreads, 1)
             tma_prefetch_map(&b48);
             int s = 0;
             uint32_t ph = 0;
-            // units come from the global counter one unit ahead: the next
-            // unit's id and description are requested when the current one
-            // starts, so that neither round trip stalls the stage sequence
-            int unit = atomicAdd(p.counter, 1), kstep = 0;
-            TcUnit u = unit < n_units ? p.units[unit] : TcUnit{0, 0, 0, 0};
-            int next = unit < n_units ? atomicAdd(p.counter, 1) : n_units;
-            TcUnit nu_ = next < n_units ? p.units[next] : TcUnit{0, 0, 0, 0};
-            while (true) {
-                if (!mbar_wait_ns(&empty[s], ph ^ 1u, kGemmWaitNs)) {
-                    set_error(p.err, kErrTimeout);
-                    break;
-                }
-                if (unit >= n_units) {
-                    meta[3 * s] = -1;
-                    meta[3 * s + 1] = 0;
-                    meta[3 * s + 2] = 0;
-                    mbar_arrive(&full[s]);
-                    break;
-                }
-                meta[3 * s] = unit;
-                meta[3 * s + 1] = kstep;
-                meta[3 * s + 2] = u.ntok;
+            bool ok = true;
+            TcUnit u = p.units[u0];
+            for (int unit = u0; ok && unit < n_units; unit += du) {
+                // the next unit's description is in flight during this one
+                const TcUnit un = unit + du < n_units ? p.units[unit + du] : u;
                 const int ng = nt_groups(u.ntok);
-                mbar_arrive_expect_tx(&full[s], L::kWeightTx + (uint32_t)(kPlanes * 16 * ng * kStageK));
-                uint8_t* st = stage(s);
+                const uint32_t tx = L::kWeightTx + (uint32_t)(kPlanes * 16 * ng * kStageK);
                 const bool sh = (u.info & kUnitShared) != 0, up = (u.info & kUnitUp) != 0;
                 const CUtensorMap* wm = sh ? (up ? &w_s1 : &w_s0) : (up ? &w_r1 : &w_r0);
-                tma_load_2d(WBITS == 8 ? st + L::kA : st + L::kRaw, wm, kstep * raw_row_bytes<WBITS>(), u.wrow0,
-                            &full[s]);
                 const CUtensorMap* bm = ng == 1 ? &b16 : ng == 2 ? &b32 : &b48;
-                tma_load_2d(st + L::kB, bm, kstep * kStageK, u.prow0 * kPlanes, &full[s]);
-                if (++kstep == p.nstage) {
-                    kstep = 0;
-                    unit = next;
-                    u = nu_;
-                    next = unit < n_units ? atomicAdd(p.counter, 1) : n_units;
-                    if (next < n_units) nu_ = p.units[next];
+                for (int kstep = 0; kstep < p.nstage; ++kstep) {
+                    if (!mbar_wait_ns(&empty[s], ph ^ 1u, kGemmWaitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[s], tx);
+                    uint8_t* st = stage(s);
+                    tma_load_2d(WBITS == 8 ? st + L::kA : st + L::kRaw, wm, kstep * raw_row_bytes<WBITS>(), u.wrow0,
+                                &full[s]);
+                    tma_load_2d(st + L::kB, bm, kstep * kStageK, u.prow0 * kPlanes, &full[s]);
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
-                if (++s == S) {
-                    s = 0;
-                    ph ^= 1u;
-                }
+                u = un;
             }
+            if (!ok) set_error(p.err, kErrTimeout);
         }
         __syncwarp();
     } else if (warp == kDpMmaWarp) {
         // ---------------- MMA issuer ----------------
-        if (lane == 0) {
-            int s = 0, cur = -1, nu = -1;
-            uint32_t ph = 0, idesc = 0, acc = 0;
+        if (lane == 0 && my_units > 0) {
+            int s = 0;
+            uint32_t ph = 0;
             bool ok = true;
-            while (ok) {
-                if (!mbar_wait_ns(&full[s], ph, kGemmWaitNs)) {
-                    set_error(p.err, kErrTimeout);
+            int ntok = p.units[u0].ntok;
+            for (int unit = u0, nu = 0; ok && unit < n_units; unit += du, ++nu) {
+                const int ntok_next = unit + du < n_units ? p.units[unit + du].ntok : 0;
+                // the unit takes the next accumulator once the epilogue has
+                // read that accumulator's previous unit
+                const int buf = nu & 1;
+                if (nu >= 2 && !mbar_wait_short(&acce[buf], ((nu >> 1) - 1) & 1, kGemmWaitNs)) {
+                    ok = false;
                     break;
                 }
-                const int unit = meta[3 * s];
-                const int kstep = meta[3 * s + 1];
-                if (unit < 0 || unit != cur) {
-                    // a new unit (or the end) takes the next accumulator, once
-                    // the epilogue has read that accumulator's previous unit;
-                    // the epilogue learns the unit id through unit_of
-                    ++nu;
-                    const int buf = nu & 1;
-                    if (nu >= 2 && !mbar_wait_ns(&acce[buf], ((nu >> 1) - 1) & 1, kGemmWaitNs)) {
-                        set_error(p.err, kErrTimeout);
+                const uint32_t idesc = idesc_i8(kPlanes * 16 * nt_groups(ntok));
+                const uint32_t acc = tmem + (uint32_t)(buf * kDpAccCols);
+                for (int kstep = 0; kstep < p.nstage; ++kstep) {
+                    if (!mbar_wait_short(&full[s], ph, kGemmWaitNs) ||
+                        (WBITS != 8 && !mbar_wait_short(&conv[s], ph, kGemmWaitNs))) {
+                        ok = false;
                         break;
                     }
-                    unit_of[buf] = unit;
-                    mbar_arrive(&uready[buf]);
-                    if (unit < 0) break;
-                    cur = unit;
-                    idesc = idesc_i8(kPlanes * 16 * nt_groups(meta[3 * s + 2]));
-                    acc = tmem + (uint32_t)(buf * kDpAccCols);
-                }
-                if (WBITS != 8 && !mbar_wait_ns(&conv[s], ph, kGemmWaitNs)) {
-                    set_error(p.err, kErrTimeout);
-                    break;
-                }
-                tc_fence_after_sync();
-                uint8_t* st = stage(s);
-                const uint64_t bdsc = desc_k128_sw128(st + L::kB);
-                const uint64_t adsc = desc_k128_sw128(st + L::kA);
+                    tc_fence_after_sync();
+                    uint8_t* st = stage(s);
+                    const uint64_t bdsc = desc_k128_sw128(st + L::kB);
+                    const uint64_t adsc = desc_k128_sw128(st + L::kA);
 #pragma unroll
-                for (int j = 0; j < kBlocksPerStage; ++j)
-                    if (kstep * kBlocksPerStage + j < p.nbK)
-                        mma_i8(acc, adsc + 2 * j, bdsc + 2 * j, idesc, kstep > 0 || j > 0);
-                mma_commit(&empty[s]);
-                if (kstep == p.nstage - 1) mma_commit(&accf[nu & 1]);
-                if (++s == S) {
-                    s = 0;
-                    ph ^= 1u;
+                    for (int j = 0; j < kBlocksPerStage; ++j)
+                        if (kstep * kBlocksPerStage + j < p.nbK)
+                            mma_i8(acc, adsc + 2 * j, bdsc + 2 * j, idesc, kstep > 0 || j > 0);
+                    mma_commit(&empty[s]);
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
+                if (!ok) break;
+                mma_commit(&accf[buf]);
+                ntok = ntok_next;
             }
+            if (!ok) set_error(p.err, kErrTimeout);
         }
         __syncwarp();
     } else if (warp >= kDpEpiWarps) {
         // ---------------- widening ----------------
         if constexpr (WBITS != 8) {
-            const int r0 = threadIdx.x - kDpEpiWarps * 32;  // rows r0, r0 + 32 kDpConvWarps, ... of the tile
+            // thread i widens part i / 128 of row i % 128 of the tile
+            const int ci = threadIdx.x - kDpEpiWarps * 32;
+            const int crow = ci % kTileRows, cpart = ci / kTileRows;
+            const int n_st = my_units * p.nstage;
             int s = 0;
             uint32_t ph = 0;
-            while (true) {
+            for (int i = 0; i < n_st; ++i) {
                 if (!mbar_wait_ns(&full[s], ph, kGemmWaitNs)) {
                     set_error(p.err, kErrTimeout);
                     break;
                 }
-                if (meta[3 * s] < 0) break;
                 uint8_t* st = stage(s);
-#pragma unroll
-                for (int r = r0; r < kTileRows; r += 32 * kDpConvWarps) widen_row_top<WBITS>(st + L::kRaw, st + L::kA, r);
+                widen_row_top<WBITS, kDpWidenParts>(st + L::kRaw, st + L::kA, crow, cpart);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&conv[s]);
@@ -1067,24 +1054,13 @@ __global__ void __launch_bounds__(kDpThreads, 1)
         }
     } else {
         // ---------------- epilogue ----------------
-        // the MMA warp hands over each accumulator's unit id (uready), then
-        // its completion (accf)
         const uint32_t tlane = (uint32_t)(32 * warp) << 16;
         const int rl = 32 * warp + lane;  // the thread's row in the tile
-        for (int nu = 0;; ++nu) {
+        for (int unit = u0, nu = 0; unit < n_units; unit += du, ++nu) {
             const int buf = nu & 1;
             const uint32_t par = (uint32_t)(nu >> 1) & 1u;
-            if (!mbar_wait_ns(&uready[buf], par, kGemmWaitNs)) {
-                set_error(p.err, kErrTimeout);
-                break;
-            }
-            const int unit = unit_of[buf];
-            if (unit < 0) break;
-            if (!mbar_wait_ns(&accf[buf], par, kGemmWaitNs)) {
-                set_error(p.err, kErrTimeout);
-                break;
-            }
-            tc_fence_after_sync();
+            // the unit's description, row scale, 2^E and (down) slots are
+            // loaded while its MMAs run; one token per lane (kChunk <= 64)
             const TcUnit u = p.units[unit];
             const int tile = u.info & 0xFFFF;
             const bool sh = (u.info & kUnitShared) != 0, up = (u.info & kUnitUp) != 0;
@@ -1092,13 +1068,16 @@ __global__ void __launch_bounds__(kDpThreads, 1)
             const double sr = (double)__ldg(sc + u.wrow0 + rl);
             const int r = tile * kTileRows + rl;  // output row of this thread
             const int ng = nt_groups(u.ntok);
-            // the chunk's 2^E and (down) slots, one token per lane (kChunk <= 64),
-            // loaded together and broadcast per token below
             const bool ina = lane < u.ntok, inb = lane + 32 < u.ntok;
             const double pea = ina ? __ldg(p.pe + u.prow0 + lane) : 0.0;
             const double peb = inb ? __ldg(p.pe + u.prow0 + lane + 32) : 0.0;
             const int sla = (p.mode == 1 && ina) ? __ldg(p.row_slot + u.prow0 + lane) : -1;
             const int slb = (p.mode == 1 && inb) ? __ldg(p.row_slot + u.prow0 + lane + 32) : -1;
+            if (!mbar_wait_ns(&accf[buf], par, kGemmWaitNs)) {
+                set_error(p.err, kErrTimeout);
+                break;
+            }
+            tc_fence_after_sync();
             for (int g = 0; g < ng; ++g) {
                 uint32_t v[kPlanes * 16];
 #pragma unroll

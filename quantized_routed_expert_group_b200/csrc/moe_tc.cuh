@@ -278,48 +278,67 @@ __device__ __forceinline__ void widen_row(const uint8_t* raw, uint8_t* tile, int
 // byte, i.e. 2^(8 - WBITS) * code as an int8 (16 code for int4, 64 code for
 // int2; int8 rows are not widened), so that only shifts, masks and byte
 // permutes are needed; the GEMM's epilogue removes the power of two exactly
-// (kWidenShift).  Same staging layouts and output layout as widen_row.
+// (kWidenShift).  Same output layout as widen_row.
 template <int WBITS>
 constexpr int kWidenShift = WBITS == 4 ? 4 : WBITS == 2 ? 6 : 0;
 
+// One 16-byte chunk c of packed row r (32 int4 or 64 int2 codes), held in
+// registers -> its 32 or 64 widened bytes of the SW128 tile.
 template <int WBITS>
-__device__ __forceinline__ void widen_row_top(const uint8_t* raw, uint8_t* tile, int r) {
+__device__ __forceinline__ void widen_chunk_regs_top(const uint4 w, uint8_t* tile, int r, int c) {
     if constexpr (WBITS == 4) {
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        uint32_t o[8];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const uint4 w = *reinterpret_cast<const uint4*>(raw + r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
-            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-            uint32_t o[8];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint32_t ev = (ww[q] << 4) & 0xF0F0F0F0u;  // elements 0, 2, 4, 6 of the word: 16 code
-                const uint32_t od = ww[q] & 0xF0F0F0F0u;         // elements 1, 3, 5, 7
-                o[2 * q] = __byte_perm(ev, od, 0x5140);
-                o[2 * q + 1] = __byte_perm(ev, od, 0x7362);
-            }
-            *reinterpret_cast<uint4*>(tile + sw128_chunk(r, 2 * c)) = make_uint4(o[0], o[1], o[2], o[3]);
-            *reinterpret_cast<uint4*>(tile + sw128_chunk(r, 2 * c + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t ev = (ww[q] << 4) & 0xF0F0F0F0u;  // elements 0, 2, 4, 6 of the word: 16 code
+            const uint32_t od = ww[q] & 0xF0F0F0F0u;         // elements 1, 3, 5, 7
+            o[2 * q] = __byte_perm(ev, od, 0x5140);
+            o[2 * q + 1] = __byte_perm(ev, od, 0x7362);
         }
+        *reinterpret_cast<uint4*>(tile + sw128_chunk(r, 2 * c)) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(tile + sw128_chunk(r, 2 * c + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
     } else if constexpr (WBITS == 2) {
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            const uint4 w = *reinterpret_cast<const uint4*>(raw + r * 32 + ((c ^ ((r >> 2) & 1)) << 4));
-            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        for (int q = 0; q < 4; ++q) {
+            uint32_t f[4];  // f[m]: field m of bytes 0..3 at the top of its byte (64 code of element 4j + m)
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t f[4];  // f[m]: field m of bytes 0..3 at the top of its byte (64 code of element 4j + m)
-#pragma unroll
-                for (int m = 0; m < 4; ++m) f[m] = (ww[q] << (6 - 2 * m)) & 0xC0C0C0C0u;
-                const uint32_t t0 = __byte_perm(f[0], f[1], 0x5140);
-                const uint32_t t1 = __byte_perm(f[2], f[3], 0x5140);
-                const uint32_t u0 = __byte_perm(f[0], f[1], 0x7362);
-                const uint32_t u1 = __byte_perm(f[2], f[3], 0x7362);
-                *reinterpret_cast<uint4*>(tile + sw128_chunk(r, 4 * c + q)) =
-                    make_uint4(__byte_perm(t0, t1, 0x5410), __byte_perm(t0, t1, 0x7632), __byte_perm(u0, u1, 0x5410),
-                               __byte_perm(u0, u1, 0x7632));
-            }
+            for (int m = 0; m < 4; ++m) f[m] = (ww[q] << (6 - 2 * m)) & 0xC0C0C0C0u;
+            const uint32_t t0 = __byte_perm(f[0], f[1], 0x5140);
+            const uint32_t t1 = __byte_perm(f[2], f[3], 0x5140);
+            const uint32_t u0 = __byte_perm(f[0], f[1], 0x7362);
+            const uint32_t u1 = __byte_perm(f[2], f[3], 0x7362);
+            *reinterpret_cast<uint4*>(tile + sw128_chunk(r, 4 * c + q)) =
+                make_uint4(__byte_perm(t0, t1, 0x5410), __byte_perm(t0, t1, 0x7632), __byte_perm(u0, u1, 0x5410),
+                           __byte_perm(u0, u1, 0x7632));
         }
     }
+}
+
+// The same from a packed staging row in shared memory, TMA-loaded with the
+// 64-byte (int4) or 32-byte (int2) swizzle, so that eight consecutive rows
+// read eight distinct bank groups.
+template <int WBITS>
+__device__ __forceinline__ void widen_chunk_top(const uint8_t* raw, uint8_t* tile, int r, int c) {
+    const uint4 w = WBITS == 4 ? *reinterpret_cast<const uint4*>(raw + r * 64 + ((c ^ ((r >> 1) & 3)) << 4))
+                               : *reinterpret_cast<const uint4*>(raw + r * 32 + ((c ^ ((r >> 2) & 1)) << 4));
+    widen_chunk_regs_top<WBITS>(w, tile, r, c);
+}
+
+// 16-byte chunks of one packed staging row.
+template <int WBITS>
+constexpr int raw_row_chunks() {
+    return kStageK * WBITS / 8 / 16;
+}
+
+// Part `part` of `PARTS` of packed row r: its raw_row_chunks / PARTS chunks.
+template <int WBITS, int PARTS>
+__device__ __forceinline__ void widen_row_top(const uint8_t* raw, uint8_t* tile, int r, int part) {
+    constexpr int kPer = raw_row_chunks<WBITS>() / PARTS;
+    static_assert(kPer * PARTS == raw_row_chunks<WBITS>(), "row parts of whole chunks");
+#pragma unroll
+    for (int c = 0; c < kPer; ++c) widen_chunk_top<WBITS>(raw, tile, r, part * kPer + c);
 }
 
 // Bytes of one packed staging row of a stage (kStageK codes).
