@@ -1792,10 +1792,17 @@ __global__ void __launch_bounds__(Roles<TM>::kThreads, 1) k_moe_small(const __gr
         uint8_t* data = s.slots + (size_t)slot * g.slot_bytes;
         uint64_t* empty = &s.empty[slot];
         if (m.kind == kItemGateUp) {
-            do_gateup<WBITS, TM>(p, s, m, data, gtid, empty);
+            // the loops are unrolled over the entry's own token count (an
+            // entry with fewer tokens than the batch does not compute the
+            // clamped copies)
+            if (TM == 1 || m.n <= 1) do_gateup<WBITS, 1>(p, s, m, data, gtid, empty);
+            else if (TM == 2 || m.n == 2) do_gateup<WBITS, TM == 1 ? 1 : 2>(p, s, m, data, gtid, empty);
+            else do_gateup<WBITS, TM>(p, s, m, data, gtid, empty);
             units = max(units, m.uc + 1);
         } else if (m.kind == kItemDown) {
-            do_down<WBITS, TM>(p, s, m, data, gtid, empty);
+            if (TM == 1 || m.n <= 1) do_down<WBITS, 1>(p, s, m, data, gtid, empty);
+            else if (TM == 2 || m.n == 2) do_down<WBITS, TM == 1 ? 1 : 2>(p, s, m, data, gtid, empty);
+            else do_down<WBITS, TM>(p, s, m, data, gtid, empty);
         } else if (m.kind == kItemSelect) {
             // always group 0's: the first item; every CTA's logits first
             if (s.misc[9]) {
