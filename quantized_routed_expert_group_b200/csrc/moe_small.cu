@@ -507,8 +507,10 @@ __device__ __forceinline__ int router_rows_in_slot(const SmallParams& p, int c, 
 // and stored to s.xq; CTA 0 also publishes xq and xd), then the CTA's router
 // logits, published to the workspace, from the rows the producer copied into
 // `rows` (ring slot 0) and, past those, rows read directly.  Ends with the
-// CTA's arrival on the router barrier.
-template <int WBITS>
+// CTA's arrival on the router barrier.  TM bounds the tokens: the loads of
+// all of a warp's x blocks, and of every token's part of x for a router job,
+// are in flight together (one round trip each, not one per token).
+template <int WBITS, int TM>
 __device__ __forceinline__ void consumers_start(const SmallParams& p, const SmemPtrs& s, const uint8_t* rows,
                                                 const CtrlSnap& snap, int tid, int nthr) {
     const int warp = tid >> 5, lane = tid & 31, nw = nthr >> 5;
@@ -518,19 +520,20 @@ __device__ __forceinline__ void consumers_start(const SmallParams& p, const Smem
     const int n_slot = router_rows_in_slot(p, c, grid);     // of which the producer copies these
     const float bias_v = tid < E ? __ldg(p.bias + tid) : 0.f;  // stored below: its load overlaps x's
     // Q8_0 of x: a warp takes 4 blocks at a time (8 lanes, a float4 each);
-    // the loads of up to 8 steps are issued before any is used
+    // the loads of up to QB steps are issued before any is used
     {
+        constexpr int QB = TM == 1 ? 8 : 6 * TM;  // steps per warp at hidden 6144: 3 (T = 1, two groups), 6 T
         const int nblk = T * nb, nstep = (nblk + 3) / 4, l8 = lane & 7;
-        for (int s0 = warp; s0 < nstep; s0 += 8 * nw) {
-            float4 v[8];
+        for (int s0 = warp; s0 < nstep; s0 += QB * nw) {
+            float4 v[QB];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < QB; ++j) {
                 const int blk = 4 * (s0 + j * nw) + (lane >> 3);
                 v[j] = blk < nblk ? __ldg(reinterpret_cast<const float4*>(p.x) + (int64_t)blk * 8 + l8)
                                   : make_float4(0.f, 0.f, 0.f, 0.f);
             }
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < QB; ++j) {
                 const int st = s0 + j * nw;
                 if (st >= nstep) break;  // the same for the whole warp
                 const int blk = 4 * st + (lane >> 3);
@@ -590,15 +593,22 @@ __device__ __forceinline__ void consumers_start(const SmallParams& p, const Smem
             } else {
                 load_router_row(p.router_w, e, E, H, w8, lane, w);
             }
-#pragma unroll 1
-            for (int t = 0; t < T; ++t) {
-                const float4* xr = reinterpret_cast<const float4*>(p.x + (int64_t)t * H) + w8 * n8;
-                DFAcc acc[4];
+            float4 xv[TM][kRouterVec];
+#pragma unroll
+            for (int t = 0; t < TM; ++t) {
+                const float4* xr = reinterpret_cast<const float4*>(p.x + (int64_t)(t < T ? t : 0) * H) + w8 * n8;
 #pragma unroll
                 for (int u = 0; u < kRouterVec; ++u) {
                     const int j = lane + 32 * u;
-                    dfacc4_add(acc, j < n8 ? __ldg(xr + j) : make_float4(0.f, 0.f, 0.f, 0.f), w[u]);
+                    xv[t][u] = (t < T && j < n8) ? __ldg(xr + j) : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
+            }
+#pragma unroll
+            for (int t = 0; t < TM; ++t) {
+                if (t >= T) break;  // the same for the whole warp
+                DFAcc acc[4];
+#pragma unroll
+                for (int u = 0; u < kRouterVec; ++u) dfacc4_add(acc, xv[t][u], w[u]);
                 double v = (acc[0].value() + acc[1].value()) + (acc[2].value() + acc[3].value());
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
@@ -1778,7 +1788,7 @@ __global__ void __launch_bounds__(Roles<TM>::kThreads, 1) k_moe_small(const __gr
     // ------------------------- consumers -------------------------
     const int group = warp / kConsumerWarps;     // consumer group
     const int gtid = tid - group * kConsumers;   // thread index inside the group
-    consumers_start<WBITS>(p, s, s.slots, snap, tid, G * kConsumers);
+    consumers_start<WBITS, TM>(p, s, s.slots, snap, tid, G * kConsumers);
     // group g takes ring slots g, g + G, ... in order
     int slot = group;
     uint32_t pf = 0;
