@@ -71,14 +71,16 @@ __global__ void __launch_bounds__(256) k_router_logits(const float* __restrict__
     }
 }
 
-// Batched logits (T >= kRouterTiledMinTokens): a tiled fp64 GEMM on the CUDA
-// cores.  CTA = 64 tokens x 64 experts x one K split; each thread keeps a
-// 4 x 4 tile of fp64 sums; x and the router rows are staged per 32-column
-// chunk in shared memory, widened to fp64 (every fp32 product is then exact
-// and every sum rounds in fp64, as the definition's).  The K splits' partial
-// sums go to parts [S][T][E] and are added in split order by
-// k_router_reduce, so the logits do not depend on the launch.
-constexpr int kRtT = 64, kRtE = 64, kRtK = 32, kRtPad = 2;
+// Batched logits (T >= kRouterTiledMinTokens): a tiled fp64 GEMM on the fp64
+// tensor cores (mma.sync m8n8k4 .f64).  CTA = 64 tokens x 64 experts x one K
+// split, 8 warps of 32 tokens x 16 experts (4 x 2 MMA tiles); x and the
+// router rows are staged per 32-column chunk in shared memory, widened to
+// fp64 (every fp32 product is then exact and every sum rounds in fp64, as
+// the definition's), the next chunk's loads in flight during the MMAs.  The
+// K splits' partial sums go to parts [S][T][E] and are added in split order
+// by k_router_reduce, so the logits do not depend on the launch.
+constexpr int kRtT = 64, kRtE = 64, kRtK = 32;
+constexpr int kRtPad = 4;  // rows of 68 doubles: the fragments' 8-byte loads hit distinct banks per half warp
 
 int router_splits(const moe_config& c, int T) {
     if (T < kRouterTiledMinTokens || c.hidden % kRtK) return 0;
@@ -88,65 +90,86 @@ int router_splits(const moe_config& c, int T) {
     return want < chunks ? want : chunks;
 }
 
+// D += A (8 x 4) x B (4 x 8) in fp64 on one warp: lane l holds A[l / 4][l % 4],
+// B[l % 4][l / 4] and D[l / 4][2 (l % 4) + j], j = 0, 1.
+__device__ __forceinline__ void dmma_8x8x4(double (&d)[2], double a, double b) {
+    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                 : "+d"(d[0]), "+d"(d[1])
+                 : "d"(a), "d"(b));
+}
+
 __global__ void __launch_bounds__(256) k_router_logits_f64(const float* __restrict__ x, int T, int H,
                                                            const float* __restrict__ Wr, int E, int chunks_per_split,
                                                            double* __restrict__ parts) {
-    __shared__ __align__(16) double xs[kRtK][kRtT + kRtPad];
-    __shared__ __align__(16) double ws[kRtK][kRtE + kRtPad];
-    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    __shared__ __align__(16) double xs[kRtK][kRtT + kRtPad];  // [k][token]
+    __shared__ __align__(16) double ws[kRtK][kRtE + kRtPad];  // [k][expert]
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, q = lane & 3;
     const int t0 = blockIdx.y * kRtT, e0 = blockIdx.x * kRtE, split = blockIdx.z;
+    const int wt = (warp & 1) * 32, we = (warp >> 1) * 16;  // the warp's tokens and experts in the tile
     const int nchunks = H / kRtK;
     const int kc0 = split * chunks_per_split;
     const int kc1 = min(nchunks, kc0 + chunks_per_split);
-    double acc[4][4];
+    double acc[4][2][2];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
-    for (int kc = kc0; kc < kc1; ++kc) {
-        // 64 rows x 32 columns of x and of the router rows: 512 float4 each
+        for (int c = 0; c < 2; ++c) acc[i][c][0] = acc[i][c][1] = 0.0;
+    // 64 rows x 32 columns of x and of the router rows per chunk: 512 float4
+    // each, two of each per thread
+    float4 xv[2], wv[2];
+    auto gload = [&](int kc) {
 #pragma unroll
-        for (int i = tid; i < 512; i += 256) {
-            const int r = i >> 3, k4 = i & 7;
+        for (int u = 0; u < 2; ++u) {
+            const int i = tid + 256 * u, r = i >> 3, k4 = i & 7;
             const int t = t0 + r, e = e0 + r;
-            const float4 xv = t < T ? __ldg(reinterpret_cast<const float4*>(x + (int64_t)t * H + kc * kRtK) + k4)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-            const float4 wv = e < E ? __ldg(reinterpret_cast<const float4*>(Wr + (int64_t)e * H + kc * kRtK) + k4)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-            xs[4 * k4 + 0][r] = (double)xv.x;
-            xs[4 * k4 + 1][r] = (double)xv.y;
-            xs[4 * k4 + 2][r] = (double)xv.z;
-            xs[4 * k4 + 3][r] = (double)xv.w;
-            ws[4 * k4 + 0][r] = (double)wv.x;
-            ws[4 * k4 + 1][r] = (double)wv.y;
-            ws[4 * k4 + 2][r] = (double)wv.z;
-            ws[4 * k4 + 3][r] = (double)wv.w;
+            xv[u] = t < T ? __ldg(reinterpret_cast<const float4*>(x + (int64_t)t * H + kc * kRtK) + k4)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+            wv[u] = e < E ? __ldg(reinterpret_cast<const float4*>(Wr + (int64_t)e * H + kc * kRtK) + k4)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    };
+    if (kc0 < kc1) gload(kc0);
+    for (int kc = kc0; kc < kc1; ++kc) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int i = tid + 256 * u, r = i >> 3, k4 = i & 7;
+            xs[4 * k4 + 0][r] = (double)xv[u].x;
+            xs[4 * k4 + 1][r] = (double)xv[u].y;
+            xs[4 * k4 + 2][r] = (double)xv[u].z;
+            xs[4 * k4 + 3][r] = (double)xv[u].w;
+            ws[4 * k4 + 0][r] = (double)wv[u].x;
+            ws[4 * k4 + 1][r] = (double)wv[u].y;
+            ws[4 * k4 + 2][r] = (double)wv[u].z;
+            ws[4 * k4 + 3][r] = (double)wv[u].w;
         }
         __syncthreads();
-#pragma unroll 8
-        for (int k = 0; k < kRtK; ++k) {
-            const double2 a01 = *reinterpret_cast<const double2*>(&xs[k][4 * ty]);
-            const double2 a23 = *reinterpret_cast<const double2*>(&xs[k][4 * ty + 2]);
-            const double2 b01 = *reinterpret_cast<const double2*>(&ws[k][4 * tx]);
-            const double2 b23 = *reinterpret_cast<const double2*>(&ws[k][4 * tx + 2]);
-            const double a[4] = {a01.x, a01.y, a23.x, a23.y};
-            const double b[4] = {b01.x, b01.y, b23.x, b23.y};
+        if (kc + 1 < kc1) gload(kc + 1);
+#pragma unroll
+        for (int k0 = 0; k0 < kRtK; k0 += 4) {
+            double a[4], b[2];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = xs[k0 + q][wt + 8 * i + g];
+#pragma unroll
+            for (int c = 0; c < 2; ++c) b[c] = ws[k0 + q][we + 8 * c + g];
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = __fma_rn(a[i], b[j], acc[i][j]);
+                for (int c = 0; c < 2; ++c) dmma_8x8x4(acc[i][c], a[i], b[c]);
         }
         __syncthreads();
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int t = t0 + 4 * ty + i;
+        const int t = t0 + wt + 8 * i + g;
         if (t >= T) continue;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int e = e0 + 4 * tx + j;
-            if (e < E) parts[((int64_t)split * T + t) * E + e] = acc[i][j];
-        }
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int e = e0 + we + 8 * c + 2 * q + j;
+                if (e < E) parts[((int64_t)split * T + t) * E + e] = acc[i][c][j];
+            }
     }
 }
 
