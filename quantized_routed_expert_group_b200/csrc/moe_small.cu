@@ -520,7 +520,10 @@ __device__ __forceinline__ void consumers_start(const SmallParams& p, const Smem
     const int n_slot = router_rows_in_slot(p, c, grid);     // of which the producer copies these
     const float bias_v = tid < E ? __ldg(p.bias + tid) : 0.f;  // stored below: its load overlaps x's
     // Q8_0 of x: a warp takes 4 blocks at a time (8 lanes, a float4 each);
-    // the loads of up to QB steps are issued before any is used
+    // the loads of up to QB steps are issued before any is used, and the
+    // steps' scales and codes (each a chain of shuffles and two exact
+    // divisions) are computed together, with no early exit, so that the
+    // chains overlap; steps past the end see zeros and store nothing
     {
         constexpr int QB = TM == 1 ? 8 : 6 * TM;  // steps per warp at hidden 6144: 3 (T = 1, two groups), 6 T
         const int nblk = T * nb, nstep = (nblk + 3) / 4, l8 = lane & 7;
@@ -532,13 +535,17 @@ __device__ __forceinline__ void consumers_start(const SmallParams& p, const Smem
                 v[j] = blk < nblk ? __ldg(reinterpret_cast<const float4*>(p.x) + (int64_t)blk * 8 + l8)
                                   : make_float4(0.f, 0.f, 0.f, 0.f);
             }
+            uint32_t qv[QB];
+            float dv[QB];
+#pragma unroll
+            for (int j = 0; j < QB; ++j) qv[j] = q8_0_octet(v[j], dv[j]);  // natural codes 4 l8 .. 4 l8 + 3
 #pragma unroll
             for (int j = 0; j < QB; ++j) {
                 const int st = s0 + j * nw;
                 if (st >= nstep) break;  // the same for the whole warp
                 const int blk = 4 * st + (lane >> 3);
-                float d;
-                const uint32_t q = q8_0_octet(v[j], d);  // natural codes 4 l8 .. 4 l8 + 3
+                const uint32_t q = qv[j];
+                const float d = dv[j];
                 // word l8 of the block in the weights' order (ActBlock layout)
                 uint32_t o;
                 if constexpr (WBITS == 4) {

@@ -855,7 +855,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 //   acc = 2^E_c (D_0 + 2^8 D_1 + 2^16 D_2 + 2^24 D_3 + 2^32 D_4)
 // is formed exactly in int64 (a double while it stays below 2^53), and the
 // output is fp32(s_row * acc) in fp64, as the oracle rounds it.
-// warps 0-3  epilogue (warp w: TMEM lanes 32 w .. 32 w + 31 = its 32 rows)
+// warps 0-3, 10-13  epilogue (warp w: TMEM lanes 32 (w % 4) .. + 31 = its 32
+//            rows; warps 0-3 take tokens 0-7 of each 16-token group, 10-13
+//            tokens 8-15)
 // warps 4-7  widening of the packed int4 / int2 staging rows (one row per
 //            thread; codes at the top of their bytes, see widen_row_top)
 // warp 8     producer: TMA per stage of the weight rows and of the chunk's
@@ -865,13 +867,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 //            (mbar_wait_short): with the default suspend the tensor pipe sat
 //            idle long after a stage's operands had landed
 // Every wait is bounded by the global timer and records kErrTimeout.
-constexpr int kDpEpiWarps = 4;
+constexpr int kDpEpiWarps = 4;  // of each of the two epilogue sets
 constexpr int kDpConvWarps = 4;
 constexpr int kDpWidenParts = kDpConvWarps * 32 / kTileRows;  // threads per widened row
 static_assert(kDpWidenParts * kTileRows == kDpConvWarps * 32, "whole rows per widening pass");
 constexpr int kDpProdWarp = kDpEpiWarps + kDpConvWarps;
 constexpr int kDpMmaWarp = kDpProdWarp + 1;
-constexpr int kDpThreads = (kDpMmaWarp + 1) * 32;
+constexpr int kDpEpiWarps2 = kDpMmaWarp + 1;  // the second epilogue set: warps 10-13
+constexpr int kDpThreads = (kDpEpiWarps2 + kDpEpiWarps) * 32;
 constexpr int kDpAccCols = 256;
 
 template <int WBITS>
@@ -920,7 +923,7 @@ __global__ void __launch_bounds__(kDpThreads, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&accf[a], 1);
-            mbar_init(&acce[a], kDpEpiWarps);
+            mbar_init(&acce[a], 2 * kDpEpiWarps);
         }
         fence_barrier_init();
     }
@@ -1027,7 +1030,7 @@ __global__ void __launch_bounds__(kDpThreads, 1)
             if (!ok) set_error(p.err, kErrTimeout);
         }
         __syncwarp();
-    } else if (warp >= kDpEpiWarps) {
+    } else if (warp >= kDpEpiWarps && warp < kDpEpiWarps + kDpConvWarps) {
         // ---------------- widening ----------------
         if constexpr (WBITS != 8) {
             // thread i widens part i / 128 of row i % 128 of the tile
@@ -1054,8 +1057,9 @@ __global__ void __launch_bounds__(kDpThreads, 1)
         }
     } else {
         // ---------------- epilogue ----------------
-        const uint32_t tlane = (uint32_t)(32 * warp) << 16;
-        const int rl = 32 * warp + lane;  // the thread's row in the tile
+        const int quad = warp & 3, part = warp >= kDpEpiWarps2 ? 1 : 0;  // TMEM lane quarter; tokens 8 part ..
+        const uint32_t tlane = (uint32_t)(32 * quad) << 16;
+        const int rl = 32 * quad + lane;  // the thread's row in the tile
         for (int unit = u0, nu = 0; unit < n_units; unit += du, ++nu) {
             const int buf = nu & 1;
             const uint32_t par = (uint32_t)(nu >> 1) & 1u;
@@ -1079,18 +1083,28 @@ __global__ void __launch_bounds__(kDpThreads, 1)
             }
             tc_fence_after_sync();
             for (int g = 0; g < ng; ++g) {
-                uint32_t v[kPlanes * 16];
+                // this set's 8 tokens of the group: accumulator columns
+                // 80 g + 40 part .. + 39 (column 5 c + p: token c's plane p)
+                if (16 * g + 8 * part >= u.ntok) break;  // the same in the whole warp
+                uint32_t v[kPlanes * 8];
+                const uint32_t col = (uint32_t)(buf * kDpAccCols + kPlanes * 16 * g + kPlanes * 8 * part);
+                {
+                    uint32_t a16[16], b16[16], c8[8];
+                    tmem_ld16(tmem + tlane + col, a16);
+                    tmem_ld16(tmem + tlane + col + 16, b16);
+                    tmem_ld8(tmem + tlane + col + 32, c8);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < kPlanes; ++i) {
-                    uint32_t w16[16];
-                    tmem_ld16(tmem + tlane + (uint32_t)(buf * kDpAccCols + kPlanes * 16 * g + 16 * i), w16);
+                    for (int k = 0; k < 16; ++k) {
+                        v[k] = a16[k];
+                        v[16 + k] = b16[k];
+                    }
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) v[16 * i + k] = w16[k];
+                    for (int k = 0; k < 8; ++k) v[32 + k] = c8[k];
                 }
-                tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    const int tk = 16 * g + c;
+                for (int c = 0; c < 8; ++c) {
+                    const int tk = 16 * g + 8 * part + c;
                     if (tk >= u.ntok) break;  // the same in the whole warp
                     const double pe = __shfl_sync(kFull, tk < 32 ? pea : peb, tk & 31);
                     const int slot = __shfl_sync(kFull, tk < 32 ? sla : slb, tk & 31);
