@@ -363,6 +363,7 @@ struct SmemPtrs {
     uint64_t* gexit;    // every consumer warp has left its loop
     uint64_t* rowsin;   // the producer's copy of the CTA's router rows into slot 0 has landed
     uint64_t* ctrl;     // the control snapshot (s.base, misc[8], misc[9]) is in shared memory
+    uint64_t* xqin;     // the selecting group has staged every token's Q8_0 codes in xq / xd
     UnitRec* urec;      // [2] the unit to finish
     SlotMeta* meta;
     float* gpart;    // [2][32][2][2][4] gate/up partial dots of a unit: [buffer][pair][gate/up][half][token]
@@ -393,6 +394,7 @@ __device__ __forceinline__ SmemPtrs carve(uint8_t* base, const SmallGeom& g) {
     s.gexit = s.gsync + 1;
     s.rowsin = s.gexit + 1;
     s.ctrl = s.rowsin + 1;
+    s.xqin = s.ctrl + 1;
     s.meta = reinterpret_cast<SlotMeta*>(base + g.o_meta);
     s.urec = reinterpret_cast<UnitRec*>(base + g.o_urec);
     s.gpart = reinterpret_cast<float*>(base + g.o_gpart);
@@ -502,6 +504,63 @@ __device__ __forceinline__ int router_rows_in_slot(const SmallParams& p, int c, 
     return min(min(n_mine, fit), kRouterRound);
 }
 
+// Every token's Q8_0 codes and scales, as the CTAs published them, into
+// shared memory in the weights' order (xq: each block's two 16-byte halves;
+// xd): all of a thread's loads are issued before its stores.  The workspace
+// was written in this call: L2 loads, after the router barrier's acquire.
+template <int WBITS, int TM>
+struct XqStage {
+    static constexpr int kPer = (TM * 192 + kConsumers - 1) / kConsumers;  // blocks a thread holds at hidden <= 6144
+    uint4 lo[kPer], hi[kPer];
+    float d[kPer];
+    __device__ __forceinline__ void load(const SmallParams& p, int tid) {
+        const int nblk = p.T * (p.H / 32);
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int blk = tid + kConsumers * i;
+            if (blk < nblk) {
+                lo[i] = __ldcg(reinterpret_cast<const uint4*>(p.xq) + 2 * blk);
+                hi[i] = __ldcg(reinterpret_cast<const uint4*>(p.xq) + 2 * blk + 1);
+                d[i] = __ldcg(p.xd + blk);
+            }
+        }
+    }
+    __device__ __forceinline__ void store(const SmallParams& p, const SmemPtrs& s, int tid) {
+        const int nb = p.H / 32, nblk = p.T * nb;
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int blk = tid + kConsumers * i;
+            if (blk < nblk) {
+                ActBlock a;
+                if constexpr (WBITS == 4) a = act_nibble_order(lo[i], hi[i]);
+                else if constexpr (WBITS == 2) a = act_crumb_order(lo[i], hi[i]);
+                else a = act_natural(lo[i], hi[i]);
+                const int t = blk / nb, b = blk - t * nb;
+                *reinterpret_cast<uint4*>(s.xq + ((size_t)(t * 2 + 0) * nb + b) * 16) =
+                    make_uint4(a.v[0], a.v[1], a.v[2], a.v[3]);
+                *reinterpret_cast<uint4*>(s.xq + ((size_t)(t * 2 + 1) * nb + b) * 16) =
+                    make_uint4(a.v[4], a.v[5], a.v[6], a.v[7]);
+                s.xd[blk] = d[i];
+            }
+        }
+        // blocks past kPer per thread (hidden above 6144): loaded and stored at once
+        for (int blk = tid + kConsumers * kPer; blk < nblk; blk += kConsumers) {
+            const uint4 l = __ldcg(reinterpret_cast<const uint4*>(p.xq) + 2 * blk);
+            const uint4 h = __ldcg(reinterpret_cast<const uint4*>(p.xq) + 2 * blk + 1);
+            ActBlock a;
+            if constexpr (WBITS == 4) a = act_nibble_order(l, h);
+            else if constexpr (WBITS == 2) a = act_crumb_order(l, h);
+            else a = act_natural(l, h);
+            const int t = blk / nb, b = blk - t * nb;
+            *reinterpret_cast<uint4*>(s.xq + ((size_t)(t * 2 + 0) * nb + b) * 16) =
+                make_uint4(a.v[0], a.v[1], a.v[2], a.v[3]);
+            *reinterpret_cast<uint4*>(s.xq + ((size_t)(t * 2 + 1) * nb + b) * 16) =
+                make_uint4(a.v[4], a.v[5], a.v[6], a.v[7]);
+            s.xd[blk] = __ldcg(p.xd + blk);
+        }
+    }
+};
+
 // The consumers' start (all G consumer groups, nthr threads, tid < nthr):
 // the Q8_0 of x (each block's codes put in the weights' order in registers
 // and stored to s.xq; CTA 0 also publishes xq and xd), then the CTA's router
@@ -519,56 +578,23 @@ __device__ __forceinline__ void consumers_start(const SmallParams& p, const Smem
     const int n_mine = c < E ? (E - 1 - c) / grid + 1 : 0;  // router rows of this CTA
     const int n_slot = router_rows_in_slot(p, c, grid);     // of which the producer copies these
     const float bias_v = tid < E ? __ldg(p.bias + tid) : 0.f;  // stored below: its load overlaps x's
-    // Q8_0 of x: a warp takes 4 blocks at a time (8 lanes, a float4 each);
-    // the loads of up to QB steps are issued before any is used, and the
-    // steps' scales and codes (each a chain of shuffles and two exact
-    // divisions) are computed together, with no early exit, so that the
-    // chains overlap; steps past the end see zeros and store nothing
+    // Q8_0 of x: the CTAs share the blocks (CTA c takes the steps of 4
+    // blocks [c S / grid, (c + 1) S / grid)) and publish the codes and scales
+    // to the workspace (xq, xd); after the router barrier every CTA stages
+    // all of them in shared memory (XqStage).  A warp takes 4 blocks at a
+    // time (8 lanes, a float4 each).
     {
-        constexpr int QB = TM == 1 ? 8 : 6 * TM;  // steps per warp at hidden 6144: 3 (T = 1, two groups), 6 T
         const int nblk = T * nb, nstep = (nblk + 3) / 4, l8 = lane & 7;
-        for (int s0 = warp; s0 < nstep; s0 += QB * nw) {
-            float4 v[QB];
-#pragma unroll
-            for (int j = 0; j < QB; ++j) {
-                const int blk = 4 * (s0 + j * nw) + (lane >> 3);
-                v[j] = blk < nblk ? __ldg(reinterpret_cast<const float4*>(p.x) + (int64_t)blk * 8 + l8)
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-            uint32_t qv[QB];
-            float dv[QB];
-#pragma unroll
-            for (int j = 0; j < QB; ++j) qv[j] = q8_0_octet(v[j], dv[j]);  // natural codes 4 l8 .. 4 l8 + 3
-#pragma unroll
-            for (int j = 0; j < QB; ++j) {
-                const int st = s0 + j * nw;
-                if (st >= nstep) break;  // the same for the whole warp
-                const int blk = 4 * st + (lane >> 3);
-                const uint32_t q = qv[j];
-                const float d = dv[j];
-                // word l8 of the block in the weights' order (ActBlock layout)
-                uint32_t o;
-                if constexpr (WBITS == 4) {
-                    const uint32_t nb2 = __shfl_xor_sync(kFull, q, 1);
-                    o = (l8 & 1) ? __byte_perm(nb2, q, 0x7531) : __byte_perm(q, nb2, 0x6420);
-                } else if constexpr (WBITS == 2) {
-                    const int qb = lane & ~3;
-                    const uint32_t w0 = __shfl_sync(kFull, q, qb), w1 = __shfl_sync(kFull, q, qb + 1);
-                    const uint32_t w2 = __shfl_sync(kFull, q, qb + 2), w3 = __shfl_sync(kFull, q, qb + 3);
-                    const uint32_t m = (uint32_t)(l8 & 3), sel = m | ((m + 4) << 4);
-                    o = __byte_perm(__byte_perm(w0, w1, sel), __byte_perm(w2, w3, sel), 0x5410);
-                } else {
-                    o = q;
-                }
-                if (blk < nblk) {
-                    const int t = blk / nb, b = blk - t * nb;
-                    reinterpret_cast<uint32_t*>(s.xq + ((size_t)(t * 2 + (l8 >> 2)) * nb + b) * 16)[l8 & 3] = o;
-                    if (l8 == 0) s.xd[blk] = d;
-                    if (c == 0) {
-                        reinterpret_cast<uint32_t*>(p.xq)[(int64_t)blk * 8 + l8] = q;
-                        if (l8 == 0) p.xd[blk] = d;
-                    }
-                }
+        const int st0 = (int)((int64_t)c * nstep / grid), st1 = (int)((int64_t)(c + 1) * nstep / grid);
+        for (int st = st0 + warp; st < st1; st += nw) {
+            const int blk = 4 * st + (lane >> 3);
+            const float4 v = blk < nblk ? __ldg(reinterpret_cast<const float4*>(p.x) + (int64_t)blk * 8 + l8)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+            float d;
+            const uint32_t q = q8_0_octet(v, d);  // natural codes 4 l8 .. 4 l8 + 3
+            if (blk < nblk) {
+                reinterpret_cast<uint32_t*>(p.xq)[(int64_t)blk * 8 + l8] = q;
+                if (l8 == 0) p.xd[blk] = d;
             }
         }
     }
@@ -610,13 +636,17 @@ __device__ __forceinline__ void consumers_start(const SmallParams& p, const Smem
                     xv[t][u] = (t < T && j < n8) ? __ldg(xr + j) : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
+            // every token's four compensated sums advance together (4 TM
+            // independent chains; each sum sees its terms in the same order)
+            DFAcc acc[TM][4];
+#pragma unroll
+            for (int u = 0; u < kRouterVec; ++u)
+#pragma unroll
+                for (int t = 0; t < TM; ++t) dfacc4_add(acc[t], xv[t][u], w[u]);
 #pragma unroll
             for (int t = 0; t < TM; ++t) {
                 if (t >= T) break;  // the same for the whole warp
-                DFAcc acc[4];
-#pragma unroll
-                for (int u = 0; u < kRouterVec; ++u) dfacc4_add(acc, xv[t][u], w[u]);
-                double v = (acc[0].value() + acc[1].value()) + (acc[2].value() + acc[3].value());
+                double v = (acc[t][0].value() + acc[t][1].value()) + (acc[t][2].value() + acc[t][3].value());
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
                 if (lane == 0) s.part[(i * 8 + w8) * 4 + t] = v;
@@ -1687,6 +1717,7 @@ __global__ void __launch_bounds__(Roles<TM>::kThreads, 1) k_moe_small(const __gr
         mbar_init(s.gexit, G * kConsumerWarps);
         mbar_init(s.rowsin, 1);
         mbar_init(s.ctrl, 1);
+        mbar_init(s.xqin, kConsumerWarps);
         fence_barrier_init();
     }
     // warp 0 reads the control region now (the values are stored to shared
@@ -1800,6 +1831,7 @@ __global__ void __launch_bounds__(Roles<TM>::kThreads, 1) k_moe_small(const __gr
     int slot = group;
     uint32_t pf = 0;
     int units = 0;  // the CTA's gate/up units, from the DONE marker (or the last unit seen)
+    bool xq_staged = false;
     while (true) {
         if (!mbar_wait_ns(&s.full[slot], pf, kSlackWaits * p.wait_ns)) {
             set_error(p.err, kErrTimeout);
@@ -1809,6 +1841,13 @@ __global__ void __launch_bounds__(Roles<TM>::kThreads, 1) k_moe_small(const __gr
         uint8_t* data = s.slots + (size_t)slot * g.slot_bytes;
         uint64_t* empty = &s.empty[slot];
         if (m.kind == kItemGateUp) {
+            if (!xq_staged) {  // the first gate/up item: the selecting group has staged xq
+                int okx = 1;
+                if (lane == 0) okx = mbar_wait_ns(s.xqin, 0, kSlackWaits * p.wait_ns) ? 1 : 0;
+                if (!__shfl_sync(kFull, okx, 0) && lane == 0) set_error(p.err, kErrTimeout);
+                __syncwarp();  // lane 0's acquire orders the other lanes' reads
+                xq_staged = true;
+            }
             // the loops are unrolled over the entry's own token count (an
             // entry with fewer tokens than the batch does not compute the
             // clamped copies)
@@ -1831,8 +1870,19 @@ __global__ void __launch_bounds__(Roles<TM>::kThreads, 1) k_moe_small(const __gr
                 s.misc[1] = 0;
                 mbar_arrive(s.routing);
             }
+            // every CTA's share of xq is published (the router barrier), and
+            // the producer is already streaming the routed experts: their
+            // latency covers this staging
+            {
+                XqStage<WBITS, TM> xs;
+                xs.load(p, gtid);
+                xs.store(p, s, gtid);
+            }
             __syncwarp();
-            if (lane == 0) mbar_arrive(empty);  // the slot was the scratch
+            if (lane == 0) {
+                mbar_arrive(s.xqin);
+                mbar_arrive(empty);  // the slot was the scratch
+            }
         } else if (m.kind == kItemSync) {
             do_sync(s, gtid, empty);
         } else if (m.kind == kItemCombine) {
