@@ -40,8 +40,10 @@
 //   The control words it shares between CTAs are never reset (see
 //   kFcMarker): each CTA reads their values before its router arrival and
 //   counts from there.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
+#include <mutex>
 
 #include "moe_device.cuh"
 #include "moe_internal.h"
@@ -77,6 +79,8 @@ constexpr int kMaxEntryWords = 5;  // ready bitmask words (entries <= 160)
 constexpr int kRouterRound = 4;    // router rows a CTA computes at a time
 constexpr int kMaxKeptFast = 4;    // kept groups of the groups-of-32 selection
 constexpr double kDownCost = 1.5;  // one token: time of a down byte over a gate/up byte (see owned_rows)
+constexpr double kSharedUnitCost = 0.6;  // one token: a shared-expert gate/up unit against a routed one
+constexpr int kOwnTab = 34;              // entry counts the down-row split is tabled for (top_k <= 33)
 constexpr uint64_t kFcMarkerValue = 0x3130646573756646ull;
 // Thread layout of the gate/up and down chunks: the 64 threads of a warp
 // pair (w, w+1) split the columns (K blocks c, c + 64, ...), the 4 warp pairs
@@ -190,6 +194,9 @@ struct SmallParams {
     int fault_entry;   // test hook: the entry whose first unit's h codes are never published (-1: none)
     int rows_bulk;     // the router matrix is 16-byte aligned: router rows by bulk copy
     SmallGeom g;
+    // one token: the down-row split's common finish time for each entry
+    // count (see owned_rows), computed on the host
+    double own_tt[kOwnTab];
 };
 
 struct SlotMeta {
@@ -1647,43 +1654,82 @@ __device__ __forceinline__ void do_combine(const SmallParams& p, const SmemPtrs&
 
 // Output rows [r0, r1) that CTA c owns in the down projection and combine.
 // More than one token: an even split.  One token: the gate/up units go round
-// robin (unit u to CTA u mod grid), so the first n1 = units mod grid CTAs
-// stream one unit more; they own fewer rows, so that every CTA spends about
-// the same time (gate/up units + its rows of every entry's down matrix), as
-// far as the row cap allows.  A down byte counts kDownCost times a gate/up
-// byte: measured per SM, down chunks stream at about two thirds of the
-// gate/up chunks' rate (~37 vs ~54 GB/s at one token).  Every CTA computes
-// the same split.
+// robin (unit u to CTA u mod grid, the shared expert's first), so the CTAs
+// stream different numbers of units after the routing; they own rows in
+// inverse measure, so that every CTA spends about the same time (its gate/up
+// units + its rows of every entry's down matrix), as far as the row cap
+// allows.  A shared-expert unit counts kSharedUnitCost of a routed one (its
+// copies are issued before the routing and have landed when the consumers
+// reach it); a down byte counts kDownCost times a gate/up byte (measured per
+// SM, down chunks stream at about two thirds of the gate/up chunks' rate).
+// With m = units - 1 = Q grid + rho and n_pre shared units (n_pre <= grid),
+// the CTAs fall into four contiguous classes:
+//   [0, min(n_pre, rho + 1))        Q routed units, one shared
+//   [.., n_pre)                     Q - 1 routed, one shared
+//   [n_pre, rho + 1)                Q + 1 routed
+//   [max(n_pre, rho + 1), grid)     Q routed
+// and a CTA of class X owns clamp((tt - w_X) unit_rows, 0, cap) rows, w_X its
+// units, tt the common finish time that makes the rows add up to H (found
+// on the host, own_tt).  Every CTA computes the same split.
+struct OwnSplit {
+    int lo[5];  // class X is CTAs [lo[X], lo[X + 1])
+    double w[4], unit_rows, cap;
+    bool even;  // an even split instead
+    __host__ __device__ OwnSplit(int H, int I, int nu, int ns, int T, int grid, int rpc, int rd, int n_entries) {
+        const int n_pre = ns ? nu : 0, n_all = n_entries * nu;
+        even = T > 1 || n_entries <= 0 || n_pre > grid || n_all <= n_pre;
+        const int Q = n_all > 0 ? (n_all - 1) / grid : 0, rho = n_all > 0 ? (n_all - 1) - Q * grid : 0;
+        lo[0] = 0;
+        lo[1] = n_pre < rho + 1 ? n_pre : rho + 1;
+        lo[2] = n_pre;
+        lo[3] = n_pre > rho + 1 ? n_pre : rho + 1;
+        lo[4] = grid;
+        w[0] = Q + kSharedUnitCost;
+        w[1] = Q - 1 + kSharedUnitCost;
+        w[2] = Q + 1;
+        w[3] = Q;
+        unit_rows = n_entries > 0 ? (double)(2 * kUnit * H) / (double)(n_entries * I) / kDownCost : 0.0;
+        cap = (double)(rpc < rd ? rpc : rd);  // one down chunk per entry at most
+        if (cap * grid < (double)H) even = true;  // the cap binds everywhere
+    }
+    __host__ __device__ double rows_of(int x, double tt) const {
+        const double r = (tt - w[x]) * unit_rows;
+        return r < 0.0 ? 0.0 : (r > cap ? cap : r);
+    }
+    __host__ __device__ double prefix(int cc, double tt) const {  // rows of CTAs [0, cc)
+        double v = 0.0;
+        for (int x = 0; x < 4; ++x) {
+            const int hi = cc < lo[x + 1] ? cc : lo[x + 1];
+            if (hi > lo[x]) v += (double)(hi - lo[x]) * rows_of(x, tt);
+        }
+        return v;
+    }
+};
+
+// The common finish time of the split (host; bisection to well below a row).
+static double own_split_tt(const OwnSplit& o, int H, int grid) {
+    if (o.even) return 0.0;
+    double t0 = o.w[1] - 1.0, t1 = o.w[2] + 1.0 + (o.unit_rows > 0.0 ? (double)H / o.unit_rows : 0.0);
+    for (int it = 0; it < 60; ++it) {
+        const double tm = 0.5 * (t0 + t1);
+        if (o.prefix(grid, tm) < (double)H) t0 = tm;
+        else t1 = tm;
+    }
+    return t1;
+}
+
 __device__ __forceinline__ void owned_rows(const SmallParams& p, int n_entries, int c, int grid, int& r0, int& r1) {
     const int H = p.H;
-    if (p.T > 1 || n_entries <= 0) {
+    const OwnSplit o(H, p.I, p.g.nu, p.ns, p.T, grid, p.g.rpc, p.g.rd, n_entries);
+    if (o.even || n_entries >= kOwnTab) {
         r0 = (int)((int64_t)H * c / grid);
         r1 = (int)((int64_t)H * (c + 1) / grid);
         return;
     }
-    const int n_units = n_entries * p.g.nu;
-    const int n1 = n_units % grid;
-    // a unit's time in rows of every entry's down matrix
-    const double unit_rows = (double)(2 * kUnit * p.H) / (double)(n_entries * p.I) / kDownCost;
-    double a = ((double)H - (double)(grid - n1) * unit_rows) / (double)grid;  // rows of a CTA with one more unit
-    a = fmax(a, 0.0);
-    double b = n1 < grid ? ((double)H - (double)n1 * a) / (double)(grid - n1) : a;
-    // at most one down chunk per entry (a second, short chunk costs more
-    // than its rows): the CTAs with fewer units take at most rd rows
-    const double cap = (double)min(p.g.rpc, p.g.rd);
-    if (b > cap && n1 > 0) {
-        b = cap;
-        a = ((double)H - (double)(grid - n1) * b) / (double)n1;
-    }
-    if (a > cap || b > cap) {  // the cap binds on both: even split instead
-        r0 = (int)((int64_t)H * c / grid);
-        r1 = (int)((int64_t)H * (c + 1) / grid);
-        return;
-    }
+    const double tt = p.own_tt[n_entries];
     auto start = [&](int cc) -> int {
         if (cc >= grid) return H;
-        const double v = cc <= n1 ? cc * a : n1 * a + (cc - n1) * b;
-        const int r = (int)floor(v + 1e-6);
+        const int r = (int)floor(o.prefix(cc, tt) + 1e-6);
         return r < H ? r : H;
     };
     r0 = start(c);
@@ -1976,6 +2022,23 @@ cudaError_t launch_small(const SmallArgs& a, cudaStream_t st) {
     p.fault_entry = g_fault_entry.load();
     p.rows_bulk = (reinterpret_cast<uintptr_t>(a.router_w) % 16 == 0) ? 1 : 0;
     p.g = small_geometry(c, a.T, device_info().sm_count);
+    {
+        // the down-row split's finish times, per entry count (one token);
+        // recomputed only when the split's inputs change
+        static std::mutex mu;
+        static int key[8] = {-1, -1, -1, -1, -1, -1, -1, -1};
+        static double tab[kOwnTab];
+        const int k8[8] = {p.H, p.I, p.g.nu, p.ns, a.T == 1 ? 1 : 2, p.g.grid, p.g.rpc, p.g.rd};
+        std::lock_guard<std::mutex> lock(mu);
+        if (!std::equal(k8, k8 + 8, key)) {
+            for (int n = 0; n < kOwnTab; ++n) {
+                const OwnSplit o(p.H, p.I, p.g.nu, p.ns, a.T, p.g.grid, p.g.rpc, p.g.rd, n);
+                tab[n] = own_split_tt(o, p.H, p.g.grid);
+            }
+            std::copy(k8, k8 + 8, key);
+        }
+        std::copy(tab, tab + kOwnTab, p.own_tt);
+    }
     if (p.g.smem_bytes > device_info().max_smem_optin) return cudaErrorInvalidConfiguration;
     const int tm = p.g.tmax;
     if (c.wbits == 4) {
