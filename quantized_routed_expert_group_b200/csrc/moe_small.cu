@@ -79,7 +79,7 @@ constexpr int kMaxEntryWords = 5;  // ready bitmask words (entries <= 160)
 constexpr int kRouterRound = 4;    // router rows a CTA computes at a time
 constexpr int kMaxKeptFast = 4;    // kept groups of the groups-of-32 selection
 constexpr double kDownCost = 1.5;  // one token: time of a down byte over a gate/up byte (see owned_rows)
-constexpr double kSharedUnitCost = 0.6;  // one token: a shared-expert gate/up unit against a routed one
+constexpr double kSharedUnitCost = 0.0;  // one token: a shared-expert gate/up unit against a routed one (measured: free)
 constexpr int kOwnTab = 34;              // entry counts the down-row split is tabled for (top_k <= 33)
 constexpr uint64_t kFcMarkerValue = 0x3130646573756646ull;
 // Thread layout of the gate/up and down chunks: the 64 threads of a warp
@@ -1658,10 +1658,12 @@ __device__ __forceinline__ void do_combine(const SmallParams& p, const SmemPtrs&
 // stream different numbers of units after the routing; they own rows in
 // inverse measure, so that every CTA spends about the same time (its gate/up
 // units + its rows of every entry's down matrix), as far as the row cap
-// allows.  A shared-expert unit counts kSharedUnitCost of a routed one (its
+// allows.  A shared-expert unit counts kSharedUnitCost of a routed one: its
 // copies are issued before the routing and have landed when the consumers
-// reach it); a down byte counts kDownCost times a gate/up byte (measured per
-// SM, down chunks stream at about two thirds of the gate/up chunks' rate).
+// reach it, which they do while the routed experts' first copies are in
+// flight (measured: weights 0, 0.3 and 0.6 gave 40.3, 40.55 and 40.6 us per
+// decode step).  A down byte counts kDownCost times a gate/up byte (measured
+// per SM, down chunks stream at about two thirds of the gate/up chunks' rate).
 // With m = units - 1 = Q grid + rho and n_pre shared units (n_pre <= grid),
 // the CTAs fall into four contiguous classes:
 //   [0, min(n_pre, rho + 1))        Q routed units, one shared
