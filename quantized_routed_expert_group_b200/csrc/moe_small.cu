@@ -569,13 +569,13 @@ struct XqStage {
 };
 
 // The consumers' start (all G consumer groups, nthr threads, tid < nthr):
-// the Q8_0 of x (each block's codes put in the weights' order in registers
-// and stored to s.xq; CTA 0 also publishes xq and xd), then the CTA's router
-// logits, published to the workspace, from the rows the producer copied into
-// `rows` (ring slot 0) and, past those, rows read directly.  Ends with the
-// CTA's arrival on the router barrier.  TM bounds the tokens: the loads of
-// all of a warp's x blocks, and of every token's part of x for a router job,
-// are in flight together (one round trip each, not one per token).
+// the Q8_0 of the CTA's share of x's blocks, published to the workspace (xq,
+// xd; every CTA stages all of them after the router barrier, XqStage), then
+// the CTA's router logits, published to the workspace, from the rows the
+// producer copied into `rows` (ring slot 0) and, past those, rows read
+// directly.  Ends with the CTA's arrival on the router barrier.  TM bounds
+// the tokens: every token's part of x for a router job is loaded together,
+// and the tokens' compensated sums advance together.
 template <int WBITS, int TM>
 __device__ __forceinline__ void consumers_start(const SmallParams& p, const SmemPtrs& s, const uint8_t* rows,
                                                 const CtrlSnap& snap, int tid, int nthr) {
