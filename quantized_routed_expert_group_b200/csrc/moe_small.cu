@@ -859,6 +859,20 @@ struct Producer {
         return i <= U && (uint32_t)ld_acquire_gpu(p.ctrl + kFcDone + i) - s.base[1 + i] >= (uint32_t)(p.g.nu * s.ent[i].n);
     }
 
+    // One poll of every entry's counter (one round trip for the warp): the
+    // entries found complete need no wait later.
+    __forceinline__ __device__ void poll_entries(int U) {
+        const bool f0 = entry_done(lane, U), f1 = entry_done(lane + 32, U), f2 = entry_done(lane + 64, U);
+        const bool f3 = entry_done(lane + 96, U), f4 = entry_done(lane + 128, U);
+        rdy0 |= __ballot_sync(kFull, f0);
+        rdy1 |= __ballot_sync(kFull, f1);
+        rdy2 |= __ballot_sync(kFull, f2);
+        rdy3 |= __ballot_sync(kFull, f3);
+        rdy4 |= __ballot_sync(kFull, f4);
+        need_proxy_fence = true;
+        __syncwarp();  // the polling lanes' acquires order the copying lanes' reads
+    }
+
     // Wait until every unit of entry e has published its h codes.  Each poll
     // reads all entries' counters at once (one round trip for the warp).
     __forceinline__ __device__ bool wait_entry(int e, int U) {
@@ -1843,6 +1857,11 @@ __global__ void __launch_bounds__(Roles<TM>::kThreads, 1) k_moe_small(const __gr
             const int n_pre_all = p.ns ? g.nu : 0;
             for (int u = c; u < n_pre_all + n_routed && !pr.aborted; u += grid) {
                 if (u < n_pre_all) continue;
+                // before the CTA's last unit: one poll of the entries' h
+                // counters, so that the first down chunks (of entries that
+                // completed in the earlier rounds) follow it without a round
+                // trip (the producer would wait for a ring slot meanwhile)
+                if (u + grid >= n_pre_all + n_routed) pr.poll_entries(U);
                 const int entry = 1 + (u - n_pre_all) / g.nu, blk = (u - n_pre_all) % g.nu;
                 const EntryInfo ei = s.ent[entry];
                 for (int ch = 0; ch < g.cpu; ++ch) pr.gateup(entry, ei, blk, ch);
