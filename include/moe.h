@@ -361,6 +361,18 @@ int moe_get_device_error(void *workspace, void *stream, int32_t *code);
  * [0, 10 s]. */
 int moe_debug_fault_injection(int withhold_entry, int64_t wait_budget_ns);
 
+/* Test export of the one-token fused forward's down-row split (no GPU work,
+ * no device needed): the output rows [starts[c], starts[c + 1]) that CTA c of
+ * a grid of `grid` CTAs owns in the down projection and the combine, for a
+ * batch of T tokens whose union holds n_entries experts (the selected ones and
+ * the shared one), as every CTA of k_moe_small computes it.  starts has
+ * grid + 1 entries (starts[grid] = hidden); the caller owns it.  *row_cap
+ * receives the per-CTA row cap of the split (0 for an even split).  Returns
+ * MOE_EINVAL for an invalid config, T outside [1, 4], n_entries outside
+ * [1, 1 + min(experts, T * top_k)], grid outside [1, 4096] or null
+ * pointers. */
+int moe_debug_down_rows(const moe_config* cfg, int T, int n_entries, int grid, int32_t* starts, int* row_cap);
+
 /* Device copy of the seeded input generator (SplitMix64, counter-based; see
  * the package's synth module): out[i] = sigma * z(seed, tid, offset + i) with z
  * the centred Irwin-Hall sum of twelve 16-bit uniforms.  Used to draw

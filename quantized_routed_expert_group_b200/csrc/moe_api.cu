@@ -577,6 +577,15 @@ MOE_API int moe_debug_fault_injection(int withhold_entry, int64_t wait_budget_ns
     return MOE_OK;
 }
 
+MOE_API int moe_debug_down_rows(const moe_config* cfg, int T, int n_entries, int grid, int32_t* starts,
+                                int* row_cap) {
+    if (check_config(cfg) != MOE_OK || !starts || !row_cap) return MOE_EINVAL;
+    const int max_ent = 1 + (cfg->n_experts < T * cfg->top_k ? cfg->n_experts : T * cfg->top_k);
+    if (T < 1 || T > 4 || n_entries < 1 || n_entries > max_ent || grid < 1 || grid > 4096) return MOE_EINVAL;
+    *row_cap = small_down_rows(*cfg, T, n_entries, grid, starts);
+    return MOE_OK;
+}
+
 MOE_API int moe_synth_normal(uint64_t seed, uint64_t tid, int64_t offset, int64_t n, float sigma, float* out,
                              void* stream) {
     if (n < 0 || offset < 0) return MOE_EINVAL;

@@ -97,6 +97,9 @@ struct ExpertArgs {
 };
 // ev (optional, 3 events): recorded after gate/up, down and combine.
 cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t s, cudaEvent_t const* ev);
+// The one-token down-row split (fused path) as every CTA computes it; returns
+// the row cap, 0 for an even split (test export).
+int small_down_rows(const moe_config& c, int T, int n_entries, int grid, int32_t* starts);
 int router_splits(const moe_config& c, int T);
 constexpr int kForwardLaunches = 7;  // quantise, logits, select, bucket, gate/up, down, combine
 // (+1 when the router logits take the split-K form: router_splits > 0)

@@ -1708,17 +1708,39 @@ struct OwnSplit {
         cap = (double)(rpc < rd ? rpc : rd);  // one down chunk per entry at most
         if (cap * grid < (double)H) even = true;  // the cap binds everywhere
     }
+    // products and sums rounded one by one, in the same order on the host
+    // (the table, the test export) and in every CTA
+    static __host__ __device__ double mul(double a, double b) {
+#ifdef __CUDA_ARCH__
+        return __dmul_rn(a, b);
+#else
+        return a * b;
+#endif
+    }
+    static __host__ __device__ double add(double a, double b) {
+#ifdef __CUDA_ARCH__
+        return __dadd_rn(a, b);
+#else
+        return a + b;
+#endif
+    }
     __host__ __device__ double rows_of(int x, double tt) const {
-        const double r = (tt - w[x]) * unit_rows;
+        const double r = mul(add(tt, -w[x]), unit_rows);
         return r < 0.0 ? 0.0 : (r > cap ? cap : r);
     }
     __host__ __device__ double prefix(int cc, double tt) const {  // rows of CTAs [0, cc)
         double v = 0.0;
         for (int x = 0; x < 4; ++x) {
             const int hi = cc < lo[x + 1] ? cc : lo[x + 1];
-            if (hi > lo[x]) v += (double)(hi - lo[x]) * rows_of(x, tt);
+            if (hi > lo[x]) v = add(v, mul((double)(hi - lo[x]), rows_of(x, tt)));
         }
         return v;
+    }
+    // first row of CTA cc (grid: H)
+    __host__ __device__ int start(int cc, int grid, int H, double tt) const {
+        if (cc >= grid) return H;
+        const int r = (int)floor(add(prefix(cc, tt), 1e-6));
+        return r < H ? r : H;
     }
 };
 
@@ -1743,13 +1765,8 @@ __device__ __forceinline__ void owned_rows(const SmallParams& p, int n_entries, 
         return;
     }
     const double tt = p.own_tt[n_entries];
-    auto start = [&](int cc) -> int {
-        if (cc >= grid) return H;
-        const int r = (int)floor(o.prefix(cc, tt) + 1e-6);
-        return r < H ? r : H;
-    };
-    r0 = start(c);
-    r1 = start(c + 1);
+    r0 = o.start(c, grid, H, tt);
+    r1 = o.start(c + 1, grid, H, tt);
 }
 
 // ---------------------------------------------------------------------------
@@ -2018,6 +2035,20 @@ static cudaError_t launch_small_t(const SmallParams& prm, cudaStream_t st) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, k_moe_small<WBITS, TM>, prm);
+}
+
+// The one-token down-row split of a grid, as every CTA computes it (test
+// export): starts[c] = the first row of CTA c, starts[grid] = hidden.
+int small_down_rows(const moe_config& c, int T, int n_entries, int grid, int32_t* starts) {
+    const SmallGeom g = small_geometry(c, T, grid);
+    const OwnSplit o(c.hidden, c.inter, g.nu, c.n_shared, T, grid, g.rpc, g.rd, n_entries);
+    if (o.even || n_entries >= kOwnTab) {
+        for (int cc = 0; cc <= grid; ++cc) starts[cc] = (int32_t)((int64_t)c.hidden * cc / grid);
+        return 0;
+    }
+    const double tt = own_split_tt(o, c.hidden, grid);
+    for (int cc = 0; cc <= grid; ++cc) starts[cc] = o.start(cc, grid, c.hidden, tt);
+    return (int)o.cap;
 }
 
 // Test hook state (moe_debug_fault_injection): read by every launch.

@@ -67,6 +67,7 @@ _SIGS = {
     "moe_noalloc_device_error": ([_vp, ctypes.POINTER(ctypes.c_int32)], _int),
     "moe_synth_normal": ([_u64, _u64, _i64, _i64, _flt, _vp, _vp], _int),
     "moe_debug_fault_injection": ([_int, _i64], _int),
+    "moe_debug_down_rows": ([ctypes.POINTER(MoeConfig), _int, _int, _int, ctypes.c_void_p, ctypes.POINTER(_int)], _int),
     "moe_profile_events": ([ctypes.POINTER(_vp), _int], _int),
     "moe_forward_launches": ([ctypes.POINTER(MoeConfig), _int], _int),
     "moe_forward_phases": ([ctypes.POINTER(MoeConfig), _int], _int),
@@ -206,6 +207,17 @@ def block_dots(packed: torch.Tensor, cols: int, wbits: int, q: torch.Tensor, str
                                           _stream(stream))
     _check(st, "block_dots")
     return out
+
+
+def debug_down_rows(cfg: MoeConfig, T: int, n_entries: int, grid: int):
+    """Test export (see moe_debug_down_rows): the first output row of each CTA of
+    the one-token fused forward's down split (grid + 1 values) and its row cap."""
+    import numpy as np
+    starts = np.zeros(grid + 1, np.int32)
+    cap = _int(0)
+    _check(lib().moe_debug_down_rows(ctypes.byref(cfg), T, n_entries, grid, starts.ctypes.data, ctypes.byref(cap)),
+           "debug_down_rows")
+    return starts, cap.value
 
 
 def debug_fault_injection(withhold_entry: int, wait_budget_ns: int = 0) -> None:
