@@ -1134,20 +1134,23 @@ __global__ void __launch_bounds__(kDpThreads, 1)
     if (warp == kDpMmaWarp) tmem_dealloc(tmem, 2 * kDpAccCols);
 }
 
-// SwiGLU and Q8_0 of h, one CTA per padded row (warp w takes the row's
-// blocks w, w + 8, ..., lane = element): h = silu(g) * u evaluated in fp64
-// and rounded to fp32, then Q8_0; the codes and scales go to the slot's h
-// (hq, hd), to the row's codes and transposed fp64 scales (hg, hdT: the
-// fp64-epilogue GEMM's operands) and, as in k_tc_quantize, to the row's
-// digit planes [5][inter] with 2^E in peh (a row too wide for the planes
-// sets *wide).  Padding rows: zero planes and scales.
+// SwiGLU and Q8_0 of h, one CTA per padded row, four consecutive elements a
+// thread (a Q8_0 block of 32 is eight lanes): h = silu(g) * u evaluated in
+// fp64 and rounded to fp32, then Q8_0 (the arithmetic of q8_0_warp, the
+// block's |h| maximum taken over its eight lanes); the codes and scales go to
+// the slot's h (hq, hd), to the row's codes and transposed fp64 scales (hg,
+// hdT: the fp64-epilogue GEMM's operands) and, as in k_tc_quantize, to the
+// row's digit planes [5][inter] with 2^E in peh (a row too wide for the
+// planes sets *wide).  The codes stay in registers between the two passes.
+// Padding rows: zero planes and scales.
+constexpr int kSwigluSpan = 4 * kQuantThreads;              // elements of the row per pass of the CTA
+constexpr int kSwigluIters = kMaxQuantCols / kSwigluSpan;   // passes at the widest row
 __global__ void __launch_bounds__(kQuantThreads) k_tc_swiglu(const float* __restrict__ gu, int I, int prows_cap,
                                                              const int32_t* __restrict__ row_slot,
                                                              const int32_t* __restrict__ ctrl, int8_t* __restrict__ hg,
                                                              double* __restrict__ hdT, int8_t* __restrict__ hq,
                                                              float* __restrict__ hd, int8_t* __restrict__ hp,
                                                              double* __restrict__ peh, int* wide) {
-    __shared__ int8_t s_q[kMaxQuantCols];
     __shared__ uint32_t s_m[kMaxQuantCols / 32];
     __shared__ int s_e[kMaxQuantCols / 32];
     __shared__ int s_red[2 * kQuantThreads / 32];
@@ -1158,27 +1161,54 @@ __global__ void __launch_bounds__(kQuantThreads) k_tc_swiglu(const float* __rest
     int8_t* dst = hp + (int64_t)q * kPlanes * I;
     if (slot < 0) {  // a padding row
         for (int b = threadIdx.x; b < nbI; b += kQuantThreads) hdT[(int64_t)b * prows_cap + q] = 0.0;
-        for (int i = threadIdx.x; i < kPlanes * I; i += kQuantThreads) dst[i] = 0;
+        uint4* d16 = reinterpret_cast<uint4*>(dst);
+        for (int i = threadIdx.x; i < kPlanes * I / 16; i += kQuantThreads) d16[i] = make_uint4(0u, 0u, 0u, 0u);
         if (threadIdx.x == 0) peh[q] = 0.0;
         return;
     }
-    const float* gr = gu + (int64_t)q * I;
-    const float* ur = gu + ((int64_t)prows_cap + q) * I;
-    float g = warp < nbI ? gr[32 * warp + lane] : 0.f, u = warp < nbI ? ur[32 * warp + lane] : 0.f;
-    for (int b = warp; b < nbI; b += nw) {
-        // the next block's loads in flight while this one is computed
-        const bool nx = b + nw < nbI;
-        const float gn = nx ? gr[32 * (b + nw) + lane] : 0.f, un = nx ? ur[32 * (b + nw) + lane] : 0.f;
-        const int i = 32 * b + lane;
-        const double gd = (double)g;
-        const float h = __double2float_rn(__dmul_rn(__ddiv_rn(gd, __dadd_rn(1.0, exp(-gd))), (double)u));
-        int8_t qq;
-        float d;
-        q8_0_warp(h, qq, d);
-        hg[(int64_t)q * I + i] = qq;
-        hq[(int64_t)slot * I + i] = qq;
-        s_q[i] = qq;
-        if (lane == 0) {
+    const float4* gr = reinterpret_cast<const float4*>(gu + (int64_t)q * I);
+    const float4* ur = reinterpret_cast<const float4*>(gu + ((int64_t)prows_cap + q) * I);
+    uint32_t codes[kSwigluIters];
+    // I is a multiple of 128, so a warp's 128 elements are all in the row or all past it
+    float4 g = 4 * threadIdx.x < I ? gr[threadIdx.x] : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 u = 4 * threadIdx.x < I ? ur[threadIdx.x] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < kSwigluIters; ++j) {
+        const int v = threadIdx.x + j * kQuantThreads, i = 4 * v;  // first element of this thread
+        if (i >= I) break;
+        // the next pass's loads in flight while this one is computed
+        const bool nx = i + kSwigluSpan < I;
+        const float4 gn = nx ? gr[v + kQuantThreads] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 un = nx ? ur[v + kQuantThreads] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float gv[4] = {g.x, g.y, g.z, g.w}, uv[4] = {u.x, u.y, u.z, u.w};
+        float h[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const double gd = (double)gv[e];
+            h[e] = __double2float_rn(__dmul_rn(__ddiv_rn(gd, __dadd_rn(1.0, exp(-gd))), (double)uv[e]));
+        }
+        // Q8_0 of the block (eight lanes): d = amax / 127, q = round-half-away(h * (1/d)) in [-127, 127]
+        float a = fmaxf(fmaxf(fabsf(h[0]), fabsf(h[1])), fmaxf(fabsf(h[2]), fabsf(h[3])));
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, o));
+        float d = 0.0f;
+        uint32_t c = 0u;
+        if (a >= FLT_MIN) {
+            d = __fdiv_rn(a, 127.0f);
+            const float id = __fdiv_rn(1.0f, d);
+            uint32_t b4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float r = fminf(fmaxf(roundf(__fmul_rn(h[e], id)), -127.0f), 127.0f);
+                b4[e] = (uint32_t)(int)r;
+            }
+            c = __byte_perm(__byte_perm(b4[0], b4[1], 0x0040), __byte_perm(b4[2], b4[3], 0x0040), 0x5410);
+        }
+        codes[j] = c;
+        *reinterpret_cast<uint32_t*>(hg + (int64_t)q * I + i) = c;
+        *reinterpret_cast<uint32_t*>(hq + (int64_t)slot * I + i) = c;
+        if ((lane & 7) == 0) {
+            const int b = i >> 5;
             hdT[(int64_t)b * prows_cap + q] = (double)d;
             hd[(int64_t)slot * nbI + b] = d;
             f32_mant_exp(d, s_m[b], s_e[b]);
@@ -1187,7 +1217,58 @@ __global__ void __launch_bounds__(kQuantThreads) k_tc_swiglu(const float* __rest
         u = un;
     }
     __syncthreads();
-    row_planes(s_q, s_m, s_e, I, s_red, dst, peh + q, wide);
+    // the row's smallest block exponent and spread (as row_planes)
+    int emin = 0x7FFFFFFF, emax = -0x7FFFFFFF;
+    for (int b = threadIdx.x; b < nbI; b += kQuantThreads)
+        if (s_m[b]) {
+            emin = min(emin, s_e[b]);
+            emax = max(emax, s_e[b]);
+        }
+    emin = __reduce_min_sync(kFull, emin);
+    emax = __reduce_max_sync(kFull, emax);
+    if (lane == 0) {
+        s_red[warp] = emin;
+        s_red[nw + warp] = emax;
+    }
+    __syncthreads();
+    for (int w = 0; w < nw; ++w) {
+        emin = min(emin, s_red[w]);
+        emax = max(emax, s_red[nw + w]);
+    }
+    const bool any = emin <= emax;  // some block is not zero
+    if (any && emax - emin > kMaxSpread) {
+        if (threadIdx.x == 0) atomicOr(wide, 1);
+        return;
+    }
+    // digits: q m + 0x8080808080 (in [0, 2^40) for |q| <= 127, m < 2^32) has
+    // the bytes c_p + 128 of the signed base-256 digits c_p of q m
+#pragma unroll
+    for (int j = 0; j < kSwigluIters; ++j) {
+        const int i = 4 * (threadIdx.x + j * kQuantThreads);
+        if (i >= I) break;
+        const int b = i >> 5;
+        const uint32_t m = s_m[b] ? s_m[b] << (s_e[b] - emin) : 0u;
+        uint32_t lo[4], hi[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int qe = (int)(int8_t)(codes[j] >> (8 * e));
+            const uint64_t t = (uint64_t)((int64_t)qe * (int64_t)m) + 0x8080808080ull;
+            lo[e] = (uint32_t)t;
+            hi[e] = (uint32_t)(t >> 32);
+        }
+        const uint32_t a01 = __byte_perm(lo[0], lo[1], 0x5140), b01 = __byte_perm(lo[0], lo[1], 0x7362);
+        const uint32_t a23 = __byte_perm(lo[2], lo[3], 0x5140), b23 = __byte_perm(lo[2], lo[3], 0x7362);
+        uint32_t pw[kPlanes];
+        pw[0] = __byte_perm(a01, a23, 0x5410);
+        pw[1] = __byte_perm(a01, a23, 0x7632);
+        pw[2] = __byte_perm(b01, b23, 0x5410);
+        pw[3] = __byte_perm(b01, b23, 0x7632);
+        pw[4] = __byte_perm(__byte_perm(hi[0], hi[1], 0x0040), __byte_perm(hi[2], hi[3], 0x0040), 0x5410);
+#pragma unroll
+        for (int pl = 0; pl < kPlanes; ++pl)
+            *reinterpret_cast<uint32_t*>(dst + (int64_t)pl * I + i) = pw[pl] ^ 0x80808080u;
+    }
+    if (threadIdx.x == 0) peh[q] = any ? ldexp(1.0, emin) : 0.0;
 }
 
 }  // namespace tc
