@@ -78,14 +78,18 @@ __global__ void __launch_bounds__(256) k_router_logits(const float* __restrict__
 // fp64 (every fp32 product is then exact and every sum rounds in fp64, as
 // the definition's), the next chunk's loads in flight during the MMAs.  The
 // K splits' partial sums go to parts [S][T][E] and are added in split order
-// by k_router_reduce, so the logits do not depend on the launch.
+// by k_router_reduce, so the logits do not depend on the launch.  The split
+// count aims at three CTAs on each of 148 SMs (the kernel is latency-bound:
+// more resident warps, not fewer chunks, shorten it).
 constexpr int kRtT = 64, kRtE = 64, kRtK = 32;
-constexpr int kRtPad = 4;  // rows of 68 doubles: the fragments' 8-byte loads hit distinct banks per half warp
+constexpr int kRtPad = 4;  // rows of 36 doubles: conflict-free fragment loads and staging stores
+constexpr int kRtTargetCtas = 3 * 148;
 
 int router_splits(const moe_config& c, int T) {
     if (T < kRouterTiledMinTokens || c.hidden % kRtK) return 0;
     const int tiles = ((T + kRtT - 1) / kRtT) * ((c.n_experts + kRtE - 1) / kRtE);
-    const int want = tiles <= 16 ? 16 : tiles <= 64 ? 8 : 4;
+    int want = kRtTargetCtas / tiles;  // never a second, partial wave
+    want = want < 1 ? 1 : want > 16 ? 16 : want;
     const int chunks = c.hidden / kRtK;
     return want < chunks ? want : chunks;
 }
@@ -101,8 +105,8 @@ __device__ __forceinline__ void dmma_8x8x4(double (&d)[2], double a, double b) {
 __global__ void __launch_bounds__(256) k_router_logits_f64(const float* __restrict__ x, int T, int H,
                                                            const float* __restrict__ Wr, int E, int chunks_per_split,
                                                            double* __restrict__ parts) {
-    __shared__ __align__(16) double xs[kRtK][kRtT + kRtPad];  // [k][token]
-    __shared__ __align__(16) double ws[kRtK][kRtE + kRtPad];  // [k][expert]
+    __shared__ __align__(16) double xs[kRtT][kRtK + kRtPad];  // [token][k]
+    __shared__ __align__(16) double ws[kRtE][kRtK + kRtPad];  // [expert][k]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, q = lane & 3;
     const int t0 = blockIdx.y * kRtT, e0 = blockIdx.x * kRtE, split = blockIdx.z;
@@ -133,15 +137,21 @@ __global__ void __launch_bounds__(256) k_router_logits_f64(const float* __restri
     for (int kc = kc0; kc < kc1; ++kc) {
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
+            // row r, columns 4 k4 .. 4 k4 + 3 as two 16-byte stores; lanes
+            // with k4 >= 4 store their upper half first, so that each
+            // store instruction of 8 lanes covers all 32 banks once
             const int i = tid + 256 * u, r = i >> 3, k4 = i & 7;
-            xs[4 * k4 + 0][r] = (double)xv[u].x;
-            xs[4 * k4 + 1][r] = (double)xv[u].y;
-            xs[4 * k4 + 2][r] = (double)xv[u].z;
-            xs[4 * k4 + 3][r] = (double)xv[u].w;
-            ws[4 * k4 + 0][r] = (double)wv[u].x;
-            ws[4 * k4 + 1][r] = (double)wv[u].y;
-            ws[4 * k4 + 2][r] = (double)wv[u].z;
-            ws[4 * k4 + 3][r] = (double)wv[u].w;
+            const bool sw = k4 >= 4;
+            double2* xr = reinterpret_cast<double2*>(&xs[r][4 * k4]);
+            double2* wr = reinterpret_cast<double2*>(&ws[r][4 * k4]);
+            const double2 xlo = make_double2((double)xv[u].x, (double)xv[u].y);
+            const double2 xhi = make_double2((double)xv[u].z, (double)xv[u].w);
+            const double2 wlo = make_double2((double)wv[u].x, (double)wv[u].y);
+            const double2 whi = make_double2((double)wv[u].z, (double)wv[u].w);
+            xr[sw ? 1 : 0] = sw ? xhi : xlo;
+            wr[sw ? 1 : 0] = sw ? whi : wlo;
+            xr[sw ? 0 : 1] = sw ? xlo : xhi;
+            wr[sw ? 0 : 1] = sw ? wlo : whi;
         }
         __syncthreads();
         if (kc + 1 < kc1) gload(kc + 1);
@@ -149,9 +159,9 @@ __global__ void __launch_bounds__(256) k_router_logits_f64(const float* __restri
         for (int k0 = 0; k0 < kRtK; k0 += 4) {
             double a[4], b[2];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] = xs[k0 + q][wt + 8 * i + g];
+            for (int i = 0; i < 4; ++i) a[i] = xs[wt + 8 * i + g][k0 + q];
 #pragma unroll
-            for (int c = 0; c < 2; ++c) b[c] = ws[k0 + q][we + 8 * c + g];
+            for (int c = 0; c < 2; ++c) b[c] = ws[we + 8 * c + g][k0 + q];
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll

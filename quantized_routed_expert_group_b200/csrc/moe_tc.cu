@@ -412,17 +412,41 @@ __global__ void __launch_bounds__(kPlanThreads) k_tc_plan(PlanParams p) {
 constexpr int kQuantThreads = 256;
 constexpr int kMaxQuantCols = 8192;  // hidden and inter of the batched path
 
-// The digit planes of one row of n codes (Q8_0 blocks of 32) from its codes
-// and block scales in shared memory: the row's smallest block exponent E
-// and spread (CTA-wide), then each thread's elements split into kPlanes
-// digits written to planes [kPlanes][n]; 2^E to *pe (0 for an all-zero row).
-// A row whose exponents spread over more than kMaxSpread sets *wide and
-// writes no planes.  Every thread of the CTA calls it.
-__device__ __forceinline__ void row_planes(const int8_t* s_q, const uint32_t* s_m, const int* s_e, int n,
-                                           int* s_red, int8_t* __restrict__ planes, double* __restrict__ pe,
-                                           int* wide) {
-    const int nb = n / 32, warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-    int emin = 0x7FFFFFFF, emax = -0x7FFFFFFF;
+// Row quantisers of the batched path, four consecutive elements a thread:
+// a Q8_0 block of 32 is eight lanes, and a thread keeps its codes in
+// registers between the row's two passes (Q8_0, then the digit planes,
+// which need the smallest block exponent E of the whole row).
+constexpr int kQuadSpan = 4 * kQuantThreads;           // elements of a row per pass of the CTA
+constexpr int kQuadIters = kMaxQuantCols / kQuadSpan;  // passes at the widest row
+
+// Q8_0 of four values of a block whose other 28 sit in the thread's seven
+// neighbours (lanes 8j .. 8j+7): the arithmetic of q8_0_warp (d = amax/127,
+// q = round-half-away(v * (1/d)) clamped to [-127, 127], amax < FLT_MIN gives
+// d = 0 and zero codes); returns the four codes packed, element 0 lowest.
+// Every lane of the warp must call it.
+__device__ __forceinline__ uint32_t q8_0_quad(const float (&v)[4], float& d) {
+    float a = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, o));
+    d = 0.0f;
+    if (!(a >= FLT_MIN)) return 0u;
+    d = __fdiv_rn(a, 127.0f);
+    const float id = __fdiv_rn(1.0f, d);
+    uint32_t b4[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) b4[e] = (uint32_t)(int)fminf(fmaxf(roundf(__fmul_rn(v[e], id)), -127.0f), 127.0f);
+    return __byte_perm(__byte_perm(b4[0], b4[1], 0x0040), __byte_perm(b4[2], b4[3], 0x0040), 0x5410);
+}
+
+// The row's smallest and largest block exponent over its nonzero blocks (the
+// mantissas and exponents of its nb block scales in shared memory), the
+// same in every thread (emin > emax: all blocks zero).  Every thread of the
+// CTA calls it, after the scales are written and a __syncthreads.
+__device__ __forceinline__ void row_exp_span(const uint32_t* s_m, const int* s_e, int nb, int* s_red, int& emin,
+                                             int& emax) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    emin = 0x7FFFFFFF;
+    emax = -0x7FFFFFFF;
     for (int b = threadIdx.x; b < nb; b += blockDim.x)
         if (s_m[b]) {
             emin = min(emin, s_e[b]);
@@ -439,53 +463,96 @@ __device__ __forceinline__ void row_planes(const int8_t* s_q, const uint32_t* s_
         emin = min(emin, s_red[w]);
         emax = max(emax, s_red[nw + w]);
     }
+}
+
+// The kPlanes digit-plane words of four packed codes q_e (element 0 lowest)
+// of one block with mantissa m (< 2^32): q m + 0x8080808080 lies in
+// [0, 2^40) for |q| <= 127, and its bytes are the signed base-256 digits c_p
+// of q m (q m = sum_p 256^p c_p, c_p in [-128, 127]) plus 128, so each plane
+// word is a byte transpose of the four sums with the top bits flipped.
+__device__ __forceinline__ void quad_planes(uint32_t codes, uint32_t m, uint32_t (&pw)[kPlanes]) {
+    uint32_t lo[4], hi[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int qe = (int)(int8_t)(codes >> (8 * e));
+        const uint64_t t = (uint64_t)((int64_t)qe * (int64_t)m) + 0x8080808080ull;
+        lo[e] = (uint32_t)t;
+        hi[e] = (uint32_t)(t >> 32);
+    }
+    const uint32_t a01 = __byte_perm(lo[0], lo[1], 0x5140), b01 = __byte_perm(lo[0], lo[1], 0x7362);
+    const uint32_t a23 = __byte_perm(lo[2], lo[3], 0x5140), b23 = __byte_perm(lo[2], lo[3], 0x7362);
+    pw[0] = __byte_perm(a01, a23, 0x5410) ^ 0x80808080u;
+    pw[1] = __byte_perm(a01, a23, 0x7632) ^ 0x80808080u;
+    pw[2] = __byte_perm(b01, b23, 0x5410) ^ 0x80808080u;
+    pw[3] = __byte_perm(b01, b23, 0x7632) ^ 0x80808080u;
+    pw[4] = __byte_perm(__byte_perm(hi[0], hi[1], 0x0040), __byte_perm(hi[2], hi[3], 0x0040), 0x5410) ^ 0x80808080u;
+}
+
+// Second pass of a row quantiser: the row's digit planes [kPlanes][n] from
+// the codes the thread kept (codes[j]: the four elements from 4 (threadIdx.x
+// + j kQuantThreads)) and 2^E to *pe (0 for an all-zero row); a row whose
+// exponents spread over more than kMaxSpread sets *wide and writes no
+// planes.  Every thread of the CTA calls it, after writing its block scales.
+__device__ __forceinline__ void row_planes_quad(const uint32_t (&codes)[kQuadIters], const uint32_t* s_m,
+                                                const int* s_e, int n, int* s_red, int8_t* __restrict__ planes,
+                                                double* __restrict__ pe, int* wide) {
+    __syncthreads();
+    int emin, emax;
+    row_exp_span(s_m, s_e, n / 32, s_red, emin, emax);
     const bool any = emin <= emax;  // some block is not zero
     if (any && emax - emin > kMaxSpread) {
         if (threadIdx.x == 0) atomicOr(wide, 1);
         return;
     }
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+#pragma unroll
+    for (int j = 0; j < kQuadIters; ++j) {
+        const int i = 4 * (threadIdx.x + j * kQuantThreads);
+        if (i >= n) break;
         const int b = i >> 5;
         const uint32_t m = s_m[b] ? s_m[b] << (s_e[b] - emin) : 0u;
-        int c[kPlanes];
-        digits5((int)s_q[i], m, c);
+        uint32_t pw[kPlanes];
+        quad_planes(codes[j], m, pw);
 #pragma unroll
-        for (int pl = 0; pl < kPlanes; ++pl) planes[(int64_t)pl * n + i] = (int8_t)c[pl];
+        for (int pl = 0; pl < kPlanes; ++pl) *reinterpret_cast<uint32_t*>(planes + (int64_t)pl * n + i) = pw[pl];
     }
     if (threadIdx.x == 0) *pe = any ? ldexp(1.0, emin) : 0.0;
 }
 
-// Q8_0 of x, one CTA per token (as k_quantize_q8_0: one warp per block of 32,
-// lane = element), and the token's digit planes [5][hidden] with its 2^E
+// Q8_0 of x, one CTA per token (the arithmetic of k_quantize_q8_0, four
+// elements a thread), and the token's digit planes [5][hidden] with its 2^E
 // (see kPlanes); a token too wide for the planes sets *wide (the call then
-// takes the fp64-epilogue GEMMs).
+// takes the fp64-epilogue GEMMs).  hidden is a multiple of 128, so a warp's
+// 128 elements are all in the row or all past it.
 __global__ void __launch_bounds__(kQuantThreads) k_tc_quantize(const float* __restrict__ x, int H,
                                                                int8_t* __restrict__ xq, float* __restrict__ xd,
                                                                int8_t* __restrict__ xpt, double* __restrict__ pet,
                                                                int* wide) {
-    __shared__ int8_t s_q[kMaxQuantCols];
     __shared__ uint32_t s_m[kMaxQuantCols / 32];
     __shared__ int s_e[kMaxQuantCols / 32];
     __shared__ int s_red[2 * kQuantThreads / 32];
-    const int t = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nb = H / 32, nw = kQuantThreads / 32;
-    const float* xt = x + (int64_t)t * H;
-    float v = warp < nb ? __ldg(xt + 32 * warp + lane) : 0.f;
-    for (int b = warp; b < nb; b += nw) {
-        const float vn = b + nw < nb ? __ldg(xt + 32 * (b + nw) + lane) : 0.f;  // the next block's load in flight
-        int8_t q;
+    const int t = blockIdx.x, lane = threadIdx.x & 31;
+    const int nb = H / 32;
+    const float4* xt = reinterpret_cast<const float4*>(x + (int64_t)t * H);
+    uint32_t codes[kQuadIters];
+    float4 v = 4 * threadIdx.x < H ? __ldg(xt + threadIdx.x) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < kQuadIters; ++j) {
+        const int u = threadIdx.x + j * kQuantThreads, i = 4 * u;
+        if (i >= H) break;
+        // the next pass's load in flight
+        const float4 vn = i + kQuadSpan < H ? __ldg(xt + u + kQuantThreads) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float vv[4] = {v.x, v.y, v.z, v.w};
         float d;
-        q8_0_warp(v, q, d);
-        xq[(int64_t)t * H + 32 * b + lane] = q;
-        s_q[32 * b + lane] = q;
-        if (lane == 0) {
+        codes[j] = q8_0_quad(vv, d);
+        *reinterpret_cast<uint32_t*>(xq + (int64_t)t * H + i) = codes[j];
+        if ((lane & 7) == 0) {
+            const int b = i >> 5;
             xd[(int64_t)t * nb + b] = d;
             f32_mant_exp(d, s_m[b], s_e[b]);
         }
         v = vn;
     }
-    __syncthreads();
-    row_planes(s_q, s_m, s_e, H, s_red, xpt + (int64_t)t * kPlanes * H, pet + t, wide);
+    row_planes_quad(codes, s_m, s_e, H, s_red, xpt + (int64_t)t * kPlanes * H, pet + t, wide);
 }
 
 // One warp per padded row: its token's digit planes and 2^E (zeros for a
@@ -1135,16 +1202,13 @@ __global__ void __launch_bounds__(kDpThreads, 1)
 }
 
 // SwiGLU and Q8_0 of h, one CTA per padded row, four consecutive elements a
-// thread (a Q8_0 block of 32 is eight lanes): h = silu(g) * u evaluated in
-// fp64 and rounded to fp32, then Q8_0 (the arithmetic of q8_0_warp, the
-// block's |h| maximum taken over its eight lanes); the codes and scales go to
-// the slot's h (hq, hd), to the row's codes and transposed fp64 scales (hg,
-// hdT: the fp64-epilogue GEMM's operands) and, as in k_tc_quantize, to the
-// row's digit planes [5][inter] with 2^E in peh (a row too wide for the
-// planes sets *wide).  The codes stay in registers between the two passes.
-// Padding rows: zero planes and scales.
-constexpr int kSwigluSpan = 4 * kQuantThreads;              // elements of the row per pass of the CTA
-constexpr int kSwigluIters = kMaxQuantCols / kSwigluSpan;   // passes at the widest row
+// thread: h = silu(g) * u evaluated in fp64 and rounded to fp32, then Q8_0;
+// the codes and scales go to the slot's h (hq, hd), to the row's codes and
+// transposed fp64 scales (hg, hdT: the fp64-epilogue GEMM's operands) and,
+// as in k_tc_quantize, to the row's digit planes [5][inter] with 2^E in peh
+// (a row too wide for the planes sets *wide).  Padding rows: zero planes and
+// scales.  inter is a multiple of 128 (a warp's elements are all in the row
+// or all past it).
 __global__ void __launch_bounds__(kQuantThreads) k_tc_swiglu(const float* __restrict__ gu, int I, int prows_cap,
                                                              const int32_t* __restrict__ row_slot,
                                                              const int32_t* __restrict__ ctrl, int8_t* __restrict__ hg,
@@ -1154,9 +1218,9 @@ __global__ void __launch_bounds__(kQuantThreads) k_tc_swiglu(const float* __rest
     __shared__ uint32_t s_m[kMaxQuantCols / 32];
     __shared__ int s_e[kMaxQuantCols / 32];
     __shared__ int s_red[2 * kQuantThreads / 32];
-    const int q = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = blockIdx.x, lane = threadIdx.x & 31;
     if (q >= ctrl[2]) return;
-    const int nbI = I / 32, nw = kQuantThreads / 32;
+    const int nbI = I / 32;
     const int slot = row_slot[q];
     int8_t* dst = hp + (int64_t)q * kPlanes * I;
     if (slot < 0) {  // a padding row
@@ -1168,16 +1232,15 @@ __global__ void __launch_bounds__(kQuantThreads) k_tc_swiglu(const float* __rest
     }
     const float4* gr = reinterpret_cast<const float4*>(gu + (int64_t)q * I);
     const float4* ur = reinterpret_cast<const float4*>(gu + ((int64_t)prows_cap + q) * I);
-    uint32_t codes[kSwigluIters];
-    // I is a multiple of 128, so a warp's 128 elements are all in the row or all past it
+    uint32_t codes[kQuadIters];
     float4 g = 4 * threadIdx.x < I ? gr[threadIdx.x] : make_float4(0.f, 0.f, 0.f, 0.f);
     float4 u = 4 * threadIdx.x < I ? ur[threadIdx.x] : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int j = 0; j < kSwigluIters; ++j) {
-        const int v = threadIdx.x + j * kQuantThreads, i = 4 * v;  // first element of this thread
+    for (int j = 0; j < kQuadIters; ++j) {
+        const int v = threadIdx.x + j * kQuantThreads, i = 4 * v;
         if (i >= I) break;
         // the next pass's loads in flight while this one is computed
-        const bool nx = i + kSwigluSpan < I;
+        const bool nx = i + kQuadSpan < I;
         const float4 gn = nx ? gr[v + kQuantThreads] : make_float4(0.f, 0.f, 0.f, 0.f);
         const float4 un = nx ? ur[v + kQuantThreads] : make_float4(0.f, 0.f, 0.f, 0.f);
         const float gv[4] = {g.x, g.y, g.z, g.w}, uv[4] = {u.x, u.y, u.z, u.w};
@@ -1187,23 +1250,8 @@ __global__ void __launch_bounds__(kQuantThreads) k_tc_swiglu(const float* __rest
             const double gd = (double)gv[e];
             h[e] = __double2float_rn(__dmul_rn(__ddiv_rn(gd, __dadd_rn(1.0, exp(-gd))), (double)uv[e]));
         }
-        // Q8_0 of the block (eight lanes): d = amax / 127, q = round-half-away(h * (1/d)) in [-127, 127]
-        float a = fmaxf(fmaxf(fabsf(h[0]), fabsf(h[1])), fmaxf(fabsf(h[2]), fabsf(h[3])));
-#pragma unroll
-        for (int o = 4; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, o));
-        float d = 0.0f;
-        uint32_t c = 0u;
-        if (a >= FLT_MIN) {
-            d = __fdiv_rn(a, 127.0f);
-            const float id = __fdiv_rn(1.0f, d);
-            uint32_t b4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float r = fminf(fmaxf(roundf(__fmul_rn(h[e], id)), -127.0f), 127.0f);
-                b4[e] = (uint32_t)(int)r;
-            }
-            c = __byte_perm(__byte_perm(b4[0], b4[1], 0x0040), __byte_perm(b4[2], b4[3], 0x0040), 0x5410);
-        }
+        float d;
+        const uint32_t c = q8_0_quad(h, d);
         codes[j] = c;
         *reinterpret_cast<uint32_t*>(hg + (int64_t)q * I + i) = c;
         *reinterpret_cast<uint32_t*>(hq + (int64_t)slot * I + i) = c;
@@ -1216,59 +1264,7 @@ __global__ void __launch_bounds__(kQuantThreads) k_tc_swiglu(const float* __rest
         g = gn;
         u = un;
     }
-    __syncthreads();
-    // the row's smallest block exponent and spread (as row_planes)
-    int emin = 0x7FFFFFFF, emax = -0x7FFFFFFF;
-    for (int b = threadIdx.x; b < nbI; b += kQuantThreads)
-        if (s_m[b]) {
-            emin = min(emin, s_e[b]);
-            emax = max(emax, s_e[b]);
-        }
-    emin = __reduce_min_sync(kFull, emin);
-    emax = __reduce_max_sync(kFull, emax);
-    if (lane == 0) {
-        s_red[warp] = emin;
-        s_red[nw + warp] = emax;
-    }
-    __syncthreads();
-    for (int w = 0; w < nw; ++w) {
-        emin = min(emin, s_red[w]);
-        emax = max(emax, s_red[nw + w]);
-    }
-    const bool any = emin <= emax;  // some block is not zero
-    if (any && emax - emin > kMaxSpread) {
-        if (threadIdx.x == 0) atomicOr(wide, 1);
-        return;
-    }
-    // digits: q m + 0x8080808080 (in [0, 2^40) for |q| <= 127, m < 2^32) has
-    // the bytes c_p + 128 of the signed base-256 digits c_p of q m
-#pragma unroll
-    for (int j = 0; j < kSwigluIters; ++j) {
-        const int i = 4 * (threadIdx.x + j * kQuantThreads);
-        if (i >= I) break;
-        const int b = i >> 5;
-        const uint32_t m = s_m[b] ? s_m[b] << (s_e[b] - emin) : 0u;
-        uint32_t lo[4], hi[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int qe = (int)(int8_t)(codes[j] >> (8 * e));
-            const uint64_t t = (uint64_t)((int64_t)qe * (int64_t)m) + 0x8080808080ull;
-            lo[e] = (uint32_t)t;
-            hi[e] = (uint32_t)(t >> 32);
-        }
-        const uint32_t a01 = __byte_perm(lo[0], lo[1], 0x5140), b01 = __byte_perm(lo[0], lo[1], 0x7362);
-        const uint32_t a23 = __byte_perm(lo[2], lo[3], 0x5140), b23 = __byte_perm(lo[2], lo[3], 0x7362);
-        uint32_t pw[kPlanes];
-        pw[0] = __byte_perm(a01, a23, 0x5410);
-        pw[1] = __byte_perm(a01, a23, 0x7632);
-        pw[2] = __byte_perm(b01, b23, 0x5410);
-        pw[3] = __byte_perm(b01, b23, 0x7632);
-        pw[4] = __byte_perm(__byte_perm(hi[0], hi[1], 0x0040), __byte_perm(hi[2], hi[3], 0x0040), 0x5410);
-#pragma unroll
-        for (int pl = 0; pl < kPlanes; ++pl)
-            *reinterpret_cast<uint32_t*>(dst + (int64_t)pl * I + i) = pw[pl] ^ 0x80808080u;
-    }
-    if (threadIdx.x == 0) peh[q] = any ? ldexp(1.0, emin) : 0.0;
+    row_planes_quad(codes, s_m, s_e, I, s_red, dst, peh + q, wide);
 }
 
 }  // namespace tc

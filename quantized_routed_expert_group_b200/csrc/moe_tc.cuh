@@ -54,21 +54,6 @@ __device__ __forceinline__ void f32_mant_exp(float v, uint32_t& m, int& e) {
     e = f ? (int)f - 150 : -149;
 }
 
-// The kPlanes signed base-256 digits of q * m (|q| <= 127, m < 2^32): q m =
-// sum_p 256^p c_p with c_p in [-128, 127], lowest first.  q m is split as
-// q (m >> 16) 2^16 + q (m & 0xFFFF), both products below 2^23.
-__device__ __forceinline__ void digits5(int q, uint32_t m, int (&c)[kPlanes]) {
-    const int lo = q * (int)(m & 0xFFFFu), hi = q * (int)(m >> 16);
-    c[0] = (int)(int8_t)lo;
-    int r = (lo - c[0]) >> 8;
-    c[1] = (int)(int8_t)r;
-    r = ((r - c[1]) >> 8) + hi;
-    c[2] = (int)(int8_t)r;
-    r = (r - c[2]) >> 8;
-    c[3] = (int)(int8_t)r;
-    c[4] = (r - c[3]) >> 8;
-}
-
 // A unit of work of the grouped GEMMs: one 128-row tile of one expert's
 // weight matrix applied to a chunk of <= kChunk of the expert's tokens.
 struct TcUnit {

@@ -79,6 +79,26 @@ def test_tiny_host_entry_point(tiny):
     assert torch.equal(out, ref)
 
 
+@pytest.mark.parametrize("T", [1, 4, 9])
+def test_tiny_host_entry_repeated(tiny, T):
+    """Repeated host-entry calls on the same pinned buffers: each copies the
+    buffer's current contents (new tokens every call), whichever of two
+    buffer pairs it is given, and a pageable pair agrees."""
+    base = torch.from_numpy(synth.make_x(tiny.wl.with_tokens(T)))
+    bufs = [(torch.empty_like(base).pin_memory(), torch.empty_like(base).pin_memory()) for _ in range(2)]
+    for i in range(6):
+        x = base * (1.0 + 0.25 * i) - 0.01 * i
+        xh, oh = bufs[i % 2]
+        xh.copy_(x)
+        oh.fill_(float("nan"))
+        tiny.layer.forward_host(xh, oh)
+        ref = tiny.layer.forward(x.cuda()).cpu()
+        assert torch.equal(oh, ref), f"call {i}"
+    xp, op = base.clone(), torch.empty_like(base)
+    tiny.layer.forward_host(xp, op)
+    assert torch.equal(op, tiny.layer.forward(base.cuda()).cpu())
+
+
 @pytest.mark.parametrize("shape,T,seed,x_kind", [
     # multi-kernel path (T > 4)
     (MID4, 37, 11, "normal"), (MID8, 19, 12, "normal"), (MID4_NOSHARED, 5, 14, "normal"),
