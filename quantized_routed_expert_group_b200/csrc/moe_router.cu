@@ -272,6 +272,84 @@ __global__ void __launch_bounds__(128) k_router_select(const double* __restrict_
     }
 }
 
+// The same selection for groups of 32 experts (warp g = group g), one CTA
+// per token and one thread per expert, by ranks instead of rounds: a group
+// is kept when fewer than topk_groups groups beat its score (larger, ties to
+// the lower group), an expert of a kept group is pick r when r experts of
+// the kept groups beat it (larger c, ties to the lower index) -- the order
+// in which the rounds of k_router_select take them, so the picks, their
+// order and the weights are the same.
+__global__ void __launch_bounds__(1024) k_router_select_g32(const double* __restrict__ logits,
+                                                            const float* __restrict__ bias, int E, int G, int tg,
+                                                            int k, float rsf, float topp, int32_t* __restrict__ idx,
+                                                            float* __restrict__ wout) {
+    __shared__ double sc[1024], ss[1024], gsc[32];
+    __shared__ int kg[32], sel[32];
+    const int t = blockIdx.x, e = threadIdx.x, warp = e >> 5, lane = e & 31;
+    {
+        const double l = logits[(int64_t)t * E + e];
+        const double sv = 1.0 / (1.0 + exp(-l));
+        ss[e] = sv;
+        sc[e] = sv + (double)bias[e];
+    }
+    __syncwarp();
+    // group score: the sum of the group's two best c (ties to the lower index)
+    {
+        const double c = sc[e];
+        double v = c;
+        int a = e;
+        warp_argmax(v, a);
+        double v2 = e == a ? -INFINITY : c;
+        int b = e == a ? 0x7fffffff : e;
+        warp_argmax(v2, b);
+        if (lane == 0) gsc[warp] = sc[a] + sc[b & 1023];
+    }
+    __syncthreads();
+    if (e < G) {
+        const double gs = gsc[e];
+        int rank = 0;
+        for (int g2 = 0; g2 < G; ++g2) rank += (gsc[g2] > gs || (gsc[g2] == gs && g2 < e)) ? 1 : 0;
+        if (rank < tg) kg[rank] = e;
+    }
+    __syncthreads();
+    // rank of this expert among the kept groups' experts
+    bool mine = false;
+    for (int q = 0; q < tg; ++q) mine |= kg[q] == warp;
+    if (mine) {
+        const double c = sc[e];
+        int rank = 0;
+        for (int q = 0; q < tg; ++q) {
+            const int g2 = kg[q];
+#pragma unroll 8
+            for (int l2 = 0; l2 < 32; ++l2) {
+                const int e2 = 32 * g2 + l2;
+                const double c2 = sc[e2];
+                rank += (c2 > c || (c2 == c && e2 < e)) ? 1 : 0;
+            }
+        }
+        if (rank < k) sel[rank] = e;
+    }
+    __syncthreads();
+    if (warp != 0) return;
+    const int pick = lane < k ? sel[lane] : 0;
+    const double sj = lane < k ? ss[pick] : 0.0;
+    double ssum = 0.0;
+    for (int n = 0; n < k; ++n) ssum += __shfl_sync(kFull, sj, n);  // pick order: s_0 + s_1 + ...
+    if (topp > 0.f && topp < 1.f) {
+        double skept;
+        const bool keep = topp_keep(sj, ssum, k, topp, lane, &skept);
+        if (lane < k) {
+            idx[(int64_t)t * k + lane] = keep ? pick : -1;
+            wout[(int64_t)t * k + lane] = keep ? (float)(sj / skept * (double)rsf) : 0.f;
+        }
+        return;
+    }
+    if (lane < k) {
+        idx[(int64_t)t * k + lane] = pick;
+        wout[(int64_t)t * k + lane] = (float)(sj / ssum * (double)rsf);
+    }
+}
+
 size_t router_ws_bytes(const moe_config& c, int T) {
     const size_t logits = ((size_t)T * c.n_experts * sizeof(double) + 255) & ~(size_t)255;
     const int S = router_splits(c, T);
@@ -302,6 +380,11 @@ cudaError_t launch_router(const moe_config& c, const float* x, int T, const floa
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    if (c.n_experts / c.n_groups == 32 && c.top_k <= 32) {  // E = 32 G <= 1024: one thread per expert
+        k_router_select_g32<<<T, c.n_experts, 0, s>>>(logits, bias, c.n_experts, c.n_groups, c.topk_groups,
+                                                      c.top_k, c.routed_scaling_factor, c.expert_topp, idx, w);
+        return cudaGetLastError();
+    }
     const size_t smem = (size_t)4 * 2 * c.n_experts * sizeof(double);
     if (smem > 48 * 1024) {
         e = cudaFuncSetAttribute(k_router_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

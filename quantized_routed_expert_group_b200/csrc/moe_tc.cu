@@ -201,11 +201,12 @@ cudaError_t launch_tc_block_dots(const uint8_t* packed, int64_t rows, int cols, 
 //
 // Data flow (T at or above kTcMinTokens, see tc_path_supported):
 //   Q8_0 of x, router, bucketing   (the multi-kernel path's kernels)
-//   k_tc_plan     one CTA: the batch-union entries (each selected expert, then
+//   k_tc_plan     the batch-union entries (each selected expert, then
 //                 the shared expert), their rows in a padded row space (each
 //                 entry's tokens start on a multiple of 16 rows), and the work
 //                 units (entry, 128-row weight tile, matrix, chunk of <= 64
-//                 tokens), heaviest entries first
+//                 tokens), heaviest entries first; every CTA of a few builds
+//                 the entry tables, and they split the units and rows
 //   k_tc_gather   the entries' Q8_0 codes of x into the padded row space
 //                 (xg [prows][hidden]) and their block scales, transposed and
 //                 widened to fp64 (xdT [hidden/32][prows]), so that every
@@ -242,6 +243,7 @@ struct PlanParams {
 };
 
 constexpr int kPlanThreads = 1024;
+constexpr int kPlanCtas = 16;  // every CTA builds the entry tables; the units and rows are split over them
 constexpr int kMaxEntries = 1025;
 constexpr int kUnitUp = 1 << 17;  // TcUnit::info: the unit's matrix is W_up (gate/up GEMM)
 
@@ -335,7 +337,7 @@ __global__ void __launch_bounds__(kPlanThreads) k_tc_plan(PlanParams p) {
     }
     if (prows > p.prows_cap || rgu > p.units_gu_cap || rdn > p.units_dn_cap) {
         // cannot happen for a consistent bucketing; leave no work
-        if (tid == 0) {
+        if (blockIdx.x == 0 && tid == 0) {
             set_error(p.err, kErrIndex);
             for (int i = 0; i < 5; ++i) p.ctrl[i] = 0;
         }
@@ -354,7 +356,8 @@ __global__ void __launch_bounds__(kPlanThreads) k_tc_plan(PlanParams p) {
         }
         return lo;
     };
-    for (int u = tid; u < rgu; u += kPlanThreads) {
+    const int g0 = blockIdx.x * kPlanThreads + tid, gstep = gridDim.x * kPlanThreads;
+    for (int u = g0; u < rgu; u += gstep) {
         const int r = entry_of(s_ugu0, u), i = s_sched[r];
         const int n = s_n[i], nch = (n + kChunk - 1) / kChunk;
         const int l = u - s_ugu0[r], c = l % nch, tm = l / nch, m = tm & 1, t = tm >> 1;
@@ -366,7 +369,7 @@ __global__ void __launch_bounds__(kPlanThreads) k_tc_plan(PlanParams p) {
         w.info = t | (shared ? kUnitShared : 0) | (m ? kUnitUp : 0);
         p.units_gu[u] = w;
     }
-    for (int u = tid; u < rdn; u += kPlanThreads) {
+    for (int u = g0; u < rdn; u += gstep) {
         const int r = entry_of(s_udn0, u), i = s_sched[r];
         const int n = s_n[i], nch = (n + kChunk - 1) / kChunk;
         const int l = u - s_udn0[r], c = l % nch, t = l / nch;
@@ -379,7 +382,7 @@ __global__ void __launch_bounds__(kPlanThreads) k_tc_plan(PlanParams p) {
         p.units_dn[u] = w;
     }
     // padded row -> token and slot (-1 for the padding rows)
-    for (int q = tid; q < prows; q += kPlanThreads) {
+    for (int q = g0; q < prows; q += gstep) {
         int lo = 0, hi = ne - 1;
         while (lo < hi) {  // last entry whose first row is <= q
             const int mid = (lo + hi + 1) >> 1;
@@ -395,7 +398,7 @@ __global__ void __launch_bounds__(kPlanThreads) k_tc_plan(PlanParams p) {
         p.row_tok[q] = tok;
         p.row_slot[q] = slot;
     }
-    if (tid == 0) {
+    if (blockIdx.x == 0 && tid == 0) {
         p.ctrl[0] = rgu;
         p.ctrl[1] = rdn;
         p.ctrl[2] = prows;
@@ -1300,7 +1303,7 @@ cudaError_t launch_tc_prepare(const TcArgs& a, cudaStream_t s) {
     pp.units_gu = static_cast<tc::TcUnit*>(a.units_gu);
     pp.units_dn = static_cast<tc::TcUnit*>(a.units_dn);
     pp.row_tok = a.row_tok; pp.row_slot = a.row_slot; pp.ctrl = a.ctrl; pp.err = a.ex.err;
-    tc::k_tc_plan<<<1, tc::kPlanThreads, 0, s>>>(pp);
+    tc::k_tc_plan<<<tc::kPlanCtas, tc::kPlanThreads, 0, s>>>(pp);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int grid = (a.sz.prows_cap + 7) / 8;
