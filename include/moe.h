@@ -254,7 +254,7 @@ int moe_layer_forward_host(const moe_config *cfg, const float *x_host, int T, co
  * Limit: the layer's workspace for T tokens must fit in 8 MiB
  * (moe_workspace_bytes(cfg, T) <= 8388608); larger T returns MOE_EWORKSPACE
  * and launches nothing.  For the GLM-5.2 layer (hidden 6144, 256 experts,
- * top-8 + 1 shared) that allows T <= 22.
+ * top-8 + 1 shared) that allows T <= 17.
  *
  * The first call on each device looks up the array's device address with that
  * device current (once per device); make that first call before any stream

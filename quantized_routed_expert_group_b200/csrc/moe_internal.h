@@ -66,7 +66,7 @@ cudaError_t launch_requant_fp8(const uint8_t* w8, const float* block_scales, int
                                int wbits, uint8_t* packed, float* scales, cudaStream_t s);
 // The router's workspace: logits [T][E] fp64, then (T >= kRouterTiledMinTokens)
 // the tiled kernel's K-split partial sums.
-constexpr int kRouterTiledMinTokens = 64;
+constexpr int kRouterTiledMinTokens = 5;  // below: the per-token kernel (the fused path's sizes)
 size_t router_ws_bytes(const moe_config& c, int T);
 cudaError_t launch_router(const moe_config& c, const float* x, int T, const float* router_w,
                           const float* bias, double* logits, int32_t* idx, float* w, cudaStream_t s);

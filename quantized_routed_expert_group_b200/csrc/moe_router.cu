@@ -84,12 +84,13 @@ __global__ void __launch_bounds__(256) k_router_logits(const float* __restrict__
 constexpr int kRtT = 64, kRtE = 64, kRtK = 32;
 constexpr int kRtPad = 4;  // rows of 36 doubles: conflict-free fragment loads and staging stores
 constexpr int kRtTargetCtas = 3 * 148;
+constexpr int kRtMaxSplits = 48;  // a few tokens: a few tiles, split finely (parts: S x T x E doubles)
 
 int router_splits(const moe_config& c, int T) {
     if (T < kRouterTiledMinTokens || c.hidden % kRtK) return 0;
     const int tiles = ((T + kRtT - 1) / kRtT) * ((c.n_experts + kRtE - 1) / kRtE);
     int want = kRtTargetCtas / tiles;  // never a second, partial wave
-    want = want < 1 ? 1 : want > 16 ? 16 : want;
+    want = want < 1 ? 1 : want > kRtMaxSplits ? kRtMaxSplits : want;
     const int chunks = c.hidden / kRtK;
     return want < chunks ? want : chunks;
 }

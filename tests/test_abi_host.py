@@ -147,13 +147,14 @@ def test_other_entry_point_errors(L):
 
 
 def test_forward_paths_and_phases(L):
-    """T <= 4 takes the fused small-batch path (2 launches, one traced phase);
-    larger batches the multi-kernel path (7 launches, five phases)."""
+    """T <= 4 takes the fused small-batch path (one launch, one traced phase);
+    larger batches the multi-kernel path (five phases; 8 launches at 16
+    tokens: the router's split-K logits add their reduction from 5 tokens)."""
     c = _cfg(L)
     assert L.forward_phases(c, 1) == ["fused"] and L.forward_launches(c, 1) == 1
     assert L.forward_phases(c, 4) == ["fused"]
     assert L.forward_phases(c, 5) == ["route", "bucket", "gate_up", "down", "combine"]
-    assert L.forward_launches(c, 16) == 7 and L.forward_launches(c, 0) == 0
+    assert L.forward_launches(c, 16) == 8 and L.forward_launches(c, 0) == 0
     big = _cfg(L, n_experts=512, n_groups=16)   # beyond the fused path's 256 experts
     assert L.forward_phases(big, 1) == ["route", "bucket", "gate_up", "down", "combine"]
     assert L.lib().moe_profile_events(None, 3) == -1
@@ -173,4 +174,5 @@ def test_path_selection(L, shape, T, fused):
     c = L.config(shape)
     phases = L.forward_phases(c, T)
     assert (phases == ["fused"]) == fused, phases
-    assert L.forward_launches(c, T) == (1 if fused else 7)
+    # multi-kernel: 7 launches, one more (the split-K router reduction) from 5 tokens
+    assert L.forward_launches(c, T) == (1 if fused else 8 if T >= 5 else 7)
