@@ -188,7 +188,16 @@ __global__ void __launch_bounds__(256) k_router_reduce(const double* __restrict_
                                                        double* __restrict__ logits) {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
         double v = parts[i];
-        for (int sp = 1; sp < S; ++sp) v = __dadd_rn(v, parts[(int64_t)sp * n + i]);
+        int sp = 1;
+        // eight loads in flight at a time; the adds stay in split order
+        for (; sp + 8 <= S; sp += 8) {
+            double u[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) u[j] = parts[(int64_t)(sp + j) * n + i];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v = __dadd_rn(v, u[j]);
+        }
+        for (; sp < S; ++sp) v = __dadd_rn(v, parts[(int64_t)sp * n + i]);
         logits[i] = v;
     }
 }
