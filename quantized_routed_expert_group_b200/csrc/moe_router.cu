@@ -296,6 +296,10 @@ __global__ void __launch_bounds__(1024) k_router_select_g32(const double* __rest
     __shared__ double sc[1024], ss[1024], gsc[32];
     __shared__ int kg[32], sel[32];
     const int t = blockIdx.x, e = threadIdx.x, warp = e >> 5, lane = e & 31;
+    if (e < 32) {  // in bounds whatever the scores (non-finite ones rank nothing)
+        kg[e] = 0;
+        sel[e] = 0;
+    }
     {
         const double l = logits[(int64_t)t * E + e];
         const double sv = 1.0 / (1.0 + exp(-l));
